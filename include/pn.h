@@ -1,0 +1,162 @@
+/*
+ * pn.h -- C ABI of libpn: parallel Newton evaluation of nonlinear sequences
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The problem (web article "并行牛顿方法：加速非线性序列评估的计算革命",
+ * "Parallel Newton methods for nonlinear sequence evaluation", jsqmd.com news
+ * item 789890; cited below as "page §X"):
+ *   given s0 and f_1..f_T, compute every state s_t = f_t(s_{t-1})   (§1.1)
+ * by the fixed-point iteration s^(i+1) = s^(i) - J~^{-1}(s^(i)) F(s^(i))
+ * (§1.2), where F_t(s) = s_t - f_t(s_{t-1}) and J~ = I - subdiag(A~_t):
+ *   PN_JACOBI  A~_t = 0                      (J~ ~ I, §1.2)
+ *   PN_PICARD  A~_t = I                      (identity approximation, §2.2.3)
+ *   PN_QUASI   A~_t = diag(df_t/ds)          (diagonal approximation, §2.2.1)
+ *   PN_NEWTON  A~_t = df_t/ds, dense D x D   (exact Jacobian, §1.2)
+ * Each iteration evaluates f_t and A~_t at all t in parallel and then solves
+ * the linear recurrence s^(i+1)_t = A~_t s^(i+1)_{t-1} + (f_t(s^(i)_{t-1}) -
+ * A~_t s^(i)_{t-1}) with a parallel scan (§2.1).  The loop stops at the first
+ * i whose residual r^(i) = max_{b,t,d} |F_t(s^(i))| satisfies r^(i) <= tol,
+ * or at i == max_iters (residual monitoring, §5.3; the infinity norm over the
+ * whole batch and the "<=" tie-break are this library's reading).  The
+ * initial guess is s^(0)_t = s0 for every t.
+ *
+ * Conventions for every entry point:
+ *  - All tensors are row-major float32.  x is [B][T][d_in], s0 is [B][D],
+ *    states is [B][T][D] (channels innermost).
+ *  - "device" pointers must be CUDA device (or managed) memory of the device
+ *    that was current at pn_create; "host" pointers are ordinary or pinned
+ *    host memory.  The caller owns every pointer it passes; the library never
+ *    frees or retains them past the call.
+ *  - Work is ordered on the handle's stream (set at pn_create or with
+ *    pn_set_stream).  pn_eval and pn_eval_host synchronise that stream before
+ *    returning, so every output is complete on return.
+ *  - Errors are reported by the return code; pn_last_error gives the text.
+ *    A handle is not thread-safe: one call at a time per handle.
+ */
+#ifndef PN_H
+#define PN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct pn_ctx* pn_handle;
+
+typedef enum {
+  PN_OK = 0,              /* converged: r^(iters) <= tol                         */
+  PN_NOT_CONVERGED = 1,   /* soft: iters == max_iters and r > tol; outputs valid */
+  PN_ERR_INVALID = -1,    /* bad argument; nothing was launched                  */
+  PN_ERR_NOMEM = -2,      /* device or pinned-host allocation failed             */
+  PN_ERR_CUDA = -3,       /* a CUDA runtime call failed (text in pn_last_error)  */
+  PN_ERR_NONFINITE = -4,  /* r^(i) was NaN or Inf; states hold that s^(i)        */
+  PN_ERR_TIMEOUT = -5     /* a bounded device wait gave up; states are invalid   */
+} pn_status;
+
+typedef enum {
+  PN_CELL_TANH_RNN = 0,   /* f_t(s) = tanh(W s + U x_t + b)                       */
+  PN_CELL_GRU = 1,        /* GRU, gates r, z, n (PyTorch convention)              */
+  PN_CELL_EULER_TANH = 2  /* f_t(s) = s + eps * tanh(W s + c_t), c_t = x_t, d_in=D */
+} pn_cell;
+
+typedef enum { PN_JACOBI = 0, PN_PICARD = 1, PN_QUASI = 2, PN_NEWTON = 3 } pn_mode;
+
+typedef enum {
+  /* Bound, in nanoseconds, on every device-side spin wait of the chunked scan
+   * (default 1e9).  When it runs out the iteration stops with PN_ERR_TIMEOUT. */
+  PN_OPT_WAIT_TIMEOUT_NS = 0,
+  /* Test hook: the scan tile with this ticket number never publishes its
+   * result, so its successors' bounded waits run out (-1 = off, default). */
+  PN_OPT_DEBUG_STALL_TICKET = 1,
+  /* 1 (default): the convergence loop runs on the device inside a CUDA graph
+   * (conditional WHILE node); 0: the host launches one iteration at a time and
+   * reads the stop decision back after each. */
+  PN_OPT_DEVICE_LOOP = 2
+} pn_option;
+
+/* Per-handle counters, cumulative since pn_create (or pn_reset_stats). */
+typedef struct {
+  long long iteration_launches;  /* fused iteration kernels launched           */
+  long long iteration_ns;        /* their summed device durations (first CTA
+                                    start to last CTA end, %globaltimer)       */
+  long long evals;               /* completed pn_eval / pn_eval_host calls     */
+} pn_stats;
+
+/* Supported sizes: 1 <= D <= 256 for PN_JACOBI/PN_PICARD/PN_QUASI and
+ * 1 <= D <= 64 for PN_NEWTON; d_in >= 1 (d_in == D for the Euler cell);
+ * T >= 1, B >= 1, B*T*max(D,d_in)*4 bytes must fit in device memory. */
+#define PN_MAX_D_DIAG 256
+#define PN_MAX_D_NEWTON 64
+
+/* Create a solver for one cell and one problem shape.
+ *   params   host, float32, n_params entries, copied to the device (the caller
+ *            keeps ownership).  Packing, row-major:
+ *              tanh RNN : W[D][D], U[D][d_in], b[D]
+ *              GRU      : W_ih[3D][d_in], W_hh[3D][D], b_ih[3D], b_hh[3D]
+ *              Euler    : W[D][D]
+ *   eps      Euler step (ignored by the other cells).
+ *   cuda_stream  a cudaStream_t (NULL = the legacy default stream).
+ * Allocates every work buffer for (D, d_in, T, B) up front.  On error *out is
+ * set to NULL and the message is available from pn_last_error(NULL). */
+pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
+                    const float* params, size_t n_params, float eps,
+                    void* cuda_stream);
+
+/* Evaluate all states.
+ *   x       device [B][T][d_in]  (Euler: c_t, d_in == D)
+ *   s0      device [B][D]
+ *   mode    iteration, see pn_mode
+ *   max_iters  >= 0; at most this many updates are applied
+ *   tol     >= 0 and finite
+ *   states  device [B][T][D], written with s^(iters); also used as one of
+ *           the two iterate buffers while the call runs
+ *   iters_out, resid_out  host; receive the iteration count and r^(iters)
+ *           (either may be NULL)
+ * Returns PN_OK, PN_NOT_CONVERGED, or an error (see pn_status). */
+pn_status pn_eval(pn_handle h, const float* x, const float* s0, pn_mode mode,
+                  int max_iters, float tol, float* states, int* iters_out,
+                  float* resid_out);
+
+/* pn_eval with HOST buffers: copies x and s0 to library-owned device buffers,
+ * evaluates, and copies the states back into states_host, all on the handle's
+ * stream (pinned host memory makes the copies asynchronous).  The device
+ * buffers are allocated on the first call and reused. */
+pn_status pn_eval_host(pn_handle h, const float* x_host, const float* s0_host,
+                       pn_mode mode, int max_iters, float tol,
+                       float* states_host, int* iters_out, float* resid_out);
+
+/* Copy min(n, iters+1) residuals r^(0..iters) of the last evaluation into the
+ * host array out; *n_written (may be NULL) receives the count. */
+pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written);
+
+/* Time the fused iteration kernel of `mode` alone: after a pn_eval on this
+ * handle (its x, s0 and states must still be valid), launch exactly
+ * n_launches iteration kernels back to back on the handle's stream, with no
+ * stop rule, bracketed by CUDA events.  *avg_ms receives the mean duration per
+ * launch.  The states buffer of that pn_eval is overwritten with later
+ * iterates. */
+pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* avg_ms);
+
+pn_status pn_get_stats(pn_handle h, pn_stats* out);
+pn_status pn_reset_stats(pn_handle h);
+pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
+pn_status pn_set_stream(pn_handle h, void* cuda_stream);
+
+/* Shape queries (for the binding); each returns -1 for a NULL handle. */
+int pn_dim(pn_handle h, int which /* 0=D 1=d_in 2=T 3=B 4=cell */);
+
+/* Last error message of this handle, or of the calling thread's last failed
+ * pn_create when h is NULL.  Never NULL; "" when there was no error. */
+const char* pn_last_error(pn_handle h);
+
+/* Release every device and host resource of the handle (NULL is a no-op). */
+void pn_destroy(pn_handle h);
+
+/* Library version string. */
+const char* pn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PN_H */
