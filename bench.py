@@ -1,0 +1,359 @@
+"""Benchmark: converged sequence-steps x batch per second of parallel Newton evaluation.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pn|reference]
+                    [--workload I] [--mode M] [--all]
+
+A step is one full evaluation (pn_eval: input projection, the device-side
+convergence loop of fused iteration kernels, result copy) of one synthetic
+workload, by default the tanh RNN D=64, T=16384, B=16 with diagonal
+quasi-Newton (tol 1e-5).  The timed region holds exactly K steps between a
+barrier + device synchronisation on both sides, timed with CUDA events; for N>1
+(launched by torch.distributed.run, one rank per GPU) every rank evaluates its
+own copy of the workload (independent problem instances, no collective in the
+data path: weak scaling) and the time is the max over ranks.
+
+Also reported, on rank 0: the end-to-end number through pn_eval_host with the
+host<->device copies inside the timed region; the roofline of the fused
+iteration kernel (algorithmic bytes per launch / its mean launch time, CUDA
+events around back-to-back launches on the library's stream); and the fp64
+oracle timed on this host's cores on a bounded sample of the same workload.
+``--impl reference`` times that oracle alone as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import pn_inputs as pi  # noqa: E402
+
+METRIC = "converged sequence-steps x batch /sec per mode; % of HBM roofline"
+UNIT = "steps*batch/s"
+DEFAULT_WORKLOAD = 1
+CSRC = os.path.join(ROOT, "newton_evaluation_nonlinear_b200", "csrc")
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="pn", choices=["pn", "reference"])
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--mode", default=None, help="jacobi|picard|quasi|newton (default: the workload's first)")
+    ap.add_argument("--all", action="store_true", help="one line per workload and mode (report runs)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--host-loop", action="store_true",
+                    help="host-driven convergence loop (plain kernel launches, e.g. for ncu) instead of the "
+                         "device-side CUDA graph loop")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# algorithmic cost model of one fused iteration launch (per sequence step)
+# ----------------------------------------------------------------------------
+
+def alg_bytes_per_step(prob) -> int:
+    """Bytes one iteration must move per (b, t): read the step input (u_t, gx_t or c_t), read
+    s^(i)_t (s^(i)_{t-1} is the previous step's row), write s^(i+1)_t; float32."""
+    rin = 3 if prob.cell == pi.CELL_GRU else 1
+    return 4 * (rin * prob.D + 2 * prob.D)
+
+
+def alg_flops_per_step(prob, mode) -> int:
+    R = 3 if prob.cell == pi.CELL_GRU else 1
+    f = 2 * R * prob.D * prob.D
+    if mode == pi.MODE_NEWTON:
+        f += 2 * prob.D * prob.D * (prob.D + 1)   # prefix chain [P|q] <- A [P|q]
+    return f
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cuh", ".cu")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(prob, mode):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current source."""
+    path = os.path.join(PROFILES, "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    e = d.get(f"{prob.name}:{pi.MODE_NAMES[mode]}")
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline / reference arm)
+# ----------------------------------------------------------------------------
+
+def cpu_sample(prob, mode, b_sample):
+    import oracle
+    m = oracle.Model.from_problem(prob)
+    x = np.ascontiguousarray(prob.x[:b_sample])
+    s0 = np.ascontiguousarray(prob.s0[:b_sample])
+    threads = oracle.default_threads(b_sample)
+    t0 = time.perf_counter()
+    _, it, _, _, _ = m.iterate(mode, x, s0, prob.iters_cap, prob.tol, nthreads=threads)
+    wall = time.perf_counter() - t0
+    return prob.T * b_sample / wall, wall, it, threads
+
+
+def cpu_baseline(prob, mode):
+    b_sample = max(1, min(prob.B, os.cpu_count() or 1))
+    v, wall, it, threads = cpu_sample(prob, mode, b_sample)
+    return {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"fp64 oracle {pi.MODE_NAMES[mode]} iteration (serial over t, threads over b) on the "
+                      f"first {b_sample} of {prob.B} sequences at full T={prob.T}: {it} iterations, "
+                      f"{wall:.1f} s wall"}
+
+
+def reference_arm(args, prob, mode, rank, world):
+    if rank != 0:
+        return
+    b_sample = max(1, min(prob.B, os.cpu_count() or 1))
+    for _ in range(args.warmup):
+        cpu_sample(prob, mode, b_sample)
+    walls, its = [], []
+    for _ in range(args.steps):
+        _, wall, it, threads = cpu_sample(prob, mode, b_sample)
+        walls.append(wall)
+        its.append(it)
+    tot = sum(walls)
+    value = prob.T * b_sample * args.steps / tot
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": prob.name, "mode": pi.MODE_NAMES[mode], "T": prob.T, "B": prob.B,
+                       "D": prob.D, "tol": prob.tol, "sample_sequences": b_sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"fp64 oracle {pi.MODE_NAMES[mode]} iteration on the first {b_sample} "
+                                       f"sequences at full T, {its[-1]} iterations per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------
+
+def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
+    import torch
+
+    import newton_evaluation_nonlinear_b200 as pn
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    solver = pn.Solver.from_problem(prob, stream=stream, device=dev)
+    if args.host_loop:
+        solver.set_option(pn.PN_OPT_DEVICE_LOOP, 0)
+    x = torch.from_numpy(prob.x).to(dev)
+    s0 = torch.from_numpy(prob.s0).to(dev)
+    states = torch.empty((prob.B, prob.T, prob.D), device=dev, dtype=torch.float32)
+    mi, tol = prob.iters_cap, prob.tol
+
+    for _ in range(max(3, args.warmup)):
+        _, iters, resid, st = solver.eval(x, s0, mode, mi, tol, states)
+    torch.cuda.synchronize(dev)
+    solver.reset_stats()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            _, iters, resid, st = solver.eval(x, s0, mode, mi, tol, states)
+        e1.record(stream)
+        barrier()
+    ms = e0.elapsed_time(e1)
+    stats = solver.stats()
+    if dist is not None:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    units = prob.T * prob.B * world * args.steps
+    value = units / (ms / 1e3)
+    launches_per_step = (iters + 1) + 2 + (0 if prob.cell == pi.CELL_EULER else 1)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": prob.name, "mode": pi.MODE_NAMES[mode], "cell": pi.CELL_NAMES[prob.cell],
+                       "D": prob.D, "d_in": prob.d_in, "T": prob.T, "B": prob.B, "tol": prob.tol,
+                       "max_iters": mi, "iters": iters, "final_resid": resid, "status": st,
+                       "parallelism": f"independent instances x{world}",
+                       "loop": "host" if args.host_loop else "device (CUDA graph WHILE node)",
+                       "l2": "inputs larger than L2 (x, u, two iterate buffers: "
+                             f"{(prob.x.nbytes + 3 * prob.B * prob.T * prob.D * 4) / 1e6:.0f} MB)"},
+            "clocks": clk.summary(), "gpu_launches": launches_per_step * args.steps}
+    if not with_extras:
+        solver.close()
+        return line
+
+    # roofline of the fused iteration kernel: CUDA events around back-to-back launches
+    n_l = max(10, 3 * (iters + 1))
+    kms = solver.time_iterations(mode, n_l)
+    in_graph_us = stats["iteration_ns"] / max(1, stats["iteration_launches"]) / 1e3
+    hbm, src = peaks()
+    bytes_launch = alg_bytes_per_step(prob) * prob.B * prob.T
+    achieved = bytes_launch / (kms / 1e3) / 1e9
+    traffic = traffic_from_profile(prob, mode)
+    line["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                        "frac": achieved / hbm, "traffic": traffic, "peak_source": src,
+                        "kernel": "fused iteration (cell + Jacobian + chunked scan + residual)",
+                        "alg_bytes_per_launch": bytes_launch, "launch_ms": kms,
+                        "in_graph_launch_us": in_graph_us,
+                        "fp32_tflops": alg_flops_per_step(prob, mode) * prob.B * prob.T / (kms / 1e3) / 1e12}
+
+    # end to end through the host-buffer entry point, copies inside the timed region
+    hx = torch.from_numpy(prob.x).pin_memory()
+    hs0 = torch.from_numpy(prob.s0).pin_memory()
+    hst = torch.empty((prob.B, prob.T, prob.D), dtype=torch.float32).pin_memory()
+    hxn, hs0n, hstn = hx.numpy(), hs0.numpy(), hst.numpy()
+    for _ in range(2):
+        solver.eval_host(hxn, hs0n, mode, mi, tol, hstn)
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        solver.eval_host(hxn, hs0n, mode, mi, tol, hstn)
+    e1.record(stream)
+    barrier()
+    ems = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ems], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    line["e2e"] = {"value": units / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(prob.x.nbytes + prob.s0.nbytes),
+                   "d2h_bytes_per_step": int(prob.B * prob.T * prob.D * 4), "ms_per_step": ems / args.steps}
+    solver.close()
+    return line
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        backend = "nccl" if args.impl == "pn" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        tdist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        jobs = []
+        if args.all:
+            for idx in range(5):
+                for m in pi.WORKLOAD_MODES[idx]:
+                    jobs.append((idx, m))
+        else:
+            m = pi.MODE_BY_NAME[args.mode] if args.mode else pi.WORKLOAD_MODES[args.workload][0]
+            jobs.append((args.workload, m))
+        for idx, mode in jobs:
+            prob = pi.benchmark_workload(idx)
+            if args.impl == "reference":
+                reference_arm(args, prob, mode, rank, world)
+                continue
+            line = bench_pn(args, prob, mode, rank, world, local_rank, dist)
+            if rank == 0:
+                if world == 1 and not args.no_cpu_baseline:
+                    line["cpu_baseline"] = cpu_baseline(prob, mode)
+                print(json.dumps(line), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -38,6 +38,12 @@
 
 #include <stddef.h>
 
+#if defined(__GNUC__)
+#define PN_API __attribute__((visibility("default")))
+#else
+#define PN_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -99,7 +105,7 @@ typedef struct {
  *   cuda_stream  a cudaStream_t (NULL = the legacy default stream).
  * Allocates every work buffer for (D, d_in, T, B) up front.  On error *out is
  * set to NULL and the message is available from pn_last_error(NULL). */
-pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
+PN_API pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
                     const float* params, size_t n_params, float eps,
                     void* cuda_stream);
 
@@ -114,7 +120,7 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
  *   iters_out, resid_out  host; receive the iteration count and r^(iters)
  *           (either may be NULL)
  * Returns PN_OK, PN_NOT_CONVERGED, or an error (see pn_status). */
-pn_status pn_eval(pn_handle h, const float* x, const float* s0, pn_mode mode,
+PN_API pn_status pn_eval(pn_handle h, const float* x, const float* s0, pn_mode mode,
                   int max_iters, float tol, float* states, int* iters_out,
                   float* resid_out);
 
@@ -122,13 +128,13 @@ pn_status pn_eval(pn_handle h, const float* x, const float* s0, pn_mode mode,
  * evaluates, and copies the states back into states_host, all on the handle's
  * stream (pinned host memory makes the copies asynchronous).  The device
  * buffers are allocated on the first call and reused. */
-pn_status pn_eval_host(pn_handle h, const float* x_host, const float* s0_host,
+PN_API pn_status pn_eval_host(pn_handle h, const float* x_host, const float* s0_host,
                        pn_mode mode, int max_iters, float tol,
                        float* states_host, int* iters_out, float* resid_out);
 
 /* Copy min(n, iters+1) residuals r^(0..iters) of the last evaluation into the
  * host array out; *n_written (may be NULL) receives the count. */
-pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written);
+PN_API pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written);
 
 /* Time the fused iteration kernel of `mode` alone: after a pn_eval on this
  * handle (its x, s0 and states must still be valid), launch exactly
@@ -136,25 +142,25 @@ pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written
  * stop rule, bracketed by CUDA events.  *avg_ms receives the mean duration per
  * launch.  The states buffer of that pn_eval is overwritten with later
  * iterates. */
-pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* avg_ms);
+PN_API pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* avg_ms);
 
-pn_status pn_get_stats(pn_handle h, pn_stats* out);
-pn_status pn_reset_stats(pn_handle h);
-pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
-pn_status pn_set_stream(pn_handle h, void* cuda_stream);
+PN_API pn_status pn_get_stats(pn_handle h, pn_stats* out);
+PN_API pn_status pn_reset_stats(pn_handle h);
+PN_API pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
+PN_API pn_status pn_set_stream(pn_handle h, void* cuda_stream);
 
 /* Shape queries (for the binding); each returns -1 for a NULL handle. */
-int pn_dim(pn_handle h, int which /* 0=D 1=d_in 2=T 3=B 4=cell */);
+PN_API int pn_dim(pn_handle h, int which /* 0=D 1=d_in 2=T 3=B 4=cell */);
 
 /* Last error message of this handle, or of the calling thread's last failed
  * pn_create when h is NULL.  Never NULL; "" when there was no error. */
-const char* pn_last_error(pn_handle h);
+PN_API const char* pn_last_error(pn_handle h);
 
 /* Release every device and host resource of the handle (NULL is a no-op). */
-void pn_destroy(pn_handle h);
+PN_API void pn_destroy(pn_handle h);
 
 /* Library version string. */
-const char* pn_version(void);
+PN_API const char* pn_version(void);
 
 #ifdef __cplusplus
 }

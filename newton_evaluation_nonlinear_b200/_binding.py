@@ -1,0 +1,252 @@
+"""ctypes binding of libpn (include/pn.h): argument marshalling only.
+
+Every computation happens inside libpn's CUDA kernels.  The module-level
+functions carry the C names (``pn_create``, ``pn_eval``, ...) and take plain
+integers for pointers and streams; :class:`Solver` wraps them for torch tensors.
+There is no fallback: if ``libpn.so`` is missing or fails to load, importing
+this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpn.so")
+
+PN_OK, PN_NOT_CONVERGED = 0, 1
+PN_ERR_INVALID, PN_ERR_NOMEM, PN_ERR_CUDA, PN_ERR_NONFINITE, PN_ERR_TIMEOUT = -1, -2, -3, -4, -5
+PN_CELL_TANH_RNN, PN_CELL_GRU, PN_CELL_EULER_TANH = 0, 1, 2
+PN_JACOBI, PN_PICARD, PN_QUASI, PN_NEWTON = 0, 1, 2, 3
+PN_OPT_WAIT_TIMEOUT_NS, PN_OPT_DEBUG_STALL_TICKET, PN_OPT_DEVICE_LOOP = 0, 1, 2
+PN_MAX_D_DIAG, PN_MAX_D_NEWTON = 256, 64
+
+STATUS_NAMES = {PN_OK: "PN_OK", PN_NOT_CONVERGED: "PN_NOT_CONVERGED", PN_ERR_INVALID: "PN_ERR_INVALID",
+                PN_ERR_NOMEM: "PN_ERR_NOMEM", PN_ERR_CUDA: "PN_ERR_CUDA",
+                PN_ERR_NONFINITE: "PN_ERR_NONFINITE", PN_ERR_TIMEOUT: "PN_ERR_TIMEOUT"}
+MODES = {"jacobi": PN_JACOBI, "picard": PN_PICARD, "quasi": PN_QUASI, "newton": PN_NEWTON}
+
+# Every symbol include/pn.h declares, with (restype, argtypes).
+_c_int, _c_float, _vp, _c_ll = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_longlong
+
+
+class pn_stats(ctypes.Structure):
+    _fields_ = [("iteration_launches", ctypes.c_longlong), ("iteration_ns", ctypes.c_longlong),
+                ("evals", ctypes.c_longlong)]
+
+
+SIGNATURES = {
+    "pn_create": (_c_int, [ctypes.POINTER(_vp), _c_int, _c_int, _c_int, _c_int, _c_int, _vp,
+                           ctypes.c_size_t, _c_float, _vp]),
+    "pn_eval": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_float, _vp, ctypes.POINTER(_c_int),
+                         ctypes.POINTER(_c_float)]),
+    "pn_eval_host": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_float, _vp, ctypes.POINTER(_c_int),
+                              ctypes.POINTER(_c_float)]),
+    "pn_get_residual_history": (_c_int, [_vp, _vp, _c_int, ctypes.POINTER(_c_int)]),
+    "pn_time_iterations": (_c_int, [_vp, _c_int, _c_int, ctypes.POINTER(_c_float)]),
+    "pn_get_stats": (_c_int, [_vp, ctypes.POINTER(pn_stats)]),
+    "pn_reset_stats": (_c_int, [_vp]),
+    "pn_set_option": (_c_int, [_vp, _c_int, _c_ll]),
+    "pn_set_stream": (_c_int, [_vp, _vp]),
+    "pn_dim": (_c_int, [_vp, _c_int]),
+    "pn_last_error": (ctypes.c_char_p, [_vp]),
+    "pn_destroy": (None, [_vp]),
+    "pn_version": (ctypes.c_char_p, []),
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m newton_evaluation_nonlinear_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+class PnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+# ----------------------------------------------------------------------------
+# C-named functions (plain ints for pointers/streams)
+# ----------------------------------------------------------------------------
+
+def pn_version() -> str:
+    return lib.pn_version().decode()
+
+
+def pn_last_error(h: Optional[int]) -> str:
+    return lib.pn_last_error(h).decode()
+
+
+def pn_create(cell: int, D: int, d_in: int, T: int, B: int, params: np.ndarray, eps: float = 0.0,
+              stream: int = 0) -> Tuple[int, Optional[int]]:
+    p = np.ascontiguousarray(params, dtype=np.float32).ravel()
+    h = _vp()
+    st = lib.pn_create(ctypes.byref(h), int(cell), int(D), int(d_in), int(T), int(B),
+                       p.ctypes.data, p.size, float(eps), stream or None)
+    return st, h.value
+
+
+def pn_eval(h: int, x_ptr: int, s0_ptr: int, mode: int, max_iters: int, tol: float,
+            states_ptr: int) -> Tuple[int, int, float]:
+    it, r = _c_int(-1), _c_float(float("nan"))
+    st = lib.pn_eval(h, x_ptr, s0_ptr, int(mode), int(max_iters), float(tol), states_ptr,
+                     ctypes.byref(it), ctypes.byref(r))
+    return st, it.value, r.value
+
+
+def pn_eval_host(h: int, x: np.ndarray, s0: np.ndarray, mode: int, max_iters: int, tol: float,
+                 states: np.ndarray) -> Tuple[int, int, float]:
+    for a in (x, s0, states):
+        if a.dtype != np.float32 or not a.flags.c_contiguous:
+            raise ValueError("host buffers must be C-contiguous float32")
+    it, r = _c_int(-1), _c_float(float("nan"))
+    st = lib.pn_eval_host(h, x.ctypes.data, s0.ctypes.data, int(mode), int(max_iters), float(tol),
+                          states.ctypes.data, ctypes.byref(it), ctypes.byref(r))
+    return st, it.value, r.value
+
+
+def pn_get_residual_history(h: int, n: int) -> Tuple[int, np.ndarray]:
+    out = np.zeros(max(int(n), 1), np.float32)
+    w = _c_int(0)
+    st = lib.pn_get_residual_history(h, out.ctypes.data, int(n), ctypes.byref(w))
+    return st, out[: w.value]
+
+
+def pn_time_iterations(h: int, mode: int, n_launches: int) -> Tuple[int, float]:
+    ms = _c_float(0.0)
+    st = lib.pn_time_iterations(h, int(mode), int(n_launches), ctypes.byref(ms))
+    return st, ms.value
+
+
+def pn_get_stats(h: int) -> Tuple[int, dict]:
+    s = pn_stats()
+    st = lib.pn_get_stats(h, ctypes.byref(s))
+    return st, {"iteration_launches": s.iteration_launches, "iteration_ns": s.iteration_ns,
+                "evals": s.evals}
+
+
+def pn_reset_stats(h: int) -> int:
+    return lib.pn_reset_stats(h)
+
+
+def pn_set_option(h: int, opt: int, value: int) -> int:
+    return lib.pn_set_option(h, int(opt), int(value))
+
+
+def pn_set_stream(h: int, stream: int) -> int:
+    return lib.pn_set_stream(h, stream or None)
+
+
+def pn_dim(h: int, which: int) -> int:
+    return lib.pn_dim(h, int(which))
+
+
+def pn_destroy(h: Optional[int]) -> None:
+    lib.pn_destroy(h)
+
+
+# ----------------------------------------------------------------------------
+# torch-facing wrapper
+# ----------------------------------------------------------------------------
+
+class Solver:
+    """One libpn handle: a cell with fixed shape (D, d_in, T, B) and parameters.
+
+    ``eval`` takes CUDA float32 tensors (x [B,T,d_in], s0 [B,D]) and returns
+    ``(states, iters, resid, status)``; statuses PN_OK and PN_NOT_CONVERGED
+    return normally, every error raises :class:`PnError`.
+    """
+
+    def __init__(self, cell: int, D: int, d_in: int, T: int, B: int, params, eps: float = 0.0,
+                 stream=None, device=None):
+        import torch
+        self.cell, self.D, self.d_in, self.T, self.B = int(cell), int(D), int(d_in), int(T), int(B)
+        self.device = torch.device(device if device is not None else "cuda")
+        with torch.cuda.device(self.device):
+            if stream is None:
+                stream = torch.cuda.current_stream(self.device)
+            self._stream = stream
+            st, h = pn_create(cell, D, d_in, T, B, np.asarray(params), eps, int(stream.cuda_stream))
+        if st != PN_OK:
+            raise PnError(st, pn_last_error(None))
+        self.h = h
+
+    @classmethod
+    def from_problem(cls, prob, stream=None, device=None) -> "Solver":
+        return cls(prob.cell, prob.D, prob.d_in, prob.T, prob.B, prob.params, prob.eps, stream, device)
+
+    def _check(self, st: int) -> int:
+        if st < 0:
+            raise PnError(st, pn_last_error(self.h))
+        return st
+
+    def eval(self, x, s0, mode, max_iters: Optional[int] = None, tol: float = 1e-5, states=None):
+        import torch
+        mode = MODES[mode] if isinstance(mode, str) else int(mode)
+        max_iters = self.T if max_iters is None else int(max_iters)
+        if states is None:
+            states = torch.empty((self.B, self.T, self.D), device=x.device, dtype=torch.float32)
+        for name, t, shape in (("x", x, (self.B, self.T, self.d_in)), ("s0", s0, (self.B, self.D)),
+                               ("states", states, (self.B, self.T, self.D))):
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
+                raise ValueError(f"{name} must be a contiguous CUDA float32 tensor of shape {shape}")
+        st, it, r = pn_eval(self.h, x.data_ptr(), s0.data_ptr(), mode, max_iters, tol, states.data_ptr())
+        self._check(st)
+        return states, it, r, st
+
+    def eval_host(self, x: np.ndarray, s0: np.ndarray, mode, max_iters: Optional[int] = None,
+                  tol: float = 1e-5, states: Optional[np.ndarray] = None):
+        mode = MODES[mode] if isinstance(mode, str) else int(mode)
+        max_iters = self.T if max_iters is None else int(max_iters)
+        if states is None:
+            states = np.empty((self.B, self.T, self.D), np.float32)
+        st, it, r = pn_eval_host(self.h, x, s0, mode, max_iters, tol, states)
+        self._check(st)
+        return states, it, r, st
+
+    def residual_history(self, n: int = 1 << 16) -> np.ndarray:
+        st, h = pn_get_residual_history(self.h, n)
+        self._check(st)
+        return h
+
+    def time_iterations(self, mode, n_launches: int) -> float:
+        mode = MODES[mode] if isinstance(mode, str) else int(mode)
+        st, ms = pn_time_iterations(self.h, mode, n_launches)
+        self._check(st)
+        return ms
+
+    def stats(self) -> dict:
+        st, s = pn_get_stats(self.h)
+        self._check(st)
+        return s
+
+    def reset_stats(self) -> None:
+        self._check(pn_reset_stats(self.h))
+
+    def set_option(self, opt: int, value: int) -> None:
+        self._check(pn_set_option(self.h, opt, value))
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            pn_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

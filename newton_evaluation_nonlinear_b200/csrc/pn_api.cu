@@ -1,0 +1,767 @@
+// pn_api.cu -- the C ABI of libpn (declared in include/pn.h).
+//
+// Host side of the solver: argument validation, weight packing, device buffer
+// ownership, the CUDA graph that holds the device-side convergence loop (a
+// conditional WHILE node around the fused iteration kernel), and the
+// host-driven loop used when the device loop is switched off.
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "pn_aux.cuh"
+#include "pn_dispatch.cuh"
+
+using namespace pn;
+
+namespace {
+
+thread_local std::string g_create_error;
+
+int padded_width(int D) {
+  int dp = 4;
+  while (dp < D) dp <<= 1;
+  return dp;
+}
+
+int cell_R(int cell) { return cell == PN_CELL_GRU ? 3 : 1; }
+
+struct Family {
+  KInfo k[4];        // per mode (jacobi, picard, quasi, newton); fn == nullptr if unsupported
+  int ngroups[4];
+  int nchunks[4];
+  int ntiles[4];     // ngroups * B * nchunks
+  int grid[4];       // persistent CTAs: a multiple of ngroups, at most ntiles
+};
+
+}  // namespace
+
+struct pn_ctx {
+  int cell = 0, D = 0, d_in = 0, T = 0, B = 0, DP = 0, device = 0;
+  float eps = 0.0f;
+  cudaStream_t stream = nullptr;
+  Family fam{};
+  // device memory
+  float* wt_diag = nullptr;    // [ngroups][DP][R*G] transposed recurrent weights
+  float* wt_dense = nullptr;   // [DP][R*DP] transposed + [R][DP][DP] row-major
+  float* bhn = nullptr;        // [DP]
+  float* proj_w = nullptr;     // U [D][d_in] or W_ih [3D][d_in]
+  float* proj_b = nullptr;     // b [D] or b_ih + [b_hr; b_hz; 0] [3D]
+  float* xin = nullptr;        // hoisted step inputs [B][T][R*D]
+  float* buf1 = nullptr;       // second iterate buffer [B][T][D]
+  unsigned* flags = nullptr;
+  float* agg = nullptr;
+  float* pref = nullptr;
+  size_t agg_floats = 0, pref_floats = 0, nflags = 0;
+  Ctrl* ctrl = nullptr;
+  Args* args = nullptr;
+  float* hist = nullptr;
+  // host pinned mirrors
+  Args* args_h = nullptr;
+  Ctrl* ctrl_h = nullptr;
+  // host-buffer evaluation staging (allocated on first pn_eval_host)
+  float* hx = nullptr;
+  float* hs0 = nullptr;
+  float* hst = nullptr;
+  // graphs, one per mode, built on first use
+  cudaGraph_t graph[4] = {nullptr, nullptr, nullptr, nullptr};
+  cudaGraphExec_t exec[4] = {nullptr, nullptr, nullptr, nullptr};
+  // options
+  long long timeout_ns = 1000000000LL;
+  int stall_ticket = -1;
+  int device_loop = 1;
+  long long evals = 0;
+  int last_iters = -1;
+  std::string err;
+};
+
+namespace {
+
+pn_status fail(pn_ctx* h, pn_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  if (h) h->err = buf;
+  else g_create_error = buf;
+  return st;
+}
+
+#define PN_CUDA(h, call)                                                                  \
+  do {                                                                                    \
+    cudaError_t e_ = (call);                                                              \
+    if (e_ != cudaSuccess)                                                                \
+      return fail((h), e_ == cudaErrorMemoryAllocation ? PN_ERR_NOMEM : PN_ERR_CUDA,      \
+                  "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__, __LINE__); \
+  } while (0)
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) cudaSetDevice(dev);
+    else prev = -1;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+template <class T>
+pn_status dalloc(pn_ctx* h, T** p, size_t count) {
+  *p = nullptr;
+  if (count == 0) count = 1;
+  cudaError_t e = cudaMalloc((void**)p, count * sizeof(T));
+  if (e != cudaSuccess) {
+    *p = nullptr;
+    return fail(h, PN_ERR_NOMEM, "cudaMalloc of %zu bytes failed: %s", count * sizeof(T),
+                cudaGetErrorString(e));
+  }
+  return PN_OK;
+}
+
+void free_all(pn_ctx* h) {
+  for (int m = 0; m < 4; ++m) {
+    if (h->exec[m]) cudaGraphExecDestroy(h->exec[m]);
+    if (h->graph[m]) cudaGraphDestroy(h->graph[m]);
+    h->exec[m] = nullptr;
+    h->graph[m] = nullptr;
+  }
+  float** fbufs[] = {&h->wt_diag, &h->wt_dense, &h->bhn, &h->proj_w, &h->proj_b, &h->xin,
+                     &h->buf1,    &h->agg,      &h->pref, &h->hist,  &h->hx,     &h->hs0, &h->hst};
+  for (float** p : fbufs) {
+    if (*p) cudaFree(*p);
+    *p = nullptr;
+  }
+  if (h->flags) cudaFree(h->flags);
+  if (h->ctrl) cudaFree(h->ctrl);
+  if (h->args) cudaFree(h->args);
+  if (h->args_h) cudaFreeHost(h->args_h);
+  if (h->ctrl_h) cudaFreeHost(h->ctrl_h);
+  h->flags = nullptr;
+  h->ctrl = nullptr;
+  h->args = nullptr;
+  h->args_h = nullptr;
+  h->ctrl_h = nullptr;
+}
+
+// Recurrent weight block q of the cell, element [row][col] (rows, cols < D).
+float w_block(const pn_ctx* h, const float* params, int q, int row, int col) {
+  const int D = h->D;
+  if (h->cell == PN_CELL_GRU) return params[(size_t)3 * D * h->d_in + ((size_t)q * D + row) * D + col];
+  return params[(size_t)row * D + col];
+}
+
+IterParams make_params(const pn_ctx* h, int mode) {
+  IterParams P{};
+  const bool dense = (mode == PN_NEWTON);
+  P.wt = dense ? h->wt_dense : h->wt_diag;
+  P.bhn = h->bhn;
+  P.xin = h->xin;
+  P.buf1 = h->buf1;
+  P.flags = h->flags;
+  P.agg = h->agg;
+  P.pref = h->pref;
+  P.ctrl = h->ctrl;
+  P.args = h->args;
+  P.hist = h->hist;
+  P.eps = h->eps;
+  P.D = h->D;
+  P.d_in = h->d_in;
+  P.T = h->T;
+  P.B = h->B;
+  P.ngroups = h->fam.ngroups[mode];
+  P.nchunks = h->fam.nchunks[mode];
+  P.tiles_per_group = h->B * h->fam.nchunks[mode];
+  const int G = h->fam.k[mode].G;
+  P.agg_stride = dense ? G * (G + 1) : 2 * G;
+  P.pref_stride = G;
+  P.cond = 0;
+  return P;
+}
+
+unsigned grid_1d(size_t n, int threads, unsigned cap) {
+  size_t g = (n + threads - 1) / threads;
+  if (g < 1) g = 1;
+  if (g > cap) g = cap;
+  return (unsigned)g;
+}
+
+// Kernels that run before the loop: projection (tanh RNN, GRU) and init.
+struct PreLaunch {
+  bool has_proj = false;
+  dim3 proj_grid;
+  int M = 0, N = 0, K = 0;
+  unsigned init_grid = 1, fin_grid = 1;
+};
+
+PreLaunch pre_launch(const pn_ctx* h) {
+  PreLaunch p;
+  p.has_proj = (h->cell != PN_CELL_EULER_TANH);
+  p.M = h->B * h->T;
+  p.N = cell_R(h->cell) * h->D;
+  p.K = h->d_in;
+  p.proj_grid = dim3((unsigned)((p.M + kProjTile - 1) / kProjTile), (unsigned)((p.N + kProjTile - 1) / kProjTile));
+  const size_t n = (size_t)h->B * h->T * h->D;
+  p.init_grid = grid_1d(n, 256, 148u * 16u);
+  p.fin_grid = grid_1d(n / 4 + 1, 256, 148u * 16u);
+  return p;
+}
+
+pn_status build_graph(pn_ctx* h, int mode) {
+  if (h->exec[mode]) return PN_OK;
+  const KInfo& ki = h->fam.k[mode];
+  const PreLaunch pl = pre_launch(h);
+  cudaGraph_t g = nullptr;
+  PN_CUDA(h, cudaGraphCreate(&g, 0));
+  cudaGraphNode_t prev = nullptr, node = nullptr;
+  auto add_kernel = [&](cudaGraph_t graph, const void* fn, dim3 grid, dim3 block, size_t smem,
+                        void** kargs, cudaGraphNode_t* dep, cudaGraphNode_t* out) -> cudaError_t {
+    cudaKernelNodeParams kp{};
+    kp.func = const_cast<void*>(fn);
+    kp.gridDim = grid;
+    kp.blockDim = block;
+    kp.sharedMemBytes = (unsigned)smem;
+    kp.kernelParams = kargs;
+    kp.extra = nullptr;
+    return cudaGraphAddKernelNode(out, graph, dep, dep ? 1 : 0, &kp);
+  };
+  cudaError_t e = cudaSuccess;
+  // 1. input projection
+  const Args* a_d = h->args;
+  if (pl.has_proj) {
+    const float* w = h->proj_w;
+    const float* bb = h->proj_b;
+    float* o = h->xin;
+    int M = pl.M, N = pl.N, K = pl.K;
+    void* kargs[] = {(void*)&a_d, (void*)&w, (void*)&bb, (void*)&o, (void*)&M, (void*)&N, (void*)&K};
+    e = add_kernel(g, (const void*)&proj_kernel, pl.proj_grid, dim3(256), 0, kargs, nullptr, &node);
+    if (e != cudaSuccess) goto fail_graph;
+    prev = node;
+  }
+  {
+    // 2. init
+    Ctrl* c = h->ctrl;
+    int D = h->D, T = h->T, B = h->B;
+    void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&D, (void*)&T, (void*)&B};
+    e = add_kernel(g, (const void*)&init_kernel, dim3(pl.init_grid), dim3(256), 0, kargs,
+                   prev ? &prev : nullptr, &node);
+    if (e != cudaSuccess) goto fail_graph;
+    prev = node;
+  }
+  {
+    // 3. WHILE (condition set to 0 by the iteration kernel's last CTA)
+    cudaGraphConditionalHandle cond;
+    e = cudaGraphConditionalHandleCreate(&cond, g, 1u, cudaGraphCondAssignDefault);
+    if (e != cudaSuccess) goto fail_graph;
+    cudaGraphNodeParams cp{};
+    cp.type = cudaGraphNodeTypeConditional;
+    cp.conditional.handle = cond;
+    cp.conditional.type = cudaGraphCondTypeWhile;
+    cp.conditional.size = 1;
+    e = cudaGraphAddNode(&node, g, &prev, 1, &cp);
+    if (e != cudaSuccess) goto fail_graph;
+    cudaGraph_t body = cp.conditional.phGraph_out[0];
+    IterParams P = make_params(h, mode);
+    P.cond = cond;
+    void* kargs[] = {(void*)&P};
+    cudaGraphNode_t knode;
+    e = add_kernel(body, ki.fn, dim3((unsigned)h->fam.grid[mode]), dim3(ki.nt), ki.smem, kargs,
+                   nullptr, &knode);
+    if (e != cudaSuccess) goto fail_graph;
+    prev = node;
+  }
+  {
+    // 4. result copy
+    const Ctrl* c = h->ctrl;
+    const float* b1 = h->buf1;
+    size_t n = (size_t)h->B * h->T * h->D;
+    void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&b1, (void*)&n};
+    e = add_kernel(g, (const void*)&finish_kernel, dim3(pl.fin_grid), dim3(256), 0, kargs, &prev, &node);
+    if (e != cudaSuccess) goto fail_graph;
+  }
+  e = cudaGraphInstantiate(&h->exec[mode], g, 0);
+  if (e != cudaSuccess) goto fail_graph;
+  h->graph[mode] = g;
+  return PN_OK;
+fail_graph:
+  cudaGraphDestroy(g);
+  h->exec[mode] = nullptr;
+  return fail(h, PN_ERR_CUDA, "building the CUDA graph for mode %d failed: %s", mode, cudaGetErrorString(e));
+}
+
+pn_status launch_iter(pn_ctx* h, int mode) {
+  const KInfo& ki = h->fam.k[mode];
+  IterParams P = make_params(h, mode);
+  void* kargs[] = {(void*)&P};
+  PN_CUDA(h, cudaLaunchKernel(ki.fn, dim3((unsigned)h->fam.grid[mode]), dim3(ki.nt), kargs, ki.smem, h->stream));
+  return PN_OK;
+}
+
+pn_status launch_pre(pn_ctx* h) {
+  const PreLaunch pl = pre_launch(h);
+  const Args* a_d = h->args;
+  if (pl.has_proj) {
+    const float* w = h->proj_w;
+    const float* bb = h->proj_b;
+    float* o = h->xin;
+    int M = pl.M, N = pl.N, K = pl.K;
+    void* kargs[] = {(void*)&a_d, (void*)&w, (void*)&bb, (void*)&o, (void*)&M, (void*)&N, (void*)&K};
+    PN_CUDA(h, cudaLaunchKernel((const void*)&proj_kernel, pl.proj_grid, dim3(256), kargs, 0, h->stream));
+  }
+  Ctrl* c = h->ctrl;
+  int D = h->D, T = h->T, B = h->B;
+  void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&D, (void*)&T, (void*)&B};
+  PN_CUDA(h, cudaLaunchKernel((const void*)&init_kernel, dim3(pl.init_grid), dim3(256), kargs, 0, h->stream));
+  return PN_OK;
+}
+
+pn_status launch_finish(pn_ctx* h) {
+  const PreLaunch pl = pre_launch(h);
+  const Args* a_d = h->args;
+  const Ctrl* c = h->ctrl;
+  const float* b1 = h->buf1;
+  size_t n = (size_t)h->B * h->T * h->D;
+  void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&b1, (void*)&n};
+  PN_CUDA(h, cudaLaunchKernel((const void*)&finish_kernel, dim3(pl.fin_grid), dim3(256), kargs, 0, h->stream));
+  return PN_OK;
+}
+
+pn_status check_device_ptr(pn_ctx* h, const void* p, const char* name) {
+  if (!p) return fail(h, PN_ERR_INVALID, "%s is NULL", name);
+  if (((uintptr_t)p) & 15u) return fail(h, PN_ERR_INVALID, "%s must be 16-byte aligned", name);
+  cudaPointerAttributes at{};
+  cudaError_t e = cudaPointerGetAttributes(&at, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(h, PN_ERR_INVALID, "%s is not a CUDA pointer (%s)", name, cudaGetErrorString(e));
+  }
+  if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+    return fail(h, PN_ERR_INVALID, "%s must be device memory", name);
+  if (at.type == cudaMemoryTypeDevice && at.device != h->device)
+    return fail(h, PN_ERR_INVALID, "%s lives on device %d, the handle on device %d", name, at.device, h->device);
+  return PN_OK;
+}
+
+pn_status validate_mode(pn_ctx* h, int mode, int max_iters, float tol) {
+  if (mode < PN_JACOBI || mode > PN_NEWTON) return fail(h, PN_ERR_INVALID, "mode %d out of range", mode);
+  if (!h->fam.k[mode].fn)
+    return fail(h, PN_ERR_INVALID, "mode %d is not supported for D=%d (newton needs D <= %d)", mode, h->D,
+                PN_MAX_D_NEWTON);
+  if (max_iters < 0) return fail(h, PN_ERR_INVALID, "max_iters must be >= 0");
+  if (!(tol >= 0.0f) || !std::isfinite(tol)) return fail(h, PN_ERR_INVALID, "tol must be finite and >= 0");
+  return PN_OK;
+}
+
+pn_status reset_flags_if_needed(pn_ctx* h) {
+  // Flags carry the 30-bit launch epoch; clear them long before it wraps.
+  if (h->ctrl_h->epoch > (1u << 29)) {
+    PN_CUDA(h, cudaMemsetAsync(h->flags, 0, h->nflags * sizeof(unsigned), h->stream));
+    PN_CUDA(h, cudaMemsetAsync(&h->ctrl->epoch, 0, sizeof(unsigned), h->stream));
+    h->ctrl_h->epoch = 0;
+  }
+  return PN_OK;
+}
+
+// The loop body shared by pn_eval and pn_eval_host: args already point at
+// device buffers.
+pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
+  pn_status st = reset_flags_if_needed(h);
+  if (st != PN_OK) return st;
+  h->args_h->use_cond = h->device_loop ? 1 : 0;
+  PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
+  if (h->device_loop) {
+    st = build_graph(h, mode);
+    if (st != PN_OK) return st;
+    PN_CUDA(h, cudaGraphLaunch(h->exec[mode], h->stream));
+  } else {
+    st = launch_pre(h);
+    if (st != PN_OK) return st;
+    for (long it = 0;; ++it) {
+      st = launch_iter(h, mode);
+      if (st != PN_OK) return st;
+      PN_CUDA(h, cudaMemcpyAsync(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, h->stream));
+      PN_CUDA(h, cudaStreamSynchronize(h->stream));
+      if (h->ctrl_h->status != kRunning) break;
+      if (it > (long)h->args_h->max_iters + 2)
+        return fail(h, PN_ERR_CUDA, "host loop did not stop after max_iters launches");
+    }
+    st = launch_finish(h);
+    if (st != PN_OK) return st;
+  }
+  PN_CUDA(h, cudaMemcpyAsync(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, h->stream));
+  PN_CUDA(h, cudaStreamSynchronize(h->stream));
+  const Ctrl& c = *h->ctrl_h;
+  h->last_iters = c.final_iter;
+  h->evals += 1;
+  if (iters_out) *iters_out = c.final_iter;
+  if (resid_out) *resid_out = c.final_resid;
+  if (c.status == PN_ERR_TIMEOUT)
+    return fail(h, PN_ERR_TIMEOUT, "a look-back wait gave up after %lld ns (tile ticket %d)",
+                (long long)h->args_h->timeout_ns, c.timeout_ticket);
+  if (c.status == PN_ERR_NONFINITE)
+    return fail(h, PN_ERR_NONFINITE, "residual became non-finite at iteration %d", c.final_iter);
+  if (c.status == kRunning) return fail(h, PN_ERR_CUDA, "the convergence loop did not finish");
+  h->err.clear();
+  return (pn_status)c.status;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pn_version(void) { return "libpn 0.1 (sm_100a)"; }
+
+const char* pn_last_error(pn_handle h) {
+  if (!h) return g_create_error.c_str();
+  return h->err.c_str();
+}
+
+pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B, const float* params,
+                    size_t n_params, float eps, void* cuda_stream) {
+  g_create_error.clear();
+  if (!out) return fail(nullptr, PN_ERR_INVALID, "out is NULL");
+  *out = nullptr;
+  if (cell < PN_CELL_TANH_RNN || cell > PN_CELL_EULER_TANH) return fail(nullptr, PN_ERR_INVALID, "unknown cell %d", (int)cell);
+  if (D < 1 || D > PN_MAX_D_DIAG) return fail(nullptr, PN_ERR_INVALID, "D=%d outside 1..%d", D, PN_MAX_D_DIAG);
+  if (d_in < 1) return fail(nullptr, PN_ERR_INVALID, "d_in must be >= 1");
+  if (cell == PN_CELL_EULER_TANH && d_in != D) return fail(nullptr, PN_ERR_INVALID, "the Euler cell needs d_in == D");
+  if (T < 1 || B < 1) return fail(nullptr, PN_ERR_INVALID, "T and B must be >= 1");
+  if ((long long)B * T > INT_MAX) return fail(nullptr, PN_ERR_INVALID, "B*T must fit in int");
+  if (!params) return fail(nullptr, PN_ERR_INVALID, "params is NULL");
+  if (!std::isfinite(eps)) return fail(nullptr, PN_ERR_INVALID, "eps must be finite");
+  size_t need = 0;
+  if (cell == PN_CELL_TANH_RNN) need = (size_t)D * D + (size_t)D * d_in + D;
+  else if (cell == PN_CELL_GRU) need = 3 * (size_t)D * d_in + 3 * (size_t)D * D + 6 * (size_t)D;
+  else need = (size_t)D * D;
+  if (n_params != need) return fail(nullptr, PN_ERR_INVALID, "n_params=%zu, the cell needs %zu", n_params, need);
+
+  pn_ctx* h = new pn_ctx();
+  h->cell = cell;
+  h->D = D;
+  h->d_in = d_in;
+  h->T = T;
+  h->B = B;
+  h->eps = eps;
+  h->DP = padded_width(D);
+  h->stream = (cudaStream_t)cuda_stream;
+  if (cudaGetDevice(&h->device) != cudaSuccess) {
+    delete h;
+    return fail(nullptr, PN_ERR_CUDA, "no CUDA device");
+  }
+  const int R = cell_R(cell);
+  const int DP = h->DP;
+  const size_t BT = (size_t)B * T;
+
+  // kernels and tilings
+  for (int m = 0; m < 4; ++m) {
+    KInfo ki = (m == PN_NEWTON && DP > PN_MAX_D_NEWTON) ? KInfo{nullptr, 0, 0, 0, 0} : lookup(cell, m, DP);
+    h->fam.k[m] = ki;
+    if (!ki.fn) continue;
+    h->fam.ngroups[m] = (m == PN_NEWTON) ? 1 : (D + ki.G - 1) / ki.G;
+    if (h->fam.ngroups[m] > kMaxGroups) {
+      delete h;
+      return fail(nullptr, PN_ERR_INVALID, "D=%d needs %d channel groups (max %d)", D, h->fam.ngroups[m], kMaxGroups);
+    }
+    h->fam.nchunks[m] = (T + ki.L - 1) / ki.L;
+    h->fam.ntiles[m] = h->fam.ngroups[m] * B * h->fam.nchunks[m];
+    if (ki.smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.smem);
+      if (e != cudaSuccess) {
+        delete h;
+        return fail(nullptr, PN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      }
+    }
+    int per_sm = 0, nsm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ki.fn, ki.nt, ki.smem) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || per_sm < 1) {
+      delete h;
+      return fail(nullptr, PN_ERR_CUDA, "occupancy query failed for mode %d (D=%d)", m, D);
+    }
+    {
+      const int ng = h->fam.ngroups[m];
+      long long want = (long long)per_sm * nsm;
+      want = std::max<long long>(ng, (want / ng) * ng);
+      h->fam.grid[m] = (int)std::min<long long>(want, h->fam.ntiles[m]);
+    }
+    const size_t G = (size_t)ki.G;
+    const size_t nt = (size_t)h->fam.ntiles[m];
+    const size_t aggf = nt * ((m == PN_NEWTON) ? G * (G + 1) : 2 * G);
+    h->agg_floats = std::max(h->agg_floats, aggf);
+    h->pref_floats = std::max(h->pref_floats, nt * G);
+    h->nflags = std::max(h->nflags, nt);
+  }
+
+  pn_status st = PN_OK;
+#define PN_TRY(expr)           \
+  do {                         \
+    st = (expr);               \
+    if (st != PN_OK) goto bad; \
+  } while (0)
+  {
+    // weights, packed on the host
+    const int Gd = h->fam.k[PN_QUASI].G;
+    const int ng = (D + Gd - 1) / Gd;
+    std::vector<float> wt((size_t)ng * DP * R * Gd, 0.0f);
+    for (int g = 0; g < ng; ++g)
+      for (int k = 0; k < D; ++k)
+        for (int q = 0; q < R; ++q)
+          for (int j = 0; j < Gd; ++j) {
+            const int row = g * Gd + j;
+            if (row < D) wt[(((size_t)g * DP + k) * R + q) * Gd + j] = w_block(h, params, q, row, k);
+          }
+    std::vector<float> wd((size_t)DP * R * DP + (size_t)R * DP * DP, 0.0f);
+    for (int k = 0; k < D; ++k)
+      for (int q = 0; q < R; ++q)
+        for (int j = 0; j < D; ++j) wd[((size_t)k * R + q) * DP + j] = w_block(h, params, q, j, k);
+    float* wr = wd.data() + (size_t)DP * R * DP;
+    for (int q = 0; q < R; ++q)
+      for (int i = 0; i < D; ++i)
+        for (int k = 0; k < D; ++k) wr[((size_t)q * DP + i) * DP + k] = w_block(h, params, q, i, k);
+    std::vector<float> bhn(DP, 0.0f);
+    std::vector<float> pw, pb;
+    if (cell == PN_CELL_TANH_RNN) {
+      pw.assign(params + (size_t)D * D, params + (size_t)D * D + (size_t)D * d_in);
+      pb.assign(params + (size_t)D * D + (size_t)D * d_in, params + need);
+    } else if (cell == PN_CELL_GRU) {
+      const float* W_ih = params;
+      const float* b_ih = params + 3 * (size_t)D * d_in + 3 * (size_t)D * D;
+      const float* b_hh = b_ih + 3 * D;
+      pw.assign(W_ih, W_ih + 3 * (size_t)D * d_in);
+      pb.resize(3 * (size_t)D);
+      for (int c = 0; c < D; ++c) {
+        pb[c] = b_ih[c] + b_hh[c];               // r: b_ir + b_hr
+        pb[D + c] = b_ih[D + c] + b_hh[D + c];   // z: b_iz + b_hz
+        pb[2 * D + c] = b_ih[2 * D + c];         // n: b_in (b_hn stays inside r * (...))
+        bhn[c] = b_hh[2 * D + c];
+      }
+    }
+    PN_TRY(dalloc(h, &h->wt_diag, wt.size()));
+    PN_TRY(dalloc(h, &h->wt_dense, wd.size()));
+    PN_TRY(dalloc(h, &h->bhn, bhn.size()));
+    if (cudaMemcpy(h->wt_diag, wt.data(), wt.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(h->wt_dense, wd.data(), wd.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(h->bhn, bhn.data(), bhn.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess) {
+      st = fail(h, PN_ERR_CUDA, "weight upload failed");
+      goto bad;
+    }
+    if (!pw.empty()) {
+      PN_TRY(dalloc(h, &h->proj_w, pw.size()));
+      PN_TRY(dalloc(h, &h->proj_b, pb.size()));
+      PN_TRY(dalloc(h, &h->xin, BT * R * D));
+      if (cudaMemcpy(h->proj_w, pw.data(), pw.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+          cudaMemcpy(h->proj_b, pb.data(), pb.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess) {
+        st = fail(h, PN_ERR_CUDA, "weight upload failed");
+        goto bad;
+      }
+    }
+    PN_TRY(dalloc(h, &h->buf1, BT * D));
+    PN_TRY(dalloc(h, &h->flags, h->nflags));
+    PN_TRY(dalloc(h, &h->agg, h->agg_floats));
+    PN_TRY(dalloc(h, &h->pref, h->pref_floats));
+    PN_TRY(dalloc(h, &h->ctrl, 1));
+    PN_TRY(dalloc(h, &h->args, 1));
+    PN_TRY(dalloc(h, &h->hist, kHistCap));
+    if (cudaMemset(h->flags, 0, h->nflags * sizeof(unsigned)) != cudaSuccess ||
+        cudaMemset(h->ctrl, 0, sizeof(Ctrl)) != cudaSuccess ||
+        cudaMemset(h->hist, 0, kHistCap * sizeof(float)) != cudaSuccess) {
+      st = fail(h, PN_ERR_CUDA, "memset failed");
+      goto bad;
+    }
+    if (cudaMallocHost((void**)&h->args_h, sizeof(Args)) != cudaSuccess ||
+        cudaMallocHost((void**)&h->ctrl_h, sizeof(Ctrl)) != cudaSuccess) {
+      st = fail(h, PN_ERR_NOMEM, "pinned host allocation failed");
+      goto bad;
+    }
+    memset(h->args_h, 0, sizeof(Args));
+    memset(h->ctrl_h, 0, sizeof(Ctrl));
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+      st = fail(h, PN_ERR_CUDA, "device synchronisation after create failed");
+      goto bad;
+    }
+  }
+#undef PN_TRY
+  *out = h;
+  return PN_OK;
+bad:
+  g_create_error = h->err;
+  free_all(h);
+  delete h;
+  return st;
+}
+
+pn_status pn_eval(pn_handle h, const float* x, const float* s0, pn_mode mode, int max_iters, float tol,
+                  float* states, int* iters_out, float* resid_out) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  DeviceGuard dg(h->device);
+  pn_status st = validate_mode(h, mode, max_iters, tol);
+  if (st != PN_OK) return st;
+  if ((st = check_device_ptr(h, x, "x")) != PN_OK) return st;
+  if ((st = check_device_ptr(h, s0, "s0")) != PN_OK) return st;
+  if ((st = check_device_ptr(h, states, "states")) != PN_OK) return st;
+  Args& a = *h->args_h;
+  a.x = x;
+  a.s0 = s0;
+  a.states = states;
+  a.tol = tol;
+  a.max_iters = max_iters;
+  a.timeout_ns = h->timeout_ns;
+  a.stall_ticket = h->stall_ticket;
+  return run_eval(h, mode, iters_out, resid_out);
+}
+
+pn_status pn_eval_host(pn_handle h, const float* x_host, const float* s0_host, pn_mode mode, int max_iters,
+                       float tol, float* states_host, int* iters_out, float* resid_out) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  DeviceGuard dg(h->device);
+  pn_status st = validate_mode(h, mode, max_iters, tol);
+  if (st != PN_OK) return st;
+  if (!x_host || !s0_host || !states_host) return fail(h, PN_ERR_INVALID, "NULL host buffer");
+  const size_t nx = (size_t)h->B * h->T * h->d_in;
+  const size_t ns = (size_t)h->B * h->T * h->D;
+  const size_t n0 = (size_t)h->B * h->D;
+  if (!h->hx) {
+    if ((st = dalloc(h, &h->hx, nx)) != PN_OK) return st;
+    if ((st = dalloc(h, &h->hs0, n0)) != PN_OK) return st;
+    if ((st = dalloc(h, &h->hst, ns)) != PN_OK) return st;
+  }
+  PN_CUDA(h, cudaMemcpyAsync(h->hx, x_host, nx * sizeof(float), cudaMemcpyHostToDevice, h->stream));
+  PN_CUDA(h, cudaMemcpyAsync(h->hs0, s0_host, n0 * sizeof(float), cudaMemcpyHostToDevice, h->stream));
+  Args& a = *h->args_h;
+  a.x = h->hx;
+  a.s0 = h->hs0;
+  a.states = h->hst;
+  a.tol = tol;
+  a.max_iters = max_iters;
+  a.timeout_ns = h->timeout_ns;
+  a.stall_ticket = h->stall_ticket;
+  st = run_eval(h, mode, iters_out, resid_out);
+  if (st < 0 && st != PN_ERR_NONFINITE) return st;
+  cudaError_t e = cudaMemcpyAsync(states_host, h->hst, ns * sizeof(float), cudaMemcpyDeviceToHost, h->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
+  if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "copying states to the host failed: %s", cudaGetErrorString(e));
+  return st;
+}
+
+pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  if (n < 0 || (n > 0 && !out)) return fail(h, PN_ERR_INVALID, "bad output buffer");
+  DeviceGuard dg(h->device);
+  int avail = h->last_iters < 0 ? 0 : std::min(h->last_iters + 1, kHistCap);
+  int cnt = std::min(n, avail);
+  if (cnt > 0) {
+    PN_CUDA(h, cudaMemcpyAsync(out, h->hist, cnt * sizeof(float), cudaMemcpyDeviceToHost, h->stream));
+    PN_CUDA(h, cudaStreamSynchronize(h->stream));
+  }
+  if (n_written) *n_written = cnt;
+  return PN_OK;
+}
+
+pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* avg_ms) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  if (n_launches < 1 || !avg_ms) return fail(h, PN_ERR_INVALID, "n_launches must be >= 1 and avg_ms non-NULL");
+  DeviceGuard dg(h->device);
+  pn_status st = validate_mode(h, mode, 0, 0.0f);
+  if (st != PN_OK) return st;
+  if (!h->args_h->states) return fail(h, PN_ERR_INVALID, "call pn_eval on this handle first");
+  // every launch re-evaluates the same iterate: r <= +inf stops the counter
+  h->args_h->tol = INFINITY;
+  h->args_h->max_iters = INT_MAX;
+  h->args_h->use_cond = 0;
+  PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
+  cudaEvent_t e0, e1;
+  PN_CUDA(h, cudaEventCreate(&e0));
+  PN_CUDA(h, cudaEventCreate(&e1));
+  st = PN_OK;
+  cudaError_t ce = cudaEventRecord(e0, h->stream);
+  for (int i = 0; i < n_launches && ce == cudaSuccess && st == PN_OK; ++i) st = launch_iter(h, mode);
+  if (ce == cudaSuccess) ce = cudaEventRecord(e1, h->stream);
+  if (ce == cudaSuccess) ce = cudaEventSynchronize(e1);
+  float ms = 0.0f;
+  if (ce == cudaSuccess) ce = cudaEventElapsedTime(&ms, e0, e1);
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  if (st != PN_OK) return st;
+  if (ce != cudaSuccess) return fail(h, PN_ERR_CUDA, "timing failed: %s", cudaGetErrorString(ce));
+  PN_CUDA(h, cudaMemcpy(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost));
+  if (h->ctrl_h->error) return fail(h, PN_ERR_TIMEOUT, "a look-back wait gave up during timing");
+  *avg_ms = ms / (float)n_launches;
+  return PN_OK;
+}
+
+pn_status pn_get_stats(pn_handle h, pn_stats* out) {
+  if (!h || !out) return fail(h, PN_ERR_INVALID, "NULL argument");
+  DeviceGuard dg(h->device);
+  PN_CUDA(h, cudaStreamSynchronize(h->stream));
+  PN_CUDA(h, cudaMemcpy(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost));
+  out->iteration_launches = (long long)h->ctrl_h->launches;
+  out->iteration_ns = (long long)h->ctrl_h->kernel_ns;
+  out->evals = h->evals;
+  return PN_OK;
+}
+
+pn_status pn_reset_stats(pn_handle h) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  DeviceGuard dg(h->device);
+  PN_CUDA(h, cudaStreamSynchronize(h->stream));
+  unsigned long long z[2] = {0ull, 0ull};
+  PN_CUDA(h, cudaMemcpy(&h->ctrl->kernel_ns, z, 2 * sizeof(unsigned long long), cudaMemcpyHostToDevice));
+  h->evals = 0;
+  return PN_OK;
+}
+
+pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  switch (opt) {
+    case PN_OPT_WAIT_TIMEOUT_NS:
+      if (value < 1000) return fail(h, PN_ERR_INVALID, "timeout must be >= 1000 ns");
+      h->timeout_ns = value;
+      return PN_OK;
+    case PN_OPT_DEBUG_STALL_TICKET:
+      if (value < -1 || value > INT_MAX) return fail(h, PN_ERR_INVALID, "bad ticket");
+      h->stall_ticket = (int)value;
+      return PN_OK;
+    case PN_OPT_DEVICE_LOOP:
+      if (value != 0 && value != 1) return fail(h, PN_ERR_INVALID, "device loop option is 0 or 1");
+      h->device_loop = (int)value;
+      return PN_OK;
+  }
+  return fail(h, PN_ERR_INVALID, "unknown option %d", (int)opt);
+}
+
+pn_status pn_set_stream(pn_handle h, void* cuda_stream) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  h->stream = (cudaStream_t)cuda_stream;
+  return PN_OK;
+}
+
+int pn_dim(pn_handle h, int which) {
+  if (!h) return -1;
+  switch (which) {
+    case 0: return h->D;
+    case 1: return h->d_in;
+    case 2: return h->T;
+    case 3: return h->B;
+    case 4: return h->cell;
+    default: return -1;
+  }
+}
+
+void pn_destroy(pn_handle h) {
+  if (!h) return;
+  {
+    DeviceGuard dg(h->device);
+    if (h->stream) cudaStreamSynchronize(h->stream);
+    else cudaDeviceSynchronize();
+    free_all(h);
+  }
+  delete h;
+}
+
+}  // extern "C"

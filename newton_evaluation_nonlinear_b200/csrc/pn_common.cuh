@@ -1,0 +1,202 @@
+// pn_common.cuh -- shared device-side definitions of libpn (sm_100a).
+//
+// Control block, kernel parameter blocks, memory-ordering helpers for the
+// single-pass chunked scan with decoupled look-back, and bounded waits.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pn.h"
+
+namespace pn {
+
+constexpr int kRunning = 100;          // ctrl.status while a loop is in flight
+constexpr int kHistCap = 65537;        // residual history entries kept per handle
+constexpr unsigned kFlagAgg = 1u;      // tile published its aggregate
+constexpr unsigned kFlagPrefix = 2u;   // tile published its inclusive prefix (a state)
+constexpr int kMaxGroups = 8;          // channel groups of the diagonal-family kernels (D / G)
+
+// Device control block: one per handle, in device memory.
+struct Ctrl {
+  int iter;            // index i of the iterate s^(i) the next launch evaluates
+  int status;          // kRunning, or the final pn_status of the loop
+  int error;           // sticky device error (PN_ERR_TIMEOUT), 0 if none
+  int final_iter;      // iteration count of the result
+  float final_resid;   // r^(final_iter)
+  unsigned resid_bits; // running max of |F| for the current launch (float bits)
+  unsigned ticket[kMaxGroups];  // tile tickets handed out per channel group, current launch
+  unsigned done;       // CTAs finished in the current launch
+  unsigned epoch;      // launch sequence number; tags the look-back flags
+  int timeout_ticket;  // ticket whose wait gave up (diagnostics), -1 if none
+  unsigned long long t_start;    // min %globaltimer at CTA entry, current launch
+  unsigned long long kernel_ns;  // summed launch durations
+  unsigned long long launches;   // fused iteration launches
+};
+
+// Per-call arguments, written by the host before each evaluation.
+struct Args {
+  const float* x;      // caller x [B][T][d_in]
+  const float* s0;     // caller s0 [B][D]
+  float* states;       // caller states [B][T][D] (iterate buffer 0)
+  float tol;
+  int max_iters;
+  long long timeout_ns;
+  int stall_ticket;    // -1 = off
+  int use_cond;        // 1 inside the device loop graph
+};
+
+// Fixed per-handle parameters of the fused iteration kernels.
+struct IterParams {
+  const float* wt;     // recurrent weights, pre-packed per group: [ngroups][DP][R*G]
+  const float* wdiag;  // diagonal entries per gate: [R][DP] (quasi mode)
+  const float* bhn;    // GRU b_hn [DP] (zero-padded); unused otherwise
+  const float* xin;    // per-step cell input: u [B][T][D] (tanh), gx [B][T][3D] (GRU); NULL for Euler
+  float* buf1;         // iterate buffer 1 [B][T][D]
+  unsigned* flags;     // look-back flags, one per tile
+  float* agg;          // look-back aggregates, agg_stride floats per tile
+  float* pref;         // look-back inclusive prefixes (states), pref_stride floats per tile
+  Ctrl* ctrl;
+  Args* args;
+  float* hist;         // residual history [kHistCap]
+  float eps;           // Euler step
+  int D, d_in, T, B;
+  int ngroups, nchunks;
+  int tiles_per_group;  // B * nchunks: tickets of one channel group
+  int agg_stride, pref_stride;
+  cudaGraphConditionalHandle cond;
+};
+
+// ---------------------------------------------------------------------------
+// memory ordering
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_volatile(const int* p) { return *(const volatile int*)p; }
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Look-back, phase A (called by all 32 lanes of one warp).
+// The tile at chunk `chunk` of a scan chain looks at its predecessors
+// chunk-1, chunk-2, ... (flag index k - d*stride for distance d) 32 at a time,
+// one lane per predecessor, until it finds the nearest one that has published
+// its inclusive prefix; chunk -1 counts as a published prefix (the state s0).
+// It waits (bounded) until every predecessor nearer than that one has at least
+// published its aggregate.  Returns the number of aggregate-only tiles between
+// this tile and that prefix, or -1 when it gave up (timeout, or another CTA's
+// error).
+__device__ __forceinline__ int lookback_find_prefix(const unsigned* flags, size_t k, size_t stride,
+                                                    int chunk, unsigned epoch, Ctrl* ctrl,
+                                                    long long timeout_ns) {
+  const int lane = threadIdx.x & 31;
+  int n_agg = 0;
+  int base = chunk - 1;   // nearest chunk of this window
+  const unsigned long long t0 = globaltimer();
+  unsigned spins = 0;
+  while (true) {
+    const int p = base - lane;
+    bool valid = true, pfx = true;
+    if (p >= 0) {
+      const unsigned f = ld_acquire(flags + (k - (size_t)(chunk - p) * stride));
+      valid = ((f >> 2) == epoch) && (f & 3u);
+      pfx = valid && ((f & 3u) == kFlagPrefix);
+    }
+    const unsigned pm = __ballot_sync(0xffffffffu, pfx);
+    const unsigned vm = __ballot_sync(0xffffffffu, valid);
+    const int nearest = pm ? (__ffs(pm) - 1) : 32;
+    const unsigned need = (nearest >= 31) ? 0xffffffffu : ((2u << nearest) - 1u);
+    if ((vm & need) == need) {
+      if (nearest < 32) return n_agg + nearest;
+      n_agg += 32;
+      base -= 32;
+      continue;
+    }
+    int give_up = 0;
+    ++spins;
+    if (lane == 0) {
+      if (ld_volatile(&ctrl->error)) give_up = 1;
+      else if (((spins & 15u) == 0u) && (long long)(globaltimer() - t0) > timeout_ns) {
+        if (atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT) == 0) ctrl->timeout_ticket = (int)k;
+        give_up = 1;
+      }
+    }
+    if (__shfl_sync(0xffffffffu, give_up, 0)) return -1;
+    if (spins > 64u) __nanosleep(32);
+  }
+}
+
+__device__ __forceinline__ unsigned make_flag(unsigned epoch, unsigned state) {
+  return (epoch << 2) | state;
+}
+
+// |F| values are >= 0, so their float bits order like unsigned integers, and
+// NaN (0x7fc00000 and up) compares above +Inf: an integer max propagates NaN.
+__device__ __forceinline__ unsigned abs_bits(float v) { return __float_as_uint(fabsf(v)); }
+
+__device__ __forceinline__ unsigned warp_max_u32(unsigned v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float sigmoidf_acc(float v) { return 1.0f / (1.0f + expf(-v)); }
+
+// ---------------------------------------------------------------------------
+// end-of-launch bookkeeping, run by the last CTA to finish
+// ---------------------------------------------------------------------------
+// Every CTA calls this once, after all of its global writes.  The last CTA
+// takes the stop decision for iterate i = ctrl->iter:
+//   non-finite r -> PN_ERR_NONFINITE; r <= tol -> PN_OK;
+//   i == max_iters -> PN_NOT_CONVERGED; otherwise continue with i+1.
+__device__ __forceinline__ void finish_launch(const IterParams& P, const Args& A,
+                                              unsigned epoch, int& is_last_smem) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    unsigned prev = atomicAdd(&P.ctrl->done, 1u);
+    is_last_smem = (prev == gridDim.x - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!is_last_smem || threadIdx.x != 0) return;
+  __threadfence();
+  Ctrl* c = P.ctrl;
+  const int i = c->iter;
+  const float r = __uint_as_float(atomicAdd(&c->resid_bits, 0u));
+  const int err = ld_volatile(&c->error);
+  if (i < kHistCap) P.hist[i] = r;
+  int st = kRunning;
+  if (err) st = err;
+  else if (!(r <= 3.402823466e38f)) st = PN_ERR_NONFINITE;
+  else if (r <= A.tol) st = PN_OK;
+  else if (i >= A.max_iters) st = PN_NOT_CONVERGED;
+  if (st != kRunning) {
+    c->status = st;
+    c->final_iter = i;
+    c->final_resid = r;
+    if (A.use_cond) cudaGraphSetConditional(P.cond, 0u);
+  } else {
+    c->iter = i + 1;
+  }
+  c->resid_bits = 0u;
+#pragma unroll
+  for (int g = 0; g < kMaxGroups; ++g) c->ticket[g] = 0u;
+  c->done = 0u;
+  c->epoch = epoch + 1u;
+  const unsigned long long t1 = globaltimer();
+  const unsigned long long t0 = c->t_start;
+  if (t1 > t0) c->kernel_ns += t1 - t0;
+  c->launches += 1ull;
+  c->t_start = ~0ull;
+  __threadfence();
+}
+
+}  // namespace pn

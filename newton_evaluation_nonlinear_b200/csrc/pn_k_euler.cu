@@ -1,0 +1,6 @@
+// pn_k_euler.cu -- fused iteration kernels instantiated for the euler cell.
+#include "pn_dispatch.cuh"
+
+namespace pn {
+KInfo lookup_euler(int mode, int DP) { return lookup_cell<PN_CELL_EULER_TANH>(mode, DP); }
+}  // namespace pn

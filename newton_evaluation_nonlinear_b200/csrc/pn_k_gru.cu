@@ -1,0 +1,6 @@
+// pn_k_gru.cu -- fused iteration kernels instantiated for the gru cell.
+#include "pn_dispatch.cuh"
+
+namespace pn {
+KInfo lookup_gru(int mode, int DP) { return lookup_cell<PN_CELL_GRU>(mode, DP); }
+}  // namespace pn

@@ -1,0 +1,6 @@
+// pn_k_tanh.cu -- fused iteration kernels instantiated for the tanh cell.
+#include "pn_dispatch.cuh"
+
+namespace pn {
+KInfo lookup_tanh(int mode, int DP) { return lookup_cell<PN_CELL_TANH_RNN>(mode, DP); }
+}  // namespace pn

@@ -216,6 +216,10 @@ def random_problem(seed: int, cell: int, D: int, d_in: Optional[int] = None, T: 
                    eps=(eps if cell == CELL_EULER else 0.0), tol=tol, max_iters=max_iters)
 
 
+WORKLOAD_MODES = {0: (MODE_NEWTON,), 1: (MODE_QUASI,), 2: (MODE_NEWTON,), 3: (MODE_QUASI,),
+                  4: (MODE_PICARD, MODE_JACOBI, MODE_QUASI)}
+
+
 def workload_names() -> List[str]:
     return ["tanh_rnn_D4_T1024_B1_newton", "tanh_rnn_D64_T16384_B16_quasi",
             "tanh_rnn_D16_T8192_B64_newton", "gru_D32_T65536_B8_quasi",

@@ -1,0 +1,61 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol include/pn.h
+declares, and rejects bad arguments before touching a device."""
+import os
+import re
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pn.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"PN_API\s+[\w\s\*]+?\b(pn_\w+)\s*\(", src)))
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for n in ("pn_create", "pn_eval", "pn_eval_host", "pn_destroy", "pn_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import ctypes
+    import newton_evaluation_nonlinear_b200 as pn
+    lib = ctypes.CDLL(pn.LIB_PATH)
+    for n in _declared():
+        assert hasattr(lib, n), n
+    assert set(_declared()) <= set(pn.SIGNATURES)
+
+
+def test_no_cuda_runtime_symbols_leak():
+    import subprocess
+    import newton_evaluation_nonlinear_b200 as pn
+    out = subprocess.run(["nm", "-D", "--defined-only", pn.LIB_PATH], capture_output=True, text=True).stdout
+    exported = [l.split()[-1] for l in out.splitlines() if " T " in l]
+    assert exported and all(n.startswith("pn_") for n in exported), exported
+
+
+def test_argument_validation_without_gpu():
+    import newton_evaluation_nonlinear_b200 as pn
+    p = np.zeros(4 * 4 + 4 * 3 + 4, np.float32)
+    cases = [
+        (dict(cell=9, D=4, d_in=3), "unknown cell"),
+        (dict(cell=0, D=0, d_in=3), "D=0"),
+        (dict(cell=0, D=300, d_in=3), "D=300"),
+        (dict(cell=2, D=4, d_in=3), "Euler"),
+        (dict(cell=0, D=4, d_in=5), "n_params"),
+    ]
+    for kw, needle in cases:
+        st, h = pn.pn_create(kw["cell"], kw["D"], kw["d_in"], 16, 2, p)
+        assert st == pn.PN_ERR_INVALID and h is None
+        assert needle in pn.pn_last_error(None)
+    st, h = pn.pn_create(0, 4, 3, 0, 2, p)
+    assert st == pn.PN_ERR_INVALID
+    assert pn.pn_dim(None, 0) == -1
+    assert pn.pn_last_error(None) != ""
+    st, _, _ = pn.pn_eval(None, 0, 0, 0, 1, 1e-5, 0)
+    assert st == pn.PN_ERR_INVALID
+    pn.pn_destroy(None)
+    assert pn.pn_version().startswith("libpn")

@@ -1,0 +1,241 @@
+"""GPU parity: libpn's CUDA path against the fp64 oracle, through the C ABI.
+
+For every cell and mode, on seeded inputs that span several tiles and a ragged
+tail, the states must match the oracle's sequential evaluation to a normwise
+relative error of 1e-4, and the iteration count must equal the oracle's serial
+iteration with the same tol (exactly, unless some oracle residual lies within
+1% of tol, where fp32 rounding may legitimately move one iteration).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import pn_inputs as pi
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 1e-4          # normwise max|s_gpu - s_ref| / max|s_ref|
+
+
+def _pn():
+    import newton_evaluation_nonlinear_b200 as pn   # raises if libpn.so is missing
+    return pn
+
+
+def _run(prob, mode, tol=None, max_iters=None, device_loop=1):
+    import torch
+    pn = _pn()
+    solver = pn.Solver.from_problem(prob)
+    solver.set_option(pn.PN_OPT_DEVICE_LOOP, device_loop)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    tol = prob.tol if tol is None else tol
+    mi = prob.iters_cap if max_iters is None else max_iters
+    states, it, r, st = solver.eval(x, s0, mode, mi, tol)
+    hist = solver.residual_history()
+    out = states.cpu().numpy()
+    solver.close()
+    return out, it, r, st, hist
+
+
+def _relerr(a, ref):
+    den = max(float(np.abs(ref).max()), 1e-30)
+    return float(np.abs(a.astype(np.float64) - ref).max()) / den
+
+
+def _check_against_oracle(prob, mode, tol=None, max_iters=None, device_loop=1):
+    """tol defaults to prob.tol * max(1, max|s|): an fp32 iterate assembled by a parallel scan carries
+    rounding of a few ulp(|s|) per step, so an absolute tol below ~1e-6 |s| would sit on the fp32
+    floor (the Euler drift reaches |s| ~ 20 on these inputs; the tanh and GRU states stay within 1)."""
+    mi = prob.iters_cap if max_iters is None else max_iters
+    m = oracle.Model.from_problem(prob)
+    seq = m.sequential(prob.x, prob.s0)
+    tol = prob.tol * max(1.0, float(np.abs(seq).max())) if tol is None else tol
+    s_or, it_or, r_or, st_or, hist_or = m.iterate(mode, prob.x, prob.s0, mi, tol)
+    s, it, r, st, hist = _run(prob, mode, tol, mi, device_loop)
+    assert np.isfinite(s).all()
+    margin = float(np.min(np.abs(hist_or / tol - 1.0))) if tol > 0 else 1.0
+    if margin > 1e-2:
+        assert it == it_or, (prob.name, mode, it, it_or, hist[:it + 1], hist_or)
+        assert st == st_or
+    else:
+        assert abs(it - it_or) <= 1
+    # same iterate as the oracle's serial iteration (fp32 vs fp64 arithmetic only)
+    if it == it_or:
+        assert _relerr(s, s_or) <= REL_TOL, _relerr(s, s_or)
+    if st == oracle.OK:
+        # the GPU's distance to the sequential states is the oracle iterate's own iteration error
+        # plus fp32 rounding
+        assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq)), (_relerr(s, seq), _relerr(s_or, seq))
+    # residual history: fp32 residuals track the fp64 ones
+    n = min(len(hist), len(hist_or))
+    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=1e-2, atol=5e-6)
+    return it, s
+
+
+CELLS = [pi.CELL_TANH_RNN, pi.CELL_GRU, pi.CELL_EULER]
+DIAG_MODES = [pi.MODE_JACOBI, pi.MODE_PICARD, pi.MODE_QUASI]
+
+
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("mode", DIAG_MODES + [pi.MODE_NEWTON])
+@pytest.mark.parametrize("D,T,B", [(1, 5, 1), (3, 70, 2), (4, 300, 3), (7, 129, 2), (16, 517, 2),
+                                   (33, 200, 2), (64, 133, 3)])
+def test_small_shapes(cell, mode, D, T, B):
+    if mode == pi.MODE_PICARD and cell != pi.CELL_EULER:
+        # A~ = I is only a contraction for near-identity dynamics (page §2.2.3); on the RNN cells the
+        # not-yet-converged tail grows geometrically until causality reaches it, so keep T short.
+        T = min(T, 12)
+    d_in = D if cell == pi.CELL_EULER else max(1, D - 1)
+    prob = pi.random_problem(1000 + 7 * D + T, cell, D, d_in, T=T, B=B, rho=0.6, eps=0.05,
+                             s0_scale=0.3, tol=1e-5)
+    if mode == pi.MODE_JACOBI:
+        prob.max_iters = T
+    _check_against_oracle(prob, mode)
+
+
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("mode", DIAG_MODES)
+@pytest.mark.parametrize("D", [100, 256])
+def test_wide_states(cell, mode, D):
+    T = 12 if (mode == pi.MODE_PICARD and cell != pi.CELL_EULER) else 150
+    prob = pi.random_problem(77 + D, cell, D, D, T=T, B=2, rho=0.6, eps=0.05, s0_scale=0.2, tol=1e-5)
+    _check_against_oracle(prob, mode)
+
+
+def test_picard_divergence_is_reported():
+    """Picard on a tanh RNN far from the identity: the tail grows until it overflows; the loop must
+    stop with PN_ERR_NONFINITE (or run out of iterations), never hang or return garbage as PN_OK."""
+    import torch
+    pn = _pn()
+    prob = pi.random_problem(13, pi.CELL_TANH_RNN, 8, 8, T=600, B=2, rho=0.6, s0_scale=0.3)
+    solver = pn.Solver.from_problem(prob)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    try:
+        _, it, r, st = solver.eval(x, s0, "picard", prob.T, 1e-6)
+        assert st == pn.PN_NOT_CONVERGED or it > 100
+    except pn.PnError as e:
+        assert e.status == pn.PN_ERR_NONFINITE
+    solver.close()
+
+
+@pytest.mark.parametrize("mode", [pi.MODE_QUASI, pi.MODE_NEWTON])
+def test_host_loop_matches_device_loop(mode):
+    prob = pi.random_problem(5, pi.CELL_TANH_RNN, 16, 16, T=700, B=3, rho=0.7, tol=1e-6)
+    a = _run(prob, mode, device_loop=1)
+    b = _run(prob, mode, device_loop=0)
+    assert a[1] == b[1]
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[4], b[4])
+
+
+def test_repeatable_bitwise():
+    prob = pi.random_problem(6, pi.CELL_GRU, 32, 32, T=1000, B=4, rho=0.9, tol=1e-6)
+    a = _run(prob, pi.MODE_QUASI)
+    b = _run(prob, pi.MODE_QUASI)
+    np.testing.assert_array_equal(a[0], b[0])
+    assert a[1] == b[1]
+
+
+def test_edge_cases():
+    import torch
+    pn = _pn()
+    prob = pi.random_problem(8, pi.CELL_TANH_RNN, 8, 5, T=100, B=2, rho=0.5, s0_scale=0.4)
+    solver = pn.Solver.from_problem(prob)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    m = oracle.Model.from_problem(prob)
+    # max_iters = 0: states are s0 broadcast, resid is r^(0)
+    states, it, r, st = solver.eval(x, s0, "quasi", 0, 1e-9)
+    assert (it, st) == (0, pn.PN_NOT_CONVERGED)
+    np.testing.assert_array_equal(states.cpu().numpy(), np.repeat(prob.s0[:, None, :], prob.T, 1))
+    _, r0 = m.residual(prob.x, prob.s0, np.repeat(prob.s0[:, None, :], prob.T, 1))
+    assert abs(r - r0) <= 1e-6 * max(1.0, r0)
+    # huge tol: converged at iteration 0
+    states, it, r, st = solver.eval(x, s0, "newton", 50, 1e9)
+    assert (it, st) == (0, pn.PN_OK)
+    # NaN input -> PN_ERR_NONFINITE, and the handle keeps working
+    bad = x.clone()
+    bad[1, 50, 2] = float("nan")
+    with pytest.raises(pn.PnError) as e:
+        solver.eval(bad, s0, "quasi", 20, 1e-6)
+    assert e.value.status == pn.PN_ERR_NONFINITE
+    states, it, r, st = solver.eval(x, s0, "quasi", prob.T, 1e-6)
+    assert st == pn.PN_OK and np.isfinite(states.cpu().numpy()).all()
+    # invalid arguments are rejected before any launch
+    st2, _, _ = pn.pn_eval(solver.h, 0, s0.data_ptr(), pn.PN_QUASI, 5, 1e-5, states.data_ptr())
+    assert st2 == pn.PN_ERR_INVALID
+    host = np.zeros((prob.B, prob.T, prob.d_in), np.float32)
+    st2, _, _ = pn.pn_eval(solver.h, host.ctypes.data, s0.data_ptr(), pn.PN_QUASI, 5, 1e-5, states.data_ptr())
+    assert st2 == pn.PN_ERR_INVALID
+    st2, _, _ = pn.pn_eval(solver.h, x.data_ptr(), s0.data_ptr(), 7, 5, 1e-5, states.data_ptr())
+    assert st2 == pn.PN_ERR_INVALID
+    st2, _, _ = pn.pn_eval(solver.h, x.data_ptr(), s0.data_ptr(), pn.PN_QUASI, -1, 1e-5, states.data_ptr())
+    assert st2 == pn.PN_ERR_INVALID
+    st2, _, _ = pn.pn_eval(solver.h, x.data_ptr() + 4, s0.data_ptr(), pn.PN_QUASI, 5, 1e-5, states.data_ptr())
+    assert st2 == pn.PN_ERR_INVALID   # misaligned
+    solver.close()
+
+
+def test_newton_rejects_wide_state():
+    import torch
+    pn = _pn()
+    prob = pi.random_problem(9, pi.CELL_EULER, 100, T=20, B=1)
+    solver = pn.Solver.from_problem(prob)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    with pytest.raises(pn.PnError) as e:
+        solver.eval(x, s0, "newton", 5, 1e-5)
+    assert e.value.status == pn.PN_ERR_INVALID
+    solver.close()
+
+
+def test_bounded_wait_times_out_and_recovers():
+    """A tile that never publishes (test hook) makes its successor's bounded wait run out:
+    the call returns PN_ERR_TIMEOUT and the context stays usable."""
+    import torch
+    pn = _pn()
+    prob = pi.random_problem(10, pi.CELL_TANH_RNN, 64, 64, T=2000, B=2, rho=0.5)
+    solver = pn.Solver.from_problem(prob)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    solver.set_option(pn.PN_OPT_WAIT_TIMEOUT_NS, 20_000_000)   # 20 ms
+    solver.set_option(pn.PN_OPT_DEBUG_STALL_TICKET, 0)
+    for mode in ("quasi", "newton"):
+        with pytest.raises(pn.PnError) as e:
+            solver.eval(x, s0, mode, 10, 1e-6)
+        assert e.value.status == pn.PN_ERR_TIMEOUT
+    solver.set_option(pn.PN_OPT_DEBUG_STALL_TICKET, -1)
+    states, it, r, st = solver.eval(x, s0, "quasi", prob.T, 1e-6)
+    assert st == pn.PN_OK
+    seq = oracle.Model.from_problem(prob).sequential(prob.x, prob.s0)
+    assert _relerr(states.cpu().numpy(), seq) <= REL_TOL
+    solver.close()
+
+
+def test_eval_host_matches_eval():
+    pn = _pn()
+    prob = pi.random_problem(11, pi.CELL_GRU, 32, 32, T=900, B=3, rho=0.8, tol=1e-6)
+    a = _run(prob, pi.MODE_QUASI)
+    solver = pn.Solver.from_problem(prob)
+    states, it, r, st = solver.eval_host(prob.x, prob.s0, "quasi", prob.T, prob.tol)
+    solver.close()
+    assert it == a[1]
+    np.testing.assert_array_equal(states, a[0])
+
+
+def test_stats_and_timing():
+    import torch
+    pn = _pn()
+    prob = pi.random_problem(12, pi.CELL_TANH_RNN, 64, 64, T=4096, B=4, rho=0.7, tol=1e-5)
+    solver = pn.Solver.from_problem(prob)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    solver.reset_stats()
+    _, it, _, _ = solver.eval(x, s0, "quasi", prob.T, prob.tol)
+    s = solver.stats()
+    assert s["iteration_launches"] == it + 1 and s["iteration_ns"] > 0 and s["evals"] == 1
+    ms = solver.time_iterations("quasi", 5)
+    assert 0.0 < ms < 1000.0
+    solver.close()
