@@ -26,7 +26,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -116,25 +115,41 @@ def traffic_from_profile(prob, mode):
 # ----------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """nvidia-smi sampling (read-only) of the SM clock and clock-event reasons every 20 ms, started
+    before the warm-up; samples whose timestamp falls inside [mark_start, mark_end] are the ones
+    taken during the timed region."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.t0 = self.t1 = None
+        self.lines = []
 
     def __enter__(self):
+        import subprocess
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)   # let it start sampling before the timed region
         except Exception:
             self.proc = None
         return self
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+        time.sleep(0.05)
+
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -145,22 +160,29 @@ class ClockSampler:
             self.lines = [l for l in out.splitlines() if l.strip()]
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        import datetime
+        rows = []
+        for l in self.lines:
             parts = [p.strip() for p in l.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 7:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[3:7]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+        inside = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= (self.t1 or 0)]
+        window = inside
+        if not window and rows and self.t0 is not None:   # region shorter than the sampling period
+            window = sorted(rows, key=lambda r: abs(r[0] - 0.5 * (self.t0 + (self.t1 or self.t0))))[:2]
+        reasons = set()
+        for r in window:
+            for n, v in zip(self.NAMES, r[3]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median([r[1] for r in window]) if window else None,
+                "sm_max_mhz": window[0][2] if window else None, "reasons": sorted(reasons),
+                "samples": len(inside), "nearest_used": bool(window) and not inside}
 
 
 # ----------------------------------------------------------------------------
@@ -246,11 +268,13 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         barrier()
+        clk.mark_start()
         e0.record(stream)
         for _ in range(args.steps):
             _, iters, resid, st = solver.eval(x, s0, mode, mi, tol, states)
         e1.record(stream)
         barrier()
+        clk.mark_end()
     ms = e0.elapsed_time(e1)
     stats = solver.stats()
     if dist is not None:

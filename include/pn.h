@@ -78,7 +78,11 @@ typedef enum {
   /* 1 (default): the convergence loop runs on the device inside a CUDA graph
    * (conditional WHILE node); 0: the host launches one iteration at a time and
    * reads the stop decision back after each. */
-  PN_OPT_DEVICE_LOOP = 2
+  PN_OPT_DEVICE_LOOP = 2,
+  /* 1 (default where available): the diagonal-mode kernels form the cell's
+   * recurrent matvec on the tensor cores (3 TF32 passes, fp32-level accuracy;
+   * D = 32, or D = 64 for the tanh RNN and Euler cells); 0: FP32 FMA. */
+  PN_OPT_TENSOR_CORES = 3
 } pn_option;
 
 /* Per-handle counters, cumulative since pn_create (or pn_reset_stats). */
@@ -148,6 +152,12 @@ PN_API pn_status pn_get_stats(pn_handle h, pn_stats* out);
 PN_API pn_status pn_reset_stats(pn_handle h);
 PN_API pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
 PN_API pn_status pn_set_stream(pn_handle h, void* cuda_stream);
+
+/* Evaluate the activations the cell kernels use, element-wise, on device
+ * arrays: which = 0 gives tanh(x), 1 gives 1 / (1 + exp(-x)).  x and y are
+ * device float32 arrays of n elements (they may alias); the work is ordered
+ * on cuda_stream and the call synchronises it.  For accuracy tests. */
+PN_API pn_status pn_activation(int which, const float* x, float* y, long long n, void* cuda_stream);
 
 /* Shape queries (for the binding); each returns -1 for a NULL handle. */
 PN_API int pn_dim(pn_handle h, int which /* 0=D 1=d_in 2=T 3=B 4=cell */);

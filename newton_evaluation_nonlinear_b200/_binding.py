@@ -21,7 +21,7 @@ PN_OK, PN_NOT_CONVERGED = 0, 1
 PN_ERR_INVALID, PN_ERR_NOMEM, PN_ERR_CUDA, PN_ERR_NONFINITE, PN_ERR_TIMEOUT = -1, -2, -3, -4, -5
 PN_CELL_TANH_RNN, PN_CELL_GRU, PN_CELL_EULER_TANH = 0, 1, 2
 PN_JACOBI, PN_PICARD, PN_QUASI, PN_NEWTON = 0, 1, 2, 3
-PN_OPT_WAIT_TIMEOUT_NS, PN_OPT_DEBUG_STALL_TICKET, PN_OPT_DEVICE_LOOP = 0, 1, 2
+PN_OPT_WAIT_TIMEOUT_NS, PN_OPT_DEBUG_STALL_TICKET, PN_OPT_DEVICE_LOOP, PN_OPT_TENSOR_CORES = 0, 1, 2, 3
 PN_MAX_D_DIAG, PN_MAX_D_NEWTON = 256, 64
 
 STATUS_NAMES = {PN_OK: "PN_OK", PN_NOT_CONVERGED: "PN_NOT_CONVERGED", PN_ERR_INVALID: "PN_ERR_INVALID",
@@ -52,6 +52,7 @@ SIGNATURES = {
     "pn_set_option": (_c_int, [_vp, _c_int, _c_ll]),
     "pn_set_stream": (_c_int, [_vp, _vp]),
     "pn_dim": (_c_int, [_vp, _c_int]),
+    "pn_activation": (_c_int, [_c_int, _vp, _vp, _c_ll, _vp]),
     "pn_last_error": (ctypes.c_char_p, [_vp]),
     "pn_destroy": (None, [_vp]),
     "pn_version": (ctypes.c_char_p, []),
@@ -61,7 +62,7 @@ SIGNATURES = {
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m newton_evaluation_nonlinear_b200.build`")
+                          "`python newton_evaluation_nonlinear_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)
@@ -149,6 +150,10 @@ def pn_set_option(h: int, opt: int, value: int) -> int:
 
 def pn_set_stream(h: int, stream: int) -> int:
     return lib.pn_set_stream(h, stream or None)
+
+
+def pn_activation(which: int, x_ptr: int, y_ptr: int, n: int, stream: int = 0) -> int:
+    return lib.pn_activation(int(which), x_ptr, y_ptr, int(n), stream or None)
 
 
 def pn_dim(h: int, which: int) -> int:

@@ -1,6 +1,8 @@
 """Build libpn.so (the CUDA library behind include/pn.h) in-tree for sm_100a.
 
-    python -m newton_evaluation_nonlinear_b200.build [--force]
+    python newton_evaluation_nonlinear_b200/build.py [--force]
+
+(run it by path: importing the package loads libpn.so, which is what this builds)
 
 Each translation unit under csrc/ is compiled by nvcc in parallel (one per
 cell holds that cell's kernel instantiations), then linked into one shared

@@ -49,6 +49,8 @@ struct pn_ctx {
   // device memory
   float* wt_diag = nullptr;    // [ngroups][DP][R*G] transposed recurrent weights
   float* wt_dense = nullptr;   // [DP][R*DP] transposed + [R][DP][DP] row-major
+  float* wt_tc = nullptr;      // [W ; W_lo] rows of W_q, TF32-rounded, K-major core-matrix layout
+  float* wdiag = nullptr;      // [R][DP] diagonal entries W_q[c][c]
   float* bhn = nullptr;        // [DP]
   float* proj_w = nullptr;     // U [D][d_in] or W_ih [3D][d_in]
   float* proj_b = nullptr;     // b [D] or b_ih + [b_hr; b_hz; 0] [3D]
@@ -75,6 +77,9 @@ struct pn_ctx {
   long long timeout_ns = 1000000000LL;
   int stall_ticket = -1;
   int device_loop = 1;
+  bool use_tma = false;        // pipelined bulk-copy kernels (D % 4 == 0, DP >= 32)
+  bool use_tc = false;         // tensor-core matvec kernels (D == DP in {32, 64})
+  bool tc_capable = false;
   long long evals = 0;
   int last_iters = -1;
   std::string err;
@@ -133,8 +138,8 @@ void free_all(pn_ctx* h) {
     h->exec[m] = nullptr;
     h->graph[m] = nullptr;
   }
-  float** fbufs[] = {&h->wt_diag, &h->wt_dense, &h->bhn, &h->proj_w, &h->proj_b, &h->xin,
-                     &h->buf1,    &h->agg,      &h->pref, &h->hist,  &h->hx,     &h->hs0, &h->hst};
+  float** fbufs[] = {&h->wt_diag, &h->wt_dense, &h->wt_tc, &h->wdiag, &h->bhn, &h->proj_w, &h->proj_b,
+                     &h->xin,     &h->buf1,     &h->agg,   &h->pref,  &h->hist, &h->hx,     &h->hs0, &h->hst};
   for (float** p : fbufs) {
     if (*p) cudaFree(*p);
     *p = nullptr;
@@ -161,7 +166,9 @@ float w_block(const pn_ctx* h, const float* params, int q, int row, int col) {
 IterParams make_params(const pn_ctx* h, int mode) {
   IterParams P{};
   const bool dense = (mode == PN_NEWTON);
-  P.wt = dense ? h->wt_dense : h->wt_diag;
+  const int kind = h->fam.k[mode].kind;
+  P.wt = dense ? h->wt_dense : (kind == kKindDiagTc ? h->wt_tc : h->wt_diag);
+  P.wdiag = h->wdiag;
   P.bhn = h->bhn;
   P.xin = h->xin;
   P.buf1 = h->buf1;
@@ -412,6 +419,48 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   return (pn_status)c.status;
 }
 
+// Chooses the kernel of every mode for the handle's shape and options and
+// records the tilings; grows the look-back buffer sizes to cover them.
+pn_status select_kernels(pn_ctx* h) {
+  const int D = h->D, T = h->T, B = h->B, DP = h->DP;
+  for (int m = 0; m < 4; ++m) {
+    KInfo ki = (m == PN_NEWTON && DP > PN_MAX_D_NEWTON) ? KInfo{nullptr, 0, 0, 0, 0, 0}
+                                                         : lookup(h->cell, m, DP, h->use_tma, h->use_tc);
+    h->fam.k[m] = ki;
+    if (!ki.fn) continue;
+    h->fam.ngroups[m] = (m == PN_NEWTON) ? 1 : (D + ki.G - 1) / ki.G;
+    if (h->fam.ngroups[m] > kMaxGroups)
+      return fail(h, PN_ERR_INVALID, "D=%d needs %d channel groups (max %d)", D, h->fam.ngroups[m], kMaxGroups);
+    h->fam.nchunks[m] = (T + ki.L - 1) / ki.L;
+    h->fam.ntiles[m] = h->fam.ngroups[m] * B * h->fam.nchunks[m];
+    if (ki.smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.smem);
+      if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    }
+    int per_sm = 0, nsm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ki.fn, ki.nt, ki.smem) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || per_sm < 1)
+      return fail(h, PN_ERR_CUDA, "occupancy query failed for mode %d (D=%d)", m, D);
+    const int ng = h->fam.ngroups[m];
+    long long want = (long long)per_sm * nsm;
+    want = std::max<long long>(ng, (want / ng) * ng);
+    h->fam.grid[m] = (int)std::min<long long>(want, h->fam.ntiles[m]);
+    const size_t G = (size_t)ki.G;
+    const size_t nt = (size_t)h->fam.ntiles[m];
+    const size_t aggf = nt * ((m == PN_NEWTON) ? G * (G + 1) : 2 * G);
+    h->agg_floats = std::max(h->agg_floats, aggf);
+    h->pref_floats = std::max(h->pref_floats, nt * G);
+    h->nflags = std::max(h->nflags, nt);
+  }
+  for (int m = 0; m < 4; ++m) {
+    if (h->exec[m]) cudaGraphExecDestroy(h->exec[m]);
+    if (h->graph[m]) cudaGraphDestroy(h->graph[m]);
+    h->exec[m] = nullptr;
+    h->graph[m] = nullptr;
+  }
+  return PN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -450,6 +499,8 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
   h->B = B;
   h->eps = eps;
   h->DP = padded_width(D);
+  h->use_tma = (D % 4) == 0;
+  h->tc_capable = (D == h->DP) && (D == 32 || (D == 64 && cell != PN_CELL_GRU));
   h->stream = (cudaStream_t)cuda_stream;
   if (cudaGetDevice(&h->device) != cudaSuccess) {
     delete h;
@@ -459,43 +510,18 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
   const int DP = h->DP;
   const size_t BT = (size_t)B * T;
 
-  // kernels and tilings
-  for (int m = 0; m < 4; ++m) {
-    KInfo ki = (m == PN_NEWTON && DP > PN_MAX_D_NEWTON) ? KInfo{nullptr, 0, 0, 0, 0} : lookup(cell, m, DP);
-    h->fam.k[m] = ki;
-    if (!ki.fn) continue;
-    h->fam.ngroups[m] = (m == PN_NEWTON) ? 1 : (D + ki.G - 1) / ki.G;
-    if (h->fam.ngroups[m] > kMaxGroups) {
+  // kernels and tilings; buffers are sized for both the tensor-core and the FP32 kernel sets
+  {
+    pn_status sk = PN_OK;
+    for (int pass = 0; pass < 2 && sk == PN_OK; ++pass) {
+      h->use_tc = (pass == 0) ? false : h->tc_capable;
+      sk = select_kernels(h);
+    }
+    if (sk != PN_OK) {
+      g_create_error = h->err;
       delete h;
-      return fail(nullptr, PN_ERR_INVALID, "D=%d needs %d channel groups (max %d)", D, h->fam.ngroups[m], kMaxGroups);
+      return sk;
     }
-    h->fam.nchunks[m] = (T + ki.L - 1) / ki.L;
-    h->fam.ntiles[m] = h->fam.ngroups[m] * B * h->fam.nchunks[m];
-    if (ki.smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.smem);
-      if (e != cudaSuccess) {
-        delete h;
-        return fail(nullptr, PN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-      }
-    }
-    int per_sm = 0, nsm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ki.fn, ki.nt, ki.smem) != cudaSuccess ||
-        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || per_sm < 1) {
-      delete h;
-      return fail(nullptr, PN_ERR_CUDA, "occupancy query failed for mode %d (D=%d)", m, D);
-    }
-    {
-      const int ng = h->fam.ngroups[m];
-      long long want = (long long)per_sm * nsm;
-      want = std::max<long long>(ng, (want / ng) * ng);
-      h->fam.grid[m] = (int)std::min<long long>(want, h->fam.ntiles[m]);
-    }
-    const size_t G = (size_t)ki.G;
-    const size_t nt = (size_t)h->fam.ntiles[m];
-    const size_t aggf = nt * ((m == PN_NEWTON) ? G * (G + 1) : 2 * G);
-    h->agg_floats = std::max(h->agg_floats, aggf);
-    h->pref_floats = std::max(h->pref_floats, nt * G);
-    h->nflags = std::max(h->nflags, nt);
   }
 
   pn_status st = PN_OK;
@@ -506,7 +532,7 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
   } while (0)
   {
     // weights, packed on the host
-    const int Gd = h->fam.k[PN_QUASI].G;
+    const int Gd = lookup(cell, PN_QUASI, DP, h->use_tma, false).G;
     const int ng = (D + Gd - 1) / Gd;
     std::vector<float> wt((size_t)ng * DP * R * Gd, 0.0f);
     for (int g = 0; g < ng; ++g)
@@ -524,6 +550,23 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
     for (int q = 0; q < R; ++q)
       for (int i = 0; i < D; ++i)
         for (int k = 0; k < D; ++k) wr[((size_t)q * DP + i) * DP + k] = w_block(h, params, q, i, k);
+    // tensor-core operand: rows n = q*DP + j of the R stacked blocks, K = DP inputs;
+    // W (TF32-rounded) then W_lo = tf32(W - tf32(W)), each in the K-major core-matrix layout
+    const int NN = R * DP;
+    std::vector<float> wtc(2 * (size_t)NN * DP, 0.0f);
+    for (int q = 0; q < R; ++q)
+      for (int j = 0; j < D; ++j)
+        for (int k = 0; k < D; ++k) {
+          const float w = w_block(h, params, q, j, k);
+          const float hi = tf32_round(w);
+          const float lo = tf32_round(w - hi);
+          const size_t off = kmajor_offset(q * DP + j, k, DP) / 4;
+          wtc[off] = hi;
+          wtc[(size_t)NN * DP + off] = lo;
+        }
+    std::vector<float> wdg((size_t)R * DP, 0.0f);
+    for (int q = 0; q < R; ++q)
+      for (int j = 0; j < D; ++j) wdg[(size_t)q * DP + j] = w_block(h, params, q, j, j);
     std::vector<float> bhn(DP, 0.0f);
     std::vector<float> pw, pb;
     if (cell == PN_CELL_TANH_RNN) {
@@ -545,7 +588,11 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
     PN_TRY(dalloc(h, &h->wt_diag, wt.size()));
     PN_TRY(dalloc(h, &h->wt_dense, wd.size()));
     PN_TRY(dalloc(h, &h->bhn, bhn.size()));
-    if (cudaMemcpy(h->wt_diag, wt.data(), wt.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+    PN_TRY(dalloc(h, &h->wt_tc, wtc.size()));
+    PN_TRY(dalloc(h, &h->wdiag, wdg.size()));
+    if (cudaMemcpy(h->wt_tc, wtc.data(), wtc.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(h->wdiag, wdg.data(), wdg.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(h->wt_diag, wt.data(), wt.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(h->wt_dense, wd.data(), wd.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(h->bhn, bhn.data(), bhn.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess) {
       st = fail(h, PN_ERR_CUDA, "weight upload failed");
@@ -731,6 +778,16 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
       if (value != 0 && value != 1) return fail(h, PN_ERR_INVALID, "device loop option is 0 or 1");
       h->device_loop = (int)value;
       return PN_OK;
+    case PN_OPT_TENSOR_CORES: {
+      if (value != 0 && value != 1) return fail(h, PN_ERR_INVALID, "tensor-core option is 0 or 1");
+      const bool want = (value == 1) && h->tc_capable;
+      if (want == h->use_tc) return PN_OK;
+      DeviceGuard dg(h->device);
+      if (h->stream) cudaStreamSynchronize(h->stream);
+      else cudaDeviceSynchronize();
+      h->use_tc = want;
+      return select_kernels(h);
+    }
   }
   return fail(h, PN_ERR_INVALID, "unknown option %d", (int)opt);
 }
@@ -738,6 +795,19 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
 pn_status pn_set_stream(pn_handle h, void* cuda_stream) {
   if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
   h->stream = (cudaStream_t)cuda_stream;
+  return PN_OK;
+}
+
+pn_status pn_activation(int which, const float* x, float* y, long long n, void* cuda_stream) {
+  if (which != 0 && which != 1) return fail(nullptr, PN_ERR_INVALID, "which must be 0 (tanh) or 1 (sigmoid)");
+  if (n < 0 || (n > 0 && (!x || !y))) return fail(nullptr, PN_ERR_INVALID, "bad arrays");
+  if (n == 0) return PN_OK;
+  cudaStream_t st = (cudaStream_t)cuda_stream;
+  const unsigned grid = (unsigned)std::min<long long>((n + 255) / 256, 148LL * 32);
+  void* kargs[] = {(void*)&which, (void*)&x, (void*)&y, (void*)&n};
+  cudaError_t e = cudaLaunchKernel((const void*)&activation_kernel, dim3(grid), dim3(256), kargs, 0, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(nullptr, PN_ERR_CUDA, "activation kernel failed: %s", cudaGetErrorString(e));
   return PN_OK;
 }
 

@@ -108,4 +108,10 @@ __global__ void finish_kernel(const Args* __restrict__ args, const Ctrl* __restr
     st[e] = buf1[e];
 }
 
+// y[e] = activation(x[e]) with the cells' device activations.
+__global__ void activation_kernel(int which, const float* __restrict__ x, float* __restrict__ y, long long n) {
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
+    y[e] = which == 0 ? tanh_pn(x[e]) : sigmoid_pn(x[e]);
+}
+
 }  // namespace pn

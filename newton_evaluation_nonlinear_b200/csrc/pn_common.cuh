@@ -148,7 +148,30 @@ __device__ __forceinline__ unsigned warp_max_u32(unsigned v) {
   return v;
 }
 
-__device__ __forceinline__ float sigmoidf_acc(float v) { return 1.0f / (1.0f + expf(-v)); }
+// Activations from the exponential identities, on the SFU's approximate base-2
+// exponential and reciprocal (ex2.approx / rcp.approx, both within 2 ulp):
+//   tanh(v) = 1 - 2 / (exp(2v) + 1),   sigmoid(v) = 1 / (1 + exp(-v)).
+// Absolute error below 4e-7 over all finite v (the identity loses relative
+// accuracy only where |tanh v| is tiny, never absolute accuracy); saturates
+// to +-1 / 0 / 1 for large |v|.  A GPU test bounds it against CUDA's tanhf.
+__device__ __forceinline__ float ex2_approx(float v) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ float rcp_approx(float v) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ float tanh_pn(float v) {
+  const float e = ex2_approx(v * 2.8853900817779268f);   // 2 / ln 2
+  return fmaf(-2.0f, rcp_approx(e + 1.0f), 1.0f);
+}
+__device__ __forceinline__ float sigmoid_pn(float v) {
+  return rcp_approx(1.0f + ex2_approx(v * -1.4426950408889634f));   // -1 / ln 2
+}
+__device__ __forceinline__ float sigmoidf_acc(float v) { return sigmoid_pn(v); }
 
 // ---------------------------------------------------------------------------
 // end-of-launch bookkeeping, run by the last CTA to finish

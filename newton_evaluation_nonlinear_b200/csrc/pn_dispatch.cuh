@@ -8,8 +8,12 @@
 
 #include "pn_iter_dense.cuh"
 #include "pn_iter_diag.cuh"
+#include "pn_iter_diag_tc.cuh"
+#include "pn_iter_diag_tma.cuh"
 
 namespace pn {
+
+enum KKind { kKindDiag = 0, kKindDiagTc = 1, kKindDense = 2 };
 
 struct KInfo {
   const void* fn;   // __global__ function
@@ -17,13 +21,14 @@ struct KInfo {
   int L;            // steps per tile
   int G;            // channels per tile
   size_t smem;      // dynamic shared memory bytes
+  int kind;         // KKind: which weight packing the kernel reads
 };
 
 template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS>
 inline KInfo diag_kinfo() {
   using C = DiagCfg<CELL, MODE, DP, G, TM, TN, TS>;
   return KInfo{(const void*)&diag_iter_kernel<CELL, MODE, DP, G, TM, TN, TS>, C::NT, C::L, G,
-               C::SMEM_BYTES};
+               C::SMEM_BYTES, kKindDiag};
 }
 
 template <int CELL, int MODE, int DP>
@@ -47,10 +52,43 @@ inline KInfo diag_pick() {
   }
 }
 
+template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS>
+inline KInfo diag_tma_kinfo() {
+  using C = DiagTmaCfg<CELL, MODE, DP, G, TM, TN, TS>;
+  return KInfo{(const void*)&diag_tma_kernel<CELL, MODE, DP, G, TM, TN, TS>, C::NT, C::L, G, C::SMEM_BYTES,
+               kKindDiag};
+}
+
+// Pipelined (producer warp + bulk copies) variant, for D a multiple of 4 and DP >= 32.
+template <int CELL, int MODE, int DP>
+inline KInfo diag_tma_pick() {
+  constexpr bool gru = (CELL == PN_CELL_GRU);
+  if constexpr (DP == 32) {
+    if constexpr (gru) return diag_tma_kinfo<CELL, MODE, 32, 32, 4, 2, 16>();
+    else return diag_tma_kinfo<CELL, MODE, 32, 32, 4, 4, 32>();
+  } else if constexpr (DP == 64) {
+    if constexpr (gru) return diag_tma_kinfo<CELL, MODE, 64, 64, 4, 2, 8>();
+    else return diag_tma_kinfo<CELL, MODE, 64, 64, 4, 4, 16>();
+  } else if constexpr (DP == 128) {
+    if constexpr (gru) return diag_tma_kinfo<CELL, MODE, 128, 32, 2, 2, 16>();
+    else return diag_tma_kinfo<CELL, MODE, 128, 64, 2, 4, 16>();
+  } else {
+    if constexpr (gru) return diag_tma_kinfo<CELL, MODE, 256, 32, 2, 2, 16>();
+    else return diag_tma_kinfo<CELL, MODE, 256, 64, 2, 4, 16>();
+  }
+}
+
+// Tensor-core variant: D == DP in {32, 64}; the GRU's three gates fit only at D = 32.
+template <int CELL, int MODE, int DP>
+inline KInfo diag_tc_kinfo() {
+  using C = DiagTcCfg<CELL, MODE, DP>;
+  return KInfo{(const void*)&diag_tc_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTc};
+}
+
 template <int CELL, int DP, int L>
 inline KInfo dense_kinfo() {
   using C = DenseCfg<CELL, DP, L>;
-  return KInfo{(const void*)&dense_iter_kernel<CELL, DP, L>, C::NT, L, DP, C::SMEM_BYTES};
+  return KInfo{(const void*)&dense_iter_kernel<CELL, DP, L>, C::NT, L, DP, C::SMEM_BYTES, kKindDense};
 }
 
 template <int CELL, int DP>
@@ -65,19 +103,36 @@ inline KInfo dense_pick() {
   }
 }
 
+// tma: use the pipelined variant where it exists (the caller checks D % 4 == 0);
+// tc: use the tensor-core variant where it exists (the caller checks D == DP).
 template <int CELL>
-inline KInfo lookup_cell(int mode, int DP) {
-  KInfo none{nullptr, 0, 0, 0, 0};
-#define PN_DIAG_CASES(MODE)                                 \
-  switch (DP) {                                             \
-    case 4: return diag_pick<CELL, MODE, 4>();              \
-    case 8: return diag_pick<CELL, MODE, 8>();              \
-    case 16: return diag_pick<CELL, MODE, 16>();            \
-    case 32: return diag_pick<CELL, MODE, 32>();            \
-    case 64: return diag_pick<CELL, MODE, 64>();            \
-    case 128: return diag_pick<CELL, MODE, 128>();          \
-    case 256: return diag_pick<CELL, MODE, 256>();          \
-    default: return none;                                   \
+inline KInfo lookup_cell(int mode, int DP, bool tma, bool tc) {
+  KInfo none{nullptr, 0, 0, 0, 0, 0};
+  if (tc && mode != PN_NEWTON) {
+    constexpr bool gru = (CELL == PN_CELL_GRU);
+    if (DP == 32) {
+      if (mode == PN_JACOBI) return diag_tc_kinfo<CELL, PN_JACOBI, 32>();
+      if (mode == PN_PICARD) return diag_tc_kinfo<CELL, PN_PICARD, 32>();
+      return diag_tc_kinfo<CELL, PN_QUASI, 32>();
+    }
+    if constexpr (!gru) {
+      if (DP == 64) {
+        if (mode == PN_JACOBI) return diag_tc_kinfo<CELL, PN_JACOBI, 64>();
+        if (mode == PN_PICARD) return diag_tc_kinfo<CELL, PN_PICARD, 64>();
+        return diag_tc_kinfo<CELL, PN_QUASI, 64>();
+      }
+    }
+  }
+#define PN_DIAG_CASES(MODE)                                                              \
+  switch (DP) {                                                                          \
+    case 4: return diag_pick<CELL, MODE, 4>();                                           \
+    case 8: return diag_pick<CELL, MODE, 8>();                                           \
+    case 16: return diag_pick<CELL, MODE, 16>();                                         \
+    case 32: return tma ? diag_tma_pick<CELL, MODE, 32>() : diag_pick<CELL, MODE, 32>();     \
+    case 64: return tma ? diag_tma_pick<CELL, MODE, 64>() : diag_pick<CELL, MODE, 64>();     \
+    case 128: return tma ? diag_tma_pick<CELL, MODE, 128>() : diag_pick<CELL, MODE, 128>(); \
+    case 256: return tma ? diag_tma_pick<CELL, MODE, 256>() : diag_pick<CELL, MODE, 256>(); \
+    default: return none;                                                                \
   }
   switch (mode) {
     case PN_JACOBI: PN_DIAG_CASES(PN_JACOBI)
@@ -98,16 +153,16 @@ inline KInfo lookup_cell(int mode, int DP) {
 }
 
 // Defined in one translation unit per cell (compiled in parallel).
-KInfo lookup_tanh(int mode, int DP);
-KInfo lookup_gru(int mode, int DP);
-KInfo lookup_euler(int mode, int DP);
+KInfo lookup_tanh(int mode, int DP, bool tma, bool tc);
+KInfo lookup_gru(int mode, int DP, bool tma, bool tc);
+KInfo lookup_euler(int mode, int DP, bool tma, bool tc);
 
-inline KInfo lookup(int cell, int mode, int DP) {
+inline KInfo lookup(int cell, int mode, int DP, bool tma, bool tc) {
   switch (cell) {
-    case PN_CELL_TANH_RNN: return lookup_tanh(mode, DP);
-    case PN_CELL_GRU: return lookup_gru(mode, DP);
-    case PN_CELL_EULER_TANH: return lookup_euler(mode, DP);
-    default: return KInfo{nullptr, 0, 0, 0, 0};
+    case PN_CELL_TANH_RNN: return lookup_tanh(mode, DP, tma, tc);
+    case PN_CELL_GRU: return lookup_gru(mode, DP, tma, tc);
+    case PN_CELL_EULER_TANH: return lookup_euler(mode, DP, tma, tc);
+    default: return KInfo{nullptr, 0, 0, 0, 0, 0};
   }
 }
 

@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
       float bb, res;
       if constexpr (CELL == PN_CELL_TANH_RNN) {
         // A = diag(1 - y^2) W
-        const float y = tanhf(acc[0] + xv[0]);
+        const float y = tanh_pn(acc[0] + xv[0]);
         const float d = 1.0f - y * y;
         coef[0] = 0.0f;
         coef[1] = d;
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
         res = sc - y;
       } else if constexpr (CELL == PN_CELL_EULER_TANH) {
         // A = I + diag(eps (1 - g^2)) W
-        const float gg = tanhf(acc[0] + xv[0]);
+        const float gg = tanh_pn(acc[0] + xv[0]);
         const float eg = P.eps * gg;
         const float e = P.eps * (1.0f - gg * gg);
         coef[0] = 1.0f;
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
         const float r = sigmoidf_acc(xv[0] + acc[0]);
         const float z = sigmoidf_acc(xv[1] + acc[1]);
         const float hn = acc[2] + bhn_i;
-        const float nn = tanhf(xv[2] + r * hn);
+        const float nn = tanh_pn(xv[2] + r * hn);
         const float y = nn + z * (sp - nn);
         const float omz = 1.0f - z;
         const float dn = omz * (1.0f - nn * nn);

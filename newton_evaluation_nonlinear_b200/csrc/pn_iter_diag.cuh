@@ -236,12 +236,12 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
         const float sc = sT[cw * LP + m0 + m + 1];   // s^(i)_t
         float y, a, bb, res;
         if constexpr (CELL == PN_CELL_TANH_RNN) {
-          y = tanhf(acc[m][0][n] + xv[m][0][n]);
+          y = tanh_pn(acc[m][0][n] + xv[m][0][n]);
           res = sc - y;
           a = (MODE == PN_QUASI) ? (1.0f - y * y) * wd[n][0] : (MODE == PN_PICARD ? 1.0f : 0.0f);
           bb = (MODE == PN_JACOBI) ? y : y - a * sp;
         } else if constexpr (CELL == PN_CELL_EULER_TANH) {
-          const float gg = tanhf(acc[m][0][n] + xv[m][0][n]);
+          const float gg = tanh_pn(acc[m][0][n] + xv[m][0][n]);
           const float eg = P.eps * gg;
           y = sp + eg;
           res = (sc - sp) - eg;
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
           const float r = sigmoidf_acc(xv[m][0][n] + acc[m][0][n]);
           const float z = sigmoidf_acc(xv[m][1][n] + acc[m][1][n]);
           const float hn = acc[m][2][n] + bhn[n];
-          const float nn = tanhf(xv[m][2][n] + r * hn);
+          const float nn = tanh_pn(xv[m][2][n] + r * hn);
           y = nn + z * (sp - nn);
           res = sc - y;
           if (MODE == PN_QUASI) {

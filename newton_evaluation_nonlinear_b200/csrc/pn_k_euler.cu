@@ -2,5 +2,5 @@
 #include "pn_dispatch.cuh"
 
 namespace pn {
-KInfo lookup_euler(int mode, int DP) { return lookup_cell<PN_CELL_EULER_TANH>(mode, DP); }
+KInfo lookup_euler(int mode, int DP, bool tma, bool tc) { return lookup_cell<PN_CELL_EULER_TANH>(mode, DP, tma, tc); }
 }  // namespace pn

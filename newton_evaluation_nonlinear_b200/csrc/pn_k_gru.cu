@@ -2,5 +2,5 @@
 #include "pn_dispatch.cuh"
 
 namespace pn {
-KInfo lookup_gru(int mode, int DP) { return lookup_cell<PN_CELL_GRU>(mode, DP); }
+KInfo lookup_gru(int mode, int DP, bool tma, bool tc) { return lookup_cell<PN_CELL_GRU>(mode, DP, tma, tc); }
 }  // namespace pn

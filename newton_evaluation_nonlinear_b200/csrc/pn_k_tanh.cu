@@ -2,5 +2,5 @@
 #include "pn_dispatch.cuh"
 
 namespace pn {
-KInfo lookup_tanh(int mode, int DP) { return lookup_cell<PN_CELL_TANH_RNN>(mode, DP); }
+KInfo lookup_tanh(int mode, int DP, bool tma, bool tc) { return lookup_cell<PN_CELL_TANH_RNN>(mode, DP, tma, tc); }
 }  // namespace pn

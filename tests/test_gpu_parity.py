@@ -22,11 +22,12 @@ def _pn():
     return pn
 
 
-def _run(prob, mode, tol=None, max_iters=None, device_loop=1):
+def _run(prob, mode, tol=None, max_iters=None, device_loop=1, tc=1):
     import torch
     pn = _pn()
     solver = pn.Solver.from_problem(prob)
     solver.set_option(pn.PN_OPT_DEVICE_LOOP, device_loop)
+    solver.set_option(pn.PN_OPT_TENSOR_CORES, tc)
     x = torch.from_numpy(prob.x).cuda()
     s0 = torch.from_numpy(prob.s0).cuda()
     tol = prob.tol if tol is None else tol
@@ -43,7 +44,7 @@ def _relerr(a, ref):
     return float(np.abs(a.astype(np.float64) - ref).max()) / den
 
 
-def _check_against_oracle(prob, mode, tol=None, max_iters=None, device_loop=1):
+def _check_against_oracle(prob, mode, tol=None, max_iters=None, device_loop=1, tc=1):
     """tol defaults to prob.tol * max(1, max|s|): an fp32 iterate assembled by a parallel scan carries
     rounding of a few ulp(|s|) per step, so an absolute tol below ~1e-6 |s| would sit on the fp32
     floor (the Euler drift reaches |s| ~ 20 on these inputs; the tanh and GRU states stay within 1)."""
@@ -52,7 +53,7 @@ def _check_against_oracle(prob, mode, tol=None, max_iters=None, device_loop=1):
     seq = m.sequential(prob.x, prob.s0)
     tol = prob.tol * max(1.0, float(np.abs(seq).max())) if tol is None else tol
     s_or, it_or, r_or, st_or, hist_or = m.iterate(mode, prob.x, prob.s0, mi, tol)
-    s, it, r, st, hist = _run(prob, mode, tol, mi, device_loop)
+    s, it, r, st, hist = _run(prob, mode, tol, mi, device_loop, tc)
     assert np.isfinite(s).all()
     margin = float(np.min(np.abs(hist_or / tol - 1.0))) if tol > 0 else 1.0
     if margin > 1e-2:
@@ -67,9 +68,11 @@ def _check_against_oracle(prob, mode, tol=None, max_iters=None, device_loop=1):
         # the GPU's distance to the sequential states is the oracle iterate's own iteration error
         # plus fp32 rounding
         assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq)), (_relerr(s, seq), _relerr(s_or, seq))
-    # residual history: fp32 residuals track the fp64 ones
+    # residual history: fp32 residuals track the fp64 ones, up to rounding of the scanned iterate
+    # (a few ulp of max|s| per step, accumulated along the chain)
     n = min(len(hist), len(hist_or))
-    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=1e-2, atol=5e-6)
+    scale = max(1.0, float(np.abs(seq).max()))
+    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=2e-2, atol=1e-5 * scale)
     return it, s
 
 
@@ -92,6 +95,22 @@ def test_small_shapes(cell, mode, D, T, B):
     if mode == pi.MODE_JACOBI:
         prob.max_iters = T
     _check_against_oracle(prob, mode)
+
+
+@pytest.mark.parametrize("tc", [1, 0])
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("mode", DIAG_MODES)
+@pytest.mark.parametrize("D,T,B", [(32, 300, 3), (32, 1000, 2), (64, 257, 2), (64, 2100, 3)])
+def test_tensor_core_and_fp32_paths(tc, cell, mode, D, T, B):
+    """D = 32 and 64 run the tensor-core matvec kernels by default (GRU: D = 32 only); both those
+    and the FP32 kernels must match the oracle, across several 128-step tiles and a ragged tail."""
+    if mode == pi.MODE_PICARD and cell != pi.CELL_EULER:
+        T = 12
+    prob = pi.random_problem(500 + D + T + cell, cell, D, D, T=T, B=B, rho=0.7, eps=0.05, s0_scale=0.3,
+                             tol=1e-5)
+    if mode == pi.MODE_JACOBI:
+        prob.max_iters = T
+    _check_against_oracle(prob, mode, tc=tc)
 
 
 @pytest.mark.parametrize("cell", CELLS)
