@@ -153,6 +153,33 @@ PN_API pn_status pn_reset_stats(pn_handle h);
 PN_API pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
 PN_API pn_status pn_set_stream(pn_handle h, void* cuda_stream);
 
+/* pn_eval without allocation, for the tanh RNN cell and the diagonal modes.
+ * (An addition of this library; the paper has no counterpart.)
+ *
+ * For callers that cannot call cudaMalloc once they are running -- a loop with
+ * its device memory budget fixed at start-up, code whose device memory belongs
+ * to another framework's allocator, a plug-in that may not grow its footprint:
+ * pn_create allocates its work buffers, this call does not.  All of its scratch
+ * (second iterate buffer, projected inputs, packed weights, scan descriptors,
+ * control block, residual history) lives in one fixed 24 MiB device array that
+ * every device loading the library holds until the process exits.
+ *   params  host, tanh RNN packing W[D][D], U[D][d_in], b[D] (n_params entries)
+ *   x, s0, states, mode, max_iters, tol, iters_out, resid_out: as in pn_eval
+ *           (device pointers, 16-byte aligned; mode jacobi, picard or quasi)
+ *   cuda_stream  the stream the work is ordered on; the call synchronises it.
+ * Limits: 1 <= D <= 64, d_in <= 1024, and the scratch of the shape must fit in
+ * 24 MiB (about B*T*D <= 2.9 million at D = 64); larger shapes return
+ * PN_ERR_INVALID with the needed size in pn_last_error(NULL), which also holds
+ * the text of every other error of this call.
+ * The first call on each device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  Every call
+ * reuses the same array and leaves its contents behind: calls that overlap on
+ * the GPU (other threads, other streams) race and corrupt each other.  The loop
+ * runs from the host, one kernel launch per iteration. */
+PN_API pn_status pn_eval_static(const float* params, size_t n_params, int D, int d_in, int T, int B,
+                                const float* x, const float* s0, pn_mode mode, int max_iters, float tol,
+                                float* states, int* iters_out, float* resid_out, void* cuda_stream);
+
 /* Evaluate the activations the cell kernels use, element-wise, on device
  * arrays: which = 0 gives tanh(x), 1 gives 1 / (1 + exp(-x)).  x and y are
  * device float32 arrays of n elements (they may alias); the work is ordered

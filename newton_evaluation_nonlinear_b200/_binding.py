@@ -53,6 +53,8 @@ SIGNATURES = {
     "pn_set_stream": (_c_int, [_vp, _vp]),
     "pn_dim": (_c_int, [_vp, _c_int]),
     "pn_activation": (_c_int, [_c_int, _vp, _vp, _c_ll, _vp]),
+    "pn_eval_static": (_c_int, [_vp, ctypes.c_size_t, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _c_int,
+                                _c_float, _vp, ctypes.POINTER(_c_int), ctypes.POINTER(_c_float), _vp]),
     "pn_last_error": (ctypes.c_char_p, [_vp]),
     "pn_destroy": (None, [_vp]),
     "pn_version": (ctypes.c_char_p, []),
@@ -150,6 +152,16 @@ def pn_set_option(h: int, opt: int, value: int) -> int:
 
 def pn_set_stream(h: int, stream: int) -> int:
     return lib.pn_set_stream(h, stream or None)
+
+
+def pn_eval_static(params: np.ndarray, D: int, d_in: int, T: int, B: int, x_ptr: int, s0_ptr: int, mode: int,
+                   max_iters: int, tol: float, states_ptr: int, stream: int = 0) -> Tuple[int, int, float]:
+    p = np.ascontiguousarray(params, dtype=np.float32).ravel()
+    it, r = _c_int(-1), _c_float(float("nan"))
+    st = lib.pn_eval_static(p.ctypes.data, p.size, int(D), int(d_in), int(T), int(B), x_ptr, s0_ptr, int(mode),
+                            int(max_iters), float(tol), states_ptr, ctypes.byref(it), ctypes.byref(r),
+                            stream or None)
+    return st, it.value, r.value
 
 
 def pn_activation(which: int, x_ptr: int, y_ptr: int, n: int, stream: int = 0) -> int:

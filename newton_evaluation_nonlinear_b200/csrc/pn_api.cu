@@ -463,6 +463,22 @@ pn_status select_kernels(pn_ctx* h) {
 
 }  // namespace
 
+namespace pn {
+// Sets the calling thread's handle-less error message (pn_last_error(NULL)).
+void set_thread_error(const char* msg) { g_create_error = msg ? msg : ""; }
+
+// Host stubs of the kernels around the convergence loop, for the other
+// translation units of the library: 0 = projection, 1 = init, 2 = result copy.
+const void* aux_kernel(int which) {
+  switch (which) {
+    case 0: return (const void*)&proj_kernel;
+    case 1: return (const void*)&init_kernel;
+    case 2: return (const void*)&finish_kernel;
+    default: return nullptr;
+  }
+}
+}  // namespace pn
+
 extern "C" {
 
 const char* pn_version(void) { return "libpn 0.1 (sm_100a)"; }
