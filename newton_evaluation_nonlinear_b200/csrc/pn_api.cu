@@ -4,6 +4,8 @@
 // ownership, the CUDA graph that holds the device-side convergence loop (a
 // conditional WHILE node around the fused iteration kernel), and the
 // host-driven loop used when the device loop is switched off.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <climits>
@@ -11,6 +13,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -63,9 +66,11 @@ struct pn_ctx {
   Ctrl* ctrl = nullptr;
   Args* args = nullptr;
   float* hist = nullptr;
+  CUtensorMap* tmaps = nullptr;   // TMA descriptors of the tensor-core kernels (3, see IterParams)
   // host pinned mirrors
   Args* args_h = nullptr;
   Ctrl* ctrl_h = nullptr;
+  CUtensorMap* tmaps_h = nullptr;
   // host-buffer evaluation staging (allocated on first pn_eval_host)
   float* hx = nullptr;
   float* hs0 = nullptr;
@@ -145,6 +150,10 @@ void free_all(pn_ctx* h) {
     *p = nullptr;
   }
   if (h->flags) cudaFree(h->flags);
+  if (h->tmaps) cudaFree(h->tmaps);
+  if (h->tmaps_h) cudaFreeHost(h->tmaps_h);
+  h->tmaps = nullptr;
+  h->tmaps_h = nullptr;
   if (h->ctrl) cudaFree(h->ctrl);
   if (h->args) cudaFree(h->args);
   if (h->args_h) cudaFreeHost(h->args_h);
@@ -178,6 +187,7 @@ IterParams make_params(const pn_ctx* h, int mode) {
   P.ctrl = h->ctrl;
   P.args = h->args;
   P.hist = h->hist;
+  P.tmaps = h->tmaps;
   P.eps = h->eps;
   P.D = h->D;
   P.d_in = h->d_in;
@@ -198,6 +208,50 @@ unsigned grid_1d(size_t n, int threads, unsigned cap) {
   if (g < 1) g = 1;
   if (g > cap) g = cap;
   return (unsigned)g;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// Map over a row-major fp32 array [rows][cols] whose box is box_rows rows of
+// box_cols floats; box_cols may exceed cols, the extra columns read as zero.
+bool encode_rows(CUtensorMap* m, const void* base, int cols, long long rows, int box_cols, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (!fn || !base) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(float)};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Fills the pinned mirror of the three maps of the tensor-core kernels for
+// the buffers of the current call: [0] the caller's states (iterate buffer
+// 0), [1] buf1, [2] the step inputs (hoisted projection, or x itself for the
+// Euler cell).  Rows are padded by 4 floats through the box width.
+bool encode_tc_maps(const pn_ctx* h, int mode, CUtensorMap* out) {
+  const int L = h->fam.k[mode].L;
+  const int R = cell_R(h->cell);
+  const long long rows = (long long)h->B * h->T;
+  const void* xs = (h->cell == PN_CELL_EULER_TANH) ? (const void*)h->args_h->x : (const void*)h->xin;
+  return encode_rows(&out[0], h->args_h->states, h->D, rows, h->DP + 4, L + 1) &&
+         encode_rows(&out[1], h->buf1, h->D, rows, h->DP + 4, L + 1) &&
+         encode_rows(&out[2], xs, R * h->D, rows, R * h->DP + 4, L);
 }
 
 // Kernels that run before the loop: projection (tanh RNN, GRU) and init.
@@ -376,6 +430,17 @@ pn_status reset_flags_if_needed(pn_ctx* h) {
   return PN_OK;
 }
 
+// Encodes and uploads the tensor maps when the mode runs a tensor-core kernel.
+// The copy is ordered before the launches on the same stream; the pinned
+// mirror is not touched again before the call's final synchronisation.
+pn_status upload_tc_maps(pn_ctx* h, int mode) {
+  if (h->fam.k[mode].kind != kKindDiagTc) return PN_OK;
+  if (!encode_tc_maps(h, mode, h->tmaps_h))
+    return fail(h, PN_ERR_CUDA, "encoding the TMA tensor maps failed (D=%d, T=%d, B=%d)", h->D, h->T, h->B);
+  PN_CUDA(h, cudaMemcpyAsync(h->tmaps, h->tmaps_h, 3 * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
+  return PN_OK;
+}
+
 // The loop body shared by pn_eval and pn_eval_host: args already point at
 // device buffers.
 pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
@@ -383,6 +448,7 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   if (st != PN_OK) return st;
   h->args_h->use_cond = h->device_loop ? 1 : 0;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
+  if ((st = upload_tc_maps(h, mode)) != PN_OK) return st;
   if (h->device_loop) {
     st = build_graph(h, mode);
     if (st != PN_OK) return st;
@@ -644,6 +710,25 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
     }
     memset(h->args_h, 0, sizeof(Args));
     memset(h->ctrl_h, 0, sizeof(Ctrl));
+    if (h->tc_capable) {
+      // the tensor-core kernels stage their tiles with TMA tensor maps; without
+      // an encoder (or if the shape cannot be encoded) they are not used
+      bool ok = cudaMalloc((void**)&h->tmaps, 3 * sizeof(CUtensorMap)) == cudaSuccess &&
+                cudaMallocHost((void**)&h->tmaps_h, 3 * sizeof(CUtensorMap)) == cudaSuccess;
+      if (ok) {
+        h->args_h->states = h->buf1;   // probe encode with buffers of the same shapes
+        h->args_h->x = (cell == PN_CELL_EULER_TANH) ? h->buf1 : nullptr;
+        ok = encode_tc_maps(h, PN_QUASI, h->tmaps_h);
+        h->args_h->states = nullptr;
+        h->args_h->x = nullptr;
+      }
+      if (!ok) {
+        cudaGetLastError();
+        h->tc_capable = false;
+        h->use_tc = false;
+        PN_TRY(select_kernels(h));
+      }
+    }
     if (cudaDeviceSynchronize() != cudaSuccess) {
       st = fail(h, PN_ERR_CUDA, "device synchronisation after create failed");
       goto bad;
@@ -738,6 +823,7 @@ pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* a
   h->args_h->max_iters = INT_MAX;
   h->args_h->use_cond = 0;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
+  if ((st = upload_tc_maps(h, mode)) != PN_OK) return st;
   cudaEvent_t e0, e1;
   PN_CUDA(h, cudaEventCreate(&e0));
   PN_CUDA(h, cudaEventCreate(&e1));

@@ -4,6 +4,7 @@
 // single-pass chunked scan with decoupled look-back, and bounded waits.
 #pragma once
 
+#include <cuda.h>   // CUtensorMap (type only)
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -59,6 +60,7 @@ struct IterParams {
   Ctrl* ctrl;
   Args* args;
   float* hist;         // residual history [kHistCap]
+  const CUtensorMap* tmaps;  // [0] s rows of iterate buffer 0 (states), [1] of buffer 1, [2] step inputs
   float eps;           // Euler step
   int D, d_in, T, B;
   int ngroups, nchunks;

@@ -12,23 +12,26 @@
 // which keeps the products to about 2^-22 relative error (fp32 level) while
 // the tensor pipe does the multiply-adds.
 //
-// Warp roles (one CTA per SM, 11 warps):
-//   warp 0     producer: claims tiles (ticket order), stages the s rows
-//              t0-1..t0+L-1 and the step inputs with bulk async copies
-//              (TMA) into padded rows; allocates / frees TMEM;
+// Warp roles (one CTA per SM, 3 + D/4 warps):
+//   warp 0     producer: claims tiles (ticket order) and stages the s rows
+//              t0-1..t0+L-1 and the step inputs with ONE 2-D TMA tensor load
+//              each.  The boxes are 4 columns wider than the tensors, so the
+//              hardware zero-fills 16 bytes at the end of every row and the
+//              rows land padded (conflict-free column reads);
 //   warp 1     MMA issuer: one thread issues the 3 x D/8 tcgen05.mma of a
 //              tile into one of two TMEM accumulators, commits to an mbarrier;
-//   warp 2     look-back: publishes nothing itself but the tile's inclusive
-//              prefix; finds the nearest published prefix, folds the
-//              aggregates in between, hands the carry to the epilogue;
-//   warps 3-10 epilogue, one thread per step row (TMEM lane) and half of the
-//              channels: reads Z from TMEM, evaluates the cell, the diagonal
-//              Jacobian and |F|, scans along the rows (warp shuffles, then
-//              across the four row quarters), publishes the tile aggregate,
-//              prepares the next tile's tensor-core operands (S and S_lo in
-//              the K-major core-matrix layout), and applies the carry.
-// The look-back runs one tile behind the epilogue: while the look-back warp
-// waits for the chain, the epilogue warps already split the next tile.
+//   warp 2     look-back: finds the nearest predecessor with a published
+//              state, folds the aggregates in between, publishes the tile's
+//              end state and hands the carry to the epilogue;
+//   warps 3..  epilogue, four row quarters x D/16 channel groups: one thread
+//              per step row (TMEM lane) and 16 channels.  Reads Z from TMEM,
+//              evaluates the cell, the diagonal Jacobian and |F|, scans along
+//              the rows (warp shuffles, all 16 channels level by level, then
+//              across the row quarters), publishes the tile aggregate,
+//              prepares the next tile's tensor-core operands and parks the
+//              in-tile prefixes in TMEM.  A tile's states are written one tile
+//              later, when the look-back warp has had a whole tile of time to
+//              deliver its carry.
 #pragma once
 
 #include <string.h>
@@ -106,19 +109,34 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// The tensor map was written to global memory by a host copy before this
+// launch: order that write before the tensor-map proxy reads it.
+__device__ __forceinline__ void tmap_acquire(const CUtensorMap* map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
+}
+
+// 2-D TMA tensor load of one box at element coordinates (c0, c1) into this
+// CTA's shared memory (128-byte aligned), counted on `bar`.  c0 is 0 here
+// (16-byte aligned); c1 may be -1, where the hardware zero-fills the row.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_addr(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // Round to the nearest TF32 value (10 explicit mantissa bits): the tensor
 // core ignores the low 13 bits, so pre-rounded operands lose nothing more.
+// The device form skips the inf/NaN guard: a non-finite iterate ends the
+// solve as non-finite whatever its rounding.
 __host__ __device__ __forceinline__ float tf32_round(float x) {
 #ifdef __CUDA_ARCH__
-  uint32_t u = __float_as_uint(x);
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 #else
   uint32_t u;
   memcpy(&u, &x, 4);
-#endif
   if ((u & 0x7F800000u) != 0x7F800000u) u = (u + 0x1000u) & 0xFFFFE000u;
-#ifdef __CUDA_ARCH__
-  return __uint_as_float(u);
-#else
   float r;
   memcpy(&r, &u, 4);
   return r;
@@ -159,12 +177,13 @@ struct DiagTcCfg {
   static constexpr int STASH0 = 2 * TCOLS;                              // first stash column
   static constexpr int USED_COLS = STASH0 + (MODE == PN_JACOBI ? 0 : 2 * SCOLS);
   static constexpr int ALLOC_COLS = USED_COLS <= 128 ? 128 : (USED_COLS <= 256 ? 256 : 512);
-  static constexpr int CH = DP / 2;             // channels per epilogue thread
-  static constexpr int NEW = 8;                 // epilogue warps
+  static constexpr int CH = 16;                 // channels per epilogue thread
+  static constexpr int NCG = DP / CH;           // channel groups
+  static constexpr int NEW = 4 * NCG;           // epilogue warps: 4 row quarters x channel groups
   static constexpr int NTE = 32 * NEW;          // epilogue threads
   static constexpr int NT = 32 * (3 + NEW);
-  static constexpr int SP = DP + 4;             // padded s row (floats)
-  static constexpr int XP = R * DP + 4;         // padded step-input row (floats)
+  static constexpr int SP = DP + 4;             // padded s row (floats) = TMA box width
+  static constexpr int XP = R * DP + 4;         // padded step-input row (floats) = TMA box width
   static constexpr int NQ = (DP + 31) / 32;
   static constexpr uint32_t SBO_A = (K / 4) * 128;
   static constexpr uint32_t SBO_B = (K / 4) * 128;
@@ -176,19 +195,21 @@ struct DiagTcCfg {
   static constexpr int OFF_S0 = 0;
   static constexpr int OFF_S1 = align(OFF_S0 + S_BYTES, 128);
   static constexpr int OFF_X = align(OFF_S1 + S_BYTES, 128);
-  static constexpr int OFF_AH = align(OFF_X + X_BYTES, 1024);
+  static constexpr int OFF_AH = align(OFF_X + X_BYTES, 128);
   static constexpr int OFF_AL = OFF_AH + A_BYTES;
   static constexpr int OFF_BH = OFF_AL + A_BYTES;
   static constexpr int OFF_BL = OFF_BH + B_BYTES;
-  static constexpr int OFF_WD = OFF_BL + B_BYTES;              // R*DP floats: diagonals of W_q
-  static constexpr int OFF_BHN = OFF_WD + R * DP * 4;          // DP floats
-  static constexpr int OFF_TOT = OFF_BHN + DP * 4;             // [2 halves][4 quarters][CH][2]
-  static constexpr int OFF_AGG = OFF_TOT + 2 * 4 * CH * 2 * 4; // [2 slots][DP][2]
-  static constexpr int OFF_CARRY = OFF_AGG + 2 * DP * 2 * 4;   // [2 slots][DP]
-  static constexpr int OFF_RED = OFF_CARRY + 2 * DP * 4;       // NT/32 floats
-  static constexpr int SMEM_BYTES = OFF_RED + (NT / 32) * 4;
+  static constexpr int OFF_WD = OFF_BL + B_BYTES;                // R*DP floats: diagonals of W_q
+  static constexpr int OFF_BHN = OFF_WD + R * DP * 4;            // DP floats
+  static constexpr int OFF_TOT = OFF_BHN + DP * 4;               // [NCG][4 quarters][CH][2]
+  static constexpr int OFF_AGG = OFF_TOT + NCG * 4 * CH * 2 * 4; // [2 slots][DP][2]
+  static constexpr int OFF_CARRY = OFF_AGG + 2 * DP * 2 * 4;     // [2 slots][DP]
+  static constexpr int OFF_RED = OFF_CARRY + 2 * DP * 4;         // NT/32 floats
+  static constexpr int SMEM_USED = OFF_RED + (NT / 32) * 4;
+  static constexpr int SMEM_BYTES = SMEM_USED + 128;             // + slack to align the base to 128 bytes
   static_assert(DP == 32 || DP == 64, "tensor-core path covers D = 32 and D = 64");
   static_assert(USED_COLS <= 512, "TMEM columns");
+  static_assert(SP <= 256 && XP <= 256 && L + 1 <= 256, "TMA box extents");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -206,7 +227,9 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   constexpr bool kScan = (MODE != PN_JACOBI);
   constexpr bool kHasA = (MODE == PN_QUASI);
 
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  extern __shared__ __align__(128) unsigned char smem_tc[];
+  // TMA destinations want 128-byte alignment: round the dynamic base up (the launch adds 128 bytes)
+  unsigned char* smem_raw = smem_tc + ((128u - (smem_addr(smem_tc) & 127u)) & 127u);
   float* sS[2] = {reinterpret_cast<float*>(smem_raw + C::OFF_S0), reinterpret_cast<float*>(smem_raw + C::OFF_S1)};
   float* sX = reinterpret_cast<float*>(smem_raw + C::OFF_X);
   unsigned char* sAH = smem_raw + C::OFF_AH;
@@ -223,7 +246,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull, bar_xempty, bar_afull,
       bar_mma[2], bar_tempty[2], bar_lb[2], bar_cfull[2], bar_cempty[2];
   __shared__ int s_tk[2];        // ticket staged in s stage 0/1 (-1: no more tiles)
-  __shared__ int s_atk;          // ticket whose operands sit in the A buffers (-1: none)
+  __shared__ int s_atk;          // ticket whose operands sit in the A buffers (-1: stop)
   __shared__ int s_lbtk[2];      // ticket handed to the look-back warp per slot (-1: stop)
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
@@ -257,7 +280,6 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   }
   const unsigned epoch = *(volatile unsigned*)&ctrl->epoch;
   const int iter = *(volatile int*)&ctrl->iter;
-  const float* __restrict__ src = (iter & 1) ? P.buf1 : A.states;
   float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;
 
   // weights: W and W_lo in the K-major core-matrix layout (pre-packed), diagonals, b_hn
@@ -284,7 +306,12 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
 
   if (warp == 0) {
     // =========================== producer ===================================
-    const float* xin = (CELL == PN_CELL_EULER_TANH) ? A.x : P.xin;
+    const CUtensorMap* tm_s = P.tmaps + ((iter & 1) ? 1 : 0);   // rows of s^(i)
+    const CUtensorMap* tm_x = P.tmaps + 2;                      // step inputs
+    if (lane == 0) {
+      tmap_acquire(tm_s);
+      tmap_acquire(tm_x);
+    }
     int it = 0;
     int x_issued = 0;
     for (;; ++it) {
@@ -301,35 +328,30 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
         ++it;
         break;
       }
-      const int b = kg % B;
-      const int t0 = (kg / B) * L;
-      const int s_rows = min(L + 1, T - t0 + 1);
-      const int x_rows = min(L, T - t0);
+      const int row0 = (kg % B) * T + (kg / B) * L;   // global row of step t0
       if (lane == 0) {
+        // rows t0-1 .. t0+L-1; for the first chunk of a sequence row t0-1 is replaced by s0
+        // when the stage is split, rows past the end are zero-filled or unused
         s_tk[st] = kg;
-        mbar_arrive_expect_tx(&bar_sfull[st], (unsigned)(s_rows * D) * 4u);
-      }
-      __syncwarp();
-      for (int r = lane; r < s_rows; r += 32) {
-        const int t = t0 - 1 + r;
-        const float* row = (t < 0) ? A.s0 + (size_t)b * D : src + ((size_t)b * T + t) * D;
-        bulk_copy_g2s(sS[st] + r * SP, row, (unsigned)D * 4u, &bar_sfull[st]);
+        mbar_arrive_expect_tx(&bar_sfull[st], (unsigned)C::S_BYTES);
+        tma_load_2d(sS[st], tm_s, 0, row0 - 1, &bar_sfull[st]);
       }
       // the single step-input buffer: wait until the previous tile's inputs were consumed
-      if (it >= 1 && !mbar_wait_flag(&bar_xempty, ((unsigned)(it - 1)) & 1u, ctrl, tmo, &s_abort)) { ++it; break; }
-      if (lane == 0) mbar_arrive_expect_tx(&bar_xfull, (unsigned)(x_rows * R * D) * 4u);
-      __syncwarp();
-      for (int e = lane; e < x_rows * R; e += 32) {
-        const int r = e / R;
-        const int q = e % R;
-        bulk_copy_g2s(sX + r * XP + q * DP, xin + ((size_t)b * T + t0 + r) * (R * D) + (size_t)q * D,
-                      (unsigned)D * 4u, &bar_xfull);
+      if (it >= 1 && !mbar_wait_flag(&bar_xempty, ((unsigned)(it - 1)) & 1u, ctrl, tmo, &s_abort)) {
+        ++it;
+        break;
       }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar_xfull, (unsigned)C::X_BYTES);
+        tma_load_2d(sX, tm_x, 0, row0, &bar_xfull);
+      }
+      __syncwarp();
       x_issued = it + 1;
     }
     // drain every fill this warp issued
     for (int j = max(0, it - 2); j < it; ++j)
-      if (!mbar_drain(&bar_sfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0) atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+      if (!mbar_drain(&bar_sfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
+        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
     if (x_issued > 0 && !mbar_drain(&bar_xfull, ((unsigned)(x_issued - 1)) & 1u, tmo) && lane == 0)
       atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
   } else if (warp == 1) {
@@ -351,8 +373,8 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
           const uint32_t bb = (pass == 1) ? bl : bh;
 #pragma unroll
           for (int kb = 0; kb < K / 8; ++kb)
-            umma_tf32(d, umma_smem_desc(a + kb * 256, 128, C::SBO_A), umma_smem_desc(bb + kb * 256, 128, C::SBO_B), idesc,
-                      (pass > 0 || kb > 0) ? 1u : 0u);
+            umma_tf32(d, umma_smem_desc(a + kb * 256, 128, C::SBO_A), umma_smem_desc(bb + kb * 256, 128, C::SBO_B),
+                      idesc, (pass > 0 || kb > 0) ? 1u : 0u);
         }
         umma_commit(&bar_mma[buf]);
       }
@@ -361,7 +383,8 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     }
     // every issued product must have completed before TMEM is released
     for (int j = max(0, issued - 2); j < issued; ++j)
-      if (!mbar_drain(&bar_mma[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0) atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+      if (!mbar_drain(&bar_mma[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
+        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
   } else if (warp == 2) {
     // =========================== look-back ==================================
     if constexpr (kScan) {
@@ -388,7 +411,8 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
             else v = (j < D) ? __ldg(A.s0 + (size_t)b * D + j) : 0.0f;
 #pragma unroll 4
             for (int d = n_agg; d >= 1; --d) {
-              const float2 ab = __ldcg(reinterpret_cast<const float2*>(P.agg + (k - (size_t)d * stride) * P.agg_stride) + j);
+              const float2 ab =
+                  __ldcg(reinterpret_cast<const float2*>(P.agg + (k - (size_t)d * stride) * P.agg_stride) + j);
               v = fmaf(ab.x, v, ab.y);
             }
           }
@@ -400,11 +424,10 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
             const int j = lane + 32 * q;
             if (j < DP) P.pref[k * P.pref_stride + j] = fmaf(agg[2 * j], carry[q], agg[2 * j + 1]);
           }
+          // the warp barrier orders the other lanes' stores before lane 0's release,
+          // which is cumulative: a reader that acquires the flag sees all of them
           __syncwarp();
-          if (lane == 0) {
-            __threadfence();
-            st_release(P.flags + k, make_flag(epoch, kFlagPrefix));
-          }
+          if (lane == 0) st_release(P.flags + k, make_flag(epoch, kFlagPrefix));
         }
         if (n_agg < 0) s_abort = 1;
 #pragma unroll
@@ -418,19 +441,30 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     }
   } else {
     // =========================== epilogue ===================================
-    const int e = warp - 3;                 // 0..7
+    const int e = warp - 3;                 // 0 .. NEW-1
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
-    const int half = e >> 2;                // channel half
+    const int cg = e >> 2;                  // channel group
     const int row = quarter * 32 + lane;    // step row within the tile
-    const int cbase = half * CH;            // first channel of this thread
-    const int te = tid - 96;                // 0..255 among epilogue threads
+    const int cbase = cg * CH;              // first channel of this thread
+    const int te = tid - 96;                // 0 .. NTE-1 among the epilogue threads
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
 
-    // operand split: S (raw, the tensor core reads it as TF32) and S_lo, K-major core-matrix layout
-    auto split = [&](const float* S) {
+    // Operand split of stage S: tf32(S) and tf32(S - tf32(S)) in the K-major
+    // core-matrix layout.  For the first chunk of a sequence the stage's row 0
+    // (time -1) is s0, written into the stage here as well for the cell phase.
+    auto split = [&](float* S, int kgs) {
+      const bool first = (kgs / B) == 0;
+      const float* s0row = A.s0 + (size_t)(kgs % B) * D;
       for (int c = te; c < L * (K / 4); c += NTE) {
         const int r = (c & 7) + 8 * ((c >> 3) / (K / 4));
         const int kq = (c >> 3) % (K / 4);
-        const float4 v = *reinterpret_cast<const float4*>(S + r * SP + kq * 4);
+        float4 v;
+        if (first && r == 0) {
+          v = __ldg(reinterpret_cast<const float4*>(s0row) + kq);
+          *reinterpret_cast<float4*>(S + kq * 4) = v;
+        } else {
+          v = *reinterpret_cast<const float4*>(S + r * SP + kq * 4);
+        }
         const float4 hi = make_float4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z), tf32_round(v.w));
         const float4 lo = make_float4(tf32_round(v.x - hi.x), tf32_round(v.y - hi.y), tf32_round(v.z - hi.z),
                                       tf32_round(v.w - hi.w));
@@ -438,15 +472,47 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
         *reinterpret_cast<float4*>(sAH + off) = hi;
         *reinterpret_cast<float4*>(sAL + off) = lo;
       }
-      fence_async_smem();
+      fence_async_smem();   // generic writes -> async proxy (tensor cores, next TMA fill)
+    };
+
+    // s^(i+1) of tile j from its parked prefixes and the carry of the look-back warp
+    auto write_out = [&](int j, int kgj) {
+      const int slot = j & 1;
+      mbar_wait_flag(&bar_cfull[slot], ((unsigned)j >> 1) & 1u, ctrl, tmo, &s_abort);
+      const float* cr = sCarry + slot * DP + cbase;
+      const int bj = kgj % B;
+      const int tj = (kgj / B) * L + row;
+      const bool okj = (tj < T) && !s_abort;
+      const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS) + lane_off;
+      float bb[16], aa[16];
+      tmem_ld16(sbase + (uint32_t)((kHasA ? DP : 0) + cbase), bb);
+      if constexpr (kHasA) tmem_ld16(sbase + (uint32_t)cbase, aa);
+      if (okj) {
+        float* o = dst + ((size_t)bj * T + tj) * D + cbase;
+#pragma unroll
+        for (int c4 = 0; c4 < CH; c4 += 4) {
+          const float4 c = *reinterpret_cast<const float4*>(cr + c4);
+          float4 v;
+          if constexpr (kHasA) {
+            v = make_float4(fmaf(aa[c4], c.x, bb[c4]), fmaf(aa[c4 + 1], c.y, bb[c4 + 1]),
+                            fmaf(aa[c4 + 2], c.z, bb[c4 + 2]), fmaf(aa[c4 + 3], c.w, bb[c4 + 3]));
+          } else {
+            v = make_float4(c.x + bb[c4], c.y + bb[c4 + 1], c.z + bb[c4 + 2], c.w + bb[c4 + 3]);
+          }
+          *reinterpret_cast<float4*>(o + c4) = v;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_cempty[slot]);
     };
 
     // prologue: operands of the first tile
     {
       int kg0 = -1;
       if (mbar_wait_flag(&bar_sfull[0], 0u, ctrl, tmo, &s_abort)) kg0 = s_tk[0];
-      if (kg0 >= 0) split(sS[0]);
+      if (kg0 >= 0) split(sS[0], kg0);
       __syncwarp();
+      named_barrier(1, NTE);
       if (lane == 0) {
         if (te == 0) s_atk = s_abort ? -1 : kg0;
         mbar_arrive(&bar_afull);
@@ -455,44 +521,13 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     named_barrier(1, NTE);
     int kg = s_atk;   // written by te == 0 before the barrier
     int it = 0;
-    // s^(i+1) of tile j from its parked prefixes and the carry of the look-back warp
-    auto write_out = [&](int j, int kgj) {
-      const int slot = j & 1;
-      mbar_wait_flag(&bar_cfull[slot], ((unsigned)j >> 1) & 1u, ctrl, tmo, &s_abort);
-      const float* cr = sCarry + slot * DP + cbase;   // read in place; released after the loop below
-      const int bj = kgj % B;
-      const int tj = (kgj / B) * L + row;
-      const bool okj = (tj < T) && !s_abort;
-      const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS) + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll
-      for (int c16 = 0; c16 < CH; c16 += 16) {
-        float bb[16], aa[16];
-        tmem_ld16(sbase + (uint32_t)((kHasA ? DP : 0) + cbase + c16), bb);
-        if constexpr (kHasA) tmem_ld16(sbase + (uint32_t)(cbase + c16), aa);
-        if (okj) {
-#pragma unroll
-          for (int c4 = 0; c4 < 16; c4 += 4) {
-            float4 o;
-            o.x = kHasA ? fmaf(aa[c4 + 0], cr[c16 + c4 + 0], bb[c4 + 0]) : cr[c16 + c4 + 0] + bb[c4 + 0];
-            o.y = kHasA ? fmaf(aa[c4 + 1], cr[c16 + c4 + 1], bb[c4 + 1]) : cr[c16 + c4 + 1] + bb[c4 + 1];
-            o.z = kHasA ? fmaf(aa[c4 + 2], cr[c16 + c4 + 2], bb[c4 + 2]) : cr[c16 + c4 + 2] + bb[c4 + 2];
-            o.w = kHasA ? fmaf(aa[c4 + 3], cr[c16 + c4 + 3], bb[c4 + 3]) : cr[c16 + c4 + 3] + bb[c4 + 3];
-            *reinterpret_cast<float4*>(dst + ((size_t)bj * T + tj) * D + cbase + c16 + c4) = o;
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_cempty[slot]);
-    };
-
     int prev_kg = -1;
     for (; kg >= 0; ++it) {
       const int st = it & 1;
       const int buf = it & 1;
       const int b = kg % B;
       const int chunk = kg / B;
-      const int t0 = chunk * L;
-      const int t = t0 + row;
+      const int t = chunk * L + row;
       const float* S = sS[st];
 
       // ---- Z from TMEM, then the cell --------------------------------------
@@ -500,14 +535,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
       tc_fence_after();
       float z[R][CH];
 #pragma unroll
-      for (int q = 0; q < R; ++q)
-#pragma unroll
-        for (int c16 = 0; c16 < CH; c16 += 16) {
-          float v[16];
-          tmem_ld16(tmem + (uint32_t)(buf * C::TCOLS) + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(q * DP + cbase + c16), v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) z[q][c16 + j] = v[j];
-        }
+      for (int q = 0; q < R; ++q) tmem_ld16(tmem + (uint32_t)(buf * C::TCOLS) + lane_off + (uint32_t)(q * DP + cbase), z[q]);
       mbar_wait_flag(&bar_xfull, (unsigned)it & 1u, ctrl, tmo, &s_abort);
       const bool tok = (t < T);
       float av[CH], bv[CH];
@@ -590,7 +618,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
       {
         int kn = -1;
         if (mbar_wait_flag(&bar_sfull[st ^ 1], (((unsigned)it + 1u) >> 1) & 1u, ctrl, tmo, &s_abort)) kn = s_tk[st ^ 1];
-        if (kn >= 0 && !s_abort) split(sS[st ^ 1]);
+        if (kn >= 0 && !s_abort) split(sS[st ^ 1], kn);
         __syncwarp();
         named_barrier(1, NTE);   // every epilogue thread has written its part of the split
         if (lane == 0) {
@@ -605,57 +633,69 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
 
       if constexpr (!kScan) {
         if (tok && !s_abort) {
+          float* o = dst + ((size_t)b * T + t) * D + cbase;
 #pragma unroll
           for (int c4 = 0; c4 < CH; c4 += 4)
-            *reinterpret_cast<float4*>(dst + ((size_t)b * T + t) * D + cbase + c4) =
-                make_float4(bv[c4], bv[c4 + 1], bv[c4 + 2], bv[c4 + 3]);
+            *reinterpret_cast<float4*>(o + c4) = make_float4(bv[c4], bv[c4 + 1], bv[c4 + 2], bv[c4 + 3]);
         }
       } else {
-        // ---- scan along the rows: within the warp, then across the quarters --
+        // ---- scan along the rows: within the warp (a level at a time over all 16
+        //      channels, so the shuffles of one level are independent), then across quarters
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-          float a_ = av[c], b_ = bv[c];
+        for (int off = 1; off < 32; off <<= 1) {
 #pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const float ub = __shfl_up_sync(0xffffffffu, b_, off);
-            float ua = 1.0f;
-            if (kHasA) ua = __shfl_up_sync(0xffffffffu, a_, off);
-            if (lane >= off) {
-              b_ = fmaf(a_, ub, b_);
-              if (kHasA) a_ *= ua;
+          for (int c = 0; c < CH; ++c) {
+            const float ub = __shfl_up_sync(0xffffffffu, bv[c], off);
+            if constexpr (kHasA) {
+              const float ua = __shfl_up_sync(0xffffffffu, av[c], off);
+              if (lane >= off) {
+                bv[c] = fmaf(av[c], ub, bv[c]);
+                av[c] *= ua;
+              }
+            } else {
+              if (lane >= off) bv[c] += ub;
             }
           }
-          av[c] = a_;
-          bv[c] = b_;
         }
         if (lane == 31) {
 #pragma unroll
-          for (int c = 0; c < CH; ++c) {
-            sTot[((half * 4 + quarter) * CH + c) * 2 + 0] = av[c];
-            sTot[((half * 4 + quarter) * CH + c) * 2 + 1] = bv[c];
-          }
+          for (int c = 0; c < CH; c += 2)
+            *reinterpret_cast<float4*>(sTot + ((cg * 4 + quarter) * CH + c) * 2) =
+                make_float4(kHasA ? av[c] : 1.0f, bv[c], kHasA ? av[c + 1] : 1.0f, bv[c + 1]);
         }
         named_barrier(1, NTE);
+        if (quarter > 0) {
+          // prefix of the earlier quarters: tot_{quarter-1} o ... o tot_0
+          float PA[CH], PB[CH];
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-          float PA = 1.0f, PB = 0.0f;
-          for (int qq = 0; qq < quarter; ++qq) {
-            const float wa = sTot[((half * 4 + qq) * CH + c) * 2 + 0];
-            const float wb = sTot[((half * 4 + qq) * CH + c) * 2 + 1];
-            PB = fmaf(wa, PB, wb);
-            PA *= wa;
+          for (int c = 0; c < CH; ++c) {
+            PA[c] = 1.0f;
+            PB[c] = 0.0f;
           }
-          bv[c] = fmaf(av[c], PB, bv[c]);
-          if (kHasA) av[c] *= PA;
+          for (int qq = 0; qq < quarter; ++qq) {
+            const float* tq = sTot + (cg * 4 + qq) * CH * 2;
+#pragma unroll
+            for (int c = 0; c < CH; c += 2) {
+              const float4 w = *reinterpret_cast<const float4*>(tq + c * 2);
+              PB[c] = fmaf(w.x, PB[c], w.y);
+              PA[c] *= w.x;
+              PB[c + 1] = fmaf(w.z, PB[c + 1], w.w);
+              PA[c + 1] *= w.z;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < CH; ++c) {
+            bv[c] = kHasA ? fmaf(av[c], PB[c], bv[c]) : bv[c] + PB[c];
+            if (kHasA) av[c] *= PA[c];
+          }
         }
         // the last row holds the tile aggregate
         const int slot = it & 1;
         if (quarter == 3 && lane == 31) {
 #pragma unroll
-          for (int c = 0; c < CH; ++c) {
-            sAgg[(slot * DP + cbase + c) * 2 + 0] = kHasA ? av[c] : 1.0f;
-            sAgg[(slot * DP + cbase + c) * 2 + 1] = bv[c];
-          }
+          for (int c = 0; c < CH; c += 2)
+            *reinterpret_cast<float4*>(sAgg + (slot * DP + cbase + c) * 2) =
+                make_float4(kHasA ? av[c] : 1.0f, bv[c], kHasA ? av[c + 1] : 1.0f, bv[c + 1]);
         }
         named_barrier(1, NTE);
         if (e == 0) {   // publish the aggregate, then wake the look-back warp
@@ -667,13 +707,10 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
               const int j = lane + 32 * q;
               if (j < DP)
                 reinterpret_cast<float2*>(P.agg + (size_t)kg * P.agg_stride)[j] =
-                    make_float2(sAgg[(slot * DP + j) * 2], sAgg[(slot * DP + j) * 2 + 1]);
+                    *reinterpret_cast<const float2*>(sAgg + (slot * DP + j) * 2);
             }
-            __syncwarp();
-            if (lane == 0) {
-              __threadfence();
-              st_release(P.flags + kg, make_flag(epoch, kFlagAgg));
-            }
+            __syncwarp();   // lane 0's release is cumulative over the lanes' stores ordered before it
+            if (lane == 0) st_release(P.flags + kg, make_flag(epoch, kFlagAgg));
           }
           __syncwarp();
           if (lane == 0) {
@@ -681,26 +718,16 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
             mbar_arrive(&bar_lb[slot]);
           }
         }
-        // ---- park this tile's in-tile prefixes in TMEM; written out next iteration
+        // ---- park this tile's in-tile prefixes in TMEM; written out next tile
         {
-          const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS) + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll
-          for (int c16 = 0; c16 < CH; c16 += 16) {
-            float v[16];
-            if constexpr (kHasA) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j) v[j] = av[c16 + j];
-              tmem_st16(sbase + (uint32_t)(cbase + c16), v);
-            }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = bv[c16 + j];
-            tmem_st16(sbase + (uint32_t)((kHasA ? DP : 0) + cbase + c16), v);
-          }
+          const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS) + lane_off;
+          if constexpr (kHasA) tmem_st16(sbase + (uint32_t)cbase, av);
+          tmem_st16(sbase + (uint32_t)((kHasA ? DP : 0) + cbase), bv);
           tmem_st_wait();
         }
         prev_kg = kg;
       }
-      named_barrier(1, NTE);   // uniform exit decision (s_atk was set by te == 0 in step 4)
+      named_barrier(1, NTE);   // uniform exit decision (s_atk was set by te == 0 above)
       kg = s_atk;
     }
     if constexpr (kScan) {
@@ -719,7 +746,9 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::ALLOC_COLS) : "memory");
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::ALLOC_COLS)
+                 : "memory");
   if (tid == 0) {
     unsigned v = 0u;
     for (int w = 0; w < C::NT / 32; ++w) v = max(v, __float_as_uint(sRed[w]));
