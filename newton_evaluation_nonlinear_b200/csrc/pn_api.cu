@@ -66,7 +66,7 @@ struct pn_ctx {
   Ctrl* ctrl = nullptr;
   Args* args = nullptr;
   float* hist = nullptr;
-  CUtensorMap* tmaps = nullptr;   // TMA descriptors of the tensor-core kernels (3, see IterParams)
+  CUtensorMap* tmaps = nullptr;   // TMA descriptors of the tensor-core kernels (kTcMaps, see IterParams)
   // host pinned mirrors
   Args* args_h = nullptr;
   Ctrl* ctrl_h = nullptr;
@@ -226,32 +226,40 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// Map over a row-major fp32 array [rows][cols] whose box is box_rows rows of
-// box_cols floats; box_cols may exceed cols, the extra columns read as zero.
-bool encode_rows(CUtensorMap* m, const void* base, int cols, long long rows, int box_cols, int box_rows) {
+// Map over an fp32 array [B][T][cols] (one sequence after the other) whose
+// box is box_rows steps of box_cols floats of one sequence.  Box elements
+// outside the array (columns >= cols, steps < 0 or >= T) read as zero and are
+// not written by stores, so a box never reaches into the next sequence.
+bool encode_seq(CUtensorMap* m, const void* base, int cols, int T, int B, int box_cols, int box_rows, bool swizzle128) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
   if (!fn || !base) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(float)};
-  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1u, 1u};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * sizeof(float), (cuuint64_t)cols * sizeof(float) * (cuuint64_t)T};
+  cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Fills the pinned mirror of the three maps of the tensor-core kernels for
-// the buffers of the current call: [0] the caller's states (iterate buffer
-// 0), [1] buf1, [2] the step inputs (hoisted projection, or x itself for the
-// Euler cell).  Rows are padded by 4 floats through the box width.
+// Fills the pinned mirror of the maps of the tensor-core kernels for the
+// buffers of the current call (iterate buffer 0 is the caller's states,
+// buffer 1 is buf1; the step inputs are the hoisted projection, or x itself
+// for the Euler cell):
+//   [0], [1]  s^(i) loads from buffer 0 / 1: 32-float column halves of L+1
+//             steps, 128-byte swizzled (the tensor cores' operand layout);
+//   [2]       step-input loads, rows padded by 4 floats through the box width;
+//   [3], [4]  state stores into buffer 0 / 1, from rows padded by 4 floats.
 bool encode_tc_maps(const pn_ctx* h, int mode, CUtensorMap* out) {
   const int L = h->fam.k[mode].L;
   const int R = cell_R(h->cell);
-  const long long rows = (long long)h->B * h->T;
+  const int D = h->D, T = h->T, B = h->B, DP = h->DP;
   const void* xs = (h->cell == PN_CELL_EULER_TANH) ? (const void*)h->args_h->x : (const void*)h->xin;
-  return encode_rows(&out[0], h->args_h->states, h->D, rows, h->DP + 4, L + 1) &&
-         encode_rows(&out[1], h->buf1, h->D, rows, h->DP + 4, L + 1) &&
-         encode_rows(&out[2], xs, R * h->D, rows, R * h->DP + 4, L);
+  return encode_seq(&out[0], h->args_h->states, D, T, B, 32, L + 1, true) &&
+         encode_seq(&out[1], h->buf1, D, T, B, 32, L + 1, true) &&
+         encode_seq(&out[2], xs, R * D, T, B, R * DP + 4, L, false) &&
+         encode_seq(&out[3], h->args_h->states, D, T, B, DP + 4, L, false) &&
+         encode_seq(&out[4], h->buf1, D, T, B, DP + 4, L, false);
 }
 
 // Kernels that run before the loop: projection (tanh RNN, GRU) and init.
@@ -437,7 +445,7 @@ pn_status upload_tc_maps(pn_ctx* h, int mode) {
   if (h->fam.k[mode].kind != kKindDiagTc) return PN_OK;
   if (!encode_tc_maps(h, mode, h->tmaps_h))
     return fail(h, PN_ERR_CUDA, "encoding the TMA tensor maps failed (D=%d, T=%d, B=%d)", h->D, h->T, h->B);
-  PN_CUDA(h, cudaMemcpyAsync(h->tmaps, h->tmaps_h, 3 * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
+  PN_CUDA(h, cudaMemcpyAsync(h->tmaps, h->tmaps_h, kTcMaps * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
   return PN_OK;
 }
 
@@ -713,8 +721,8 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
     if (h->tc_capable) {
       // the tensor-core kernels stage their tiles with TMA tensor maps; without
       // an encoder (or if the shape cannot be encoded) they are not used
-      bool ok = cudaMalloc((void**)&h->tmaps, 3 * sizeof(CUtensorMap)) == cudaSuccess &&
-                cudaMallocHost((void**)&h->tmaps_h, 3 * sizeof(CUtensorMap)) == cudaSuccess;
+      bool ok = cudaMalloc((void**)&h->tmaps, kTcMaps * sizeof(CUtensorMap)) == cudaSuccess &&
+                cudaMallocHost((void**)&h->tmaps_h, kTcMaps * sizeof(CUtensorMap)) == cudaSuccess;
       if (ok) {
         h->args_h->states = h->buf1;   // probe encode with buffers of the same shapes
         h->args_h->x = (cell == PN_CELL_EULER_TANH) ? h->buf1 : nullptr;

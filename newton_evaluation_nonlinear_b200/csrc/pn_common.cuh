@@ -17,6 +17,7 @@ constexpr int kHistCap = 65537;        // residual history entries kept per hand
 constexpr unsigned kFlagAgg = 1u;      // tile published its aggregate
 constexpr unsigned kFlagPrefix = 2u;   // tile published its inclusive prefix (a state)
 constexpr int kMaxGroups = 8;          // channel groups of the diagonal-family kernels (D / G)
+constexpr int kTcMaps = 5;             // TMA tensor maps of the tensor-core kernels
 
 // Device control block: one per handle, in device memory.
 struct Ctrl {
@@ -60,7 +61,8 @@ struct IterParams {
   Ctrl* ctrl;
   Args* args;
   float* hist;         // residual history [kHistCap]
-  const CUtensorMap* tmaps;  // [0] s rows of iterate buffer 0 (states), [1] of buffer 1, [2] step inputs
+  const CUtensorMap* tmaps;  // tensor-core kernels: [0]/[1] s^(i) loads from iterate buffer 0 (states) / 1,
+                             // [2] step-input loads, [3]/[4] state stores into buffer 0 / 1
   float eps;           // Euler step
   int D, d_in, T, B;
   int ngroups, nchunks;
@@ -77,6 +79,14 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// With a preceding relaxed load that observed a release store, this fence
+// makes the later loads of this thread see what the releasing thread wrote.
+__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -95,7 +105,9 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 // It waits (bounded) until every predecessor nearer than that one has at least
 // published its aggregate.  Returns the number of aggregate-only tiles between
 // this tile and that prefix, or -1 when it gave up (timeout, or another CTA's
-// error).
+// error).  Flags are polled with relaxed loads; one fence after the final
+// poll gives the caller's subsequent loads of the aggregates and the prefix
+// acquire semantics.
 __device__ __forceinline__ int lookback_find_prefix(const unsigned* flags, size_t k, size_t stride,
                                                     int chunk, unsigned epoch, Ctrl* ctrl,
                                                     long long timeout_ns) {
@@ -108,7 +120,7 @@ __device__ __forceinline__ int lookback_find_prefix(const unsigned* flags, size_
     const int p = base - lane;
     bool valid = true, pfx = true;
     if (p >= 0) {
-      const unsigned f = ld_acquire(flags + (k - (size_t)(chunk - p) * stride));
+      const unsigned f = ld_relaxed(flags + (k - (size_t)(chunk - p) * stride));
       valid = ((f >> 2) == epoch) && (f & 3u);
       pfx = valid && ((f & 3u) == kFlagPrefix);
     }
@@ -117,21 +129,26 @@ __device__ __forceinline__ int lookback_find_prefix(const unsigned* flags, size_
     const int nearest = pm ? (__ffs(pm) - 1) : 32;
     const unsigned need = (nearest >= 31) ? 0xffffffffu : ((2u << nearest) - 1u);
     if ((vm & need) == need) {
-      if (nearest < 32) return n_agg + nearest;
+      if (nearest < 32) {
+        fence_acquire_gpu();
+        return n_agg + nearest;
+      }
       n_agg += 32;
       base -= 32;
       continue;
     }
-    int give_up = 0;
     ++spins;
-    if (lane == 0) {
-      if (ld_volatile(&ctrl->error)) give_up = 1;
-      else if (((spins & 15u) == 0u) && (long long)(globaltimer() - t0) > timeout_ns) {
-        if (atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT) == 0) ctrl->timeout_ticket = (int)k;
-        give_up = 1;
+    if ((spins & 15u) == 0u) {
+      int give_up = 0;
+      if (lane == 0) {
+        if (ld_volatile(&ctrl->error)) give_up = 1;
+        else if ((long long)(globaltimer() - t0) > timeout_ns) {
+          if (atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT) == 0) ctrl->timeout_ticket = (int)k;
+          give_up = 1;
+        }
       }
+      if (__shfl_sync(0xffffffffu, give_up, 0)) return -1;
     }
-    if (__shfl_sync(0xffffffffu, give_up, 0)) return -1;
     if (spins > 64u) __nanosleep(32);
   }
 }

@@ -8,30 +8,39 @@
 // matvec W s_{t-1} of all L = 128 steps of a tile is formed: as one
 // 128 x N x D product Z = S W^T (S = the tile's s^(i) rows, N = R*D) on the
 // tensor cores, split into three TF32 products
-//     Z = S W + S W_lo + S_lo W,   x_lo = x - tf32(x),
-// which keeps the products to about 2^-22 relative error (fp32 level) while
-// the tensor pipe does the multiply-adds.
+//     Z = S_hi W_hi + S_hi W_lo + S_lo W_hi,
+// where the tensor core reads S as S_hi (it ignores the low 13 mantissa bits
+// of an fp32 operand), S_lo = S - S_hi is formed in shared memory, and W_hi,
+// W_lo come pre-split from the host.  The dropped S_lo W_lo term and the
+// truncation of S_lo are below 2^-20 relative, about fp32 level.
 //
-// Warp roles (one CTA per SM, 3 + D/4 warps):
-//   warp 0     producer: claims tiles (ticket order) and stages the s rows
-//              t0-1..t0+L-1 and the step inputs with ONE 2-D TMA tensor load
-//              each.  The boxes are 4 columns wider than the tensors, so the
-//              hardware zero-fills 16 bytes at the end of every row and the
-//              rows land padded (conflict-free column reads);
-//   warp 1     MMA issuer: one thread issues the 3 x D/8 tcgen05.mma of a
-//              tile into one of two TMEM accumulators, commits to an mbarrier;
-//   warp 2     look-back: finds the nearest predecessor with a published
-//              state, folds the aggregates in between, publishes the tile's
-//              end state and hands the carry to the epilogue;
-//   warps 3..  epilogue, four row quarters x D/16 channel groups: one thread
-//              per step row (TMEM lane) and 16 channels.  Reads Z from TMEM,
-//              evaluates the cell, the diagonal Jacobian and |F|, scans along
-//              the rows (warp shuffles, all 16 channels level by level, then
-//              across the row quarters), publishes the tile aggregate,
-//              prepares the next tile's tensor-core operands and parks the
-//              in-tile prefixes in TMEM.  A tile's states are written one tile
-//              later, when the look-back warp has had a whole tile of time to
-//              deliver its carry.
+// Data movement (all TMA, never multicast):
+//   s^(i) rows t0-1 .. t0+L-1 of one sequence arrive in the tensor cores'
+//   128-byte-swizzled K-major layout, one 32-float column half per load; the
+//   epilogue reads them there directly (the swizzle keeps column reads
+//   conflict-free).  Step t0-1 < 0 reads as zero and is replaced by s0.
+//   Step inputs arrive as rows padded by 4 floats (box wider than the array).
+//   New states leave through a padded-row staging buffer and one TMA tensor
+//   store per tile; steps >= T are clipped by the store itself.
+//
+// Warp roles (one CTA per SM):
+//   warp 0      producer: claims tiles (ticket order), issues the loads;
+//   warp 1      MMA and store issuer: one thread issues the 3 x D/8
+//               tcgen05.mma of a tile into one of two TMEM accumulators,
+//               commits to an mbarrier, then issues the TMA store of the
+//               newest finished output tile while the tensor cores work;
+//   warps 2-3   look-back (scan modes), alternate tiles: publish the tile
+//               aggregate, find the nearest predecessor with a published
+//               state, fold the aggregates in between, hand the carry to the
+//               epilogue, then publish the tile's end state;
+//   the rest    epilogue, four row quarters x D/16 channel groups: one thread
+//               per step row (TMEM lane) and 16 channels.  Reads Z from TMEM,
+//               evaluates the cell, the diagonal Jacobian and |F|, forms the
+//               next tile's S_lo, scans along the rows (warp shuffles a level
+//               at a time over all 16 channels, then across the row quarters)
+//               and parks the in-tile prefixes in TMEM.  A tile's states are
+//               formed two tiles later, so the look-back has two tiles of time
+//               to deliver its carry.
 #pragma once
 
 #include <string.h>
@@ -41,22 +50,31 @@
 
 namespace pn {
 
-// --- tcgen05 helpers (inline PTX) ------------------------------------------
+// --- tcgen05 / TMA helpers (inline PTX) ------------------------------------
 
 // Canonical K-major layout without swizzle ("interleaved" core matrices):
 // a core matrix is 8 rows x 16 bytes stored contiguously; core matrices
 // adjacent along K are 128 bytes apart (leading byte offset) and groups of 8
-// rows are K/4 * 128 bytes apart (stride byte offset).
+// rows are K/4 * 128 bytes apart (stride byte offset).  Used for W.
 __host__ __device__ __forceinline__ uint32_t kmajor_offset(int row, int k, int K) {
   return (uint32_t)((row >> 3) * (K / 4) * 128 + (k >> 2) * 128 + (row & 7) * 16 + (k & 3) * 4);
 }
 
+// 128-byte-swizzled K-major layout of a 32-float column half (base 1024-byte
+// aligned): row r occupies bytes [128 r, 128 r + 128) and its 16-byte chunk j
+// sits at chunk position j ^ (r mod 8).  This is the layout a TMA load with
+// 128-byte swizzle writes.  Used for S and S_lo.
+__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
+  return (uint32_t)(r * 128 + ((((c >> 2) ^ r) & 7) << 4) + (c & 3) * 4);
+}
+
 // Shared-memory matrix descriptor (sm_100): start address >> 4 in bits 0-13,
 // leading byte offset >> 4 in bits 16-29, stride byte offset >> 4 in bits
-// 32-45, version 1 in bits 46-47, no swizzle (bits 61-63 = 0).
-__device__ __forceinline__ uint64_t umma_smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// 32-45, version 1 in bits 46-47, layout in bits 61-63 (0: no swizzle,
+// 2: 128-byte swizzle).
+__device__ __forceinline__ uint64_t umma_smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)layout << 61);
 }
 
 // Instruction descriptor for kind::tf32: D fp32 (bit 4), A and B tf32 (code 2
@@ -115,33 +133,43 @@ __device__ __forceinline__ void tmap_acquire(const CUtensorMap* map) {
   asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
 }
 
-// 2-D TMA tensor load of one box at element coordinates (c0, c1) into this
-// CTA's shared memory (128-byte aligned), counted on `bar`.  c0 is 0 here
-// (16-byte aligned); c1 may be -1, where the hardware zero-fills the row.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+// 3-D TMA tensor load of one box at element coordinates (column c0, step c1,
+// sequence c2) into this CTA's shared memory, counted on `bar`.  c0 is a
+// multiple of 32 (16-byte aligned); c1 may be -1 (that row reads as zero).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
           smem_addr(dst)),
-      "l"(map), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
       : "memory");
 }
 
-// Round to the nearest TF32 value (10 explicit mantissa bits): the tensor
-// core ignores the low 13 bits, so pre-rounded operands lose nothing more.
-// The device form skips the inf/NaN guard: a non-finite iterate ends the
-// solve as non-finite whatever its rounding.
+// 3-D TMA tensor store of one box from shared memory (coordinates >= 0);
+// elements outside the array are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int c0, int c1, int c2, const void* src) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(map), "r"(c0),
+               "r"(c1), "r"(c2), "r"(smem_addr(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's committed bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and have completed their global writes
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Round to the nearest TF32 value (10 explicit mantissa bits), for the host
+// split of W: W_hi = tf32(W), W_lo = tf32(W - W_hi).
 __host__ __device__ __forceinline__ float tf32_round(float x) {
-#ifdef __CUDA_ARCH__
-  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
-#else
   uint32_t u;
   memcpy(&u, &x, 4);
   if ((u & 0x7F800000u) != 0x7F800000u) u = (u + 0x1000u) & 0xFFFFE000u;
   float r;
   memcpy(&r, &u, 4);
   return r;
-#endif
 }
+
+// The part of x below its TF32 truncation (exact in fp32).
+__device__ __forceinline__ float tf32_tail(float x) { return x - __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
 
 // Bounded mbarrier wait that never leaves the caller's control flow: on
 // timeout / error it records the failure in *abort and returns false.
@@ -169,48 +197,56 @@ __device__ __forceinline__ bool mbar_wait_flag(uint64_t* bar, unsigned parity, C
 template <int CELL, int MODE, int DP>
 struct DiagTcCfg {
   static constexpr int R = CellInfo<CELL>::R;
+  static constexpr bool kScan = (MODE != PN_JACOBI);
   static constexpr int L = 128;                 // steps per tile = MMA M
   static constexpr int K = DP;                  // MMA K (input channels)
   static constexpr int N = R * DP;              // MMA N (output rows of W)
+  static constexpr int NKH = DP / 32;           // 32-float column halves of S (one swizzle atom wide)
   static constexpr int TCOLS = N <= 64 ? 64 : (N <= 128 ? 128 : 256);   // TMEM columns per accumulator
   static constexpr int SCOLS = (MODE == PN_QUASI ? 2 : 1) * DP;        // stash columns per tile: [A |] B
-  static constexpr int STASH0 = 2 * TCOLS;                              // first stash column
-  static constexpr int USED_COLS = STASH0 + (MODE == PN_JACOBI ? 0 : 2 * SCOLS);
+  static constexpr int NSLOT = 3;               // tiles between their scan and their write-out, + 1
+  static constexpr int DEFER = NSLOT - 1;       // a tile's states are formed DEFER tiles later
+  static constexpr int NLB = kScan ? 2 : 0;     // look-back warps, alternating tiles
+  static constexpr int STASH0 = 2 * TCOLS;      // first stash column
+  static constexpr int USED_COLS = STASH0 + (kScan ? NSLOT * SCOLS : 0);
   static constexpr int ALLOC_COLS = USED_COLS <= 128 ? 128 : (USED_COLS <= 256 ? 256 : 512);
   static constexpr int CH = 16;                 // channels per epilogue thread
   static constexpr int NCG = DP / CH;           // channel groups
   static constexpr int NEW = 4 * NCG;           // epilogue warps: 4 row quarters x channel groups
   static constexpr int NTE = 32 * NEW;          // epilogue threads
-  static constexpr int NT = 32 * (3 + NEW);
-  static constexpr int SP = DP + 4;             // padded s row (floats) = TMA box width
-  static constexpr int XP = R * DP + 4;         // padded step-input row (floats) = TMA box width
+  static constexpr int WE0 = 2 + NLB;           // first epilogue warp
+  static constexpr int OUT_LAG = kScan ? DEFER : 0;   // output tile j is staged in epilogue tile j + OUT_LAG
+  static constexpr int NT = 32 * (WE0 + NEW);
+  static constexpr int SP = DP + 4;             // padded output row (floats) = store box width
+  static constexpr int XP = R * DP + 4;         // padded step-input row (floats) = load box width
   static constexpr int NQ = (DP + 31) / 32;
-  static constexpr uint32_t SBO_A = (K / 4) * 128;
-  static constexpr uint32_t SBO_B = (K / 4) * 128;
   static constexpr int align(int v, int a) { return (v + a - 1) / a * a; }
-  static constexpr int S_BYTES = (L + 1) * SP * 4;
+  static constexpr int SH_LOAD = (L + 1) * 128;                  // bytes of one S column-half load
+  static constexpr int SH_BYTES = align(SH_LOAD, 1024);          // S column-half buffer
+  static constexpr int LO_BYTES = L * 128;                       // S_lo column-half buffer
   static constexpr int X_BYTES = L * XP * 4;
-  static constexpr int A_BYTES = L * K * 4;
+  static constexpr int O_BYTES = L * SP * 4;
   static constexpr int B_BYTES = N * K * 4;
-  static constexpr int OFF_S0 = 0;
-  static constexpr int OFF_S1 = align(OFF_S0 + S_BYTES, 128);
-  static constexpr int OFF_X = align(OFF_S1 + S_BYTES, 128);
-  static constexpr int OFF_AH = align(OFF_X + X_BYTES, 128);
-  static constexpr int OFF_AL = OFF_AH + A_BYTES;
-  static constexpr int OFF_BH = OFF_AL + A_BYTES;
+  static constexpr int TOT_FLOATS = NCG * 4 * CH * 2;            // one buffer of quarter totals
+  static constexpr int OFF_S = 0;                                // [2 stages][NKH][SH_BYTES]
+  static constexpr int OFF_LO = OFF_S + 2 * NKH * SH_BYTES;      // [NKH][LO_BYTES]
+  static constexpr int OFF_X = OFF_LO + NKH * LO_BYTES;
+  static constexpr int OFF_O = align(OFF_X + X_BYTES, 128);
+  static constexpr int OFF_BH = align(OFF_O + O_BYTES, 128);
   static constexpr int OFF_BL = OFF_BH + B_BYTES;
   static constexpr int OFF_WD = OFF_BL + B_BYTES;                // R*DP floats: diagonals of W_q
   static constexpr int OFF_BHN = OFF_WD + R * DP * 4;            // DP floats
-  static constexpr int OFF_TOT = OFF_BHN + DP * 4;               // [NCG][4 quarters][CH][2]
-  static constexpr int OFF_AGG = OFF_TOT + NCG * 4 * CH * 2 * 4; // [2 slots][DP][2]
-  static constexpr int OFF_CARRY = OFF_AGG + 2 * DP * 2 * 4;     // [2 slots][DP]
-  static constexpr int OFF_RED = OFF_CARRY + 2 * DP * 4;         // NT/32 floats
+  static constexpr int OFF_TOT = OFF_BHN + DP * 4;               // [2][NCG][4 quarters][CH][2]
+  static constexpr int OFF_AGG = OFF_TOT + 2 * TOT_FLOATS * 4;   // [NSLOT][DP][2]
+  static constexpr int OFF_CARRY = OFF_AGG + NSLOT * DP * 2 * 4; // [NSLOT][DP]
+  static constexpr int OFF_RED = OFF_CARRY + NSLOT * DP * 4;     // NT/32 floats
   static constexpr int SMEM_USED = OFF_RED + (NT / 32) * 4;
-  static constexpr int SMEM_BYTES = SMEM_USED + 128;             // + slack to align the base to 128 bytes
+  static constexpr int SMEM_BYTES = SMEM_USED + 1024;            // + slack to align the base to 1024 bytes
   static_assert(DP == 32 || DP == 64, "tensor-core path covers D = 32 and D = 64");
   static_assert(USED_COLS <= 512, "TMEM columns");
   static_assert(SP <= 256 && XP <= 256 && L + 1 <= 256, "TMA box extents");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(DEFER == 2, "the epilogue keeps the tickets of the last two tiles");
 };
 
 template <int CELL, int MODE, int DP>
@@ -220,20 +256,22 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   constexpr int L = C::L;
   constexpr int K = C::K;
   constexpr int N = C::N;
+  constexpr int NKH = C::NKH;
   constexpr int SP = C::SP;
   constexpr int XP = C::XP;
   constexpr int CH = C::CH;
   constexpr int NTE = C::NTE;
-  constexpr bool kScan = (MODE != PN_JACOBI);
+  constexpr int NSLOT = C::NSLOT;
+  constexpr bool kScan = C::kScan;
   constexpr bool kHasA = (MODE == PN_QUASI);
 
-  extern __shared__ __align__(128) unsigned char smem_tc[];
-  // TMA destinations want 128-byte alignment: round the dynamic base up (the launch adds 128 bytes)
-  unsigned char* smem_raw = smem_tc + ((128u - (smem_addr(smem_tc) & 127u)) & 127u);
-  float* sS[2] = {reinterpret_cast<float*>(smem_raw + C::OFF_S0), reinterpret_cast<float*>(smem_raw + C::OFF_S1)};
+  extern __shared__ __align__(1024) unsigned char smem_tc[];
+  // 128-byte swizzled TMA destinations want 1024-byte alignment: round the base up (the launch adds 1 KB)
+  unsigned char* smem_raw = smem_tc + ((1024u - (smem_addr(smem_tc) & 1023u)) & 1023u);
+  unsigned char* sS = smem_raw + C::OFF_S;       // stage st, half h at sS + (st * NKH + h) * SH_BYTES
+  unsigned char* sLo = smem_raw + C::OFF_LO;     // half h at sLo + h * LO_BYTES
   float* sX = reinterpret_cast<float*>(smem_raw + C::OFF_X);
-  unsigned char* sAH = smem_raw + C::OFF_AH;
-  unsigned char* sAL = smem_raw + C::OFF_AL;
+  float* sO = reinterpret_cast<float*>(smem_raw + C::OFF_O);
   unsigned char* sBH = smem_raw + C::OFF_BH;
   unsigned char* sBL = smem_raw + C::OFF_BL;
   float* sWd = reinterpret_cast<float*>(smem_raw + C::OFF_WD);
@@ -243,11 +281,12 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   float* sCarry = reinterpret_cast<float*>(smem_raw + C::OFF_CARRY);
   float* sRed = reinterpret_cast<float*>(smem_raw + C::OFF_RED);
 
-  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull, bar_xempty, bar_afull,
-      bar_mma[2], bar_tempty[2], bar_lb[2], bar_cfull[2], bar_cempty[2];
+  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull, bar_xempty, bar_afull, bar_mma[2],
+      bar_tempty[2], bar_ofull, bar_oempty, bar_lb[NSLOT], bar_cfull[NSLOT], bar_cempty[NSLOT];
   __shared__ int s_tk[2];        // ticket staged in s stage 0/1 (-1: no more tiles)
-  __shared__ int s_atk;          // ticket whose operands sit in the A buffers (-1: stop)
-  __shared__ int s_lbtk[2];      // ticket handed to the look-back warp per slot (-1: stop)
+  __shared__ int s_atk[2];       // ticket of tile i's operands, by the parity of i (-1: stop)
+  __shared__ int s_otk[2];       // ticket of output tile j, by the parity of j (-1: stop, -2: skip)
+  __shared__ int s_lbtk[NSLOT];  // ticket handed to the look-back per slot (-1: stop)
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ int s_last;
@@ -268,21 +307,24 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
       mbar_init(&bar_sempty[s], (unsigned)C::NEW);
       mbar_init(&bar_mma[s], 1u);
       mbar_init(&bar_tempty[s], (unsigned)C::NEW);
-      mbar_init(&bar_lb[s], 1u);
+    }
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(&bar_lb[s], (unsigned)C::NCG);
       mbar_init(&bar_cfull[s], 1u);
       mbar_init(&bar_cempty[s], (unsigned)C::NEW);
     }
     mbar_init(&bar_xfull, 1u);
     mbar_init(&bar_xempty, (unsigned)C::NEW);
     mbar_init(&bar_afull, (unsigned)C::NEW);
+    mbar_init(&bar_ofull, (unsigned)C::NEW);
+    mbar_init(&bar_oempty, 1u);
     mbar_init_fence();
     s_abort = 0;
   }
   const unsigned epoch = *(volatile unsigned*)&ctrl->epoch;
   const int iter = *(volatile int*)&ctrl->iter;
-  float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;
 
-  // weights: W and W_lo in the K-major core-matrix layout (pre-packed), diagonals, b_hn
+  // weights: W_hi and W_lo in the K-major core-matrix layout (pre-packed), diagonals, b_hn
   {
     const float4* w4 = reinterpret_cast<const float4*>(P.wt);
     float4* d4 = reinterpret_cast<float4*>(sBH);   // sBH and sBL are contiguous
@@ -306,7 +348,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
 
   if (warp == 0) {
     // =========================== producer ===================================
-    const CUtensorMap* tm_s = P.tmaps + ((iter & 1) ? 1 : 0);   // rows of s^(i)
+    const CUtensorMap* tm_s = P.tmaps + ((iter & 1) ? 1 : 0);   // s^(i)
     const CUtensorMap* tm_x = P.tmaps + 2;                      // step inputs
     if (lane == 0) {
       tmap_acquire(tm_s);
@@ -328,13 +370,14 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
         ++it;
         break;
       }
-      const int row0 = (kg % B) * T + (kg / B) * L;   // global row of step t0
+      const int b = kg % B;
+      const int t0 = (kg / B) * L;
       if (lane == 0) {
-        // rows t0-1 .. t0+L-1; for the first chunk of a sequence row t0-1 is replaced by s0
-        // when the stage is split, rows past the end are zero-filled or unused
+        // steps t0-1 .. t0+L-1 (step -1 reads as zero and is replaced by s0 in the split)
         s_tk[st] = kg;
-        mbar_arrive_expect_tx(&bar_sfull[st], (unsigned)C::S_BYTES);
-        tma_load_2d(sS[st], tm_s, 0, row0 - 1, &bar_sfull[st]);
+        mbar_arrive_expect_tx(&bar_sfull[st], (unsigned)(NKH * C::SH_LOAD));
+#pragma unroll
+        for (int h = 0; h < NKH; ++h) tma_load_3d(sS + (st * NKH + h) * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[st]);
       }
       // the single step-input buffer: wait until the previous tile's inputs were consumed
       if (it >= 1 && !mbar_wait_flag(&bar_xempty, ((unsigned)(it - 1)) & 1u, ctrl, tmo, &s_abort)) {
@@ -343,7 +386,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
       }
       if (lane == 0) {
         mbar_arrive_expect_tx(&bar_xfull, (unsigned)C::X_BYTES);
-        tma_load_2d(sX, tm_x, 0, row0, &bar_xfull);
+        tma_load_3d(sX, tm_x, 0, t0, b, &bar_xfull);
       }
       __syncwarp();
       x_issued = it + 1;
@@ -355,52 +398,103 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     if (x_issued > 0 && !mbar_drain(&bar_xfull, ((unsigned)(x_issued - 1)) & 1u, tmo) && lane == 0)
       atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
   } else if (warp == 1) {
-    // =========================== MMA issuer =================================
+    // ======================= MMA and store issuer ============================
     constexpr uint32_t idesc = umma_idesc_tf32(L, N);
+    constexpr uint32_t SBO_B = (K / 4) * 128;
+    const CUtensorMap* tm_o = P.tmaps + ((iter & 1) ? 3 : 4);   // s^(i+1) goes to the other buffer
+    if (lane == 0) tmap_acquire(tm_o);
+    int nstored = 0;   // output tiles taken so far
+    // output tile j: wait until it is staged, store it, release the staging buffer.
+    // Returns false at the stop marker or when the wait gave up.
+    auto store_tile = [&](int j) -> bool {
+      if (!mbar_wait_flag(&bar_ofull, (unsigned)j & 1u, ctrl, tmo, &s_abort)) return false;
+      const int kgj = s_otk[j & 1];
+      if (kgj == -1) return false;
+      if (lane == 0) {
+        if (kgj >= 0) {
+          tma_store_3d(tm_o, 0, (kgj / B) * L, kgj % B, sO);
+          bulk_commit();
+          bulk_wait_read();
+        }
+        mbar_arrive(&bar_oempty);
+      }
+      __syncwarp();
+      nstored = j + 1;
+      return true;
+    };
     int issued = 0;
     for (int it = 0;; ++it) {
       if (!mbar_wait_flag(&bar_afull, (unsigned)it & 1u, ctrl, tmo, &s_abort)) break;
-      if (s_atk < 0) break;
+      if (s_atk[it & 1] < 0) break;
       const int buf = it & 1;
       if (it >= 2 && !mbar_wait_flag(&bar_tempty[buf], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t d = tmem + (uint32_t)(buf * C::TCOLS);
-        const uint32_t ah = smem_addr(sAH), al = smem_addr(sAL), bh = smem_addr(sBH), bl = smem_addr(sBL);
+        const uint32_t s_hi = smem_addr(sS + (it & 1) * NKH * C::SH_BYTES), s_lo = smem_addr(sLo);
+        const uint32_t bh = smem_addr(sBH), bl = smem_addr(sBL);
 #pragma unroll 1
         for (int pass = 0; pass < 3; ++pass) {
-          const uint32_t a = (pass == 2) ? al : ah;
-          const uint32_t bb = (pass == 1) ? bl : bh;
+          // pass 0: S_hi W_hi, pass 1: S_hi W_lo, pass 2: S_lo W_hi
 #pragma unroll
-          for (int kb = 0; kb < K / 8; ++kb)
-            umma_tf32(d, umma_smem_desc(a + kb * 256, 128, C::SBO_A), umma_smem_desc(bb + kb * 256, 128, C::SBO_B),
+          for (int kb = 0; kb < K / 8; ++kb) {
+            const int h = kb >> 2;   // column half; 4 K-steps of 32 bytes per 128-byte swizzled row
+            const uint32_t a = (pass == 2) ? (s_lo + h * C::LO_BYTES) : (s_hi + h * C::SH_BYTES);
+            const uint32_t bb = (pass == 1) ? bl : bh;
+            umma_tf32(d, umma_smem_desc(a + (kb & 3) * 32, 16, 1024, 2), umma_smem_desc(bb + kb * 256, 128, SBO_B, 0),
                       idesc, (pass > 0 || kb > 0) ? 1u : 0u);
+          }
         }
         umma_commit(&bar_mma[buf]);
       }
       __syncwarp();
       issued = it + 1;
+      // the output tile staged in epilogue tile it-1 (after it released the operands of tile it)
+      const int j = it - 1 - C::OUT_LAG;
+      if (j >= 0 && !store_tile(j)) break;
     }
     // every issued product must have completed before TMEM is released
     for (int j = max(0, issued - 2); j < issued; ++j)
       if (!mbar_drain(&bar_mma[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
         atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
-  } else if (warp == 2) {
+    // the remaining output tiles, up to the stop marker
+    for (int j = nstored;; ++j)
+      if (!store_tile(j)) break;
+    if (lane == 0) bulk_wait_all();   // the states are in global memory before the CTA retires
+  } else if (warp < C::WE0) {
     // =========================== look-back ==================================
+    // warp 2 + j takes tiles j, j + NLB, j + 2 NLB, ... of this CTA
     if constexpr (kScan) {
-      for (int it = 0;; ++it) {
-        const int slot = it & 1;
-        if (!mbar_wait_flag(&bar_lb[slot], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort)) break;
+      for (int it = warp - 2;; it += C::NLB) {
+        const int slot = it % NSLOT;
+        const unsigned ph = (unsigned)(it / NSLOT) & 1u;
+        if (!mbar_wait_flag(&bar_lb[slot], ph, ctrl, tmo, &s_abort)) break;
         const int kg = s_lbtk[slot];
         if (kg < 0) break;
-        if (it >= 2 && !mbar_wait_flag(&bar_cempty[slot], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
         const int b = kg % B;
         const int chunk = kg / B;
         const size_t k = (size_t)kg;
         const bool stall = (A.stall_ticket == kg);
-        const float* agg = sAgg + slot * DP * 2;
+        float2 ag[C::NQ];
+#pragma unroll
+        for (int q = 0; q < C::NQ; ++q) {
+          const int j = lane + 32 * q;
+          ag[q] = (j < DP) ? *reinterpret_cast<const float2*>(sAgg + (slot * DP + j) * 2) : make_float2(1.0f, 0.0f);
+        }
+        // 1. the tile aggregate, for successors that reach this tile before its state
+        if (chunk > 0 && !stall) {
+#pragma unroll
+          for (int q = 0; q < C::NQ; ++q) {
+            const int j = lane + 32 * q;
+            if (j < DP) reinterpret_cast<float2*>(P.agg + k * P.agg_stride)[j] = ag[q];
+          }
+          // the warp barrier orders the other lanes' stores before lane 0's release,
+          // which is cumulative: a reader that acquires the flag sees all of them
+          __syncwarp();
+          if (lane == 0) st_release(P.flags + k, make_flag(epoch, kFlagAgg));
+        }
+        // 2. the carry: nearest published state, then the aggregates in between
         const int n_agg = lookback_find_prefix(P.flags, k, stride, chunk, epoch, ctrl, tmo);
-        __syncwarp();
         float carry[C::NQ];
 #pragma unroll
         for (int q = 0; q < C::NQ; ++q) {
@@ -418,18 +512,9 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
           }
           carry[q] = v;
         }
-        if (n_agg >= 0 && !stall) {
-#pragma unroll
-          for (int q = 0; q < C::NQ; ++q) {
-            const int j = lane + 32 * q;
-            if (j < DP) P.pref[k * P.pref_stride + j] = fmaf(agg[2 * j], carry[q], agg[2 * j + 1]);
-          }
-          // the warp barrier orders the other lanes' stores before lane 0's release,
-          // which is cumulative: a reader that acquires the flag sees all of them
-          __syncwarp();
-          if (lane == 0) st_release(P.flags + k, make_flag(epoch, kFlagPrefix));
-        }
         if (n_agg < 0) s_abort = 1;
+        // 3. hand the carry to the epilogue (its slot is free once tile it - NSLOT was formed)
+        if (it >= NSLOT && !mbar_wait_flag(&bar_cempty[slot], ph ^ 1u, ctrl, tmo, &s_abort)) break;
 #pragma unroll
         for (int q = 0; q < C::NQ; ++q) {
           const int j = lane + 32 * q;
@@ -437,130 +522,153 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_cfull[slot]);
+        // 4. the tile's end state
+        if (n_agg >= 0 && !stall) {
+#pragma unroll
+          for (int q = 0; q < C::NQ; ++q) {
+            const int j = lane + 32 * q;
+            if (j < DP) P.pref[k * P.pref_stride + j] = fmaf(ag[q].x, carry[q], ag[q].y);
+          }
+          __syncwarp();
+          if (lane == 0) st_release(P.flags + k, make_flag(epoch, kFlagPrefix));
+        }
       }
     }
   } else {
     // =========================== epilogue ===================================
-    const int e = warp - 3;                 // 0 .. NEW-1
+    const int e = warp - C::WE0;            // 0 .. NEW-1
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int cg = e >> 2;                  // channel group
     const int row = quarter * 32 + lane;    // step row within the tile
     const int cbase = cg * CH;              // first channel of this thread
-    const int te = tid - 96;                // 0 .. NTE-1 among the epilogue threads
+    const int te = tid - 32 * C::WE0;       // 0 .. NTE-1 among the epilogue threads
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int hh = cbase >> 5;              // column half of this thread's channels
+    const int cw = cbase & 31;              // first column within that half
 
-    // Operand split of stage S: tf32(S) and tf32(S - tf32(S)) in the K-major
-    // core-matrix layout.  For the first chunk of a sequence the stage's row 0
-    // (time -1) is s0, written into the stage here as well for the cell phase.
-    auto split = [&](float* S, int kgs) {
+    // S_lo of stage `stg` (rows 0..L-1), in the same swizzled layout.  For the first
+    // chunk of a sequence, row 0 (step -1, loaded as zero) becomes s0 first.
+    auto split = [&](int stg, int kgs) {
       const bool first = (kgs / B) == 0;
       const float* s0row = A.s0 + (size_t)(kgs % B) * D;
-      for (int c = te; c < L * (K / 4); c += NTE) {
-        const int r = (c & 7) + 8 * ((c >> 3) / (K / 4));
-        const int kq = (c >> 3) % (K / 4);
+      for (int u = te; u < NKH * L * 8; u += NTE) {
+        const int q = u & 7;             // 16-byte chunk within the 128-byte row
+        const int r = (u >> 3) % L;
+        const int h = (u >> 3) / L;
+        const uint32_t off = sw128_offset(r, 4 * q);
+        unsigned char* srow = sS + (stg * NKH + h) * C::SH_BYTES;
         float4 v;
         if (first && r == 0) {
-          v = __ldg(reinterpret_cast<const float4*>(s0row) + kq);
-          *reinterpret_cast<float4*>(S + kq * 4) = v;
+          v = __ldg(reinterpret_cast<const float4*>(s0row + 32 * h) + q);
+          *reinterpret_cast<float4*>(srow + off) = v;
         } else {
-          v = *reinterpret_cast<const float4*>(S + r * SP + kq * 4);
+          v = *reinterpret_cast<const float4*>(srow + off);
         }
-        const float4 hi = make_float4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z), tf32_round(v.w));
-        const float4 lo = make_float4(tf32_round(v.x - hi.x), tf32_round(v.y - hi.y), tf32_round(v.z - hi.z),
-                                      tf32_round(v.w - hi.w));
-        const uint32_t off = kmajor_offset(r, kq * 4, K);
-        *reinterpret_cast<float4*>(sAH + off) = hi;
-        *reinterpret_cast<float4*>(sAL + off) = lo;
+        *reinterpret_cast<float4*>(sLo + h * C::LO_BYTES + off) =
+            make_float4(tf32_tail(v.x), tf32_tail(v.y), tf32_tail(v.z), tf32_tail(v.w));
       }
-      fence_async_smem();   // generic writes -> async proxy (tensor cores, next TMA fill)
+      fence_async_smem();   // generic writes -> async proxy (tensor cores)
     };
 
-    // s^(i+1) of tile j from its parked prefixes and the carry of the look-back warp
+    // hand the staged rows of output tile j (ticket kgj) to the store issuer
+    auto publish_out = [&](int j, int kgj) {
+      fence_async_smem();   // this thread's staging writes -> async proxy (the TMA store)
+      __syncwarp();
+      if (lane == 0) {
+        if (te == 0) s_otk[j & 1] = s_abort ? -2 : kgj;
+        mbar_arrive(&bar_ofull);
+      }
+    };
+
+    // s^(i+1) of tile j from its parked prefixes and the carry of the look-back
     auto write_out = [&](int j, int kgj) {
-      const int slot = j & 1;
-      mbar_wait_flag(&bar_cfull[slot], ((unsigned)j >> 1) & 1u, ctrl, tmo, &s_abort);
+      const int slot = j % NSLOT;
+      mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort);
+      if (j >= 1) mbar_wait_flag(&bar_oempty, (unsigned)(j - 1) & 1u, ctrl, tmo, &s_abort);   // staging free
       const float* cr = sCarry + slot * DP + cbase;
-      const int bj = kgj % B;
-      const int tj = (kgj / B) * L + row;
-      const bool okj = (tj < T) && !s_abort;
       const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS) + lane_off;
       float bb[16], aa[16];
       tmem_ld16(sbase + (uint32_t)((kHasA ? DP : 0) + cbase), bb);
       if constexpr (kHasA) tmem_ld16(sbase + (uint32_t)cbase, aa);
-      if (okj) {
-        float* o = dst + ((size_t)bj * T + tj) * D + cbase;
+      float* o = sO + row * SP + cbase;
 #pragma unroll
-        for (int c4 = 0; c4 < CH; c4 += 4) {
-          const float4 c = *reinterpret_cast<const float4*>(cr + c4);
-          float4 v;
-          if constexpr (kHasA) {
-            v = make_float4(fmaf(aa[c4], c.x, bb[c4]), fmaf(aa[c4 + 1], c.y, bb[c4 + 1]),
-                            fmaf(aa[c4 + 2], c.z, bb[c4 + 2]), fmaf(aa[c4 + 3], c.w, bb[c4 + 3]));
-          } else {
-            v = make_float4(c.x + bb[c4], c.y + bb[c4 + 1], c.z + bb[c4 + 2], c.w + bb[c4 + 3]);
-          }
-          *reinterpret_cast<float4*>(o + c4) = v;
+      for (int c4 = 0; c4 < CH; c4 += 4) {
+        const float4 c = *reinterpret_cast<const float4*>(cr + c4);
+        float4 v;
+        if constexpr (kHasA) {
+          v = make_float4(fmaf(aa[c4], c.x, bb[c4]), fmaf(aa[c4 + 1], c.y, bb[c4 + 1]),
+                          fmaf(aa[c4 + 2], c.z, bb[c4 + 2]), fmaf(aa[c4 + 3], c.w, bb[c4 + 3]));
+        } else {
+          v = make_float4(c.x + bb[c4], c.y + bb[c4 + 1], c.z + bb[c4 + 2], c.w + bb[c4 + 3]);
         }
+        *reinterpret_cast<float4*>(o + c4) = v;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_cempty[slot]);
+      publish_out(j, kgj);
     };
 
     // prologue: operands of the first tile
     {
       int kg0 = -1;
       if (mbar_wait_flag(&bar_sfull[0], 0u, ctrl, tmo, &s_abort)) kg0 = s_tk[0];
-      if (kg0 >= 0) split(sS[0], kg0);
+      if (kg0 >= 0) split(0, kg0);
       __syncwarp();
-      named_barrier(1, NTE);
       if (lane == 0) {
-        if (te == 0) s_atk = s_abort ? -1 : kg0;
+        if (te == 0) s_atk[0] = s_abort ? -1 : kg0;
         mbar_arrive(&bar_afull);
       }
     }
     named_barrier(1, NTE);
-    int kg = s_atk;   // written by te == 0 before the barrier
+    int kg = s_atk[0];   // written by te == 0 before the barrier
     int it = 0;
-    int prev_kg = -1;
+    int kg_m1 = -1, kg_m2 = -1;   // tickets of tiles it-1 and it-2
     for (; kg >= 0; ++it) {
       const int st = it & 1;
       const int buf = it & 1;
-      const int b = kg % B;
       const int chunk = kg / B;
       const int t = chunk * L + row;
-      const float* S = sS[st];
+      const unsigned char* Sst = sS + st * NKH * C::SH_BYTES + hh * C::SH_BYTES;
 
       // ---- Z from TMEM, then the cell --------------------------------------
       mbar_wait_flag(&bar_mma[buf], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort);
       tc_fence_after();
       float z[R][CH];
 #pragma unroll
-      for (int q = 0; q < R; ++q) tmem_ld16(tmem + (uint32_t)(buf * C::TCOLS) + lane_off + (uint32_t)(q * DP + cbase), z[q]);
+      for (int q = 0; q < R; ++q)
+        tmem_ld16(tmem + (uint32_t)(buf * C::TCOLS) + lane_off + (uint32_t)(q * DP + cbase), z[q]);
       mbar_wait_flag(&bar_xfull, (unsigned)it & 1u, ctrl, tmo, &s_abort);
       const bool tok = (t < T);
       float av[CH], bv[CH];
 #pragma unroll
       for (int c4 = 0; c4 < CH; c4 += 4) {
         const int c = cbase + c4;
-        const float4 sp4 = *reinterpret_cast<const float4*>(S + row * SP + c);
-        const float4 sc4 = *reinterpret_cast<const float4*>(S + (row + 1) * SP + c);
+        const float4 sp4 = *reinterpret_cast<const float4*>(Sst + sw128_offset(row, cw + c4));
+        const float4 sc4 = *reinterpret_cast<const float4*>(Sst + sw128_offset(row + 1, cw + c4));
         float4 x4[R];
 #pragma unroll
         for (int q = 0; q < R; ++q) x4[q] = *reinterpret_cast<const float4*>(sX + row * XP + q * DP + c);
+        float4 wd4[R];
+#pragma unroll
+        for (int q = 0; q < R; ++q) wd4[q] = *reinterpret_cast<const float4*>(sWd + q * DP + c);
+        const float4 bhn4 = *reinterpret_cast<const float4*>(sBhn + c);
         const float spv[4] = {sp4.x, sp4.y, sp4.z, sp4.w};
         const float scv[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
+        const float bhv[4] = {bhn4.x, bhn4.y, bhn4.z, bhn4.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int cc = c + u;
-          float xv[R];
+          float xv[R], wd[R];
 #pragma unroll
-          for (int q = 0; q < R; ++q) xv[q] = (u == 0) ? x4[q].x : (u == 1) ? x4[q].y : (u == 2) ? x4[q].z : x4[q].w;
+          for (int q = 0; q < R; ++q) {
+            xv[q] = (u == 0) ? x4[q].x : (u == 1) ? x4[q].y : (u == 2) ? x4[q].z : x4[q].w;
+            wd[q] = (u == 0) ? wd4[q].x : (u == 1) ? wd4[q].y : (u == 2) ? wd4[q].z : wd4[q].w;
+          }
           const float sp = spv[u], sc = scv[u];
           float y, a, bb, res;
           if constexpr (CELL == PN_CELL_TANH_RNN) {
             y = tanh_pn(z[0][c4 + u] + xv[0]);
             res = sc - y;
-            a = (MODE == PN_QUASI) ? (1.0f - y * y) * sWd[cc] : (MODE == PN_PICARD ? 1.0f : 0.0f);
+            a = (MODE == PN_QUASI) ? (1.0f - y * y) * wd[0] : (MODE == PN_PICARD ? 1.0f : 0.0f);
             bb = (MODE == PN_JACOBI) ? y : y - a * sp;
           } else if constexpr (CELL == PN_CELL_EULER_TANH) {
             const float gg = tanh_pn(z[0][c4 + u] + xv[0]);
@@ -568,7 +676,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
             y = sp + eg;
             res = (sc - sp) - eg;
             if (MODE == PN_QUASI) {
-              const float ed = P.eps * (1.0f - gg * gg) * sWd[cc];
+              const float ed = P.eps * (1.0f - gg * gg) * wd[0];
               a = 1.0f + ed;
               bb = eg - ed * sp;
             } else if (MODE == PN_PICARD) {
@@ -581,15 +689,14 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
           } else {
             const float rr = sigmoidf_acc(xv[0] + z[0][c4 + u]);
             const float zz = sigmoidf_acc(xv[1] + z[1][c4 + u]);
-            const float hn = z[2][c4 + u] + sBhn[cc];
+            const float hn = z[2][c4 + u] + bhv[u];
             const float nn = tanh_pn(xv[2] + rr * hn);
             y = nn + zz * (sp - nn);
             res = sc - y;
             if (MODE == PN_QUASI) {
               const float omz = 1.0f - zz;
               const float dn = omz * (1.0f - nn * nn);
-              a = zz + (sp - nn) * zz * omz * sWd[DP + cc] +
-                  dn * (rr * sWd[2 * DP + cc] + hn * rr * (1.0f - rr) * sWd[cc]);
+              a = zz + (sp - nn) * zz * omz * wd[1] + dn * (rr * wd[2] + hn * rr * (1.0f - rr) * wd[0]);
             } else {
               a = (MODE == PN_PICARD) ? 1.0f : 0.0f;
             }
@@ -618,27 +725,29 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
       {
         int kn = -1;
         if (mbar_wait_flag(&bar_sfull[st ^ 1], (((unsigned)it + 1u) >> 1) & 1u, ctrl, tmo, &s_abort)) kn = s_tk[st ^ 1];
-        if (kn >= 0 && !s_abort) split(sS[st ^ 1], kn);
+        if (kn >= 0 && !s_abort) split(st ^ 1, kn);
         __syncwarp();
-        named_barrier(1, NTE);   // every epilogue thread has written its part of the split
         if (lane == 0) {
-          if (te == 0) s_atk = s_abort ? -1 : kn;   // also the loop's exit decision, read after the last barrier
+          // the ticket of tile it+1 is also the loop's exit decision, read after the next barrier
+          if (te == 0) s_atk[(it + 1) & 1] = s_abort ? -1 : kn;
           mbar_arrive(&bar_afull);
         }
       }
-      // the previous tile's carry had this tile's cell phase to arrive: write it out now
-      if constexpr (kScan) {
-        if (it > 0) write_out(it - 1, prev_kg);
-      }
 
       if constexpr (!kScan) {
-        if (tok && !s_abort) {
-          float* o = dst + ((size_t)b * T + t) * D + cbase;
+        // s^(i+1) = f(s^(i)) row by row: stage it for the store issuer
+        if (it >= 1) mbar_wait_flag(&bar_oempty, (unsigned)(it - 1) & 1u, ctrl, tmo, &s_abort);
+        float* o = sO + row * SP + cbase;
 #pragma unroll
-          for (int c4 = 0; c4 < CH; c4 += 4)
-            *reinterpret_cast<float4*>(o + c4) = make_float4(bv[c4], bv[c4 + 1], bv[c4 + 2], bv[c4 + 3]);
-        }
+        for (int c4 = 0; c4 < CH; c4 += 4)
+          *reinterpret_cast<float4*>(o + c4) = make_float4(bv[c4], bv[c4 + 1], bv[c4 + 2], bv[c4 + 3]);
+        publish_out(it, kg);
+        named_barrier(1, NTE);
+        kg = s_atk[(it + 1) & 1];
       } else {
+        // the states of tile it-2: its carry had two tiles of time to arrive
+        if (it >= C::DEFER) write_out(it - C::DEFER, kg_m2);
+
         // ---- scan along the rows: within the warp (a level at a time over all 16
         //      channels, so the shuffles of one level are independent), then across quarters
 #pragma unroll
@@ -657,13 +766,15 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
             }
           }
         }
+        float* tot = sTot + (it & 1) * C::TOT_FLOATS;
         if (lane == 31) {
 #pragma unroll
           for (int c = 0; c < CH; c += 2)
-            *reinterpret_cast<float4*>(sTot + ((cg * 4 + quarter) * CH + c) * 2) =
+            *reinterpret_cast<float4*>(tot + ((cg * 4 + quarter) * CH + c) * 2) =
                 make_float4(kHasA ? av[c] : 1.0f, bv[c], kHasA ? av[c + 1] : 1.0f, bv[c + 1]);
         }
-        named_barrier(1, NTE);
+        named_barrier(1, NTE);   // quarter totals, and the ticket of tile it+1
+        const int kg_next = s_atk[(it + 1) & 1];
         if (quarter > 0) {
           // prefix of the earlier quarters: tot_{quarter-1} o ... o tot_0
           float PA[CH], PB[CH];
@@ -673,7 +784,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
             PB[c] = 0.0f;
           }
           for (int qq = 0; qq < quarter; ++qq) {
-            const float* tq = sTot + (cg * 4 + qq) * CH * 2;
+            const float* tq = tot + (cg * 4 + qq) * CH * 2;
 #pragma unroll
             for (int c = 0; c < CH; c += 2) {
               const float4 w = *reinterpret_cast<const float4*>(tq + c * 2);
@@ -689,54 +800,46 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
             if (kHasA) av[c] *= PA[c];
           }
         }
-        // the last row holds the tile aggregate
-        const int slot = it & 1;
+        // the last row holds the tile aggregate: hand it to the look-back
+        const int slot = it % NSLOT;
         if (quarter == 3 && lane == 31) {
 #pragma unroll
           for (int c = 0; c < CH; c += 2)
             *reinterpret_cast<float4*>(sAgg + (slot * DP + cbase + c) * 2) =
                 make_float4(kHasA ? av[c] : 1.0f, bv[c], kHasA ? av[c + 1] : 1.0f, bv[c + 1]);
+          if (cg == 0) s_lbtk[slot] = s_abort ? -1 : kg;
+          mbar_arrive(&bar_lb[slot]);
         }
-        named_barrier(1, NTE);
-        if (e == 0) {   // publish the aggregate, then wake the look-back warp
-          const bool stall = (A.stall_ticket == kg);
-          const int ab = __shfl_sync(0xffffffffu, (int)s_abort, 0);   // one value for the whole warp
-          if (chunk > 0 && !stall && !ab) {
-#pragma unroll
-            for (int q = 0; q < C::NQ; ++q) {
-              const int j = lane + 32 * q;
-              if (j < DP)
-                reinterpret_cast<float2*>(P.agg + (size_t)kg * P.agg_stride)[j] =
-                    *reinterpret_cast<const float2*>(sAgg + (slot * DP + j) * 2);
-            }
-            __syncwarp();   // lane 0's release is cumulative over the lanes' stores ordered before it
-            if (lane == 0) st_release(P.flags + kg, make_flag(epoch, kFlagAgg));
-          }
-          __syncwarp();
-          if (lane == 0) {
-            s_lbtk[slot] = ab ? -1 : kg;
-            mbar_arrive(&bar_lb[slot]);
-          }
-        }
-        // ---- park this tile's in-tile prefixes in TMEM; written out next tile
+        // ---- park this tile's in-tile prefixes in TMEM; formed two tiles later
         {
           const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS) + lane_off;
           if constexpr (kHasA) tmem_st16(sbase + (uint32_t)cbase, av);
           tmem_st16(sbase + (uint32_t)((kHasA ? DP : 0) + cbase), bv);
           tmem_st_wait();
         }
-        prev_kg = kg;
+        kg_m2 = kg_m1;
+        kg_m1 = kg;
+        kg = kg_next;
       }
-      named_barrier(1, NTE);   // uniform exit decision (s_atk was set by te == 0 above)
-      kg = s_atk;
     }
     if constexpr (kScan) {
-      if (it > 0) write_out(it - 1, prev_kg);
-      // stop the look-back warp: its next slot is the `it`-th
-      if (e == 0 && lane == 0) {
-        s_lbtk[it & 1] = -1;
-        mbar_arrive(&bar_lb[it & 1]);
+      if (it >= 2) write_out(it - 2, kg_m2);
+      if (it >= 1) write_out(it - 1, kg_m1);
+      // stop the look-back warps: their next tiles are it .. it + NLB - 1
+      if (quarter == 3 && lane == 31) {
+        for (int j = it; j < it + C::NLB; ++j) {
+          if (cg == 0) s_lbtk[j % NSLOT] = -1;
+          mbar_arrive(&bar_lb[j % NSLOT]);
+        }
       }
+    }
+    // stop the store issuer once it has taken the last tile (a warp arrives on
+    // bar_ofull again only after the previous phase completed)
+    if (it >= 1) mbar_wait_flag(&bar_oempty, (unsigned)(it - 1) & 1u, ctrl, tmo, &s_abort);
+    __syncwarp();
+    if (lane == 0) {
+      if (te == 0) s_otk[it & 1] = -1;
+      mbar_arrive(&bar_ofull);
     }
   }
 
