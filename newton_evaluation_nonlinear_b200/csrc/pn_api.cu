@@ -87,6 +87,7 @@ struct pn_ctx {
   bool tc_capable = false;
   long long evals = 0;
   int last_iters = -1;
+  int last_kind = -1;          // kernel kind of the last iteration launch (look-back buffer format)
   std::string err;
 };
 
@@ -428,13 +429,25 @@ pn_status validate_mode(pn_ctx* h, int mode, int max_iters, float tol) {
   return PN_OK;
 }
 
-pn_status reset_flags_if_needed(pn_ctx* h) {
-  // Flags carry the 30-bit launch epoch; clear them long before it wraps.
-  if (h->ctrl_h->epoch > (1u << 29)) {
+// Prepares the look-back buffers for a launch of `mode`'s kernel.  Flags and
+// tagged words carry the 30-bit launch epoch: clear them long before it
+// wraps.  The tensor-core kernels read the aggregate and state buffers as
+// tagged words, the others as plain floats: clear them when the format changes
+// so no word of one format is ever read as the other.
+pn_status prepare_lookback(pn_ctx* h, int mode) {
+  const int kind = h->fam.k[mode].kind;
+  const bool wrap = h->ctrl_h->epoch > (1u << 29);
+  const bool format = (kind != h->last_kind) && (kind == kKindDiagTc || h->last_kind == kKindDiagTc);
+  if (wrap) {
     PN_CUDA(h, cudaMemsetAsync(h->flags, 0, h->nflags * sizeof(unsigned), h->stream));
     PN_CUDA(h, cudaMemsetAsync(&h->ctrl->epoch, 0, sizeof(unsigned), h->stream));
     h->ctrl_h->epoch = 0;
   }
+  if (wrap || format) {
+    PN_CUDA(h, cudaMemsetAsync(h->agg, 0, h->agg_floats * sizeof(float), h->stream));
+    PN_CUDA(h, cudaMemsetAsync(h->pref, 0, h->pref_floats * sizeof(float), h->stream));
+  }
+  h->last_kind = kind;
   return PN_OK;
 }
 
@@ -452,7 +465,7 @@ pn_status upload_tc_maps(pn_ctx* h, int mode) {
 // The loop body shared by pn_eval and pn_eval_host: args already point at
 // device buffers.
 pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
-  pn_status st = reset_flags_if_needed(h);
+  pn_status st = prepare_lookback(h, mode);
   if (st != PN_OK) return st;
   h->args_h->use_cond = h->device_loop ? 1 : 0;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
@@ -521,9 +534,11 @@ pn_status select_kernels(pn_ctx* h) {
     h->fam.grid[m] = (int)std::min<long long>(want, h->fam.ntiles[m]);
     const size_t G = (size_t)ki.G;
     const size_t nt = (size_t)h->fam.ntiles[m];
-    const size_t aggf = nt * ((m == PN_NEWTON) ? G * (G + 1) : 2 * G);
+    // the tensor-core kernels publish 64-bit tagged words: twice the floats
+    const size_t wf = (ki.kind == kKindDiagTc) ? 2 : 1;
+    const size_t aggf = nt * ((m == PN_NEWTON) ? G * (G + 1) : 2 * G) * wf;
     h->agg_floats = std::max(h->agg_floats, aggf);
-    h->pref_floats = std::max(h->pref_floats, nt * G);
+    h->pref_floats = std::max(h->pref_floats, nt * G * wf);
     h->nflags = std::max(h->nflags, nt);
   }
   for (int m = 0; m < 4; ++m) {
@@ -830,6 +845,7 @@ pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* a
   h->args_h->tol = INFINITY;
   h->args_h->max_iters = INT_MAX;
   h->args_h->use_cond = 0;
+  if ((st = prepare_lookback(h, mode)) != PN_OK) return st;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
   if ((st = upload_tc_maps(h, mode)) != PN_OK) return st;
   cudaEvent_t e0, e1;

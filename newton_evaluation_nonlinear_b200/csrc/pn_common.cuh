@@ -90,7 +90,34 @@ __device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_re
 __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ void st_relaxed(unsigned* p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ int ld_volatile(const int* p) { return *(const volatile int*)p; }
+
+// Self-validating look-back words: a float value in the low 32 bits and the
+// launch epoch in the high 32 bits of one aligned 64-bit word.  A 64-bit
+// access is single-copy atomic, so a reader that sees the expected epoch sees
+// the value written with it; no fence is needed on either side.
+__device__ __forceinline__ unsigned long long tag_word(float v, unsigned tag) {
+  return ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(v);
+}
+__device__ __forceinline__ float word_value(unsigned long long w) { return __uint_as_float((unsigned)w); }
+__device__ __forceinline__ bool word_tagged(unsigned long long w, unsigned tag) { return (unsigned)(w >> 32) == tag; }
+__device__ __forceinline__ void st_word(unsigned long long* p, unsigned long long w) {
+  asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ void st_word2(unsigned long long* p, unsigned long long w0, unsigned long long w1) {
+  asm volatile("st.volatile.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(w0), "l"(w1) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_word(const unsigned long long* p) {
+  unsigned long long w;
+  asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+__device__ __forceinline__ void ld_word2(const unsigned long long* p, unsigned long long& w0, unsigned long long& w1) {
+  asm volatile("ld.volatile.global.v2.u64 {%0, %1}, [%2];" : "=l"(w0), "=l"(w1) : "l"(p) : "memory");
+}
 __device__ __forceinline__ unsigned long long globaltimer() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -105,12 +132,13 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 // It waits (bounded) until every predecessor nearer than that one has at least
 // published its aggregate.  Returns the number of aggregate-only tiles between
 // this tile and that prefix, or -1 when it gave up (timeout, or another CTA's
-// error).  Flags are polled with relaxed loads; one fence after the final
-// poll gives the caller's subsequent loads of the aggregates and the prefix
-// acquire semantics.
+// error).  Flags are polled with relaxed loads; with `acquire`, one fence
+// after the final poll gives the caller's subsequent loads of the aggregates
+// and the prefix acquire semantics (flags published with a release store).
+// Without it the flags are hints and the caller validates the data itself.
 __device__ __forceinline__ int lookback_find_prefix(const unsigned* flags, size_t k, size_t stride,
                                                     int chunk, unsigned epoch, Ctrl* ctrl,
-                                                    long long timeout_ns) {
+                                                    long long timeout_ns, bool acquire = true) {
   const int lane = threadIdx.x & 31;
   int n_agg = 0;
   int base = chunk - 1;   // nearest chunk of this window
@@ -130,7 +158,7 @@ __device__ __forceinline__ int lookback_find_prefix(const unsigned* flags, size_
     const unsigned need = (nearest >= 31) ? 0xffffffffu : ((2u << nearest) - 1u);
     if ((vm & need) == need) {
       if (nearest < 32) {
-        fence_acquire_gpu();
+        if (acquire) fence_acquire_gpu();
         return n_agg + nearest;
       }
       n_agg += 32;

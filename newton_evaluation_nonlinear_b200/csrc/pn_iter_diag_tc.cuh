@@ -194,6 +194,80 @@ __device__ __forceinline__ bool mbar_wait_flag(uint64_t* bar, unsigned parity, C
   }
 }
 
+// Launch tag of the self-validating look-back words: never 0, so memory that
+// was only cleared never validates.
+__device__ __forceinline__ unsigned lookback_tag(unsigned epoch) { return 0x80000000u | epoch; }
+
+// Gives up a warp-wide spin: true (for all lanes) when another CTA reported an
+// error or this wait ran past timeout_ns (then it reports PN_ERR_TIMEOUT).
+__device__ __forceinline__ bool spin_give_up(unsigned& spins, unsigned long long t0, Ctrl* ctrl, long long timeout_ns) {
+  int g = 0;
+  if ((++spins & 15u) == 0u && (threadIdx.x & 31) == 0) {
+    if (ld_volatile(&ctrl->error)) g = 1;
+    else if ((long long)(globaltimer() - t0) > timeout_ns) {
+      atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+      g = 1;
+    }
+  }
+  return __shfl_sync(0xffffffffu, g, 0) != 0;
+}
+
+// A published state: the DP words of one tile, lane j holding channels
+// j + 32 q.  Spins (bounded) until every word carries `tag`.
+template <int DP, int NQ>
+__device__ __forceinline__ bool ld_tagged_state(const unsigned long long* src, unsigned tag, float (&v)[NQ], Ctrl* ctrl,
+                                                long long timeout_ns) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long w[NQ];
+  unsigned long long t0 = 0;
+  unsigned spins = 0;
+  while (true) {
+    bool ok = true;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int j = lane + 32 * q;
+      w[q] = (j < DP) ? ld_word(src + j) : tag_word(0.0f, tag);
+      ok = ok && word_tagged(w[q], tag);
+    }
+    if (__all_sync(0xffffffffu, ok)) break;
+    if (spins == 0) t0 = globaltimer();
+    if (spin_give_up(spins, t0, ctrl, timeout_ns)) return false;
+  }
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) v[q] = word_value(w[q]);
+  return true;
+}
+
+// Aggregates of the tiles d0, d0-1, .., d0-3 places back (k - d * stride,
+// those with d >= 1), loaded together; spins (bounded) until all validate.
+template <int DP, int NQ>
+__device__ __forceinline__ bool ld_tagged_aggs(const unsigned long long* aggw, size_t k, size_t stride, int d0,
+                                               unsigned tag, float (&fa)[4][NQ], float (&fb)[4][NQ], Ctrl* ctrl,
+                                               long long timeout_ns) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long t0 = 0;
+  unsigned spins = 0;
+  while (true) {
+    bool ok = true;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int d = d0 - u;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int j = lane + 32 * q;
+        unsigned long long wa = tag_word(1.0f, tag), wb = tag_word(0.0f, tag);
+        if (d >= 1 && j < DP) ld_word2(aggw + ((k - (size_t)d * stride) * DP + j) * 2, wa, wb);
+        ok = ok && word_tagged(wa, tag) && word_tagged(wb, tag);
+        fa[u][q] = word_value(wa);
+        fb[u][q] = word_value(wb);
+      }
+    }
+    if (__all_sync(0xffffffffu, ok)) return true;
+    if (spins == 0) t0 = globaltimer();
+    if (spin_give_up(spins, t0, ctrl, timeout_ns)) return false;
+  }
+}
+
 template <int CELL, int MODE, int DP>
 struct DiagTcCfg {
   static constexpr int R = CellInfo<CELL>::R;
@@ -463,8 +537,13 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     if (lane == 0) bulk_wait_all();   // the states are in global memory before the CTA retires
   } else if (warp < C::WE0) {
     // =========================== look-back ==================================
-    // warp 2 + j takes tiles j, j + NLB, j + 2 NLB, ... of this CTA
+    // warp 2 + j takes tiles j, j + NLB, j + 2 NLB, ... of this CTA.  Aggregates
+    // and states are published as self-validating words (value + launch tag);
+    // the flags only tell a reader where to look, so no fences are needed.
     if constexpr (kScan) {
+      unsigned long long* aggw = reinterpret_cast<unsigned long long*>(P.agg);    // [tile][DP] x {A, B}
+      unsigned long long* prefw = reinterpret_cast<unsigned long long*>(P.pref);  // [tile][DP]
+      const unsigned tag = lookback_tag(epoch);
       for (int it = warp - 2;; it += C::NLB) {
         const int slot = it % NSLOT;
         const unsigned ph = (unsigned)(it / NSLOT) & 1u;
@@ -486,31 +565,40 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
 #pragma unroll
           for (int q = 0; q < C::NQ; ++q) {
             const int j = lane + 32 * q;
-            if (j < DP) reinterpret_cast<float2*>(P.agg + k * P.agg_stride)[j] = ag[q];
+            if (j < DP) st_word2(aggw + (k * DP + j) * 2, tag_word(ag[q].x, tag), tag_word(ag[q].y, tag));
           }
-          // the warp barrier orders the other lanes' stores before lane 0's release,
-          // which is cumulative: a reader that acquires the flag sees all of them
           __syncwarp();
-          if (lane == 0) st_release(P.flags + k, make_flag(epoch, kFlagAgg));
+          if (lane == 0) st_relaxed(P.flags + k, make_flag(epoch, kFlagAgg));
         }
         // 2. the carry: nearest published state, then the aggregates in between
-        const int n_agg = lookback_find_prefix(P.flags, k, stride, chunk, epoch, ctrl, tmo);
+        int n_agg = lookback_find_prefix(P.flags, k, stride, chunk, epoch, ctrl, tmo, false);
         float carry[C::NQ];
 #pragma unroll
-        for (int q = 0; q < C::NQ; ++q) {
-          const int j = lane + 32 * q;
-          float v = 0.0f;
-          if (n_agg >= 0 && j < DP) {
-            if (chunk - 1 - n_agg >= 0) v = __ldcg(P.pref + (k - (size_t)(n_agg + 1) * stride) * P.pref_stride + j);
-            else v = (j < D) ? __ldg(A.s0 + (size_t)b * D + j) : 0.0f;
-#pragma unroll 4
-            for (int d = n_agg; d >= 1; --d) {
-              const float2 ab =
-                  __ldcg(reinterpret_cast<const float2*>(P.agg + (k - (size_t)d * stride) * P.agg_stride) + j);
-              v = fmaf(ab.x, v, ab.y);
+        for (int q = 0; q < C::NQ; ++q) carry[q] = 0.0f;
+        if (n_agg >= 0) {
+          if (chunk - 1 - n_agg >= 0) {
+            if (!ld_tagged_state<DP, C::NQ>(prefw + (k - (size_t)(n_agg + 1) * stride) * DP, tag, carry, ctrl, tmo))
+              n_agg = -1;
+          } else {
+#pragma unroll
+            for (int q = 0; q < C::NQ; ++q) {
+              const int j = lane + 32 * q;
+              carry[q] = (j < D) ? __ldg(A.s0 + (size_t)b * D + j) : 0.0f;
             }
           }
-          carry[q] = v;
+        }
+        for (int d0 = n_agg; d0 >= 1; d0 -= 4) {   // oldest aggregate first, four loads in flight
+          float fa[4][C::NQ], fb[4][C::NQ];
+          if (!ld_tagged_aggs<DP, C::NQ>(aggw, k, stride, d0, tag, fa, fb, ctrl, tmo)) {
+            n_agg = -1;
+            break;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (d0 - u >= 1) {
+#pragma unroll
+              for (int q = 0; q < C::NQ; ++q) carry[q] = fmaf(fa[u][q], carry[q], fb[u][q]);
+            }
         }
         if (n_agg < 0) s_abort = 1;
         // 3. hand the carry to the epilogue (its slot is free once tile it - NSLOT was formed)
@@ -527,10 +615,10 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
 #pragma unroll
           for (int q = 0; q < C::NQ; ++q) {
             const int j = lane + 32 * q;
-            if (j < DP) P.pref[k * P.pref_stride + j] = fmaf(ag[q].x, carry[q], ag[q].y);
+            if (j < DP) st_word(prefw + k * DP + j, tag_word(fmaf(ag[q].x, carry[q], ag[q].y), tag));
           }
           __syncwarp();
-          if (lane == 0) st_release(P.flags + k, make_flag(epoch, kFlagPrefix));
+          if (lane == 0) st_relaxed(P.flags + k, make_flag(epoch, kFlagPrefix));
         }
       }
     }
