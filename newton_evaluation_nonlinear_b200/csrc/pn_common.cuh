@@ -105,18 +105,18 @@ __device__ __forceinline__ unsigned long long tag_word(float v, unsigned tag) {
 __device__ __forceinline__ float word_value(unsigned long long w) { return __uint_as_float((unsigned)w); }
 __device__ __forceinline__ bool word_tagged(unsigned long long w, unsigned tag) { return (unsigned)(w >> 32) == tag; }
 __device__ __forceinline__ void st_word(unsigned long long* p, unsigned long long w) {
-  asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
 __device__ __forceinline__ void st_word2(unsigned long long* p, unsigned long long w0, unsigned long long w1) {
-  asm volatile("st.volatile.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(w0), "l"(w1) : "memory");
+  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(w0), "l"(w1) : "memory");
 }
 __device__ __forceinline__ unsigned long long ld_word(const unsigned long long* p) {
   unsigned long long w;
-  asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
   return w;
 }
 __device__ __forceinline__ void ld_word2(const unsigned long long* p, unsigned long long& w0, unsigned long long& w1) {
-  asm volatile("ld.volatile.global.v2.u64 {%0, %1}, [%2];" : "=l"(w0), "=l"(w1) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(w0), "=l"(w1) : "l"(p) : "memory");
 }
 __device__ __forceinline__ unsigned long long globaltimer() {
   unsigned long long t;
@@ -161,6 +161,51 @@ __device__ __forceinline__ int lookback_find_prefix(const unsigned* flags, size_
         if (acquire) fence_acquire_gpu();
         return n_agg + nearest;
       }
+      n_agg += 32;
+      base -= 32;
+      continue;
+    }
+    ++spins;
+    if ((spins & 15u) == 0u) {
+      int give_up = 0;
+      if (lane == 0) {
+        if (ld_volatile(&ctrl->error)) give_up = 1;
+        else if ((long long)(globaltimer() - t0) > timeout_ns) {
+          if (atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT) == 0) ctrl->timeout_ticket = (int)k;
+          give_up = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, give_up, 0)) return -1;
+    }
+    if (spins > 64u) __nanosleep(32);
+  }
+}
+
+// Look-back for self-validating data (called by all 32 lanes of one warp):
+// the distance to the nearest predecessor whose flag says it published its
+// state, as the number n of tiles in between (chunk -1 = s0 counts as
+// published).  Unlike lookback_find_prefix it does not wait for the flags of
+// the n tiles in between: the caller waits on their tagged aggregate words
+// directly, which saves a round trip.  The window moves on only when all of
+// its 32 tiles have at least flagged an aggregate.  Returns -1 when it gave up.
+__device__ __forceinline__ int lookback_nearest_state(const unsigned* flags, size_t k, size_t stride, int chunk,
+                                                      unsigned epoch, Ctrl* ctrl, long long timeout_ns) {
+  const int lane = threadIdx.x & 31;
+  int n_agg = 0;
+  int base = chunk - 1;
+  const unsigned long long t0 = globaltimer();
+  unsigned spins = 0;
+  while (true) {
+    const int p = base - lane;
+    bool valid = true, pfx = true;
+    if (p >= 0) {
+      const unsigned f = ld_relaxed(flags + (k - (size_t)(chunk - p) * stride));
+      valid = ((f >> 2) == epoch) && (f & 3u);
+      pfx = valid && ((f & 3u) == kFlagPrefix);
+    }
+    const unsigned pm = __ballot_sync(0xffffffffu, pfx);
+    if (pm) return n_agg + (__ffs(pm) - 1);
+    if (__ballot_sync(0xffffffffu, valid) == 0xffffffffu) {
       n_agg += 32;
       base -= 32;
       continue;

@@ -560,8 +560,9 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
           const int j = lane + 32 * q;
           ag[q] = (j < DP) ? *reinterpret_cast<const float2*>(sAgg + (slot * DP + j) * 2) : make_float2(1.0f, 0.0f);
         }
-        // 1. the tile aggregate, for successors that reach this tile before its state
-        if (chunk > 0 && !stall) {
+        // 1. the tile aggregate, for successors that reach this tile before its state (the
+        //    first chunk too: a successor may start from s0 before that chunk's state is out)
+        if (!stall) {
 #pragma unroll
           for (int q = 0; q < C::NQ; ++q) {
             const int j = lane + 32 * q;
@@ -571,7 +572,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
           if (lane == 0) st_relaxed(P.flags + k, make_flag(epoch, kFlagAgg));
         }
         // 2. the carry: nearest published state, then the aggregates in between
-        int n_agg = lookback_find_prefix(P.flags, k, stride, chunk, epoch, ctrl, tmo, false);
+        int n_agg = lookback_nearest_state(P.flags, k, stride, chunk, epoch, ctrl, tmo);
         float carry[C::NQ];
 #pragma unroll
         for (int q = 0; q < C::NQ; ++q) carry[q] = 0.0f;

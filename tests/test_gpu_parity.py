@@ -139,21 +139,29 @@ def test_picard_divergence_is_reported():
     solver.close()
 
 
+# The decoupled look-back combines a tile's carry from whichever predecessor state is published
+# first, so two runs may associate the same fp32 products differently: results agree to rounding,
+# not bit for bit.
+RUN_TO_RUN = 1e-6
+
+
 @pytest.mark.parametrize("mode", [pi.MODE_QUASI, pi.MODE_NEWTON])
 def test_host_loop_matches_device_loop(mode):
     prob = pi.random_problem(5, pi.CELL_TANH_RNN, 16, 16, T=700, B=3, rho=0.7, tol=1e-6)
     a = _run(prob, mode, device_loop=1)
     b = _run(prob, mode, device_loop=0)
     assert a[1] == b[1]
-    np.testing.assert_array_equal(a[0], b[0])
-    np.testing.assert_array_equal(a[4], b[4])
+    scale = max(1.0, float(np.abs(a[0]).max()))
+    np.testing.assert_allclose(a[0], b[0], rtol=0, atol=RUN_TO_RUN * scale)
+    np.testing.assert_allclose(a[4], b[4], rtol=1e-3, atol=RUN_TO_RUN * scale)
 
 
-def test_repeatable_bitwise():
+def test_repeatable():
     prob = pi.random_problem(6, pi.CELL_GRU, 32, 32, T=1000, B=4, rho=0.9, tol=1e-6)
     a = _run(prob, pi.MODE_QUASI)
     b = _run(prob, pi.MODE_QUASI)
-    np.testing.assert_array_equal(a[0], b[0])
+    scale = max(1.0, float(np.abs(a[0]).max()))
+    np.testing.assert_allclose(a[0], b[0], rtol=0, atol=RUN_TO_RUN * scale)
     assert a[1] == b[1]
 
 
