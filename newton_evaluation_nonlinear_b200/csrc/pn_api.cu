@@ -53,6 +53,7 @@ struct pn_ctx {
   float* wt_diag = nullptr;    // [ngroups][DP][R*G] transposed recurrent weights
   float* wt_dense = nullptr;   // [DP][R*DP] transposed + [R][DP][DP] row-major
   float* wt_tc = nullptr;      // [W ; W_lo] rows of W_q, TF32-rounded, K-major core-matrix layout
+  float* wt_tct = nullptr;     // zero-banded [Z; W_hi; Z; W_lo; Z] (one-gate cells), same layout
   float* wdiag = nullptr;      // [R][DP] diagonal entries W_q[c][c]
   float* bhn = nullptr;        // [DP]
   float* proj_w = nullptr;     // U [D][d_in] or W_ih [3D][d_in]
@@ -144,8 +145,8 @@ void free_all(pn_ctx* h) {
     h->exec[m] = nullptr;
     h->graph[m] = nullptr;
   }
-  float** fbufs[] = {&h->wt_diag, &h->wt_dense, &h->wt_tc, &h->wdiag, &h->bhn, &h->proj_w, &h->proj_b,
-                     &h->xin,     &h->buf1,     &h->agg,   &h->pref,  &h->hist, &h->hx,     &h->hs0, &h->hst};
+  float** fbufs[] = {&h->wt_diag, &h->wt_dense, &h->wt_tc, &h->wt_tct, &h->wdiag, &h->bhn, &h->proj_w, &h->proj_b,
+                     &h->xin,     &h->buf1,     &h->agg,   &h->pref,   &h->hist,  &h->hx,  &h->hs0,    &h->hst};
   for (float** p : fbufs) {
     if (*p) cudaFree(*p);
     *p = nullptr;
@@ -177,7 +178,8 @@ IterParams make_params(const pn_ctx* h, int mode) {
   IterParams P{};
   const bool dense = (mode == PN_NEWTON);
   const int kind = h->fam.k[mode].kind;
-  P.wt = dense ? h->wt_dense : (kind == kKindDiagTc ? h->wt_tc : h->wt_diag);
+  P.wt = dense ? h->wt_dense
+               : (kind == kKindDiagTc ? h->wt_tc : (kind == kKindDiagTct ? h->wt_tct : h->wt_diag));
   P.wdiag = h->wdiag;
   P.bhn = h->bhn;
   P.xin = h->xin;
@@ -249,16 +251,19 @@ bool encode_seq(CUtensorMap* m, const void* base, int cols, int T, int B, int bo
 // for the Euler cell):
 //   [0], [1]  s^(i) loads from buffer 0 / 1: 32-float column halves of L+1
 //             steps, 128-byte swizzled (the tensor cores' operand layout);
-//   [2]       step-input loads, rows padded by 4 floats through the box width;
-//   [3], [4]  state stores into buffer 0 / 1, from rows padded by 4 floats.
+//   [2]       step-input loads: rows padded by 4 floats through the box width
+//             for the row-major kernel, plain rows for the channel-major one;
+//   [3], [4]  state stores into buffer 0 / 1, from rows padded by 4 floats
+//             (row-major kernel).
 bool encode_tc_maps(const pn_ctx* h, int mode, CUtensorMap* out) {
   const int L = h->fam.k[mode].L;
+  const bool padded_x = (h->fam.k[mode].kind == kKindDiagTc);
   const int R = cell_R(h->cell);
   const int D = h->D, T = h->T, B = h->B, DP = h->DP;
   const void* xs = (h->cell == PN_CELL_EULER_TANH) ? (const void*)h->args_h->x : (const void*)h->xin;
   return encode_seq(&out[0], h->args_h->states, D, T, B, 32, L + 1, true) &&
          encode_seq(&out[1], h->buf1, D, T, B, 32, L + 1, true) &&
-         encode_seq(&out[2], xs, R * D, T, B, R * DP + 4, L, false) &&
+         encode_seq(&out[2], xs, R * D, T, B, padded_x ? R * DP + 4 : R * DP, L, false) &&
          encode_seq(&out[3], h->args_h->states, D, T, B, DP + 4, L, false) &&
          encode_seq(&out[4], h->buf1, D, T, B, DP + 4, L, false);
 }
@@ -437,7 +442,7 @@ pn_status validate_mode(pn_ctx* h, int mode, int max_iters, float tol) {
 pn_status prepare_lookback(pn_ctx* h, int mode) {
   const int kind = h->fam.k[mode].kind;
   const bool wrap = h->ctrl_h->epoch > (1u << 29);
-  const bool format = (kind != h->last_kind) && (kind == kKindDiagTc || h->last_kind == kKindDiagTc);
+  const bool format = (kind != h->last_kind) && (tagged_lookback(kind) || tagged_lookback(h->last_kind));
   if (wrap) {
     PN_CUDA(h, cudaMemsetAsync(h->flags, 0, h->nflags * sizeof(unsigned), h->stream));
     PN_CUDA(h, cudaMemsetAsync(&h->ctrl->epoch, 0, sizeof(unsigned), h->stream));
@@ -455,7 +460,7 @@ pn_status prepare_lookback(pn_ctx* h, int mode) {
 // The copy is ordered before the launches on the same stream; the pinned
 // mirror is not touched again before the call's final synchronisation.
 pn_status upload_tc_maps(pn_ctx* h, int mode) {
-  if (h->fam.k[mode].kind != kKindDiagTc) return PN_OK;
+  if (!tagged_lookback(h->fam.k[mode].kind)) return PN_OK;
   if (!encode_tc_maps(h, mode, h->tmaps_h))
     return fail(h, PN_ERR_CUDA, "encoding the TMA tensor maps failed (D=%d, T=%d, B=%d)", h->D, h->T, h->B);
   PN_CUDA(h, cudaMemcpyAsync(h->tmaps, h->tmaps_h, kTcMaps * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
@@ -535,7 +540,7 @@ pn_status select_kernels(pn_ctx* h) {
     const size_t G = (size_t)ki.G;
     const size_t nt = (size_t)h->fam.ntiles[m];
     // the tensor-core kernels publish 64-bit tagged words: twice the floats
-    const size_t wf = (ki.kind == kKindDiagTc) ? 2 : 1;
+    const size_t wf = tagged_lookback(ki.kind) ? 2 : 1;
     const size_t aggf = nt * ((m == PN_NEWTON) ? G * (G + 1) : 2 * G) * wf;
     h->agg_floats = std::max(h->agg_floats, aggf);
     h->pref_floats = std::max(h->pref_floats, nt * G * wf);
@@ -669,6 +674,21 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
           wtc[off] = hi;
           wtc[(size_t)NN * DP + off] = lo;
         }
+    // channel-major tensor-core operand (one-gate cells, D == DP): rows of the zero-banded
+    // buffer [Z(128-D); W_hi; Z(128-D); W_lo; Z(128-D)], K = DP, K-major core-matrix layout
+    std::vector<float> wtct;
+    if (h->tc_capable && cell != PN_CELL_GRU) {
+      const int rows = 384 - DP;
+      wtct.assign((size_t)rows * DP, 0.0f);
+      for (int j = 0; j < D; ++j)
+        for (int k = 0; k < D; ++k) {
+          const float w = w_block(h, params, 0, j, k);
+          const float hi = tf32_round(w);
+          const float lo = tf32_round(w - hi);
+          wtct[kmajor_offset((128 - DP) + j, k, DP) / 4] = hi;
+          wtct[kmajor_offset((256 - DP) + j, k, DP) / 4] = lo;
+        }
+    }
     std::vector<float> wdg((size_t)R * DP, 0.0f);
     for (int q = 0; q < R; ++q)
       for (int j = 0; j < D; ++j) wdg[(size_t)q * DP + j] = w_block(h, params, q, j, j);
@@ -695,6 +715,13 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
     PN_TRY(dalloc(h, &h->bhn, bhn.size()));
     PN_TRY(dalloc(h, &h->wt_tc, wtc.size()));
     PN_TRY(dalloc(h, &h->wdiag, wdg.size()));
+    if (!wtct.empty()) {
+      PN_TRY(dalloc(h, &h->wt_tct, wtct.size()));
+      if (cudaMemcpy(h->wt_tct, wtct.data(), wtct.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess) {
+        st = fail(h, PN_ERR_CUDA, "weight upload failed");
+        goto bad;
+      }
+    }
     if (cudaMemcpy(h->wt_tc, wtc.data(), wtc.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(h->wdiag, wdg.data(), wdg.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(h->wt_diag, wt.data(), wt.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||

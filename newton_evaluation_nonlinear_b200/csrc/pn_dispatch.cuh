@@ -9,11 +9,16 @@
 #include "pn_iter_dense.cuh"
 #include "pn_iter_diag.cuh"
 #include "pn_iter_diag_tc.cuh"
+#include "pn_iter_diag_tct.cuh"
 #include "pn_iter_diag_tma.cuh"
 
 namespace pn {
 
-enum KKind { kKindDiag = 0, kKindDiagTc = 1, kKindDense = 2 };
+// Which weight packing and look-back format a kernel uses.
+enum KKind { kKindDiag = 0, kKindDiagTc = 1, kKindDense = 2, kKindDiagTct = 3 };
+
+// Kernels whose look-back aggregates and states are tagged 64-bit words.
+inline bool tagged_lookback(int kind) { return kind == kKindDiagTc || kind == kKindDiagTct; }
 
 struct KInfo {
   const void* fn;   // __global__ function
@@ -85,6 +90,13 @@ inline KInfo diag_tc_kinfo() {
   return KInfo{(const void*)&diag_tc_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTc};
 }
 
+// Channel-major tensor-core variant for the one-gate cells: D == DP in {32, 64}.
+template <int CELL, int MODE, int DP>
+inline KInfo diag_tct_kinfo() {
+  using C = DiagTctCfg<CELL, MODE, DP>;
+  return KInfo{(const void*)&diag_tct_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTct};
+}
+
 template <int CELL, int DP, int L>
 inline KInfo dense_kinfo() {
   using C = DenseCfg<CELL, DP, L>;
@@ -109,17 +121,25 @@ template <int CELL>
 inline KInfo lookup_cell(int mode, int DP, bool tma, bool tc) {
   KInfo none{nullptr, 0, 0, 0, 0, 0};
   if (tc && mode != PN_NEWTON) {
-    constexpr bool gru = (CELL == PN_CELL_GRU);
-    if (DP == 32) {
-      if (mode == PN_JACOBI) return diag_tc_kinfo<CELL, PN_JACOBI, 32>();
-      if (mode == PN_PICARD) return diag_tc_kinfo<CELL, PN_PICARD, 32>();
-      return diag_tc_kinfo<CELL, PN_QUASI, 32>();
-    }
-    if constexpr (!gru) {
+    if constexpr (CELL == PN_CELL_GRU) {
+      // three gates per channel: the row-major kernel (D = 32)
+      if (DP == 32) {
+        if (mode == PN_JACOBI) return diag_tc_kinfo<CELL, PN_JACOBI, 32>();
+        if (mode == PN_PICARD) return diag_tc_kinfo<CELL, PN_PICARD, 32>();
+        return diag_tc_kinfo<CELL, PN_QUASI, 32>();
+      }
+    } else {
+      // quasi-Newton: the channel-major kernel (sequential in-register scan); Jacobi and
+      // Picard: the row-major one (half the tensor-core operand traffic, cheap scan)
+      if (DP == 32) {
+        if (mode == PN_JACOBI) return diag_tc_kinfo<CELL, PN_JACOBI, 32>();
+        if (mode == PN_PICARD) return diag_tc_kinfo<CELL, PN_PICARD, 32>();
+        return diag_tct_kinfo<CELL, PN_QUASI, 32>();
+      }
       if (DP == 64) {
         if (mode == PN_JACOBI) return diag_tc_kinfo<CELL, PN_JACOBI, 64>();
         if (mode == PN_PICARD) return diag_tc_kinfo<CELL, PN_PICARD, 64>();
-        return diag_tc_kinfo<CELL, PN_QUASI, 64>();
+        return diag_tct_kinfo<CELL, PN_QUASI, 64>();
       }
     }
   }

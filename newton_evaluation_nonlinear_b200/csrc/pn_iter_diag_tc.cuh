@@ -397,6 +397,28 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   }
   const unsigned epoch = *(volatile unsigned*)&ctrl->epoch;
   const int iter = *(volatile int*)&ctrl->iter;
+  if (tid == 0) {
+    // The first tile of every CTA has a static ticket (blockIdx.x < tiles: the grid is never
+    // larger) and is fetched right away, overlapping the weight load and TMEM set-up below.
+    const CUtensorMap* tm_s = P.tmaps + ((iter & 1) ? 1 : 0);
+    const CUtensorMap* tm_x = P.tmaps + 2;
+    tmap_acquire(tm_s);
+    tmap_acquire(tm_x);
+    const int kg = (int)blockIdx.x;
+    if (kg < P.tiles_per_group) {
+      const int b = kg % B;
+      const int t0 = (kg / B) * L;
+      s_tk[0] = kg;
+      mbar_arrive_expect_tx(&bar_sfull[0], (unsigned)(NKH * C::SH_LOAD));
+#pragma unroll
+      for (int h = 0; h < NKH; ++h) tma_load_3d(sS + h * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[0]);
+      mbar_arrive_expect_tx(&bar_xfull, (unsigned)C::X_BYTES);
+      tma_load_3d(sX, tm_x, 0, t0, b, &bar_xfull);
+    } else {
+      s_tk[0] = -1;
+      mbar_arrive(&bar_sfull[0]);
+    }
+  }
 
   // weights: W_hi and W_lo in the K-major core-matrix layout (pre-packed), diagonals, b_hn
   {
@@ -424,17 +446,15 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     // =========================== producer ===================================
     const CUtensorMap* tm_s = P.tmaps + ((iter & 1) ? 1 : 0);   // s^(i)
     const CUtensorMap* tm_x = P.tmaps + 2;                      // step inputs
-    if (lane == 0) {
-      tmap_acquire(tm_s);
-      tmap_acquire(tm_x);
-    }
-    int it = 0;
-    int x_issued = 0;
-    for (;; ++it) {
+    // tile 0 was issued before the block-wide sync (static ticket blockIdx.x)
+    const bool none = (int)blockIdx.x >= P.tiles_per_group;
+    int it = 1;
+    int x_issued = none ? 0 : 1;
+    for (; !none; ++it) {
       const int st = it & 1;
       if (it >= 2 && !mbar_wait_flag(&bar_sempty[st], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
       int kg = 0;
-      if (lane == 0) kg = (int)atomicAdd(&ctrl->ticket[0], 1u);
+      if (lane == 0) kg = (int)(gridDim.x + atomicAdd(&ctrl->ticket[0], 1u));
       kg = __shfl_sync(0xffffffffu, kg, 0);
       if (kg >= P.tiles_per_group) {
         if (lane == 0) {
@@ -475,6 +495,9 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     // ======================= MMA and store issuer ============================
     constexpr uint32_t idesc = umma_idesc_tf32(L, N);
     constexpr uint32_t SBO_B = (K / 4) * 128;
+    const uint64_t a_base0 = umma_smem_desc(smem_addr(sS), 16, 1024, 2);
+    const uint64_t a_lo = umma_smem_desc(smem_addr(sLo), 16, 1024, 2);
+    const uint64_t b_base = umma_smem_desc(smem_addr(sBH), 128, SBO_B, 0);   // W_lo follows W_hi
     const CUtensorMap* tm_o = P.tmaps + ((iter & 1) ? 3 : 4);   // s^(i+1) goes to the other buffer
     if (lane == 0) tmap_acquire(tm_o);
     int nstored = 0;   // output tiles taken so far
@@ -504,19 +527,19 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
       if (it >= 2 && !mbar_wait_flag(&bar_tempty[buf], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
       tc_fence_after();
       if (lane == 0) {
+        // descriptors differ only in the start-address field: base + compile-time offsets
         const uint32_t d = tmem + (uint32_t)(buf * C::TCOLS);
-        const uint32_t s_hi = smem_addr(sS + (it & 1) * NKH * C::SH_BYTES), s_lo = smem_addr(sLo);
-        const uint32_t bh = smem_addr(sBH), bl = smem_addr(sBL);
-#pragma unroll 1
+        const uint64_t a_hi = a_base0 + (uint64_t)(((it & 1) * NKH * C::SH_BYTES) >> 4);
+#pragma unroll
         for (int pass = 0; pass < 3; ++pass) {
           // pass 0: S_hi W_hi, pass 1: S_hi W_lo, pass 2: S_lo W_hi
 #pragma unroll
           for (int kb = 0; kb < K / 8; ++kb) {
             const int h = kb >> 2;   // column half; 4 K-steps of 32 bytes per 128-byte swizzled row
-            const uint32_t a = (pass == 2) ? (s_lo + h * C::LO_BYTES) : (s_hi + h * C::SH_BYTES);
-            const uint32_t bb = (pass == 1) ? bl : bh;
-            umma_tf32(d, umma_smem_desc(a + (kb & 3) * 32, 16, 1024, 2), umma_smem_desc(bb + kb * 256, 128, SBO_B, 0),
-                      idesc, (pass > 0 || kb > 0) ? 1u : 0u);
+            const uint64_t ad = (pass == 2) ? a_lo + (uint64_t)((h * C::LO_BYTES + (kb & 3) * 32) >> 4)
+                                            : a_hi + (uint64_t)((h * C::SH_BYTES + (kb & 3) * 32) >> 4);
+            const uint64_t bd = b_base + (uint64_t)(((pass == 1 ? C::B_BYTES : 0) + kb * 256) >> 4);
+            umma_tf32(d, ad, bd, idesc, (pass > 0 || kb > 0) ? 1u : 0u);
           }
         }
         umma_commit(&bar_mma[buf]);

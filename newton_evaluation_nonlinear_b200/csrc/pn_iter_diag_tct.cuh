@@ -1,0 +1,609 @@
+// pn_iter_diag_tct.cuh -- tensor-core iteration kernel with a channel-major
+// accumulator, for the one-gate cells (tanh RNN, Euler drift) at D = 32, 64,
+// in the Jacobi, Picard and diagonal quasi-Newton modes.
+//
+// Same iteration as pn_iter_diag_tc.cuh (the page's unified update, "Parallel
+// Newton methods..." page §1.2, with a diagonal A~_t, §2.2.1 / §2.2.3, solved
+// by the chunked scan of §2.1), with the roles of the two MMA operands
+// swapped: Z = W S^T, so a TMEM lane holds one channel and its columns hold
+// consecutive steps.  The 128 lanes hold 128 / D step segments side by side:
+// lane g D + c is channel c of steps t0 + g RS .. t0 + (g+1) RS - 1
+// (RS = D L / 128).  Segment g's MMA reads its steps of S as the B operand and
+// a window of a zero-banded copy of W as the A operand, whose nonzero rows are
+// exactly lanes g D .. g D + D - 1; the accumulations of all segments land in
+// one 128-lane accumulator.  Products are 3xTF32 as in the row-major kernel:
+// S_hi W_hi + S_hi W_lo + S_lo W_hi, with S_hi the tensor core's truncation.
+//
+// Each epilogue thread owns one lane (channel c of one segment) and 16
+// consecutive steps: it evaluates the cell, the Jacobian diagonal and the
+// residual, and scans those steps sequentially in registers -- no shuffles.
+// The 8 sixteen-step pieces of a channel are combined through shared memory;
+// the piece prefix (PA, PB) stays in registers, the in-piece prefixes are
+// parked in TMEM, and the states are formed two tiles later from the carry of
+// the look-back warps, stored straight from registers (a warp writes 32
+// consecutive channels of one step: 128 contiguous bytes).
+//
+// Warp roles (one CTA per SM): 0 producer (tickets, TMA loads); 1 MMA issuer;
+// 2-3 look-back (scan modes, alternate tiles); the rest epilogue (4 TMEM lane
+// quarters x RS / 16 step groups).  The epilogue forms the next tile's S_lo
+// right after the current tile's cell phase, so the tensor cores compute the
+// next tile's products while the epilogue finishes the current one.
+#pragma once
+
+#include "pn_iter_diag_tc.cuh"
+
+namespace pn {
+
+template <int CELL, int MODE, int DP>
+struct DiagTctCfg {
+  static_assert(CELL != PN_CELL_GRU, "one-gate cells only");
+  static_assert(DP == 32 || DP == 64, "D = 32 or 64");
+  static constexpr bool kScan = (MODE != PN_JACOBI);
+  static constexpr int L = 128;                  // steps per tile
+  static constexpr int K = DP;                   // MMA K (input channels)
+  static constexpr int NSEG = 128 / DP;          // step segments side by side on the TMEM lanes
+  static constexpr int RS = L / NSEG;            // steps per segment = MMA N
+  static constexpr int NRG = RS / 16;            // 16-step groups per segment
+  static constexpr int NPC = NSEG * NRG;         // pieces per channel (L / 16)
+  static constexpr int NKH = DP / 32;            // 32-float column halves of S
+  static constexpr int SCOLS = (MODE == PN_QUASI ? 2 : 1) * RS;   // stash columns per tile: [A |] B
+  static constexpr int NSLOT = 3;                // tiles between their scan and their write-out, + 1
+  static constexpr int DEFER = NSLOT - 1;
+  static constexpr int NLB = kScan ? 2 : 0;      // look-back warps, alternating tiles
+  static constexpr int STASH0 = 2 * RS;          // accumulators: 2 x RS columns
+  static constexpr int USED_COLS = STASH0 + (kScan ? NSLOT * SCOLS : 0);
+  static constexpr int ALLOC_COLS =
+      USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128 : USED_COLS <= 256 ? 256 : 512;
+  static constexpr int NEW = 4 * NRG;            // epilogue warps
+  static constexpr int NTE = 32 * NEW;
+  static constexpr int WE0 = 2 + NLB;            // first epilogue warp
+  static constexpr int NT = 32 * (WE0 + NEW);
+  static constexpr int NQ = DP / 32;             // channels per look-back lane; warps holding the last piece
+  static constexpr int WROWS = 384 - DP;         // banded W: Z(128-D) W_hi Z(128-D) W_lo Z(128-D)
+  static constexpr int align(int v, int a) { return (v + a - 1) / a * a; }
+  static constexpr int SH_LOAD = (L + 1) * 128;
+  static constexpr int SH_BYTES = align(SH_LOAD, 1024);
+  static constexpr int LO_BYTES = L * 128;
+  static constexpr int X_BYTES = L * DP * 4;
+  static constexpr int W_BYTES = WROWS * DP * 4;
+  static constexpr uint32_t SBO_W = (K / 4) * 128;
+  static constexpr int OFF_S = 0;                                 // [2 stages][NKH][SH_BYTES]
+  static constexpr int OFF_LO = OFF_S + 2 * NKH * SH_BYTES;       // [NKH][LO_BYTES]
+  static constexpr int OFF_X = OFF_LO + NKH * LO_BYTES;           // [L][DP]
+  static constexpr int OFF_W = align(OFF_X + X_BYTES, 128);
+  static constexpr int OFF_WD = OFF_W + W_BYTES;                  // DP floats
+  static constexpr int OFF_TOT = OFF_WD + DP * 4;                 // [2][NPC][DP] float2
+  static constexpr int OFF_AGG = OFF_TOT + 2 * NPC * DP * 8;      // [NSLOT][DP] float2
+  static constexpr int OFF_CARRY = OFF_AGG + NSLOT * DP * 8;      // [NSLOT][DP]
+  static constexpr int OFF_RED = OFF_CARRY + NSLOT * DP * 4;      // NT/32 floats
+  static constexpr int SMEM_USED = OFF_RED + (NT / 32) * 4;
+  static constexpr int SMEM_BYTES = SMEM_USED + 1024;             // + slack to align the base to 1024 bytes
+  // first row of segment g's window of the banded W (hi: W_hi at window rows g D .. g D + D - 1)
+  static constexpr int win_hi(int g) { return (128 - DP) - g * DP; }
+  static constexpr int win_lo(int g) { return (256 - DP) - g * DP; }
+  static_assert(USED_COLS <= 512, "TMEM columns");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+template <int CELL, int MODE, int DP>
+__global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_kernel(const IterParams P) {
+  using C = DiagTctCfg<CELL, MODE, DP>;
+  constexpr int L = C::L;
+  constexpr int K = C::K;
+  constexpr int NKH = C::NKH;
+  constexpr int RS = C::RS;
+  constexpr int NTE = C::NTE;
+  constexpr int NSLOT = C::NSLOT;
+  constexpr bool kScan = C::kScan;
+  constexpr bool kHasA = (MODE == PN_QUASI);
+
+  extern __shared__ __align__(1024) unsigned char smem_tct[];
+  unsigned char* smem_raw = smem_tct + ((1024u - (smem_addr(smem_tct) & 1023u)) & 1023u);
+  unsigned char* sS = smem_raw + C::OFF_S;       // stage st, half h at sS + (st * NKH + h) * SH_BYTES
+  unsigned char* sLo = smem_raw + C::OFF_LO;     // half h at sLo + h * LO_BYTES
+  const float* sX = reinterpret_cast<const float*>(smem_raw + C::OFF_X);
+  unsigned char* sW = smem_raw + C::OFF_W;
+  float* sWd = reinterpret_cast<float*>(smem_raw + C::OFF_WD);
+  float* sTot = reinterpret_cast<float*>(smem_raw + C::OFF_TOT);
+  float* sAgg = reinterpret_cast<float*>(smem_raw + C::OFF_AGG);
+  float* sCarry = reinterpret_cast<float*>(smem_raw + C::OFF_CARRY);
+  float* sRed = reinterpret_cast<float*>(smem_raw + C::OFF_RED);
+
+  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull, bar_xempty, bar_afull, bar_mma[2],
+      bar_tempty[2], bar_lb[NSLOT], bar_cfull[NSLOT], bar_cempty[NSLOT];
+  __shared__ int s_tk[2];        // ticket staged in s stage 0/1 (-1: no more tiles)
+  __shared__ int s_atk[2];       // ticket of tile i's operands, by the parity of i (-1: stop)
+  __shared__ int s_lbtk[NSLOT];  // ticket handed to the look-back per slot (-1: stop)
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  Ctrl* ctrl = P.ctrl;
+  const Args A = *P.args;
+  const int D = P.D, T = P.T, B = P.B;
+  const size_t stride = (size_t)B;   // consecutive chunks of a sequence are B tickets apart
+  const long long tmo = A.timeout_ns;
+
+  if (tid == 0) {
+    atomicMin(&ctrl->t_start, globaltimer());
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_sfull[s], 1u);
+      mbar_init(&bar_sempty[s], (unsigned)C::NEW);
+      mbar_init(&bar_mma[s], 1u);
+      mbar_init(&bar_tempty[s], (unsigned)C::NEW);
+    }
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(&bar_lb[s], (unsigned)C::NQ);
+      mbar_init(&bar_cfull[s], 1u);
+      mbar_init(&bar_cempty[s], (unsigned)C::NEW);
+    }
+    mbar_init(&bar_xfull, 1u);
+    mbar_init(&bar_xempty, (unsigned)C::NEW);
+    mbar_init(&bar_afull, (unsigned)C::NEW);
+    mbar_init_fence();
+    s_abort = 0;
+  }
+  const unsigned epoch = *(volatile unsigned*)&ctrl->epoch;
+  const int iter = *(volatile int*)&ctrl->iter;
+  if (tid == 0) {
+    // The first tile of every CTA has a static ticket (blockIdx.x < tiles: the grid is never
+    // larger) and is fetched right away, overlapping the weight load and TMEM set-up below.
+    const CUtensorMap* tm_s = P.tmaps + ((iter & 1) ? 1 : 0);
+    const CUtensorMap* tm_x = P.tmaps + 2;
+    tmap_acquire(tm_s);
+    tmap_acquire(tm_x);
+    const int kg = (int)blockIdx.x;
+    if (kg < P.tiles_per_group) {
+      const int b = kg % B;
+      const int t0 = (kg / B) * L;
+      s_tk[0] = kg;
+      mbar_arrive_expect_tx(&bar_sfull[0], (unsigned)(NKH * C::SH_LOAD));
+#pragma unroll
+      for (int h = 0; h < NKH; ++h) tma_load_3d(sS + h * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[0]);
+      mbar_arrive_expect_tx(&bar_xfull, (unsigned)C::X_BYTES);
+      tma_load_3d(smem_raw + C::OFF_X, tm_x, 0, t0, b, &bar_xfull);
+    } else {
+      s_tk[0] = -1;
+      mbar_arrive(&bar_sfull[0]);
+    }
+  }
+  float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;
+
+  // banded W (hi and lo in the K-major core-matrix layout): the zero bands are written here,
+  // only the W_hi and W_lo row blocks (pre-packed by the host at their band offsets) are loaded
+  {
+    const float4* w4 = reinterpret_cast<const float4*>(P.wt);
+    float4* d4 = reinterpret_cast<float4*>(sW);
+    constexpr int ROW16 = DP / 4;                 // float4s per row of the K-major layout (on average)
+    constexpr int HI0 = (128 - DP) * ROW16, HI1 = 128 * ROW16;            // W_hi rows, in float4 units
+    constexpr int LO0 = (256 - DP) * ROW16, LO1 = 256 * ROW16;            // W_lo rows
+    for (int e = tid; e < C::W_BYTES / 16; e += C::NT) {
+      const bool wrow = (e >= HI0 && e < HI1) || (e >= LO0 && e < LO1);
+      d4[e] = wrow ? __ldg(w4 + e) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+    for (int e = tid; e < DP; e += C::NT) sWd[e] = __ldg(P.wdiag + e);
+    fence_async_smem();   // the tensor cores read sW through the async proxy
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
+                 "r"((uint32_t)C::ALLOC_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  unsigned rbits = 0u;
+
+  if (warp == 0) {
+    // =========================== producer ===================================
+    const CUtensorMap* tm_s = P.tmaps + ((iter & 1) ? 1 : 0);   // s^(i)
+    const CUtensorMap* tm_x = P.tmaps + 2;                      // step inputs
+    // tile 0 was issued before the block-wide sync (static ticket blockIdx.x)
+    const bool none = (int)blockIdx.x >= P.tiles_per_group;
+    int it = 1;
+    int x_issued = none ? 0 : 1;
+    for (; !none; ++it) {
+      const int st = it & 1;
+      if (it >= 2 && !mbar_wait_flag(&bar_sempty[st], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
+      int kg = 0;
+      if (lane == 0) kg = (int)(gridDim.x + atomicAdd(&ctrl->ticket[0], 1u));
+      kg = __shfl_sync(0xffffffffu, kg, 0);
+      if (kg >= P.tiles_per_group) {
+        if (lane == 0) {
+          s_tk[st] = -1;
+          mbar_arrive(&bar_sfull[st]);
+        }
+        ++it;
+        break;
+      }
+      const int b = kg % B;
+      const int t0 = (kg / B) * L;
+      if (lane == 0) {
+        // steps t0-1 .. t0+L-1 (step -1 reads as zero and is replaced by s0 in the split)
+        s_tk[st] = kg;
+        mbar_arrive_expect_tx(&bar_sfull[st], (unsigned)(NKH * C::SH_LOAD));
+#pragma unroll
+        for (int h = 0; h < NKH; ++h) tma_load_3d(sS + (st * NKH + h) * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[st]);
+      }
+      // the single step-input buffer: wait until the previous tile's inputs were consumed
+      if (it >= 1 && !mbar_wait_flag(&bar_xempty, ((unsigned)(it - 1)) & 1u, ctrl, tmo, &s_abort)) {
+        ++it;
+        break;
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar_xfull, (unsigned)C::X_BYTES);
+        tma_load_3d(smem_raw + C::OFF_X, tm_x, 0, t0, b, &bar_xfull);
+      }
+      __syncwarp();
+      x_issued = it + 1;
+    }
+    for (int j = max(0, it - 2); j < it; ++j)
+      if (!mbar_drain(&bar_sfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
+        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+    if (x_issued > 0 && !mbar_drain(&bar_xfull, ((unsigned)(x_issued - 1)) & 1u, tmo) && lane == 0)
+      atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+  } else if (warp == 1) {
+    // =========================== MMA issuer =================================
+    constexpr uint32_t idesc = umma_idesc_tf32(128, RS);
+    // Descriptors differ between MMAs only in the start address (bits 0-13, address >> 4;
+    // shared addresses stay below 2^18 so the field never carries): precompute the bases
+    // and add compile-time offsets in the fully unrolled issue loop.
+    const uint64_t a_base = umma_smem_desc(smem_addr(sW), 128, C::SBO_W, 0);
+    const uint64_t b_base0 = umma_smem_desc(smem_addr(sS), 16, 1024, 2);
+    const uint64_t b_lo = umma_smem_desc(smem_addr(sLo), 16, 1024, 2);
+    int issued = 0;
+    for (int it = 0;; ++it) {
+      if (!mbar_wait_flag(&bar_afull, (unsigned)it & 1u, ctrl, tmo, &s_abort)) break;
+      if (s_atk[it & 1] < 0) break;
+      const int buf = it & 1;
+      if (it >= 2 && !mbar_wait_flag(&bar_tempty[buf], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t d = tmem + (uint32_t)(buf * RS);
+        const uint64_t b_hi = b_base0 + (uint64_t)(((it & 1) * NKH * C::SH_BYTES) >> 4);
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass) {
+          // pass 0: W_hi S_hi, pass 1: W_lo S_hi, pass 2: W_hi S_lo
+#pragma unroll
+          for (int kb = 0; kb < K / 8; ++kb) {
+            const int h = kb >> 2;   // column half of S; 4 K-steps of 32 bytes per 128-byte swizzled row
+#pragma unroll
+            for (int g = 0; g < C::NSEG; ++g) {
+              const int ws = (pass == 1) ? C::win_lo(g) : C::win_hi(g);
+              const uint64_t ad = a_base + (uint64_t)(((ws / 8) * C::SBO_W + kb * 256) >> 4);
+              const uint64_t bd = (pass == 2 ? b_lo + (uint64_t)((h * C::LO_BYTES + g * RS * 128 + (kb & 3) * 32) >> 4)
+                                             : b_hi + (uint64_t)((h * C::SH_BYTES + g * RS * 128 + (kb & 3) * 32) >> 4));
+              umma_tf32(d, ad, bd, idesc, (pass | kb | g) ? 1u : 0u);
+            }
+          }
+        }
+        umma_commit(&bar_mma[buf]);
+      }
+      __syncwarp();
+      issued = it + 1;
+    }
+    for (int j = max(0, issued - 2); j < issued; ++j)
+      if (!mbar_drain(&bar_mma[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
+        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+  } else if (warp < C::WE0) {
+    // =========================== look-back ==================================
+    // warp 2 + j takes tiles j, j + NLB, ...; self-validating words, flags as hints
+    if constexpr (kScan) {
+      unsigned long long* aggw = reinterpret_cast<unsigned long long*>(P.agg);    // [tile][DP] x {A, B}
+      unsigned long long* prefw = reinterpret_cast<unsigned long long*>(P.pref);  // [tile][DP]
+      const unsigned tag = lookback_tag(epoch);
+      for (int it = warp - 2;; it += C::NLB) {
+        const int slot = it % NSLOT;
+        const unsigned ph = (unsigned)(it / NSLOT) & 1u;
+        if (!mbar_wait_flag(&bar_lb[slot], ph, ctrl, tmo, &s_abort)) break;
+        const int kg = s_lbtk[slot];
+        if (kg < 0) break;
+        const int b = kg % B;
+        const int chunk = kg / B;
+        const size_t k = (size_t)kg;
+        const bool stall = (A.stall_ticket == kg);
+        float2 ag[C::NQ];
+#pragma unroll
+        for (int q = 0; q < C::NQ; ++q)
+          ag[q] = *reinterpret_cast<const float2*>(sAgg + (slot * DP + lane + 32 * q) * 2);
+        // 1. the tile aggregate (the first chunk too: a successor may start from s0)
+        if (!stall) {
+#pragma unroll
+          for (int q = 0; q < C::NQ; ++q)
+            st_word2(aggw + (k * DP + lane + 32 * q) * 2, tag_word(ag[q].x, tag), tag_word(ag[q].y, tag));
+          __syncwarp();
+          if (lane == 0) st_relaxed(P.flags + k, make_flag(epoch, kFlagAgg));
+        }
+        // 2. the carry: nearest published state, then the aggregates in between
+        int n_agg = lookback_nearest_state(P.flags, k, stride, chunk, epoch, ctrl, tmo);
+        float carry[C::NQ];
+#pragma unroll
+        for (int q = 0; q < C::NQ; ++q) carry[q] = 0.0f;
+        if (n_agg >= 0) {
+          if (chunk - 1 - n_agg >= 0) {
+            if (!ld_tagged_state<DP, C::NQ>(prefw + (k - (size_t)(n_agg + 1) * stride) * DP, tag, carry, ctrl, tmo))
+              n_agg = -1;
+          } else {
+#pragma unroll
+            for (int q = 0; q < C::NQ; ++q) {
+              const int j = lane + 32 * q;
+              carry[q] = (j < D) ? __ldg(A.s0 + (size_t)b * D + j) : 0.0f;
+            }
+          }
+        }
+        for (int d0 = n_agg; d0 >= 1; d0 -= 4) {   // oldest aggregate first, four loads in flight
+          float fa[4][C::NQ], fb[4][C::NQ];
+          if (!ld_tagged_aggs<DP, C::NQ>(aggw, k, stride, d0, tag, fa, fb, ctrl, tmo)) {
+            n_agg = -1;
+            break;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (d0 - u >= 1) {
+#pragma unroll
+              for (int q = 0; q < C::NQ; ++q) carry[q] = fmaf(fa[u][q], carry[q], fb[u][q]);
+            }
+        }
+        if (n_agg < 0) s_abort = 1;
+        // 3. hand the carry to the epilogue (its slot is free once tile it - NSLOT was formed)
+        if (it >= NSLOT && !mbar_wait_flag(&bar_cempty[slot], ph ^ 1u, ctrl, tmo, &s_abort)) break;
+#pragma unroll
+        for (int q = 0; q < C::NQ; ++q) sCarry[slot * DP + lane + 32 * q] = carry[q];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_cfull[slot]);
+        // 4. the tile's end state
+        if (n_agg >= 0 && !stall) {
+#pragma unroll
+          for (int q = 0; q < C::NQ; ++q)
+            st_word(prefw + k * DP + lane + 32 * q, tag_word(fmaf(ag[q].x, carry[q], ag[q].y), tag));
+          __syncwarp();
+          if (lane == 0) st_relaxed(P.flags + k, make_flag(epoch, kFlagPrefix));
+        }
+      }
+    }
+  } else {
+    // =========================== epilogue ===================================
+    const int e = warp - C::WE0;            // 0 .. NEW-1
+    const int quarter = warp & 3;           // TMEM lane quarter this warp may access
+    const int rg = e >> 2;                  // 16-step group within the segment
+    const int ln = quarter * 32 + lane;     // TMEM lane = g * DP + c
+    const int g = ln / DP;                  // step segment (warp-uniform)
+    const int c = ln % DP;                  // channel
+    const int row0 = g * RS + 16 * rg;      // first step (tile row) of this thread
+    const int piece = g * C::NRG + rg;      // warp-uniform
+    const int te = tid - 32 * C::WE0;       // 0 .. NTE-1 among the epilogue threads
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int hc = c >> 5;                  // column half of channel c in S
+    const int cc = c & 31;                  // its column within the half
+    const float wdc = sWd[c];
+
+    // S_lo of stage `stg` (rows 0..L-1), swizzled like S.  For the first chunk of a
+    // sequence, row 0 (step -1, loaded as zero) becomes s0 first.
+    auto split = [&](int stg, int kgs) {
+      const bool first = (kgs / B) == 0;
+      const float* s0row = A.s0 + (size_t)(kgs % B) * D;
+      for (int u = te; u < NKH * L * 8; u += NTE) {
+        const int q = u & 7;
+        const int r = (u >> 3) % L;
+        const int h = (u >> 3) / L;
+        const uint32_t off = sw128_offset(r, 4 * q);
+        unsigned char* srow = sS + (stg * NKH + h) * C::SH_BYTES;
+        float4 v;
+        if (first && r == 0) {
+          v = __ldg(reinterpret_cast<const float4*>(s0row + 32 * h) + q);
+          *reinterpret_cast<float4*>(srow + off) = v;
+        } else {
+          v = *reinterpret_cast<const float4*>(srow + off);
+        }
+        *reinterpret_cast<float4*>(sLo + h * C::LO_BYTES + off) =
+            make_float4(tf32_tail(v.x), tf32_tail(v.y), tf32_tail(v.z), tf32_tail(v.w));
+      }
+      fence_async_smem();   // generic writes -> the tensor cores (async proxy)
+    };
+
+    // operands of the tile after `itn - 1`: wait for its stage, split it, publish its ticket
+    // (the exit decision, read by everyone after the next named barrier) and wake the MMA warp
+    auto prepare = [&](int itn) {
+      const int stg = itn & 1;
+      int kn = -1;
+      if (mbar_wait_flag(&bar_sfull[stg], ((unsigned)itn >> 1) & 1u, ctrl, tmo, &s_abort)) kn = s_tk[stg];
+      if (kn >= 0 && !s_abort) split(stg, kn);
+      __syncwarp();
+      if (lane == 0) {
+        if (te == 0) s_atk[itn & 1] = s_abort ? -1 : kn;
+        mbar_arrive(&bar_afull);
+      }
+    };
+
+    // s^(i+1) of tile j (ticket kgj): piece carry from the look-back carry, then the parked prefixes
+    auto write_out = [&](int j, int kgj, float pa, float pb) {
+      const int slot = j % NSLOT;
+      mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort);
+      const float carry = sCarry[slot * DP + c];
+      const float cp = kHasA ? fmaf(pa, carry, pb) : carry + pb;
+      const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + 16 * rg) + lane_off;
+      float bb[16], aa[16];
+      tmem_ld16(sbase + (uint32_t)(kHasA ? RS : 0), bb);
+      if constexpr (kHasA) tmem_ld16(sbase, aa);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_cempty[slot]);
+      if (!s_abort) {
+        const int tj = (kgj / B) * L + row0;
+        float* o = dst + ((size_t)(kgj % B) * T + tj) * D + c;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (tj + i < T) o[(size_t)i * D] = kHasA ? fmaf(aa[i], cp, bb[i]) : cp + bb[i];
+      }
+    };
+
+    // The loop's exit decision is one thread's reading of the next stage's ticket,
+    // published before a named barrier, so every epilogue thread takes the same path.
+    prepare(0);
+    named_barrier(1, NTE);
+    int kg = s_atk[0];
+    int it = 0;
+    int kg_m1 = -1, kg_m2 = -1;              // tickets of tiles it-1, it-2
+    float pa1 = 1.0f, pb1 = 0.0f, pa2 = 1.0f, pb2 = 0.0f;   // their piece prefixes
+    for (; kg >= 0; ++it) {
+      const int st = it & 1;
+      const int buf = it & 1;
+      const int b = kg % B;
+      const int t0 = (kg / B) * L;
+
+      // ---- Z of this thread's channel and 16 steps, then cell + sequential scan
+      mbar_wait_flag(&bar_mma[buf], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort);
+      tc_fence_after();
+      float z[16];
+      tmem_ld16(tmem + (uint32_t)(buf * RS + 16 * rg) + lane_off, z);
+      mbar_wait_flag(&bar_xfull, (unsigned)it & 1u, ctrl, tmo, &s_abort);
+      const unsigned char* Sh = sS + (st * NKH + hc) * C::SH_BYTES;
+      // step t0 + row0 - 1; for the first step of a sequence that is s0 (the stage's row 0
+      // holds s0 only for the tensor cores)
+      float sp = (t0 + row0 == 0) ? __ldg(A.s0 + (size_t)b * D + c)
+                                  : *reinterpret_cast<const float*>(Sh + sw128_offset(row0, cc));
+      float SA = 1.0f, SB = 0.0f;
+      float av[16], bv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = row0 + i;
+        const float sc = *reinterpret_cast<const float*>(Sh + sw128_offset(r + 1, cc));
+        const float xv = sX[r * DP + c];
+        float y, a, bb, res;
+        if constexpr (CELL == PN_CELL_TANH_RNN) {
+          y = tanh_pn(z[i] + xv);
+          res = sc - y;
+          a = (MODE == PN_QUASI) ? (1.0f - y * y) * wdc : (MODE == PN_PICARD ? 1.0f : 0.0f);
+          bb = (MODE == PN_JACOBI) ? y : y - a * sp;
+        } else {
+          const float gg = tanh_pn(z[i] + xv);
+          const float eg = P.eps * gg;
+          y = sp + eg;
+          res = (sc - sp) - eg;
+          if (MODE == PN_QUASI) {
+            const float ed = P.eps * (1.0f - gg * gg) * wdc;
+            a = 1.0f + ed;
+            bb = eg - ed * sp;
+          } else if (MODE == PN_PICARD) {
+            a = 1.0f;
+            bb = eg;
+          } else {
+            a = 0.0f;
+            bb = y;
+          }
+        }
+        if (t0 + r < T) {
+          rbits = max(rbits, abs_bits(res));
+        } else {
+          a = 1.0f;
+          bb = 0.0f;
+        }
+        if constexpr (kHasA) {
+          SB = fmaf(a, SB, bb);
+          SA *= a;
+        } else {
+          SB += bb;   // Picard: a = 1; Jacobi: SB unused
+        }
+        av[i] = SA;
+        bv[i] = (MODE == PN_JACOBI) ? bb : SB;
+        sp = sc;
+      }
+      // this tile's TMEM accumulator, step inputs and s stage are consumed
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar_tempty[buf]);
+        mbar_arrive(&bar_xempty);
+        mbar_arrive(&bar_sempty[st]);
+      }
+      // the next tile's operands (S_lo is free: this tile's products are done)
+      prepare(it + 1);
+
+
+      if constexpr (!kScan) {
+        if (!s_abort) {
+          float* o = dst + ((size_t)b * T + t0 + row0) * D + c;
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (t0 + row0 + i < T) o[(size_t)i * D] = bv[i];
+        }
+        named_barrier(1, NTE);   // the ticket of tile it+1
+        kg = s_atk[(it + 1) & 1];
+      } else {
+        // the states of tile it-2: its carry had two tiles of time to arrive
+        if (it >= C::DEFER) write_out(it - C::DEFER, kg_m2, pa2, pb2);
+
+        // ---- combine the 8 pieces of each channel
+        float* tot = sTot + (it & 1) * C::NPC * DP * 2;
+        *reinterpret_cast<float2*>(tot + (piece * DP + c) * 2) = make_float2(SA, SB);
+        named_barrier(1, NTE);   // piece totals, and the ticket of tile it+1
+        const int kg_next = s_atk[(it + 1) & 1];
+        float PA = 1.0f, PB = 0.0f;   // prefix of the earlier pieces
+        for (int p = 0; p < piece; ++p) {
+          const float2 w = *reinterpret_cast<const float2*>(tot + (p * DP + c) * 2);
+          PB = kHasA ? fmaf(w.x, PB, w.y) : PB + w.y;
+          if (kHasA) PA *= w.x;
+        }
+        // the last piece's inclusive prefix is the tile aggregate: hand it to the look-back
+        const int slot = it % NSLOT;
+        if (piece == C::NPC - 1) {
+          *reinterpret_cast<float2*>(sAgg + (slot * DP + c) * 2) =
+              kHasA ? make_float2(SA * PA, fmaf(SA, PB, SB)) : make_float2(1.0f, PB + SB);
+          __syncwarp();
+          if (lane == 0) {
+            if (c == 0) s_lbtk[slot] = s_abort ? -1 : kg;
+            mbar_arrive(&bar_lb[slot]);
+          }
+        }
+        // ---- park the in-piece prefixes in TMEM; formed two tiles later
+        {
+          const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + 16 * rg) + lane_off;
+          if constexpr (kHasA) tmem_st16(sbase, av);
+          tmem_st16(sbase + (uint32_t)(kHasA ? RS : 0), bv);
+          tmem_st_wait();
+        }
+        pa2 = pa1;
+        pb2 = pb1;
+        pa1 = PA;
+        pb1 = PB;
+        kg_m2 = kg_m1;
+        kg_m1 = kg;
+        kg = kg_next;
+      }
+    }
+    if constexpr (kScan) {
+      if (it >= 2) write_out(it - 2, kg_m2, pa2, pb2);
+      if (it >= 1) write_out(it - 1, kg_m1, pa1, pb1);
+      // stop the look-back warps: their next tiles are it .. it + NLB - 1
+      if (piece == C::NPC - 1 && lane == 0) {
+        for (int j = it; j < it + C::NLB; ++j) {
+          if (c == 0) s_lbtk[j % NSLOT] = -1;
+          mbar_arrive(&bar_lb[j % NSLOT]);
+        }
+      }
+    }
+  }
+
+  // ---- residual, TMEM release, end-of-launch decision ------------------------
+  rbits = warp_max_u32(rbits);
+  if (lane == 0) sRed[warp] = __uint_as_float(rbits);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::ALLOC_COLS)
+                 : "memory");
+  if (tid == 0) {
+    unsigned v = 0u;
+    for (int w = 0; w < C::NT / 32; ++w) v = max(v, __float_as_uint(sRed[w]));
+    if (v) atomicMax(&ctrl->resid_bits, v);
+  }
+  finish_launch(P, A, epoch, s_last);
+}
+
+}  // namespace pn
