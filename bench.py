@@ -237,6 +237,26 @@ def reference_arm(args, prob, mode, rank, world):
 
 
 # ----------------------------------------------------------------------------
+# multi-rank aggregation (independent instances, one per rank: weak scaling)
+# ----------------------------------------------------------------------------
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time for the same timed region; every rank calls this at the same point
+    (a collective). Without a process group it is the local time."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
+# ----------------------------------------------------------------------------
 # the CUDA path
 # ----------------------------------------------------------------------------
 
@@ -275,14 +295,9 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
         e1.record(stream)
         barrier()
         clk.mark_end()
-    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     stats = solver.stats()
-    if dist is not None:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    units = prob.T * prob.B * world * args.steps
-    value = units / (ms / 1e3)
+    value = job_throughput(prob.T * prob.B * args.steps, world, ms)
     launches_per_step = (iters + 1) + 2 + (0 if prob.cell == pi.CELL_EULER else 1)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -328,12 +343,8 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
         solver.eval_host(hxn, hs0n, mode, mi, tol, hstn)
     e1.record(stream)
     barrier()
-    ems = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ems], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
-    line["e2e"] = {"value": units / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(prob.x.nbytes + prob.s0.nbytes),
+    ems = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    line["e2e"] = {"value": job_throughput(prob.T * prob.B * args.steps, world, ems), "unit": UNIT, "h2d_bytes_per_step": int(prob.x.nbytes + prob.s0.nbytes),
                    "d2h_bytes_per_step": int(prob.B * prob.T * prob.D * 4), "ms_per_step": ems / args.steps}
     solver.close()
     return line
