@@ -141,11 +141,14 @@ PN_API pn_status pn_eval_host(pn_handle h, const float* x_host, const float* s0_
 PN_API pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written);
 
 /* Time the fused iteration kernel of `mode` alone: after a pn_eval on this
- * handle (its x, s0 and states must still be valid), launch exactly
- * n_launches iteration kernels back to back on the handle's stream, with no
- * stop rule, bracketed by CUDA events.  *avg_ms receives the mean duration per
- * launch.  The states buffer of that pn_eval is overwritten with later
- * iterates. */
+ * handle (its x, s0 and states must still be valid), run exactly n_launches
+ * iterations on the handle's stream with no stop rule, bracketed by CUDA
+ * events, and return the mean time per iteration in *avg_ms.  Kernels that
+ * launch once per iteration are launched n_launches times back to back;
+ * kernels that loop over iterations on the device (the quasi-Newton
+ * tensor-core kernel of the one-gate cells) run one launch of n_launches
+ * iterations, as in pn_eval.  The states buffer of that pn_eval is
+ * overwritten with later iterates. */
 PN_API pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* avg_ms);
 
 PN_API pn_status pn_get_stats(pn_handle h, pn_stats* out);

@@ -273,7 +273,8 @@ struct PreLaunch {
   bool has_proj = false;
   dim3 proj_grid;
   int M = 0, N = 0, K = 0;
-  unsigned init_grid = 1, fin_grid = 1;
+  dim3 init_grid{1, 1, 1};
+  unsigned fin_grid = 1;
 };
 
 PreLaunch pre_launch(const pn_ctx* h) {
@@ -284,7 +285,10 @@ PreLaunch pre_launch(const pn_ctx* h) {
   p.K = h->d_in;
   p.proj_grid = dim3((unsigned)((p.M + kProjTile - 1) / kProjTile), (unsigned)((p.N + kProjTile - 1) / kProjTile));
   const size_t n = (size_t)h->B * h->T * h->D;
-  p.init_grid = grid_1d(n, 256, 148u * 16u);
+  // init: about 8 CTAs per SM in all, whole sequences per grid row
+  const unsigned gy = (unsigned)std::min(h->B, 65535);
+  const unsigned gx = std::max(1u, std::min(grid_1d((size_t)h->T * h->D / 4 + 1, 256, 1u << 20), (148u * 8u) / gy));
+  p.init_grid = dim3(gx, gy);
   p.fin_grid = grid_1d(n / 4 + 1, 256, 148u * 16u);
   return p;
 }
@@ -325,12 +329,20 @@ pn_status build_graph(pn_ctx* h, int mode) {
     Ctrl* c = h->ctrl;
     int D = h->D, T = h->T, B = h->B;
     void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&D, (void*)&T, (void*)&B};
-    e = add_kernel(g, (const void*)&init_kernel, dim3(pl.init_grid), dim3(256), 0, kargs,
+    e = add_kernel(g, (const void*)&init_kernel, pl.init_grid, dim3(256), 0, kargs,
                    prev ? &prev : nullptr, &node);
     if (e != cudaSuccess) goto fail_graph;
     prev = node;
   }
-  {
+  if (ki.kind == kKindDiagTct) {
+    // 3. one launch of the looping kernel: it iterates on the device until the stop rule
+    IterParams P = make_params(h, mode);
+    P.persist = 1;
+    void* kargs[] = {(void*)&P};
+    e = add_kernel(g, ki.fn, dim3((unsigned)h->fam.grid[mode]), dim3(ki.nt), ki.smem, kargs, &prev, &node);
+    if (e != cudaSuccess) goto fail_graph;
+    prev = node;
+  } else {
     // 3. WHILE (condition set to 0 by the iteration kernel's last CTA)
     cudaGraphConditionalHandle cond;
     e = cudaGraphConditionalHandleCreate(&cond, g, 1u, cudaGraphCondAssignDefault);
@@ -371,9 +383,10 @@ fail_graph:
   return fail(h, PN_ERR_CUDA, "building the CUDA graph for mode %d failed: %s", mode, cudaGetErrorString(e));
 }
 
-pn_status launch_iter(pn_ctx* h, int mode) {
+pn_status launch_iter(pn_ctx* h, int mode, int persist = 0) {
   const KInfo& ki = h->fam.k[mode];
   IterParams P = make_params(h, mode);
+  P.persist = persist;
   void* kargs[] = {(void*)&P};
   PN_CUDA(h, cudaLaunchKernel(ki.fn, dim3((unsigned)h->fam.grid[mode]), dim3(ki.nt), kargs, ki.smem, h->stream));
   return PN_OK;
@@ -393,7 +406,7 @@ pn_status launch_pre(pn_ctx* h) {
   Ctrl* c = h->ctrl;
   int D = h->D, T = h->T, B = h->B;
   void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&D, (void*)&T, (void*)&B};
-  PN_CUDA(h, cudaLaunchKernel((const void*)&init_kernel, dim3(pl.init_grid), dim3(256), kargs, 0, h->stream));
+  PN_CUDA(h, cudaLaunchKernel((const void*)&init_kernel, pl.init_grid, dim3(256), kargs, 0, h->stream));
   return PN_OK;
 }
 
@@ -868,9 +881,23 @@ pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* a
   pn_status st = validate_mode(h, mode, 0, 0.0f);
   if (st != PN_OK) return st;
   if (!h->args_h->states) return fail(h, PN_ERR_INVALID, "call pn_eval on this handle first");
-  // every launch re-evaluates the same iterate: r <= +inf stops the counter
-  h->args_h->tol = INFINITY;
-  h->args_h->max_iters = INT_MAX;
+  // Kernels that iterate on the device (the graph runs them as one launch per evaluation) are
+  // timed the same way: one launch that runs n_launches iterations (a tolerance below zero never
+  // stops it early, max_iters ends it), average = elapsed / n_launches.  The others: n_launches
+  // launches that each re-evaluate the same iterate (r <= +inf stops after one iteration).
+  const bool looping = (h->fam.k[mode].kind == kKindDiagTct);
+  if (looping) {
+    PN_CUDA(h, cudaMemcpy(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost));
+    const long long last = (long long)h->ctrl_h->iter + n_launches - 1;
+    if (last > INT_MAX) return fail(h, PN_ERR_INVALID, "n_launches too large");
+    h->args_h->tol = -1.0f;
+    h->args_h->max_iters = (int)last;
+    const int running[2] = {kRunning, 0};   // ctrl->status, ctrl->error
+    PN_CUDA(h, cudaMemcpy(&h->ctrl->status, running, sizeof running, cudaMemcpyHostToDevice));
+  } else {
+    h->args_h->tol = INFINITY;
+    h->args_h->max_iters = INT_MAX;
+  }
   h->args_h->use_cond = 0;
   if ((st = prepare_lookback(h, mode)) != PN_OK) return st;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
@@ -880,7 +907,8 @@ pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* a
   PN_CUDA(h, cudaEventCreate(&e1));
   st = PN_OK;
   cudaError_t ce = cudaEventRecord(e0, h->stream);
-  for (int i = 0; i < n_launches && ce == cudaSuccess && st == PN_OK; ++i) st = launch_iter(h, mode);
+  if (looping) st = launch_iter(h, mode, 1);
+  for (int i = 0; !looping && i < n_launches && ce == cudaSuccess && st == PN_OK; ++i) st = launch_iter(h, mode);
   if (ce == cudaSuccess) ce = cudaEventRecord(e1, h->stream);
   if (ce == cudaSuccess) ce = cudaEventSynchronize(e1);
   float ms = 0.0f;
@@ -891,6 +919,9 @@ pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* a
   if (ce != cudaSuccess) return fail(h, PN_ERR_CUDA, "timing failed: %s", cudaGetErrorString(ce));
   PN_CUDA(h, cudaMemcpy(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost));
   if (h->ctrl_h->error) return fail(h, PN_ERR_TIMEOUT, "a look-back wait gave up during timing");
+  if (looping && h->ctrl_h->final_iter != (int)h->args_h->max_iters)
+    return fail(h, PN_ERR_CUDA, "timing run stopped at iteration %d, expected %d", h->ctrl_h->final_iter,
+                h->args_h->max_iters);
   *avg_ms = ms / (float)n_launches;
   return PN_OK;
 }

@@ -64,19 +64,27 @@ __global__ void __launch_bounds__(256) proj_kernel(const Args* __restrict__ args
   }
 }
 
-// s^(0)_t = s0 for every t, and a fresh control block for the loop.
+// s^(0)_t = s0 for every t, and a fresh control block for the loop.  Each
+// blockIdx.y takes whole sequences (b = blockIdx.y, + gridDim.y, ...), the x
+// dimension strides over one sequence; 16-byte stores when D % 4 == 0.
 __global__ void init_kernel(const Args* __restrict__ args, Ctrl* __restrict__ ctrl, int D, int T,
                             int B) {
-  const float* s0 = args->s0;
-  float* st = args->states;
-  const size_t n = (size_t)B * T * D;
-  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
-       e += (size_t)gridDim.x * blockDim.x) {
-    const size_t b = e / ((size_t)T * D);
-    const size_t c = e % D;
-    st[e] = __ldg(s0 + b * D + c);
+  const size_t per_seq = (size_t)T * D;
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t nthr = (size_t)gridDim.x * blockDim.x;
+  for (int b = blockIdx.y; b < B; b += gridDim.y) {
+    const float* s0 = args->s0 + (size_t)b * D;
+    float* st = args->states + (size_t)b * per_seq;
+    if ((D & 3) == 0) {
+      const size_t D4 = (size_t)(D >> 2);
+      const float4* s04 = reinterpret_cast<const float4*>(s0);
+      float4* st4 = reinterpret_cast<float4*>(st);
+      for (size_t e = tid; e < per_seq / 4; e += nthr) st4[e] = __ldg(s04 + e % D4);
+    } else {
+      for (size_t e = tid; e < per_seq; e += nthr) st[e] = __ldg(s0 + e % (size_t)D);
+    }
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
+  if (blockIdx.y == 0 && blockIdx.x == 0 && threadIdx.x == 0) {
     ctrl->iter = 0;
     ctrl->status = kRunning;
     ctrl->error = 0;

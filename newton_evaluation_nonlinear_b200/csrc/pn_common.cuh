@@ -33,7 +33,8 @@ struct Ctrl {
   int timeout_ticket;  // ticket whose wait gave up (diagnostics), -1 if none
   unsigned long long t_start;    // min %globaltimer at CTA entry, current launch
   unsigned long long kernel_ns;  // summed launch durations
-  unsigned long long launches;   // fused iteration launches
+  unsigned long long launches;   // iterations run by the fused iteration kernels
+  unsigned gen;        // grid-barrier generation of the looping kernels (iterations completed)
 };
 
 // Per-call arguments, written by the host before each evaluation.
@@ -68,6 +69,7 @@ struct IterParams {
   int ngroups, nchunks;
   int tiles_per_group;  // B * nchunks: tickets of one channel group
   int agg_stride, pref_stride;
+  int persist;          // looping kernels: 1 = run iterations until the stop rule, 0 = one iteration
   cudaGraphConditionalHandle cond;
 };
 
@@ -312,6 +314,71 @@ __device__ __forceinline__ void finish_launch(const IterParams& P, const Args& A
   c->launches += 1ull;
   c->t_start = ~0ull;
   __threadfence();
+}
+
+// Looping kernels (P.persist = 1): every CTA calls this at the end of an
+// iteration, after all of its global writes and with its residual folded into
+// ctrl->resid_bits.  The last CTA to arrive applies the stop rule exactly as
+// finish_launch does and opens the next iteration (generation gen_before + 1);
+// the others wait for it, bounded by the handle's timeout.  Returns, for every
+// thread of the CTA, whether another iteration follows.
+__device__ __forceinline__ bool finish_iteration(const IterParams& P, const Args& A, unsigned epoch,
+                                                 int& flag_smem, unsigned gen_before) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Ctrl* c = P.ctrl;
+    __threadfence();
+    const unsigned prev = atomicAdd(&c->done, 1u);
+    int go = 0;
+    if (prev == gridDim.x - 1) {
+      __threadfence();
+      const int i = c->iter;
+      const float r = __uint_as_float(atomicAdd(&c->resid_bits, 0u));
+      const int err = ld_volatile(&c->error);
+      if (i < kHistCap) P.hist[i] = r;
+      int st = kRunning;
+      if (err) st = err;
+      else if (!(r <= 3.402823466e38f)) st = PN_ERR_NONFINITE;
+      else if (r <= A.tol) st = PN_OK;
+      else if (i >= A.max_iters) st = PN_NOT_CONVERGED;
+      c->launches += 1ull;
+      if (st != kRunning) {
+        c->status = st;
+        c->final_iter = i;
+        c->final_resid = r;
+        const unsigned long long t1 = globaltimer();
+        const unsigned long long t0 = c->t_start;
+        if (t1 > t0) c->kernel_ns += t1 - t0;
+        c->t_start = ~0ull;
+      } else {
+        c->iter = i + 1;
+        go = 1;
+      }
+      c->resid_bits = 0u;
+#pragma unroll
+      for (int g = 0; g < kMaxGroups; ++g) c->ticket[g] = 0u;
+      c->done = 0u;
+      c->epoch = epoch + 1u;
+      __threadfence();
+      st_release(&c->gen, gen_before + 1u);
+    } else {
+      const unsigned long long t0 = globaltimer();
+      unsigned spins = 0;
+      bool ok = true;
+      while (ld_acquire(&c->gen) == gen_before) {
+        if (((++spins) & 15u) == 0u && (long long)(globaltimer() - t0) > A.timeout_ns) {
+          atomicCAS(&c->error, 0, (int)PN_ERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+        if (spins > 64u) __nanosleep(128);
+      }
+      go = ok && ld_volatile(&c->status) == kRunning;
+    }
+    flag_smem = go;
+  }
+  __syncthreads();
+  return flag_smem != 0;
 }
 
 }  // namespace pn

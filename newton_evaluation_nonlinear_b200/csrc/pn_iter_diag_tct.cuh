@@ -23,6 +23,11 @@
 // the look-back warps, stored straight from registers (a warp writes 32
 // consecutive channels of one step: 128 contiguous bytes).
 //
+// With P.persist = 1 the kernel runs the whole fixed-point loop in one launch:
+// after each iteration the CTAs meet at a bounded grid barrier whose last
+// arrival applies the stop rule, then the next iteration starts with the
+// weights, TMEM and barrier memory of the CTA kept (no launch gap, no set-up).
+//
 // Warp roles (one CTA per SM): 0 producer (tickets, TMA loads); 1 MMA issuer;
 // 2-3 look-back (scan modes, alternate tiles); the rest epilogue (4 TMEM lane
 // quarters x RS / 16 step groups).  The epilogue forms the next tile's S_lo
@@ -127,8 +132,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   const size_t stride = (size_t)B;   // consecutive chunks of a sequence are B tickets apart
   const long long tmo = A.timeout_ns;
 
-  if (tid == 0) {
-    atomicMin(&ctrl->t_start, globaltimer());
+  auto init_barriers = [&]() {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_sfull[s], 1u);
       mbar_init(&bar_sempty[s], (unsigned)C::NEW);
@@ -144,13 +148,31 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     mbar_init(&bar_xempty, (unsigned)C::NEW);
     mbar_init(&bar_afull, (unsigned)C::NEW);
     mbar_init_fence();
+  };
+  auto inval_barriers = [&]() {
+    uint64_t* bars[] = {&bar_sfull[0], &bar_sfull[1], &bar_sempty[0], &bar_sempty[1], &bar_mma[0], &bar_mma[1],
+                        &bar_tempty[0], &bar_tempty[1], &bar_xfull, &bar_xempty, &bar_afull};
+    for (uint64_t* bb : bars) mbar_inval(bb);
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_inval(&bar_lb[s]);
+      mbar_inval(&bar_cfull[s]);
+      mbar_inval(&bar_cempty[s]);
+    }
+  };
+  const unsigned gen0 = *(volatile unsigned*)&ctrl->gen;
+  unsigned epoch = 0u;
+  for (int round = 0;; ++round) {
+  if (tid == 0) {
+    if (round == 0) atomicMin(&ctrl->t_start, globaltimer());
+    else inval_barriers();   // every operation on them of the last iteration has completed
+    init_barriers();
     s_abort = 0;
   }
-  const unsigned epoch = *(volatile unsigned*)&ctrl->epoch;
+  epoch = *(volatile unsigned*)&ctrl->epoch;
   const int iter = *(volatile int*)&ctrl->iter;
   if (tid == 0) {
     // The first tile of every CTA has a static ticket (blockIdx.x < tiles: the grid is never
-    // larger) and is fetched right away, overlapping the weight load and TMEM set-up below.
+    // larger) and is fetched right away, overlapping the remaining set-up.
     const CUtensorMap* tm_s = P.tmaps + ((iter & 1) ? 1 : 0);
     const CUtensorMap* tm_x = P.tmaps + 2;
     tmap_acquire(tm_s);
@@ -172,9 +194,9 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   }
   float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;
 
-  // banded W (hi and lo in the K-major core-matrix layout): the zero bands are written here,
-  // only the W_hi and W_lo row blocks (pre-packed by the host at their band offsets) are loaded
-  {
+  if (round == 0) {
+    // banded W (hi and lo in the K-major core-matrix layout): the zero bands are written here,
+    // only the W_hi and W_lo row blocks (pre-packed by the host at their band offsets) are loaded
     const float4* w4 = reinterpret_cast<const float4*>(P.wt);
     float4* d4 = reinterpret_cast<float4*>(sW);
     constexpr int ROW16 = DP / 4;                 // float4s per row of the K-major layout (on average)
@@ -186,12 +208,12 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     }
     for (int e = tid; e < DP; e += C::NT) sWd[e] = __ldg(P.wdiag + e);
     fence_async_smem();   // the tensor cores read sW through the async proxy
-  }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
-                 "r"((uint32_t)C::ALLOC_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (warp == 0) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
+                   "r"((uint32_t)C::ALLOC_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -589,21 +611,28 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     }
   }
 
-  // ---- residual, TMEM release, end-of-launch decision ------------------------
+  // ---- residual of this iteration; next iteration or end of the launch ------
   rbits = warp_max_u32(rbits);
   if (lane == 0) sRed[warp] = __uint_as_float(rbits);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::ALLOC_COLS)
-                 : "memory");
   if (tid == 0) {
     unsigned v = 0u;
     for (int w = 0; w < C::NT / 32; ++w) v = max(v, __float_as_uint(sRed[w]));
     if (v) atomicMax(&ctrl->resid_bits, v);
   }
-  finish_launch(P, A, epoch, s_last);
+  if (!P.persist) break;
+  if (!finish_iteration(P, A, epoch, s_last, gen0 + (unsigned)round)) break;
+  }   // iterations
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(s_tmem), "r"((uint32_t)C::ALLOC_COLS)
+                 : "memory");
+  if (!P.persist) finish_launch(P, A, epoch, s_last);
 }
 
 }  // namespace pn
