@@ -88,9 +88,10 @@ def peaks():
 
 
 def kernel_source_sha() -> str:
+    """Hash of the device code: the kernel headers and the per-cell kernel units (host code excluded)."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cuh", ".cu")):
+        if name.endswith(".cuh") or (name.startswith("pn_k_") and name.endswith(".cu")):
             with open(os.path.join(CSRC, name), "rb") as f:
                 h.update(f.read())
     return h.hexdigest()[:16]
@@ -298,7 +299,9 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
     ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     stats = solver.stats()
     value = job_throughput(prob.T * prob.B * args.steps, world, ms)
-    launches_per_step = (iters + 1) + 2 + (0 if prob.cell == pi.CELL_EULER else 1)
+    looping = pn.pn_dim(solver.h, 5 + mode) == 1 and not args.host_loop
+    # projection (not for the Euler cell), init, the iteration kernel(s), result copy
+    launches_per_step = (1 if looping else iters + 1) + 2 + (0 if prob.cell == pi.CELL_EULER else 1)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -307,7 +310,8 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
                        "D": prob.D, "d_in": prob.d_in, "T": prob.T, "B": prob.B, "tol": prob.tol,
                        "max_iters": mi, "iters": iters, "final_resid": resid, "status": st,
                        "parallelism": f"independent instances x{world}",
-                       "loop": "host" if args.host_loop else "device (CUDA graph WHILE node)",
+                       "loop": "host" if args.host_loop else ("device (one launch iterating to the stop rule)"
+                                                               if looping else "device (CUDA graph WHILE node)"),
                        "l2": "inputs larger than L2 (x, u, two iterate buffers: "
                              f"{(prob.x.nbytes + 3 * prob.B * prob.T * prob.D * 4) / 1e6:.0f} MB)"},
             "clocks": clk.summary(), "gpu_launches": launches_per_step * args.steps}
@@ -318,16 +322,17 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
     # roofline of the fused iteration kernel: CUDA events around back-to-back launches
     n_l = max(10, 3 * (iters + 1))
     kms = solver.time_iterations(mode, n_l)
-    in_graph_us = stats["iteration_ns"] / max(1, stats["iteration_launches"]) / 1e3
+    in_eval_us = stats["iteration_ns"] / max(1, stats["iteration_launches"]) / 1e3
     hbm, src = peaks()
     bytes_launch = alg_bytes_per_step(prob) * prob.B * prob.T
     achieved = bytes_launch / (kms / 1e3) / 1e9
     traffic = traffic_from_profile(prob, mode)
     line["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                         "frac": achieved / hbm, "traffic": traffic, "peak_source": src,
-                        "kernel": "fused iteration (cell + Jacobian + chunked scan + residual)",
+                        "kernel": "fused iteration (cell + Jacobian + chunked scan + residual)"
+                                  + (", one launch looping over iterations: figures per iteration" if looping else ""),
                         "alg_bytes_per_launch": bytes_launch, "launch_ms": kms,
-                        "in_graph_launch_us": in_graph_us,
+                        "in_eval_us_per_iteration": in_eval_us,
                         "fp32_tflops": alg_flops_per_step(prob, mode) * prob.B * prob.T / (kms / 1e3) / 1e12}
 
     # end to end through the host-buffer entry point, copies inside the timed region

@@ -189,8 +189,11 @@ PN_API pn_status pn_eval_static(const float* params, size_t n_params, int D, int
  * on cuda_stream and the call synchronises it.  For accuracy tests. */
 PN_API pn_status pn_activation(int which, const float* x, float* y, long long n, void* cuda_stream);
 
-/* Shape queries (for the binding); each returns -1 for a NULL handle. */
-PN_API int pn_dim(pn_handle h, int which /* 0=D 1=d_in 2=T 3=B 4=cell */);
+/* Shape queries (for the binding); each returns -1 for a NULL handle.
+ * which = 0..4: D, d_in, T, B, cell.  which = 5 + mode: 1 when that mode's
+ * iteration kernel loops over the iterations on the device (one launch per
+ * evaluation), 0 when pn_eval launches it once per iteration. */
+PN_API int pn_dim(pn_handle h, int which);
 
 /* Last error message of this handle, or of the calling thread's last failed
  * pn_create when h is NULL.  Never NULL; "" when there was no error. */

@@ -334,15 +334,7 @@ pn_status build_graph(pn_ctx* h, int mode) {
     if (e != cudaSuccess) goto fail_graph;
     prev = node;
   }
-  if (ki.kind == kKindDiagTct) {
-    // 3. one launch of the looping kernel: it iterates on the device until the stop rule
-    IterParams P = make_params(h, mode);
-    P.persist = 1;
-    void* kargs[] = {(void*)&P};
-    e = add_kernel(g, ki.fn, dim3((unsigned)h->fam.grid[mode]), dim3(ki.nt), ki.smem, kargs, &prev, &node);
-    if (e != cudaSuccess) goto fail_graph;
-    prev = node;
-  } else {
+  {
     // 3. WHILE (condition set to 0 by the iteration kernel's last CTA)
     cudaGraphConditionalHandle cond;
     e = cudaGraphConditionalHandleCreate(&cond, g, 1u, cudaGraphCondAssignDefault);
@@ -488,7 +480,12 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   h->args_h->use_cond = h->device_loop ? 1 : 0;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
   if ((st = upload_tc_maps(h, mode)) != PN_OK) return st;
-  if (h->device_loop) {
+  if (h->device_loop && h->fam.k[mode].kind == kKindDiagTct) {
+    // the iteration kernel loops on the device: four plain launches, no graph needed
+    if ((st = launch_pre(h)) != PN_OK) return st;
+    if ((st = launch_iter(h, mode, 1)) != PN_OK) return st;
+    if ((st = launch_finish(h)) != PN_OK) return st;
+  } else if (h->device_loop) {
     st = build_graph(h, mode);
     if (st != PN_OK) return st;
     PN_CUDA(h, cudaGraphLaunch(h->exec[mode], h->stream));
@@ -1003,6 +1000,10 @@ int pn_dim(pn_handle h, int which) {
     case 2: return h->T;
     case 3: return h->B;
     case 4: return h->cell;
+    case 5 + PN_JACOBI:
+    case 5 + PN_PICARD:
+    case 5 + PN_QUASI:
+    case 5 + PN_NEWTON: return h->fam.k[which - 5].kind == kKindDiagTct ? 1 : 0;
     default: return -1;
   }
 }
