@@ -51,7 +51,8 @@ struct DiagTctCfg {
   static constexpr int NRG = RS / 16;            // 16-step groups per segment
   static constexpr int NPC = NSEG * NRG;         // pieces per channel (L / 16)
   static constexpr int NKH = DP / 32;            // 32-float column halves of S
-  static constexpr int SCOLS = (MODE == PN_QUASI ? 2 : 1) * RS;   // stash columns per tile: [A |] B
+  static constexpr int SCOLS = (MODE == PN_QUASI ? 2 : 1) * RS;   // stash columns per tile: per 16-step
+                                                                     // group, [A (16) |] B (16)
   static constexpr int NSLOT = 3;                // tiles between their scan and their write-out, + 1
   static constexpr int DEFER = NSLOT - 1;
   static constexpr int NLB = kScan ? 2 : 0;      // look-back warps, alternating tiles
@@ -449,18 +450,29 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort);
       const float carry = sCarry[slot * DP + c];
       const float cp = kHasA ? fmaf(pa, carry, pb) : carry + pb;
-      const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + 16 * rg) + lane_off;
-      float bb[16], aa[16];
-      tmem_ld16(sbase + (uint32_t)(kHasA ? RS : 0), bb);
-      if constexpr (kHasA) tmem_ld16(sbase, aa);
+      const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + (kHasA ? 32 : 16) * rg) + lane_off;
+      float ab[32];   // [A (16) | B (16)] of this thread's 16 steps (quasi); B only (Picard)
+      if constexpr (kHasA) {
+        tmem_ld32(sbase, ab);
+      } else {
+        float bb[16];
+        tmem_ld16(sbase, bb);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ab[16 + i] = bb[i];
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_cempty[slot]);
       if (!s_abort) {
         const int tj = (kgj / B) * L + row0;
         float* o = dst + ((size_t)(kgj % B) * T + tj) * D + c;
+        if (tj + 16 <= T) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (tj + i < T) o[(size_t)i * D] = kHasA ? fmaf(aa[i], cp, bb[i]) : cp + bb[i];
+          for (int i = 0; i < 16; ++i) o[(size_t)i * D] = kHasA ? fmaf(ab[i], cp, ab[16 + i]) : cp + ab[16 + i];
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (tj + i < T) o[(size_t)i * D] = kHasA ? fmaf(ab[i], cp, ab[16 + i]) : cp + ab[16 + i];
+        }
       }
     };
 
@@ -484,18 +496,22 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       float z[16];
       tmem_ld16(tmem + (uint32_t)(buf * RS + 16 * rg) + lane_off, z);
       mbar_wait_flag(&bar_xfull, (unsigned)it & 1u, ctrl, tmo, &s_abort);
-      const unsigned char* Sh = sS + (st * NKH + hc) * C::SH_BYTES;
+      // rows row0 .. row0 + 16 of the swizzled stage (row0 is a multiple of 16, so the swizzle
+      // phase of row row0 + i is i mod 8): byte offset = 128 (row0 + i) + (cq ^ (i mod 8)) 16 + (cc mod 4) 4
+      const unsigned char* Sh = sS + (st * NKH + hc) * C::SH_BYTES + row0 * 128 + (cc & 3) * 4;
+      const uint32_t cq16 = (uint32_t)(cc >> 2) << 4;
       // step t0 + row0 - 1; for the first step of a sequence that is s0 (the stage's row 0
       // holds s0 only for the tensor cores)
-      float sp = (t0 + row0 == 0) ? __ldg(A.s0 + (size_t)b * D + c)
-                                  : *reinterpret_cast<const float*>(Sh + sw128_offset(row0, cc));
+      float sp = (t0 + row0 == 0) ? __ldg(A.s0 + (size_t)b * D + c) : *reinterpret_cast<const float*>(Sh + cq16);
+      const bool full = (t0 + row0 + 16 <= T);   // no step of this thread lies past the sequence end
+      const float* xr = sX + row0 * DP + c;
       float SA = 1.0f, SB = 0.0f;
       float av[16], bv[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int r = row0 + i;
-        const float sc = *reinterpret_cast<const float*>(Sh + sw128_offset(r + 1, cc));
-        const float xv = sX[r * DP + c];
+        const float sc = *reinterpret_cast<const float*>(Sh + (i + 1) * 128 + (cq16 ^ (uint32_t)(((i + 1) & 7) << 4)));
+        const float xv = xr[i * DP];
         float y, a, bb, res;
         if constexpr (CELL == PN_CELL_TANH_RNN) {
           y = tanh_pn(z[i] + xv);
@@ -519,7 +535,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
             bb = y;
           }
         }
-        if (t0 + r < T) {
+        if (full || t0 + r < T) {
           rbits = max(rbits, abs_bits(res));
         } else {
           a = 1.0f;
@@ -557,9 +573,6 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         named_barrier(1, NTE);   // the ticket of tile it+1
         kg = s_atk[(it + 1) & 1];
       } else {
-        // the states of tile it-2: its carry had two tiles of time to arrive
-        if (it >= C::DEFER) write_out(it - C::DEFER, kg_m2, pa2, pb2);
-
         // ---- combine the 8 pieces of each channel
         float* tot = sTot + (it & 1) * C::NPC * DP * 2;
         *reinterpret_cast<float2*>(tot + (piece * DP + c) * 2) = make_float2(SA, SB);
@@ -584,11 +597,14 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         }
         // ---- park the in-piece prefixes in TMEM; formed two tiles later
         {
-          const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + 16 * rg) + lane_off;
-          if constexpr (kHasA) tmem_st16(sbase, av);
-          tmem_st16(sbase + (uint32_t)(kHasA ? RS : 0), bv);
+          const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + (kHasA ? 32 : 16) * rg) + lane_off;
+          if constexpr (kHasA) tmem_st32(sbase, av, bv);
+          else tmem_st16(sbase, bv);
           tmem_st_wait();
         }
+        // the states of tile it-2 (its carry had two tiles of time to arrive; this tile's
+        // prefixes are parked, so few registers are live)
+        if (it >= C::DEFER) write_out(it - C::DEFER, kg_m2, pa2, pb2);
         pa2 = pa1;
         pb2 = pb1;
         pa1 = PA;
