@@ -53,7 +53,7 @@ struct pn_ctx {
   float* wt_diag = nullptr;    // [ngroups][DP][R*G] transposed recurrent weights
   float* wt_dense = nullptr;   // [DP][R*DP] transposed + [R][DP][DP] row-major
   float* wt_tc = nullptr;      // [W ; W_lo] rows of W_q, TF32-rounded, K-major core-matrix layout
-  float* wt_tct = nullptr;     // zero-banded [Z; W_hi; Z; W_lo; Z] (one-gate cells), same layout
+  float* wt_tct = nullptr;     // banded [Z; W_hi; Z; W_lo; Z] (one-gate cells; no Z for D = 64), same layout
   float* wdiag = nullptr;      // [R][DP] diagonal entries W_q[c][c]
   float* bhn = nullptr;        // [DP]
   float* proj_w = nullptr;     // U [D][d_in] or W_ih [3D][d_in]
@@ -684,19 +684,20 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
           wtc[off] = hi;
           wtc[(size_t)NN * DP + off] = lo;
         }
-    // channel-major tensor-core operand (one-gate cells, D == DP): rows of the zero-banded
-    // buffer [Z(128-D); W_hi; Z(128-D); W_lo; Z(128-D)], K = DP, K-major core-matrix layout
+    // channel-major tensor-core operand (one-gate cells, D == DP): rows of the banded
+    // buffer [Z(64-D); W_hi; Z(64-D); W_lo; Z(64-D)] (no zero rows for D = 64), K = DP,
+    // K-major core-matrix layout; the kernel reads 64-row windows of it
     std::vector<float> wtct;
     if (h->tc_capable && cell != PN_CELL_GRU) {
-      const int rows = 384 - DP;
+      const int rows = 192 - DP;
       wtct.assign((size_t)rows * DP, 0.0f);
       for (int j = 0; j < D; ++j)
         for (int k = 0; k < D; ++k) {
           const float w = w_block(h, params, 0, j, k);
           const float hi = tf32_round(w);
           const float lo = tf32_round(w - hi);
-          wtct[kmajor_offset((128 - DP) + j, k, DP) / 4] = hi;
-          wtct[kmajor_offset((256 - DP) + j, k, DP) / 4] = lo;
+          wtct[kmajor_offset((64 - DP) + j, k, DP) / 4] = hi;
+          wtct[kmajor_offset((128 - DP) + j, k, DP) / 4] = lo;
         }
     }
     std::vector<float> wdg((size_t)R * DP, 0.0f);
@@ -889,8 +890,9 @@ pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* a
     if (last > INT_MAX) return fail(h, PN_ERR_INVALID, "n_launches too large");
     h->args_h->tol = -1.0f;
     h->args_h->max_iters = (int)last;
-    const int running[2] = {kRunning, 0};   // ctrl->status, ctrl->error
-    PN_CUDA(h, cudaMemcpy(&h->ctrl->status, running, sizeof running, cudaMemcpyHostToDevice));
+    const int running = kRunning, no_error = 0;
+    PN_CUDA(h, cudaMemcpy(&h->ctrl->status, &running, sizeof running, cudaMemcpyHostToDevice));
+    PN_CUDA(h, cudaMemcpy(&h->ctrl->error, &no_error, sizeof no_error, cudaMemcpyHostToDevice));
   } else {
     h->args_h->tol = INFINITY;
     h->args_h->max_iters = INT_MAX;

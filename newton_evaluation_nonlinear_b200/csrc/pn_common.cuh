@@ -21,19 +21,22 @@ constexpr int kTcMaps = 5;             // TMA tensor maps of the tensor-core ker
 
 // Device control block: one per handle, in device memory.
 struct Ctrl {
+  // read at launch or iteration start, written by one thread
   int iter;            // index i of the iterate s^(i) the next launch evaluates
   int status;          // kRunning, or the final pn_status of the loop
-  int error;           // sticky device error (PN_ERR_TIMEOUT), 0 if none
   int final_iter;      // iteration count of the result
   float final_resid;   // r^(final_iter)
-  unsigned resid_bits; // running max of |F| for the current launch (float bits)
-  unsigned ticket[kMaxGroups];  // tile tickets handed out per channel group, current launch
-  unsigned done;       // CTAs finished in the current launch
   unsigned epoch;      // launch sequence number; tags the look-back flags
   int timeout_ticket;  // ticket whose wait gave up (diagnostics), -1 if none
   unsigned long long t_start;    // min %globaltimer at CTA entry, current launch
   unsigned long long kernel_ns;  // summed launch durations
   unsigned long long launches;   // iterations run by the fused iteration kernels
+  // The words below are hot and each sits in a 128-byte line of its own, so that
+  // the ticket atomics do not queue behind the polls of the error word.
+  alignas(128) int error;        // sticky device error (PN_ERR_TIMEOUT), 0 if none; polled by waiting warps
+  alignas(128) unsigned ticket[kMaxGroups];  // tile tickets handed out per channel group, current launch
+  alignas(128) unsigned resid_bits;  // running max of |F| for the current launch (float bits)
+  unsigned done;       // CTAs finished in the current launch
   unsigned gen;        // grid-barrier generation of the looping kernels (iterations completed)
 };
 

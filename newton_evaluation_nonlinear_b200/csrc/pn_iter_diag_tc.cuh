@@ -212,8 +212,12 @@ __device__ __forceinline__ bool mbar_wait_flag(uint64_t* bar, unsigned parity, C
   unsigned spins = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (((++spins) & 15u) == 0u) {
-      if (*abort || ld_volatile(&ctrl->error)) {
+    ++spins;
+    // the CTA's own abort flag (shared memory) often; the grid's error word and the clock
+    // rarely: thousands of waiting warps polling one global word make its L2 slice a hot spot
+    if ((spins & 15u) == 0u && *abort) return false;
+    if ((spins & 255u) == 0u) {
+      if (ld_volatile(&ctrl->error)) {
         *abort = 1;
         return false;
       }

@@ -6,15 +6,19 @@
 // Newton methods..." page §1.2, with a diagonal A~_t, §2.2.1 / §2.2.3, solved
 // by the chunked scan of §2.1), with the roles of the two MMA operands
 // swapped: Z = W S^T, so a TMEM lane holds one channel and its columns hold
-// consecutive steps.  The 128 lanes hold 128 / D step segments side by side:
-// lane g D + c is channel c of steps t0 + g RS .. t0 + (g+1) RS - 1
-// (RS = D L / 128).  Segment g's MMA reads its steps of S as the B operand and
-// a window of a zero-banded copy of W as the A operand, whose nonzero rows are
-// exactly lanes g D .. g D + D - 1; the accumulations of all segments land in
-// one 128-lane accumulator.  Products are 3xTF32 as in the row-major kernel:
-// S_hi W_hi + S_hi W_lo + S_lo W_hi, with S_hi the tensor core's truncation.
+// consecutive steps.  The MMAs are M = 64: an M = 64 accumulator takes 16
+// lanes of each 32-lane quarter (row m at lane 32 (m / 16) + m mod 16), and a
+// second one sits beside it at lane offset 16, so the 128 lanes hold two
+// halves.  Each half holds 64 / D bands of D channels, and each (half, band)
+// pair is one step segment: RS = D L / 128 consecutive steps of all D
+// channels.  Segment (h, j)'s MMA reads its steps of S as the B operand and a
+// 64-row window of a banded copy of W as the A operand, whose nonzero rows are
+// exactly band j (for D = 64 the window is W itself, with no zero rows).
+// Products are 3xTF32 as in the row-major kernel: S_hi W_hi + S_hi W_lo +
+// S_lo W_hi, with S_hi the tensor core's truncation.
 //
-// Each epilogue thread owns one lane (channel c of one segment) and 16
+// Each epilogue thread owns one lane (channel c of one segment: the two lane
+// halves of a warp hold two different segments) and 16
 // consecutive steps: it evaluates the cell, the Jacobian diagonal and the
 // residual, and scans those steps sequentially in registers -- no shuffles.
 // The 8 sixteen-step pieces of a channel are combined through shared memory;
@@ -28,6 +32,9 @@
 // arrival applies the stop rule, then the next iteration starts with the
 // weights, TMEM and barrier memory of the CTA kept (no launch gap, no set-up).
 //
+// The step inputs are double-buffered with the S stages and released with
+// them, so both are fetched two tiles ahead of their use.
+//
 // Warp roles (one CTA per SM): 0 producer (tickets, TMA loads); 1 MMA issuer;
 // 2-3 look-back (scan modes, alternate tiles); the rest epilogue (4 TMEM lane
 // quarters x RS / 16 step groups).  The epilogue forms the next tile's S_lo
@@ -39,6 +46,71 @@
 
 namespace pn {
 
+// The carry into tile k: the published state n_agg + 1 places back (unless
+// `from_s0`: the chain starts at s0, which the caller put in `carry`) folded
+// with the aggregates n_agg .. 1 places back, oldest first.  Each round trip
+// loads up to FB aggregates, the first one the state as well; a round spins
+// (bounded) until all its words carry `tag`.  Returns false when a wait gave up.
+template <int DP, int NQ, int FB>
+__device__ __forceinline__ bool lookback_fold(const unsigned long long* aggw, const unsigned long long* prefw, size_t k,
+                                              size_t stride, int n_agg, bool from_s0, unsigned tag, float (&carry)[NQ],
+                                              Ctrl* ctrl, long long timeout_ns) {
+  const int lane = threadIdx.x & 31;
+  bool need_state = !from_s0;
+  const unsigned long long* src = prefw + (k - (size_t)(n_agg + 1) * stride) * DP;
+  for (int d0 = n_agg; need_state || d0 >= 1; d0 -= FB) {
+    unsigned long long ws[NQ], wa[FB][NQ], wb[FB][NQ];
+    unsigned long long t0 = 0;
+    unsigned spins = 0;
+    while (true) {
+      bool ok = true;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int j = lane + 32 * q;
+        ws[q] = (need_state && j < DP) ? ld_word(src + j) : tag_word(0.0f, tag);
+#pragma unroll
+        for (int u = 0; u < FB; ++u) {
+          const int d = d0 - u;
+          wa[u][q] = tag_word(1.0f, tag);
+          wb[u][q] = tag_word(0.0f, tag);
+          if (d >= 1 && j < DP) ld_word2(aggw + ((k - (size_t)d * stride) * DP + j) * 2, wa[u][q], wb[u][q]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        ok = ok && word_tagged(ws[q], tag);
+#pragma unroll
+        for (int u = 0; u < FB; ++u) ok = ok && word_tagged(wa[u][q], tag) && word_tagged(wb[u][q], tag);
+      }
+      if (__all_sync(0xffffffffu, ok)) break;
+      if (spins == 0) t0 = globaltimer();
+      if (spin_give_up(spins, t0, ctrl, timeout_ns)) return false;
+    }
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      if (need_state) carry[q] = word_value(ws[q]);
+#pragma unroll
+      for (int u = 0; u < FB; ++u) carry[q] = fmaf(word_value(wa[u][q]), carry[q], word_value(wb[u][q]));
+    }
+    need_state = false;
+  }
+  return true;
+}
+
+// 32 TMEM columns of this warp's lanes from a[16], b[16] in the order
+// [a 0-7 | b 0-7 | a 8-15 | b 8-15], so that each half can be read back alone.
+__device__ __forceinline__ void tmem_st32_split8(uint32_t taddr, const float (&a)[16], const float (&b)[16]) {
+  float lo[16], hi[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    lo[i] = a[i];
+    lo[8 + i] = b[i];
+    hi[i] = a[8 + i];
+    hi[8 + i] = b[8 + i];
+  }
+  tmem_st32(taddr, lo, hi);
+}
+
 template <int CELL, int MODE, int DP>
 struct DiagTctCfg {
   static_assert(CELL != PN_CELL_GRU, "one-gate cells only");
@@ -46,16 +118,21 @@ struct DiagTctCfg {
   static constexpr bool kScan = (MODE != PN_JACOBI);
   static constexpr int L = 128;                  // steps per tile
   static constexpr int K = DP;                   // MMA K (input channels)
-  static constexpr int NSEG = 128 / DP;          // step segments side by side on the TMEM lanes
+  static constexpr int MT = 64;                  // MMA M: one accumulator half (16 lanes of each lane quarter)
+  static constexpr int NB = MT / DP;             // channel bands per accumulator half (1 for D = 64, 2 for D = 32)
+  static constexpr int NSEG = 2 * NB;            // step segments: 2 halves x NB bands = 128 / D
   static constexpr int RS = L / NSEG;            // steps per segment = MMA N
   static constexpr int NRG = RS / 16;            // 16-step groups per segment
   static constexpr int NPC = NSEG * NRG;         // pieces per channel (L / 16)
   static constexpr int NKH = DP / 32;            // 32-float column halves of S
   static constexpr int SCOLS = (MODE == PN_QUASI ? 2 : 1) * RS;   // stash columns per tile: per 16-step
                                                                      // group, [A (16) |] B (16)
-  static constexpr int NSLOT = 3;                // tiles between their scan and their write-out, + 1
-  static constexpr int DEFER = NSLOT - 1;
+  static constexpr int NSLOT = 3;                // TMEM stash slots (and look-back carry slots)
+  static constexpr int DEFER = NSLOT;            // a tile's states are formed 3 tiles later, just before
+                                                 // that tile's prefixes take over its stash slot
+  static constexpr int NAG = NSLOT + 1;          // slots of the aggregate hand-off to the look-back
   static constexpr int NLB = kScan ? 2 : 0;      // look-back warps, alternating tiles
+  static constexpr int FB = 6;                   // aggregates per look-back round trip
   static constexpr int STASH0 = 2 * RS;          // accumulators: 2 x RS columns
   static constexpr int USED_COLS = STASH0 + (kScan ? NSLOT * SCOLS : 0);
   static constexpr int ALLOC_COLS =
@@ -64,8 +141,9 @@ struct DiagTctCfg {
   static constexpr int NTE = 32 * NEW;
   static constexpr int WE0 = 2 + NLB;            // first epilogue warp
   static constexpr int NT = 32 * (WE0 + NEW);
-  static constexpr int NQ = DP / 32;             // channels per look-back lane; warps holding the last piece
-  static constexpr int WROWS = 384 - DP;         // banded W: Z(128-D) W_hi Z(128-D) W_lo Z(128-D)
+  static constexpr int NQ = DP / 32;             // channels per look-back lane
+  static constexpr int NLASTW = 4 / NB;          // epilogue warps holding the last piece of a channel
+  static constexpr int WROWS = 3 * MT - DP;      // banded W: Z(64-D) W_hi Z(64-D) W_lo Z(64-D)
   static constexpr int align(int v, int a) { return (v + a - 1) / a * a; }
   static constexpr int SH_LOAD = (L + 1) * 128;
   static constexpr int SH_BYTES = align(SH_LOAD, 1024);
@@ -75,18 +153,18 @@ struct DiagTctCfg {
   static constexpr uint32_t SBO_W = (K / 4) * 128;
   static constexpr int OFF_S = 0;                                 // [2 stages][NKH][SH_BYTES]
   static constexpr int OFF_LO = OFF_S + 2 * NKH * SH_BYTES;       // [NKH][LO_BYTES]
-  static constexpr int OFF_X = OFF_LO + NKH * LO_BYTES;           // [L][DP]
-  static constexpr int OFF_W = align(OFF_X + X_BYTES, 128);
+  static constexpr int OFF_X = OFF_LO + NKH * LO_BYTES;           // [2 stages][L][DP]
+  static constexpr int OFF_W = align(OFF_X + 2 * X_BYTES, 128);
   static constexpr int OFF_WD = OFF_W + W_BYTES;                  // DP floats
   static constexpr int OFF_TOT = OFF_WD + DP * 4;                 // [2][NPC][DP] float2
-  static constexpr int OFF_AGG = OFF_TOT + 2 * NPC * DP * 8;      // [NSLOT][DP] float2
-  static constexpr int OFF_CARRY = OFF_AGG + NSLOT * DP * 8;      // [NSLOT][DP]
+  static constexpr int OFF_AGG = OFF_TOT + 2 * NPC * DP * 8;      // [NAG][DP] float2
+  static constexpr int OFF_CARRY = OFF_AGG + NAG * DP * 8;        // [NSLOT][DP]
   static constexpr int OFF_RED = OFF_CARRY + NSLOT * DP * 4;      // NT/32 floats
   static constexpr int SMEM_USED = OFF_RED + (NT / 32) * 4;
   static constexpr int SMEM_BYTES = SMEM_USED + 1024;             // + slack to align the base to 1024 bytes
-  // first row of segment g's window of the banded W (hi: W_hi at window rows g D .. g D + D - 1)
-  static constexpr int win_hi(int g) { return (128 - DP) - g * DP; }
-  static constexpr int win_lo(int g) { return (256 - DP) - g * DP; }
+  // first row of band j's 64-row window of the banded W (W_hi or W_lo at window rows j D .. j D + D - 1)
+  static constexpr int win_hi(int j) { return (MT - DP) - j * DP; }
+  static constexpr int win_lo(int j) { return (2 * MT - DP) - j * DP; }
   static_assert(USED_COLS <= 512, "TMEM columns");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -115,11 +193,11 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   float* sCarry = reinterpret_cast<float*>(smem_raw + C::OFF_CARRY);
   float* sRed = reinterpret_cast<float*>(smem_raw + C::OFF_RED);
 
-  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull, bar_xempty, bar_afull, bar_mma[2],
-      bar_tempty[2], bar_lb[NSLOT], bar_cfull[NSLOT], bar_cempty[NSLOT];
+  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull[2], bar_afull, bar_mma[2],
+      bar_tempty[2], bar_lb[C::NAG], bar_cfull[NSLOT], bar_cempty[NSLOT];
   __shared__ int s_tk[2];        // ticket staged in s stage 0/1 (-1: no more tiles)
   __shared__ int s_atk[2];       // ticket of tile i's operands, by the parity of i (-1: stop)
-  __shared__ int s_lbtk[NSLOT];  // ticket handed to the look-back per slot (-1: stop)
+  __shared__ int s_lbtk[C::NAG];  // ticket handed to the look-back per slot (-1: stop)
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ int s_last;
@@ -136,26 +214,25 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   auto init_barriers = [&]() {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_sfull[s], 1u);
+      mbar_init(&bar_xfull[s], 1u);
       mbar_init(&bar_sempty[s], (unsigned)C::NEW);
       mbar_init(&bar_mma[s], 1u);
       mbar_init(&bar_tempty[s], (unsigned)C::NEW);
     }
+    for (int s = 0; s < C::NAG; ++s) mbar_init(&bar_lb[s], (unsigned)C::NLASTW);
     for (int s = 0; s < NSLOT; ++s) {
-      mbar_init(&bar_lb[s], (unsigned)C::NQ);
       mbar_init(&bar_cfull[s], 1u);
       mbar_init(&bar_cempty[s], (unsigned)C::NEW);
     }
-    mbar_init(&bar_xfull, 1u);
-    mbar_init(&bar_xempty, (unsigned)C::NEW);
     mbar_init(&bar_afull, (unsigned)C::NEW);
     mbar_init_fence();
   };
   auto inval_barriers = [&]() {
     uint64_t* bars[] = {&bar_sfull[0], &bar_sfull[1], &bar_sempty[0], &bar_sempty[1], &bar_mma[0], &bar_mma[1],
-                        &bar_tempty[0], &bar_tempty[1], &bar_xfull, &bar_xempty, &bar_afull};
+                        &bar_tempty[0], &bar_tempty[1], &bar_xfull[0], &bar_xfull[1], &bar_afull};
     for (uint64_t* bb : bars) mbar_inval(bb);
+    for (int s = 0; s < C::NAG; ++s) mbar_inval(&bar_lb[s]);
     for (int s = 0; s < NSLOT; ++s) {
-      mbar_inval(&bar_lb[s]);
       mbar_inval(&bar_cfull[s]);
       mbar_inval(&bar_cempty[s]);
     }
@@ -186,8 +263,8 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       mbar_arrive_expect_tx(&bar_sfull[0], (unsigned)(NKH * C::SH_LOAD));
 #pragma unroll
       for (int h = 0; h < NKH; ++h) tma_load_3d(sS + h * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[0]);
-      mbar_arrive_expect_tx(&bar_xfull, (unsigned)C::X_BYTES);
-      tma_load_3d(smem_raw + C::OFF_X, tm_x, 0, t0, b, &bar_xfull);
+      mbar_arrive_expect_tx(&bar_xfull[0], (unsigned)C::X_BYTES);
+      tma_load_3d(smem_raw + C::OFF_X, tm_x, 0, t0, b, &bar_xfull[0]);
     } else {
       s_tk[0] = -1;
       mbar_arrive(&bar_sfull[0]);
@@ -201,8 +278,8 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     const float4* w4 = reinterpret_cast<const float4*>(P.wt);
     float4* d4 = reinterpret_cast<float4*>(sW);
     constexpr int ROW16 = DP / 4;                 // float4s per row of the K-major layout (on average)
-    constexpr int HI0 = (128 - DP) * ROW16, HI1 = 128 * ROW16;            // W_hi rows, in float4 units
-    constexpr int LO0 = (256 - DP) * ROW16, LO1 = 256 * ROW16;            // W_lo rows
+    constexpr int HI0 = (C::MT - DP) * ROW16, HI1 = C::MT * ROW16;            // W_hi rows, in float4 units
+    constexpr int LO0 = (2 * C::MT - DP) * ROW16, LO1 = 2 * C::MT * ROW16;    // W_lo rows
     for (int e = tid; e < C::W_BYTES / 16; e += C::NT) {
       const bool wrow = (e >= HI0 && e < HI1) || (e >= LO0 && e < LO1);
       d4[e] = wrow ? __ldg(w4 + e) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -230,9 +307,11 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     // tile 0 was issued before the block-wide sync (static ticket blockIdx.x)
     const bool none = (int)blockIdx.x >= P.tiles_per_group;
     int it = 1;
-    int x_issued = none ? 0 : 1;
+    int n_loaded = none ? 0 : 1;   // tiles whose S and x loads were issued
     for (; !none; ++it) {
       const int st = it & 1;
+      // stage st (S and step inputs) is free once tile it-2's cell phase is done; the ticket
+      // is claimed only then, so a CTA holds no ticket it cannot start loading
       if (it >= 2 && !mbar_wait_flag(&bar_sempty[st], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
       int kg = 0;
       if (lane == 0) kg = (int)(gridDim.x + atomicAdd(&ctrl->ticket[0], 1u));
@@ -253,59 +332,84 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         mbar_arrive_expect_tx(&bar_sfull[st], (unsigned)(NKH * C::SH_LOAD));
 #pragma unroll
         for (int h = 0; h < NKH; ++h) tma_load_3d(sS + (st * NKH + h) * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[st]);
-      }
-      // the single step-input buffer: wait until the previous tile's inputs were consumed
-      if (it >= 1 && !mbar_wait_flag(&bar_xempty, ((unsigned)(it - 1)) & 1u, ctrl, tmo, &s_abort)) {
-        ++it;
-        break;
-      }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bar_xfull, (unsigned)C::X_BYTES);
-        tma_load_3d(smem_raw + C::OFF_X, tm_x, 0, t0, b, &bar_xfull);
+        mbar_arrive_expect_tx(&bar_xfull[st], (unsigned)C::X_BYTES);
+        tma_load_3d(smem_raw + C::OFF_X + st * C::X_BYTES, tm_x, 0, t0, b, &bar_xfull[st]);
       }
       __syncwarp();
-      x_issued = it + 1;
+      n_loaded = it + 1;
     }
+    // the last two stages' loads (and the stop marker) complete before the CTA moves on
     for (int j = max(0, it - 2); j < it; ++j)
       if (!mbar_drain(&bar_sfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
         atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
-    if (x_issued > 0 && !mbar_drain(&bar_xfull, ((unsigned)(x_issued - 1)) & 1u, tmo) && lane == 0)
-      atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+    for (int j = max(0, n_loaded - 2); j < n_loaded; ++j)
+      if (!mbar_drain(&bar_xfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
+        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
   } else if (warp == 1) {
     // =========================== MMA issuer =================================
-    constexpr uint32_t idesc = umma_idesc_tf32(128, RS);
+    constexpr uint32_t idesc = umma_idesc_tf32(C::MT, RS);
     // Descriptors differ between MMAs only in the start address (bits 0-13, address >> 4;
     // shared addresses stay below 2^18 so the field never carries): precompute the bases
     // and add compile-time offsets in the fully unrolled issue loop.
     const uint64_t a_base = umma_smem_desc(smem_addr(sW), 128, C::SBO_W, 0);
     const uint64_t b_base0 = umma_smem_desc(smem_addr(sS), 16, 1024, 2);
     const uint64_t b_lo = umma_smem_desc(smem_addr(sLo), 16, 1024, 2);
-    int issued = 0;
-    for (int it = 0;; ++it) {
-      if (!mbar_wait_flag(&bar_afull, (unsigned)it & 1u, ctrl, tmo, &s_abort)) break;
-      if (s_atk[it & 1] < 0) break;
+    // products of stage `it` for passes p0 .. p1-1 (pass 0: W_hi S_hi, 1: W_lo S_hi, 2: W_hi S_lo)
+    auto issue = [&](int it, int p0, int p1) {
       const int buf = it & 1;
-      if (it >= 2 && !mbar_wait_flag(&bar_tempty[buf], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t d = tmem + (uint32_t)(buf * RS);
-        const uint64_t b_hi = b_base0 + (uint64_t)(((it & 1) * NKH * C::SH_BYTES) >> 4);
+      const uint32_t d = tmem + (uint32_t)(buf * RS);
+      const uint64_t b_hi = b_base0 + (uint64_t)(((it & 1) * NKH * C::SH_BYTES) >> 4);
 #pragma unroll
-        for (int pass = 0; pass < 3; ++pass) {
-          // pass 0: W_hi S_hi, pass 1: W_lo S_hi, pass 2: W_hi S_lo
+      for (int pass = 0; pass < 3; ++pass) {
+        if (pass < p0 || pass >= p1) continue;
 #pragma unroll
-          for (int kb = 0; kb < K / 8; ++kb) {
-            const int h = kb >> 2;   // column half of S; 4 K-steps of 32 bytes per 128-byte swizzled row
+        for (int kb = 0; kb < K / 8; ++kb) {
+          const int h = kb >> 2;   // column half of S; 4 K-steps of 32 bytes per 128-byte swizzled row
 #pragma unroll
-            for (int g = 0; g < C::NSEG; ++g) {
-              const int ws = (pass == 1) ? C::win_lo(g) : C::win_hi(g);
-              const uint64_t ad = a_base + (uint64_t)(((ws / 8) * C::SBO_W + kb * 256) >> 4);
-              const uint64_t bd = (pass == 2 ? b_lo + (uint64_t)((h * C::LO_BYTES + g * RS * 128 + (kb & 3) * 32) >> 4)
-                                             : b_hi + (uint64_t)((h * C::SH_BYTES + g * RS * 128 + (kb & 3) * 32) >> 4));
-              umma_tf32(d, ad, bd, idesc, (pass | kb | g) ? 1u : 0u);
-            }
+          for (int g = 0; g < C::NSEG; ++g) {
+            // segment g = accumulator half g / NB (lane offset 16), band g % NB; the first
+            // product of each half overwrites it (its other bands receive zeros)
+            const int band = g % C::NB;
+            const int ws = (pass == 1) ? C::win_lo(band) : C::win_hi(band);
+            const uint64_t ad = a_base + (uint64_t)(((ws / 8) * C::SBO_W + kb * 256) >> 4);
+            const uint64_t bd = (pass == 2 ? b_lo + (uint64_t)((h * C::LO_BYTES + g * RS * 128 + (kb & 3) * 32) >> 4)
+                                           : b_hi + (uint64_t)((h * C::SH_BYTES + g * RS * 128 + (kb & 3) * 32) >> 4));
+            umma_tf32(d + ((uint32_t)(16 * (g / C::NB)) << 16), ad, bd, idesc, (pass | kb | band) ? 1u : 0u);
           }
         }
+      }
+    };
+    // The two S_hi passes need only the loaded stage (the tensor core truncates S itself), so
+    // they are issued as soon as it lands and run under the epilogue's cell phase of the
+    // previous tile; only the S_lo pass waits for the split.  A sequence's first chunk is the
+    // exception: its row 0 (step -1) becomes s0 in the split, so all its passes wait.
+    int issued = 0;
+    for (int it = 0;; ++it) {
+      const int buf = it & 1;
+      if (!mbar_wait_flag(&bar_sfull[it & 1], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort)) break;
+      const int kn = s_tk[it & 1];
+      bool early = false;
+      if (kn >= 0 && kn / B != 0) {
+        if (it >= 2 && !mbar_wait_flag(&bar_tempty[buf], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
+        tc_fence_after();
+        if (lane == 0) issue(it, 0, 2);
+        __syncwarp();
+        early = true;
+      }
+      const bool ok = mbar_wait_flag(&bar_afull, (unsigned)it & 1u, ctrl, tmo, &s_abort);
+      if (!ok || s_atk[it & 1] < 0) {
+        if (early) {   // let the issued products complete before the accumulator is released
+          if (lane == 0) umma_commit(&bar_mma[buf]);
+          __syncwarp();
+          issued = it + 1;
+        }
+        break;
+      }
+      if (!early && it >= 2 && !mbar_wait_flag(&bar_tempty[buf], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort))
+        break;
+      tc_fence_after();
+      if (lane == 0) {
+        issue(it, early ? 2 : 0, 3);
         umma_commit(&bar_mma[buf]);
       }
       __syncwarp();
@@ -322,10 +426,11 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       unsigned long long* prefw = reinterpret_cast<unsigned long long*>(P.pref);  // [tile][DP]
       const unsigned tag = lookback_tag(epoch);
       for (int it = warp - 2;; it += C::NLB) {
-        const int slot = it % NSLOT;
+        const int aslot = it % C::NAG;   // aggregate hand-off slot
+        const int slot = it % NSLOT;     // carry slot
         const unsigned ph = (unsigned)(it / NSLOT) & 1u;
-        if (!mbar_wait_flag(&bar_lb[slot], ph, ctrl, tmo, &s_abort)) break;
-        const int kg = s_lbtk[slot];
+        if (!mbar_wait_flag(&bar_lb[aslot], (unsigned)(it / C::NAG) & 1u, ctrl, tmo, &s_abort)) break;
+        const int kg = s_lbtk[aslot];
         if (kg < 0) break;
         const int b = kg % B;
         const int chunk = kg / B;
@@ -334,7 +439,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         float2 ag[C::NQ];
 #pragma unroll
         for (int q = 0; q < C::NQ; ++q)
-          ag[q] = *reinterpret_cast<const float2*>(sAgg + (slot * DP + lane + 32 * q) * 2);
+          ag[q] = *reinterpret_cast<const float2*>(sAgg + (aslot * DP + lane + 32 * q) * 2);
         // 1. the tile aggregate (the first chunk too: a successor may start from s0)
         if (!stall) {
 #pragma unroll
@@ -349,29 +454,15 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
 #pragma unroll
         for (int q = 0; q < C::NQ; ++q) carry[q] = 0.0f;
         if (n_agg >= 0) {
-          if (chunk - 1 - n_agg >= 0) {
-            if (!ld_tagged_state<DP, C::NQ>(prefw + (k - (size_t)(n_agg + 1) * stride) * DP, tag, carry, ctrl, tmo))
-              n_agg = -1;
-          } else {
+          const bool from_s0 = chunk - 1 - n_agg < 0;
+          if (from_s0) {
 #pragma unroll
             for (int q = 0; q < C::NQ; ++q) {
               const int j = lane + 32 * q;
               carry[q] = (j < D) ? __ldg(A.s0 + (size_t)b * D + j) : 0.0f;
             }
           }
-        }
-        for (int d0 = n_agg; d0 >= 1; d0 -= 4) {   // oldest aggregate first, four loads in flight
-          float fa[4][C::NQ], fb[4][C::NQ];
-          if (!ld_tagged_aggs<DP, C::NQ>(aggw, k, stride, d0, tag, fa, fb, ctrl, tmo)) {
-            n_agg = -1;
-            break;
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (d0 - u >= 1) {
-#pragma unroll
-              for (int q = 0; q < C::NQ; ++q) carry[q] = fmaf(fa[u][q], carry[q], fb[u][q]);
-            }
+          if (!lookback_fold<DP, C::NQ, C::FB>(aggw, prefw, k, stride, n_agg, from_s0, tag, carry, ctrl, tmo)) n_agg = -1;
         }
         if (n_agg < 0) s_abort = 1;
         // 3. hand the carry to the epilogue (its slot is free once tile it - NSLOT was formed)
@@ -395,11 +486,15 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     const int e = warp - C::WE0;            // 0 .. NEW-1
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int rg = e >> 2;                  // 16-step group within the segment
-    const int ln = quarter * 32 + lane;     // TMEM lane = g * DP + c
-    const int g = ln / DP;                  // step segment (warp-uniform)
-    const int c = ln % DP;                  // channel
+    // TMEM lane quarter * 32 + lane = row m of accumulator half `half`
+    const int m = 16 * quarter + (lane & 15);
+    const int half = lane >> 4;
+    const int c = m % DP;                   // channel
+    const int g = half * C::NB + m / DP;    // step segment (differs between the lane halves)
     const int row0 = g * RS + 16 * rg;      // first step (tile row) of this thread
-    const int piece = g * C::NRG + rg;      // warp-uniform
+    const int piece = g * C::NRG + rg;
+    // the warps holding the last piece (last step group of the last band of half 1)
+    const bool lastw = (rg == C::NRG - 1) && ((16 * quarter) / DP == C::NB - 1);
     const int te = tid - 32 * C::WE0;       // 0 .. NTE-1 among the epilogue threads
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int hc = c >> 5;                  // column half of channel c in S
@@ -409,23 +504,28 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     // S_lo of stage `stg` (rows 0..L-1), swizzled like S.  For the first chunk of a
     // sequence, row 0 (step -1, loaded as zero) becomes s0 first.
     auto split = [&](int stg, int kgs) {
+      constexpr int NU = NKH * L * 8 / NTE;   // 16-byte chunks per thread
+      static_assert(NU * NTE == NKH * L * 8, "split covers the stage exactly");
       const bool first = (kgs / B) == 0;
-      const float* s0row = A.s0 + (size_t)(kgs % B) * D;
-      for (int u = te; u < NKH * L * 8; u += NTE) {
-        const int q = u & 7;
+      float4 v[NU];
+#pragma unroll
+      for (int k = 0; k < NU; ++k) {   // all loads first
+        const int u = te + k * NTE;
+        const int h = (u >> 3) / L;
+        v[k] = *reinterpret_cast<const float4*>(sS + (stg * NKH + h) * C::SH_BYTES + sw128_offset((u >> 3) % L, 4 * (u & 7)));
+      }
+#pragma unroll
+      for (int k = 0; k < NU; ++k) {
+        const int u = te + k * NTE;
         const int r = (u >> 3) % L;
         const int h = (u >> 3) / L;
-        const uint32_t off = sw128_offset(r, 4 * q);
-        unsigned char* srow = sS + (stg * NKH + h) * C::SH_BYTES;
-        float4 v;
+        const uint32_t off = sw128_offset(r, 4 * (u & 7));
         if (first && r == 0) {
-          v = __ldg(reinterpret_cast<const float4*>(s0row + 32 * h) + q);
-          *reinterpret_cast<float4*>(srow + off) = v;
-        } else {
-          v = *reinterpret_cast<const float4*>(srow + off);
+          v[k] = __ldg(reinterpret_cast<const float4*>(A.s0 + (size_t)(kgs % B) * D + 32 * h) + (u & 7));
+          *reinterpret_cast<float4*>(sS + (stg * NKH + h) * C::SH_BYTES + off) = v[k];
         }
         *reinterpret_cast<float4*>(sLo + h * C::LO_BYTES + off) =
-            make_float4(tf32_tail(v.x), tf32_tail(v.y), tf32_tail(v.z), tf32_tail(v.w));
+            make_float4(tf32_tail(v[k].x), tf32_tail(v[k].y), tf32_tail(v[k].z), tf32_tail(v[k].w));
       }
       fence_async_smem();   // generic writes -> the tensor cores (async proxy)
     };
@@ -444,34 +544,34 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       }
     };
 
-    // s^(i+1) of tile j (ticket kgj): piece carry from the look-back carry, then the parked prefixes
+    // s^(i+1) of tile j (ticket kgj): piece carry from the look-back carry, then the parked
+    // prefixes (the stash holds [A 0-7 | B 0-7 | A 8-15 | B 8-15] per 16 steps; B only for Picard)
     auto write_out = [&](int j, int kgj, float pa, float pb) {
       const int slot = j % NSLOT;
       mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort);
       const float carry = sCarry[slot * DP + c];
       const float cp = kHasA ? fmaf(pa, carry, pb) : carry + pb;
       const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + (kHasA ? 32 : 16) * rg) + lane_off;
-      float ab[32];   // [A (16) | B (16)] of this thread's 16 steps (quasi); B only (Picard)
+      float v[32];
       if constexpr (kHasA) {
-        tmem_ld32(sbase, ab);
+        tmem_ld32(sbase, v);
       } else {
         float bb[16];
         tmem_ld16(sbase, bb);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) ab[16 + i] = bb[i];
+        for (int i = 0; i < 16; ++i) v[i] = bb[i];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_cempty[slot]);
       if (!s_abort) {
         const int tj = (kgj / B) * L + row0;
         float* o = dst + ((size_t)(kgj % B) * T + tj) * D + c;
-        if (tj + 16 <= T) {
+        const bool whole = (tj + 16 <= T);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) o[(size_t)i * D] = kHasA ? fmaf(ab[i], cp, ab[16 + i]) : cp + ab[16 + i];
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (tj + i < T) o[(size_t)i * D] = kHasA ? fmaf(ab[i], cp, ab[16 + i]) : cp + ab[16 + i];
+        for (int i = 0; i < 16; ++i) {
+          const int q = (i & 8) * 2 + (i & 7);   // A of step i at column q, its B at q + 8
+          const float sv = kHasA ? fmaf(v[q], cp, v[q + 8]) : cp + v[i];
+          if (whole || tj + i < T) o[(size_t)i * D] = sv;
         }
       }
     };
@@ -482,20 +582,26 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     named_barrier(1, NTE);
     int kg = s_atk[0];
     int it = 0;
-    int kg_m1 = -1, kg_m2 = -1;              // tickets of tiles it-1, it-2
-    float pa1 = 1.0f, pb1 = 0.0f, pa2 = 1.0f, pb2 = 0.0f;   // their piece prefixes
+    int kg_m1 = -1, kg_m2 = -1, kg_m3 = -1;  // tickets of tiles it-1, it-2, it-3
+    float pa1 = 1.0f, pb1 = 0.0f, pa2 = 1.0f, pb2 = 0.0f, pa3 = 1.0f, pb3 = 0.0f;   // their piece prefixes
     for (; kg >= 0; ++it) {
       const int st = it & 1;
       const int buf = it & 1;
       const int b = kg % B;
       const int t0 = (kg / B) * L;
 
+      // the states of tile it-3 (its carry had nearly three tiles of time to arrive); this
+      // frees the stash slot this tile's prefixes go to, and overlaps the wait for the products
+      if constexpr (kScan) {
+        if (it >= C::DEFER) write_out(it - C::DEFER, kg_m3, pa3, pb3);
+      }
+
       // ---- Z of this thread's channel and 16 steps, then cell + sequential scan
       mbar_wait_flag(&bar_mma[buf], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort);
       tc_fence_after();
       float z[16];
       tmem_ld16(tmem + (uint32_t)(buf * RS + 16 * rg) + lane_off, z);
-      mbar_wait_flag(&bar_xfull, (unsigned)it & 1u, ctrl, tmo, &s_abort);
+      mbar_wait_flag(&bar_xfull[st], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort);
       // rows row0 .. row0 + 16 of the swizzled stage (row0 is a multiple of 16, so the swizzle
       // phase of row row0 + i is i mod 8): byte offset = 128 (row0 + i) + (cq ^ (i mod 8)) 16 + (cc mod 4) 4
       const unsigned char* Sh = sS + (st * NKH + hc) * C::SH_BYTES + row0 * 128 + (cc & 3) * 4;
@@ -504,7 +610,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       // holds s0 only for the tensor cores)
       float sp = (t0 + row0 == 0) ? __ldg(A.s0 + (size_t)b * D + c) : *reinterpret_cast<const float*>(Sh + cq16);
       const bool full = (t0 + row0 + 16 <= T);   // no step of this thread lies past the sequence end
-      const float* xr = sX + row0 * DP + c;
+      const float* xr = sX + st * (L * DP) + row0 * DP + c;
       float SA = 1.0f, SB = 0.0f;
       float av[16], bv[16];
 #pragma unroll
@@ -551,12 +657,11 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         bv[i] = (MODE == PN_JACOBI) ? bb : SB;
         sp = sc;
       }
-      // this tile's TMEM accumulator, step inputs and s stage are consumed
+      // this tile's TMEM accumulator and its stage (S and step inputs) are consumed
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bar_tempty[buf]);
-        mbar_arrive(&bar_xempty);
         mbar_arrive(&bar_sempty[st]);
       }
       // the next tile's operands (S_lo is free: this tile's products are done)
@@ -579,49 +684,58 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         named_barrier(1, NTE);   // piece totals, and the ticket of tile it+1
         const int kg_next = s_atk[(it + 1) & 1];
         float PA = 1.0f, PB = 0.0f;   // prefix of the earlier pieces
-        for (int p = 0; p < piece; ++p) {
-          const float2 w = *reinterpret_cast<const float2*>(tot + (p * DP + c) * 2);
-          PB = kHasA ? fmaf(w.x, PB, w.y) : PB + w.y;
-          if (kHasA) PA *= w.x;
+        {
+          float2 w[C::NPC - 1];   // all loads in flight together
+#pragma unroll
+          for (int p = 0; p < C::NPC - 1; ++p) w[p] = *reinterpret_cast<const float2*>(tot + (p * DP + c) * 2);
+#pragma unroll
+          for (int p = 0; p < C::NPC - 1; ++p)
+            if (p < piece) {
+              PB = kHasA ? fmaf(w[p].x, PB, w[p].y) : PB + w[p].y;
+              if (kHasA) PA *= w[p].x;
+            }
         }
         // the last piece's inclusive prefix is the tile aggregate: hand it to the look-back
-        const int slot = it % NSLOT;
-        if (piece == C::NPC - 1) {
-          *reinterpret_cast<float2*>(sAgg + (slot * DP + c) * 2) =
-              kHasA ? make_float2(SA * PA, fmaf(SA, PB, SB)) : make_float2(1.0f, PB + SB);
+        const int aslot = it % C::NAG;
+        if (lastw) {
+          if (piece == C::NPC - 1)
+            *reinterpret_cast<float2*>(sAgg + (aslot * DP + c) * 2) =
+                kHasA ? make_float2(SA * PA, fmaf(SA, PB, SB)) : make_float2(1.0f, PB + SB);
           __syncwarp();
           if (lane == 0) {
-            if (c == 0) s_lbtk[slot] = s_abort ? -1 : kg;
-            mbar_arrive(&bar_lb[slot]);
+            if (c == 0) s_lbtk[aslot] = s_abort ? -1 : kg;
+            mbar_arrive(&bar_lb[aslot]);
           }
         }
-        // ---- park the in-piece prefixes in TMEM; formed two tiles later
+        // ---- park the in-piece prefixes in TMEM
         {
-          const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + (kHasA ? 32 : 16) * rg) + lane_off;
-          if constexpr (kHasA) tmem_st32(sbase, av, bv);
+          const uint32_t sbase =
+              tmem + (uint32_t)(C::STASH0 + (it % NSLOT) * C::SCOLS + (kHasA ? 32 : 16) * rg) + lane_off;
+          if constexpr (kHasA) tmem_st32_split8(sbase, av, bv);
           else tmem_st16(sbase, bv);
           tmem_st_wait();
         }
-        // the states of tile it-2 (its carry had two tiles of time to arrive; this tile's
-        // prefixes are parked, so few registers are live)
-        if (it >= C::DEFER) write_out(it - C::DEFER, kg_m2, pa2, pb2);
+        pa3 = pa2;
+        pb3 = pb2;
         pa2 = pa1;
         pb2 = pb1;
         pa1 = PA;
         pb1 = PB;
+        kg_m3 = kg_m2;
         kg_m2 = kg_m1;
         kg_m1 = kg;
         kg = kg_next;
       }
     }
     if constexpr (kScan) {
+      if (it >= 3) write_out(it - 3, kg_m3, pa3, pb3);
       if (it >= 2) write_out(it - 2, kg_m2, pa2, pb2);
       if (it >= 1) write_out(it - 1, kg_m1, pa1, pb1);
       // stop the look-back warps: their next tiles are it .. it + NLB - 1
-      if (piece == C::NPC - 1 && lane == 0) {
+      if (lastw && lane == 0) {
         for (int j = it; j < it + C::NLB; ++j) {
-          if (c == 0) s_lbtk[j % NSLOT] = -1;
-          mbar_arrive(&bar_lb[j % NSLOT]);
+          if (c == 0) s_lbtk[j % C::NAG] = -1;
+          mbar_arrive(&bar_lb[j % C::NAG]);
         }
       }
     }
