@@ -37,7 +37,7 @@ struct Ctrl {
   alignas(128) unsigned ticket[kMaxGroups];  // tile tickets handed out per channel group, current launch
   alignas(128) unsigned resid_bits;  // running max of |F| for the current launch (float bits)
   unsigned done;       // CTAs finished in the current launch
-  unsigned gen;        // grid-barrier generation of the looping kernels (iterations completed)
+  unsigned gen;        // grid barrier of the looping kernels: (iterations completed << 1) | (another follows)
 };
 
 // Per-call arguments, written by the host before each evaluation.
@@ -319,14 +319,17 @@ __device__ __forceinline__ void finish_launch(const IterParams& P, const Args& A
   __threadfence();
 }
 
-// Looping kernels (P.persist = 1): every CTA calls this at the end of an
-// iteration, after all of its global writes and with its residual folded into
-// ctrl->resid_bits.  The last CTA to arrive applies the stop rule exactly as
-// finish_launch does and opens the next iteration (generation gen_before + 1);
-// the others wait for it, bounded by the handle's timeout.  Returns, for every
-// thread of the CTA, whether another iteration follows.
-__device__ __forceinline__ bool finish_iteration(const IterParams& P, const Args& A, unsigned epoch,
-                                                 int& flag_smem, unsigned gen_before) {
+// Grid barrier between the iterations of a looping kernel.  Every CTA calls
+// it (all threads) after its part of the iteration, after all of its global
+// writes and with its residual folded into ctrl->resid_bits.  The last CTA to
+// arrive applies the stop rule exactly as finish_launch does (iteration `iter`,
+// look-back epoch `epoch`) and publishes the next generation of ctrl->gen
+// together with the decision in its low bit, so the other CTAs learn both from
+// the one word they wait on.  `gen_count` is the number of iterations this
+// handle completed before this one.  Returns, for every thread of the CTA,
+// whether another iteration follows (its iteration and epoch are one more).
+__device__ __forceinline__ bool finish_iteration(const IterParams& P, const Args& A, int iter, unsigned epoch,
+                                                 int& flag_smem, unsigned gen_count) {
   __syncthreads();
   if (threadIdx.x == 0) {
     Ctrl* c = P.ctrl;
@@ -335,26 +338,25 @@ __device__ __forceinline__ bool finish_iteration(const IterParams& P, const Args
     int go = 0;
     if (prev == gridDim.x - 1) {
       __threadfence();
-      const int i = c->iter;
       const float r = __uint_as_float(atomicAdd(&c->resid_bits, 0u));
       const int err = ld_volatile(&c->error);
-      if (i < kHistCap) P.hist[i] = r;
+      if (iter < kHistCap) P.hist[iter] = r;
       int st = kRunning;
       if (err) st = err;
       else if (!(r <= 3.402823466e38f)) st = PN_ERR_NONFINITE;
       else if (r <= A.tol) st = PN_OK;
-      else if (i >= A.max_iters) st = PN_NOT_CONVERGED;
+      else if (iter >= A.max_iters) st = PN_NOT_CONVERGED;
       c->launches += 1ull;
       if (st != kRunning) {
         c->status = st;
-        c->final_iter = i;
+        c->final_iter = iter;
         c->final_resid = r;
         const unsigned long long t1 = globaltimer();
         const unsigned long long t0 = c->t_start;
         if (t1 > t0) c->kernel_ns += t1 - t0;
         c->t_start = ~0ull;
       } else {
-        c->iter = i + 1;
+        c->iter = iter + 1;
         go = 1;
       }
       c->resid_bits = 0u;
@@ -363,20 +365,19 @@ __device__ __forceinline__ bool finish_iteration(const IterParams& P, const Args
       c->done = 0u;
       c->epoch = epoch + 1u;
       __threadfence();
-      st_release(&c->gen, gen_before + 1u);
+      st_release(&c->gen, ((gen_count + 1u) << 1) | (unsigned)go);
     } else {
       const unsigned long long t0 = globaltimer();
       unsigned spins = 0;
-      bool ok = true;
-      while (ld_acquire(&c->gen) == gen_before) {
+      unsigned g;
+      while (((g = ld_acquire(&c->gen)) >> 1) == (gen_count & 0x7fffffffu)) {
         if (((++spins) & 15u) == 0u && (long long)(globaltimer() - t0) > A.timeout_ns) {
           atomicCAS(&c->error, 0, (int)PN_ERR_TIMEOUT);
-          ok = false;
           break;
         }
-        if (spins > 64u) __nanosleep(128);
+        if (spins > 64u) __nanosleep(64);
       }
-      go = ok && ld_volatile(&c->status) == kRunning;
+      go = ((g >> 1) != (gen_count & 0x7fffffffu)) && (g & 1u);
     }
     flag_smem = go;
   }

@@ -237,17 +237,23 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       mbar_inval(&bar_cempty[s]);
     }
   };
+  // iteration and look-back epoch of this launch's first iteration; each further
+  // iteration of a looping launch adds one to both
   const unsigned gen0 = *(volatile unsigned*)&ctrl->gen;
-  unsigned epoch = 0u;
+  const unsigned epoch0 = *(volatile unsigned*)&ctrl->epoch;
+  const int iter0 = *(volatile int*)&ctrl->iter;
+  const bool has_tile0 = (int)blockIdx.x < P.tiles_per_group;
+  unsigned epoch = epoch0;
   for (int round = 0;; ++round) {
   if (tid == 0) {
-    if (round == 0) atomicMin(&ctrl->t_start, globaltimer());
-    else inval_barriers();   // every operation on them of the last iteration has completed
-    init_barriers();
+    if (round == 0) {
+      atomicMin(&ctrl->t_start, globaltimer());
+      init_barriers();   // later iterations: re-initialised at the end of the previous one
+    }
     s_abort = 0;
   }
-  epoch = *(volatile unsigned*)&ctrl->epoch;
-  const int iter = *(volatile int*)&ctrl->iter;
+  epoch = epoch0 + (unsigned)round;
+  const int iter = iter0 + round;
   if (tid == 0) {
     // The first tile of every CTA has a static ticket (blockIdx.x < tiles: the grid is never
     // larger) and is fetched right away, overlapping the remaining set-up.
@@ -263,8 +269,10 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       mbar_arrive_expect_tx(&bar_sfull[0], (unsigned)(NKH * C::SH_LOAD));
 #pragma unroll
       for (int h = 0; h < NKH; ++h) tma_load_3d(sS + h * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[0]);
-      mbar_arrive_expect_tx(&bar_xfull[0], (unsigned)C::X_BYTES);
-      tma_load_3d(smem_raw + C::OFF_X, tm_x, 0, t0, b, &bar_xfull[0]);
+      if (round == 0) {   // later iterations: fetched before the grid barrier
+        mbar_arrive_expect_tx(&bar_xfull[0], (unsigned)C::X_BYTES);
+        tma_load_3d(smem_raw + C::OFF_X, tm_x, 0, t0, b, &bar_xfull[0]);
+      }
     } else {
       s_tk[0] = -1;
       mbar_arrive(&bar_sfull[0]);
@@ -753,7 +761,22 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     if (v) atomicMax(&ctrl->resid_bits, v);
   }
   if (!P.persist) break;
-  if (!finish_iteration(P, A, epoch, s_last, gen0 + (unsigned)round)) break;
+  // Set-up of the next iteration ahead of the grid barrier: fresh barriers (every operation on
+  // the old ones has completed) and the first tile's step inputs, which every iteration reads.
+  if (tid == 0) {
+    inval_barriers();
+    init_barriers();
+    if (has_tile0) {
+      const int kg = (int)blockIdx.x;
+      mbar_arrive_expect_tx(&bar_xfull[0], (unsigned)C::X_BYTES);
+      tma_load_3d(smem_raw + C::OFF_X, P.tmaps + 2, 0, (kg / B) * L, kg % B, &bar_xfull[0]);
+    }
+  }
+  if (!finish_iteration(P, A, iter, epoch, s_last, (gen0 >> 1) + (unsigned)round)) {
+    // no next iteration: the prefetched step inputs land before the CTA exits
+    if (tid == 0 && has_tile0 && !mbar_drain(&bar_xfull[0], 0u, tmo)) atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+    break;
+  }
   }   // iterations
 
   tc_fence_before();
