@@ -264,8 +264,8 @@ bool encode_tc_maps(const pn_ctx* h, int mode, CUtensorMap* out) {
   return encode_seq(&out[0], h->args_h->states, D, T, B, 32, L + 1, true) &&
          encode_seq(&out[1], h->buf1, D, T, B, 32, L + 1, true) &&
          encode_seq(&out[2], xs, R * D, T, B, padded_x ? R * DP + 4 : R * DP, L, false) &&
-         encode_seq(&out[3], h->args_h->states, D, T, B, DP + 4, L, false) &&
-         encode_seq(&out[4], h->buf1, D, T, B, DP + 4, L, false);
+         encode_seq(&out[3], h->args_h->states, D, T, B, padded_x ? DP + 4 : DP, L, false) &&
+         encode_seq(&out[4], h->buf1, D, T, B, padded_x ? DP + 4 : DP, L, false);
 }
 
 // Kernels that run before the loop: projection (tanh RNN, GRU) and init.

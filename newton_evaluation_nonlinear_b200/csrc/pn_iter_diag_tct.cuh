@@ -193,11 +193,12 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   float* sCarry = reinterpret_cast<float*>(smem_raw + C::OFF_CARRY);
   float* sRed = reinterpret_cast<float*>(smem_raw + C::OFF_RED);
 
-  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull[2], bar_afull, bar_mma[2],
+  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull[2], bar_ofull[2], bar_afull, bar_mma[2],
       bar_tempty[2], bar_lb[C::NAG], bar_cfull[NSLOT], bar_cempty[NSLOT];
   __shared__ int s_tk[2];        // ticket staged in s stage 0/1 (-1: no more tiles)
   __shared__ int s_atk[2];       // ticket of tile i's operands, by the parity of i (-1: stop)
   __shared__ int s_lbtk[C::NAG];  // ticket handed to the look-back per slot (-1: stop)
+  __shared__ int s_otk[2];        // ticket of the states staged in step-input buffer i (-1: none)
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ int s_last;
@@ -215,6 +216,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_sfull[s], 1u);
       mbar_init(&bar_xfull[s], 1u);
+      mbar_init(&bar_ofull[s], (unsigned)C::NEW);
       mbar_init(&bar_sempty[s], (unsigned)C::NEW);
       mbar_init(&bar_mma[s], 1u);
       mbar_init(&bar_tempty[s], (unsigned)C::NEW);
@@ -229,7 +231,8 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   };
   auto inval_barriers = [&]() {
     uint64_t* bars[] = {&bar_sfull[0], &bar_sfull[1], &bar_sempty[0], &bar_sempty[1], &bar_mma[0], &bar_mma[1],
-                        &bar_tempty[0], &bar_tempty[1], &bar_xfull[0], &bar_xfull[1], &bar_afull};
+                        &bar_tempty[0], &bar_tempty[1], &bar_xfull[0], &bar_xfull[1], &bar_ofull[0],
+                        &bar_ofull[1], &bar_afull};
     for (uint64_t* bb : bars) mbar_inval(bb);
     for (int s = 0; s < C::NAG; ++s) mbar_inval(&bar_lb[s]);
     for (int s = 0; s < NSLOT; ++s) {
@@ -261,6 +264,9 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     const CUtensorMap* tm_x = P.tmaps + 2;
     tmap_acquire(tm_s);
     tmap_acquire(tm_x);
+    // the last iteration's states (other CTAs' stores, ordered before the grid barrier) are
+    // read by the tensor-copy loads below
+    asm volatile("fence.proxy.async.global;" ::: "memory");
     const int kg = (int)blockIdx.x;
     if (kg < P.tiles_per_group) {
       const int b = kg % B;
@@ -312,14 +318,34 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     // =========================== producer ===================================
     const CUtensorMap* tm_s = P.tmaps + ((iter & 1) ? 1 : 0);   // s^(i)
     const CUtensorMap* tm_x = P.tmaps + 2;                      // step inputs
+    const CUtensorMap* tm_o = P.tmaps + ((iter & 1) ? 3 : 4);   // s^(i+1), into the other buffer
+    if (lane == 0) tmap_acquire(tm_o);
+    // The states epilogue tile e staged in step-input buffer e & 1: one tensor store, and a wait
+    // until it has read the buffer, which tile e + 2's step inputs reuse.
+    int n_served = 0;
+    auto serve = [&](int e) -> bool {
+      if (!mbar_wait_flag(&bar_ofull[e & 1], ((unsigned)e >> 1) & 1u, ctrl, tmo, &s_abort)) return false;
+      if (lane == 0) {
+        const int ko = s_otk[e & 1];
+        if (ko >= 0) {
+          tma_store_3d(tm_o, 0, (ko / B) * L, ko % B, smem_raw + C::OFF_X + (e & 1) * C::X_BYTES);
+          bulk_commit();
+          bulk_wait_read();
+        }
+      }
+      __syncwarp();
+      n_served = e + 1;
+      return true;
+    };
     // tile 0 was issued before the block-wide sync (static ticket blockIdx.x)
     const bool none = (int)blockIdx.x >= P.tiles_per_group;
     int it = 1;
-    int n_loaded = none ? 0 : 1;   // tiles whose S and x loads were issued
+    int n_tiles = none ? 0 : 1;    // tiles claimed (their S loads issued)
+    int n_loaded = none ? 0 : 1;   // of them, with their step inputs issued too
     for (; !none; ++it) {
       const int st = it & 1;
-      // stage st (S and step inputs) is free once tile it-2's cell phase is done; the ticket
-      // is claimed only then, so a CTA holds no ticket it cannot start loading
+      // stage st's S buffer is free once tile it-2's cell phase is done; the ticket is claimed
+      // only then, so a CTA holds no ticket it cannot start loading
       if (it >= 2 && !mbar_wait_flag(&bar_sempty[st], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
       int kg = 0;
       if (lane == 0) kg = (int)(gridDim.x + atomicAdd(&ctrl->ticket[0], 1u));
@@ -340,12 +366,24 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         mbar_arrive_expect_tx(&bar_sfull[st], (unsigned)(NKH * C::SH_LOAD));
 #pragma unroll
         for (int h = 0; h < NKH; ++h) tma_load_3d(sS + (st * NKH + h) * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[st]);
+      }
+      __syncwarp();
+      n_tiles = it + 1;
+      // step-input buffer st: free once the states tile it-2's epilogue staged there are read
+      if (it >= 2 && !serve(it - 2)) {
+        ++it;
+        break;
+      }
+      if (lane == 0) {
         mbar_arrive_expect_tx(&bar_xfull[st], (unsigned)C::X_BYTES);
         tma_load_3d(smem_raw + C::OFF_X + st * C::X_BYTES, tm_x, 0, t0, b, &bar_xfull[st]);
       }
       __syncwarp();
       n_loaded = it + 1;
     }
+    // the remaining tiles' staged states
+    for (int e = n_served; e < n_tiles && !s_abort; ++e)
+      if (!serve(e)) break;
     // the last two stages' loads (and the stop marker) complete before the CTA moves on
     for (int j = max(0, it - 2); j < it; ++j)
       if (!mbar_drain(&bar_sfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
@@ -353,6 +391,12 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     for (int j = max(0, n_loaded - 2); j < n_loaded; ++j)
       if (!mbar_drain(&bar_xfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
         atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+    // the stored states are in global memory, ordered before this CTA's part of the grid barrier
+    if (lane == 0) {
+      bulk_wait_all();
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // =========================== MMA issuer =================================
     constexpr uint32_t idesc = umma_idesc_tf32(C::MT, RS);
@@ -584,6 +628,30 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       }
     };
 
+    // s^(i+1) of tile j as above, staged for the producer's tensor store in step-input buffer
+    // `stg` (whose inputs every epilogue warp has consumed), eight steps at a time
+    auto stage_out = [&](int j, float pa, float pb, int stg) {
+      const int slot = j % NSLOT;
+      mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort);
+      const float carry = sCarry[slot * DP + c];
+      const float cp = kHasA ? fmaf(pa, carry, pb) : carry + pb;
+      const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + (kHasA ? 32 : 16) * rg) + lane_off;
+      float* xo = reinterpret_cast<float*>(smem_raw + C::OFF_X + stg * C::X_BYTES) + row0 * DP + c;
+#pragma unroll
+      for (int h8 = 0; h8 < (kHasA ? 2 : 1); ++h8) {
+        float v[16];   // quasi: A then B of steps 8 h8 .. 8 h8 + 7; Picard: B of all 16 steps
+        tmem_ld16(sbase + (uint32_t)(16 * h8), v);
+#pragma unroll
+        for (int i = 0; i < (kHasA ? 8 : 16); ++i) {
+          const int ii = (kHasA ? 8 * h8 : 0) + i;
+          xo[ii * DP] = kHasA ? fmaf(v[i], cp, v[8 + i]) : cp + v[i];
+        }
+      }
+      fence_async_smem();   // generic writes -> the tensor store (async proxy)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_cempty[slot]);
+    };
+
     // The loop's exit decision is one thread's reading of the next stage's ticket,
     // published before a named barrier, so every epilogue thread takes the same path.
     prepare(0);
@@ -597,12 +665,6 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       const int buf = it & 1;
       const int b = kg % B;
       const int t0 = (kg / B) * L;
-
-      // the states of tile it-3 (its carry had nearly three tiles of time to arrive); this
-      // frees the stash slot this tile's prefixes go to, and overlaps the wait for the products
-      if constexpr (kScan) {
-        if (it >= C::DEFER) write_out(it - C::DEFER, kg_m3, pa3, pb3);
-      }
 
       // ---- Z of this thread's channel and 16 steps, then cell + sequential scan
       mbar_wait_flag(&bar_mma[buf], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort);
@@ -684,6 +746,9 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
             if (t0 + row0 + i < T) o[(size_t)i * D] = bv[i];
         }
         named_barrier(1, NTE);   // the ticket of tile it+1
+        if (te == 0) s_otk[st] = -1;   // nothing staged: the step-input buffer is free
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_ofull[st]);
         kg = s_atk[(it + 1) & 1];
       } else {
         // ---- combine the 8 pieces of each channel
@@ -715,6 +780,13 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
             mbar_arrive(&bar_lb[aslot]);
           }
         }
+        // the states of tile it-3 (its carry had three tiles of time to arrive), staged in this
+        // tile's step-input buffer for the producer's tensor store; this frees the stash slot
+        // this tile's prefixes take
+        if (it >= C::DEFER) stage_out(it - C::DEFER, pa3, pb3, st);
+        if (te == 0) s_otk[st] = (it >= C::DEFER && !s_abort) ? kg_m3 : -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_ofull[st]);
         // ---- park the in-piece prefixes in TMEM
         {
           const uint32_t sbase =
