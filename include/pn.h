@@ -136,6 +136,23 @@ PN_API pn_status pn_eval_host(pn_handle h, const float* x_host, const float* s0_
                        pn_mode mode, int max_iters, float tol,
                        float* states_host, int* iters_out, float* resid_out);
 
+/* pn_eval_host over n independent batches in a pipeline: batch k+1's inputs
+ * are copied in while batch k is evaluated and batch k-1's states are copied
+ * out, on two internal copy streams ordered against the handle's stream by
+ * events, through two device staging slots (allocated on the first call,
+ * 2 x (x, s0, states) of this handle's shapes).  x_host[k], s0_host[k] and
+ * states_host[k] are batch k's host buffers (pinned memory lets the copies
+ * overlap; states_host may repeat a buffer only for batches whose results
+ * are not kept); iters_out[k] and resid_out[k] (arrays of n, either may be
+ * NULL) receive each batch's count and final residual.  Every batch gives
+ * the same result pn_eval_host gives for it.  Returns the first error, else
+ * PN_NOT_CONVERGED if any batch did not converge, else PN_OK; the call is
+ * complete (all copies done) on return. */
+PN_API pn_status pn_eval_host_many(pn_handle h, int n, const float* const* x_host,
+                                   const float* const* s0_host, pn_mode mode, int max_iters,
+                                   float tol, float* const* states_host, int* iters_out,
+                                   float* resid_out);
+
 /* Copy min(n, iters+1) residuals r^(0..iters) of the last evaluation into the
  * host array out; *n_written (may be NULL) receives the count. */
 PN_API pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written);

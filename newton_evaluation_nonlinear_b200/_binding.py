@@ -45,6 +45,7 @@ SIGNATURES = {
                          ctypes.POINTER(_c_float)]),
     "pn_eval_host": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_float, _vp, ctypes.POINTER(_c_int),
                               ctypes.POINTER(_c_float)]),
+    "pn_eval_host_many": (_c_int, [_vp, _c_int, _vp, _vp, _c_int, _c_int, _c_float, _vp, _vp, _vp]),
     "pn_get_residual_history": (_c_int, [_vp, _vp, _c_int, ctypes.POINTER(_c_int)]),
     "pn_time_iterations": (_c_int, [_vp, _c_int, _c_int, ctypes.POINTER(_c_float)]),
     "pn_get_stats": (_c_int, [_vp, ctypes.POINTER(pn_stats)]),
@@ -120,6 +121,24 @@ def pn_eval_host(h: int, x: np.ndarray, s0: np.ndarray, mode: int, max_iters: in
     st = lib.pn_eval_host(h, x.ctypes.data, s0.ctypes.data, int(mode), int(max_iters), float(tol),
                           states.ctypes.data, ctypes.byref(it), ctypes.byref(r))
     return st, it.value, r.value
+
+
+def pn_eval_host_many(h: int, xs, s0s, mode: int, max_iters: int, tol: float, states_list):
+    """Pipelined pn_eval_host over len(xs) batches; returns (status, iters[], resids[])."""
+    n = len(xs)
+    if len(s0s) != n or len(states_list) != n:
+        raise ValueError("one x, s0 and states buffer per batch")
+    for a in list(xs) + list(s0s) + list(states_list):
+        if a.dtype != np.float32 or not a.flags.c_contiguous:
+            raise ValueError("host buffers must be C-contiguous float32")
+    px = (_vp * max(n, 1))(*[a.ctypes.data for a in xs])
+    ps0 = (_vp * max(n, 1))(*[a.ctypes.data for a in s0s])
+    pst = (_vp * max(n, 1))(*[a.ctypes.data for a in states_list])
+    its = np.full(max(n, 1), -1, np.int32)
+    rs = np.full(max(n, 1), np.nan, np.float32)
+    st = lib.pn_eval_host_many(h, n, px, ps0, int(mode), int(max_iters), float(tol), pst, its.ctypes.data,
+                               rs.ctypes.data)
+    return st, its[:n], rs[:n]
 
 
 def pn_get_residual_history(h: int, n: int) -> Tuple[int, np.ndarray]:
@@ -234,6 +253,18 @@ class Solver:
         st, it, r = pn_eval_host(self.h, x, s0, mode, max_iters, tol, states)
         self._check(st)
         return states, it, r, st
+
+    def eval_host_many(self, xs, s0s, mode, max_iters: Optional[int] = None, tol: float = 1e-5,
+                       states_list=None):
+        """Evaluate several batches from host buffers, overlapping each batch's copies with the
+        neighbouring batches' evaluations.  Returns (states_list, iters, resids, status)."""
+        mode = MODES[mode] if isinstance(mode, str) else int(mode)
+        max_iters = self.T if max_iters is None else int(max_iters)
+        if states_list is None:
+            states_list = [np.empty((self.B, self.T, self.D), np.float32) for _ in xs]
+        st, its, rs = pn_eval_host_many(self.h, xs, s0s, mode, max_iters, tol, states_list)
+        self._check(st)
+        return states_list, its, rs, st
 
     def residual_history(self, n: int = 1 << 16) -> np.ndarray:
         st, h = pn_get_residual_history(self.h, n)

@@ -76,6 +76,12 @@ struct pn_ctx {
   float* hx = nullptr;
   float* hs0 = nullptr;
   float* hst = nullptr;
+  // pipelined host-buffer evaluation (pn_eval_host_many): two staging slots, copy streams, events
+  float* px[2] = {nullptr, nullptr};
+  float* ps0[2] = {nullptr, nullptr};
+  float* pst[2] = {nullptr, nullptr};
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_done[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
   // graphs, one per mode, built on first use
   cudaGraph_t graph[4] = {nullptr, nullptr, nullptr, nullptr};
   cudaGraphExec_t exec[4] = {nullptr, nullptr, nullptr, nullptr};
@@ -145,8 +151,19 @@ void free_all(pn_ctx* h) {
     h->exec[m] = nullptr;
     h->graph[m] = nullptr;
   }
-  float** fbufs[] = {&h->wt_diag, &h->wt_dense, &h->wt_tc, &h->wt_tct, &h->wdiag, &h->bhn, &h->proj_w, &h->proj_b,
-                     &h->xin,     &h->buf1,     &h->agg,   &h->pref,   &h->hist,  &h->hx,  &h->hs0,    &h->hst};
+  float** fbufs[] = {&h->wt_diag, &h->wt_dense, &h->wt_tc, &h->wt_tct, &h->wdiag, &h->bhn,    &h->proj_w,
+                     &h->proj_b,  &h->xin,      &h->buf1,  &h->agg,    &h->pref,  &h->hist, &h->hx,
+                     &h->hs0,     &h->hst,      &h->px[0], &h->px[1],  &h->ps0[0], &h->ps0[1], &h->pst[0],
+                     &h->pst[1]};
+  for (int q = 0; q < 2; ++q) {
+    if (h->ev_in[q]) cudaEventDestroy(h->ev_in[q]);
+    if (h->ev_done[q]) cudaEventDestroy(h->ev_done[q]);
+    if (h->ev_out[q]) cudaEventDestroy(h->ev_out[q]);
+    h->ev_in[q] = h->ev_done[q] = h->ev_out[q] = nullptr;
+  }
+  if (h->s_in) cudaStreamDestroy(h->s_in);
+  if (h->s_out) cudaStreamDestroy(h->s_out);
+  h->s_in = h->s_out = nullptr;
   for (float** p : fbufs) {
     if (*p) cudaFree(*p);
     *p = nullptr;
@@ -856,6 +873,81 @@ pn_status pn_eval_host(pn_handle h, const float* x_host, const float* s0_host, p
   if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
   if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "copying states to the host failed: %s", cudaGetErrorString(e));
   return st;
+}
+
+pn_status pn_eval_host_many(pn_handle h, int n, const float* const* x_host, const float* const* s0_host,
+                            pn_mode mode, int max_iters, float tol, float* const* states_host, int* iters_out,
+                            float* resid_out) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  DeviceGuard dg(h->device);
+  pn_status st = validate_mode(h, mode, max_iters, tol);
+  if (st != PN_OK) return st;
+  if (n < 0) return fail(h, PN_ERR_INVALID, "n = %d < 0", n);
+  if (n == 0) return PN_OK;
+  if (!x_host || !s0_host || !states_host) return fail(h, PN_ERR_INVALID, "NULL host buffer array");
+  for (int k = 0; k < n; ++k)
+    if (!x_host[k] || !s0_host[k] || !states_host[k]) return fail(h, PN_ERR_INVALID, "NULL host buffer (batch %d)", k);
+  const size_t nx = (size_t)h->B * h->T * h->d_in;
+  const size_t ns = (size_t)h->B * h->T * h->D;
+  const size_t n0 = (size_t)h->B * h->D;
+  if (!h->px[0]) {
+    for (int q = 0; q < 2; ++q) {
+      if ((st = dalloc(h, &h->px[q], nx)) != PN_OK) return st;
+      if ((st = dalloc(h, &h->ps0[q], n0)) != PN_OK) return st;
+      if ((st = dalloc(h, &h->pst[q], ns)) != PN_OK) return st;
+      PN_CUDA(h, cudaEventCreateWithFlags(&h->ev_in[q], cudaEventDisableTiming));
+      PN_CUDA(h, cudaEventCreateWithFlags(&h->ev_done[q], cudaEventDisableTiming));
+      PN_CUDA(h, cudaEventCreateWithFlags(&h->ev_out[q], cudaEventDisableTiming));
+    }
+    PN_CUDA(h, cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking));
+    PN_CUDA(h, cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking));
+  }
+  // batch k uses slot k & 1.  Its inputs go in on s_in once batch k-2's evaluation has read that
+  // slot; it is evaluated on the handle's stream once they are in and batch k-2's states have
+  // left the slot; its states go out on s_out once it is evaluated.
+  auto copy_in = [&](int k) -> pn_status {
+    const int q = k & 1;
+    if (k >= 2) PN_CUDA(h, cudaStreamWaitEvent(h->s_in, h->ev_done[q], 0));
+    PN_CUDA(h, cudaMemcpyAsync(h->px[q], x_host[k], nx * sizeof(float), cudaMemcpyHostToDevice, h->s_in));
+    PN_CUDA(h, cudaMemcpyAsync(h->ps0[q], s0_host[k], n0 * sizeof(float), cudaMemcpyHostToDevice, h->s_in));
+    PN_CUDA(h, cudaEventRecord(h->ev_in[q], h->s_in));
+    return PN_OK;
+  };
+  pn_status result = PN_OK;
+  if ((st = copy_in(0)) != PN_OK) return st;
+  for (int k = 0; k < n; ++k) {
+    const int q = k & 1;
+    if (k + 1 < n && (st = copy_in(k + 1)) != PN_OK) return st;
+    PN_CUDA(h, cudaStreamWaitEvent(h->stream, h->ev_in[q], 0));
+    if (k >= 2) PN_CUDA(h, cudaStreamWaitEvent(h->stream, h->ev_out[q], 0));
+    Args& a = *h->args_h;
+    a.x = h->px[q];
+    a.s0 = h->ps0[q];
+    a.states = h->pst[q];
+    a.tol = tol;
+    a.max_iters = max_iters;
+    a.timeout_ns = h->timeout_ns;
+    a.stall_ticket = h->stall_ticket;
+    int it = -1;
+    float r = NAN;
+    st = run_eval(h, mode, &it, &r);   // returns after the evaluation is complete
+    if (iters_out) iters_out[k] = it;
+    if (resid_out) resid_out[k] = r;
+    if (st < 0 && st != PN_ERR_NONFINITE) {
+      cudaStreamSynchronize(h->s_in);
+      cudaStreamSynchronize(h->s_out);
+      return st;
+    }
+    if (st != PN_OK && result == PN_OK) result = st;
+    PN_CUDA(h, cudaEventRecord(h->ev_done[q], h->stream));
+    PN_CUDA(h, cudaStreamWaitEvent(h->s_out, h->ev_done[q], 0));
+    PN_CUDA(h, cudaMemcpyAsync(states_host[k], h->pst[q], ns * sizeof(float), cudaMemcpyDeviceToHost, h->s_out));
+    PN_CUDA(h, cudaEventRecord(h->ev_out[q], h->s_out));
+  }
+  cudaError_t e = cudaStreamSynchronize(h->s_out);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(h->s_in);
+  if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "copying states to the host failed: %s", cudaGetErrorString(e));
+  return result;
 }
 
 pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written) {

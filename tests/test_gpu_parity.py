@@ -252,6 +252,24 @@ def test_eval_host_matches_eval():
     np.testing.assert_array_equal(states, a[0])
 
 
+@pytest.mark.parametrize("cell,D,T,B", [(pi.CELL_TANH_RNN, 64, 4096, 4), (pi.CELL_GRU, 32, 900, 3)])
+def test_eval_host_many_matches_eval_host(cell, D, T, B):
+    """The pipelined host entry point gives every batch the result pn_eval_host gives it (to
+    rounding: the look-back may fold in a different order), with the same iteration count."""
+    pn = _pn()
+    probs = [pi.random_problem(40 + j, cell, D, D, T=T, B=B, rho=0.7, tol=1e-5) for j in range(3)]
+    solver = pn.Solver.from_problem(probs[0])   # the weights of batch 0; the other batches differ in x, s0
+    xs = [np.ascontiguousarray(p.x) for p in probs]
+    s0s = [np.ascontiguousarray(p.s0) for p in probs]
+    outs, its, rs, st = solver.eval_host_many(xs, s0s, "quasi", T, 1e-5)
+    assert st in (pn.PN_OK, pn.PN_NOT_CONVERGED)
+    for j in range(3):
+        ref, it, r, st1 = solver.eval_host(xs[j], s0s[j], "quasi", T, 1e-5)
+        assert its[j] == it
+        np.testing.assert_allclose(outs[j], ref, rtol=0, atol=1e-6 * max(1.0, float(np.abs(ref).max())))
+    solver.close()
+
+
 def test_stats_and_timing():
     import torch
     pn = _pn()
