@@ -57,5 +57,15 @@ def test_argument_validation_without_gpu():
     assert pn.pn_last_error(None) != ""
     st, _, _ = pn.pn_eval(None, 0, 0, 0, 1, 1e-5, 0)
     assert st == pn.PN_ERR_INVALID
+    x = np.zeros((2, 16, 3), np.float32)
+    s0 = np.zeros((2, 4), np.float32)
+    out = np.zeros((2, 16, 4), np.float32)
+    st, its, rs = pn.pn_eval_host_many(None, [x, x], [s0, s0], 0, 1, 1e-5, [out, out])
+    assert st == pn.PN_ERR_INVALID and len(its) == 2 and len(rs) == 2
+    try:
+        pn.pn_eval_host_many(None, [x], [s0, s0], 0, 1, 1e-5, [out])
+        raise AssertionError("mismatched batch lists accepted")
+    except ValueError:
+        pass
     pn.pn_destroy(None)
     assert pn.pn_version().startswith("libpn")
