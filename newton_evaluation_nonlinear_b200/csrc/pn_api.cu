@@ -534,6 +534,9 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   if (c.status == PN_ERR_NONFINITE)
     return fail(h, PN_ERR_NONFINITE, "residual became non-finite at iteration %d", c.final_iter);
   if (c.status == kRunning) return fail(h, PN_ERR_CUDA, "the convergence loop did not finish");
+  if (c.error)   // a bounded wait gave up after the stop rule had fired: the launch stalled
+    return fail(h, PN_ERR_TIMEOUT, "a device wait gave up after the stop decision (%lld ns)",
+                (long long)h->args_h->timeout_ns);
   h->err.clear();
   return (pn_status)c.status;
 }
