@@ -23,9 +23,9 @@
 // residual, and scans those steps sequentially in registers -- no shuffles.
 // The 8 sixteen-step pieces of a channel are combined through shared memory;
 // the piece prefix (PA, PB) stays in registers, the in-piece prefixes are
-// parked in TMEM, and the states are formed two tiles later from the carry of
-// the look-back warps, stored straight from registers (a warp writes 32
-// consecutive channels of one step: 128 contiguous bytes).
+// parked in TMEM, and the states are formed three tiles later from the carry
+// of the look-back warps, staged in the step-input buffer the tile has
+// consumed and written by one TMA tensor store from the producer warp.
 //
 // With P.persist = 1 the kernel runs the whole fixed-point loop in one launch:
 // after each iteration the CTAs meet at a bounded grid barrier whose last
@@ -35,7 +35,7 @@
 // The step inputs are double-buffered with the S stages and released with
 // them, so both are fetched two tiles ahead of their use.
 //
-// Warp roles (one CTA per SM): 0 producer (tickets, TMA loads); 1 MMA issuer;
+// Warp roles (one CTA per SM): 0 producer (tickets, TMA loads and state stores); 1 MMA issuer;
 // 2-3 look-back (scan modes, alternate tiles); the rest epilogue (4 TMEM lane
 // quarters x RS / 16 step groups).  The epilogue forms the next tile's S_lo
 // right after the current tile's cell phase, so the tensor cores compute the
@@ -193,7 +193,8 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   float* sCarry = reinterpret_cast<float*>(smem_raw + C::OFF_CARRY);
   float* sRed = reinterpret_cast<float*>(smem_raw + C::OFF_RED);
 
-  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull[2], bar_ofull[2], bar_afull, bar_mma[2],
+  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull[2], bar_ofull[2], bar_oempty[2], bar_afull,
+      bar_mma[2],
       bar_tempty[2], bar_lb[C::NAG], bar_cfull[NSLOT], bar_cempty[NSLOT];
   __shared__ int s_tk[2];        // ticket staged in s stage 0/1 (-1: no more tiles)
   __shared__ int s_atk[2];       // ticket of tile i's operands, by the parity of i (-1: stop)
@@ -217,6 +218,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       mbar_init(&bar_sfull[s], 1u);
       mbar_init(&bar_xfull[s], 1u);
       mbar_init(&bar_ofull[s], (unsigned)C::NEW);
+      mbar_init(&bar_oempty[s], 1u);
       mbar_init(&bar_sempty[s], (unsigned)C::NEW);
       mbar_init(&bar_mma[s], 1u);
       mbar_init(&bar_tempty[s], (unsigned)C::NEW);
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   auto inval_barriers = [&]() {
     uint64_t* bars[] = {&bar_sfull[0], &bar_sfull[1], &bar_sempty[0], &bar_sempty[1], &bar_mma[0], &bar_mma[1],
                         &bar_tempty[0], &bar_tempty[1], &bar_xfull[0], &bar_xfull[1], &bar_ofull[0],
-                        &bar_ofull[1], &bar_afull};
+                        &bar_ofull[1], &bar_oempty[0], &bar_oempty[1], &bar_afull};
     for (uint64_t* bb : bars) mbar_inval(bb);
     for (int s = 0; s < C::NAG; ++s) mbar_inval(&bar_lb[s]);
     for (int s = 0; s < NSLOT; ++s) {
@@ -320,8 +322,10 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     const CUtensorMap* tm_x = P.tmaps + 2;                      // step inputs
     const CUtensorMap* tm_o = P.tmaps + ((iter & 1) ? 3 : 4);   // s^(i+1), into the other buffer
     if (lane == 0) tmap_acquire(tm_o);
-    // The states epilogue tile e staged in step-input buffer e & 1: one tensor store, and a wait
-    // until it has read the buffer, which tile e + 2's step inputs reuse.
+    // The states the epilogue staged at its event e (one event per tile, and three more for the
+    // last write-outs) in step-input buffer e & 1: one tensor store, and a wait until it has
+    // read the buffer, which is then free again (for tile e + 2's step inputs, or, signalled on
+    // bar_oempty, for the epilogue's last events).
     int n_served = 0;
     auto serve = [&](int e) -> bool {
       if (!mbar_wait_flag(&bar_ofull[e & 1], ((unsigned)e >> 1) & 1u, ctrl, tmo, &s_abort)) return false;
@@ -332,6 +336,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
           bulk_commit();
           bulk_wait_read();
         }
+        mbar_arrive(&bar_oempty[e & 1]);
       }
       __syncwarp();
       n_served = e + 1;
@@ -381,8 +386,8 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       __syncwarp();
       n_loaded = it + 1;
     }
-    // the remaining tiles' staged states
-    for (int e = n_served; e < n_tiles && !s_abort; ++e)
+    // the remaining events: the last tiles', and three more for the last write-outs
+    for (int e = n_served; e < n_tiles + (kScan ? C::DEFER : 0) && !s_abort; ++e)
       if (!serve(e)) break;
     // the last two stages' loads (and the stop marker) complete before the CTA moves on
     for (int j = max(0, it - 2); j < it; ++j)
@@ -596,40 +601,10 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       }
     };
 
-    // s^(i+1) of tile j (ticket kgj): piece carry from the look-back carry, then the parked
-    // prefixes (the stash holds [A 0-7 | B 0-7 | A 8-15 | B 8-15] per 16 steps; B only for Picard)
-    auto write_out = [&](int j, int kgj, float pa, float pb) {
-      const int slot = j % NSLOT;
-      mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort);
-      const float carry = sCarry[slot * DP + c];
-      const float cp = kHasA ? fmaf(pa, carry, pb) : carry + pb;
-      const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + (kHasA ? 32 : 16) * rg) + lane_off;
-      float v[32];
-      if constexpr (kHasA) {
-        tmem_ld32(sbase, v);
-      } else {
-        float bb[16];
-        tmem_ld16(sbase, bb);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = bb[i];
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_cempty[slot]);
-      if (!s_abort) {
-        const int tj = (kgj / B) * L + row0;
-        float* o = dst + ((size_t)(kgj % B) * T + tj) * D + c;
-        const bool whole = (tj + 16 <= T);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int q = (i & 8) * 2 + (i & 7);   // A of step i at column q, its B at q + 8
-          const float sv = kHasA ? fmaf(v[q], cp, v[q + 8]) : cp + v[i];
-          if (whole || tj + i < T) o[(size_t)i * D] = sv;
-        }
-      }
-    };
-
-    // s^(i+1) of tile j as above, staged for the producer's tensor store in step-input buffer
-    // `stg` (whose inputs every epilogue warp has consumed), eight steps at a time
+    // s^(i+1) of tile j: piece carry from the look-back carry, then the parked prefixes (the
+    // stash holds [A 0-7 | B 0-7 | A 8-15 | B 8-15] per 16 steps; B only for Picard), staged for
+    // the producer's tensor store in step-input buffer `stg` (whose inputs every epilogue warp
+    // has consumed), eight steps at a time
     auto stage_out = [&](int j, float pa, float pb, int stg) {
       const int slot = j % NSLOT;
       mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort);
@@ -808,9 +783,22 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       }
     }
     if constexpr (kScan) {
-      if (it >= 3) write_out(it - 3, kg_m3, pa3, pb3);
-      if (it >= 2) write_out(it - 2, kg_m2, pa2, pb2);
-      if (it >= 1) write_out(it - 1, kg_m1, pa1, pb1);
+      // the last three tiles' states: events it .. it+2, each in the step-input buffer of its
+      // parity once the store of the event two before has read that buffer
+#pragma unroll
+      for (int j = 0; j < C::DEFER; ++j) {
+        const int ev = it + j;
+        const int tj = ev - C::DEFER;
+        const int st = ev & 1;
+        if (ev >= 2) mbar_wait_flag(&bar_oempty[st], ((unsigned)(ev - 2) >> 1) & 1u, ctrl, tmo, &s_abort);
+        const int kj = (j == 0) ? kg_m3 : (j == 1 ? kg_m2 : kg_m1);
+        const float pa = (j == 0) ? pa3 : (j == 1 ? pa2 : pa1);
+        const float pb = (j == 0) ? pb3 : (j == 1 ? pb2 : pb1);
+        if (tj >= 0) stage_out(tj, pa, pb, st);
+        if (te == 0) s_otk[st] = (tj >= 0 && !s_abort) ? kj : -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_ofull[st]);
+      }
       // stop the look-back warps: their next tiles are it .. it + NLB - 1
       if (lastw && lane == 0) {
         for (int j = it; j < it + C::NLB; ++j) {
