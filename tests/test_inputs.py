@@ -71,3 +71,15 @@ def test_full_workloads_match_stored_fingerprints(index):
     p = pi.benchmark_workload(index)
     assert (p.B, p.T, p.D, p.d_in) == (stored["B"], stored["T"], stored["D"], stored["d_in"])
     assert p.fingerprint() == stored["fingerprint"]
+
+
+def test_stored_oracle_results_regenerate():
+    """The stored oracle results are the oracle's: workload 0 (small enough to rerun here)
+    gives the same count, status and residual history again."""
+    import oracle
+    stored = json.load(open(GOLDEN))["0"]["modes_result"]["newton"]
+    p = pi.benchmark_workload(0)
+    _, it, r, st, hist = oracle.Model.from_problem(p).iterate(pi.MODE_NEWTON, p.x, p.s0, p.iters_cap, p.tol)
+    assert (int(it), int(st)) == (stored["iters"], stored["status"])
+    np.testing.assert_allclose(np.asarray(hist, np.float64), np.asarray(stored["history"]), rtol=1e-12, atol=0)
+    assert abs(float(r) - stored["resid"]) <= 1e-12 * abs(stored["resid"])
