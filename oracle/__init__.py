@@ -25,7 +25,8 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-JACOBI, PICARD, QUASI, NEWTON = 0, 1, 2, 3
+JACOBI, PICARD, QUASI, NEWTON, BANDED = 0, 1, 2, 3, 4
+STORE_F64, STORE_F32, STORE_BF16, STORE_F16 = 0, 1, 2, 3
 OK, NOT_CONVERGED, ERR_INVALID, ERR_NOMEM, ERR_NONFINITE = 0, 1, -1, -2, -4
 
 
@@ -60,8 +61,14 @@ def _load():
             lib.orc_update.argtypes = [i, i, i, i, dp, d, i, i, dp, dp, dp, dp, i]
             lib.orc_iterate.argtypes = [i, i, i, i, dp, d, i, i, dp, dp, i, d, dp, ip, dp, dp, i, i]
             lib.orc_affine_recurrence.argtypes = [i, i, dp, dp, dp, dp]
+            lib.orc_banded_jacobian.argtypes = [i, i, i, i, dp, d, dp, dp, dp]
+            lib.orc_round_storage.argtypes = [i, dp, ctypes.c_long]
+            lib.orc_update_ex.argtypes = [i, i, i, d, i, i, dp, d, i, i, dp, dp, dp, dp, i]
+            lib.orc_iterate_ex.argtypes = [i, i, i, d, i, d, i, d, i, i, i, dp, d, i, i, dp, dp, i, d,
+                                           dp, ip, dp, dp, ip, i, ip, i]
             for fn in ("orc_cell", "orc_jacobian", "orc_approx_jacobian", "orc_sequential",
-                       "orc_residual", "orc_update", "orc_iterate", "orc_affine_recurrence"):
+                       "orc_residual", "orc_update", "orc_iterate", "orc_affine_recurrence",
+                       "orc_banded_jacobian", "orc_round_storage", "orc_update_ex", "orc_iterate_ex"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -173,6 +180,66 @@ class Model:
         if st in (ERR_INVALID, ERR_NOMEM):
             _check(st, "iterate")
         return s, it.value, r.value, st, hist[: min(it.value + 1, cap)].copy()
+
+
+    # --- the page's refinements: banded Jacobian, damping, adaptive switching,
+    # --- reduced-precision iterate storage, windowed solve (readings in oracle.h)
+    def banded_jacobian(self, band: int, x_t, s_prev) -> np.ndarray:
+        x_t, s_prev = _f64(x_t), _f64(s_prev)
+        A = np.empty((self.D, self.D))
+        _check(_load().orc_banded_jacobian(self.cell, int(band), self.D, self.d_in, _ptr(self.p),
+                                           self.eps, _ptr(x_t), _ptr(s_prev), _ptr(A)),
+               "banded_jacobian")
+        return A
+
+    def update_ex(self, mode: int, x, s0, s_cur, band: int = 0, damping: float = 1.0,
+                  nthreads: int = 0) -> np.ndarray:
+        x, s0, B, T = self._shapes(x, s0)
+        s_cur = _f64(s_cur)
+        s_next = np.empty((B, T, self.D))
+        _check(_load().orc_update_ex(self.cell, int(mode), int(band), float(damping), self.D,
+                                     self.d_in, _ptr(self.p), self.eps, T, B, _ptr(x), _ptr(s0),
+                                     _ptr(s_cur), _ptr(s_next), nthreads or default_threads(B)),
+               "update_ex")
+        return s_next
+
+    def iterate_ex(self, mode: int, x, s0, max_iters: int, tol: float, band: int = 0,
+                   damping: float = 1.0, adapt: bool = False, stall: float = 0.9,
+                   store: int = STORE_F64, store_until: float = 0.0, window: int = 0,
+                   nthreads: int = 0, hist_cap: int = None):
+        """Returns (states, iters, resid, status, history, modes, window_iters).
+
+        history / modes: each measured residual and the mode of the update that
+        followed it (-1 after a window's last residual), window after window."""
+        x, s0, B, T = self._shapes(x, s0)
+        Wn = T if (window <= 0 or window >= T) else int(window)
+        nwin = 0 if T == 0 else (T + Wn - 1) // Wn
+        s = np.empty((B, T, self.D))
+        cap = nwin * (max_iters + 1) if hist_cap is None else int(hist_cap)
+        hist = np.zeros(max(cap, 1))
+        modes = np.full(max(cap, 1), -2, dtype=np.intc)
+        wit = np.zeros(max(nwin, 1), dtype=np.intc)
+        ip = ctypes.POINTER(ctypes.c_int)
+        it = ctypes.c_int(0)
+        r = ctypes.c_double(0.0)
+        st = _load().orc_iterate_ex(self.cell, int(mode), int(band), float(damping), int(bool(adapt)),
+                                    float(stall), int(store), float(store_until), int(window),
+                                    self.D, self.d_in, _ptr(self.p), self.eps, T, B, _ptr(x),
+                                    _ptr(s0), int(max_iters), float(tol), _ptr(s),
+                                    ctypes.byref(it), ctypes.byref(r), _ptr(hist),
+                                    modes.ctypes.data_as(ip), cap, wit.ctypes.data_as(ip),
+                                    nthreads or default_threads(B))
+        if st in (ERR_INVALID, ERR_NOMEM):
+            _check(st, "iterate_ex")
+        used = min(int(np.sum(wit[:nwin])) + nwin, cap)
+        return s, it.value, r.value, st, hist[:used].copy(), modes[:used].copy(), wit[:nwin].copy()
+
+
+def round_storage(values, store: int) -> np.ndarray:
+    """Values rounded to a storage format (STORE_*), returned as float64."""
+    v = _f64(values).copy()
+    _check(_load().orc_round_storage(int(store), _ptr(v), v.size), "round_storage")
+    return v
 
 
 def affine_recurrence(A, b, s_init) -> np.ndarray:

@@ -204,6 +204,8 @@ typedef struct {
   const double* s_in;  /* current iterate (residual / update) */
   double* out;         /* sequential states, F, or s_next */
   const double* F;     /* precomputed residual for the update, or NULL */
+  int band;            /* half-bandwidth for ORC_BANDED */
+  double damping;      /* lambda of s_next = s + lambda * delta (1 = undamped) */
   int b_begin, b_end;
   double rmax;
   int rc;
@@ -357,6 +359,8 @@ static void* update_worker(void* arg) {
       }
       if (!rc && (j->mode == ORC_QUASI || j->mode == ORC_NEWTON))
         rc = orc_approx_jacobian(j->cell, j->mode, D, d_in, j->p, j->eps, xt, prev, A);
+      else if (!rc && j->mode == ORC_BANDED)
+        rc = orc_banded_jacobian(j->cell, j->band, D, d_in, j->p, j->eps, xt, prev, A);
       if (rc) { j->rc = rc; free(buf); return NULL; }
       for (int r = 0; r < D; ++r) {
         double acc;
@@ -366,7 +370,7 @@ static void* update_worker(void* arg) {
           acc = dprev[r];
         } else if (j->mode == ORC_QUASI) {
           acc = A[(long)r * D + r] * dprev[r];
-        } else {
+        } else { /* newton, and banded with its zeros outside the band */
           acc = 0.0;
           for (int k = 0; k < D; ++k) acc += A[(long)r * D + k] * dprev[k];
         }
@@ -374,7 +378,9 @@ static void* update_worker(void* arg) {
       }
       double* nxt = j->out + ((long)b * T + t) * D;
       for (int r = 0; r < D; ++r) {
-        nxt[r] = cur[r] + dcur[r];
+        /* the recurrence runs on the full delta; damping scales only the
+           step taken (lambda * delta solves J~ v = -lambda F) */
+        nxt[r] = cur[r] + j->damping * dcur[r];
         dprev[r] = dcur[r];
       }
       prev = cur;
@@ -393,7 +399,7 @@ int orc_update(int cell, int mode, int D, int d_in, const double* p,
   orc_job proto = {0};
   proto.cell = cell; proto.mode = mode; proto.D = D; proto.d_in = d_in;
   proto.T = T; proto.p = p; proto.eps = eps; proto.x = x; proto.s0 = s0;
-  proto.s_in = s_cur; proto.out = s_next;
+  proto.s_in = s_cur; proto.out = s_next; proto.damping = 1.0;
   return run_jobs(update_worker, &proto, B, nthreads, NULL);
 }
 
@@ -428,7 +434,7 @@ int orc_iterate(int cell, int mode, int D, int d_in, const double* p,
       orc_job proto = {0};
       proto.cell = cell; proto.mode = mode; proto.D = D; proto.d_in = d_in;
       proto.T = T; proto.p = p; proto.eps = eps; proto.x = x; proto.s0 = s0;
-      proto.s_in = cur; proto.out = nxt; proto.F = F;
+      proto.s_in = cur; proto.out = nxt; proto.F = F; proto.damping = 1.0;
       rc = run_jobs(update_worker, &proto, B, nthreads, NULL);
     }
     if (rc) { free(other); free(F); return rc; }
@@ -457,4 +463,202 @@ int orc_affine_recurrence(int D, int T, const double* A, const double* b,
     prev = cur;
   }
   return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* extensions: banded Jacobian, storage rounding, damping, adaptive     */
+/* switching, windowed solve (declarations and readings in oracle.h)    */
+/* ------------------------------------------------------------------ */
+
+int orc_banded_jacobian(int cell, int band, int D, int d_in, const double* p,
+                        double eps, const double* x_t, const double* s_prev,
+                        double* A) {
+  if (band < 0) return ORC_ERR_INVALID;
+  int rc = orc_jacobian(cell, D, d_in, p, eps, x_t, s_prev, A);
+  if (rc) return rc;
+  for (int j = 0; j < D; ++j)
+    for (int k = 0; k < D; ++k)
+      if (abs(j - k) > band) A[(long)j * D + k] = 0.0;
+  return ORC_OK;
+}
+
+/* Nearest value of a binary format with `prec` significand bits (the
+ * leading one included) and normal exponents emin..emax, ties to even.
+ * Below 2^emin the spacing stays 2^(emin - prec + 1) (gradual underflow);
+ * a rounded magnitude above the largest finite value becomes infinite. */
+static double round_to_format(double v, int prec, int emin, int emax) {
+  if (v == 0.0 || !isfinite(v)) return v;
+  int e;
+  (void)frexp(v, &e);            /* |v| in [2^(e-1), 2^e) */
+  int lead = e - 1;              /* exponent of v's leading bit */
+  if (lead < emin) lead = emin;
+  /* scale so that one unit in the last place of the format is 1; the
+     scaling by a power of two is exact, nearbyint rounds ties to even in
+     the default rounding mode */
+  double q = nearbyint(ldexp(v, prec - 1 - lead));
+  double r = ldexp(q, lead - (prec - 1));
+  double maxv = ldexp(2.0 - ldexp(1.0, 1 - prec), emax);
+  if (fabs(r) > maxv) return copysign(INFINITY, v);
+  return r;
+}
+
+int orc_round_storage(int store, double* v, long n) {
+  int prec, emin, emax;
+  switch (store) {
+    case ORC_STORE_F64: return ORC_OK;
+    case ORC_STORE_F32: prec = 24; emin = -126; emax = 127; break;
+    case ORC_STORE_BF16: prec = 8; emin = -126; emax = 127; break;
+    case ORC_STORE_F16: prec = 11; emin = -14; emax = 15; break;
+    default: return ORC_ERR_INVALID;
+  }
+  for (long i = 0; i < n; ++i) v[i] = round_to_format(v[i], prec, emin, emax);
+  return ORC_OK;
+}
+
+static int mode_valid(int mode, int band) {
+  if (mode == ORC_BANDED) return band >= 0;
+  return mode >= ORC_JACOBI && mode <= ORC_NEWTON;
+}
+
+int orc_update_ex(int cell, int mode, int band, double damping, int D,
+                  int d_in, const double* p, double eps, int T, int B,
+                  const double* x, const double* s0, const double* s_cur,
+                  double* s_next, int nthreads) {
+  if (orc_param_count(cell, D, d_in) < 0 || T < 0 || B < 0) return ORC_ERR_INVALID;
+  if (!mode_valid(mode, band) || !(damping > 0.0 && damping <= 1.0)) return ORC_ERR_INVALID;
+  if (T == 0 || B == 0) return ORC_OK;
+  orc_job proto = {0};
+  proto.cell = cell; proto.mode = mode; proto.D = D; proto.d_in = d_in;
+  proto.T = T; proto.p = p; proto.eps = eps; proto.x = x; proto.s0 = s0;
+  proto.s_in = s_cur; proto.out = s_next; proto.band = band; proto.damping = damping;
+  return run_jobs(update_worker, &proto, B, nthreads, NULL);
+}
+
+/* One rung up the ladder of Jacobian approximations (adaptive switching). */
+static int stronger_mode(int mode, int band) {
+  switch (mode) {
+    case ORC_JACOBI:
+    case ORC_PICARD: return ORC_QUASI;
+    case ORC_QUASI: return band >= 1 ? ORC_BANDED : ORC_NEWTON;
+    default: return ORC_NEWTON;
+  }
+}
+
+/* The iteration over one block of contiguous sequences [B][T]: orc_iterate
+ * with the damping, adaptive switching and storage rounding of
+ * orc_iterate_ex.  history / modes receive at most hist_cap entries. */
+static int iterate_block(int cell, int mode, int band, double damping,
+                         int adapt, double stall, int store,
+                         double store_until, int D, int d_in, const double* p,
+                         double eps, int T, int B, const double* x,
+                         const double* s0, int max_iters, double tol,
+                         double* s_out, int* iters, double* resid,
+                         double* history, int* modes, int hist_cap,
+                         int nthreads) {
+  size_t n = (size_t)B * (size_t)T * (size_t)D;
+  double* other = (double*)malloc(sizeof(double) * (n ? n : 1));
+  double* F = (double*)malloc(sizeof(double) * (n ? n : 1));
+  if (!other || !F) { free(other); free(F); return ORC_ERR_NOMEM; }
+  for (int b = 0; b < B; ++b)
+    for (int t = 0; t < T; ++t)
+      memcpy(s_out + ((size_t)b * T + t) * D, s0 + (size_t)b * D, sizeof(double) * (size_t)D);
+  orc_round_storage(store, s_out, (long)n);   /* the initial guess is stored too */
+  double* cur = s_out;
+  double* nxt = other;
+  int status = ORC_NOT_CONVERGED;
+  int i = 0;
+  double r = 0.0, r_prev = 0.0;
+  for (;; ++i) {
+    int rc = orc_residual(cell, D, d_in, p, eps, T, B, x, s0, cur, F, &r, nthreads);
+    if (rc) { free(other); free(F); return rc; }
+    if (i < hist_cap) {
+      if (history) history[i] = r;
+      if (modes) modes[i] = -1;
+    }
+    if (!isfinite(r)) { status = ORC_ERR_NONFINITE; break; }
+    if (r <= tol) { status = ORC_OK; break; }
+    if (i >= max_iters) { status = ORC_NOT_CONVERGED; break; }
+    if (adapt && i >= 1 && r > stall * r_prev) mode = stronger_mode(mode, band);
+    if (modes && i < hist_cap) modes[i] = mode;
+    {
+      orc_job proto = {0};
+      proto.cell = cell; proto.mode = mode; proto.D = D; proto.d_in = d_in;
+      proto.T = T; proto.p = p; proto.eps = eps; proto.x = x; proto.s0 = s0;
+      proto.s_in = cur; proto.out = nxt; proto.F = F;
+      proto.band = band; proto.damping = damping;
+      rc = run_jobs(update_worker, &proto, B, nthreads, NULL);
+    }
+    if (rc) { free(other); free(F); return rc; }
+    if (r > store_until) orc_round_storage(store, nxt, (long)n);
+    double* tmp = cur; cur = nxt; nxt = tmp;
+    r_prev = r;
+  }
+  if (cur != s_out) memcpy(s_out, cur, sizeof(double) * n);
+  free(other);
+  free(F);
+  *iters = i;
+  *resid = r;
+  return status;
+}
+
+int orc_iterate_ex(int cell, int mode, int band, double damping, int adapt,
+                   double stall, int store, double store_until, int window,
+                   int D, int d_in, const double* p, double eps, int T, int B,
+                   const double* x, const double* s0, int max_iters,
+                   double tol, double* s_out, int* iters, double* resid,
+                   double* history, int* modes_used, int hist_cap,
+                   int* window_iters, int nthreads) {
+  if (orc_param_count(cell, D, d_in) < 0 || T < 0 || B < 0) return ORC_ERR_INVALID;
+  if (!mode_valid(mode, band) || !(damping > 0.0 && damping <= 1.0)) return ORC_ERR_INVALID;
+  if (max_iters < 0 || !(tol >= 0.0) || (adapt && !(stall >= 0.0))) return ORC_ERR_INVALID;
+  if (store < ORC_STORE_F64 || store > ORC_STORE_F16 || store_until != store_until) return ORC_ERR_INVALID;
+  if (hist_cap < 0) hist_cap = 0;
+  int Wn = (window <= 0 || window >= T) ? T : window;
+  int nwin = T == 0 ? 0 : (T + Wn - 1) / Wn;
+  size_t xw_n = (size_t)B * Wn * d_in, sw_n = (size_t)B * Wn * D, s0_n = (size_t)B * D;
+  double* xw = (double*)malloc(sizeof(double) * (xw_n ? xw_n : 1));
+  double* sw = (double*)malloc(sizeof(double) * (sw_n ? sw_n : 1));
+  double* s0w = (double*)malloc(sizeof(double) * (s0_n ? s0_n : 1));
+  if (!xw || !sw || !s0w) { free(xw); free(sw); free(s0w); return ORC_ERR_NOMEM; }
+  int status = ORC_OK, total = 0, hpos = 0;
+  double rmax = 0.0;
+  for (int w = 0; w < nwin; ++w) {
+    int t0 = w * Wn;
+    int L = T - t0 < Wn ? T - t0 : Wn;
+    for (int b = 0; b < B; ++b) {
+      memcpy(xw + (size_t)b * L * d_in, x + ((size_t)b * T + t0) * d_in, sizeof(double) * (size_t)L * d_in);
+      const double* init = w == 0 ? s0 + (size_t)b * D : s_out + ((size_t)b * T + t0 - 1) * D;
+      memcpy(s0w + (size_t)b * D, init, sizeof(double) * (size_t)D);
+    }
+    if (status == ORC_ERR_NONFINITE) {
+      /* an earlier window failed: this one keeps its initial guess */
+      for (int b = 0; b < B; ++b)
+        for (int t = 0; t < L; ++t)
+          memcpy(s_out + ((size_t)b * T + t0 + t) * D, s0w + (size_t)b * D, sizeof(double) * (size_t)D);
+      if (window_iters) window_iters[w] = 0;
+      continue;
+    }
+    int it = 0;
+    double r = 0.0;
+    int st = iterate_block(cell, mode, band, damping, adapt, stall, store, store_until, D,
+                           d_in, p, eps, L, B, xw, s0w, max_iters, tol, sw, &it, &r,
+                           history ? history + hpos : NULL, modes_used ? modes_used + hpos : NULL,
+                           hist_cap - hpos, nthreads);
+    if (st == ORC_ERR_INVALID || st == ORC_ERR_NOMEM) { free(xw); free(sw); free(s0w); return st; }
+    for (int b = 0; b < B; ++b)
+      memcpy(s_out + ((size_t)b * T + t0) * D, sw + (size_t)b * L * D, sizeof(double) * (size_t)L * D);
+    if (window_iters) window_iters[w] = it;
+    hpos += (it + 1 < hist_cap - hpos) ? it + 1 : hist_cap - hpos;
+    total += it;
+    if (r != r) rmax = r;                 /* NaN sticks */
+    else if (rmax == rmax && r > rmax) rmax = r;
+    if (st == ORC_ERR_NONFINITE) status = ORC_ERR_NONFINITE;
+    else if (st == ORC_NOT_CONVERGED && status == ORC_OK) status = ORC_NOT_CONVERGED;
+  }
+  free(xw);
+  free(sw);
+  free(s0w);
+  *iters = total;
+  *resid = rmax;
+  return status;
 }

@@ -25,13 +25,19 @@
  *   - the full iteration with the stop rule r^(i) = max|F(s^(i))| <= tol
  *     (page §5.3, residual monitoring; the norm and tie-break are a reading).
  *   - a serial affine recurrence s_t = A_t s_{t-1} + b_t, the object the
- *     parallel scan of page §2.1 evaluates.
+ *     parallel scan of page §2.1 evaluates;
+ *   - the page's refinements of the iteration: a banded Jacobian
+ *     approximation (page §2.2.2), damping (page §4.3, §5.3), adaptive
+ *     switching to a more exact approximation when the residual stalls
+ *     (page §5.3), reduced-precision storage of the iterate (page §2.3) and
+ *     a windowed solve (page §1.3.1, §2.3); the readings are stated at
+ *     orc_iterate_ex.
  *
  * Parity status: every function here is pinned by the CPU tests (library
  * cells, finite differences, a dense linear solve of J~ delta = -F,
- * causality, closed forms).  The iteration COUNTS at the benchmark sizes
- * are pinned only through those pins of the update step; the page prints no
- * count for them.
+ * causality, closed forms, numpy's and PyTorch's float conversions).  The
+ * iteration COUNTS at the benchmark sizes are pinned only through those pins
+ * of the update step; the page prints no count for them.
  */
 #ifndef PN_ORACLE_H
 #define PN_ORACLE_H
@@ -41,7 +47,9 @@ extern "C" {
 #endif
 
 enum { ORC_TANH_RNN = 0, ORC_GRU = 1, ORC_EULER = 2 };
-enum { ORC_JACOBI = 0, ORC_PICARD = 1, ORC_QUASI = 2, ORC_NEWTON = 3 };
+enum { ORC_JACOBI = 0, ORC_PICARD = 1, ORC_QUASI = 2, ORC_NEWTON = 3, ORC_BANDED = 4 };
+/* formats the stored iterate can be rounded to (round to nearest, ties to even) */
+enum { ORC_STORE_F64 = 0, ORC_STORE_F32 = 1, ORC_STORE_BF16 = 2, ORC_STORE_F16 = 3 };
 enum {
   ORC_OK = 0,
   ORC_NOT_CONVERGED = 1,
@@ -97,6 +105,75 @@ int orc_iterate(int cell, int mode, int D, int d_in, const double* p,
                 double eps, int T, int B, const double* x, const double* s0,
                 int max_iters, double tol, double* s_out, int* iters,
                 double* resid, double* history, int hist_cap, int nthreads);
+
+/* ---- extensions of the iteration (the page's optimisation sections) ----
+ *
+ * Banded Jacobian approximation (page §2.2.2): A~ keeps the entries of
+ * df_t/ds with |j - k| <= band and zeroes the rest.  band = 0 is the
+ * diagonal (quasi-Newton); band >= D - 1 is the full Jacobian (Newton). */
+int orc_banded_jacobian(int cell, int band, int D, int d_in, const double* p,
+                        double eps, const double* x_t, const double* s_prev,
+                        double* A);
+
+/* Round n values in place to a storage format (ORC_STORE_*), to nearest
+ * with ties to even, overflow to +-inf, gradual underflow (IEEE 754
+ * binary32 / binary16; bfloat16 = binary32's exponent range with an
+ * 8-bit significand).  ORC_STORE_F64 leaves the values unchanged. */
+int orc_round_storage(int store, double* v, long n);
+
+/* orc_update with a mode that may be ORC_BANDED (with its band) and a
+ * damping factor lambda in (0, 1]: s_next = s_cur + lambda * delta, where
+ * delta solves J~ delta = -F(s_cur) as in orc_update (page §4.3 and §5.3
+ * name damping as the remedy for a stalled iteration). */
+int orc_update_ex(int cell, int mode, int band, double damping, int D,
+                  int d_in, const double* p, double eps, int T, int B,
+                  const double* x, const double* s0, const double* s_cur,
+                  double* s_next, int nthreads);
+
+/* The full iteration with the page's optional refinements.  With
+ * band = 0, damping = 1, adapt = 0, store = ORC_STORE_F64 and window <= 0
+ * it is orc_iterate.
+ *
+ *   mode, band   starting approximation (ORC_JACOBI..ORC_BANDED).
+ *   damping      lambda in (0, 1] applied to every update.
+ *   adapt, stall adaptive switching (page §5.3: when the residual curve
+ *                stalls, move to a more exact Jacobian approximation).
+ *                Reading: after the residual r^(i) (i >= 1) is measured,
+ *                if r^(i) > stall * r^(i-1) the mode moves one rung up the
+ *                ladder jacobi/picard -> quasi -> banded (only when
+ *                band >= 1) -> newton before update i is taken; newton
+ *                stays newton.
+ *   store,       reduced-precision iterate storage (page §2.3: states kept
+ *   store_until  in a narrow format, arithmetic in a wider one).  The
+ *                initial guess, and every iterate s^(i+1) whose
+ *                predecessor's residual r^(i) > store_until, is rounded to
+ *                the format before it is stored; the residual and the
+ *                update are then computed in double from the stored values.
+ *   window       windowed solve (page §1.3.1: the long sequence is split
+ *                into blocks that fit in memory; page §2.3, chunks such as
+ *                1024 steps).  Reading: t = 1..T is cut into consecutive
+ *                windows of `window` steps (the last one ragged); each is
+ *                solved in turn by the iteration above, from the start
+ *                mode, with its initial state the last state of the
+ *                previous window, until its own residual max-norm <= tol or
+ *                max_iters.  window <= 0 or >= T: one window.
+ *
+ * Results: s_out [B][T][D]; *iters = iterations summed over windows;
+ * *resid = the largest final window residual, which is the max-norm of F
+ * over the whole sequence; status OK when every window converged,
+ * NOT_CONVERGED when one ran out of iterations (the next windows still
+ * run), NONFINITE when a residual is not finite (the windows after it keep
+ * their initial guess).  history[] / modes_used[] hold, window after
+ * window, each measured residual and the mode of the update that followed
+ * it (-1 after a window's last residual), hist_cap entries at most;
+ * window_iters[w] (may be NULL) each window's count. */
+int orc_iterate_ex(int cell, int mode, int band, double damping, int adapt,
+                   double stall, int store, double store_until, int window,
+                   int D, int d_in, const double* p, double eps, int T, int B,
+                   const double* x, const double* s0, int max_iters,
+                   double tol, double* s_out, int* iters, double* resid,
+                   double* history, int* modes_used, int hist_cap,
+                   int* window_iters, int nthreads);
 
 /* s[t] = A[t] s[t-1] + b[t] for t = 0..T-1 with s_init before t = 0.
  * A: [T][D][D], b: [T][D], s: [T][D].  A serial loop. */
