@@ -153,6 +153,40 @@ PN_API pn_status pn_eval_host_many(pn_handle h, int n, const float* const* x_hos
                                    float tol, float* const* states_host, int* iters_out,
                                    float* resid_out);
 
+/* Windowed solve of a sequence longer than the handle (web article "并行牛顿
+ * 方法：加速非线性序列评估的计算革命", §1.3.1, the long sequence split into
+ * blocks that fit in memory, and §2.3, chunked computation).  Steps
+ * t = 1..T_total are cut into consecutive windows of W = h's T steps; each
+ * window is solved in turn by pn_eval's iteration, with the previous
+ * window's last state as its s0 and its own stop rule (residual max-norm
+ * over the window and the batch <= tol, or max_iters), so the result is the
+ * windowed result of the oracle's orc_iterate_ex.
+ *   h        handle; its T is the window length W
+ *   tail     handle for the last window when W does not divide T_total: same
+ *            cell, D, d_in, B, eps, device, stream and PARAMETERS as h (the
+ *            parameters cannot be checked: the caller's responsibility),
+ *            T = T_total mod W; must be NULL when W divides T_total
+ *   T_total  >= 1
+ *   x        device [B][T_total][d_in];  s0 device [B][D]
+ *   states   device [B][T_total][D], written window by window
+ *   iters_out     host; the iterations summed over the windows (may be NULL)
+ *   resid_out     host; the largest final window residual, which is the
+ *                 residual max-norm over the whole sequence (may be NULL)
+ *   window_iters  host array of n_window_cap ints (may be NULL); receives
+ *                 each window's count, in order, as far as it reaches
+ * Each window's x slice and initial state are staged with strided device
+ * copies into h's host-evaluation buffers (allocated on first use, as for
+ * pn_eval_host), and its states are copied back, all on h's stream.
+ * Returns PN_OK when every window converged; PN_NOT_CONVERGED when some
+ * window used up max_iters (the windows after it still run); the first
+ * error otherwise: PN_ERR_NONFINITE leaves the windows after the failing
+ * one unwritten.  Afterwards pn_get_residual_history on h (or tail) reports
+ * the last window that handle solved. */
+PN_API pn_status pn_eval_windowed(pn_handle h, pn_handle tail, int T_total, const float* x,
+                                  const float* s0, pn_mode mode, int max_iters, float tol,
+                                  float* states, int* iters_out, float* resid_out,
+                                  int* window_iters, int n_window_cap);
+
 /* Copy min(n, iters+1) residuals r^(0..iters) of the last evaluation into the
  * host array out; *n_written (may be NULL) receives the count. */
 PN_API pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written);

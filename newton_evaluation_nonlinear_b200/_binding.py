@@ -46,6 +46,8 @@ SIGNATURES = {
     "pn_eval_host": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_float, _vp, ctypes.POINTER(_c_int),
                               ctypes.POINTER(_c_float)]),
     "pn_eval_host_many": (_c_int, [_vp, _c_int, _vp, _vp, _c_int, _c_int, _c_float, _vp, _vp, _vp]),
+    "pn_eval_windowed": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _c_float, _vp,
+                                  ctypes.POINTER(_c_int), ctypes.POINTER(_c_float), _vp, _c_int]),
     "pn_get_residual_history": (_c_int, [_vp, _vp, _c_int, ctypes.POINTER(_c_int)]),
     "pn_time_iterations": (_c_int, [_vp, _c_int, _c_int, ctypes.POINTER(_c_float)]),
     "pn_get_stats": (_c_int, [_vp, ctypes.POINTER(pn_stats)]),
@@ -139,6 +141,16 @@ def pn_eval_host_many(h: int, xs, s0s, mode: int, max_iters: int, tol: float, st
     st = lib.pn_eval_host_many(h, n, px, ps0, int(mode), int(max_iters), float(tol), pst, its.ctypes.data,
                                rs.ctypes.data)
     return st, its[:n], rs[:n]
+
+
+def pn_eval_windowed(h: int, tail: Optional[int], T_total: int, x_ptr: int, s0_ptr: int, mode: int,
+                     max_iters: int, tol: float, states_ptr: int, n_window_cap: int):
+    """Returns (status, total iters, resid, per-window iters[:n_window_cap])."""
+    it, r = _c_int(-1), _c_float(float("nan"))
+    wit = np.full(max(int(n_window_cap), 1), -1, np.int32)
+    st = lib.pn_eval_windowed(h, tail, int(T_total), x_ptr, s0_ptr, int(mode), int(max_iters), float(tol),
+                              states_ptr, ctypes.byref(it), ctypes.byref(r), wit.ctypes.data, int(n_window_cap))
+    return st, it.value, r.value, wit[:max(int(n_window_cap), 0)]
 
 
 def pn_get_residual_history(h: int, n: int) -> Tuple[int, np.ndarray]:
@@ -265,6 +277,27 @@ class Solver:
         st, its, rs = pn_eval_host_many(self.h, xs, s0s, mode, max_iters, tol, states_list)
         self._check(st)
         return states_list, its, rs, st
+
+    def eval_windowed(self, x, s0, mode, max_iters: Optional[int] = None, tol: float = 1e-5,
+                      tail: Optional["Solver"] = None, states=None):
+        """Solve a sequence of T_total = x.shape[1] steps window by window, this solver's T being
+        the window length; ``tail`` is a Solver for the last T_total % T steps (same cell, shapes,
+        parameters and stream).  Returns (states, iters, resid, status, window_iters)."""
+        import torch
+        mode = MODES[mode] if isinstance(mode, str) else int(mode)
+        max_iters = self.T if max_iters is None else int(max_iters)
+        T_total = int(x.shape[1]) if x.dim() == 3 else -1
+        if states is None:
+            states = torch.empty((self.B, max(T_total, 0), self.D), device=x.device, dtype=torch.float32)
+        for name, t, shape in (("x", x, (self.B, T_total, self.d_in)), ("s0", s0, (self.B, self.D)),
+                               ("states", states, (self.B, T_total, self.D))):
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
+                raise ValueError(f"{name} must be a contiguous CUDA float32 tensor of shape {shape}")
+        nwin = -(-T_total // self.T)
+        st, it, r, wit = pn_eval_windowed(self.h, tail.h if tail is not None else None, T_total, x.data_ptr(),
+                                          s0.data_ptr(), mode, max_iters, tol, states.data_ptr(), nwin)
+        self._check(st)
+        return states, it, r, st, wit
 
     def residual_history(self, n: int = 1 << 16) -> np.ndarray:
         st, h = pn_get_residual_history(self.h, n)

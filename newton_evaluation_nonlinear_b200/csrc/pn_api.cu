@@ -953,6 +953,92 @@ pn_status pn_eval_host_many(pn_handle h, int n, const float* const* x_host, cons
   return result;
 }
 
+pn_status pn_eval_windowed(pn_handle h, pn_handle tail, int T_total, const float* x, const float* s0,
+                           pn_mode mode, int max_iters, float tol, float* states, int* iters_out,
+                           float* resid_out, int* window_iters, int n_window_cap) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  DeviceGuard dg(h->device);
+  pn_status st = validate_mode(h, mode, max_iters, tol);
+  if (st != PN_OK) return st;
+  if (T_total < 1) return fail(h, PN_ERR_INVALID, "T_total = %d < 1", T_total);
+  if ((long long)h->B * T_total > INT_MAX) return fail(h, PN_ERR_INVALID, "B*T_total must fit in int");
+  if (n_window_cap < 0 || (n_window_cap > 0 && !window_iters)) return fail(h, PN_ERR_INVALID, "bad window_iters array");
+  const int W = h->T;
+  const int rem = T_total % W;
+  if (rem == 0 && tail) return fail(h, PN_ERR_INVALID, "tail must be NULL when the window length %d divides T_total", W);
+  if (rem != 0) {
+    if (!tail) return fail(h, PN_ERR_INVALID, "T_total %% %d = %d needs a tail handle", W, rem);
+    if (tail == h || tail->T != rem || tail->cell != h->cell || tail->D != h->D || tail->d_in != h->d_in ||
+        tail->B != h->B || tail->eps != h->eps || tail->device != h->device || tail->stream != h->stream)
+      return fail(h, PN_ERR_INVALID, "tail handle must match (cell, D, d_in, B, eps, device, stream) with T = %d", rem);
+    if ((st = validate_mode(tail, mode, max_iters, tol)) != PN_OK)
+      return fail(h, st, "tail: %s", tail->err.c_str());
+  }
+  if ((st = check_device_ptr(h, x, "x")) != PN_OK) return st;
+  if ((st = check_device_ptr(h, s0, "s0")) != PN_OK) return st;
+  if ((st = check_device_ptr(h, states, "states")) != PN_OK) return st;
+  const int B = h->B, D = h->D, d_in = h->d_in;
+  if (!h->hx) {   // staging of one window, shared with pn_eval_host (the tail's windows are shorter)
+    if ((st = dalloc(h, &h->hx, (size_t)B * W * d_in)) != PN_OK) return st;
+    if ((st = dalloc(h, &h->hs0, (size_t)B * D)) != PN_OK) return st;
+    if ((st = dalloc(h, &h->hst, (size_t)B * W * D)) != PN_OK) return st;
+  }
+  const size_t fsz = sizeof(float);
+  const int nwin = (T_total + W - 1) / W;
+  long long total = 0;
+  float rmax = 0.0f;
+  pn_status result = PN_OK;
+  for (int w = 0; w < nwin; ++w) {
+    const int t0 = w * W;
+    const int L = std::min(W, T_total - t0);
+    pn_ctx* hh = (L == W) ? h : tail;
+    // x[:, t0:t0+L, :] -> staging [B][L][d_in]
+    PN_CUDA(h, cudaMemcpy2DAsync(h->hx, (size_t)L * d_in * fsz, x + (size_t)t0 * d_in, (size_t)T_total * d_in * fsz,
+                                 (size_t)L * d_in * fsz, (size_t)B, cudaMemcpyDeviceToDevice, h->stream));
+    // the window's initial state: s0, or states[:, t0-1, :]
+    if (w == 0)
+      PN_CUDA(h, cudaMemcpyAsync(h->hs0, s0, (size_t)B * D * fsz, cudaMemcpyDeviceToDevice, h->stream));
+    else
+      PN_CUDA(h, cudaMemcpy2DAsync(h->hs0, (size_t)D * fsz, states + (size_t)(t0 - 1) * D, (size_t)T_total * D * fsz,
+                                   (size_t)D * fsz, (size_t)B, cudaMemcpyDeviceToDevice, h->stream));
+    Args& a = *hh->args_h;
+    a.x = h->hx;
+    a.s0 = h->hs0;
+    a.states = h->hst;
+    a.tol = tol;
+    a.max_iters = max_iters;
+    a.timeout_ns = hh->timeout_ns;
+    a.stall_ticket = hh->stall_ticket;
+    int it = -1;
+    float r = NAN;
+    st = run_eval(hh, mode, &it, &r);   // returns after the window is solved (stream synchronised)
+    if (st < 0 && st != PN_ERR_NONFINITE) {
+      if (hh != h) return fail(h, st, "window %d (tail): %s", w, tail->err.c_str());
+      return st;
+    }
+    // staging [B][L][D] -> states[:, t0:t0+L, :]
+    PN_CUDA(h, cudaMemcpy2DAsync(states + (size_t)t0 * D, (size_t)T_total * D * fsz, h->hst, (size_t)L * D * fsz,
+                                 (size_t)L * D * fsz, (size_t)B, cudaMemcpyDeviceToDevice, h->stream));
+    if (w < n_window_cap) window_iters[w] = it;
+    total += it;
+    if (r != r) rmax = r;                 // NaN sticks
+    else if (rmax == rmax && r > rmax) rmax = r;
+    if (st == PN_ERR_NONFINITE) {
+      result = PN_ERR_NONFINITE;
+      if (hh != h) fail(h, st, "window %d (tail): %s", w, tail->err.c_str());
+      else fail(h, st, "window %d: %s", w, std::string(h->err).c_str());
+      break;
+    }
+    if (st == PN_NOT_CONVERGED) result = PN_NOT_CONVERGED;
+  }
+  cudaError_t e = cudaStreamSynchronize(h->stream);
+  if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "windowed solve: %s", cudaGetErrorString(e));
+  if (iters_out) *iters_out = (int)std::min<long long>(total, INT_MAX);
+  if (resid_out) *resid_out = rmax;
+  if (result != PN_ERR_NONFINITE) h->err.clear();
+  return result;
+}
+
 pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written) {
   if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
   if (n < 0 || (n > 0 && !out)) return fail(h, PN_ERR_INVALID, "bad output buffer");

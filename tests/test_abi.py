@@ -67,5 +67,7 @@ def test_argument_validation_without_gpu():
         raise AssertionError("mismatched batch lists accepted")
     except ValueError:
         pass
+    st, it, r, wit = pn.pn_eval_windowed(None, None, 32, 0, 0, 0, 1, 1e-5, 0, 2)
+    assert st == pn.PN_ERR_INVALID and "NULL" in pn.pn_last_error(None) and len(wit) == 2
     pn.pn_destroy(None)
     assert pn.pn_version().startswith("libpn")
