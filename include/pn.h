@@ -28,8 +28,9 @@
  *    host memory.  The caller owns every pointer it passes; the library never
  *    frees or retains them past the call.
  *  - Work is ordered on the handle's stream (set at pn_create or with
- *    pn_set_stream).  pn_eval and pn_eval_host synchronise that stream before
- *    returning, so every output is complete on return.
+ *    pn_set_stream).  Every evaluation entry point (pn_eval, pn_eval_host,
+ *    pn_eval_host_many, pn_eval_windowed, pn_eval_static) synchronises that
+ *    stream before returning, so every output is complete on return.
  *  - Errors are reported by the return code; pn_last_error gives the text.
  *    A handle is not thread-safe: one call at a time per handle.
  */
@@ -90,7 +91,10 @@ typedef struct {
   long long iteration_launches;  /* fused iteration kernels launched           */
   long long iteration_ns;        /* their summed device durations (first CTA
                                     start to last CTA end, %globaltimer)       */
-  long long evals;               /* completed pn_eval / pn_eval_host calls     */
+  long long evals;               /* completed evaluations: one per pn_eval or
+                                    pn_eval_host call, per batch of
+                                    pn_eval_host_many, per window of
+                                    pn_eval_windowed                            */
 } pn_stats;
 
 /* Supported sizes: 1 <= D <= 256 for PN_JACOBI/PN_PICARD/PN_QUASI and
@@ -187,8 +191,10 @@ PN_API pn_status pn_eval_windowed(pn_handle h, pn_handle tail, int T_total, cons
                                   float* states, int* iters_out, float* resid_out,
                                   int* window_iters, int n_window_cap);
 
-/* Copy min(n, iters+1) residuals r^(0..iters) of the last evaluation into the
- * host array out; *n_written (may be NULL) receives the count. */
+/* Copy min(n, iters+1, 65537) residuals r^(0..) of the handle's last
+ * evaluation into the host array out (n >= 0 entries; may be NULL when
+ * n == 0); *n_written (may be NULL) receives the count, 0 before the first
+ * evaluation.  PN_ERR_INVALID for a NULL handle or a bad array. */
 PN_API pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_written);
 
 /* Time the fused iteration kernel of `mode` alone: after a pn_eval on this
@@ -202,9 +208,23 @@ PN_API pn_status pn_get_residual_history(pn_handle h, float* out, int n, int* n_
  * overwritten with later iterates. */
 PN_API pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* avg_ms);
 
+/* Fill *out (host) with the handle's counters; synchronises the handle's
+ * stream first.  PN_ERR_INVALID for a NULL handle or out. */
 PN_API pn_status pn_get_stats(pn_handle h, pn_stats* out);
+
+/* Zero the handle's counters (after synchronising its stream). */
 PN_API pn_status pn_reset_stats(pn_handle h);
+
+/* Set one pn_option.  Values: PN_OPT_WAIT_TIMEOUT_NS >= 1000;
+ * PN_OPT_DEBUG_STALL_TICKET -1 or a ticket >= 0; PN_OPT_DEVICE_LOOP and
+ * PN_OPT_TENSOR_CORES 0 or 1 (tensor cores: ignored where the shape has no
+ * tensor-core kernel; switching re-selects the kernels after synchronising the
+ * stream).  Anything else: PN_ERR_INVALID, the handle unchanged. */
 PN_API pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
+
+/* Order the handle's later work on cuda_stream (a cudaStream_t; NULL = the
+ * legacy default stream).  The caller keeps the stream alive while the handle
+ * uses it and orders it against earlier work itself. */
 PN_API pn_status pn_set_stream(pn_handle h, void* cuda_stream);
 
 /* pn_eval without allocation, for the tanh RNN cell and the diagonal modes.
@@ -246,8 +266,10 @@ PN_API pn_status pn_activation(int which, const float* x, float* y, long long n,
  * evaluation), 0 when pn_eval launches it once per iteration. */
 PN_API int pn_dim(pn_handle h, int which);
 
-/* Last error message of this handle, or of the calling thread's last failed
- * pn_create when h is NULL.  Never NULL; "" when there was no error. */
+/* Last error message of this handle; with h NULL, the calling thread's last
+ * error that had no handle to go to (pn_create, pn_eval_static,
+ * pn_activation, or any call given a NULL handle).  Never NULL; "" when there
+ * was no error. */
 PN_API const char* pn_last_error(pn_handle h);
 
 /* Release every device and host resource of the handle (NULL is a no-op). */
