@@ -202,13 +202,42 @@ def cpu_sample(prob, mode, b_sample):
     return prob.T * b_sample / wall, wall, it, threads
 
 
+def cpu_sequential(prob, b_sample, threads):
+    """The oracle's plain sequential loop s_t = f_t(s_{t-1}) on the first b_sample sequences."""
+    import oracle
+    m = oracle.Model.from_problem(prob)
+    x = np.ascontiguousarray(prob.x[:b_sample])
+    s0 = np.ascontiguousarray(prob.s0[:b_sample])
+    t0 = time.perf_counter()
+    m.sequential(x, s0, nthreads=threads)
+    return prob.T * b_sample / (time.perf_counter() - t0)
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(prob, mode):
     b_sample = max(1, min(prob.B, os.cpu_count() or 1))
     v, wall, it, threads = cpu_sample(prob, mode, b_sample)
+    # context: the sequential loop the method replaces, on the same sample and threads, and on one
+    # sequence with one thread
+    seq = cpu_sequential(prob, b_sample, threads)
+    seq1 = cpu_sequential(prob, 1, 1)
     return {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"fp64 oracle {pi.MODE_NAMES[mode]} iteration (serial over t, threads over b) on the "
                       f"first {b_sample} of {prob.B} sequences at full T={prob.T}: {it} iterations, "
-                      f"{wall:.1f} s wall"}
+                      f"{wall:.1f} s wall",
+            "sequential": {"value": seq, "unit": UNIT, "cores": threads, "value_1_thread_1_sequence": seq1},
+            "cpu_model": cpu_model(), "nproc": os.cpu_count()}
 
 
 def reference_arm(args, prob, mode, rank, world):
