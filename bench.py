@@ -12,11 +12,13 @@ barrier + device synchronisation on both sides, timed with CUDA events; for N>1
 own copy of the workload (independent problem instances, no collective in the
 data path: weak scaling) and the time is the max over ranks.
 
-Also reported, on rank 0: the end-to-end number through pn_eval_host with the
-host<->device copies inside the timed region; the roofline of the fused
-iteration kernel (algorithmic bytes per launch / its mean launch time, CUDA
-events around back-to-back launches on the library's stream); and the fp64
-oracle timed on this host's cores on a bounded sample of the same workload.
+Also reported, on rank 0: the end-to-end number through pn_eval_host_many
+(K batches from pinned host buffers, every batch's host<->device copies inside
+the timed region, overlapped with the neighbouring batches' evaluations); the
+roofline of the fused iteration kernel (algorithmic bytes per iteration / its
+mean time per iteration, CUDA events on the library's stream); and the fp64
+oracle timed on this host's cores on a bounded sample of the same workload,
+with the oracle's plain sequential loop beside it for context.
 ``--impl reference`` times that oracle alone as the reference arm.
 """
 from __future__ import annotations
