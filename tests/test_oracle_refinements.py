@@ -350,3 +350,33 @@ def test_windowed_failure_and_budget():
     np.testing.assert_array_equal(s[:, 16:], np.repeat(s[:, 15:16], 8, axis=1))
     good = m.iterate_ex(pi.MODE_QUASI, prob.x, prob.s0, T, 1e-12, window=window)
     np.testing.assert_array_equal(s[:, :8], good[0][:, :8])
+
+
+def test_refinements_combine_per_window():
+    """Windows are independent solves: with adaptive switching every window restarts from the
+    start mode, and a window's own schedule follows the rule on its own residuals."""
+    T, window = 60, 20
+    prob = pi.random_problem(171, pi.CELL_EULER, 6, T=T, B=2, rho=0.9, s0_scale=0.3, eps=0.05)
+    m = oracle.Model.from_problem(prob)
+    s, it, r, st, hist, modes, wit = m.iterate_ex(pi.MODE_JACOBI, prob.x, prob.s0, T, 1e-10, adapt=True,
+                                                  stall=0.5, damping=0.9, window=window)
+    assert st == oracle.OK and len(wit) == 3
+    pos = 0
+    for w in wit:
+        h, md = hist[pos:pos + w + 1], modes[pos:pos + w + 1]
+        assert md[0] == pi.MODE_JACOBI and md[-1] == -1
+        assert md.tolist() == _expected_schedule(pi.MODE_JACOBI, 0, 0.5, h)
+        pos += w + 1
+    np.testing.assert_allclose(s, m.sequential(prob.x, prob.s0), rtol=0, atol=1e-8)
+
+
+def test_refinements_do_not_depend_on_threads():
+    prob = pi.random_problem(172, pi.CELL_GRU, 5, 3, T=45, B=5, rho=0.9, s0_scale=0.3)
+    m = oracle.Model.from_problem(prob)
+    kw = dict(band=1, damping=0.8, adapt=True, stall=0.6, store=oracle.STORE_F32, store_until=1e-4, window=16)
+    a = m.iterate_ex(pi.MODE_PICARD, prob.x, prob.s0, 45, 1e-9, nthreads=1, **kw)
+    b = m.iterate_ex(pi.MODE_PICARD, prob.x, prob.s0, 45, 1e-9, nthreads=4, **kw)
+    assert a[1:4] == b[1:4]
+    for x, y in zip(a[4:], b[4:]):
+        np.testing.assert_array_equal(x, y)
+    np.testing.assert_array_equal(a[0], b[0])
