@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--mode", default=None, help="jacobi|picard|quasi|newton (default: the workload's first)")
     ap.add_argument("--all", action="store_true", help="one line per workload and mode (report runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--window", type=int, default=0,
+                    help="time the windowed solve (pn_eval_windowed) with windows of this many steps instead")
     ap.add_argument("--host-loop", action="store_true",
                     help="host-driven convergence loop (plain kernel launches, e.g. for ncu) instead of the "
                          "device-side CUDA graph loop")
@@ -386,6 +388,65 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
     return line
 
 
+def bench_windowed(args, prob, mode, rank, world, local_rank, dist):
+    """The same metric for the windowed solve: each step solves the whole sequence window by
+    window (windows of args.window steps, the ragged last one by a second handle)."""
+    import torch
+
+    import newton_evaluation_nonlinear_b200 as pn
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    W = min(int(args.window), prob.T)
+    rem = prob.T % W
+    win = pn.Solver(prob.cell, prob.D, prob.d_in, W, prob.B, prob.params, prob.eps, stream=stream, device=dev)
+    tail = (pn.Solver(prob.cell, prob.D, prob.d_in, rem, prob.B, prob.params, prob.eps, stream=stream, device=dev)
+            if rem else None)
+    x = torch.from_numpy(prob.x).to(dev)
+    s0 = torch.from_numpy(prob.s0).to(dev)
+    states = torch.empty((prob.B, prob.T, prob.D), device=dev, dtype=torch.float32)
+    mi, tol = min(prob.iters_cap, W), prob.tol
+    for _ in range(max(3, args.warmup)):
+        _, iters, resid, st, wit = win.eval_windowed(x, s0, mode, mi, tol, tail=tail, states=states)
+    torch.cuda.synchronize(dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        clk.mark_start()
+        e0.record(stream)
+        for _ in range(args.steps):
+            _, iters, resid, st, wit = win.eval_windowed(x, s0, mode, mi, tol, tail=tail, states=states)
+        e1.record(stream)
+        barrier()
+        clk.mark_end()
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    nwin = len(wit)
+    looping = pn.pn_dim(win.h, 5 + mode) == 1
+    per_window = [(1 if looping else int(n) + 1) + 2 + (0 if prob.cell == pi.CELL_EULER else 1) for n in wit]
+    line = {"metric": METRIC, "value": job_throughput(prob.T * prob.B * args.steps, world, ms), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": prob.name + f"_window{W}", "mode": pi.MODE_NAMES[mode],
+                       "cell": pi.CELL_NAMES[prob.cell], "D": prob.D, "d_in": prob.d_in, "T": prob.T,
+                       "B": prob.B, "tol": prob.tol, "max_iters_per_window": mi, "window": W,
+                       "windows": nwin, "iters": iters, "window_iters": [int(n) for n in wit],
+                       "final_resid": resid, "status": st,
+                       "parallelism": f"independent instances x{world}",
+                       "l2": "inputs larger than L2 (the whole sequence is read and written once per step)"},
+            "clocks": clk.summary(), "gpu_launches": sum(per_window) * args.steps}
+    win.close()
+    if tail is not None:
+        tail.close()
+    return line
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -416,9 +477,12 @@ def main():
             if args.impl == "reference":
                 reference_arm(args, prob, mode, rank, world)
                 continue
-            line = bench_pn(args, prob, mode, rank, world, local_rank, dist)
+            if args.window > 0:
+                line = bench_windowed(args, prob, mode, rank, world, local_rank, dist)
+            else:
+                line = bench_pn(args, prob, mode, rank, world, local_rank, dist)
             if rank == 0:
-                if world == 1 and not args.no_cpu_baseline:
+                if world == 1 and not args.no_cpu_baseline and args.window <= 0:
                     line["cpu_baseline"] = cpu_baseline(prob, mode)
                 print(json.dumps(line), flush=True)
     finally:
