@@ -403,6 +403,17 @@ int orc_update(int cell, int mode, int D, int d_in, const double* p,
   return run_jobs(update_worker, &proto, B, nthreads, NULL);
 }
 
+static int iterate_block(int cell, int mode, int band, double damping,
+                         int adapt, double stall, int store,
+                         double store_until, int D, int d_in, const double* p,
+                         double eps, int T, int B, const double* x,
+                         const double* s0, int max_iters, double tol,
+                         double* s_out, int* iters, double* resid,
+                         double* history, int* modes, int hist_cap,
+                         int nthreads);
+
+/* The plain iteration is the general loop below (iterate_block) with every
+ * refinement off: no band, no damping, no switching, double storage. */
 int orc_iterate(int cell, int mode, int D, int d_in, const double* p,
                 double eps, int T, int B, const double* x, const double* s0,
                 int max_iters, double tol, double* s_out, int* iters,
@@ -410,42 +421,14 @@ int orc_iterate(int cell, int mode, int D, int d_in, const double* p,
   if (orc_param_count(cell, D, d_in) < 0 || T < 0 || B < 0) return ORC_ERR_INVALID;
   if (mode < ORC_JACOBI || mode > ORC_NEWTON) return ORC_ERR_INVALID;
   if (max_iters < 0 || !(tol >= 0.0)) return ORC_ERR_INVALID;
-  size_t n = (size_t)B * (size_t)T * (size_t)D;
-  double* other = (double*)malloc(sizeof(double) * (n ? n : 1));
-  double* F = (double*)malloc(sizeof(double) * (n ? n : 1));
-  if (!other || !F) { free(other); free(F); return ORC_ERR_NOMEM; }
-  /* initial guess: s^(0)_t = s0 for every t (a reading; the page is silent) */
-  for (int b = 0; b < B; ++b)
-    for (int t = 0; t < T; ++t)
-      memcpy(s_out + ((size_t)b * T + t) * D, s0 + (size_t)b * D, sizeof(double) * (size_t)D);
-  double* cur = s_out;
-  double* nxt = other;
-  int status = ORC_NOT_CONVERGED;
-  int i = 0;
+  int it = 0;
   double r = 0.0;
-  for (;; ++i) {
-    int rc = orc_residual(cell, D, d_in, p, eps, T, B, x, s0, cur, F, &r, nthreads);
-    if (rc) { free(other); free(F); return rc; }
-    if (history && i < hist_cap) history[i] = r;
-    if (!isfinite(r)) { status = ORC_ERR_NONFINITE; break; }
-    if (r <= tol) { status = ORC_OK; break; }
-    if (i >= max_iters) { status = ORC_NOT_CONVERGED; break; }
-    {
-      orc_job proto = {0};
-      proto.cell = cell; proto.mode = mode; proto.D = D; proto.d_in = d_in;
-      proto.T = T; proto.p = p; proto.eps = eps; proto.x = x; proto.s0 = s0;
-      proto.s_in = cur; proto.out = nxt; proto.F = F; proto.damping = 1.0;
-      rc = run_jobs(update_worker, &proto, B, nthreads, NULL);
-    }
-    if (rc) { free(other); free(F); return rc; }
-    double* tmp = cur; cur = nxt; nxt = tmp;
-  }
-  if (cur != s_out) memcpy(s_out, cur, sizeof(double) * n);
-  free(other);
-  free(F);
-  if (iters) *iters = i;
+  int st = iterate_block(cell, mode, 0, 1.0, 0, 0.0, ORC_STORE_F64, 0.0, D, d_in, p, eps, T, B, x, s0,
+                         max_iters, tol, s_out, &it, &r, history, NULL, hist_cap < 0 ? 0 : hist_cap, nthreads);
+  if (st == ORC_ERR_INVALID || st == ORC_ERR_NOMEM) return st;
+  if (iters) *iters = it;
   if (resid) *resid = r;
-  return status;
+  return st;
 }
 
 int orc_affine_recurrence(int D, int T, const double* A, const double* b,
