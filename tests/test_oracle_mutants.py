@@ -34,6 +34,9 @@ MUTANTS = [
     ("adaptive rule reversed", "r > stall * r_prev", "r < stall * r_prev", 0),
     ("window hand-off from the wrong step", "s_out + ((size_t)b * T + t0 - 1) * D",
      "s_out + ((size_t)b * T + (t0 > 1 ? t0 - 2 : 0)) * D", 0),
+    ("quasi keeps the off-diagonal", "if (j != k) A[(long)j * D + k] = 0.0;", "if (j != k && 0) A[(long)j * D + k] = 0.0;", 0),
+    ("affine recurrence transposed", "acc += At[(long)r * D + k] * prev[k];", "acc += At[(long)k * D + r] * prev[k];", 0),
+    ("NaN residual not propagated", "if (a != a) r = a;", "if (a != a) r = r;", 0),
 ]
 
 
