@@ -71,3 +71,30 @@ def test_argument_validation_without_gpu():
     assert st == pn.PN_ERR_INVALID and "NULL" in pn.pn_last_error(None) and len(wit) == 2
     pn.pn_destroy(None)
     assert pn.pn_version().startswith("libpn")
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """A C99 program includes include/pn.h, links libpn.so and calls the entry points that need no
+    device (version, error text, NULL-handle validation)."""
+    import subprocess
+    import newton_evaluation_nonlinear_b200 as pn
+    src = tmp_path / "use_pn.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "pn.h"\n'
+        "int main(void) {\n"
+        "  pn_handle h = 0; int it = -1; float r = 0.0f;\n"
+        "  if (pn_eval(h, 0, 0, PN_QUASI, 1, 1e-5f, 0, &it, &r) != PN_ERR_INVALID) return 2;\n"
+        "  if (pn_last_error(NULL)[0] == '\\0') return 3;\n"
+        "  if (pn_dim(NULL, 0) != -1) return 4;\n"
+        "  pn_destroy(NULL);\n"
+        "  printf(\"%s\\n\", pn_version());\n"
+        "  return 0;\n"
+        "}\n")
+    exe = tmp_path / "use_pn"
+    lib_dir = os.path.dirname(pn.LIB_PATH)
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                         str(src), "-o", str(exe), "-L", lib_dir, "-lpn", f"-Wl,-rpath,{lib_dir}"],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0 and run.stdout.startswith("libpn"), (run.returncode, run.stdout, run.stderr)
