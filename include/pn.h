@@ -83,7 +83,14 @@ typedef enum {
   /* 1 (default where available): the diagonal-mode kernels form the cell's
    * recurrent matvec on the tensor cores (3 TF32 passes, fp32-level accuracy;
    * D = 32, or D = 64 for the tanh RNN and Euler cells); 0: FP32 FMA. */
-  PN_OPT_TENSOR_CORES = 3
+  PN_OPT_TENSOR_CORES = 3,
+  /* PN_NEWTON with a banded Jacobian approximation (page §2.2.2, banded
+   * structure of locally connected systems): k >= 0 keeps the entries of
+   * df_t/ds with |row - col| <= k (k = 0 is the diagonal, as PN_QUASI;
+   * k >= D - 1 the exact Jacobian); -1 (default) the exact Jacobian.  The
+   * cost per iteration is that of PN_NEWTON: the scan's aggregates stay
+   * dense, since products of banded matrices fill in. */
+  PN_OPT_NEWTON_BAND = 4
 } pn_option;
 
 /* Per-handle counters, cumulative since pn_create (or pn_reset_stats). */
@@ -216,7 +223,8 @@ PN_API pn_status pn_get_stats(pn_handle h, pn_stats* out);
 PN_API pn_status pn_reset_stats(pn_handle h);
 
 /* Set one pn_option.  Values: PN_OPT_WAIT_TIMEOUT_NS >= 1000;
- * PN_OPT_DEBUG_STALL_TICKET -1 or a ticket >= 0; PN_OPT_DEVICE_LOOP and
+ * PN_OPT_DEBUG_STALL_TICKET -1 or a ticket >= 0; PN_OPT_NEWTON_BAND -1 or a
+ * half-bandwidth >= 0; PN_OPT_DEVICE_LOOP and
  * PN_OPT_TENSOR_CORES 0 or 1 (tensor cores: ignored where the shape has no
  * tensor-core kernel; switching re-selects the kernels after synchronising the
  * stream).  Anything else: PN_ERR_INVALID, the handle unchanged. */

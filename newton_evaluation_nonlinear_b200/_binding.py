@@ -22,6 +22,7 @@ PN_ERR_INVALID, PN_ERR_NOMEM, PN_ERR_CUDA, PN_ERR_NONFINITE, PN_ERR_TIMEOUT = -1
 PN_CELL_TANH_RNN, PN_CELL_GRU, PN_CELL_EULER_TANH = 0, 1, 2
 PN_JACOBI, PN_PICARD, PN_QUASI, PN_NEWTON = 0, 1, 2, 3
 PN_OPT_WAIT_TIMEOUT_NS, PN_OPT_DEBUG_STALL_TICKET, PN_OPT_DEVICE_LOOP, PN_OPT_TENSOR_CORES = 0, 1, 2, 3
+PN_OPT_NEWTON_BAND = 4
 PN_MAX_D_DIAG, PN_MAX_D_NEWTON = 256, 64
 
 STATUS_NAMES = {PN_OK: "PN_OK", PN_NOT_CONVERGED: "PN_NOT_CONVERGED", PN_ERR_INVALID: "PN_ERR_INVALID",

@@ -88,6 +88,7 @@ struct pn_ctx {
   // options
   long long timeout_ns = 1000000000LL;
   int stall_ticket = -1;
+  int newton_band = -1;        // PN_OPT_NEWTON_BAND
   int device_loop = 1;
   bool use_tma = false;        // pipelined bulk-copy kernels (D % 4 == 0, DP >= 32)
   bool use_tc = false;         // tensor-core matvec kernels (D == DP in {32, 64})
@@ -495,6 +496,7 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   pn_status st = prepare_lookback(h, mode);
   if (st != PN_OK) return st;
   h->args_h->use_cond = h->device_loop ? 1 : 0;
+  h->args_h->newton_band = h->newton_band;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
   if ((st = upload_tc_maps(h, mode)) != PN_OK) return st;
   if (h->device_loop && h->fam.k[mode].kind == kKindDiagTct) {
@@ -1137,6 +1139,10 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
     case PN_OPT_DEBUG_STALL_TICKET:
       if (value < -1 || value > INT_MAX) return fail(h, PN_ERR_INVALID, "bad ticket");
       h->stall_ticket = (int)value;
+      return PN_OK;
+    case PN_OPT_NEWTON_BAND:
+      if (value < -1 || value > INT_MAX) return fail(h, PN_ERR_INVALID, "band must be -1 or >= 0");
+      h->newton_band = (int)value;
       return PN_OK;
     case PN_OPT_DEVICE_LOOP:
       if (value != 0 && value != 1) return fail(h, PN_ERR_INVALID, "device loop option is 0 or 1");
