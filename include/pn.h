@@ -230,6 +230,14 @@ PN_API pn_status pn_reset_stats(pn_handle h);
  * stream).  Anything else: PN_ERR_INVALID, the handle unchanged. */
 PN_API pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
 
+/* Damping (page §4.3 and §5.3: a damping factor for an iteration that does
+ * not converge): later evaluations store s^(i+1) = s^(i) + lambda * delta,
+ * delta the undamped update, 0 < lambda <= 1 (1, the default, is undamped).
+ * Implemented for PN_NEWTON (with or without PN_OPT_NEWTON_BAND); while
+ * lambda < 1, evaluations in the other modes return PN_ERR_INVALID.  A lambda
+ * outside (0, 1] is PN_ERR_INVALID, the handle unchanged. */
+PN_API pn_status pn_set_damping(pn_handle h, float lambda);
+
 /* Order the handle's later work on cuda_stream (a cudaStream_t; NULL = the
  * legacy default stream).  The caller keeps the stream alive while the handle
  * uses it and orders it against earlier work itself. */

@@ -55,6 +55,7 @@ SIGNATURES = {
     "pn_reset_stats": (_c_int, [_vp]),
     "pn_set_option": (_c_int, [_vp, _c_int, _c_ll]),
     "pn_set_stream": (_c_int, [_vp, _vp]),
+    "pn_set_damping": (_c_int, [_vp, _c_float]),
     "pn_dim": (_c_int, [_vp, _c_int]),
     "pn_activation": (_c_int, [_c_int, _vp, _vp, _c_ll, _vp]),
     "pn_eval_static": (_c_int, [_vp, ctypes.c_size_t, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _c_int,
@@ -180,6 +181,10 @@ def pn_reset_stats(h: int) -> int:
 
 def pn_set_option(h: int, opt: int, value: int) -> int:
     return lib.pn_set_option(h, int(opt), int(value))
+
+
+def pn_set_damping(h: int, damping: float) -> int:
+    return lib.pn_set_damping(h, float(damping))
 
 
 def pn_set_stream(h: int, stream: int) -> int:
@@ -321,6 +326,9 @@ class Solver:
 
     def set_option(self, opt: int, value: int) -> None:
         self._check(pn_set_option(self.h, opt, value))
+
+    def set_damping(self, damping: float) -> None:
+        self._check(pn_set_damping(self.h, damping))
 
     def close(self) -> None:
         if getattr(self, "h", None):

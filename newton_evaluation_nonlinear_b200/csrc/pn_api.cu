@@ -89,6 +89,7 @@ struct pn_ctx {
   long long timeout_ns = 1000000000LL;
   int stall_ticket = -1;
   int newton_band = -1;        // PN_OPT_NEWTON_BAND
+  float damping = 1.0f;        // pn_set_damping
   int device_loop = 1;
   bool use_tma = false;        // pipelined bulk-copy kernels (D % 4 == 0, DP >= 32)
   bool use_tc = false;         // tensor-core matvec kernels (D == DP in {32, 64})
@@ -454,6 +455,8 @@ pn_status validate_mode(pn_ctx* h, int mode, int max_iters, float tol) {
                 PN_MAX_D_NEWTON);
   if (max_iters < 0) return fail(h, PN_ERR_INVALID, "max_iters must be >= 0");
   if (!(tol >= 0.0f) || !std::isfinite(tol)) return fail(h, PN_ERR_INVALID, "tol must be finite and >= 0");
+  if (h->damping != 1.0f && h->fam.k[mode].kind != kKindDense)
+    return fail(h, PN_ERR_INVALID, "damping is implemented for the dense (Newton) kernel only");
   return PN_OK;
 }
 
@@ -497,6 +500,7 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   if (st != PN_OK) return st;
   h->args_h->use_cond = h->device_loop ? 1 : 0;
   h->args_h->newton_band = h->newton_band;
+  h->args_h->damping = h->damping;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
   if ((st = upload_tc_maps(h, mode)) != PN_OK) return st;
   if (h->device_loop && h->fam.k[mode].kind == kKindDiagTct) {
@@ -1160,6 +1164,13 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
     }
   }
   return fail(h, PN_ERR_INVALID, "unknown option %d", (int)opt);
+}
+
+pn_status pn_set_damping(pn_handle h, float lambda) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  if (!(lambda > 0.0f && lambda <= 1.0f)) return fail(h, PN_ERR_INVALID, "damping must be in (0, 1]");
+  h->damping = lambda;
+  return PN_OK;
 }
 
 pn_status pn_set_stream(pn_handle h, void* cuda_stream) {

@@ -12,6 +12,12 @@
 // |row - col| <= k, and b_t = f_t(s^(i)_{t-1}) - A_t s^(i)_{t-1} takes the
 // banded product.  k >= D - 1 is the exact Jacobian.
 //
+// With a damping factor lambda < 1 (Args::damping; page §4.3 and §5.3 name
+// damping as the remedy for a stalled iteration) the stored iterate is
+// s^(i) + lambda (s_full - s^(i)), where s_full is the undamped update the
+// scan produces; the scan itself, its aggregates and its carried states stay
+// undamped (lambda * delta solves J~ v = -lambda F).
+//
 // Every Jacobian of the three cells is a row-scaled sum of fixed matrices,
 //     A_t = diag(c0_t) + sum_q diag(c_{q,t}) W_q,
 // so the kernel evaluates the cell once, keeps the per-step coefficient
@@ -87,6 +93,8 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
   const int D = P.D, T = P.T, B = P.B;
   const int band = A.newton_band;
   const bool banded = band >= 0 && band < D - 1;
+  const float lambda = A.damping;
+  const bool damped = lambda != 1.0f;
   const size_t stride = (size_t)B;
 
   if (tid == 0) atomicMin(&ctrl->t_start, globaltimer());
@@ -320,6 +328,10 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
       float v = row[DP];
 #pragma unroll(DP <= 16 ? DP : 16)
       for (int kk = 0; kk < DP; ++kk) v = fmaf(row[kk], cur[kk], v);
+      if (damped) {
+        const float sc = sS[(m + 1) * C::SP + i];   // s^(i)_t, staged in step 1
+        v = fmaf(lambda, v - sc, sc);
+      }
       dst[((size_t)b * T + t) * D + i] = v;
     }
   }

@@ -69,5 +69,6 @@ def test_argument_validation_without_gpu():
         pass
     st, it, r, wit = pn.pn_eval_windowed(None, None, 32, 0, 0, 0, 1, 1e-5, 0, 2)
     assert st == pn.PN_ERR_INVALID and "NULL" in pn.pn_last_error(None) and len(wit) == 2
+    assert pn.pn_set_damping(None, 0.5) == pn.PN_ERR_INVALID
     pn.pn_destroy(None)
     assert pn.pn_version().startswith("libpn")
