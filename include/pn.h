@@ -230,6 +230,20 @@ PN_API pn_status pn_reset_stats(pn_handle h);
  * stream).  Anything else: PN_ERR_INVALID, the handle unchanged. */
 PN_API pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
 
+/* Adaptive switching (page §5.3: when the residual curve stalls, switch to
+ * a more exact Jacobian approximation).  With stall >= 0, later evaluations
+ * move one rung up the ladder jacobi/picard -> quasi -> newton (newton only
+ * where this handle supports it) whenever r^(i) > stall * r^(i-1), i >= 1,
+ * before update i is applied; the loop then runs from the host, one launch
+ * per iteration (plus one more launch per switch).  stall < 0 switches it
+ * off (default).  A NaN or infinite stall is PN_ERR_INVALID. */
+PN_API pn_status pn_set_adaptive(pn_handle h, float stall);
+
+/* The mode of each update of the handle's last evaluation (out[i] for update
+ * i, i < iters), n entries at most; *n_written (may be NULL) receives the
+ * count.  Empty unless that evaluation ran with adaptive switching. */
+PN_API pn_status pn_get_mode_history(pn_handle h, int* out, int n, int* n_written);
+
 /* Damping (page §4.3 and §5.3: a damping factor for an iteration that does
  * not converge): later evaluations store s^(i+1) = s^(i) + lambda * delta,
  * delta the undamped update, 0 < lambda <= 1 (1, the default, is undamped).

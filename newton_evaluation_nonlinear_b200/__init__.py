@@ -16,7 +16,8 @@ from ._binding import (MODES, PN_CELL_EULER_TANH, PN_CELL_GRU, PN_CELL_TANH_RNN,
                        PN_OPT_WAIT_TIMEOUT_NS,
                        PN_PICARD, PN_QUASI, SIGNATURES, STATUS_NAMES, LIB_PATH, PnError, Solver, lib,
                        pn_activation, pn_create, pn_destroy, pn_dim, pn_eval, pn_eval_host, pn_eval_host_many, pn_eval_static, pn_eval_windowed, pn_get_residual_history,
-                       pn_get_stats, pn_last_error, pn_reset_stats, pn_set_damping, pn_set_option, pn_set_stream,
+                       pn_get_mode_history, pn_get_stats, pn_last_error, pn_reset_stats, pn_set_adaptive,
+                       pn_set_damping, pn_set_option, pn_set_stream,
                        pn_time_iterations, pn_version)
 
 __version__ = "0.1.0"

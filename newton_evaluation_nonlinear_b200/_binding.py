@@ -56,6 +56,8 @@ SIGNATURES = {
     "pn_set_option": (_c_int, [_vp, _c_int, _c_ll]),
     "pn_set_stream": (_c_int, [_vp, _vp]),
     "pn_set_damping": (_c_int, [_vp, _c_float]),
+    "pn_set_adaptive": (_c_int, [_vp, _c_float]),
+    "pn_get_mode_history": (_c_int, [_vp, _vp, _c_int, ctypes.POINTER(_c_int)]),
     "pn_dim": (_c_int, [_vp, _c_int]),
     "pn_activation": (_c_int, [_c_int, _vp, _vp, _c_ll, _vp]),
     "pn_eval_static": (_c_int, [_vp, ctypes.c_size_t, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _c_int,
@@ -181,6 +183,17 @@ def pn_reset_stats(h: int) -> int:
 
 def pn_set_option(h: int, opt: int, value: int) -> int:
     return lib.pn_set_option(h, int(opt), int(value))
+
+
+def pn_set_adaptive(h: int, stall: float) -> int:
+    return lib.pn_set_adaptive(h, float(stall))
+
+
+def pn_get_mode_history(h: int, n: int) -> Tuple[int, np.ndarray]:
+    out = np.zeros(max(int(n), 1), np.int32)
+    w = _c_int(0)
+    st = lib.pn_get_mode_history(h, out.ctypes.data, int(n), ctypes.byref(w))
+    return st, out[:w.value]
 
 
 def pn_set_damping(h: int, damping: float) -> int:
@@ -329,6 +342,14 @@ class Solver:
 
     def set_damping(self, damping: float) -> None:
         self._check(pn_set_damping(self.h, damping))
+
+    def set_adaptive(self, stall: float) -> None:
+        self._check(pn_set_adaptive(self.h, stall))
+
+    def mode_history(self, n: int = 1 << 16) -> np.ndarray:
+        st, m = pn_get_mode_history(self.h, n)
+        self._check(st)
+        return m
 
     def close(self) -> None:
         if getattr(self, "h", None):

@@ -1,4 +1,4 @@
-"""GPU parity of the Newton-mode refinements (web article "并行牛顿方法：加速非线性
+"""GPU parity of the refinements of the iteration (web article "并行牛顿方法：加速非线性
 序列评估的计算革命"): the banded Jacobian approximation of §2.2.2 (PN_NEWTON with
 PN_OPT_NEWTON_BAND = k keeps the entries of df_t/ds with |row - col| <= k; k = 0
 is the diagonal approximation, k >= D - 1 the exact Jacobian) and the damping of
@@ -105,4 +105,59 @@ def test_band_option_bounds():
     with pytest.raises(pn.PnError):
         solver.set_option(pn.PN_OPT_NEWTON_BAND, -2)
     solver.set_option(pn.PN_OPT_NEWTON_BAND, 1000)      # beyond D - 1: the exact Jacobian
+    solver.close()
+
+
+# ----------------------------------------------------------------------------
+# adaptive switching (§5.3): jacobi/picard -> quasi -> newton on a stall
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("start", ["jacobi", "picard", "quasi"])
+@pytest.mark.parametrize("stall", [0.5, 0.9])
+def test_adaptive_matches_oracle(cell, start, stall):
+    import torch
+    import newton_evaluation_nonlinear_b200 as pn
+    D, T, B = 16, 400, 2
+    d_in = D if cell == pi.CELL_EULER else D - 1
+    prob = pi.random_problem(341 + cell, cell, D, d_in, T=T, B=B, rho=0.8, s0_scale=0.3, eps=0.05)
+    m = oracle.Model.from_problem(prob)
+    seq = m.sequential(prob.x, prob.s0)
+    tol = 1e-5 * max(1.0, float(np.abs(seq).max()))
+    theta = float(np.float32(stall))
+    mode = pn.MODES[start]
+    s_or, it_or, r_or, st_or, hist_or, modes_or, _ = m.iterate_ex(mode, prob.x, prob.s0, T, tol, adapt=True,
+                                                                  stall=theta)
+    solver = pn.Solver.from_problem(prob)
+    solver.set_adaptive(theta)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    states, it, r, st = solver.eval(x, s0, start, T, tol)
+    modes = solver.mode_history()
+    s = states.cpu().numpy()
+    solver.close()
+    assert np.isfinite(s).all() and len(modes) == it
+    ratios = hist_or[1:] / hist_or[:-1]
+    clear = (float(np.min(np.abs(hist_or / tol - 1.0))) > 1e-2 and
+             (len(ratios) == 0 or float(np.min(np.abs(ratios / theta - 1.0))) > 2e-2))
+    if clear:
+        assert (it, st) == (it_or, st_or), (it, it_or)
+        assert modes.tolist() == modes_or[:-1].tolist(), (modes, modes_or)
+        assert _relerr(s, s_or) <= REL_TOL, _relerr(s, s_or)
+    if st == oracle.OK:
+        assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq))
+
+
+def test_adaptive_off_leaves_no_mode_history():
+    import torch
+    import newton_evaluation_nonlinear_b200 as pn
+    prob = pi.random_problem(351, pi.CELL_TANH_RNN, 8, 8, T=60, B=1, rho=0.5)
+    solver = pn.Solver.from_problem(prob)
+    with pytest.raises(pn.PnError):
+        solver.set_adaptive(float("nan"))
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    solver.set_adaptive(-1.0)
+    states, it, r, st = solver.eval(x, s0, "quasi", 60, 1e-5)
+    assert st == pn.PN_OK and len(solver.mode_history()) == 0
     solver.close()
