@@ -1,11 +1,14 @@
-"""GPU parity of the refinements of the iteration (web article "并行牛顿方法：加速非线性
-序列评估的计算革命"): the banded Jacobian approximation of §2.2.2 (PN_NEWTON with
-PN_OPT_NEWTON_BAND = k keeps the entries of df_t/ds with |row - col| <= k; k = 0
-is the diagonal approximation, k >= D - 1 the exact Jacobian) and the damping of
-§4.3 / §5.3 (pn_set_damping: s^(i+1) = s^(i) + lambda * delta).  The oracle's
-orc_iterate_ex with the same settings is the reference: iteration counts equal
-(unless an oracle residual lies within 1% of tol), states within 1e-4 normwise
-of the oracle's iterate and of the sequential states."""
+"""GPU parity of the refinements of the iteration (web article "并行牛顿方法：加速非
+线性序列评估的计算革命"):
+- the banded Jacobian approximation of §2.2.2 (PN_NEWTON with PN_OPT_NEWTON_BAND
+  = k keeps the entries of df_t/ds with |row - col| <= k; k = 0 is the diagonal
+  approximation, k >= D - 1 the exact Jacobian);
+- damping, §4.3 and §5.3 (pn_set_damping: s^(i+1) = s^(i) + lambda * delta);
+- adaptive switching on a residual stall, §5.3 (pn_set_adaptive).
+The oracle's orc_iterate_ex with the same settings is the reference: iteration
+counts (and modes) equal unless an oracle residual lies within 1% of tol or a
+residual ratio within 2% of the stall threshold; states within 1e-4 normwise of
+the oracle's iterate and of the sequential states."""
 import numpy as np
 import pytest
 
