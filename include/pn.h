@@ -83,7 +83,14 @@ typedef enum {
   /* 1 (default where available): the diagonal-mode kernels form the cell's
    * recurrent matvec on the tensor cores (3 TF32 passes, fp32-level accuracy;
    * D = 32, or D = 64 for the tanh RNN and Euler cells); 0: FP32 FMA. */
-  PN_OPT_TENSOR_CORES = 3
+  PN_OPT_TENSOR_CORES = 3,
+  /* PN_NEWTON with a banded Jacobian approximation (page §2.2.2, banded
+   * structure of locally connected systems): k >= 0 keeps the entries of
+   * df_t/ds with |row - col| <= k (k = 0 is the diagonal, as PN_QUASI;
+   * k >= D - 1 the exact Jacobian); -1 (default) the exact Jacobian.  The
+   * cost per iteration is that of PN_NEWTON: the scan's aggregates stay
+   * dense, since products of banded matrices fill in. */
+  PN_OPT_NEWTON_BAND = 4
 } pn_option;
 
 /* Per-handle counters, cumulative since pn_create (or pn_reset_stats). */
@@ -216,11 +223,34 @@ PN_API pn_status pn_get_stats(pn_handle h, pn_stats* out);
 PN_API pn_status pn_reset_stats(pn_handle h);
 
 /* Set one pn_option.  Values: PN_OPT_WAIT_TIMEOUT_NS >= 1000;
- * PN_OPT_DEBUG_STALL_TICKET -1 or a ticket >= 0; PN_OPT_DEVICE_LOOP and
+ * PN_OPT_DEBUG_STALL_TICKET -1 or a ticket >= 0; PN_OPT_NEWTON_BAND -1 or a
+ * half-bandwidth >= 0; PN_OPT_DEVICE_LOOP and
  * PN_OPT_TENSOR_CORES 0 or 1 (tensor cores: ignored where the shape has no
  * tensor-core kernel; switching re-selects the kernels after synchronising the
  * stream).  Anything else: PN_ERR_INVALID, the handle unchanged. */
 PN_API pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
+
+/* Adaptive switching (page §5.3: when the residual curve stalls, switch to
+ * a more exact Jacobian approximation).  With stall >= 0, later evaluations
+ * move one rung up the ladder jacobi/picard -> quasi -> newton (newton only
+ * where this handle supports it) whenever r^(i) > stall * r^(i-1), i >= 1,
+ * before update i is applied; the loop then runs from the host, one launch
+ * per iteration (plus one more launch per switch).  stall < 0 switches it
+ * off (default).  A NaN or infinite stall is PN_ERR_INVALID. */
+PN_API pn_status pn_set_adaptive(pn_handle h, float stall);
+
+/* The mode of each update of the handle's last evaluation (out[i] for update
+ * i, i < iters), n entries at most; *n_written (may be NULL) receives the
+ * count.  Empty unless that evaluation ran with adaptive switching. */
+PN_API pn_status pn_get_mode_history(pn_handle h, int* out, int n, int* n_written);
+
+/* Damping (page §4.3 and §5.3: a damping factor for an iteration that does
+ * not converge): later evaluations store s^(i+1) = s^(i) + lambda * delta,
+ * delta the undamped update, 0 < lambda <= 1 (1, the default, is undamped).
+ * Implemented for PN_NEWTON (with or without PN_OPT_NEWTON_BAND); while
+ * lambda < 1, evaluations in the other modes return PN_ERR_INVALID.  A lambda
+ * outside (0, 1] is PN_ERR_INVALID, the handle unchanged. */
+PN_API pn_status pn_set_damping(pn_handle h, float lambda);
 
 /* Order the handle's later work on cuda_stream (a cudaStream_t; NULL = the
  * legacy default stream).  The caller keeps the stream alive while the handle

@@ -22,6 +22,7 @@ PN_ERR_INVALID, PN_ERR_NOMEM, PN_ERR_CUDA, PN_ERR_NONFINITE, PN_ERR_TIMEOUT = -1
 PN_CELL_TANH_RNN, PN_CELL_GRU, PN_CELL_EULER_TANH = 0, 1, 2
 PN_JACOBI, PN_PICARD, PN_QUASI, PN_NEWTON = 0, 1, 2, 3
 PN_OPT_WAIT_TIMEOUT_NS, PN_OPT_DEBUG_STALL_TICKET, PN_OPT_DEVICE_LOOP, PN_OPT_TENSOR_CORES = 0, 1, 2, 3
+PN_OPT_NEWTON_BAND = 4
 PN_MAX_D_DIAG, PN_MAX_D_NEWTON = 256, 64
 
 STATUS_NAMES = {PN_OK: "PN_OK", PN_NOT_CONVERGED: "PN_NOT_CONVERGED", PN_ERR_INVALID: "PN_ERR_INVALID",
@@ -54,6 +55,9 @@ SIGNATURES = {
     "pn_reset_stats": (_c_int, [_vp]),
     "pn_set_option": (_c_int, [_vp, _c_int, _c_ll]),
     "pn_set_stream": (_c_int, [_vp, _vp]),
+    "pn_set_damping": (_c_int, [_vp, _c_float]),
+    "pn_set_adaptive": (_c_int, [_vp, _c_float]),
+    "pn_get_mode_history": (_c_int, [_vp, _vp, _c_int, ctypes.POINTER(_c_int)]),
     "pn_dim": (_c_int, [_vp, _c_int]),
     "pn_activation": (_c_int, [_c_int, _vp, _vp, _c_ll, _vp]),
     "pn_eval_static": (_c_int, [_vp, ctypes.c_size_t, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _c_int,
@@ -179,6 +183,21 @@ def pn_reset_stats(h: int) -> int:
 
 def pn_set_option(h: int, opt: int, value: int) -> int:
     return lib.pn_set_option(h, int(opt), int(value))
+
+
+def pn_set_adaptive(h: int, stall: float) -> int:
+    return lib.pn_set_adaptive(h, float(stall))
+
+
+def pn_get_mode_history(h: int, n: int) -> Tuple[int, np.ndarray]:
+    out = np.zeros(max(int(n), 1), np.int32)
+    w = _c_int(0)
+    st = lib.pn_get_mode_history(h, out.ctypes.data, int(n), ctypes.byref(w))
+    return st, out[:w.value]
+
+
+def pn_set_damping(h: int, damping: float) -> int:
+    return lib.pn_set_damping(h, float(damping))
 
 
 def pn_set_stream(h: int, stream: int) -> int:
@@ -320,6 +339,17 @@ class Solver:
 
     def set_option(self, opt: int, value: int) -> None:
         self._check(pn_set_option(self.h, opt, value))
+
+    def set_damping(self, damping: float) -> None:
+        self._check(pn_set_damping(self.h, damping))
+
+    def set_adaptive(self, stall: float) -> None:
+        self._check(pn_set_adaptive(self.h, stall))
+
+    def mode_history(self, n: int = 1 << 16) -> np.ndarray:
+        st, m = pn_get_mode_history(self.h, n)
+        self._check(st)
+        return m
 
     def close(self) -> None:
         if getattr(self, "h", None):

@@ -88,6 +88,10 @@ struct pn_ctx {
   // options
   long long timeout_ns = 1000000000LL;
   int stall_ticket = -1;
+  int newton_band = -1;        // PN_OPT_NEWTON_BAND
+  float damping = 1.0f;        // pn_set_damping
+  float adapt_stall = -1.0f;   // pn_set_adaptive: < 0 off
+  std::vector<int> mode_hist;  // mode of every update of the last evaluation
   int device_loop = 1;
   bool use_tma = false;        // pipelined bulk-copy kernels (D % 4 == 0, DP >= 32)
   bool use_tc = false;         // tensor-core matvec kernels (D == DP in {32, 64})
@@ -453,6 +457,8 @@ pn_status validate_mode(pn_ctx* h, int mode, int max_iters, float tol) {
                 PN_MAX_D_NEWTON);
   if (max_iters < 0) return fail(h, PN_ERR_INVALID, "max_iters must be >= 0");
   if (!(tol >= 0.0f) || !std::isfinite(tol)) return fail(h, PN_ERR_INVALID, "tol must be finite and >= 0");
+  if (h->damping != 1.0f && h->fam.k[mode].kind != kKindDense)
+    return fail(h, PN_ERR_INVALID, "damping is implemented for the dense (Newton) kernel only");
   return PN_OK;
 }
 
@@ -489,15 +495,64 @@ pn_status upload_tc_maps(pn_ctx* h, int mode) {
   return PN_OK;
 }
 
+// One rung up the ladder of Jacobian approximations that the handle supports.
+int stronger_mode(const pn_ctx* h, int mode) {
+  int next = mode;
+  if (mode == PN_JACOBI || mode == PN_PICARD) next = PN_QUASI;
+  else if (mode == PN_QUASI) next = PN_NEWTON;
+  return h->fam.k[next].fn ? next : mode;
+}
+
+// Adaptive switching (the page's §5.3: when the residual curve stalls, move to
+// a more exact Jacobian approximation): a host loop, one launch per
+// iteration.  Launch i measures r^(i) and applies update i in the current
+// mode.  When r^(i) > stall * r^(i-1) (i >= 1) and a stronger mode exists,
+// update i must use that mode: the control block's iteration index is set
+// back to i and iteration i is launched again in the stronger mode (it reads
+// the same s^(i) and overwrites s^(i+1) and r^(i)).
+pn_status run_adaptive(pn_ctx* h, int mode) {
+  pn_status st = launch_pre(h);
+  if (st != PN_OK) return st;
+  int cur = mode;
+  float r_prev = 0.0f;
+  for (int i = 0;; ++i) {
+    float r = NAN;
+    for (int attempt = 0; attempt < 2; ++attempt) {
+      if ((st = launch_iter(h, cur)) != PN_OK) return st;
+      PN_CUDA(h, cudaMemcpyAsync(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, h->stream));
+      if (i < kHistCap) PN_CUDA(h, cudaMemcpyAsync(&r, h->hist + i, sizeof(float), cudaMemcpyDeviceToHost, h->stream));
+      PN_CUDA(h, cudaStreamSynchronize(h->stream));
+      if (h->ctrl_h->status != kRunning) return PN_OK;
+      if (attempt == 1 || i == 0 || !(r > h->adapt_stall * r_prev)) break;
+      const int next = stronger_mode(h, cur);
+      if (next == cur) break;
+      cur = next;
+      if ((st = prepare_lookback(h, cur)) != PN_OK) return st;
+      if ((st = upload_tc_maps(h, cur)) != PN_OK) return st;
+      PN_CUDA(h, cudaMemcpyAsync(&h->ctrl->iter, &i, sizeof(int), cudaMemcpyHostToDevice, h->stream));
+    }
+    h->mode_hist.push_back(cur);
+    r_prev = r;
+    if (i > h->args_h->max_iters + 2) return fail(h, PN_ERR_CUDA, "adaptive loop did not stop after max_iters launches");
+  }
+}
+
 // The loop body shared by pn_eval and pn_eval_host: args already point at
 // device buffers.
 pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   pn_status st = prepare_lookback(h, mode);
   if (st != PN_OK) return st;
-  h->args_h->use_cond = h->device_loop ? 1 : 0;
+  const bool adaptive = h->adapt_stall >= 0.0f;
+  h->args_h->use_cond = (h->device_loop && !adaptive) ? 1 : 0;
+  h->args_h->newton_band = h->newton_band;
+  h->args_h->damping = h->damping;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
   if ((st = upload_tc_maps(h, mode)) != PN_OK) return st;
-  if (h->device_loop && h->fam.k[mode].kind == kKindDiagTct) {
+  h->mode_hist.clear();
+  if (adaptive) {
+    if ((st = run_adaptive(h, mode)) != PN_OK) return st;
+    if ((st = launch_finish(h)) != PN_OK) return st;
+  } else if (h->device_loop && h->fam.k[mode].kind == kKindDiagTct) {
     // the iteration kernel loops on the device: four plain launches, no graph needed
     if ((st = launch_pre(h)) != PN_OK) return st;
     if ((st = launch_iter(h, mode, 1)) != PN_OK) return st;
@@ -1138,6 +1193,10 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
       if (value < -1 || value > INT_MAX) return fail(h, PN_ERR_INVALID, "bad ticket");
       h->stall_ticket = (int)value;
       return PN_OK;
+    case PN_OPT_NEWTON_BAND:
+      if (value < -1 || value > INT_MAX) return fail(h, PN_ERR_INVALID, "band must be -1 or >= 0");
+      h->newton_band = (int)value;
+      return PN_OK;
     case PN_OPT_DEVICE_LOOP:
       if (value != 0 && value != 1) return fail(h, PN_ERR_INVALID, "device loop option is 0 or 1");
       h->device_loop = (int)value;
@@ -1154,6 +1213,29 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
     }
   }
   return fail(h, PN_ERR_INVALID, "unknown option %d", (int)opt);
+}
+
+pn_status pn_set_adaptive(pn_handle h, float stall) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  if (std::isnan(stall) || std::isinf(stall)) return fail(h, PN_ERR_INVALID, "stall ratio must be finite");
+  h->adapt_stall = stall < 0.0f ? -1.0f : stall;
+  return PN_OK;
+}
+
+pn_status pn_get_mode_history(pn_handle h, int* out, int n, int* n_written) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  if (n < 0 || (n > 0 && !out)) return fail(h, PN_ERR_INVALID, "bad output buffer");
+  const int cnt = std::min(n, (int)h->mode_hist.size());
+  for (int k = 0; k < cnt; ++k) out[k] = h->mode_hist[k];
+  if (n_written) *n_written = cnt;
+  return PN_OK;
+}
+
+pn_status pn_set_damping(pn_handle h, float lambda) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  if (!(lambda > 0.0f && lambda <= 1.0f)) return fail(h, PN_ERR_INVALID, "damping must be in (0, 1]");
+  h->damping = lambda;
+  return PN_OK;
 }
 
 pn_status pn_set_stream(pn_handle h, void* cuda_stream) {

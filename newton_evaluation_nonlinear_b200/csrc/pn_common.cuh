@@ -50,6 +50,8 @@ struct Args {
   long long timeout_ns;
   int stall_ticket;    // -1 = off
   int use_cond;        // 1 inside the device loop graph
+  int newton_band;     // Newton mode: < 0 the exact Jacobian; k >= 0 its entries with |row - col| <= k only
+  float damping;       // lambda of s^(i+1) = s^(i) + lambda * delta (1 = undamped; dense kernel only)
 };
 
 // Fixed per-handle parameters of the fused iteration kernels.

@@ -7,6 +7,17 @@
 // solved with the affine-map scan of §2.1 (combine (A,b) o (A',b') =
 // (A'A, A'b + b'), (A,b) earlier) over D x D blocks.
 //
+// With a band k >= 0 (Args::newton_band) the kernel uses the banded
+// approximation of §2.2.2 instead: A_t keeps the entries of df_t/ds with
+// |row - col| <= k, and b_t = f_t(s^(i)_{t-1}) - A_t s^(i)_{t-1} takes the
+// banded product.  k >= D - 1 is the exact Jacobian.
+//
+// With a damping factor lambda < 1 (Args::damping; page §4.3 and §5.3 name
+// damping as the remedy for a stalled iteration) the stored iterate is
+// s^(i) + lambda (s_full - s^(i)), where s_full is the undamped update the
+// scan produces; the scan itself, its aggregates and its carried states stay
+// undamped (lambda * delta solves J~ v = -lambda F).
+//
 // Every Jacobian of the three cells is a row-scaled sum of fixed matrices,
 //     A_t = diag(c0_t) + sum_q diag(c_{q,t}) W_q,
 // so the kernel evaluates the cell once, keeps the per-step coefficient
@@ -80,6 +91,10 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
   Ctrl* ctrl = P.ctrl;
   const Args A = *P.args;
   const int D = P.D, T = P.T, B = P.B;
+  const int band = A.newton_band;
+  const bool banded = band >= 0 && band < D - 1;
+  const float lambda = A.damping;
+  const bool damped = lambda != 1.0f;
   const size_t stride = (size_t)B;
 
   if (tid == 0) atomicMin(&ctrl->t_start, globaltimer());
@@ -153,6 +168,21 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
       }
       const float sp = sS[m * C::SP + i];        // s^(i)_{t-1}, channel i
       const float sc = sS[(m + 1) * C::SP + i];  // s^(i)_t
+      // the products W_q s restricted to the band, for b_t = f - A s (the full products
+      // above serve the cell itself)
+      float accb[R];
+#pragma unroll
+      for (int q = 0; q < R; ++q) accb[q] = acc[q];
+      if (banded) {
+        const int k_lo = max(0, i - band);
+        const int k_hi = min(DP - 1, i + band);
+#pragma unroll
+        for (int q = 0; q < R; ++q) {
+          float v = 0.0f;
+          for (int kk = k_lo; kk <= k_hi; ++kk) v = fmaf(sWr[(q * DP + i) * DP + kk], sS[m * C::SP + kk], v);
+          accb[q] = v;
+        }
+      }
       float coef[NC];
       float bb, res;
       if constexpr (CELL == PN_CELL_TANH_RNN) {
@@ -161,7 +191,7 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
         const float d = 1.0f - y * y;
         coef[0] = 0.0f;
         coef[1] = d;
-        bb = y - d * acc[0];
+        bb = y - d * accb[0];
         res = sc - y;
       } else if constexpr (CELL == PN_CELL_EULER_TANH) {
         // A = I + diag(eps (1 - g^2)) W
@@ -170,7 +200,7 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
         const float e = P.eps * (1.0f - gg * gg);
         coef[0] = 1.0f;
         coef[1] = e;
-        bb = eg - e * acc[0];
+        bb = eg - e * accb[0];
         res = (sc - sp) - eg;
       } else {
         // A = diag(z) + diag(gam) W_hr + diag(alp) W_hz + diag(bet) W_hn
@@ -188,7 +218,7 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
         coef[1] = gam;
         coef[2] = alp;
         coef[3] = bet;
-        bb = y - (z * sp + gam * acc[0] + alp * acc[1] + bet * acc[2]);
+        bb = y - (z * sp + gam * accb[0] + alp * accb[1] + bet * accb[2]);
         res = sc - y;
       }
       if (ok) {
@@ -212,6 +242,7 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
       float v = (ii == kk) ? sCoef[(mm * NC + 0) * DP + ii] : 0.0f;
 #pragma unroll
       for (int q = 0; q < R; ++q) v = fmaf(sCoef[(mm * NC + 1 + q) * DP + ii], sWr[(q * DP + ii) * DP + kk], v);
+      if (banded && abs(ii - kk) > band) v = 0.0f;
       sA[e] = v;
       if (mm == 0) sPQ[ii * PQW + kk] = v;   // P_0 = A_0
     }
@@ -297,6 +328,10 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
       float v = row[DP];
 #pragma unroll(DP <= 16 ? DP : 16)
       for (int kk = 0; kk < DP; ++kk) v = fmaf(row[kk], cur[kk], v);
+      if (damped) {
+        const float sc = sS[(m + 1) * C::SP + i];   // s^(i)_t, staged in step 1
+        v = fmaf(lambda, v - sc, sc);
+      }
       dst[((size_t)b * T + t) * D + i] = v;
     }
   }

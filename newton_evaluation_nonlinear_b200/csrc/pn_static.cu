@@ -174,6 +174,8 @@ PN_API pn_status pn_eval_static(const float* params, size_t n_params, int D, int
   ha.timeout_ns = 1000000000LL;
   ha.stall_ticket = -1;
   ha.use_cond = 0;
+  ha.newton_band = -1;
+  ha.damping = 1.0f;
   PN_STATIC_CUDA(cudaMemcpyAsync(args, &ha, sizeof(Args), cudaMemcpyHostToDevice, stream));
 
   // u = U x + b, s^(0) = s0

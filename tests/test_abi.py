@@ -69,6 +69,10 @@ def test_argument_validation_without_gpu():
         pass
     st, it, r, wit = pn.pn_eval_windowed(None, None, 32, 0, 0, 0, 1, 1e-5, 0, 2)
     assert st == pn.PN_ERR_INVALID and "NULL" in pn.pn_last_error(None) and len(wit) == 2
+    assert pn.pn_set_damping(None, 0.5) == pn.PN_ERR_INVALID
+    assert pn.pn_set_adaptive(None, 0.5) == pn.PN_ERR_INVALID
+    st, modes = pn.pn_get_mode_history(None, 4)
+    assert st == pn.PN_ERR_INVALID and len(modes) == 0
     pn.pn_destroy(None)
     assert pn.pn_version().startswith("libpn")
 

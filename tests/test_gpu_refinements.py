@@ -1,0 +1,166 @@
+"""GPU parity of the refinements of the iteration (web article "并行牛顿方法：加速非
+线性序列评估的计算革命"):
+- the banded Jacobian approximation of §2.2.2 (PN_NEWTON with PN_OPT_NEWTON_BAND
+  = k keeps the entries of df_t/ds with |row - col| <= k; k = 0 is the diagonal
+  approximation, k >= D - 1 the exact Jacobian);
+- damping, §4.3 and §5.3 (pn_set_damping: s^(i+1) = s^(i) + lambda * delta);
+- adaptive switching on a residual stall, §5.3 (pn_set_adaptive).
+The oracle's orc_iterate_ex with the same settings is the reference: iteration
+counts (and modes) equal unless an oracle residual lies within 1% of tol or a
+residual ratio within 2% of the stall threshold; states within 1e-4 normwise of
+the oracle's iterate and of the sequential states."""
+import numpy as np
+import pytest
+
+import oracle
+import pn_inputs as pi
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 1e-4
+CELLS = [pi.CELL_TANH_RNN, pi.CELL_GRU, pi.CELL_EULER]
+
+
+def _relerr(a, ref):
+    den = max(float(np.abs(ref).max()), 1e-30)
+    return float(np.abs(a.astype(np.float64) - ref).max()) / den
+
+
+def _run(prob, band, tol, max_iters, damping=1.0):
+    import torch
+    import newton_evaluation_nonlinear_b200 as pn
+    solver = pn.Solver.from_problem(prob)
+    solver.set_option(pn.PN_OPT_NEWTON_BAND, band)
+    solver.set_damping(damping)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    states, it, r, st = solver.eval(x, s0, "newton", max_iters, tol)
+    hist = solver.residual_history()
+    out = states.cpu().numpy()
+    solver.close()
+    return out, it, r, st, hist
+
+
+def _check(cell, D, T, B, band, damping, seed):
+    d_in = D if cell == pi.CELL_EULER else D - 1
+    prob = pi.random_problem(seed, cell, D, d_in, T=T, B=B, rho=0.7, s0_scale=0.3, eps=0.05)
+    m = oracle.Model.from_problem(prob)
+    seq = m.sequential(prob.x, prob.s0)
+    tol = 1e-5 * max(1.0, float(np.abs(seq).max()))
+    mode_or, band_or = (pi.MODE_NEWTON, 0) if band < 0 else (oracle.BANDED, band)
+    lam = float(np.float32(damping))           # the library holds lambda in float32
+    s_or, it_or, r_or, st_or, hist_or, _, _ = m.iterate_ex(mode_or, prob.x, prob.s0, T, tol, band=band_or,
+                                                           damping=lam)
+    s, it, r, st, hist = _run(prob, band, tol, T, damping)
+    assert np.isfinite(s).all()
+    margin = float(np.min(np.abs(hist_or / tol - 1.0)))
+    if margin > 1e-2:
+        assert (it, st) == (it_or, st_or), (it, it_or, hist[:it + 1], hist_or)
+    else:
+        assert abs(it - it_or) <= 1
+    if it == it_or:
+        assert _relerr(s, s_or) <= REL_TOL, _relerr(s, s_or)
+    if st == oracle.OK:
+        assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq))
+    n = min(len(hist), len(hist_or))
+    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=2e-2, atol=1e-5 * max(1.0, float(np.abs(seq).max())))
+
+
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("D,T,B", [(8, 300, 2), (16, 517, 3)])
+@pytest.mark.parametrize("band", [0, 1, 3, -1])
+def test_banded_newton_matches_oracle(cell, D, T, B, band):
+    _check(cell, D, T, B, band, 1.0, 301 + cell + D + band)
+
+
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("band,damping", [(-1, 0.5), (-1, 0.8), (2, 0.7)])
+def test_damped_newton_matches_oracle(cell, band, damping):
+    _check(cell, 12, 400, 2, band, damping, 321 + cell)
+
+
+def test_damping_only_where_implemented():
+    import torch
+    import newton_evaluation_nonlinear_b200 as pn
+    prob = pi.random_problem(331, pi.CELL_TANH_RNN, 8, 8, T=40, B=1, rho=0.5)
+    solver = pn.Solver.from_problem(prob)
+    for bad in (0.0, -0.5, 1.5, float("nan")):
+        with pytest.raises(pn.PnError):
+            solver.set_damping(bad)
+    solver.set_damping(0.5)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    with pytest.raises(pn.PnError) as e:
+        solver.eval(x, s0, "quasi", 40, 1e-5)
+    assert e.value.status == pn.PN_ERR_INVALID
+    states, it, r, st = solver.eval(x, s0, "newton", 40, 1e-5)
+    assert st == pn.PN_OK
+    solver.set_damping(1.0)
+    states, it, r, st = solver.eval(x, s0, "quasi", 40, 1e-5)
+    assert st == pn.PN_OK
+    solver.close()
+
+
+def test_band_option_bounds():
+    import newton_evaluation_nonlinear_b200 as pn
+    prob = pi.random_problem(311, pi.CELL_TANH_RNN, 8, 8, T=40, B=1, rho=0.5)
+    solver = pn.Solver.from_problem(prob)
+    with pytest.raises(pn.PnError):
+        solver.set_option(pn.PN_OPT_NEWTON_BAND, -2)
+    solver.set_option(pn.PN_OPT_NEWTON_BAND, 1000)      # beyond D - 1: the exact Jacobian
+    solver.close()
+
+
+# ----------------------------------------------------------------------------
+# adaptive switching (§5.3): jacobi/picard -> quasi -> newton on a stall
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("start", ["jacobi", "picard", "quasi"])
+@pytest.mark.parametrize("stall", [0.5, 0.9])
+def test_adaptive_matches_oracle(cell, start, stall):
+    import torch
+    import newton_evaluation_nonlinear_b200 as pn
+    D, T, B = 16, 400, 2
+    d_in = D if cell == pi.CELL_EULER else D - 1
+    prob = pi.random_problem(341 + cell, cell, D, d_in, T=T, B=B, rho=0.8, s0_scale=0.3, eps=0.05)
+    m = oracle.Model.from_problem(prob)
+    seq = m.sequential(prob.x, prob.s0)
+    tol = 1e-5 * max(1.0, float(np.abs(seq).max()))
+    theta = float(np.float32(stall))
+    mode = pn.MODES[start]
+    s_or, it_or, r_or, st_or, hist_or, modes_or, _ = m.iterate_ex(mode, prob.x, prob.s0, T, tol, adapt=True,
+                                                                  stall=theta)
+    solver = pn.Solver.from_problem(prob)
+    solver.set_adaptive(theta)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    states, it, r, st = solver.eval(x, s0, start, T, tol)
+    modes = solver.mode_history()
+    s = states.cpu().numpy()
+    solver.close()
+    assert np.isfinite(s).all() and len(modes) == it
+    ratios = hist_or[1:] / hist_or[:-1]
+    clear = (float(np.min(np.abs(hist_or / tol - 1.0))) > 1e-2 and
+             (len(ratios) == 0 or float(np.min(np.abs(ratios / theta - 1.0))) > 2e-2))
+    if clear:
+        assert (it, st) == (it_or, st_or), (it, it_or)
+        assert modes.tolist() == modes_or[:-1].tolist(), (modes, modes_or)
+        assert _relerr(s, s_or) <= REL_TOL, _relerr(s, s_or)
+    if st == oracle.OK:
+        assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq))
+
+
+def test_adaptive_off_leaves_no_mode_history():
+    import torch
+    import newton_evaluation_nonlinear_b200 as pn
+    prob = pi.random_problem(351, pi.CELL_TANH_RNN, 8, 8, T=60, B=1, rho=0.5)
+    solver = pn.Solver.from_problem(prob)
+    with pytest.raises(pn.PnError):
+        solver.set_adaptive(float("nan"))
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    solver.set_adaptive(-1.0)
+    states, it, r, st = solver.eval(x, s0, "quasi", 60, 1e-5)
+    assert st == pn.PN_OK and len(solver.mode_history()) == 0
+    solver.close()
