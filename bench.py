@@ -244,6 +244,15 @@ def cpu_baseline(prob, mode):
             "cpu_model": cpu_model(), "nproc": os.cpu_count()}
 
 
+def workload_config(prob, mode, world):
+    """The workload a line measures; both arms print the same dict for the same workload."""
+    return {"workload": prob.name, "mode": pi.MODE_NAMES[mode], "cell": pi.CELL_NAMES[prob.cell],
+            "D": prob.D, "d_in": prob.d_in, "T": prob.T, "B": prob.B, "tol": prob.tol,
+            "max_iters": prob.iters_cap, "parallelism": f"independent instances x{world}",
+            "l2": "inputs larger than L2 (x, u, two iterate buffers: "
+                  f"{(prob.x.nbytes + 3 * prob.B * prob.T * prob.D * 4) / 1e6:.0f} MB)"}
+
+
 def reference_arm(args, prob, mode, rank, world):
     if rank != 0:
         return
@@ -261,11 +270,11 @@ def reference_arm(args, prob, mode, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": prob.name, "mode": pi.MODE_NAMES[mode], "T": prob.T, "B": prob.B,
-                       "D": prob.D, "tol": prob.tol, "sample_sequences": b_sample},
+            "config": workload_config(prob, mode, world),
+            "run": {"iters": its[-1], "sample_sequences": b_sample, "loop": "host (serial over t)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": f"fp64 oracle {pi.MODE_NAMES[mode]} iteration on the first {b_sample} "
-                                       f"sequences at full T, {its[-1]} iterations per step"},
+                                       f"of {prob.B} sequences at full T={prob.T}, {its[-1]} iterations per step"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -339,14 +348,10 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": prob.name, "mode": pi.MODE_NAMES[mode], "cell": pi.CELL_NAMES[prob.cell],
-                       "D": prob.D, "d_in": prob.d_in, "T": prob.T, "B": prob.B, "tol": prob.tol,
-                       "max_iters": mi, "iters": iters, "final_resid": resid, "status": st,
-                       "parallelism": f"independent instances x{world}",
-                       "loop": "host" if args.host_loop else ("device (one launch iterating to the stop rule)"
-                                                               if looping else "device (CUDA graph WHILE node)"),
-                       "l2": "inputs larger than L2 (x, u, two iterate buffers: "
-                             f"{(prob.x.nbytes + 3 * prob.B * prob.T * prob.D * 4) / 1e6:.0f} MB)"},
+            "config": workload_config(prob, mode, world),
+            "run": {"iters": iters, "final_resid": resid, "status": st,
+                    "loop": "host" if args.host_loop else ("device (one launch iterating to the stop rule)"
+                                                            if looping else "device (CUDA graph WHILE node)")},
             "clocks": clk.summary(), "gpu_launches": launches_per_step * args.steps}
     if not with_extras:
         solver.close()

@@ -40,6 +40,7 @@ struct Family {
   int nchunks[4];
   int ntiles[4];     // ngroups * B * nchunks
   int grid[4];       // persistent CTAs: a multiple of ngroups, at most ntiles
+  int resident[4];   // CTAs that can be resident at once (occupancy query x SM count)
 };
 
 }  // namespace
@@ -396,12 +397,36 @@ fail_graph:
   return fail(h, PN_ERR_CUDA, "building the CUDA graph for mode %d failed: %s", mode, cudaGetErrorString(e));
 }
 
+// The channel-major kernel's CTAs wait on one another (each starts with a
+// static ticket, blockIdx.x, whose look-back may need any lower one, and the
+// looping form meets at a grid barrier after every iteration), so all of its
+// CTAs must be resident at once.  It is launched cooperatively: the runtime
+// refuses a grid it cannot keep resident (another context's kernels, an MPS
+// limit) instead of every wait running out its timeout.  The grid was sized
+// from the occupancy query; the check below guards that sizing on the host.
 pn_status launch_iter(pn_ctx* h, int mode, int persist = 0) {
   const KInfo& ki = h->fam.k[mode];
   IterParams P = make_params(h, mode);
   P.persist = persist;
   void* kargs[] = {(void*)&P};
-  PN_CUDA(h, cudaLaunchKernel(ki.fn, dim3((unsigned)h->fam.grid[mode]), dim3(ki.nt), kargs, ki.smem, h->stream));
+  const unsigned grid = (unsigned)h->fam.grid[mode];
+  if (ki.kind != kKindDiagTct) {
+    PN_CUDA(h, cudaLaunchKernel(ki.fn, dim3(grid), dim3(ki.nt), kargs, ki.smem, h->stream));
+    return PN_OK;
+  }
+  if ((long long)grid > (long long)h->fam.resident[mode])
+    return fail(h, PN_ERR_CUDA, "grid of %u CTAs exceeds the %d that can be resident", grid, h->fam.resident[mode]);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(ki.nt);
+  cfg.dynamicSmemBytes = ki.smem;
+  cfg.stream = h->stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  PN_CUDA(h, cudaLaunchKernelExC(&cfg, ki.fn, kargs));
   return PN_OK;
 }
 
@@ -619,6 +644,7 @@ pn_status select_kernels(pn_ctx* h) {
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || per_sm < 1)
       return fail(h, PN_ERR_CUDA, "occupancy query failed for mode %d (D=%d)", m, D);
     const int ng = h->fam.ngroups[m];
+    h->fam.resident[m] = per_sm * nsm;
     long long want = (long long)per_sm * nsm;
     want = std::max<long long>(ng, (want / ng) * ng);
     h->fam.grid[m] = (int)std::min<long long>(want, h->fam.ntiles[m]);

@@ -147,15 +147,14 @@ PN_API pn_status pn_eval_static(const float* params, size_t n_params, int D, int
     if (e_ != cudaSuccess) return static_fail(PN_ERR_CUDA, "pn_eval_static: %s: %s", #call, cudaGetErrorString(e_)); \
   } while (0)
 
-  // the scratch keeps the previous call's contents: restart the look-back epochs well before they wrap
+  // The scratch keeps the previous call's contents, and the region this call reads as look-back
+  // flags may have held another shape's floats or flags: clear this call's flags on every call (a
+  // few KB), and restart the look-back epochs well before they wrap.
   Ctrl hc;
   PN_STATIC_CUDA(cudaMemcpyAsync(&hc, ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, stream));
   PN_STATIC_CUDA(cudaStreamSynchronize(stream));
-  if (hc.epoch > (1u << 29)) {
-    PN_STATIC_CUDA(cudaMemsetAsync(base + o_flags, 0, sizeof(unsigned) * ntiles, stream));
-    PN_STATIC_CUDA(cudaMemsetAsync(&ctrl->epoch, 0, sizeof(unsigned), stream));
-  }
-  // flags of this call's tiles may hold any earlier epoch; values from the current epoch cannot exist
+  PN_STATIC_CUDA(cudaMemsetAsync(base + o_flags, 0, sizeof(unsigned) * ntiles, stream));
+  if (hc.epoch > (1u << 29)) PN_STATIC_CUDA(cudaMemsetAsync(&ctrl->epoch, 0, sizeof(unsigned), stream));
   PN_STATIC_CUDA(cudaMemcpyAsync(base + o_par, params, sizeof(float) * need_params, cudaMemcpyHostToDevice, stream));
   PN_STATIC_CUDA(cudaMemsetAsync(base + o_bhn, 0, sizeof(float) * DP, stream));
   {

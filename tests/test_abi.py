@@ -102,3 +102,15 @@ def test_header_is_plain_c_and_links(tmp_path):
     assert cc.returncode == 0, cc.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert run.returncode == 0 and run.stdout.startswith("libpn"), (run.returncode, run.stdout, run.stderr)
+
+
+def test_static_entry_point_source_allocates_nothing():
+    """pn_eval_static's translation unit calls no device or host allocator (its scratch is a
+    file-scope device array) and keeps that array a fixed, stated size."""
+    src = open(os.path.join(ROOT, "newton_evaluation_nonlinear_b200", "csrc", "pn_static.cu")).read()
+    code = re.sub(r"//[^\n]*", "", src)
+    for call in ("cudaMalloc", "cudaMallocAsync", "cudaMallocHost", "cudaHostAlloc", "cudaMallocManaged",
+                 "cudaFree", "cuMemAlloc", "cuMemCreate", "malloc(", "new ", "std::vector"):
+        assert call not in code, call
+    assert re.search(r"static __device__ __align__\(256\) unsigned char pn_static_scratch\[", code)
+    assert "cudaGetSymbolAddress" in code

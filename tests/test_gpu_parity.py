@@ -15,6 +15,12 @@ import pn_inputs as pi
 pytestmark = pytest.mark.gpu
 
 REL_TOL = 1e-4          # normwise max|s_gpu - s_ref| / max|s_ref|
+# Residual histories: r^(i) = max|F(s^(i))| in fp32 from an fp32 iterate against the oracle's fp64 one.
+# Early residuals are large and agree to well under 1%; near tol the difference is absolute: the
+# iterate carries a few ulp(max|s|) of scan rounding per step, the activations are within 4e-7, and
+# F_t = s_t - f_t(s_{t-1}) cancels to ~1e-5, so an absolute floor of a few 1e-6 * max(1, max|s|) applies.
+HIST_RTOL = 1e-2
+HIST_ATOL = 5e-6
 
 
 def _pn():
@@ -72,7 +78,7 @@ def _check_against_oracle(prob, mode, tol=None, max_iters=None, device_loop=1, t
     # (a few ulp of max|s| per step, accumulated along the chain)
     n = min(len(hist), len(hist_or))
     scale = max(1.0, float(np.abs(seq).max()))
-    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=2e-2, atol=1e-5 * scale)
+    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=HIST_RTOL, atol=HIST_ATOL * scale)
     return it, s
 
 
@@ -145,11 +151,19 @@ def test_picard_divergence_is_reported():
 RUN_TO_RUN = 1e-6
 
 
-@pytest.mark.parametrize("mode", [pi.MODE_QUASI, pi.MODE_NEWTON])
-def test_host_loop_matches_device_loop(mode):
-    prob = pi.random_problem(5, pi.CELL_TANH_RNN, 16, 16, T=700, B=3, rho=0.7, tol=1e-6)
+@pytest.mark.parametrize("cell,D,mode", [(pi.CELL_TANH_RNN, 16, pi.MODE_QUASI), (pi.CELL_TANH_RNN, 16, pi.MODE_NEWTON),
+                                         (pi.CELL_TANH_RNN, 32, pi.MODE_QUASI), (pi.CELL_TANH_RNN, 64, pi.MODE_QUASI),
+                                         (pi.CELL_EULER, 64, pi.MODE_QUASI), (pi.CELL_GRU, 32, pi.MODE_QUASI)])
+def test_host_loop_matches_device_loop(cell, D, mode):
+    """The host-driven loop (one launch per iteration, PN_OPT_DEVICE_LOOP = 0) and the device loop
+    give the same count and the same states to rounding.  At D = 32 and 64 the one-gate cells' quasi
+    mode runs the channel-major tensor-core kernel, which the device loop launches once for all
+    iterations and the host loop once per iteration; both must also match the oracle."""
+    prob = pi.random_problem(5, cell, D, D, T=700, B=3, rho=0.7, eps=0.05, s0_scale=0.3, tol=1e-6)
     a = _run(prob, mode, device_loop=1)
     b = _run(prob, mode, device_loop=0)
+    if D >= 32:
+        _check_against_oracle(prob, mode, device_loop=0)
     assert a[1] == b[1]
     scale = max(1.0, float(np.abs(a[0]).max()))
     np.testing.assert_allclose(a[0], b[0], rtol=0, atol=RUN_TO_RUN * scale)

@@ -63,7 +63,7 @@ def _check(cell, D, T, B, band, damping, seed):
     if st == oracle.OK:
         assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq))
     n = min(len(hist), len(hist_or))
-    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=2e-2, atol=1e-5 * max(1.0, float(np.abs(seq).max())))
+    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=1e-2, atol=5e-6 * max(1.0, float(np.abs(seq).max())))
 
 
 @pytest.mark.parametrize("cell", CELLS)
@@ -115,15 +115,11 @@ def test_band_option_bounds():
 # adaptive switching (§5.3): jacobi/picard -> quasi -> newton on a stall
 # ----------------------------------------------------------------------------
 
-@pytest.mark.parametrize("cell", CELLS)
-@pytest.mark.parametrize("start", ["jacobi", "picard", "quasi"])
-@pytest.mark.parametrize("stall", [0.5, 0.9])
-def test_adaptive_matches_oracle(cell, start, stall):
+def _check_adaptive(cell, start, stall, D, T, B, seed):
     import torch
     import newton_evaluation_nonlinear_b200 as pn
-    D, T, B = 16, 400, 2
     d_in = D if cell == pi.CELL_EULER else D - 1
-    prob = pi.random_problem(341 + cell, cell, D, d_in, T=T, B=B, rho=0.8, s0_scale=0.3, eps=0.05)
+    prob = pi.random_problem(seed, cell, D, d_in, T=T, B=B, rho=0.8, s0_scale=0.3, eps=0.05)
     m = oracle.Model.from_problem(prob)
     seq = m.sequential(prob.x, prob.s0)
     tol = 1e-5 * max(1.0, float(np.abs(seq).max()))
@@ -149,6 +145,22 @@ def test_adaptive_matches_oracle(cell, start, stall):
         assert _relerr(s, s_or) <= REL_TOL, _relerr(s, s_or)
     if st == oracle.OK:
         assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq))
+
+
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("start", ["jacobi", "picard", "quasi"])
+@pytest.mark.parametrize("stall", [0.5, 0.9])
+def test_adaptive_matches_oracle(cell, start, stall):
+    _check_adaptive(cell, start, stall, 16, 400, 2, 341 + cell)
+
+
+@pytest.mark.parametrize("cell", [pi.CELL_TANH_RNN, pi.CELL_EULER])
+@pytest.mark.parametrize("start", ["jacobi", "picard", "quasi"])
+def test_adaptive_wide_matches_oracle(cell, start):
+    """D = 64: the one-gate cells' quasi-Newton updates run on the channel-major tensor-core kernel
+    (one launch per iteration in the adaptive loop), Jacobi and Picard on the row-major one, Newton
+    on the dense kernel; the switches and the result must match the oracle's."""
+    _check_adaptive(cell, start, 0.9, 64, 600, 2, 361 + cell)
 
 
 def test_adaptive_off_leaves_no_mode_history():
