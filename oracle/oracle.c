@@ -551,6 +551,8 @@ static int iterate_block(int cell, int mode, int band, double damping,
   int status = ORC_NOT_CONVERGED;
   int i = 0;
   double r = 0.0, r_prev = 0.0;
+  /* the residual known when update i starts: r^(i-1), none (+inf) before update 0 */
+  double r_known = INFINITY;
   for (;; ++i) {
     int rc = orc_residual(cell, D, d_in, p, eps, T, B, x, s0, cur, F, &r, nthreads);
     if (rc) { free(other); free(F); return rc; }
@@ -572,9 +574,10 @@ static int iterate_block(int cell, int mode, int band, double damping,
       rc = run_jobs(update_worker, &proto, B, nthreads, NULL);
     }
     if (rc) { free(other); free(F); return rc; }
-    if (r > store_until) orc_round_storage(store, nxt, (long)n);
+    if (r_known > store_until) orc_round_storage(store, nxt, (long)n);
     double* tmp = cur; cur = nxt; nxt = tmp;
     r_prev = r;
+    r_known = r;
   }
   if (cur != s_out) memcpy(s_out, cur, sizeof(double) * n);
   free(other);

@@ -145,10 +145,14 @@ int orc_update_ex(int cell, int mode, int band, double damping, int D,
  *                stays newton.
  *   store,       reduced-precision iterate storage (page §2.3: states kept
  *   store_until  in a narrow format, arithmetic in a wider one).  The
- *                initial guess, and every iterate s^(i+1) whose
- *                predecessor's residual r^(i) > store_until, is rounded to
- *                the format before it is stored; the residual and the
- *                update are then computed in double from the stored values.
+ *                initial guess s^(0) and the first update s^(1) are rounded
+ *                to the format before they are stored, and so is every later
+ *                iterate s^(i+1) while the residual known when its update
+ *                starts, r^(i-1), is above store_until (the page gives no
+ *                switching rule; this one can be applied by an iteration
+ *                that evaluates r^(i) and writes s^(i+1) in the same pass,
+ *                before r^(i) is complete).  The residual and the update are
+ *                computed in double from the stored values.
  *   window       windowed solve (page §1.3.1: the long sequence is split
  *                into blocks that fit in memory; page §2.3, chunks such as
  *                1024 steps).  Reading: t = 1..T is cut into consecutive

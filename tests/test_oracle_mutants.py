@@ -37,6 +37,8 @@ MUTANTS = [
     ("quasi keeps the off-diagonal", "if (j != k) A[(long)j * D + k] = 0.0;", "if (j != k && 0) A[(long)j * D + k] = 0.0;", 0),
     ("affine recurrence transposed", "acc += At[(long)r * D + k] * prev[k];", "acc += At[(long)k * D + r] * prev[k];", 0),
     ("NaN residual not propagated", "if (a != a) r = a;", "if (a != a) r = r;", 0),
+    ("storage switch decided by r^(i), not the known r^(i-1)",
+     "if (r_known > store_until) orc_round_storage", "if (r > store_until) orc_round_storage", 0),
 ]
 
 

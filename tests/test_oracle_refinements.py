@@ -191,8 +191,10 @@ def test_damped_jacobi_closed_form():
 def test_reduced_storage_closed_form(store):
     """s0 = 0, f_t(s) = c_t, Jacobi: the first update gives c exactly, stored as round(c), so
     r^(1) = max|round(c) - c|; every later update returns c and stores round(c) again, so the
-    residual stays at r^(1).  With store_until >= r^(1) the next iterate is kept in double and
-    the iteration ends at r = 0 with the states equal to c."""
+    residual stays at r^(1).  With store_until = r^(1), update i stores round(c) while the residual
+    known when it starts, r^(i-1), is above r^(1): update 0 (nothing known yet) and update 1
+    (r^(0) = max|c|) do; update 2 starts knowing r^(1), which is not above store_until, so s^(3) = c
+    is kept in double and the iteration ends at i = 3 with r = 0 and the states equal to c."""
     prob, m, c = _input_driven(102)
     rc = oracle.round_storage(c, store)
     r1 = np.max(np.abs(rc - c))
@@ -203,7 +205,8 @@ def test_reduced_storage_closed_form(store):
     np.testing.assert_array_equal(s, rc)
     s, it, r, st, hist, modes, wit = m.iterate_ex(pi.MODE_JACOBI, prob.x, prob.s0, 6, 0.0,
                                                   store=store, store_until=r1)
-    assert (it, st, r) == (2, oracle.OK, 0.0)
+    assert (it, st, r) == (3, oracle.OK, 0.0)
+    assert hist[1] == r1 and hist[2] == r1
     np.testing.assert_array_equal(s, c)
 
 
