@@ -246,11 +246,34 @@ PN_API pn_status pn_get_mode_history(pn_handle h, int* out, int n, int* n_writte
 
 /* Damping (page §4.3 and §5.3: a damping factor for an iteration that does
  * not converge): later evaluations store s^(i+1) = s^(i) + lambda * delta,
- * delta the undamped update, 0 < lambda <= 1 (1, the default, is undamped).
- * Implemented for PN_NEWTON (with or without PN_OPT_NEWTON_BAND); while
- * lambda < 1, evaluations in the other modes return PN_ERR_INVALID.  A lambda
- * outside (0, 1] is PN_ERR_INVALID, the handle unchanged. */
+ * delta the undamped update, 0 < lambda <= 1 (1, the default, is undamped),
+ * in every mode (PN_NEWTON with or without PN_OPT_NEWTON_BAND).  The scan
+ * that solves for delta is unchanged; only the stored iterate moves lambda of
+ * the way.  While lambda < 1, Picard and the GRU's quasi-Newton run on the
+ * FP32 kernels instead of the tensor-core ones.  A lambda outside (0, 1] is
+ * PN_ERR_INVALID, the handle unchanged. */
 PN_API pn_status pn_set_damping(pn_handle h, float lambda);
+
+/* Iterate storage formats for pn_set_storage. */
+typedef enum { PN_STORE_F32 = 0, PN_STORE_BF16 = 1, PN_STORE_F16 = 2 } pn_store;
+
+/* Reduced-precision iterate storage (page §2.3: intermediate states kept in
+ * FP16, the key computation in FP32; page §4.2 and §4.3: lower the precision
+ * of intermediate states).  With format PN_STORE_BF16 or PN_STORE_F16, later
+ * evaluations store the iterate in that 16-bit format (round to nearest, ties
+ * to even) while the residual known when an update starts, r^(i-1), is above
+ * store_until -- the initial guess s^(0) and the first update s^(1) always --
+ * and in float32 afterwards; every cell, Jacobian, residual and scan step
+ * still computes in float32 from the stored values.  A narrow iterate takes
+ * the first half of its float32 buffer, so each narrow iteration reads and
+ * writes half the state bytes.  The result is returned as float32 whatever
+ * its storage.  Stored narrow throughout (store_until = +inf), the residual
+ * stalls at the format's resolution (about 2^-9 of max|s| for bfloat16,
+ * 2^-12 for float16), so tol must sit above it or store_until below it.
+ * PN_STORE_F32 (default) stores float32 throughout.  While a narrow format
+ * is set the evaluations run on the FP32-FMA kernels.  An unknown format or
+ * a NaN store_until is PN_ERR_INVALID, the handle unchanged. */
+PN_API pn_status pn_set_storage(pn_handle h, int format, float store_until);
 
 /* Order the handle's later work on cuda_stream (a cudaStream_t; NULL = the
  * legacy default stream).  The caller keeps the stream alive while the handle

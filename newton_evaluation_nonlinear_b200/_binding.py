@@ -23,6 +23,7 @@ PN_CELL_TANH_RNN, PN_CELL_GRU, PN_CELL_EULER_TANH = 0, 1, 2
 PN_JACOBI, PN_PICARD, PN_QUASI, PN_NEWTON = 0, 1, 2, 3
 PN_OPT_WAIT_TIMEOUT_NS, PN_OPT_DEBUG_STALL_TICKET, PN_OPT_DEVICE_LOOP, PN_OPT_TENSOR_CORES = 0, 1, 2, 3
 PN_OPT_NEWTON_BAND = 4
+PN_STORE_F32, PN_STORE_BF16, PN_STORE_F16 = 0, 1, 2
 PN_MAX_D_DIAG, PN_MAX_D_NEWTON = 256, 64
 
 STATUS_NAMES = {PN_OK: "PN_OK", PN_NOT_CONVERGED: "PN_NOT_CONVERGED", PN_ERR_INVALID: "PN_ERR_INVALID",
@@ -57,6 +58,7 @@ SIGNATURES = {
     "pn_set_stream": (_c_int, [_vp, _vp]),
     "pn_set_damping": (_c_int, [_vp, _c_float]),
     "pn_set_adaptive": (_c_int, [_vp, _c_float]),
+    "pn_set_storage": (_c_int, [_vp, _c_int, _c_float]),
     "pn_get_mode_history": (_c_int, [_vp, _vp, _c_int, ctypes.POINTER(_c_int)]),
     "pn_dim": (_c_int, [_vp, _c_int]),
     "pn_activation": (_c_int, [_c_int, _vp, _vp, _c_ll, _vp]),
@@ -198,6 +200,10 @@ def pn_get_mode_history(h: int, n: int) -> Tuple[int, np.ndarray]:
 
 def pn_set_damping(h: int, damping: float) -> int:
     return lib.pn_set_damping(h, float(damping))
+
+
+def pn_set_storage(h: int, fmt: int, store_until: float) -> int:
+    return lib.pn_set_storage(h, int(fmt), float(store_until))
 
 
 def pn_set_stream(h: int, stream: int) -> int:
@@ -345,6 +351,11 @@ class Solver:
 
     def set_adaptive(self, stall: float) -> None:
         self._check(pn_set_adaptive(self.h, stall))
+
+    def set_storage(self, fmt: int, store_until: float = 0.0) -> None:
+        """Iterate storage: PN_STORE_F32, or a 16-bit format (PN_STORE_BF16 / PN_STORE_F16) while the
+        residual known at an update's start is above store_until."""
+        self._check(pn_set_storage(self.h, fmt, store_until))
 
     def mode_history(self, n: int = 1 << 16) -> np.ndarray:
         st, m = pn_get_mode_history(self.h, n)

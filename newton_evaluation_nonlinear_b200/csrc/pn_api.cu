@@ -91,6 +91,8 @@ struct pn_ctx {
   int stall_ticket = -1;
   int newton_band = -1;        // PN_OPT_NEWTON_BAND
   float damping = 1.0f;        // pn_set_damping
+  int store_fmt = 0;           // pn_set_storage: PN_STORE_F32 / _BF16 / _F16
+  float store_until = 0.0f;
   float adapt_stall = -1.0f;   // pn_set_adaptive: < 0 off
   std::vector<int> mode_hist;  // mode of every update of the last evaluation
   int device_loop = 1;
@@ -379,13 +381,16 @@ pn_status build_graph(pn_ctx* h, int mode) {
     prev = node;
   }
   {
-    // 4. result copy
+    // 4. result copy (a narrow result in the caller's buffer first moves to the work buffer)
     const Ctrl* c = h->ctrl;
-    const float* b1 = h->buf1;
+    float* b1 = h->buf1;
     size_t n = (size_t)h->B * h->T * h->D;
-    void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&b1, (void*)&n};
-    e = add_kernel(g, (const void*)&finish_kernel, dim3(pl.fin_grid), dim3(256), 0, kargs, &prev, &node);
-    if (e != cudaSuccess) goto fail_graph;
+    for (int pass = (h->store_fmt != 0 ? 0 : 1); pass < 2; ++pass) {
+      void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&b1, (void*)&n, (void*)&pass};
+      e = add_kernel(g, (const void*)&finish_kernel, dim3(pl.fin_grid), dim3(256), 0, kargs, &prev, &node);
+      if (e != cudaSuccess) goto fail_graph;
+      prev = node;
+    }
   }
   e = cudaGraphInstantiate(&h->exec[mode], g, 0);
   if (e != cudaSuccess) goto fail_graph;
@@ -452,10 +457,12 @@ pn_status launch_finish(pn_ctx* h) {
   const PreLaunch pl = pre_launch(h);
   const Args* a_d = h->args;
   const Ctrl* c = h->ctrl;
-  const float* b1 = h->buf1;
+  float* b1 = h->buf1;
   size_t n = (size_t)h->B * h->T * h->D;
-  void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&b1, (void*)&n};
-  PN_CUDA(h, cudaLaunchKernel((const void*)&finish_kernel, dim3(pl.fin_grid), dim3(256), kargs, 0, h->stream));
+  for (int pass = (h->store_fmt != 0 ? 0 : 1); pass < 2; ++pass) {
+    void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&b1, (void*)&n, (void*)&pass};
+    PN_CUDA(h, cudaLaunchKernel((const void*)&finish_kernel, dim3(pl.fin_grid), dim3(256), kargs, 0, h->stream));
+  }
   return PN_OK;
 }
 
@@ -482,8 +489,6 @@ pn_status validate_mode(pn_ctx* h, int mode, int max_iters, float tol) {
                 PN_MAX_D_NEWTON);
   if (max_iters < 0) return fail(h, PN_ERR_INVALID, "max_iters must be >= 0");
   if (!(tol >= 0.0f) || !std::isfinite(tol)) return fail(h, PN_ERR_INVALID, "tol must be finite and >= 0");
-  if (h->damping != 1.0f && h->fam.k[mode].kind != kKindDense)
-    return fail(h, PN_ERR_INVALID, "damping is implemented for the dense (Newton) kernel only");
   return PN_OK;
 }
 
@@ -540,9 +545,12 @@ pn_status run_adaptive(pn_ctx* h, int mode) {
   if (st != PN_OK) return st;
   int cur = mode;
   float r_prev = 0.0f;
+  // storage formats of iteration i's input and output, restored when iteration i runs again
+  int fmt[2] = {h->store_fmt != 0, h->store_fmt != 0};
   for (int i = 0;; ++i) {
     float r = NAN;
     for (int attempt = 0; attempt < 2; ++attempt) {
+      if (attempt == 1) PN_CUDA(h, cudaMemcpyAsync(&h->ctrl->fmt_in, fmt, sizeof fmt, cudaMemcpyHostToDevice, h->stream));
       if ((st = launch_iter(h, cur)) != PN_OK) return st;
       PN_CUDA(h, cudaMemcpyAsync(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, h->stream));
       if (i < kHistCap) PN_CUDA(h, cudaMemcpyAsync(&r, h->hist + i, sizeof(float), cudaMemcpyDeviceToHost, h->stream));
@@ -558,6 +566,8 @@ pn_status run_adaptive(pn_ctx* h, int mode) {
     }
     h->mode_hist.push_back(cur);
     r_prev = r;
+    fmt[0] = h->ctrl_h->fmt_in;   // iteration i+1's formats, as the last launch left them
+    fmt[1] = h->ctrl_h->fmt_out;
     if (i > h->args_h->max_iters + 2) return fail(h, PN_ERR_CUDA, "adaptive loop did not stop after max_iters launches");
   }
 }
@@ -571,6 +581,8 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   h->args_h->use_cond = (h->device_loop && !adaptive) ? 1 : 0;
   h->args_h->newton_band = h->newton_band;
   h->args_h->damping = h->damping;
+  h->args_h->store_fmt = h->store_fmt;
+  h->args_h->store_until = h->store_until;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
   if ((st = upload_tc_maps(h, mode)) != PN_OK) return st;
   h->mode_hist.clear();
@@ -626,8 +638,15 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
 pn_status select_kernels(pn_ctx* h) {
   const int D = h->D, T = h->T, B = h->B, DP = h->DP;
   for (int m = 0; m < 4; ++m) {
+    // Damped Picard and damped GRU quasi-Newton run on the FP32 kernels: the row-major tensor-core
+    // kernel releases s^(i)_t before its write-out, where damping needs it.
+    // Narrow iterate storage runs on the plain FP32 kernels (element-wise loads and stores in the
+    // storage format).
+    const bool narrow = h->store_fmt != 0;
+    const bool tc_m = h->use_tc && !narrow &&
+                      !(h->damping != 1.0f && (m == PN_PICARD || (h->cell == PN_CELL_GRU && m == PN_QUASI)));
     KInfo ki = (m == PN_NEWTON && DP > PN_MAX_D_NEWTON) ? KInfo{nullptr, 0, 0, 0, 0, 0}
-                                                         : lookup(h->cell, m, DP, h->use_tma, h->use_tc);
+                                                         : lookup(h->cell, m, DP, h->use_tma && !narrow, tc_m);
     h->fam.k[m] = ki;
     if (!ki.fn) continue;
     h->fam.ngroups[m] = (m == PN_NEWTON) ? 1 : (D + ki.G - 1) / ki.G;
@@ -1260,8 +1279,31 @@ pn_status pn_get_mode_history(pn_handle h, int* out, int n, int* n_written) {
 pn_status pn_set_damping(pn_handle h, float lambda) {
   if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
   if (!(lambda > 0.0f && lambda <= 1.0f)) return fail(h, PN_ERR_INVALID, "damping must be in (0, 1]");
+  const bool was = h->damping != 1.0f;
   h->damping = lambda;
+  if (was != (lambda != 1.0f) && h->use_tc) {   // the kernel choice of damped Picard / GRU quasi changes
+    DeviceGuard dg(h->device);
+    if (h->stream) cudaStreamSynchronize(h->stream);
+    else cudaDeviceSynchronize();
+    return select_kernels(h);
+  }
   return PN_OK;
+}
+
+pn_status pn_set_storage(pn_handle h, int format, float store_until) {
+  if (!h) return fail(nullptr, PN_ERR_INVALID, "handle is NULL");
+  if (format < PN_STORE_F32 || format > PN_STORE_F16) return fail(h, PN_ERR_INVALID, "unknown storage format %d", format);
+  if (std::isnan(store_until)) return fail(h, PN_ERR_INVALID, "store_until must not be NaN");
+  const bool changed = (format != 0) != (h->store_fmt != 0);
+  h->store_fmt = format;
+  h->store_until = store_until;
+  if (changed) {   // the kernel choice and the result copy of the graphs change
+    DeviceGuard dg(h->device);
+    if (h->stream) cudaStreamSynchronize(h->stream);
+    else cudaDeviceSynchronize();
+    return select_kernels(h);
+  }
+  return PN_OK;   // the graphs read the format and the threshold from the per-call arguments
 }
 
 pn_status pn_set_stream(pn_handle h, void* cuda_stream) {

@@ -72,10 +72,13 @@ __global__ void init_kernel(const Args* __restrict__ args, Ctrl* __restrict__ ct
   const size_t per_seq = (size_t)T * D;
   const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t nthr = (size_t)gridDim.x * blockDim.x;
+  const int fmt = args->store_fmt;   // s^(0) is stored in the narrow format when one is set
   for (int b = blockIdx.y; b < B; b += gridDim.y) {
     const float* s0 = args->s0 + (size_t)b * D;
     float* st = args->states + (size_t)b * per_seq;
-    if ((D & 3) == 0) {
+    if (fmt != 0) {
+      for (size_t e = tid; e < per_seq; e += nthr) st_state(args->states, (size_t)b * per_seq + e, __ldg(s0 + e % (size_t)D), fmt);
+    } else if ((D & 3) == 0) {
       const size_t D4 = (size_t)(D >> 2);
       const float4* s04 = reinterpret_cast<const float4*>(s0);
       float4* st4 = reinterpret_cast<float4*>(st);
@@ -95,14 +98,36 @@ __global__ void init_kernel(const Args* __restrict__ args, Ctrl* __restrict__ ct
     ctrl->done = 0u;
     ctrl->timeout_ticket = -1;
     ctrl->t_start = ~0ull;
+    ctrl->fmt_in = fmt != 0;    // s^(0) and s^(1) are narrow when a narrow format is set
+    ctrl->fmt_out = fmt != 0;
+    ctrl->final_fmt = 0;
   }
 }
 
-// The result is s^(final_iter), which lives in buffer (final_iter & 1); move
-// it into the caller's states buffer when it is in the work buffer.
+// The result is s^(final_iter), which lives in buffer (final_iter & 1), in
+// float32 or (final_fmt) in the narrow storage format.  Pass 1 moves it into
+// the caller's states buffer as float32: a copy from the work buffer, or a
+// widening of the narrow copy in the work buffer.  Pass 0 runs first when a
+// narrow format is set: a narrow result in the caller's buffer (the first half
+// of it) is moved to the work buffer, so pass 1 never widens in place.
 __global__ void finish_kernel(const Args* __restrict__ args, const Ctrl* __restrict__ ctrl,
-                              const float* __restrict__ buf1, size_t n) {
+                              float* __restrict__ buf1, size_t n, int pass) {
   const int fi = *(const volatile int*)&ctrl->final_iter;
+  const int narrow = *(const volatile int*)&ctrl->final_fmt;
+  const int fmt = args->store_fmt;
+  const size_t g0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t gs = (size_t)gridDim.x * blockDim.x;
+  if (pass == 0) {
+    if (!narrow || (fi & 1)) return;
+    const unsigned short* src = reinterpret_cast<const unsigned short*>(args->states);
+    unsigned short* dst = reinterpret_cast<unsigned short*>(buf1);
+    for (size_t e = g0; e < n; e += gs) dst[e] = src[e];
+    return;
+  }
+  if (narrow) {
+    for (size_t e = g0; e < n; e += gs) args->states[e] = ld_state(buf1, e, fmt);
+    return;
+  }
   if ((fi & 1) == 0) return;
   float* st = args->states;
   const size_t n4 = n / 4;

@@ -5,6 +5,8 @@
 #pragma once
 
 #include <cuda.h>   // CUtensorMap (type only)
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -31,6 +33,11 @@ struct Ctrl {
   unsigned long long t_start;    // min %globaltimer at CTA entry, current launch
   unsigned long long kernel_ns;  // summed launch durations
   unsigned long long launches;   // iterations run by the fused iteration kernels
+  // reduced-precision storage: 1 when s^(iter) (fmt_in) / s^(iter+1) (fmt_out) is stored in the
+  // narrow format Args::store_fmt, 0 for float32; final_fmt is fmt_in of the result s^(final_iter)
+  int fmt_in;
+  int fmt_out;
+  int final_fmt;
   // The words below are hot and each sits in a 128-byte line of its own, so that
   // the ticket atomics do not queue behind the polls of the error word.
   alignas(128) int error;        // sticky device error (PN_ERR_TIMEOUT), 0 if none; polled by waiting warps
@@ -51,7 +58,9 @@ struct Args {
   int stall_ticket;    // -1 = off
   int use_cond;        // 1 inside the device loop graph
   int newton_band;     // Newton mode: < 0 the exact Jacobian; k >= 0 its entries with |row - col| <= k only
-  float damping;       // lambda of s^(i+1) = s^(i) + lambda * delta (1 = undamped; dense kernel only)
+  float damping;       // lambda of s^(i+1) = s^(i) + lambda * delta (1 = undamped)
+  int store_fmt;       // iterate storage: 0 float32, 1 bfloat16, 2 float16 (PN_STORE_*)
+  float store_until;   // narrow storage while the residual known at an update's start is above this
 };
 
 // Fixed per-handle parameters of the fused iteration kernels.
@@ -233,6 +242,26 @@ __device__ __forceinline__ int lookback_nearest_state(const unsigned* flags, siz
   }
 }
 
+// Iterate storage: element idx of an iterate buffer in format fmt (0 float32, 1 bfloat16, 2 float16).
+// A narrow iterate occupies the first half of its float32 buffer.  Stores round to nearest, ties to
+// even (float16: overflow to infinity, gradual underflow).
+__device__ __forceinline__ float ld_state(const void* base, size_t idx, int fmt) {
+  if (fmt == 0) return __ldg(reinterpret_cast<const float*>(base) + idx);
+  const unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(base) + idx);
+  return fmt == 1 ? __uint_as_float((unsigned)h << 16) : __half2float(__ushort_as_half(h));
+}
+__device__ __forceinline__ void st_state(void* base, size_t idx, float v, int fmt) {
+  if (fmt == 0) reinterpret_cast<float*>(base)[idx] = v;
+  else if (fmt == 1) reinterpret_cast<__nv_bfloat16*>(base)[idx] = __float2bfloat16_rn(v);
+  else reinterpret_cast<__half*>(base)[idx] = __float2half_rn(v);
+}
+// The storage formats of the iteration a launch runs: of its input s^(i) and its output s^(i+1).
+__device__ __forceinline__ int2 iter_formats(const Ctrl* c, const Args& A) {
+  const int fi = *(const volatile int*)&c->fmt_in;
+  const int fo = *(const volatile int*)&c->fmt_out;
+  return make_int2(fi ? A.store_fmt : 0, fo ? A.store_fmt : 0);
+}
+
 __device__ __forceinline__ unsigned make_flag(unsigned epoch, unsigned state) {
   return (epoch << 2) | state;
 }
@@ -304,9 +333,13 @@ __device__ __forceinline__ void finish_launch(const IterParams& P, const Args& A
     c->status = st;
     c->final_iter = i;
     c->final_resid = r;
+    c->final_fmt = c->fmt_in;
     if (A.use_cond) cudaGraphSetConditional(P.cond, 0u);
   } else {
     c->iter = i + 1;
+    // s^(i+2) is stored narrow while r^(i), the residual known when update i+1 starts, is above the bar
+    c->fmt_in = c->fmt_out;
+    c->fmt_out = (A.store_fmt != 0 && r > A.store_until) ? 1 : 0;
   }
   c->resid_bits = 0u;
 #pragma unroll
@@ -353,12 +386,15 @@ __device__ __forceinline__ bool finish_iteration(const IterParams& P, const Args
         c->status = st;
         c->final_iter = iter;
         c->final_resid = r;
+        c->final_fmt = c->fmt_in;
         const unsigned long long t1 = globaltimer();
         const unsigned long long t0 = c->t_start;
         if (t1 > t0) c->kernel_ns += t1 - t0;
         c->t_start = ~0ull;
       } else {
         c->iter = iter + 1;
+        c->fmt_in = c->fmt_out;
+        c->fmt_out = (A.store_fmt != 0 && r > A.store_until) ? 1 : 0;
         go = 1;
       }
       c->resid_bits = 0u;

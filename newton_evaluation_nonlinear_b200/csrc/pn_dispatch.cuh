@@ -7,6 +7,7 @@
 #pragma once
 
 #include "pn_iter_dense.cuh"
+#include "pn_iter_dense_warp.cuh"
 #include "pn_iter_diag.cuh"
 #include "pn_iter_diag_tc.cuh"
 #include "pn_iter_diag_tct.cuh"
@@ -103,14 +104,27 @@ inline KInfo dense_kinfo() {
   return KInfo{(const void*)&dense_iter_kernel<CELL, DP, L>, C::NT, L, DP, C::SMEM_BYTES, kKindDense};
 }
 
+// One warp per tile, FP32 chain (D <= 32); NW warps per CTA, sized so two CTAs fit on an SM where
+// the per-warp staging allows it.
+template <int CELL, int DP, int NW>
+inline KInfo dense_warp_kinfo() {
+  using C = DenseWarpCfg<CELL, DP, NW>;
+  return KInfo{(const void*)&dense_warp_kernel<CELL, DP, NW>, C::NT, C::L, DP, C::SMEM_BYTES, kKindDense};
+}
+
 template <int CELL, int DP>
 inline KInfo dense_pick() {
-  if constexpr (DP == 4) return dense_kinfo<CELL, 4, 64>();
-  else if constexpr (DP == 8) return dense_kinfo<CELL, 8, 32>();
-  else if constexpr (DP == 16) return dense_kinfo<CELL, 16, 16>();
-  else if constexpr (DP == 32) return dense_kinfo<CELL, 32, 8>();
-  else {
-    if constexpr (CELL == PN_CELL_GRU) return dense_kinfo<CELL, 64, 2>();
+  constexpr bool gru = (CELL == PN_CELL_GRU);
+  if constexpr (DP == 4) return dense_warp_kinfo<CELL, 4, 8>();
+  else if constexpr (DP == 8) return dense_warp_kinfo<CELL, 8, 8>();
+  else if constexpr (DP == 16) {
+    if constexpr (gru) return dense_warp_kinfo<CELL, 16, 4>();
+    else return dense_warp_kinfo<CELL, 16, 7>();
+  } else if constexpr (DP == 32) {
+    if constexpr (gru) return dense_warp_kinfo<CELL, 32, 3>();
+    else return dense_warp_kinfo<CELL, 32, 6>();
+  } else {
+    if constexpr (gru) return dense_kinfo<CELL, 64, 2>();
     else return dense_kinfo<CELL, 64, 4>();
   }
 }

@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
   const int iter = *(volatile int*)&ctrl->iter;
   const float* __restrict__ src = (iter & 1) ? P.buf1 : A.states;
   float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;
+  const int2 fmt = iter_formats(ctrl, A);   // storage of s^(i) (x) and s^(i+1) (y)
 
   // thread (m, i): step m of the tile, channel i
   const int m = tid / DP;
@@ -144,7 +145,7 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
       float v = 0.0f;
       if (c < D) {
         if (tt < 0) v = __ldg(A.s0 + (size_t)b * D + c);
-        else if (tt < T) v = __ldg(src + ((size_t)b * T + tt) * D + c);
+        else if (tt < T) v = ld_state(src, ((size_t)b * T + tt) * D + c, fmt.x);
       }
       sS[r * C::SP + c] = v;
     }
@@ -332,7 +333,7 @@ __global__ void __launch_bounds__(DenseCfg<CELL, DP, L>::NT) dense_iter_kernel(c
         const float sc = sS[(m + 1) * C::SP + i];   // s^(i)_t, staged in step 1
         v = fmaf(lambda, v - sc, sc);
       }
-      dst[((size_t)b * T + t) * D + i] = v;
+      st_state(dst, ((size_t)b * T + t) * D + i, v, fmt.y);
     }
   }
 

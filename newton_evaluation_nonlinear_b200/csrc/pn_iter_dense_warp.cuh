@@ -1,0 +1,548 @@
+// pn_iter_dense_warp.cuh -- fused Newton iteration with one warp per tile
+// (dense or banded Jacobian, D <= 32), FP32.
+//
+// The iteration is the page's unified update with J~ = J ("Parallel Newton
+// methods..." page, §1.2), or its banded approximation (§2.2.2):
+//     s^(i+1)_t = A_t s^(i+1)_{t-1} + b_t,  A_t = df_t/ds(s^(i)_{t-1}),
+//     b_t = f_t(s^(i)_{t-1}) - A_t s^(i)_{t-1},
+// solved by the affine scan of §2.1 with the combine (A,b) o (A',b') =
+// (A'A, A'b + b') over chunks of L steps and a decoupled look-back between
+// chunks.  Every Jacobian of the three cells is a row-scaled sum of fixed
+// matrices, A_t = diag(c0_t) + sum_q diag(c_{q,t}) W_q, so a step stores only
+// its coefficient vectors, never A_t itself.
+//
+// One warp owns one tile (sequence b, steps t0 .. t0+L-1) from start to end,
+// so the chain needs no block-wide barrier:
+//   1. stage s^(i) rows t0-1 .. t0+L-1 and the step inputs in the warp's slice
+//      of shared memory;
+//   2. cell phase, lane = step: y = f_t(s_{t-1}), the coefficient vectors, b_t
+//      and |F_t|, with W from shared memory (broadcast reads);
+//   3. chain [P | q] <- A_m [P | q] + [0 | b_m], m = 1 .. L-1, from
+//      [A_0 | b_0]: lane (rg, cg) holds rows 4 rg .. 4 rg + 3 and columns
+//      cg CPL .. of P in registers and reads P_{m-1} back from shared memory
+//      (one warp-synchronous exchange per step).  With a band k the inner
+//      product runs only over the band's columns of W, 4 + 2k of them instead
+//      of D: the banded mode costs less than the dense one.  q is a matvec
+//      split over the column-group lanes and reduced with shuffles;
+//   4. decoupled look-back: publish [P_L | q_L], find the nearest published
+//      state, fold the aggregates in between (one matvec each), publish the
+//      tile's end state P_L carry + q_L;
+//   5. apply the carry sequentially, s_m = A_m s_{m-1} + b_m (a matvec per
+//      step, D^2 instead of the D^3 of the chain), stage the states and write
+//      them out (damped: s^(i) + lambda (s - s^(i))).
+// Padded steps (t >= T) and channels (i >= D) are identity maps.
+#pragma once
+
+#include "pn_cells.cuh"
+
+namespace pn {
+
+template <int CELL, int DP, int NWARP>
+struct DenseWarpCfg {
+  static constexpr int R = CellInfo<CELL>::R;
+  static constexpr int L = 32;                          // steps per tile: one per lane in the cell phase
+  static constexpr int RG = DP / 4;                     // row groups of four rows
+  static constexpr int CG = (32 / RG < DP) ? 32 / RG : DP;   // column groups
+  static constexpr int NA = RG * CG;                    // lanes active in the chain and the matvecs
+  static constexpr int CPL = DP / CG;                   // P columns per lane = k-slice per lane
+  static constexpr int NCS = R + 1;                     // coefficient vectors per step: c0, c_1 .. c_R
+  static constexpr int SP = DP + 1;                     // row stride of the staged s rows
+  static constexpr int UP = R * DP + 1;                 // row stride of the staged step inputs
+  static constexpr int a4(int v) { return (v + 3) / 4 * 4; }
+  // per-warp shared memory, in floats
+  static constexpr int O_S = 0;                         // s^(i) rows t0-1 .. t0+L-1: [L+1][SP]
+  static constexpr int O_U = a4(O_S + (L + 1) * SP);    // step inputs [L][UP]
+  static constexpr int O_C = a4(O_U + L * UP);          // coefficients [L][NCS][DP]
+  static constexpr int O_B = O_C + L * NCS * DP;        // b_m [L][DP]
+  static constexpr int O_P = O_B + L * DP;              // P double buffer [2][DP][DP]
+  static constexpr int O_Q = O_P + 2 * DP * DP;         // q double buffer [2][DP]
+  static constexpr int O_O = O_Q + 2 * DP;              // new states [L][DP]
+  static constexpr int O_X = O_O + L * DP;              // carry and fold scratch [2][DP]
+  static constexpr int WARP_FLOATS = a4(O_X + 2 * DP);
+  // per-CTA: W_q^T for the cell [DP][R*DP] (k-major rows: W_q[i][k] at k*R*DP + q*DP + i), the banded
+  // copy used by the Jacobian (same layout), then the warps' slices
+  static constexpr int C_WF = 0;
+  static constexpr int C_WB = C_WF + DP * R * DP;
+  static constexpr int C_WARPS = C_WB + DP * R * DP;
+  static constexpr int C_RED = C_WARPS + NWARP * WARP_FLOATS;
+  static constexpr int SMEM_FLOATS = C_RED + NWARP;
+  static constexpr size_t SMEM_BYTES = (size_t)SMEM_FLOATS * sizeof(float);
+  static constexpr int NT = 32 * NWARP;
+  static_assert(DP % 4 == 0 && DP <= 32, "DP in {4, 8, 16, 32}");
+  static_assert(NA <= 32 && RG * 4 == DP && CG * CPL == DP, "lane grid");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+template <int N>
+__device__ __forceinline__ void lds_n(const float* p, float (&v)[N]) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int e = 0; e < N; e += 4) {
+      const float4 t = *reinterpret_cast<const float4*>(p + e);
+      v[e] = t.x; v[e + 1] = t.y; v[e + 2] = t.z; v[e + 3] = t.w;
+    }
+  } else if constexpr (N == 2) {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    v[0] = t.x; v[1] = t.y;
+  } else {
+#pragma unroll
+    for (int e = 0; e < N; ++e) v[e] = p[e];
+  }
+}
+
+template <int CELL, int DP, int NWARP>
+__global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams P) {
+  using C = DenseWarpCfg<CELL, DP, NWARP>;
+  constexpr int R = C::R;
+  constexpr int L = C::L;
+  constexpr int NCS = C::NCS;
+  constexpr int CG = C::CG;
+  constexpr int CPL = C::CPL;
+  constexpr int SP = C::SP;
+  constexpr int UP = C::UP;
+  constexpr int WR = R * DP;   // row length of the transposed weights
+
+  extern __shared__ __align__(16) float smem_dw[];
+  float* sWf = smem_dw + C::C_WF;
+  float* sWb = smem_dw + C::C_WB;
+  float* sRed = smem_dw + C::C_RED;
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  float* ws = smem_dw + C::C_WARPS + warp * C::WARP_FLOATS;
+  float* sS = ws + C::O_S;
+  float* sU = ws + C::O_U;
+  float* sC = ws + C::O_C;
+  float* sB = ws + C::O_B;
+  float* sP = ws + C::O_P;
+  float* sQ = ws + C::O_Q;
+  float* sO = ws + C::O_O;
+  float* sX = ws + C::O_X;
+
+  Ctrl* ctrl = P.ctrl;
+  const Args A = *P.args;
+  const int D = P.D, T = P.T, B = P.B;
+  const int band = A.newton_band;
+  const bool banded = band >= 0 && band < D - 1;
+  const float lambda = A.damping;
+  const bool damped = lambda != 1.0f;
+  const size_t stride = (size_t)B;
+
+  if (tid == 0) atomicMin(&ctrl->t_start, globaltimer());
+  const unsigned epoch = *(volatile unsigned*)&ctrl->epoch;
+  const int iter = *(volatile int*)&ctrl->iter;
+  const float* __restrict__ src = (iter & 1) ? P.buf1 : A.states;
+  float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;
+  const int2 fmt = iter_formats(ctrl, A);   // storage of s^(i) (x) and s^(i+1) (y)
+  const float* xin = (CELL == PN_CELL_EULER_TANH) ? A.x : P.xin;
+
+  // weights: the cell's W_q^T, and the copy the Jacobian uses (band-masked when banded)
+  for (int e = tid; e < DP * WR; e += C::NT) {
+    const float w = __ldg(P.wt + e);   // W_q[i][k] at k * R * DP + q * DP + i
+    sWf[e] = w;
+    const int k = e / WR;
+    const int i = e % DP;
+    sWb[e] = (banded && abs(i - k) > band) ? 0.0f : w;
+  }
+  __syncthreads();
+  const float* sWj = banded ? sWb : sWf;
+
+  // chain / matvec lane grid: rows 4 rg .. 4 rg + 3, P columns (= k-slice) cg CPL .. cg CPL + CPL - 1
+  const bool act = lane < C::NA;
+  const int rg = act ? lane / CG : 0;
+  const int cg = act ? lane % CG : 0;
+  const int r0 = 4 * rg;
+  const int j0 = cg * CPL;
+  // band-limited k range of the chain's inner product for these four rows
+  const int klo = banded ? max(0, r0 - band) : 0;
+  const int khi = banded ? min(DP - 1, r0 + 3 + band) : DP - 1;
+  const float bhn_l = (CELL == PN_CELL_GRU && lane < D) ? __ldg(P.bhn + lane) : 0.0f;
+  unsigned rbits = 0u;
+  bool aborted = false;
+
+  // y = sum over the k-slice of W_q[r0 + r][k] x[k], reduced over the column-group lanes
+  auto slice_matvec = [&](const float* x, float (&out)[R][4]) {
+    float xs[CPL];
+    lds_n<CPL>(x + j0, xs);
+#pragma unroll
+    for (int q = 0; q < R; ++q)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) out[q][r] = 0.0f;
+#pragma unroll
+    for (int kk = 0; kk < CPL; ++kk) {
+#pragma unroll
+      for (int q = 0; q < R; ++q) {
+        const float4 w = *reinterpret_cast<const float4*>(sWj + (j0 + kk) * WR + q * DP + r0);
+        out[q][0] = fmaf(w.x, xs[kk], out[q][0]);
+        out[q][1] = fmaf(w.y, xs[kk], out[q][1]);
+        out[q][2] = fmaf(w.z, xs[kk], out[q][2]);
+        out[q][3] = fmaf(w.w, xs[kk], out[q][3]);
+      }
+    }
+#pragma unroll
+    for (int off = 1; off < CG; off <<= 1)
+#pragma unroll
+      for (int q = 0; q < R; ++q)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) out[q][r] += __shfl_xor_sync(0xffffffffu, out[q][r], off);
+  };
+
+  for (;;) {
+    int k = 0;
+    if (lane == 0) k = (int)atomicAdd(&ctrl->ticket[0], 1u);
+    k = __shfl_sync(0xffffffffu, k, 0);
+    if (k >= P.tiles_per_group || aborted) break;
+    const int b = k % B;
+    const int chunk = k / B;
+    const int t0 = chunk * L;
+
+    // ---- 1. stage s^(i) rows t0-1 .. t0+L-1 and the step inputs --------------
+    for (int e = lane; e < (L + 1) * DP; e += 32) {
+      const int r = e / DP, c = e % DP;
+      const int tt = t0 - 1 + r;
+      float v = 0.0f;
+      if (c < D) {
+        if (tt < 0) v = __ldg(A.s0 + (size_t)b * D + c);
+        else if (tt < T) v = ld_state(src, ((size_t)b * T + tt) * D + c, fmt.x);
+      }
+      sS[r * SP + c] = v;
+    }
+    for (int e = lane; e < L * R * DP; e += 32) {
+      const int m = e / (R * DP), qc = e % (R * DP);
+      const int q = qc / DP, c = qc % DP;
+      const int tt = t0 + m;
+      sU[m * UP + qc] = (c < D && tt < T) ? __ldg(xin + ((size_t)b * T + tt) * (R * D) + (size_t)q * D + c) : 0.0f;
+    }
+    __syncwarp();
+
+    // ---- 2. cell phase: lane = step m ------------------------------------------
+    {
+      const int m = lane;
+      const bool tok = (t0 + m) < T;
+      float sp[DP];
+#pragma unroll
+      for (int kk = 0; kk < DP; ++kk) sp[kk] = sS[m * SP + kk];
+#pragma unroll 1
+      for (int i0 = 0; i0 < DP; i0 += 4) {
+        float z[R][4], zb[R][4];
+#pragma unroll
+        for (int q = 0; q < R; ++q)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) z[q][r] = 0.0f;
+#pragma unroll
+        for (int kk = 0; kk < DP; ++kk) {
+#pragma unroll
+          for (int q = 0; q < R; ++q) {
+            const float4 w = *reinterpret_cast<const float4*>(sWf + kk * WR + q * DP + i0);
+            z[q][0] = fmaf(w.x, sp[kk], z[q][0]);
+            z[q][1] = fmaf(w.y, sp[kk], z[q][1]);
+            z[q][2] = fmaf(w.z, sp[kk], z[q][2]);
+            z[q][3] = fmaf(w.w, sp[kk], z[q][3]);
+          }
+        }
+        if (banded) {   // the Jacobian's product W_band s for b_t = f - A s
+#pragma unroll
+          for (int q = 0; q < R; ++q)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) zb[q][r] = 0.0f;
+#pragma unroll
+          for (int kk = 0; kk < DP; ++kk) {
+#pragma unroll
+            for (int q = 0; q < R; ++q) {
+              const float4 w = *reinterpret_cast<const float4*>(sWb + kk * WR + q * DP + i0);
+              zb[q][0] = fmaf(w.x, sp[kk], zb[q][0]);
+              zb[q][1] = fmaf(w.y, sp[kk], zb[q][1]);
+              zb[q][2] = fmaf(w.z, sp[kk], zb[q][2]);
+              zb[q][3] = fmaf(w.w, sp[kk], zb[q][3]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < R; ++q)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) zb[q][r] = z[q][r];
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int i = i0 + r;
+          const float spi = sS[m * SP + i];
+          const float sci = sS[(m + 1) * SP + i];
+          float cf[NCS], bb, res;
+          if constexpr (CELL == PN_CELL_TANH_RNN) {
+            const float y = tanh_pn(z[0][r] + sU[m * UP + i]);
+            cf[0] = 0.0f;
+            cf[1] = 1.0f - y * y;
+            bb = y - cf[1] * zb[0][r];
+            res = sci - y;
+          } else if constexpr (CELL == PN_CELL_EULER_TANH) {
+            const float gg = tanh_pn(z[0][r] + sU[m * UP + i]);
+            const float eg = P.eps * gg;
+            cf[0] = 1.0f;
+            cf[1] = P.eps * (1.0f - gg * gg);
+            bb = eg - cf[1] * zb[0][r];
+            res = (sci - spi) - eg;
+          } else {
+            const float bh = __shfl_sync(0xffffffffu, bhn_l, i);
+            const float rr = sigmoidf_acc(sU[m * UP + i] + z[0][r]);
+            const float zz = sigmoidf_acc(sU[m * UP + DP + i] + z[1][r]);
+            const float hn = z[2][r] + bh;
+            const float nn = tanh_pn(sU[m * UP + 2 * DP + i] + rr * hn);
+            const float y = nn + zz * (spi - nn);
+            const float omz = 1.0f - zz;
+            const float dn = omz * (1.0f - nn * nn);
+            cf[0] = zz;
+            cf[1] = dn * hn * rr * (1.0f - rr);   // gamma: W_hr
+            cf[2] = (spi - nn) * zz * omz;        // alpha: W_hz
+            cf[3] = dn * rr;                      // beta:  W_hn
+            // b_t = y - A s with the banded products of W_hr, W_hz, W_hn
+            bb = y - (zz * spi + cf[1] * zb[0][r] + cf[2] * zb[1][r] + cf[3] * zb[2][r]);
+            res = sci - y;
+          }
+          if (tok && i < D) {
+            rbits = max(rbits, abs_bits(res));
+          } else {   // identity map
+            cf[0] = 1.0f;
+#pragma unroll
+            for (int q = 1; q < NCS; ++q) cf[q] = 0.0f;
+            bb = 0.0f;
+          }
+#pragma unroll
+          for (int q = 0; q < NCS; ++q) sC[(m * NCS + q) * DP + i] = cf[q];
+          sB[m * DP + i] = bb;
+        }
+      }
+    }
+    __syncwarp();
+
+    // ---- 3. chain [P | q] over the tile --------------------------------------
+    float pold[4][CPL];
+    {
+      // P_0 = A_0, q_0 = b_0
+      float c0[4], cq[R][4];
+      lds_n<4>(sC + 0 * DP + r0, c0);
+#pragma unroll
+      for (int q = 0; q < R; ++q) lds_n<4>(sC + (1 + q) * DP + r0, cq[q]);
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          const int i = r0 + r, j = j0 + c;
+          float v = (i == j) ? c0[r] : 0.0f;
+#pragma unroll
+          for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], sWj[j * WR + q * DP + i], v);
+          pold[r][c] = v;
+        }
+      if (act) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) sP[(r0 + r) * DP + j0 + c] = pold[r][c];
+        if (cg == 0) *reinterpret_cast<float4*>(sQ + r0) = *reinterpret_cast<const float4*>(sB + r0);
+      }
+      __syncwarp();
+    }
+#pragma unroll 1
+    for (int m = 1; m < L; ++m) {
+      const float* Pk = sP + ((m - 1) & 1) * DP * DP;
+      const float* Qk = sQ + ((m - 1) & 1) * DP;
+      float acc[R][4][CPL];
+#pragma unroll
+      for (int q = 0; q < R; ++q)
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) acc[q][r][c] = 0.0f;
+      if (act) {
+#pragma unroll 4
+        for (int kk = klo; kk <= khi; ++kk) {
+          float p[CPL];
+          lds_n<CPL>(Pk + kk * DP + j0, p);
+#pragma unroll
+          for (int q = 0; q < R; ++q) {
+            const float4 w = *reinterpret_cast<const float4*>(sWj + kk * WR + q * DP + r0);
+            const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+              for (int c = 0; c < CPL; ++c) acc[q][r][c] = fmaf(wv[r], p[c], acc[q][r][c]);
+          }
+        }
+      }
+      float qa[R][4];
+      slice_matvec(Qk, qa);
+      float c0[4], cq[R][4], bm[4], qo[4];
+      lds_n<4>(sC + (m * NCS) * DP + r0, c0);
+#pragma unroll
+      for (int q = 0; q < R; ++q) lds_n<4>(sC + (m * NCS + 1 + q) * DP + r0, cq[q]);
+      lds_n<4>(sB + m * DP + r0, bm);
+      lds_n<4>(Qk + r0, qo);
+      float* Pn = sP + (m & 1) * DP * DP;
+      float qn[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          float v = c0[r] * pold[r][c];
+#pragma unroll
+          for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], acc[q][r][c], v);
+          pold[r][c] = v;
+        }
+        float v = fmaf(c0[r], qo[r], bm[r]);
+#pragma unroll
+        for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], qa[q][r], v);
+        qn[r] = v;
+      }
+      if (act) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          if constexpr (CPL % 4 == 0) {
+#pragma unroll
+            for (int c = 0; c < CPL; c += 4)
+              *reinterpret_cast<float4*>(Pn + (r0 + r) * DP + j0 + c) =
+                  make_float4(pold[r][c], pold[r][c + 1], pold[r][c + 2], pold[r][c + 3]);
+          } else if constexpr (CPL == 2) {
+            *reinterpret_cast<float2*>(Pn + (r0 + r) * DP + j0) = make_float2(pold[r][0], pold[r][1]);
+          } else {
+            Pn[(r0 + r) * DP + j0] = pold[r][0];
+          }
+        }
+        if (cg == 0) *reinterpret_cast<float4*>(sQ + (m & 1) * DP + r0) = make_float4(qn[0], qn[1], qn[2], qn[3]);
+      }
+      __syncwarp();
+    }
+    const float* Pl = sP + ((L - 1) & 1) * DP * DP;   // aggregate [P_L | q_L]
+    const float* Ql = sQ + ((L - 1) & 1) * DP;
+
+    // ---- 4. decoupled look-back ------------------------------------------------
+    const bool stall = (A.stall_ticket == k);
+    if (chunk > 0 && !stall) {
+      float* ag = P.agg + (size_t)k * P.agg_stride;
+      for (int e = lane; e < DP * (DP + 1); e += 32) {
+        const int i = e / (DP + 1), j = e % (DP + 1);
+        ag[e] = (j == DP) ? Ql[i] : Pl[i * DP + j];
+      }
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) st_release(P.flags + k, make_flag(epoch, kFlagAgg));
+    }
+    const int n_agg = lookback_find_prefix(P.flags, (size_t)k, stride, chunk, epoch, ctrl, A.timeout_ns);
+    if (n_agg < 0) {
+      aborted = true;
+      break;
+    }
+    // starting state: the end state of the tile n_agg + 1 back, or s0
+    float* cur = sX;
+    float* nxt = sX + DP;
+    if (lane < DP) {
+      float v = 0.0f;
+      if (chunk - 1 - n_agg >= 0) v = __ldcg(P.pref + ((size_t)k - (size_t)(n_agg + 1) * stride) * P.pref_stride + lane);
+      else if (lane < D) v = __ldg(A.s0 + (size_t)b * D + lane);
+      cur[lane] = v;
+    }
+    __syncwarp();
+    // fold the aggregates at distances n_agg .. 1, farthest first: carry <- P_d carry + q_d
+    for (int d = n_agg; d >= 1; --d) {
+      const float* ag = P.agg + ((size_t)k - (size_t)d * stride) * P.agg_stride;
+      float part[4], qd[4];
+      float xs[CPL];
+      lds_n<CPL>(cur + j0, xs);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        float v = 0.0f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) v = fmaf(act ? __ldcg(ag + (r0 + r) * (DP + 1) + j0 + c) : 0.0f, xs[c], v);
+        part[r] = v;
+        qd[r] = act ? __ldcg(ag + (r0 + r) * (DP + 1) + DP) : 0.0f;
+      }
+#pragma unroll
+      for (int off = 1; off < CG; off <<= 1)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
+      if (act && cg == 0)
+        *reinterpret_cast<float4*>(nxt + r0) =
+            make_float4(part[0] + qd[0], part[1] + qd[1], part[2] + qd[2], part[3] + qd[3]);
+      __syncwarp();
+      float* tmp = cur;
+      cur = nxt;
+      nxt = tmp;
+    }
+    // this tile's end state P_L carry + q_L
+    if (!stall) {
+      float xs[CPL];
+      lds_n<CPL>(cur + j0, xs);
+      float part[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        float v = 0.0f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) v = fmaf(Pl[(r0 + r) * DP + j0 + c], xs[c], v);
+        part[r] = v;
+      }
+#pragma unroll
+      for (int off = 1; off < CG; off <<= 1)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
+      if (act && cg == 0) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) P.pref[(size_t)k * P.pref_stride + r0 + r] = part[r] + Ql[r0 + r];
+      }
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) st_release(P.flags + k, make_flag(epoch, kFlagPrefix));
+    }
+
+    // ---- 5. apply the carry step by step, write the states ----------------------
+    {
+      float sold[4];
+      lds_n<4>(cur + r0, sold);
+      const float* xcur = cur;
+#pragma unroll 1
+      for (int m = 0; m < L; ++m) {
+        float pa[R][4];
+        slice_matvec(xcur, pa);
+        float c0[4], cq[R][4], bm[4];
+        lds_n<4>(sC + (m * NCS) * DP + r0, c0);
+#pragma unroll
+        for (int q = 0; q < R; ++q) lds_n<4>(sC + (m * NCS + 1 + q) * DP + r0, cq[q]);
+        lds_n<4>(sB + m * DP + r0, bm);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          float v = fmaf(c0[r], sold[r], bm[r]);
+#pragma unroll
+          for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], pa[q][r], v);
+          sold[r] = v;
+        }
+        if (act && cg == 0) *reinterpret_cast<float4*>(sO + m * DP + r0) = make_float4(sold[0], sold[1], sold[2], sold[3]);
+        __syncwarp();
+        xcur = sO + m * DP;
+      }
+      for (int e = lane; e < L * DP; e += 32) {
+        const int m = e / DP, i = e % DP;
+        const int tt = t0 + m;
+        if (tt < T && i < D) {
+          float v = sO[e];
+          if (damped) {
+            const float sc = sS[(m + 1) * SP + i];   // s^(i)_t
+            v = fmaf(lambda, v - sc, sc);
+          }
+          st_state(dst, ((size_t)b * T + tt) * D + i, v, fmt.y);
+        }
+      }
+      __syncwarp();   // the warp's slice is restaged by the next tile
+    }
+  }
+
+  rbits = warp_max_u32(rbits);
+  if (lane == 0) sRed[warp] = __uint_as_float(rbits);
+  __syncthreads();
+  if (tid == 0) {
+    unsigned v = 0u;
+    for (int w = 0; w < NWARP; ++w) v = max(v, __float_as_uint(sRed[w]));
+    if (v) atomicMax(&ctrl->resid_bits, v);
+  }
+  finish_launch(P, A, epoch, s_last);
+}
+
+}  // namespace pn

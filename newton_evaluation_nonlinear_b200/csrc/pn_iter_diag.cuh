@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
   Ctrl* ctrl = P.ctrl;
   const Args A = *P.args;
   const int D = P.D, T = P.T, B = P.B;
+  const float lambda = A.damping;   // s^(i+1) = s^(i) + lambda * delta (1: undamped)
+  const bool damped = lambda != 1.0f;
   const int g = (int)(blockIdx.x % (unsigned)P.ngroups);
   const size_t stride = (size_t)B * P.ngroups;   // flag distance between consecutive chunks
 
@@ -95,6 +97,7 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
   const int iter = *(volatile int*)&ctrl->iter;
   const float* __restrict__ src = (iter & 1) ? P.buf1 : A.states;
   float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;
+  const int2 fmt = iter_formats(ctrl, A);   // storage of s^(i) (x) and s^(i+1) (y): 0 float32, else 16-bit
 
   const int tseg = tid % TS;
   const int jg = tid / TS;
@@ -111,6 +114,16 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
     float4* wdst = reinterpret_cast<float4*>(sW);
     for (int e = tid; e < DP * C::WCOLS / 4; e += C::NT) wdst[e] = __ldg(wsrc + e);
   }
+  // s^(i+1) elements e .. e + cvalid - 1, in the storage format of the output
+  auto store_out = [&](size_t e, const float (&o)[TN]) {
+    if (fmt.y == 0) {
+      store_n<TN>(dst + e, o, cvalid, vec_ok);
+    } else {
+#pragma unroll
+      for (int n = 0; n < TN; ++n)
+        if (n < cvalid) st_state(dst, e + n, o[n], fmt.y);
+    }
+  };
   float wd[TN][R];    // W_q[c][c] for this thread's channels (quasi mode)
   float bhn[TN];
   unsigned rbits = 0u;
@@ -161,7 +174,13 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
         else if (t < T) row = src + ((size_t)b * T + t) * D;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (row != nullptr && c < D) {
-          if (dvec) {
+          if (t >= 0 && fmt.x != 0) {   // narrow s^(i)
+            const size_t e0 = ((size_t)b * T + t) * D + c;
+            v.x = ld_state(src, e0, fmt.x);
+            if (c + 1 < D) v.y = ld_state(src, e0 + 1, fmt.x);
+            if (c + 2 < D) v.z = ld_state(src, e0 + 2, fmt.x);
+            if (c + 3 < D) v.w = ld_state(src, e0 + 3, fmt.x);
+          } else if (dvec) {
             v = __ldg(reinterpret_cast<const float4*>(row + c));
           } else {
             v.x = __ldg(row + c);
@@ -292,8 +311,14 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
           if (t < T) {
             float o[TN];
 #pragma unroll
-            for (int n = 0; n < TN; ++n) o[n] = bv[m][n];
-            store_n<TN>(dst + ((size_t)b * T + t) * D + c0, o, cvalid, vec_ok);
+            for (int n = 0; n < TN; ++n) {
+              o[n] = bv[m][n];
+              if (damped && n < cvalid) {
+                const float sc = sT[(c0 + n) * LP + m0 + m + 1];   // s^(i)_t
+                o[n] = fmaf(lambda, o[n] - sc, sc);
+              }
+            }
+            store_out(((size_t)b * T + t) * D + c0, o);
           }
         }
       }
@@ -438,8 +463,12 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
           for (int n = 0; n < TN; ++n) {
             s[n] = fmaf(av[m][n], s[n], bv[m][n]);
             o[n] = s[n];
+            if (damped && n < cvalid) {   // the stored iterate moves lambda of the way; the scan stays undamped
+              const float sc = sT[(c0 + n) * LP + m0 + m + 1];
+              o[n] = fmaf(lambda, o[n] - sc, sc);
+            }
           }
-          if (t < T) store_n<TN>(dst + ((size_t)b * T + t) * D + c0, o, cvalid, vec_ok);
+          if (t < T) store_out(((size_t)b * T + t) * D + c0, o);
         }
       }
       if (s_abort) break;

@@ -407,6 +407,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   Ctrl* ctrl = P.ctrl;
   const Args A = *P.args;
   const int D = P.D, T = P.T, B = P.B;
+  const float lambda = A.damping;
   const size_t stride = (size_t)B;   // one channel group: consecutive chunks are B tickets apart
   const long long tmo = A.timeout_ns;
 
@@ -854,6 +855,9 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
             rbits = max(rbits, abs_bits(res));
             av[c4 + u] = a;
             bv[c4 + u] = bb;
+            // damping (Jacobi only here: the host routes damped Picard and GRU quasi-Newton to the
+            // FP32 kernels, whose write-out still has s^(i)_t at hand)
+            if (MODE == PN_JACOBI && lambda != 1.0f) bv[c4 + u] = fmaf(lambda, bb - sc, sc);
           } else {
             av[c4 + u] = 1.0f;
             bv[c4 + u] = 0.0f;

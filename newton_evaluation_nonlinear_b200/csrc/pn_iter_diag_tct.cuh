@@ -211,6 +211,11 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   const Args A = *P.args;
   const int D = P.D, T = P.T, B = P.B;
   const size_t stride = (size_t)B;   // consecutive chunks of a sequence are B tickets apart
+  // Damping, s^(i+1) = s^(i) + lambda * delta: the parked prefixes (A_t, B_t), from which a state is
+  // formed as A_t carry + B_t, are stored as (lambda A_t, lambda B_t + (1 - lambda) s^(i)_t); the scan,
+  // the piece totals and the look-back stay undamped.
+  const float lambda = A.damping;
+  const bool damped = lambda != 1.0f;
   const long long tmo = A.timeout_ns;
 
   auto init_barriers = [&]() {
@@ -609,7 +614,8 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       const int slot = j % NSLOT;
       mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort);
       const float carry = sCarry[slot * DP + c];
-      const float cp = kHasA ? fmaf(pa, carry, pb) : carry + pb;
+      // Picard parks only B: its damped A_t = lambda enters here
+      const float cp = kHasA ? fmaf(pa, carry, pb) : (carry + pb) * lambda;
       const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + (kHasA ? 32 : 16) * rg) + lane_off;
       float* xo = reinterpret_cast<float*>(smem_raw + C::OFF_X + stg * C::X_BYTES) + row0 * DP + c;
 #pragma unroll
@@ -700,6 +706,10 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         }
         av[i] = SA;
         bv[i] = (MODE == PN_JACOBI) ? bb : SB;
+        if (damped) {
+          av[i] *= lambda;
+          bv[i] = fmaf(lambda, bv[i], (1.0f - lambda) * sc);
+        }
         sp = sc;
       }
       // this tile's TMEM accumulator and its stage (S and step inputs) are consumed

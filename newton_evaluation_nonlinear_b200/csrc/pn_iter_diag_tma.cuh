@@ -88,6 +88,10 @@ __global__ void __launch_bounds__(DiagTmaCfg<CELL, MODE, DP, G, TM, TN, TS>::NT,
   Ctrl* ctrl = P.ctrl;
   const Args A = *P.args;
   const int D = P.D, T = P.T, B = P.B;
+  // damping: s^(i+1) = s^(i) + lambda * delta; the stage of s^(i) is released before the write-out,
+  // so a damped write re-reads s^(i)_t (the scan itself stays undamped)
+  const float lambda = A.damping;
+  const bool damped = lambda != 1.0f;
   const int g = (int)(blockIdx.x % (unsigned)P.ngroups);
   const size_t stride = (size_t)B * P.ngroups;
   const int gw = min(G, D - g * G);   // channels of this group present in D (multiple of 4)
@@ -333,7 +337,13 @@ __global__ void __launch_bounds__(DiagTmaCfg<CELL, MODE, DP, G, TM, TN, TS>::NT,
             if (t < T) {
               float o[TN];
 #pragma unroll
-              for (int n = 0; n < TN; ++n) o[n] = bv[m][n];
+              for (int n = 0; n < TN; ++n) {
+                o[n] = bv[m][n];
+                if (damped && n < cvalid) {
+                  const float sc = __ldg(src + ((size_t)b * T + t) * D + c0 + n);
+                  o[n] = fmaf(lambda, o[n] - sc, sc);
+                }
+              }
               store_n<TN>(dst + ((size_t)b * T + t) * D + c0, o, cvalid, (D % TN) == 0);
             }
           }
@@ -450,7 +460,13 @@ __global__ void __launch_bounds__(DiagTmaCfg<CELL, MODE, DP, G, TM, TN, TS>::NT,
             const int t = t0 + m * TS + tseg;
             float o[TN];
 #pragma unroll
-            for (int n = 0; n < TN; ++n) o[n] = fmaf(av[m][n], cr[n], bv[m][n]);
+            for (int n = 0; n < TN; ++n) {
+              o[n] = fmaf(av[m][n], cr[n], bv[m][n]);
+              if (damped && n < cvalid && t < T) {
+                const float sc = __ldg(src + ((size_t)b * T + t) * D + c0 + n);
+                o[n] = fmaf(lambda, o[n] - sc, sc);
+              }
+            }
             if (t < T) store_n<TN>(dst + ((size_t)b * T + t) * D + c0, o, cvalid, (D % TN) == 0);
           }
         }

@@ -234,9 +234,10 @@ PN_API pn_status pn_eval_static(const float* params, size_t n_params, int D, int
   {
     const Args* a_d = args;
     const Ctrl* c = ctrl;
-    const float* b1 = P.buf1;
+    float* b1 = P.buf1;
     size_t n = nstate;
-    void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&b1, (void*)&n};
+    int pass = 1;   // float32 storage: one pass
+    void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&b1, (void*)&n, (void*)&pass};
     const unsigned g = (unsigned)std::min<size_t>(n / 4 / 256 + 1, 148u * 16u);
     PN_STATIC_CUDA(cudaLaunchKernel(aux_kernel(2), dim3(g), dim3(256), kargs, 0, stream));
   }
