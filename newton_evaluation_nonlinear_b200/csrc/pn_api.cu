@@ -97,6 +97,7 @@ struct pn_ctx {
   std::vector<int> mode_hist;  // mode of every update of the last evaluation
   int device_loop = 1;
   bool use_tma = false;        // pipelined bulk-copy kernels (D % 4 == 0, DP >= 32)
+  bool tc_opt = true;          // PN_OPT_TENSOR_CORES
   bool use_tc = false;         // tensor-core matvec kernels (D == DP in {32, 64})
   bool tc_capable = false;
   long long evals = 0;
@@ -204,6 +205,7 @@ IterParams make_params(const pn_ctx* h, int mode) {
   const int kind = h->fam.k[mode].kind;
   P.wt = dense ? h->wt_dense
                : (kind == kKindDiagTc ? h->wt_tc : (kind == kKindDiagTct ? h->wt_tct : h->wt_diag));
+  P.wt_tc = h->wt_tc;
   P.wdiag = h->wdiag;
   P.bhn = h->bhn;
   P.xin = h->xin;
@@ -402,20 +404,21 @@ fail_graph:
   return fail(h, PN_ERR_CUDA, "building the CUDA graph for mode %d failed: %s", mode, cudaGetErrorString(e));
 }
 
-// The channel-major kernel's CTAs wait on one another (each starts with a
-// static ticket, blockIdx.x, whose look-back may need any lower one, and the
-// looping form meets at a grid barrier after every iteration), so all of its
-// CTAs must be resident at once.  It is launched cooperatively: the runtime
-// refuses a grid it cannot keep resident (another context's kernels, an MPS
-// limit) instead of every wait running out its timeout.  The grid was sized
-// from the occupancy query; the check below guards that sizing on the host.
+// The looping kernels' CTAs wait on one another (they meet at a grid barrier
+// after every iteration; the channel-major kernel also starts each CTA with a
+// static ticket, blockIdx.x, whose look-back may need any lower one), so all
+// of their CTAs must be resident at once.  They are launched cooperatively:
+// the runtime refuses a grid it cannot keep resident (another context's
+// kernels, an MPS limit) instead of every wait running out its timeout.  The
+// grid was sized from the occupancy query; the check below guards that sizing
+// on the host.
 pn_status launch_iter(pn_ctx* h, int mode, int persist = 0) {
   const KInfo& ki = h->fam.k[mode];
   IterParams P = make_params(h, mode);
   P.persist = persist;
   void* kargs[] = {(void*)&P};
   const unsigned grid = (unsigned)h->fam.grid[mode];
-  if (ki.kind != kKindDiagTct) {
+  if (!ki.loops) {
     PN_CUDA(h, cudaLaunchKernel(ki.fn, dim3(grid), dim3(ki.nt), kargs, ki.smem, h->stream));
     return PN_OK;
   }
@@ -589,7 +592,7 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   if (adaptive) {
     if ((st = run_adaptive(h, mode)) != PN_OK) return st;
     if ((st = launch_finish(h)) != PN_OK) return st;
-  } else if (h->device_loop && h->fam.k[mode].kind == kKindDiagTct) {
+  } else if (h->device_loop && h->fam.k[mode].loops) {
     // the iteration kernel loops on the device: four plain launches, no graph needed
     if ((st = launch_pre(h)) != PN_OK) return st;
     if ((st = launch_iter(h, mode, 1)) != PN_OK) return st;
@@ -643,8 +646,12 @@ pn_status select_kernels(pn_ctx* h) {
     // Narrow iterate storage runs on the plain FP32 kernels (element-wise loads and stores in the
     // storage format).
     const bool narrow = h->store_fmt != 0;
-    const bool tc_m = h->use_tc && !narrow &&
-                      !(h->damping != 1.0f && (m == PN_PICARD || (h->cell == PN_CELL_GRU && m == PN_QUASI)));
+    // Newton: the tensor-core compositions take the one-gate cells at DP = 32, 64 unless a band is set
+    const bool banded = h->newton_band >= 0 && h->newton_band < D - 1;
+    const bool tc_m = (m == PN_NEWTON)
+                          ? (h->tc_opt && h->cell != PN_CELL_GRU && (DP == 32 || DP == 64) && !banded)
+                          : (h->use_tc && !narrow &&
+                             !(h->damping != 1.0f && (m == PN_PICARD || (h->cell == PN_CELL_GRU && m == PN_QUASI))));
     KInfo ki = (m == PN_NEWTON && DP > PN_MAX_D_NEWTON) ? KInfo{nullptr, 0, 0, 0, 0, 0}
                                                          : lookup(h->cell, m, DP, h->use_tma && !narrow, tc_m);
     h->fam.k[m] = ki;
@@ -754,6 +761,7 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
   {
     pn_status sk = PN_OK;
     for (int pass = 0; pass < 2 && sk == PN_OK; ++pass) {
+      h->tc_opt = (pass == 1);
       h->use_tc = (pass == 0) ? false : h->tc_capable;
       sk = select_kernels(h);
     }
@@ -1164,7 +1172,7 @@ pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* a
   // timed the same way: one launch that runs n_launches iterations (a tolerance below zero never
   // stops it early, max_iters ends it), average = elapsed / n_launches.  The others: n_launches
   // launches that each re-evaluate the same iterate (r <= +inf stops after one iteration).
-  const bool looping = (h->fam.k[mode].kind == kKindDiagTct);
+  const bool looping = h->fam.k[mode].loops;
   if (looping) {
     PN_CUDA(h, cudaMemcpy(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost));
     const long long last = (long long)h->ctrl_h->iter + n_launches - 1;
@@ -1238,10 +1246,18 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
       if (value < -1 || value > INT_MAX) return fail(h, PN_ERR_INVALID, "bad ticket");
       h->stall_ticket = (int)value;
       return PN_OK;
-    case PN_OPT_NEWTON_BAND:
+    case PN_OPT_NEWTON_BAND: {
       if (value < -1 || value > INT_MAX) return fail(h, PN_ERR_INVALID, "band must be -1 or >= 0");
+      const bool was = h->newton_band >= 0 && h->newton_band < h->D - 1;
       h->newton_band = (int)value;
+      if (was != (h->newton_band >= 0 && h->newton_band < h->D - 1)) {   // Newton's kernel choice changes
+        DeviceGuard dg(h->device);
+        if (h->stream) cudaStreamSynchronize(h->stream);
+        else cudaDeviceSynchronize();
+        return select_kernels(h);
+      }
       return PN_OK;
+    }
     case PN_OPT_DEVICE_LOOP:
       if (value != 0 && value != 1) return fail(h, PN_ERR_INVALID, "device loop option is 0 or 1");
       h->device_loop = (int)value;
@@ -1249,10 +1265,11 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
     case PN_OPT_TENSOR_CORES: {
       if (value != 0 && value != 1) return fail(h, PN_ERR_INVALID, "tensor-core option is 0 or 1");
       const bool want = (value == 1) && h->tc_capable;
-      if (want == h->use_tc) return PN_OK;
+      if (want == h->use_tc && (value == 1) == h->tc_opt) return PN_OK;
       DeviceGuard dg(h->device);
       if (h->stream) cudaStreamSynchronize(h->stream);
       else cudaDeviceSynchronize();
+      h->tc_opt = (value == 1);
       h->use_tc = want;
       return select_kernels(h);
     }
@@ -1336,7 +1353,7 @@ int pn_dim(pn_handle h, int which) {
     case 5 + PN_JACOBI:
     case 5 + PN_PICARD:
     case 5 + PN_QUASI:
-    case 5 + PN_NEWTON: return h->fam.k[which - 5].kind == kKindDiagTct ? 1 : 0;
+    case 5 + PN_NEWTON: return h->fam.k[which - 5].loops ? 1 : 0;
     default: return -1;
   }
 }

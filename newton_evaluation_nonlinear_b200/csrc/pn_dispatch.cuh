@@ -7,6 +7,7 @@
 #pragma once
 
 #include "pn_iter_dense.cuh"
+#include "pn_iter_dense_tc.cuh"
 #include "pn_iter_dense_warp.cuh"
 #include "pn_iter_diag.cuh"
 #include "pn_iter_diag_tc.cuh"
@@ -28,6 +29,7 @@ struct KInfo {
   int G;            // channels per tile
   size_t smem;      // dynamic shared memory bytes
   int kind;         // KKind: which weight packing the kernel reads
+  bool loops = false;   // can run every iteration in one launch (IterParams::persist, grid barrier)
 };
 
 template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS>
@@ -95,7 +97,8 @@ inline KInfo diag_tc_kinfo() {
 template <int CELL, int MODE, int DP>
 inline KInfo diag_tct_kinfo() {
   using C = DiagTctCfg<CELL, MODE, DP>;
-  return KInfo{(const void*)&diag_tct_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTct};
+  return KInfo{(const void*)&diag_tct_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTct,
+               true};
 }
 
 template <int CELL, int DP, int L>
@@ -109,7 +112,7 @@ inline KInfo dense_kinfo() {
 template <int CELL, int DP, int NW>
 inline KInfo dense_warp_kinfo() {
   using C = DenseWarpCfg<CELL, DP, NW>;
-  return KInfo{(const void*)&dense_warp_kernel<CELL, DP, NW>, C::NT, C::L, DP, C::SMEM_BYTES, kKindDense};
+  return KInfo{(const void*)&dense_warp_kernel<CELL, DP, NW>, C::NT, C::L, DP, C::SMEM_BYTES, kKindDense, true};
 }
 
 template <int CELL, int DP>
@@ -129,11 +132,25 @@ inline KInfo dense_pick() {
   }
 }
 
+// Newton with the compositions on the tensor cores: one-gate cells, DP = 32 or 64.
+template <int CELL, int DP>
+inline KInfo dense_tc_kinfo() {
+  using C = DenseTcCfg<CELL, DP>;
+  return KInfo{(const void*)&dense_tc_kernel<CELL, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDense};
+}
+
 // tma: use the pipelined variant where it exists (the caller checks D % 4 == 0);
-// tc: use the tensor-core variant where it exists (the caller checks D == DP).
+// tc: use the tensor-core variant where it exists (diagonal modes: the caller checks D == DP; Newton:
+// the caller checks that the band is off).
 template <int CELL>
 inline KInfo lookup_cell(int mode, int DP, bool tma, bool tc) {
   KInfo none{nullptr, 0, 0, 0, 0, 0};
+  if constexpr (CELL != PN_CELL_GRU) {
+    if (tc && mode == PN_NEWTON) {
+      if (DP == 32) return dense_tc_kinfo<CELL, 32>();
+      if (DP == 64) return dense_tc_kinfo<CELL, 64>();
+    }
+  }
   if (tc && mode != PN_NEWTON) {
     if constexpr (CELL == PN_CELL_GRU) {
       // three gates per channel: the row-major kernel (D = 32)

@@ -131,11 +131,11 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
   const size_t stride = (size_t)B;
 
   if (tid == 0) atomicMin(&ctrl->t_start, globaltimer());
-  const unsigned epoch = *(volatile unsigned*)&ctrl->epoch;
-  const int iter = *(volatile int*)&ctrl->iter;
-  const float* __restrict__ src = (iter & 1) ? P.buf1 : A.states;
-  float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;
-  const int2 fmt = iter_formats(ctrl, A);   // storage of s^(i) (x) and s^(i+1) (y)
+  // iteration and look-back epoch of this launch's first iteration; with P.persist each further
+  // iteration of the launch adds one to both (the grid barrier's last CTA advances the control block)
+  const unsigned gen0 = *(volatile unsigned*)&ctrl->gen;
+  const unsigned epoch0 = *(volatile unsigned*)&ctrl->epoch;
+  const int iter0 = *(volatile int*)&ctrl->iter;
   const float* xin = (CELL == PN_CELL_EULER_TANH) ? A.x : P.xin;
 
   // weights: the cell's W_q^T, and the copy the Jacobian uses (band-masked when banded)
@@ -189,6 +189,15 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
         for (int r = 0; r < 4; ++r) out[q][r] += __shfl_xor_sync(0xffffffffu, out[q][r], off);
   };
 
+  unsigned epoch = epoch0;
+  for (int round = 0;; ++round) {
+  epoch = epoch0 + (unsigned)round;
+  const int iter = iter0 + round;
+  const float* __restrict__ src = (iter & 1) ? P.buf1 : A.states;
+  float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;
+  const int2 fmt = iter_formats(ctrl, A);   // storage of s^(i) (x) and s^(i+1) (y)
+  rbits = 0u;
+  aborted = false;
   for (;;) {
     int k = 0;
     if (lane == 0) k = (int)atomicAdd(&ctrl->ticket[0], 1u);
@@ -534,6 +543,7 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
     }
   }
 
+  // ---- residual of this iteration; the next one (grid barrier) or the end of the launch
   rbits = warp_max_u32(rbits);
   if (lane == 0) sRed[warp] = __uint_as_float(rbits);
   __syncthreads();
@@ -542,7 +552,10 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
     for (int w = 0; w < NWARP; ++w) v = max(v, __float_as_uint(sRed[w]));
     if (v) atomicMax(&ctrl->resid_bits, v);
   }
-  finish_launch(P, A, epoch, s_last);
+  if (!P.persist) break;
+  if (!finish_iteration(P, A, iter, epoch, s_last, (gen0 >> 1) + (unsigned)round)) break;
+  }   // iterations
+  if (!P.persist) finish_launch(P, A, epoch, s_last);
 }
 
 }  // namespace pn

@@ -298,3 +298,18 @@ def test_stats_and_timing():
     ms = solver.time_iterations("quasi", 5)
     assert 0.0 < ms < 1000.0
     solver.close()
+
+
+@pytest.mark.parametrize("tc", [1, 0])
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("D,T,B", [(24, 300, 3), (32, 517, 2), (48, 300, 2), (64, 700, 3)])
+def test_newton_tensor_core_and_fp32_compositions(tc, cell, D, T, B):
+    """Newton at D = 17..64: the one-gate cells compose the chunk aggregates on the tensor cores
+    (3xTF32 tcgen05.mma, padded width 32 or 64) unless PN_OPT_TENSOR_CORES = 0; the GRU, and every
+    cell with tc = 0, run the FP32 kernels (one warp per tile up to D = 32).  All must match the
+    oracle's serial Newton iteration and the sequential states, over several 32-step chunks and a
+    ragged tail."""
+    d_in = D if cell == pi.CELL_EULER else D - 3
+    prob = pi.random_problem(600 + D + T + cell, cell, D, d_in, T=T, B=B, rho=0.7, eps=0.05, s0_scale=0.3,
+                             tol=1e-5)
+    _check_against_oracle(prob, pi.MODE_NEWTON, tc=tc)
