@@ -281,10 +281,11 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       s_tk[0] = kg;
       mbar_arrive_expect_tx(&bar_sfull[0], (unsigned)(NKH * C::SH_LOAD));
 #pragma unroll
-      for (int h = 0; h < NKH; ++h) tma_load_3d(sS + h * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[0]);
+      for (int h = 0; h < NKH; ++h)
+        tma_load_3d_hint(sS + h * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[0], l2_policy_evict_first());
       if (round == 0) {   // later iterations: fetched before the grid barrier
         mbar_arrive_expect_tx(&bar_xfull[0], (unsigned)C::X_BYTES);
-        tma_load_3d(smem_raw + C::OFF_X, tm_x, 0, t0, b, &bar_xfull[0]);
+        tma_load_3d_hint(smem_raw + C::OFF_X, tm_x, 0, t0, b, &bar_xfull[0], l2_policy_evict_last());
       }
     } else {
       s_tk[0] = -1;
@@ -327,6 +328,9 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     const CUtensorMap* tm_x = P.tmaps + 2;                      // step inputs
     const CUtensorMap* tm_o = P.tmaps + ((iter & 1) ? 3 : 4);   // s^(i+1), into the other buffer
     if (lane == 0) tmap_acquire(tm_o);
+    // the step inputs are read by every iteration: kept in L2 ahead of the iterates, read once each
+    const uint64_t pol_keep = l2_policy_evict_last();
+    const uint64_t pol_stream = l2_policy_evict_first();
     // The states the epilogue staged at its event e (one event per tile, and three more for the
     // last write-outs) in step-input buffer e & 1: one tensor store, and a wait until it has
     // read the buffer, which is then free again (for tile e + 2's step inputs, or, signalled on
@@ -375,7 +379,8 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         s_tk[st] = kg;
         mbar_arrive_expect_tx(&bar_sfull[st], (unsigned)(NKH * C::SH_LOAD));
 #pragma unroll
-        for (int h = 0; h < NKH; ++h) tma_load_3d(sS + (st * NKH + h) * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[st]);
+        for (int h = 0; h < NKH; ++h)
+          tma_load_3d_hint(sS + (st * NKH + h) * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[st], pol_stream);
       }
       __syncwarp();
       n_tiles = it + 1;
@@ -386,7 +391,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       }
       if (lane == 0) {
         mbar_arrive_expect_tx(&bar_xfull[st], (unsigned)C::X_BYTES);
-        tma_load_3d(smem_raw + C::OFF_X + st * C::X_BYTES, tm_x, 0, t0, b, &bar_xfull[st]);
+        tma_load_3d_hint(smem_raw + C::OFF_X + st * C::X_BYTES, tm_x, 0, t0, b, &bar_xfull[st], pol_keep);
       }
       __syncwarp();
       n_loaded = it + 1;
@@ -794,8 +799,9 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     }
     if constexpr (kScan) {
       // the last three tiles' states: events it .. it+2, each in the step-input buffer of its
-      // parity once the store of the event two before has read that buffer
-#pragma unroll
+      // parity once the store of the event two before has read that buffer (a loop, not unrolled:
+      // one copy of the write-out code serves it, which keeps the epilogue's code smaller)
+#pragma unroll 1
       for (int j = 0; j < C::DEFER; ++j) {
         const int ev = it + j;
         const int tj = ev - C::DEFER;
@@ -839,7 +845,8 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     if (has_tile0) {
       const int kg = (int)blockIdx.x;
       mbar_arrive_expect_tx(&bar_xfull[0], (unsigned)C::X_BYTES);
-      tma_load_3d(smem_raw + C::OFF_X, P.tmaps + 2, 0, (kg / B) * L, kg % B, &bar_xfull[0]);
+      tma_load_3d_hint(smem_raw + C::OFF_X, P.tmaps + 2, 0, (kg / B) * L, kg % B, &bar_xfull[0],
+                       l2_policy_evict_last());
     }
   }
   if (!finish_iteration(P, A, iter, epoch, s_last, (gen0 >> 1) + (unsigned)round)) {
