@@ -14,10 +14,11 @@ from ._binding import (MODES, PN_CELL_EULER_TANH, PN_CELL_GRU, PN_CELL_TANH_RNN,
                        PN_MAX_D_DIAG, PN_MAX_D_NEWTON, PN_NEWTON, PN_NOT_CONVERGED, PN_OK,
                        PN_OPT_DEBUG_STALL_TICKET, PN_OPT_DEVICE_LOOP, PN_OPT_NEWTON_BAND, PN_OPT_TENSOR_CORES,
                        PN_OPT_WAIT_TIMEOUT_NS,
-                       PN_PICARD, PN_QUASI, SIGNATURES, STATUS_NAMES, LIB_PATH, PnError, Solver, lib,
+                       PN_PICARD, PN_QUASI, PN_STORE_BF16, PN_STORE_F16, PN_STORE_F32,
+                       SIGNATURES, STATUS_NAMES, LIB_PATH, PnError, Solver, lib,
                        pn_activation, pn_create, pn_destroy, pn_dim, pn_eval, pn_eval_host, pn_eval_host_many, pn_eval_static, pn_eval_windowed, pn_get_residual_history,
                        pn_get_mode_history, pn_get_stats, pn_last_error, pn_reset_stats, pn_set_adaptive,
-                       pn_set_damping, pn_set_option, pn_set_stream,
+                       pn_set_damping, pn_set_option, pn_set_storage, pn_set_stream,
                        pn_time_iterations, pn_version)
 
 __version__ = "0.1.0"

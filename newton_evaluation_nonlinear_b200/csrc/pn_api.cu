@@ -41,6 +41,7 @@ struct Family {
   int ntiles[4];     // ngroups * B * nchunks
   int grid[4];       // persistent CTAs: a multiple of ngroups, at most ntiles
   int resident[4];   // CTAs that can be resident at once (occupancy query x SM count)
+  int run[4];        // chunks per ticket
 };
 
 }  // namespace
@@ -225,6 +226,7 @@ IterParams make_params(const pn_ctx* h, int mode) {
   P.ngroups = h->fam.ngroups[mode];
   P.nchunks = h->fam.nchunks[mode];
   P.tiles_per_group = h->B * h->fam.nchunks[mode];
+  P.run = h->fam.run[mode];
   const int G = h->fam.k[mode].G;
   P.agg_stride = dense ? G * (G + 1) : 2 * G;
   P.pref_stride = G;
@@ -659,8 +661,6 @@ pn_status select_kernels(pn_ctx* h) {
     h->fam.ngroups[m] = (m == PN_NEWTON) ? 1 : (D + ki.G - 1) / ki.G;
     if (h->fam.ngroups[m] > kMaxGroups)
       return fail(h, PN_ERR_INVALID, "D=%d needs %d channel groups (max %d)", D, h->fam.ngroups[m], kMaxGroups);
-    h->fam.nchunks[m] = (T + ki.L - 1) / ki.L;
-    h->fam.ntiles[m] = h->fam.ngroups[m] * B * h->fam.nchunks[m];
     if (ki.smem > 48 * 1024) {
       cudaError_t e = cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.smem);
       if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -669,6 +669,17 @@ pn_status select_kernels(pn_ctx* h) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ki.fn, ki.nt, ki.smem) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || per_sm < 1)
       return fail(h, PN_ERR_CUDA, "occupancy query failed for mode %d (D=%d)", m, D);
+    // Kernels that take runs of chunks get one run per resident ticket-taker where the work allows
+    // it: fewer tickets per sequence in flight, so fewer aggregates per look-back.
+    const int chunks = (T + ki.L - 1) / ki.L;
+    int run = 1;
+    if (ki.tpc > 0) {
+      const long long takers = (long long)per_sm * nsm * ki.tpc;
+      run = (int)std::max<long long>(1, ((long long)chunks * B + takers - 1) / takers);
+    }
+    h->fam.run[m] = run;
+    h->fam.nchunks[m] = (chunks + run - 1) / run;
+    h->fam.ntiles[m] = h->fam.ngroups[m] * B * h->fam.nchunks[m];
     const int ng = h->fam.ngroups[m];
     h->fam.resident[m] = per_sm * nsm;
     long long want = (long long)per_sm * nsm;

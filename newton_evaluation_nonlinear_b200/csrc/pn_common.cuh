@@ -85,6 +85,7 @@ struct IterParams {
   int tiles_per_group;  // B * nchunks: tickets of one channel group
   int agg_stride, pref_stride;
   int persist;          // looping kernels: 1 = run iterations until the stop rule, 0 = one iteration
+  int run;              // chunks of L steps per ticket (a run; 1 for the kernels that take single chunks)
   cudaGraphConditionalHandle cond;
 };
 

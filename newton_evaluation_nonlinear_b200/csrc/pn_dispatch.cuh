@@ -30,6 +30,7 @@ struct KInfo {
   size_t smem;      // dynamic shared memory bytes
   int kind;         // KKind: which weight packing the kernel reads
   bool loops = false;   // can run every iteration in one launch (IterParams::persist, grid barrier)
+  int tpc = 0;          // > 0: takes runs of several chunks per ticket, tpc tickets in flight per CTA
 };
 
 template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS>
@@ -112,7 +113,7 @@ inline KInfo dense_kinfo() {
 template <int CELL, int DP, int NW>
 inline KInfo dense_warp_kinfo() {
   using C = DenseWarpCfg<CELL, DP, NW>;
-  return KInfo{(const void*)&dense_warp_kernel<CELL, DP, NW>, C::NT, C::L, DP, C::SMEM_BYTES, kKindDense, true};
+  return KInfo{(const void*)&dense_warp_kernel<CELL, DP, NW>, C::NT, C::L, DP, C::SMEM_BYTES, kKindDense, true, NW};
 }
 
 template <int CELL, int DP>

@@ -203,31 +203,36 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
     if (lane == 0) k = (int)atomicAdd(&ctrl->ticket[0], 1u);
     k = __shfl_sync(0xffffffffu, k, 0);
     if (k >= P.tiles_per_group || aborted) break;
+    // a ticket is a run of P.run consecutive chunks of one sequence
     const int b = k % B;
-    const int chunk = k / B;
-    const int t0 = chunk * L;
+    const int chunk = k / B;                      // run index (the look-back's chain position)
+    const int c_first = chunk * P.run;
+    const int c_end = min(c_first + P.run, (T + L - 1) / L);
 
-    // ---- 1. stage s^(i) rows t0-1 .. t0+L-1 and the step inputs --------------
-    for (int e = lane; e < (L + 1) * DP; e += 32) {
-      const int r = e / DP, c = e % DP;
-      const int tt = t0 - 1 + r;
-      float v = 0.0f;
-      if (c < D) {
-        if (tt < 0) v = __ldg(A.s0 + (size_t)b * D + c);
-        else if (tt < T) v = ld_state(src, ((size_t)b * T + tt) * D + c, fmt.x);
+    // ---- 1. stage s^(i) rows t0-1 .. t0+L-1 and the step inputs of one chunk -------------
+    auto stage = [&](int t0) {
+      __syncwarp();   // the previous chunk's readers are done with the slice
+      for (int e = lane; e < (L + 1) * DP; e += 32) {
+        const int r = e / DP, c = e % DP;
+        const int tt = t0 - 1 + r;
+        float v = 0.0f;
+        if (c < D) {
+          if (tt < 0) v = __ldg(A.s0 + (size_t)b * D + c);
+          else if (tt < T) v = ld_state(src, ((size_t)b * T + tt) * D + c, fmt.x);
+        }
+        sS[r * SP + c] = v;
       }
-      sS[r * SP + c] = v;
-    }
-    for (int e = lane; e < L * R * DP; e += 32) {
-      const int m = e / (R * DP), qc = e % (R * DP);
-      const int q = qc / DP, c = qc % DP;
-      const int tt = t0 + m;
-      sU[m * UP + qc] = (c < D && tt < T) ? __ldg(xin + ((size_t)b * T + tt) * (R * D) + (size_t)q * D + c) : 0.0f;
-    }
-    __syncwarp();
+      for (int e = lane; e < L * R * DP; e += 32) {
+        const int m = e / (R * DP), qc = e % (R * DP);
+        const int q = qc / DP, c = qc % DP;
+        const int tt = t0 + m;
+        sU[m * UP + qc] = (c < D && tt < T) ? __ldg(xin + ((size_t)b * T + tt) * (R * D) + (size_t)q * D + c) : 0.0f;
+      }
+      __syncwarp();
+    };
 
-    // ---- 2. cell phase: lane = step m ------------------------------------------
-    {
+    // ---- 2. cell phase, lane = step m: coefficient vectors, b_m (and |F_m| on the first pass) --
+    auto cell = [&](int t0, bool with_res) {
       const int m = lane;
       const bool tok = (t0 + m) < T;
       float sp[DP];
@@ -310,7 +315,7 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
             res = sci - y;
           }
           if (tok && i < D) {
-            rbits = max(rbits, abs_bits(res));
+            if (with_res) rbits = max(rbits, abs_bits(res));
           } else {   // identity map
             cf[0] = 1.0f;
 #pragma unroll
@@ -322,109 +327,109 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
           sB[m * DP + i] = bb;
         }
       }
-    }
-    __syncwarp();
-
-    // ---- 3. chain [P | q] over the tile --------------------------------------
-    float pold[4][CPL];
-    {
-      // P_0 = A_0, q_0 = b_0
-      float c0[4], cq[R][4];
-      lds_n<4>(sC + 0 * DP + r0, c0);
-#pragma unroll
-      for (int q = 0; q < R; ++q) lds_n<4>(sC + (1 + q) * DP + r0, cq[q]);
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-          const int i = r0 + r, j = j0 + c;
-          float v = (i == j) ? c0[r] : 0.0f;
-#pragma unroll
-          for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], sWj[j * WR + q * DP + i], v);
-          pold[r][c] = v;
-        }
-      if (act) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int c = 0; c < CPL; ++c) sP[(r0 + r) * DP + j0 + c] = pold[r][c];
-        if (cg == 0) *reinterpret_cast<float4*>(sQ + r0) = *reinterpret_cast<const float4*>(sB + r0);
-      }
       __syncwarp();
-    }
+    };
+
+    // ---- 3. chain [P | q] over the run, one chunk at a time --------------------------------
+    // gs counts the run's composition steps: step 0 sets [P | q] = [A_0 | b_0], step gs > 0 composes
+    // with A_m from buffer (gs - 1) & 1 into buffer gs & 1
+    float pold[4][CPL];
+    int gs = 0;
 #pragma unroll 1
-    for (int m = 1; m < L; ++m) {
-      const float* Pk = sP + ((m - 1) & 1) * DP * DP;
-      const float* Qk = sQ + ((m - 1) & 1) * DP;
-      float acc[R][4][CPL];
+    for (int c = c_first; c < c_end; ++c) {
+      const int t0 = c * L;
+      stage(t0);
+      cell(t0, true);
+#pragma unroll 1
+      for (int m = 0; m < L; ++m, ++gs) {
+        float c0[4], cq[R][4], bm[4];
+        lds_n<4>(sC + (m * NCS) * DP + r0, c0);
 #pragma unroll
-      for (int q = 0; q < R; ++q)
+        for (int q = 0; q < R; ++q) lds_n<4>(sC + (m * NCS + 1 + q) * DP + r0, cq[q]);
+        lds_n<4>(sB + m * DP + r0, bm);
+        float* Pn = sP + (gs & 1) * DP * DP;
+        float qn[4];
+        if (gs == 0) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+          for (int r = 0; r < 4; ++r) {
 #pragma unroll
-          for (int c = 0; c < CPL; ++c) acc[q][r][c] = 0.0f;
-      if (act) {
-#pragma unroll 4
-        for (int kk = klo; kk <= khi; ++kk) {
-          float p[CPL];
-          lds_n<CPL>(Pk + kk * DP + j0, p);
+            for (int cc = 0; cc < CPL; ++cc) {
+              const int i = r0 + r, j = j0 + cc;
+              float v = (i == j) ? c0[r] : 0.0f;
 #pragma unroll
-          for (int q = 0; q < R; ++q) {
-            const float4 w = *reinterpret_cast<const float4*>(sWj + kk * WR + q * DP + r0);
-            const float wv[4] = {w.x, w.y, w.z, w.w};
+              for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], sWj[j * WR + q * DP + i], v);
+              pold[r][cc] = v;
+            }
+            qn[r] = bm[r];
+          }
+        } else {
+          const float* Pk = sP + ((gs - 1) & 1) * DP * DP;
+          const float* Qk = sQ + ((gs - 1) & 1) * DP;
+          float acc[R][4][CPL];
+#pragma unroll
+          for (int q = 0; q < R; ++q)
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
-              for (int c = 0; c < CPL; ++c) acc[q][r][c] = fmaf(wv[r], p[c], acc[q][r][c]);
+              for (int cc = 0; cc < CPL; ++cc) acc[q][r][cc] = 0.0f;
+          if (act) {
+#pragma unroll 4
+            for (int kk = klo; kk <= khi; ++kk) {
+              float p[CPL];
+              lds_n<CPL>(Pk + kk * DP + j0, p);
+#pragma unroll
+              for (int q = 0; q < R; ++q) {
+                const float4 w = *reinterpret_cast<const float4*>(sWj + kk * WR + q * DP + r0);
+                const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                  for (int cc = 0; cc < CPL; ++cc) acc[q][r][cc] = fmaf(wv[r], p[cc], acc[q][r][cc]);
+              }
+            }
+          }
+          float qa[R][4];
+          slice_matvec(Qk, qa);
+          float qo[4];
+          lds_n<4>(Qk + r0, qo);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+#pragma unroll
+            for (int cc = 0; cc < CPL; ++cc) {
+              float v = c0[r] * pold[r][cc];
+#pragma unroll
+              for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], acc[q][r][cc], v);
+              pold[r][cc] = v;
+            }
+            float v = fmaf(c0[r], qo[r], bm[r]);
+#pragma unroll
+            for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], qa[q][r], v);
+            qn[r] = v;
           }
         }
-      }
-      float qa[R][4];
-      slice_matvec(Qk, qa);
-      float c0[4], cq[R][4], bm[4], qo[4];
-      lds_n<4>(sC + (m * NCS) * DP + r0, c0);
+        if (act) {
 #pragma unroll
-      for (int q = 0; q < R; ++q) lds_n<4>(sC + (m * NCS + 1 + q) * DP + r0, cq[q]);
-      lds_n<4>(sB + m * DP + r0, bm);
-      lds_n<4>(Qk + r0, qo);
-      float* Pn = sP + (m & 1) * DP * DP;
-      float qn[4];
+          for (int r = 0; r < 4; ++r) {
+            if constexpr (CPL % 4 == 0) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-          float v = c0[r] * pold[r][c];
-#pragma unroll
-          for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], acc[q][r][c], v);
-          pold[r][c] = v;
-        }
-        float v = fmaf(c0[r], qo[r], bm[r]);
-#pragma unroll
-        for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], qa[q][r], v);
-        qn[r] = v;
-      }
-      if (act) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          if constexpr (CPL % 4 == 0) {
-#pragma unroll
-            for (int c = 0; c < CPL; c += 4)
-              *reinterpret_cast<float4*>(Pn + (r0 + r) * DP + j0 + c) =
-                  make_float4(pold[r][c], pold[r][c + 1], pold[r][c + 2], pold[r][c + 3]);
-          } else if constexpr (CPL == 2) {
-            *reinterpret_cast<float2*>(Pn + (r0 + r) * DP + j0) = make_float2(pold[r][0], pold[r][1]);
-          } else {
-            Pn[(r0 + r) * DP + j0] = pold[r][0];
+              for (int cc = 0; cc < CPL; cc += 4)
+                *reinterpret_cast<float4*>(Pn + (r0 + r) * DP + j0 + cc) =
+                    make_float4(pold[r][cc], pold[r][cc + 1], pold[r][cc + 2], pold[r][cc + 3]);
+            } else if constexpr (CPL == 2) {
+              *reinterpret_cast<float2*>(Pn + (r0 + r) * DP + j0) = make_float2(pold[r][0], pold[r][1]);
+            } else {
+              Pn[(r0 + r) * DP + j0] = pold[r][0];
+            }
           }
+          if (cg == 0) *reinterpret_cast<float4*>(sQ + (gs & 1) * DP + r0) = make_float4(qn[0], qn[1], qn[2], qn[3]);
         }
-        if (cg == 0) *reinterpret_cast<float4*>(sQ + (m & 1) * DP + r0) = make_float4(qn[0], qn[1], qn[2], qn[3]);
+        __syncwarp();
       }
-      __syncwarp();
     }
-    const float* Pl = sP + ((L - 1) & 1) * DP * DP;   // aggregate [P_L | q_L]
-    const float* Ql = sQ + ((L - 1) & 1) * DP;
+    const float* Pl = sP + ((gs - 1) & 1) * DP * DP;   // the run's aggregate [P | q]
+    const float* Ql = sQ + ((gs - 1) & 1) * DP;
 
-    // ---- 4. decoupled look-back ------------------------------------------------
+    // ---- 4. decoupled look-back over the runs of the sequence ---------------------------------
     const bool stall = (A.stall_ticket == k);
     if (chunk > 0 && !stall) {
       float* ag = P.agg + (size_t)k * P.agg_stride;
@@ -441,7 +446,7 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
       aborted = true;
       break;
     }
-    // starting state: the end state of the tile n_agg + 1 back, or s0
+    // starting state: the end state of the run n_agg + 1 back, or s0
     float* cur = sX;
     float* nxt = sX + DP;
     if (lane < DP) {
@@ -451,33 +456,49 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
       cur[lane] = v;
     }
     __syncwarp();
-    // fold the aggregates at distances n_agg .. 1, farthest first: carry <- P_d carry + q_d
-    for (int d = n_agg; d >= 1; --d) {
-      const float* ag = P.agg + ((size_t)k - (size_t)d * stride) * P.agg_stride;
-      float part[4], qd[4];
-      float xs[CPL];
-      lds_n<CPL>(cur + j0, xs);
+    // fold the aggregates at distances n_agg .. 1, farthest first: carry <- P_d carry + q_d.  Each
+    // lane's blocks of FB aggregates are loaded together, so a batch costs one L2 round trip.
+    constexpr int FB = (CPL <= 2) ? 4 : 2;
+    for (int d = n_agg; d >= 1; d -= FB) {
+      float blk[FB][4][CPL], qd[FB][4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        float v = 0.0f;
+      for (int u = 0; u < FB; ++u) {
+        const bool use = act && (d - u >= 1);
+        const float* ag = P.agg + ((size_t)k - (size_t)max(d - u, 1) * stride) * P.agg_stride;
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) v = fmaf(act ? __ldcg(ag + (r0 + r) * (DP + 1) + j0 + c) : 0.0f, xs[c], v);
-        part[r] = v;
-        qd[r] = act ? __ldcg(ag + (r0 + r) * (DP + 1) + DP) : 0.0f;
+        for (int r = 0; r < 4; ++r) {
+#pragma unroll
+          for (int cc = 0; cc < CPL; ++cc) blk[u][r][cc] = use ? __ldcg(ag + (r0 + r) * (DP + 1) + j0 + cc) : 0.0f;
+          qd[u][r] = use ? __ldcg(ag + (r0 + r) * (DP + 1) + DP) : 0.0f;
+        }
       }
 #pragma unroll
-      for (int off = 1; off < CG; off <<= 1)
+      for (int u = 0; u < FB; ++u) {
+        if (d - u < 1) break;   // uniform across the warp
+        float xs[CPL];
+        lds_n<CPL>(cur + j0, xs);
+        float part[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
-      if (act && cg == 0)
-        *reinterpret_cast<float4*>(nxt + r0) =
-            make_float4(part[0] + qd[0], part[1] + qd[1], part[2] + qd[2], part[3] + qd[3]);
-      __syncwarp();
-      float* tmp = cur;
-      cur = nxt;
-      nxt = tmp;
+        for (int r = 0; r < 4; ++r) {
+          float v = 0.0f;
+#pragma unroll
+          for (int cc = 0; cc < CPL; ++cc) v = fmaf(blk[u][r][cc], xs[cc], v);
+          part[r] = v;
+        }
+#pragma unroll
+        for (int off = 1; off < CG; off <<= 1)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
+        if (act && cg == 0)
+          *reinterpret_cast<float4*>(nxt + r0) =
+              make_float4(part[0] + qd[u][0], part[1] + qd[u][1], part[2] + qd[u][2], part[3] + qd[u][3]);
+        __syncwarp();
+        float* tmp = cur;
+        cur = nxt;
+        nxt = tmp;
+      }
     }
-    // this tile's end state P_L carry + q_L
+    // this run's end state P carry + q
     if (!stall) {
       float xs[CPL];
       lds_n<CPL>(cur + j0, xs);
@@ -486,7 +507,7 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
       for (int r = 0; r < 4; ++r) {
         float v = 0.0f;
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) v = fmaf(Pl[(r0 + r) * DP + j0 + c], xs[c], v);
+        for (int cc = 0; cc < CPL; ++cc) v = fmaf(Pl[(r0 + r) * DP + j0 + cc], xs[cc], v);
         part[r] = v;
       }
 #pragma unroll
@@ -502,47 +523,61 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
       if (lane == 0) st_release(P.flags + k, make_flag(epoch, kFlagPrefix));
     }
 
-    // ---- 5. apply the carry step by step, write the states ----------------------
+    // ---- 5. apply the carry step by step over the run, chunk by chunk, write the states ------
+    // (the carry moves to the end of sO's row space: sX keeps it across the chunks' restaging)
     {
       float sold[4];
       lds_n<4>(cur + r0, sold);
-      const float* xcur = cur;
-#pragma unroll 1
-      for (int m = 0; m < L; ++m) {
-        float pa[R][4];
-        slice_matvec(xcur, pa);
-        float c0[4], cq[R][4], bm[4];
-        lds_n<4>(sC + (m * NCS) * DP + r0, c0);
-#pragma unroll
-        for (int q = 0; q < R; ++q) lds_n<4>(sC + (m * NCS + 1 + q) * DP + r0, cq[q]);
-        lds_n<4>(sB + m * DP + r0, bm);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          float v = fmaf(c0[r], sold[r], bm[r]);
-#pragma unroll
-          for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], pa[q][r], v);
-          sold[r] = v;
-        }
-        if (act && cg == 0) *reinterpret_cast<float4*>(sO + m * DP + r0) = make_float4(sold[0], sold[1], sold[2], sold[3]);
+      if (cur != sX) {   // keep the running state at sX[0 .. DP-1]
+        if (act && cg == 0) *reinterpret_cast<float4*>(sX + r0) = make_float4(sold[0], sold[1], sold[2], sold[3]);
         __syncwarp();
-        xcur = sO + m * DP;
       }
-      for (int e = lane; e < L * DP; e += 32) {
-        const int m = e / DP, i = e % DP;
-        const int tt = t0 + m;
-        if (tt < T && i < D) {
-          float v = sO[e];
-          if (damped) {
-            const float sc = sS[(m + 1) * SP + i];   // s^(i)_t
-            v = fmaf(lambda, v - sc, sc);
-          }
-          st_state(dst, ((size_t)b * T + tt) * D + i, v, fmt.y);
+#pragma unroll 1
+      for (int c = c_first; c < c_end; ++c) {
+        const int t0 = c * L;
+        if (P.run > 1) {   // the first pass's coefficients belong to the run's last chunk
+          stage(t0);
+          cell(t0, false);
         }
+        const float* xcur = sX;
+#pragma unroll 1
+        for (int m = 0; m < L; ++m) {
+          float pa[R][4];
+          slice_matvec(xcur, pa);
+          float c0[4], cq[R][4], bm[4];
+          lds_n<4>(sC + (m * NCS) * DP + r0, c0);
+#pragma unroll
+          for (int q = 0; q < R; ++q) lds_n<4>(sC + (m * NCS + 1 + q) * DP + r0, cq[q]);
+          lds_n<4>(sB + m * DP + r0, bm);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            float v = fmaf(c0[r], sold[r], bm[r]);
+#pragma unroll
+            for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], pa[q][r], v);
+            sold[r] = v;
+          }
+          if (act && cg == 0) *reinterpret_cast<float4*>(sO + m * DP + r0) = make_float4(sold[0], sold[1], sold[2], sold[3]);
+          __syncwarp();
+          xcur = sO + m * DP;
+        }
+        for (int e = lane; e < L * DP; e += 32) {
+          const int m = e / DP, i = e % DP;
+          const int tt = t0 + m;
+          if (tt < T && i < D) {
+            float v = sO[e];
+            if (damped) {
+              const float sc = sS[(m + 1) * SP + i];   // s^(i)_t
+              v = fmaf(lambda, v - sc, sc);
+            }
+            st_state(dst, ((size_t)b * T + tt) * D + i, v, fmt.y);
+          }
+        }
+        // the chunk's last state starts the next chunk
+        if (act && cg == 0) *reinterpret_cast<float4*>(sX + r0) = make_float4(sold[0], sold[1], sold[2], sold[3]);
+        __syncwarp();
       }
-      __syncwarp();   // the warp's slice is restaged by the next tile
     }
   }
-
   // ---- residual of this iteration; the next one (grid barrier) or the end of the launch
   rbits = warp_max_u32(rbits);
   if (lane == 0) sRed[warp] = __uint_as_float(rbits);

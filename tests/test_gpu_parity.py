@@ -76,10 +76,22 @@ def _check_against_oracle(prob, mode, tol=None, max_iters=None, device_loop=1, t
         assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq)), (_relerr(s, seq), _relerr(s_or, seq))
     # residual history: fp32 residuals track the fp64 ones, up to rounding of the scanned iterate
     # (a few ulp of max|s| per step, accumulated along the chain)
-    n = min(len(hist), len(hist_or))
-    scale = max(1.0, float(np.abs(seq).max()))
-    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=HIST_RTOL, atol=HIST_ATOL * scale)
+    _check_history(hist, hist_or, max(1.0, float(np.abs(seq).max())))
     return it, s
+
+
+def _check_history(hist, hist_or, scale):
+    """Residual histories, fp32 against fp64, element by element (see HIST_RTOL / HIST_ATOL).  An
+    iteration that passes through a large iterate (a residual far above max|s|: the Euler drift under
+    quasi-Newton can reach 1e5 before it contracts) carries float32 rounding at that scale into every
+    later iterate, so each later residual also gets an absolute allowance of 8 float32 ulps (2^-20)
+    of the largest oracle residual so far."""
+    n = min(len(hist), len(hist_or))
+    h, ho = np.asarray(hist[:n], np.float64), np.asarray(hist_or[:n], np.float64)
+    peak = np.maximum.accumulate(np.abs(ho)) if n else ho
+    bound = HIST_ATOL * scale + 2.0 ** -20 * peak + HIST_RTOL * np.abs(ho)
+    bad = np.nonzero(np.abs(h - ho) > bound)[0]
+    assert bad.size == 0, [(int(i), float(h[i]), float(ho[i]), float(bound[i])) for i in bad[:5]]
 
 
 CELLS = [pi.CELL_TANH_RNN, pi.CELL_GRU, pi.CELL_EULER]

@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 import pn_inputs as pi
+from test_gpu_parity import _check_history
 
 pytestmark = pytest.mark.gpu
 
@@ -66,8 +67,7 @@ def _check(cell, D, T, B, band, damping, seed, mode="newton", tc=1):
         assert _relerr(s, s_or) <= REL_TOL, _relerr(s, s_or)
     if st == oracle.OK:
         assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq))
-    n = min(len(hist), len(hist_or))
-    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=1e-2, atol=5e-6 * max(1.0, float(np.abs(seq).max())))
+    _check_history(hist, hist_or, max(1.0, float(np.abs(seq).max())))
 
 
 @pytest.mark.parametrize("cell", CELLS)
@@ -95,9 +95,11 @@ def test_damped_diagonal_modes_match_oracle(cell, mode, D, tc):
 
 
 def test_damping_arguments_and_switching():
+    """Damping toggles the kernel choice of Picard (tensor-core row-major kernel undamped, FP32 kernel
+    damped) and back; the Euler drift keeps Picard contractive over the whole sequence."""
     import torch
     import newton_evaluation_nonlinear_b200 as pn
-    prob = pi.random_problem(331, pi.CELL_TANH_RNN, 64, 64, T=300, B=1, rho=0.5)
+    prob = pi.random_problem(331, pi.CELL_EULER, 64, 64, T=300, B=1, rho=0.5, eps=0.05)
     solver = pn.Solver.from_problem(prob)
     for bad in (0.0, -0.5, 1.5, float("nan")):
         with pytest.raises(pn.PnError):
@@ -112,7 +114,8 @@ def test_damping_arguments_and_switching():
     solver.set_damping(1.0)   # back to the undamped kernels: the same result as before
     for m in ("picard", "quasi"):
         states, it, r, st = solver.eval(x, s0, m, 300, 1e-5)
-        np.testing.assert_allclose(states.cpu().numpy(), ref[m], rtol=0, atol=1e-6)
+        ref_m = ref[m]
+        np.testing.assert_allclose(states.cpu().numpy(), ref_m, rtol=0, atol=1e-6 * max(1.0, float(np.abs(ref_m).max())))
     solver.close()
 
 
