@@ -70,6 +70,13 @@ struct pn_ctx {
   Args* args = nullptr;
   float* hist = nullptr;
   CUtensorMap* tmaps = nullptr;   // TMA descriptors of the tensor-core kernels (kTcMaps, see IterParams)
+  // wide one-gate cells (D = 128, 256): the tensor-core product Y = S W^T before each iteration
+  bool wide_capable = false;
+  float* wt_hi = nullptr;          // TF32 split of W, row-major [D][D]
+  float* wt_lo = nullptr;
+  float* ypre = nullptr;           // [B*T][D]
+  CUtensorMap* wmaps = nullptr;    // [0]/[1] S of iterate buffer 0 / 1, [2] W_hi, [3] W_lo
+  CUtensorMap* wmaps_h = nullptr;
   // host pinned mirrors
   Args* args_h = nullptr;
   Ctrl* ctrl_h = nullptr;
@@ -177,6 +184,14 @@ void free_all(pn_ctx* h) {
     if (*p) cudaFree(*p);
     *p = nullptr;
   }
+  for (float** p : {&h->wt_hi, &h->wt_lo, &h->ypre}) {
+    if (*p) cudaFree(*p);
+    *p = nullptr;
+  }
+  if (h->wmaps) cudaFree(h->wmaps);
+  if (h->wmaps_h) cudaFreeHost(h->wmaps_h);
+  h->wmaps = nullptr;
+  h->wmaps_h = nullptr;
   if (h->flags) cudaFree(h->flags);
   if (h->tmaps) cudaFree(h->tmaps);
   if (h->tmaps_h) cudaFreeHost(h->tmaps_h);
@@ -207,6 +222,7 @@ IterParams make_params(const pn_ctx* h, int mode) {
   P.wt = dense ? h->wt_dense
                : (kind == kKindDiagTc ? h->wt_tc : (kind == kKindDiagTct ? h->wt_tct : h->wt_diag));
   P.wt_tc = h->wt_tc;
+  P.ypre = h->ypre;
   P.wdiag = h->wdiag;
   P.bhn = h->bhn;
   P.xin = h->xin;
@@ -273,6 +289,30 @@ bool encode_seq(CUtensorMap* m, const void* base, int cols, int T, int B, int bo
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Map over a row-major fp32 matrix [rows][cols] whose box is box_rows x box_cols,
+// 128-byte swizzled (the tensor cores' K-major operand layout for 32-float rows).
+bool encode_2d_sw128(CUtensorMap* m, const void* base, int cols, long long rows, int box_cols, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (!fn || !base) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(float)};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The wide product's maps for the current call: S of both iterate buffers (128 rows x 32
+// floats per box) and W_hi, W_lo (D rows x 32 floats).
+bool encode_wide_maps(const pn_ctx* h, CUtensorMap* out) {
+  const long long rows = (long long)h->B * h->T;
+  return encode_2d_sw128(&out[0], h->args_h->states, h->D, rows, 32, 128) &&
+         encode_2d_sw128(&out[1], h->buf1, h->D, rows, 32, 128) &&
+         encode_2d_sw128(&out[2], h->wt_hi, h->D, h->D, 32, h->D) &&
+         encode_2d_sw128(&out[3], h->wt_lo, h->D, h->D, 32, h->D);
+}
+
 // Fills the pinned mirror of the maps of the tensor-core kernels for the
 // buffers of the current call (iterate buffer 0 is the caller's states,
 // buffer 1 is buf1; the step inputs are the hoisted projection, or x itself
@@ -319,6 +359,33 @@ PreLaunch pre_launch(const pn_ctx* h) {
   p.init_grid = dim3(gx, gy);
   p.fin_grid = grid_1d(n / 4 + 1, 256, 148u * 16u);
   return p;
+}
+
+// Launch shape and arguments of the wide product (wide_gemm_kernel) of `mode`.
+struct PreArgs {
+  const CUtensorMap* maps;
+  float* y;
+  int rows;
+  Ctrl* ctrl;
+  const Args* args;
+  void* kargs[5];
+  unsigned grid;
+};
+void pre_args(pn_ctx* h, PreArgs& a) {
+  a.maps = h->wmaps;
+  a.y = h->ypre;
+  a.rows = h->B * h->T;
+  a.ctrl = h->ctrl;
+  a.args = h->args;
+  a.kargs[0] = (void*)&a.maps;
+  a.kargs[1] = (void*)&a.y;
+  a.kargs[2] = (void*)&a.rows;
+  a.kargs[3] = (void*)&a.ctrl;
+  a.kargs[4] = (void*)&a.args;
+  int nsm = 148;
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, h->device);
+  const int tiles = (a.rows + 127) / 128;
+  a.grid = (unsigned)std::max(1, std::min(nsm, tiles));
 }
 
 pn_status build_graph(pn_ctx* h, int mode) {
@@ -378,9 +445,17 @@ pn_status build_graph(pn_ctx* h, int mode) {
     IterParams P = make_params(h, mode);
     P.cond = cond;
     void* kargs[] = {(void*)&P};
-    cudaGraphNode_t knode;
+    cudaGraphNode_t knode, pnode;
+    PreArgs pa;
+    cudaGraphNode_t* dep = nullptr;
+    if (ki.pre_fn) {
+      pre_args(h, pa);
+      e = add_kernel(body, ki.pre_fn, dim3(pa.grid), dim3(ki.pre_nt), ki.pre_smem, pa.kargs, nullptr, &pnode);
+      if (e != cudaSuccess) goto fail_graph;
+      dep = &pnode;
+    }
     e = add_kernel(body, ki.fn, dim3((unsigned)h->fam.grid[mode]), dim3(ki.nt), ki.smem, kargs,
-                   nullptr, &knode);
+                   dep, &knode);
     if (e != cudaSuccess) goto fail_graph;
     prev = node;
   }
@@ -420,6 +495,11 @@ pn_status launch_iter(pn_ctx* h, int mode, int persist = 0) {
   P.persist = persist;
   void* kargs[] = {(void*)&P};
   const unsigned grid = (unsigned)h->fam.grid[mode];
+  if (ki.pre_fn) {   // the tensor-core product the iteration kernel reads
+    PreArgs pa;
+    pre_args(h, pa);
+    PN_CUDA(h, cudaLaunchKernel(ki.pre_fn, dim3(pa.grid), dim3(ki.pre_nt), pa.kargs, ki.pre_smem, h->stream));
+  }
   if (!ki.loops) {
     PN_CUDA(h, cudaLaunchKernel(ki.fn, dim3(grid), dim3(ki.nt), kargs, ki.smem, h->stream));
     return PN_OK;
@@ -523,6 +603,12 @@ pn_status prepare_lookback(pn_ctx* h, int mode) {
 // The copy is ordered before the launches on the same stream; the pinned
 // mirror is not touched again before the call's final synchronisation.
 pn_status upload_tc_maps(pn_ctx* h, int mode) {
+  if (h->fam.k[mode].pre_fn) {
+    if (!encode_wide_maps(h, h->wmaps_h))
+      return fail(h, PN_ERR_CUDA, "encoding the wide product's tensor maps failed (D=%d, T=%d, B=%d)", h->D, h->T, h->B);
+    PN_CUDA(h, cudaMemcpyAsync(h->wmaps, h->wmaps_h, 4 * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
+    return PN_OK;
+  }
   if (!tagged_lookback(h->fam.k[mode].kind)) return PN_OK;
   if (!encode_tc_maps(h, mode, h->tmaps_h))
     return fail(h, PN_ERR_CUDA, "encoding the TMA tensor maps failed (D=%d, T=%d, B=%d)", h->D, h->T, h->B);
@@ -665,6 +751,10 @@ pn_status select_kernels(pn_ctx* h) {
       cudaError_t e = cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.smem);
       if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     }
+    if (ki.pre_fn && ki.pre_smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(ki.pre_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.pre_smem);
+      if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    }
     int per_sm = 0, nsm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ki.fn, ki.nt, ki.smem) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || per_sm < 1)
@@ -759,6 +849,7 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
   h->DP = padded_width(D);
   h->use_tma = (D % 4) == 0;
   h->tc_capable = (D == h->DP) && (D == 32 || (D == 64 && cell != PN_CELL_GRU));
+  h->wide_capable = (D == h->DP) && (D == 128 || D == 256) && cell != PN_CELL_GRU;
   h->stream = (cudaStream_t)cuda_stream;
   if (cudaGetDevice(&h->device) != cudaSuccess) {
     delete h;
@@ -773,7 +864,7 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
     pn_status sk = PN_OK;
     for (int pass = 0; pass < 2 && sk == PN_OK; ++pass) {
       h->tc_opt = (pass == 1);
-      h->use_tc = (pass == 0) ? false : h->tc_capable;
+      h->use_tc = (pass == 0) ? false : (h->tc_capable || h->wide_capable);
       sk = select_kernels(h);
     }
     if (sk != PN_OK) {
@@ -891,6 +982,27 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
       }
     }
     PN_TRY(dalloc(h, &h->buf1, BT * D));
+    if (h->wide_capable) {
+      // the wide product's operands: W split into TF32 hi and lo parts (row-major, for the swizzled
+      // tensor loads), its output Y, and the tensor maps
+      std::vector<float> whi((size_t)D * D), wlo((size_t)D * D);
+      for (int j = 0; j < D; ++j)
+        for (int k = 0; k < D; ++k) {
+          const float w = w_block(h, params, 0, j, k);
+          whi[(size_t)j * D + k] = tf32_round(w);
+          wlo[(size_t)j * D + k] = tf32_round(w - tf32_round(w));
+        }
+      PN_TRY(dalloc(h, &h->wt_hi, whi.size()));
+      PN_TRY(dalloc(h, &h->wt_lo, wlo.size()));
+      PN_TRY(dalloc(h, &h->ypre, BT * D));
+      if (cudaMemcpy(h->wt_hi, whi.data(), whi.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+          cudaMemcpy(h->wt_lo, wlo.data(), wlo.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+          cudaMalloc((void**)&h->wmaps, 4 * sizeof(CUtensorMap)) != cudaSuccess ||
+          cudaMallocHost((void**)&h->wmaps_h, 4 * sizeof(CUtensorMap)) != cudaSuccess) {
+        st = fail(h, PN_ERR_NOMEM, "allocating the wide product's buffers failed");
+        goto bad;
+      }
+    }
     PN_TRY(dalloc(h, &h->flags, h->nflags));
     PN_TRY(dalloc(h, &h->agg, h->agg_floats));
     PN_TRY(dalloc(h, &h->pref, h->pref_floats));
@@ -1275,7 +1387,7 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
       return PN_OK;
     case PN_OPT_TENSOR_CORES: {
       if (value != 0 && value != 1) return fail(h, PN_ERR_INVALID, "tensor-core option is 0 or 1");
-      const bool want = (value == 1) && h->tc_capable;
+      const bool want = (value == 1) && (h->tc_capable || h->wide_capable);
       if (want == h->use_tc && (value == 1) == h->tc_opt) return PN_OK;
       DeviceGuard dg(h->device);
       if (h->stream) cudaStreamSynchronize(h->stream);

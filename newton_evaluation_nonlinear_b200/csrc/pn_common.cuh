@@ -67,6 +67,7 @@ struct Args {
 struct IterParams {
   const float* wt;     // recurrent weights, pre-packed per group: [ngroups][DP][R*G]
   const float* wt_tc;  // W_q rows split for the tensor cores: [W_hi; W_lo], K-major core-matrix layout
+  const float* ypre;   // wide states: W s^(i)_r for every row r = b T + t, from the tensor cores
   const float* wdiag;  // diagonal entries per gate: [R][DP] (quasi mode)
   const float* bhn;    // GRU b_hn [DP] (zero-padded); unused otherwise
   const float* xin;    // per-step cell input: u [B][T][D] (tanh), gx [B][T][3D] (GRU); NULL for Euler

@@ -13,6 +13,7 @@
 #include "pn_iter_diag_tc.cuh"
 #include "pn_iter_diag_tct.cuh"
 #include "pn_iter_diag_tma.cuh"
+#include "pn_wide_gemm.cuh"
 
 namespace pn {
 
@@ -31,6 +32,9 @@ struct KInfo {
   int kind;         // KKind: which weight packing the kernel reads
   bool loops = false;   // can run every iteration in one launch (IterParams::persist, grid barrier)
   int tpc = 0;          // > 0: takes runs of several chunks per ticket, tpc tickets in flight per CTA
+  const void* pre_fn = nullptr;   // launched before fn in every iteration (the tensor-core product Y = S W^T)
+  int pre_nt = 0;
+  size_t pre_smem = 0;
 };
 
 template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS>
@@ -133,6 +137,20 @@ inline KInfo dense_pick() {
   }
 }
 
+// Wide one-gate cells (DP = 128, 256): the recurrent product of every step on the tensor cores
+// (wide_gemm_kernel), then the FP32 diagonal kernel reading it.
+template <int CELL, int MODE, int DP>
+inline KInfo diag_wide_kinfo() {
+  using C = DiagCfg<CELL, MODE, DP, 64, 4, 4, 16, true>;
+  using W = WideGemmCfg<DP>;
+  KInfo k{(const void*)&diag_iter_kernel<CELL, MODE, DP, 64, 4, 4, 16, true>, C::NT, C::L, 64, C::SMEM_BYTES,
+          kKindDiag};
+  k.pre_fn = (const void*)&wide_gemm_kernel<DP>;
+  k.pre_nt = W::NT;
+  k.pre_smem = (size_t)W::SMEM_BYTES;
+  return k;
+}
+
 // Newton with the compositions on the tensor cores: one-gate cells, DP = 32 or 64.
 template <int CELL, int DP>
 inline KInfo dense_tc_kinfo() {
@@ -150,6 +168,14 @@ inline KInfo lookup_cell(int mode, int DP, bool tma, bool tc) {
     if (tc && mode == PN_NEWTON) {
       if (DP == 32) return dense_tc_kinfo<CELL, 32>();
       if (DP == 64) return dense_tc_kinfo<CELL, 64>();
+    }
+    if (tc && mode != PN_NEWTON && (DP == 128 || DP == 256)) {
+#define PN_WIDE(MODE_)                                              \
+  return DP == 128 ? diag_wide_kinfo<CELL, MODE_, 128>() : diag_wide_kinfo<CELL, MODE_, 256>();
+      if (mode == PN_JACOBI) { PN_WIDE(PN_JACOBI) }
+      if (mode == PN_PICARD) { PN_WIDE(PN_PICARD) }
+      PN_WIDE(PN_QUASI)
+#undef PN_WIDE
     }
   }
   if (tc && mode != PN_NEWTON) {

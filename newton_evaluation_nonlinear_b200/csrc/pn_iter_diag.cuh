@@ -35,7 +35,10 @@
 
 namespace pn {
 
-template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS>
+// PRE: the recurrent product W s_{t-1} of every step comes precomputed from the
+// tensor cores (pn_wide_gemm.cuh) in IterParams::ypre, row b T + t - 1 for step t
+// (step 0 forms W s0 itself); the CTA stages only its channel group's states.
+template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS, bool PRE = false>
 struct DiagCfg {
   static constexpr int R = CellInfo<CELL>::R;
   static constexpr int L = TS * TM;           // steps per tile
@@ -48,7 +51,7 @@ struct DiagCfg {
   static constexpr int NQ = (G + 31) / 32;    // channels per lane in the look-back warp
   static constexpr int OFF_S = 0;
   static constexpr int OFF_W = OFF_S + DP * LP;
-  static constexpr int OFF_AGG = OFF_W + DP * WCOLS;
+  static constexpr int OFF_AGG = OFF_W + (PRE ? 0 : DP * WCOLS);
   static constexpr int OFF_PART = OFF_AGG + 2 * G;
   static constexpr int OFF_CARRY = OFF_PART + 2 * JG * WPG * TN;
   static constexpr int OFF_RED = OFF_CARRY + G;
@@ -60,12 +63,13 @@ struct DiagCfg {
   static_assert((TS & (TS - 1)) == 0 && (TS <= 32 || TS % 32 == 0), "TS must be a power of two");
   static_assert(TN == 1 || TN == 2 || TN == 4, "TN must be 1, 2 or 4");
   static_assert(OFF_W % 4 == 0 && LP % 4 == 0, "16-byte alignment of shared tiles");
+  static_assert(!PRE || R == 1, "precomputed products: one-gate cells");
 };
 
-template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS>
-__global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
+template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS, bool PRE = false>
+__global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS, PRE>::NT)
     diag_iter_kernel(const IterParams P) {
-  using C = DiagCfg<CELL, MODE, DP, G, TM, TN, TS>;
+  using C = DiagCfg<CELL, MODE, DP, G, TM, TN, TS, PRE>;
   constexpr int R = C::R;
   constexpr int L = C::L;
   constexpr int LP = C::LP;
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
   const bool dvec = (D % 4) == 0;
 
   // weights of this group, once per launch
-  {
+  if constexpr (!PRE) {
     const float4* wsrc = reinterpret_cast<const float4*>(P.wt + (size_t)g * DP * C::WCOLS);
     float4* wdst = reinterpret_cast<float4*>(sW);
     for (int e = tid; e < DP * C::WCOLS / 4; e += C::NT) wdst[e] = __ldg(wsrc + e);
@@ -160,11 +164,11 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
 
     // ---- 1b. stage s rows t0-1 .. t0+L-1 transposed: sT[k][r], time t0-1+r
     {
-      constexpr int Q4 = DP / 4;
+      constexpr int Q4 = PRE ? G / 4 : DP / 4;   // PRE: only this group's channels are read
       constexpr int RB = (L + 1 + 7) / 8;
       for (int e = tid; e < RB * Q4 * 8; e += C::NT) {
         const int rl = e & 7;
-        const int c4 = (e >> 3) % Q4;
+        const int c4 = (e >> 3) % Q4 + (PRE ? g * (G / 4) : 0);
         const int r = ((e >> 3) / Q4) * 8 + rl;
         if (r > L) continue;
         const int c = c4 * 4;
@@ -202,7 +206,10 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
         const int cw = (n < cvalid) ? c : 0;
         const int jl = j0 + n;
 #pragma unroll
-        for (int q = 0; q < R; ++q) wd[n][q] = sW[cw * C::WCOLS + q * G + jl];
+        for (int q = 0; q < R; ++q) {
+          if constexpr (PRE) wd[n][q] = (n < cvalid) ? __ldg(P.wdiag + q * DP + c) : 0.0f;
+          else wd[n][q] = sW[cw * C::WCOLS + q * G + jl];
+        }
         bhn[n] = (CELL == PN_CELL_GRU && n < cvalid) ? __ldg(P.bhn + c) : 0.0f;
       }
     }
@@ -217,8 +224,25 @@ __global__ void __launch_bounds__(DiagCfg<CELL, MODE, DP, G, TM, TN, TS>::NT)
 #pragma unroll
         for (int n = 0; n < TN; ++n) acc[m][q][n] = 0.0f;
 
+    if constexpr (PRE) {
+      // W s_{t-1} from the tensor cores' product; step 0 of a sequence: W s0, formed here
+#pragma unroll
+      for (int m = 0; m < TM; ++m) {
+        const int t = t0 + m0 + m;
+        if (t >= 1 && t < T && cvalid > 0) {
+          load_n<TN>(P.ypre + ((size_t)b * T + t - 1) * D + c0, acc[m][0], cvalid, vec_ok);
+        } else if (t == 0) {
+          for (int kk = 0; kk < D; ++kk) {
+            const float s0k = __ldg(A.s0 + (size_t)b * D + kk);
+#pragma unroll
+            for (int n = 0; n < TN; ++n)
+              acc[m][0][n] = fmaf(__ldg(P.wt + ((size_t)g * DP + kk) * G + j0 + n), s0k, acc[m][0][n]);
+          }
+        }
+      }
+    }
 #pragma unroll(DP <= 64 ? DP : 8)
-    for (int kk = 0; kk < DP; ++kk) {
+    for (int kk = 0; kk < (PRE ? 0 : DP); ++kk) {
       const float4 sv = *reinterpret_cast<const float4*>(sT + kk * LP + m0);
       const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
       const float* wrow = sW + kk * C::WCOLS + j0;

@@ -1,0 +1,231 @@
+// pn_wide_gemm.cuh -- the cell's recurrent product for wide states (D = 128,
+// 256) on the tensor cores: Y = S W^T over all B*T steps of an iterate, as
+// 3xTF32 tcgen05.mma with W streamed from L2 in 32-column K chunks.
+//
+// At D = 256 one step's W s costs 2 D^2 = 131 kflop, so an iteration of the
+// Euler workload (B = 32, T = 1024) is 4.3 GFLOP: about 60 us of the FP32 FMA
+// peak against 15 us of HBM traffic, and W_hi + W_lo (512 KB) do not fit in
+// shared memory.  Here the product runs as a plain GEMM on the tensor cores
+// (rows r = b T + t of the iterate, Y[r][n] = sum_k S[r][k] W[n][k] =
+// (W s_r)[n]) and the fused cell + Jacobian + scan kernel reads Y instead of
+// forming W s itself ("Parallel Newton methods..." page, §5.2: tensor cores as
+// the hardware lever; the iteration itself is §1.2 and §2.2).  Products are
+// 3xTF32 as in the other tensor-core kernels: S W_hi + S W_lo + S_lo W_hi,
+// with S read by the tensor core as its TF32 truncation and S_lo the exact
+// remainder, formed in shared memory.
+//
+// Per CTA (persistent, static round-robin over 128-row tiles):
+//   warp 0   producer: per (tile, K chunk) one TMA load of the S chunk
+//            (128 rows x 32 floats) and of W_hi and W_lo (D rows x 32),
+//            128-byte swizzled, into a stage of the ring;
+//   warp 1   MMA issuer: 3 passes x 4 K-steps per chunk into one of two TMEM
+//            accumulators (128 lanes x D columns); a commit frees the stage;
+//   warps 2-3  S_lo of each landed S chunk (element-wise: the swizzled
+//            layout is the same for both);
+//   warps 4-7  epilogue: thread = row, TMEM -> registers -> Y.
+// TMA loads never use cluster multicast.  Rows past B*T read as zero and are
+// not stored.
+#pragma once
+
+#include "pn_iter_diag_tc.cuh"
+
+namespace pn {
+
+template <int DP>
+struct WideGemmCfg {
+  static_assert(DP == 128 || DP == 256, "wide states: D = 128 or 256");
+  static constexpr int BM = 128;                  // rows per tile
+  static constexpr int KC = 32;                   // K chunk: one 128-byte swizzle row of fp32
+  static constexpr int NKC = DP / KC;             // chunks per tile
+  static constexpr int S_BYTES = BM * KC * 4;     // 16 KB
+  static constexpr int W_BYTES = DP * KC * 4;     // 16 or 32 KB
+  static constexpr int STAGE = 2 * S_BYTES + 2 * W_BYTES;   // S, S_lo, W_hi, W_lo
+  static constexpr int NSTAGE = (DP == 128) ? 3 : 2;
+  static constexpr int TCOLS = 2 * DP;            // two accumulators
+  static constexpr int NT = 256;                  // 8 warps
+  static constexpr int SMEM_BYTES = NSTAGE * STAGE + 1024;   // + slack to align the ring to 1024 bytes
+  static_assert(TCOLS <= 512, "TMEM columns");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+// 2-D TMA tensor load (coordinates: column c0, row c1), counted on bar.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_addr(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// maps: [0] S of iterate buffer 0, [1] S of buffer 1, [2] W_hi, [3] W_lo.
+template <int DP>
+__global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __restrict__ maps, float* __restrict__ Y,
+                                                           int rows, Ctrl* ctrl, const Args* __restrict__ args) {
+  using C = WideGemmCfg<DP>;
+  constexpr int NS = C::NSTAGE;
+  constexpr int NKC = C::NKC;
+  extern __shared__ __align__(1024) unsigned char smem_wg[];
+  unsigned char* ring = smem_wg + ((1024u - (smem_addr(smem_wg) & 1023u)) & 1023u);
+  __shared__ __align__(8) uint64_t bar_full[NS], bar_lo[NS], bar_empty[NS], bar_acc[2], bar_accfree[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+  __shared__ int s_loaded, s_issued;   // units whose loads / products were issued (for the drain)
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const long long tmo = args->timeout_ns;
+  const int iter = *(volatile int*)&ctrl->iter;
+  const CUtensorMap* mS = maps + ((iter & 1) ? 1 : 0);   // s^(i)
+  const CUtensorMap* mWh = maps + 2;
+  const CUtensorMap* mWl = maps + 3;
+  const int ntiles = (rows + C::BM - 1) / C::BM;
+  const int my_tiles = (ntiles > (int)blockIdx.x) ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int units = my_tiles * NKC;
+
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar_full[s], 1u);
+      mbar_init(&bar_lo[s], 2u);
+      mbar_init(&bar_empty[s], 1u);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bar_acc[a], 1u);
+      mbar_init(&bar_accfree[a], 4u);
+    }
+    mbar_init_fence();
+    s_abort = 0;
+    s_loaded = 0;
+    s_issued = 0;
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
+                 "r"((uint32_t)C::TCOLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  auto sbuf = [&](int s) { return ring + s * C::STAGE; };                 // S chunk
+  auto lbuf = [&](int s) { return ring + s * C::STAGE + C::S_BYTES; };    // S_lo
+  auto hbuf = [&](int s) { return ring + s * C::STAGE + 2 * C::S_BYTES; };   // W_hi
+  auto wlbuf = [&](int s) { return hbuf(s) + C::W_BYTES; };                  // W_lo
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      tmap_acquire(mS);
+      tmap_acquire(mWh);
+      tmap_acquire(mWl);
+      asm volatile("fence.proxy.async.global;" ::: "memory");   // s^(i) written by the previous kernel
+      for (int u = 0; u < units; ++u) {
+        const int s = u % NS;
+        if (u >= NS && !mbar_wait_flag(&bar_empty[s], (unsigned)((u / NS) - 1) & 1u, ctrl, tmo, &s_abort)) break;
+        const int tile = (int)blockIdx.x + (u / NKC) * (int)gridDim.x;
+        const int kc = u % NKC;
+        mbar_arrive_expect_tx(&bar_full[s], (unsigned)(C::S_BYTES + 2 * C::W_BYTES));
+        tma_load_2d(sbuf(s), mS, kc * C::KC, tile * C::BM, &bar_full[s]);
+        tma_load_2d(hbuf(s), mWh, kc * C::KC, 0, &bar_full[s]);
+        tma_load_2d(wlbuf(s), mWl, kc * C::KC, 0, &bar_full[s]);
+        s_loaded = u + 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    constexpr uint32_t idesc = umma_idesc_tf32(C::BM, DP);
+    for (int u = 0; u < units; ++u) {
+      const int s = u % NS;
+      const int j = u / NKC;    // this CTA's tile number
+      const int kc = u % NKC;
+      const int acc = j & 1;
+      if (kc == 0 && j >= 2 && !mbar_wait_flag(&bar_accfree[acc], (unsigned)((j >> 1) - 1) & 1u, ctrl, tmo, &s_abort))
+        break;
+      if (!mbar_wait_flag(&bar_lo[s], (unsigned)(u / NS) & 1u, ctrl, tmo, &s_abort)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint64_t a_hi = umma_smem_desc(smem_addr(sbuf(s)), 16, 1024, 2);
+        const uint64_t a_lo = umma_smem_desc(smem_addr(lbuf(s)), 16, 1024, 2);
+        const uint64_t b_hi = umma_smem_desc(smem_addr(hbuf(s)), 16, 1024, 2);
+        const uint64_t b_lo = umma_smem_desc(smem_addr(wlbuf(s)), 16, 1024, 2);
+        const uint32_t d = tmem + (uint32_t)(acc * DP);
+#pragma unroll
+        for (int ks = 0; ks < C::KC / 8; ++ks) {
+          const uint64_t ko = (uint64_t)((ks * 32) >> 4);   // 8 fp32 of K = 32 bytes along the swizzled row
+          umma_tf32(d, a_hi + ko, b_hi + ko, idesc, (kc | ks) ? 1u : 0u);
+          umma_tf32(d, a_hi + ko, b_lo + ko, idesc, 1u);
+          umma_tf32(d, a_lo + ko, b_hi + ko, idesc, 1u);
+        }
+        umma_commit(&bar_empty[s]);                 // the stage is free once these products are done
+        if (kc == NKC - 1) umma_commit(&bar_acc[acc]);   // the tile's accumulator is complete
+        s_issued = u + 1;
+      }
+      __syncwarp();
+    }
+  } else if (warp < 4) {
+    // ---------------- S_lo ----------------
+    const int t = tid - 64;   // 0 .. 63
+    for (int u = 0; u < units; ++u) {
+      const int s = u % NS;
+      if (!mbar_wait_flag(&bar_full[s], (unsigned)(u / NS) & 1u, ctrl, tmo, &s_abort)) break;
+      const float4* src = reinterpret_cast<const float4*>(sbuf(s));
+      float4* dst = reinterpret_cast<float4*>(lbuf(s));
+#pragma unroll 4
+      for (int e = t; e < C::S_BYTES / 16; e += 64) {
+        const float4 v = src[e];
+        dst[e] = make_float4(tf32_tail(v.x), tf32_tail(v.y), tf32_tail(v.z), tf32_tail(v.w));
+      }
+      fence_async_smem();   // generic writes -> the tensor cores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_lo[s]);
+    }
+  } else {
+    // ---------------- epilogue: thread = row ----------------
+    const int q = warp & 3;   // TMEM lane quarter
+    for (int j = 0; j < my_tiles; ++j) {
+      const int acc = j & 1;
+      if (!mbar_wait_flag(&bar_acc[acc], (unsigned)(j >> 1) & 1u, ctrl, tmo, &s_abort)) break;
+      tc_fence_after();
+      const int tile = (int)blockIdx.x + j * (int)gridDim.x;
+      const int row = tile * C::BM + 32 * q + lane;
+      float* yr = Y + (size_t)row * DP;
+      const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * DP);
+#pragma unroll 1
+      for (int c = 0; c < DP; c += 16) {
+        float v[16];
+        tmem_ld16(base + (uint32_t)c, v);
+        if (row < rows) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(yr + c + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_accfree[acc]);
+    }
+  }
+
+  // every issued copy and product completes before the CTA releases TMEM and exits
+  if (warp == 0 && lane == 0) {
+    const int n = s_loaded;
+    for (int u = max(0, n - NS); u < n; ++u)
+      if (!mbar_drain(&bar_full[u % NS], (unsigned)(u / NS) & 1u, tmo)) atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+  }
+  if (warp == 1 && lane == 0) {
+    const int n = s_issued;
+    for (int u = max(0, n - NS); u < n; ++u)
+      if (!mbar_drain(&bar_empty[u % NS], (unsigned)(u / NS) & 1u, tmo)) atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::TCOLS)
+                 : "memory");
+}
+
+}  // namespace pn

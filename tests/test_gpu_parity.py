@@ -325,3 +325,20 @@ def test_newton_tensor_core_and_fp32_compositions(tc, cell, D, T, B):
     prob = pi.random_problem(600 + D + T + cell, cell, D, d_in, T=T, B=B, rho=0.7, eps=0.05, s0_scale=0.3,
                              tol=1e-5)
     _check_against_oracle(prob, pi.MODE_NEWTON, tc=tc)
+
+
+@pytest.mark.parametrize("tc", [1, 0])
+@pytest.mark.parametrize("cell", [pi.CELL_TANH_RNN, pi.CELL_EULER])
+@pytest.mark.parametrize("mode", DIAG_MODES)
+@pytest.mark.parametrize("D,T,B", [(128, 300, 3), (256, 333, 3), (256, 64, 1)])
+def test_wide_tensor_core_product(tc, cell, mode, D, T, B):
+    """D = 128 and 256 (one-gate cells): each iteration first forms W s^(i)_r for every step on the
+    tensor cores (3xTF32, 128-row tiles, the last one partial), then the diagonal kernel reads it; with
+    tc = 0 the FP32 kernels form the product themselves.  Both must match the oracle."""
+    if mode == pi.MODE_PICARD and cell != pi.CELL_EULER:
+        T = 12
+    prob = pi.random_problem(700 + D + T + cell, cell, D, D, T=T, B=B, rho=0.6, eps=0.05, s0_scale=0.2,
+                             tol=1e-5)
+    if mode == pi.MODE_JACOBI:
+        prob.max_iters = T
+    _check_against_oracle(prob, mode, tc=tc)
