@@ -77,6 +77,13 @@ struct pn_ctx {
   float* ypre = nullptr;           // [B*T][D]
   CUtensorMap* wmaps = nullptr;    // [0]/[1] S of iterate buffer 0 / 1, [2] W_hi, [3] W_lo
   CUtensorMap* wmaps_h = nullptr;
+  // the input projection on the tensor cores (N = R*D a multiple of 16 up to 256, d_in % 4 == 0)
+  const void* proj_gemm = nullptr;
+  size_t proj_gemm_smem = 0;
+  float* proj_hi = nullptr;        // TF32 split of U (or W_ih), row-major [R*D][d_in]
+  float* proj_lo = nullptr;
+  CUtensorMap* pmaps = nullptr;    // [0], [1] x, [2] U_hi, [3] U_lo
+  CUtensorMap* pmaps_h = nullptr;
   // host pinned mirrors
   Args* args_h = nullptr;
   Ctrl* ctrl_h = nullptr;
@@ -184,7 +191,11 @@ void free_all(pn_ctx* h) {
     if (*p) cudaFree(*p);
     *p = nullptr;
   }
-  for (float** p : {&h->wt_hi, &h->wt_lo, &h->ypre}) {
+  if (h->pmaps) cudaFree(h->pmaps);
+  if (h->pmaps_h) cudaFreeHost(h->pmaps_h);
+  h->pmaps = nullptr;
+  h->pmaps_h = nullptr;
+  for (float** p : {&h->wt_hi, &h->wt_lo, &h->ypre, &h->proj_hi, &h->proj_lo}) {
     if (*p) cudaFree(*p);
     *p = nullptr;
   }
@@ -337,6 +348,26 @@ bool encode_tc_maps(const pn_ctx* h, int mode, CUtensorMap* out) {
 }
 
 // Kernels that run before the loop: projection (tanh RNN, GRU) and init.
+// The tensor-core GEMM for N output columns (the input projection's N = R*D).
+template <int N>
+void gemm_fn_of(const void** fn, size_t* smem) {
+  *fn = (const void*)&wide_gemm_kernel<N>;
+  *smem = (size_t)WideGemmCfg<N>::SMEM_BYTES;
+}
+bool gemm_for_width(int N, const void** fn, size_t* smem) {
+  switch (N) {
+    case 16: gemm_fn_of<16>(fn, smem); return true;
+    case 32: gemm_fn_of<32>(fn, smem); return true;
+    case 48: gemm_fn_of<48>(fn, smem); return true;
+    case 64: gemm_fn_of<64>(fn, smem); return true;
+    case 96: gemm_fn_of<96>(fn, smem); return true;
+    case 128: gemm_fn_of<128>(fn, smem); return true;
+    case 192: gemm_fn_of<192>(fn, smem); return true;
+    case 256: gemm_fn_of<256>(fn, smem); return true;
+    default: return false;
+  }
+}
+
 struct PreLaunch {
   bool has_proj = false;
   dim3 proj_grid;
@@ -361,31 +392,68 @@ PreLaunch pre_launch(const pn_ctx* h) {
   return p;
 }
 
-// Launch shape and arguments of the wide product (wide_gemm_kernel) of `mode`.
-struct PreArgs {
-  const CUtensorMap* maps;
-  float* y;
-  int rows;
-  Ctrl* ctrl;
-  const Args* args;
-  void* kargs[5];
-  unsigned grid;
+// One launch of the tensor-core GEMM (wide_gemm_kernel<N>): the wide product Y = S W^T of an
+// iteration, or the input projection u = x U^T + b.
+struct GemmLaunch {
+  const void* fn = nullptr;
+  unsigned grid = 1;
+  int nt = 256;
+  size_t smem = 0;
+  const CUtensorMap* maps = nullptr;
+  float* y = nullptr;
+  int rows = 0;
+  int K = 0;
+  const float* bias = nullptr;
+  Ctrl* ctrl = nullptr;
+  const Args* args = nullptr;
+  void* kargs[7];
+  void bind() {
+    kargs[0] = (void*)&maps;
+    kargs[1] = (void*)&y;
+    kargs[2] = (void*)&rows;
+    kargs[3] = (void*)&K;
+    kargs[4] = (void*)&bias;
+    kargs[5] = (void*)&ctrl;
+    kargs[6] = (void*)&args;
+  }
 };
-void pre_args(pn_ctx* h, PreArgs& a) {
-  a.maps = h->wmaps;
-  a.y = h->ypre;
-  a.rows = h->B * h->T;
-  a.ctrl = h->ctrl;
-  a.args = h->args;
-  a.kargs[0] = (void*)&a.maps;
-  a.kargs[1] = (void*)&a.y;
-  a.kargs[2] = (void*)&a.rows;
-  a.kargs[3] = (void*)&a.ctrl;
-  a.kargs[4] = (void*)&a.args;
+
+unsigned gemm_grid(const pn_ctx* h, int rows) {
   int nsm = 148;
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, h->device);
-  const int tiles = (a.rows + 127) / 128;
-  a.grid = (unsigned)std::max(1, std::min(nsm, tiles));
+  return (unsigned)std::max(1, std::min(nsm, (rows + 127) / 128));
+}
+
+// the wide product of `mode`'s iteration (ki.pre_fn)
+void wide_launch(pn_ctx* h, const KInfo& ki, GemmLaunch& g) {
+  g.fn = ki.pre_fn;
+  g.nt = ki.pre_nt;
+  g.smem = ki.pre_smem;
+  g.maps = h->wmaps;
+  g.y = h->ypre;
+  g.rows = h->B * h->T;
+  g.K = h->D;
+  g.bias = nullptr;
+  g.ctrl = h->ctrl;
+  g.args = h->args;
+  g.grid = gemm_grid(h, g.rows);
+  g.bind();
+}
+
+// the input projection on the tensor cores (h->proj_gemm set at create)
+void proj_launch(pn_ctx* h, GemmLaunch& g) {
+  g.fn = h->proj_gemm;
+  g.nt = 256;
+  g.smem = h->proj_gemm_smem;
+  g.maps = h->pmaps;
+  g.y = h->xin;
+  g.rows = h->B * h->T;
+  g.K = h->d_in;
+  g.bias = h->proj_b;
+  g.ctrl = h->ctrl;
+  g.args = h->args;
+  g.grid = gemm_grid(h, g.rows);
+  g.bind();
 }
 
 pn_status build_graph(pn_ctx* h, int mode) {
@@ -407,9 +475,10 @@ pn_status build_graph(pn_ctx* h, int mode) {
     return cudaGraphAddKernelNode(out, graph, dep, dep ? 1 : 0, &kp);
   };
   cudaError_t e = cudaSuccess;
-  // 1. input projection
+  // 1. input projection (FP32 kernel; the tensor-core one runs after init, below)
   const Args* a_d = h->args;
-  if (pl.has_proj) {
+  GemmLaunch pg;
+  if (pl.has_proj && !(h->proj_gemm && h->tc_opt)) {
     const float* w = h->proj_w;
     const float* bb = h->proj_b;
     float* o = h->xin;
@@ -426,6 +495,13 @@ pn_status build_graph(pn_ctx* h, int mode) {
     void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&D, (void*)&T, (void*)&B};
     e = add_kernel(g, (const void*)&init_kernel, pl.init_grid, dim3(256), 0, kargs,
                    prev ? &prev : nullptr, &node);
+    if (e != cudaSuccess) goto fail_graph;
+    prev = node;
+  }
+  if (pl.has_proj && h->proj_gemm && h->tc_opt) {
+    // 2b. input projection on the tensor cores (after init, which resets the error word it polls)
+    proj_launch(h, pg);
+    e = add_kernel(g, pg.fn, dim3(pg.grid), dim3(pg.nt), pg.smem, pg.kargs, &prev, &node);
     if (e != cudaSuccess) goto fail_graph;
     prev = node;
   }
@@ -446,11 +522,11 @@ pn_status build_graph(pn_ctx* h, int mode) {
     P.cond = cond;
     void* kargs[] = {(void*)&P};
     cudaGraphNode_t knode, pnode;
-    PreArgs pa;
+    GemmLaunch wl;
     cudaGraphNode_t* dep = nullptr;
     if (ki.pre_fn) {
-      pre_args(h, pa);
-      e = add_kernel(body, ki.pre_fn, dim3(pa.grid), dim3(ki.pre_nt), ki.pre_smem, pa.kargs, nullptr, &pnode);
+      wide_launch(h, ki, wl);
+      e = add_kernel(body, wl.fn, dim3(wl.grid), dim3(wl.nt), wl.smem, wl.kargs, nullptr, &pnode);
       if (e != cudaSuccess) goto fail_graph;
       dep = &pnode;
     }
@@ -496,9 +572,9 @@ pn_status launch_iter(pn_ctx* h, int mode, int persist = 0) {
   void* kargs[] = {(void*)&P};
   const unsigned grid = (unsigned)h->fam.grid[mode];
   if (ki.pre_fn) {   // the tensor-core product the iteration kernel reads
-    PreArgs pa;
-    pre_args(h, pa);
-    PN_CUDA(h, cudaLaunchKernel(ki.pre_fn, dim3(pa.grid), dim3(ki.pre_nt), pa.kargs, ki.pre_smem, h->stream));
+    GemmLaunch wl;
+    wide_launch(h, ki, wl);
+    PN_CUDA(h, cudaLaunchKernel(wl.fn, dim3(wl.grid), dim3(wl.nt), wl.kargs, wl.smem, h->stream));
   }
   if (!ki.loops) {
     PN_CUDA(h, cudaLaunchKernel(ki.fn, dim3(grid), dim3(ki.nt), kargs, ki.smem, h->stream));
@@ -523,7 +599,7 @@ pn_status launch_iter(pn_ctx* h, int mode, int persist = 0) {
 pn_status launch_pre(pn_ctx* h) {
   const PreLaunch pl = pre_launch(h);
   const Args* a_d = h->args;
-  if (pl.has_proj) {
+  if (pl.has_proj && !(h->proj_gemm && h->tc_opt)) {
     const float* w = h->proj_w;
     const float* bb = h->proj_b;
     float* o = h->xin;
@@ -535,6 +611,11 @@ pn_status launch_pre(pn_ctx* h) {
   int D = h->D, T = h->T, B = h->B;
   void* kargs[] = {(void*)&a_d, (void*)&c, (void*)&D, (void*)&T, (void*)&B};
   PN_CUDA(h, cudaLaunchKernel((const void*)&init_kernel, pl.init_grid, dim3(256), kargs, 0, h->stream));
+  if (pl.has_proj && h->proj_gemm && h->tc_opt) {
+    GemmLaunch pg;
+    proj_launch(h, pg);
+    PN_CUDA(h, cudaLaunchKernel(pg.fn, dim3(pg.grid), dim3(pg.nt), pg.kargs, pg.smem, h->stream));
+  }
   return PN_OK;
 }
 
@@ -603,6 +684,16 @@ pn_status prepare_lookback(pn_ctx* h, int mode) {
 // The copy is ordered before the launches on the same stream; the pinned
 // mirror is not touched again before the call's final synchronisation.
 pn_status upload_tc_maps(pn_ctx* h, int mode) {
+  if (h->proj_gemm && h->tc_opt && h->cell != PN_CELL_EULER_TANH) {   // x changes from call to call
+    const long long rows = (long long)h->B * h->T;
+    const int N = cell_R(h->cell) * h->D;
+    if (!encode_2d_sw128(&h->pmaps_h[0], h->args_h->x, h->d_in, rows, 32, 128) ||
+        !encode_2d_sw128(&h->pmaps_h[2], h->proj_hi, h->d_in, N, 32, N) ||
+        !encode_2d_sw128(&h->pmaps_h[3], h->proj_lo, h->d_in, N, 32, N))
+      return fail(h, PN_ERR_CUDA, "encoding the input projection's tensor maps failed");
+    h->pmaps_h[1] = h->pmaps_h[0];
+    PN_CUDA(h, cudaMemcpyAsync(h->pmaps, h->pmaps_h, 4 * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
+  }
   if (h->fam.k[mode].pre_fn) {
     if (!encode_wide_maps(h, h->wmaps_h))
       return fail(h, PN_ERR_CUDA, "encoding the wide product's tensor maps failed (D=%d, T=%d, B=%d)", h->D, h->T, h->B);
@@ -975,6 +1066,32 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
       PN_TRY(dalloc(h, &h->proj_w, pw.size()));
       PN_TRY(dalloc(h, &h->proj_b, pb.size()));
       PN_TRY(dalloc(h, &h->xin, BT * R * D));
+      // the projection on the tensor cores where its shape allows: N = R*D a multiple of 16 up to
+      // 256 and rows of x 16-byte aligned (d_in % 4 == 0)
+      const void* gfn = nullptr;
+      size_t gsmem = 0;
+      if ((d_in % 4) == 0 && gemm_for_width(R * D, &gfn, &gsmem) &&
+          cudaFuncSetAttribute(gfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem) == cudaSuccess) {
+        const int N = R * D;
+        std::vector<float> phi((size_t)N * d_in), plo((size_t)N * d_in);
+        for (size_t e = 0; e < phi.size(); ++e) {
+          phi[e] = tf32_round(pw[e]);
+          plo[e] = tf32_round(pw[e] - phi[e]);
+        }
+        PN_TRY(dalloc(h, &h->proj_hi, phi.size()));
+        PN_TRY(dalloc(h, &h->proj_lo, plo.size()));
+        if (cudaMemcpy(h->proj_hi, phi.data(), phi.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+            cudaMemcpy(h->proj_lo, plo.data(), plo.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+            cudaMalloc((void**)&h->pmaps, 4 * sizeof(CUtensorMap)) != cudaSuccess ||
+            cudaMallocHost((void**)&h->pmaps_h, 4 * sizeof(CUtensorMap)) != cudaSuccess) {
+          st = fail(h, PN_ERR_NOMEM, "allocating the projection's tensor-core operands failed");
+          goto bad;
+        }
+        h->proj_gemm = gfn;
+        h->proj_gemm_smem = gsmem;
+      } else {
+        cudaGetLastError();
+      }
       if (cudaMemcpy(h->proj_w, pw.data(), pw.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
           cudaMemcpy(h->proj_b, pb.data(), pb.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess) {
         st = fail(h, PN_ERR_CUDA, "weight upload failed");

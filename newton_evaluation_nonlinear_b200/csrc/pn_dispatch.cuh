@@ -142,7 +142,7 @@ inline KInfo dense_pick() {
 template <int CELL, int MODE, int DP>
 inline KInfo diag_wide_kinfo() {
   using C = DiagCfg<CELL, MODE, DP, 64, 4, 4, 16, true>;
-  using W = WideGemmCfg<DP>;
+  using W = WideGemmCfg<DP>;   // N = K = DP
   KInfo k{(const void*)&diag_iter_kernel<CELL, MODE, DP, 64, 4, 4, 16, true>, C::NT, C::L, 64, C::SMEM_BYTES,
           kKindDiag};
   k.pre_fn = (const void*)&wide_gemm_kernel<DP>;

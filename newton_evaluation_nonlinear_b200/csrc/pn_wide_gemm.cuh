@@ -1,6 +1,7 @@
-// pn_wide_gemm.cuh -- the cell's recurrent product for wide states (D = 128,
-// 256) on the tensor cores: Y = S W^T over all B*T steps of an iterate, as
-// 3xTF32 tcgen05.mma with W streamed from L2 in 32-column K chunks.
+// pn_wide_gemm.cuh -- a 3xTF32 tcgen05 GEMM Y = X W^T (+ bias) over all B*T
+// rows, with W streamed from L2 in 32-column K chunks.  It forms the cell's
+// recurrent product for wide states (D = 128, 256: X = the iterate, W = the
+// recurrent weights) and the hoisted input projection (X = x, W = U or W_ih).
 //
 // At D = 256 one step's W s costs 2 D^2 = 131 kflop, so an iteration of the
 // Euler workload (B = 32, T = 1024) is 4.3 GFLOP: about 60 us of the FP32 FMA
@@ -31,20 +32,21 @@
 
 namespace pn {
 
-template <int DP>
+// N output columns (the rows of W), a multiple of 16 up to 256.
+template <int N>
 struct WideGemmCfg {
-  static_assert(DP == 128 || DP == 256, "wide states: D = 128 or 256");
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "N: a multiple of 16, at most 256");
   static constexpr int BM = 128;                  // rows per tile
   static constexpr int KC = 32;                   // K chunk: one 128-byte swizzle row of fp32
-  static constexpr int NKC = DP / KC;             // chunks per tile
   static constexpr int S_BYTES = BM * KC * 4;     // 16 KB
-  static constexpr int W_BYTES = DP * KC * 4;     // 16 or 32 KB
+  static constexpr int W_BYTES = N * KC * 4;
   static constexpr int STAGE = 2 * S_BYTES + 2 * W_BYTES;   // S, S_lo, W_hi, W_lo
-  static constexpr int NSTAGE = (DP == 128) ? 3 : 2;
-  static constexpr int TCOLS = 2 * DP;            // two accumulators
+  static constexpr int NSTAGE = (200 * 1024) / STAGE < 4 ? (200 * 1024) / STAGE : 4;
+  static constexpr int TCOLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
   static constexpr int NT = 256;                  // 8 warps
   static constexpr int SMEM_BYTES = NSTAGE * STAGE + 1024;   // + slack to align the ring to 1024 bytes
-  static_assert(TCOLS <= 512, "TMEM columns");
+  static_assert(NSTAGE >= 2, "two stages at least");
+  static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -57,13 +59,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// maps: [0] S of iterate buffer 0, [1] S of buffer 1, [2] W_hi, [3] W_lo.
-template <int DP>
+// Y[r][n] = sum_k X[r][k] W[n][k] (+ bias[n]) for r < rows, n < N, k < K.  maps: [0] X of iterate
+// buffer 0 and [1] of buffer 1 (the iteration's parity picks one; the input projection passes the
+// same map twice), [2] W_hi, [3] W_lo.  K need not be a multiple of 32 (the loads zero-fill).
+template <int N>
 __global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __restrict__ maps, float* __restrict__ Y,
-                                                           int rows, Ctrl* ctrl, const Args* __restrict__ args) {
-  using C = WideGemmCfg<DP>;
+                                                           int rows, int K, const float* __restrict__ bias, Ctrl* ctrl,
+                                                           const Args* __restrict__ args) {
+  using C = WideGemmCfg<N>;
+  constexpr int DP = N;
   constexpr int NS = C::NSTAGE;
-  constexpr int NKC = C::NKC;
+  const int NKC = (K + C::KC - 1) / C::KC;
   extern __shared__ __align__(1024) unsigned char smem_wg[];
   unsigned char* ring = smem_wg + ((1024u - (smem_addr(smem_wg) & 1023u)) & 1023u);
   __shared__ __align__(8) uint64_t bar_full[NS], bar_lo[NS], bar_empty[NS], bar_acc[2], bar_accfree[2];
@@ -197,6 +203,10 @@ __global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __
       for (int c = 0; c < DP; c += 16) {
         float v[16];
         tmem_ld16(base + (uint32_t)c, v);
+        if (bias) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] += __ldg(bias + c + e);
+        }
         if (row < rows) {
 #pragma unroll
           for (int e = 0; e < 16; e += 4)
