@@ -234,9 +234,13 @@ PN_API pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
  * a more exact Jacobian approximation).  With stall >= 0, later evaluations
  * move one rung up the ladder jacobi/picard -> quasi -> newton (newton only
  * where this handle supports it) whenever r^(i) > stall * r^(i-1), i >= 1,
- * before update i is applied; the loop then runs from the host, one launch
- * per iteration (plus one more launch per switch).  stall < 0 switches it
- * off (default).  A NaN or infinite stall is PN_ERR_INVALID. */
+ * before update i is applied: iteration i runs again in the stronger mode.
+ * With the device loop (PN_OPT_DEVICE_LOOP = 1, the default) the rule runs
+ * on the device: a CUDA graph holds one conditional IF node per mode inside
+ * its WHILE node, and the last CTA of each iteration turns on the node of the
+ * mode the next iteration runs in.  With PN_OPT_DEVICE_LOOP = 0 the host
+ * applies it, one launch per iteration.  stall < 0 switches it off
+ * (default).  A NaN or infinite stall is PN_ERR_INVALID. */
 PN_API pn_status pn_set_adaptive(pn_handle h, float stall);
 
 /* The mode of each update of the handle's last evaluation (out[i] for update

@@ -69,7 +69,7 @@ struct pn_ctx {
   Ctrl* ctrl = nullptr;
   Args* args = nullptr;
   float* hist = nullptr;
-  CUtensorMap* tmaps = nullptr;   // TMA descriptors of the tensor-core kernels (kTcMaps, see IterParams)
+  CUtensorMap* tmaps = nullptr;   // TMA descriptors of the tensor-core kernels: kTcMaps per mode (see IterParams)
   // wide one-gate cells (D = 128, 256): the tensor-core product Y = S W^T before each iteration
   bool wide_capable = false;
   float* wt_hi = nullptr;          // TF32 split of W, row-major [D][D]
@@ -98,9 +98,13 @@ struct pn_ctx {
   float* pst[2] = {nullptr, nullptr};
   cudaStream_t s_in = nullptr, s_out = nullptr;
   cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_done[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
-  // graphs, one per mode, built on first use
+  // graphs, one per mode, built on first use; the adaptive ones (one per starting mode) hold an
+  // IF node per mode inside the WHILE node
   cudaGraph_t graph[4] = {nullptr, nullptr, nullptr, nullptr};
   cudaGraphExec_t exec[4] = {nullptr, nullptr, nullptr, nullptr};
+  cudaGraph_t graph_ad[4] = {nullptr, nullptr, nullptr, nullptr};
+  cudaGraphExec_t exec_ad[4] = {nullptr, nullptr, nullptr, nullptr};
+  int* mode_hist_d = nullptr;  // [kHistCap] modes of the kept updates (adaptive graph)
   // options
   long long timeout_ns = 1000000000LL;
   int stall_ticket = -1;
@@ -167,13 +171,23 @@ pn_status dalloc(pn_ctx* h, T** p, size_t count) {
   return PN_OK;
 }
 
-void free_all(pn_ctx* h) {
+void destroy_graphs(pn_ctx* h) {
   for (int m = 0; m < 4; ++m) {
     if (h->exec[m]) cudaGraphExecDestroy(h->exec[m]);
     if (h->graph[m]) cudaGraphDestroy(h->graph[m]);
+    if (h->exec_ad[m]) cudaGraphExecDestroy(h->exec_ad[m]);
+    if (h->graph_ad[m]) cudaGraphDestroy(h->graph_ad[m]);
     h->exec[m] = nullptr;
     h->graph[m] = nullptr;
+    h->exec_ad[m] = nullptr;
+    h->graph_ad[m] = nullptr;
   }
+}
+
+void free_all(pn_ctx* h) {
+  destroy_graphs(h);
+  if (h->mode_hist_d) cudaFree(h->mode_hist_d);
+  h->mode_hist_d = nullptr;
   float** fbufs[] = {&h->wt_diag, &h->wt_dense, &h->wt_tc, &h->wt_tct, &h->wdiag, &h->bhn,    &h->proj_w,
                      &h->proj_b,  &h->xin,      &h->buf1,  &h->agg,    &h->pref,  &h->hist, &h->hx,
                      &h->hs0,     &h->hst,      &h->px[0], &h->px[1],  &h->ps0[0], &h->ps0[1], &h->pst[0],
@@ -234,6 +248,7 @@ IterParams make_params(const pn_ctx* h, int mode) {
                : (kind == kKindDiagTc ? h->wt_tc : (kind == kKindDiagTct ? h->wt_tct : h->wt_diag));
   P.wt_tc = h->wt_tc;
   P.ypre = h->ypre;
+  P.mode_hist = h->mode_hist_d;
   P.wdiag = h->wdiag;
   P.bhn = h->bhn;
   P.xin = h->xin;
@@ -244,7 +259,7 @@ IterParams make_params(const pn_ctx* h, int mode) {
   P.ctrl = h->ctrl;
   P.args = h->args;
   P.hist = h->hist;
-  P.tmaps = h->tmaps;
+  P.tmaps = h->tmaps ? h->tmaps + (size_t)mode * kTcMaps : nullptr;   // each mode's kernel has its own maps
   P.eps = h->eps;
   P.D = h->D;
   P.d_in = h->d_in;
@@ -456,8 +471,8 @@ void proj_launch(pn_ctx* h, GemmLaunch& g) {
   g.bind();
 }
 
-pn_status build_graph(pn_ctx* h, int mode) {
-  if (h->exec[mode]) return PN_OK;
+pn_status build_graph(pn_ctx* h, int mode, bool adaptive = false) {
+  if ((adaptive ? h->exec_ad[mode] : h->exec[mode])) return PN_OK;
   const KInfo& ki = h->fam.k[mode];
   const PreLaunch pl = pre_launch(h);
   cudaGraph_t g = nullptr;
@@ -518,21 +533,54 @@ pn_status build_graph(pn_ctx* h, int mode) {
     e = cudaGraphAddNode(&node, g, &prev, 1, &cp);
     if (e != cudaSuccess) goto fail_graph;
     cudaGraph_t body = cp.conditional.phGraph_out[0];
-    IterParams P = make_params(h, mode);
-    P.cond = cond;
-    void* kargs[] = {(void*)&P};
-    cudaGraphNode_t knode, pnode;
-    GemmLaunch wl;
-    cudaGraphNode_t* dep = nullptr;
-    if (ki.pre_fn) {
-      wide_launch(h, ki, wl);
-      e = add_kernel(body, wl.fn, dim3(wl.grid), dim3(wl.nt), wl.smem, wl.kargs, nullptr, &pnode);
+    // one iteration of mode m (its tensor-core product first, where it has one) into graph `gr`
+    auto add_iteration = [&](cudaGraph_t gr, int m, const cudaGraphConditionalHandle* mc) -> cudaError_t {
+      const KInfo& km = h->fam.k[m];
+      IterParams P = make_params(h, m);
+      P.cond = cond;
+      if (mc)
+        for (int q = 0; q < 4; ++q) P.mode_cond[q] = mc[q];
+      void* kargs[] = {(void*)&P};
+      cudaGraphNode_t knode, pnode;
+      GemmLaunch wl;
+      cudaGraphNode_t* dep = nullptr;
+      cudaError_t err = cudaSuccess;
+      if (km.pre_fn) {
+        wide_launch(h, km, wl);
+        err = add_kernel(gr, wl.fn, dim3(wl.grid), dim3(wl.nt), wl.smem, wl.kargs, nullptr, &pnode);
+        if (err != cudaSuccess) return err;
+        dep = &pnode;
+      }
+      return add_kernel(gr, km.fn, dim3((unsigned)h->fam.grid[m]), dim3(km.nt), km.smem, kargs, dep, &knode);
+    };
+    if (!adaptive) {
+      e = add_iteration(body, mode, nullptr);
       if (e != cudaSuccess) goto fail_graph;
-      dep = &pnode;
+    } else {
+      // adaptive switching on the device: an IF node per mode, in the ladder's order, inside the
+      // WHILE node; the starting mode's is on at every launch, and the last CTA of an iteration
+      // turns on the one of the mode the next iteration runs in (a stronger mode is reached in the
+      // same pass of the body, since its IF node comes later)
+      cudaGraphConditionalHandle mc[4];
+      for (int m = 0; m < 4 && e == cudaSuccess; ++m)
+        e = cudaGraphConditionalHandleCreate(&mc[m], g, m == mode ? 1u : 0u, cudaGraphCondAssignDefault);
+      if (e != cudaSuccess) goto fail_graph;
+      cudaGraphNode_t bprev = nullptr;
+      for (int m = 0; m < 4; ++m) {
+        if (!h->fam.k[m].fn) continue;
+        cudaGraphNodeParams ip{};
+        ip.type = cudaGraphNodeTypeConditional;
+        ip.conditional.handle = mc[m];
+        ip.conditional.type = cudaGraphCondTypeIf;
+        ip.conditional.size = 1;
+        cudaGraphNode_t inode;
+        e = cudaGraphAddNode(&inode, body, bprev ? &bprev : nullptr, bprev ? 1 : 0, &ip);
+        if (e != cudaSuccess) goto fail_graph;
+        e = add_iteration(ip.conditional.phGraph_out[0], m, mc);
+        if (e != cudaSuccess) goto fail_graph;
+        bprev = inode;
+      }
     }
-    e = add_kernel(body, ki.fn, dim3((unsigned)h->fam.grid[mode]), dim3(ki.nt), ki.smem, kargs,
-                   dep, &knode);
-    if (e != cudaSuccess) goto fail_graph;
     prev = node;
   }
   {
@@ -547,13 +595,13 @@ pn_status build_graph(pn_ctx* h, int mode) {
       prev = node;
     }
   }
-  e = cudaGraphInstantiate(&h->exec[mode], g, 0);
+  e = cudaGraphInstantiate(adaptive ? &h->exec_ad[mode] : &h->exec[mode], g, 0);
   if (e != cudaSuccess) goto fail_graph;
-  h->graph[mode] = g;
+  (adaptive ? h->graph_ad : h->graph)[mode] = g;
   return PN_OK;
 fail_graph:
   cudaGraphDestroy(g);
-  h->exec[mode] = nullptr;
+  (adaptive ? h->exec_ad : h->exec)[mode] = nullptr;
   return fail(h, PN_ERR_CUDA, "building the CUDA graph for mode %d failed: %s", mode, cudaGetErrorString(e));
 }
 
@@ -701,9 +749,10 @@ pn_status upload_tc_maps(pn_ctx* h, int mode) {
     return PN_OK;
   }
   if (!tagged_lookback(h->fam.k[mode].kind)) return PN_OK;
-  if (!encode_tc_maps(h, mode, h->tmaps_h))
+  if (!encode_tc_maps(h, mode, h->tmaps_h + (size_t)mode * kTcMaps))
     return fail(h, PN_ERR_CUDA, "encoding the TMA tensor maps failed (D=%d, T=%d, B=%d)", h->D, h->T, h->B);
-  PN_CUDA(h, cudaMemcpyAsync(h->tmaps, h->tmaps_h, kTcMaps * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
+  PN_CUDA(h, cudaMemcpyAsync(h->tmaps + (size_t)mode * kTcMaps, h->tmaps_h + (size_t)mode * kTcMaps,
+                             kTcMaps * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
   return PN_OK;
 }
 
@@ -760,15 +809,32 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   pn_status st = prepare_lookback(h, mode);
   if (st != PN_OK) return st;
   const bool adaptive = h->adapt_stall >= 0.0f;
-  h->args_h->use_cond = (h->device_loop && !adaptive) ? 1 : 0;
+  const bool device_adaptive = adaptive && h->device_loop;   // the switching rule runs on the device
+  h->args_h->use_cond = h->device_loop ? 1 : 0;
   h->args_h->newton_band = h->newton_band;
   h->args_h->damping = h->damping;
   h->args_h->store_fmt = h->store_fmt;
   h->args_h->store_until = h->store_until;
+  h->args_h->adapt = device_adaptive ? 1 : 0;
+  h->args_h->stall = h->adapt_stall;
+  h->args_h->start_mode = mode;
+  h->args_h->mode_ok = 0;
+  for (int m = 0; m < 4; ++m)
+    if (h->fam.k[m].fn) h->args_h->mode_ok |= 1 << m;
   PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
   if ((st = upload_tc_maps(h, mode)) != PN_OK) return st;
+  if (device_adaptive) {   // the maps of every mode the ladder may reach
+    for (int m = 0; m < 4; ++m)
+      if (m != mode && h->fam.k[m].fn && (st = upload_tc_maps(h, m)) != PN_OK) return st;
+  }
   h->mode_hist.clear();
-  if (adaptive) {
+  if (device_adaptive) {
+    st = build_graph(h, mode, true);
+    if (st != PN_OK) return st;
+    PN_CUDA(h, cudaGraphLaunch(h->exec_ad[mode], h->stream));
+  } else if (adaptive) {
+    h->args_h->use_cond = 0;
+    PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
     if ((st = run_adaptive(h, mode)) != PN_OK) return st;
     if ((st = launch_finish(h)) != PN_OK) return st;
   } else if (h->device_loop && h->fam.k[mode].loops) {
@@ -798,6 +864,14 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   PN_CUDA(h, cudaMemcpyAsync(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, h->stream));
   PN_CUDA(h, cudaStreamSynchronize(h->stream));
   const Ctrl& c = *h->ctrl_h;
+  if (device_adaptive) {
+    // the modes of the kept updates, and the look-back format the last one left behind
+    const int n = std::min(std::max(c.final_iter, 0), kHistCap);
+    h->mode_hist.assign((size_t)n, 0);
+    if (n > 0)
+      PN_CUDA(h, cudaMemcpy(h->mode_hist.data(), h->mode_hist_d, (size_t)n * sizeof(int), cudaMemcpyDeviceToHost));
+    if (c.cur_mode >= 0 && c.cur_mode < 4 && h->fam.k[c.cur_mode].fn) h->last_kind = h->fam.k[c.cur_mode].kind;
+  }
   h->last_iters = c.final_iter;
   h->evals += 1;
   if (iters_out) *iters_out = c.final_iter;
@@ -875,12 +949,7 @@ pn_status select_kernels(pn_ctx* h) {
     h->pref_floats = std::max(h->pref_floats, nt * G * wf);
     h->nflags = std::max(h->nflags, nt);
   }
-  for (int m = 0; m < 4; ++m) {
-    if (h->exec[m]) cudaGraphExecDestroy(h->exec[m]);
-    if (h->graph[m]) cudaGraphDestroy(h->graph[m]);
-    h->exec[m] = nullptr;
-    h->graph[m] = nullptr;
-  }
+  destroy_graphs(h);
   return PN_OK;
 }
 
@@ -1126,6 +1195,7 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
     PN_TRY(dalloc(h, &h->ctrl, 1));
     PN_TRY(dalloc(h, &h->args, 1));
     PN_TRY(dalloc(h, &h->hist, kHistCap));
+    PN_TRY(dalloc(h, &h->mode_hist_d, kHistCap));
     if (cudaMemset(h->flags, 0, h->nflags * sizeof(unsigned)) != cudaSuccess ||
         cudaMemset(h->ctrl, 0, sizeof(Ctrl)) != cudaSuccess ||
         cudaMemset(h->hist, 0, kHistCap * sizeof(float)) != cudaSuccess) {
@@ -1142,8 +1212,8 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
     if (h->tc_capable) {
       // the tensor-core kernels stage their tiles with TMA tensor maps; without
       // an encoder (or if the shape cannot be encoded) they are not used
-      bool ok = cudaMalloc((void**)&h->tmaps, kTcMaps * sizeof(CUtensorMap)) == cudaSuccess &&
-                cudaMallocHost((void**)&h->tmaps_h, kTcMaps * sizeof(CUtensorMap)) == cudaSuccess;
+      bool ok = cudaMalloc((void**)&h->tmaps, 4 * kTcMaps * sizeof(CUtensorMap)) == cudaSuccess &&
+                cudaMallocHost((void**)&h->tmaps_h, 4 * kTcMaps * sizeof(CUtensorMap)) == cudaSuccess;
       if (ok) {
         h->args_h->states = h->buf1;   // probe encode with buffers of the same shapes
         h->args_h->x = (cell == PN_CELL_EULER_TANH) ? h->buf1 : nullptr;

@@ -101,6 +101,8 @@ __global__ void init_kernel(const Args* __restrict__ args, Ctrl* __restrict__ ct
     ctrl->fmt_in = fmt != 0;    // s^(0) and s^(1) are narrow when a narrow format is set
     ctrl->fmt_out = fmt != 0;
     ctrl->final_fmt = 0;
+    ctrl->cur_mode = args->start_mode;
+    ctrl->retried = 0;
   }
 }
 

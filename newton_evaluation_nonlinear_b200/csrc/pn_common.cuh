@@ -38,6 +38,10 @@ struct Ctrl {
   int fmt_in;
   int fmt_out;
   int final_fmt;
+  // adaptive switching on the device: the mode the current iteration runs in, and whether this
+  // iteration is already the re-run of a stalled one
+  int cur_mode;
+  int retried;
   // The words below are hot and each sits in a 128-byte line of its own, so that
   // the ticket atomics do not queue behind the polls of the error word.
   alignas(128) int error;        // sticky device error (PN_ERR_TIMEOUT), 0 if none; polled by waiting warps
@@ -61,6 +65,10 @@ struct Args {
   float damping;       // lambda of s^(i+1) = s^(i) + lambda * delta (1 = undamped)
   int store_fmt;       // iterate storage: 0 float32, 1 bfloat16, 2 float16 (PN_STORE_*)
   float store_until;   // narrow storage while the residual known at an update's start is above this
+  int adapt;           // 1: adaptive switching decided on the device (graph with one IF node per mode)
+  float stall;         // switch when r^(i) > stall * r^(i-1)
+  int mode_ok;         // bit m set when mode m has a kernel (the ladder skips the others)
+  int start_mode;      // the evaluation's first mode
 };
 
 // Fixed per-handle parameters of the fused iteration kernels.
@@ -88,6 +96,8 @@ struct IterParams {
   int persist;          // looping kernels: 1 = run iterations until the stop rule, 0 = one iteration
   int run;              // chunks of L steps per ticket (a run; 1 for the kernels that take single chunks)
   cudaGraphConditionalHandle cond;
+  cudaGraphConditionalHandle mode_cond[4];   // adaptive graph: the IF node of each mode
+  int* mode_hist;       // adaptive: the mode of each kept update [kHistCap]
 };
 
 // ---------------------------------------------------------------------------
@@ -332,13 +342,30 @@ __device__ __forceinline__ void finish_launch(const IterParams& P, const Args& A
   else if (!(r <= 3.402823466e38f)) st = PN_ERR_NONFINITE;
   else if (r <= A.tol) st = PN_OK;
   else if (i >= A.max_iters) st = PN_NOT_CONVERGED;
+  // adaptive switching (page §5.3): a stall, r^(i) > stall * r^(i-1), re-runs iteration i in the
+  // next stronger mode -- the same rule as the host loop, applied here by the last CTA
+  bool rerun = false;
+  if (st == kRunning && A.adapt && A.use_cond && i >= 1 && !c->retried && i - 1 < kHistCap &&
+      r > A.stall * P.hist[i - 1]) {
+    const int mode = c->cur_mode;
+    int next = (mode == PN_JACOBI || mode == PN_PICARD) ? PN_QUASI : PN_NEWTON;
+    if (!((A.mode_ok >> next) & 1)) next = mode;
+    if (next != mode) {
+      c->cur_mode = next;
+      c->retried = 1;
+      rerun = true;
+      for (int m = 0; m < 4; ++m) cudaGraphSetConditional(P.mode_cond[m], m == next ? 1u : 0u);
+    }
+  }
   if (st != kRunning) {
     c->status = st;
     c->final_iter = i;
     c->final_resid = r;
     c->final_fmt = c->fmt_in;
     if (A.use_cond) cudaGraphSetConditional(P.cond, 0u);
-  } else {
+  } else if (!rerun) {
+    if (A.adapt && i < kHistCap) P.mode_hist[i] = c->cur_mode;   // the mode of the kept update i
+    c->retried = 0;
     c->iter = i + 1;
     // s^(i+2) is stored narrow while r^(i), the residual known when update i+1 starts, is above the bar
     c->fmt_in = c->fmt_out;

@@ -133,7 +133,7 @@ def test_band_option_bounds():
 # adaptive switching (§5.3): jacobi/picard -> quasi -> newton on a stall
 # ----------------------------------------------------------------------------
 
-def _check_adaptive(cell, start, stall, D, T, B, seed):
+def _check_adaptive(cell, start, stall, D, T, B, seed, device_loop=1):
     import torch
     import newton_evaluation_nonlinear_b200 as pn
     d_in = D if cell == pi.CELL_EULER else D - 1
@@ -147,6 +147,7 @@ def _check_adaptive(cell, start, stall, D, T, B, seed):
                                                                   stall=theta)
     solver = pn.Solver.from_problem(prob)
     solver.set_adaptive(theta)
+    solver.set_option(pn.PN_OPT_DEVICE_LOOP, device_loop)
     x = torch.from_numpy(prob.x).cuda()
     s0 = torch.from_numpy(prob.s0).cuda()
     states, it, r, st = solver.eval(x, s0, start, T, tol)
@@ -165,20 +166,24 @@ def _check_adaptive(cell, start, stall, D, T, B, seed):
         assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq))
 
 
+@pytest.mark.parametrize("device_loop", [1, 0])
 @pytest.mark.parametrize("cell", CELLS)
 @pytest.mark.parametrize("start", ["jacobi", "picard", "quasi"])
 @pytest.mark.parametrize("stall", [0.5, 0.9])
-def test_adaptive_matches_oracle(cell, start, stall):
-    _check_adaptive(cell, start, stall, 16, 400, 2, 341 + cell)
+def test_adaptive_matches_oracle(cell, start, stall, device_loop):
+    """device_loop = 1: the switching rule runs on the device (an IF node per mode inside the
+    graph's WHILE node, set by the last CTA of each iteration); 0: the host loop applies it."""
+    _check_adaptive(cell, start, stall, 16, 400, 2, 341 + cell, device_loop)
 
 
+@pytest.mark.parametrize("device_loop", [1, 0])
 @pytest.mark.parametrize("cell", [pi.CELL_TANH_RNN, pi.CELL_EULER])
 @pytest.mark.parametrize("start", ["jacobi", "picard", "quasi"])
-def test_adaptive_wide_matches_oracle(cell, start):
+def test_adaptive_wide_matches_oracle(cell, start, device_loop):
     """D = 64: the one-gate cells' quasi-Newton updates run on the channel-major tensor-core kernel
     (one launch per iteration in the adaptive loop), Jacobi and Picard on the row-major one, Newton
     on the dense kernel; the switches and the result must match the oracle's."""
-    _check_adaptive(cell, start, 0.9, 64, 600, 2, 361 + cell)
+    _check_adaptive(cell, start, 0.9, 64, 600, 2, 361 + cell, device_loop)
 
 
 def test_adaptive_off_leaves_no_mode_history():
