@@ -271,9 +271,10 @@ typedef enum { PN_STORE_F32 = 0, PN_STORE_BF16 = 1, PN_STORE_F16 = 2 } pn_store;
  * still computes in float32 from the stored values.  A narrow iterate takes
  * the first half of its float32 buffer, so each narrow iteration reads and
  * writes half the state bytes.  The result is returned as float32 whatever
- * its storage.  Stored narrow throughout (store_until = +inf), the residual
- * stalls at the format's resolution (about 2^-9 of max|s| for bfloat16,
- * 2^-12 for float16), so tol must sit above it or store_until below it.
+ * its storage.  Stored narrow throughout (store_until = 0: every residual
+ * is above it), the residual stalls at the format's resolution (about 2^-9
+ * of max|s| for bfloat16, 2^-12 for float16), so store_until must sit above
+ * that floor and tol may then go below it.
  * PN_STORE_F32 (default) stores float32 throughout.  While a narrow format
  * is set the evaluations run on the FP32-FMA kernels.  An unknown format or
  * a NaN store_until is PN_ERR_INVALID, the handle unchanged. */

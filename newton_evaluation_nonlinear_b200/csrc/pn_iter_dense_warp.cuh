@@ -40,13 +40,16 @@ namespace pn {
 template <int CELL, int DP, int NWARP>
 struct DenseWarpCfg {
   static constexpr int R = CellInfo<CELL>::R;
-  static constexpr int L = 32;                          // steps per tile: one per lane in the cell phase
-  static constexpr int RG = DP / 4;                     // row groups of four rows
+  static constexpr int L = 32;                          // steps per chunk
+  static constexpr int RPL = (DP == 4) ? 4 : 2;         // P rows per lane in the chain
+  static constexpr int RG = DP / RPL;                   // row groups
   static constexpr int CG = (32 / RG < DP) ? 32 / RG : DP;   // column groups
   static constexpr int NA = RG * CG;                    // lanes active in the chain and the matvecs
   static constexpr int CPL = DP / CG;                   // P columns per lane = k-slice per lane
+  static constexpr bool WREG = (R == 1);                // the chain keeps its W rows in registers
+  static constexpr int SPP = 32 / DP;                   // cell phase: steps per pass (lane = channel)
   static constexpr int NCS = R + 1;                     // coefficient vectors per step: c0, c_1 .. c_R
-  static constexpr int SP = DP + 1;                     // row stride of the staged s rows
+  static constexpr int SP = DP + 4;                     // row stride of the staged s rows (16-byte rows)
   static constexpr int UP = R * DP + 1;                 // row stride of the staged step inputs
   static constexpr int a4(int v) { return (v + 3) / 4 * 4; }
   // per-warp shared memory, in floats
@@ -68,11 +71,14 @@ struct DenseWarpCfg {
   static constexpr int SMEM_FLOATS = C_RED + NWARP;
   static constexpr size_t SMEM_BYTES = (size_t)SMEM_FLOATS * sizeof(float);
   static constexpr int NT = 32 * NWARP;
+  // two CTAs per SM where the shared memory allows (the register budget follows)
+  static constexpr int MINB = (2 * (SMEM_BYTES + 1024) <= 228 * 1024) ? 2 : 1;
   static_assert(DP % 4 == 0 && DP <= 32, "DP in {4, 8, 16, 32}");
-  static_assert(NA <= 32 && RG * 4 == DP && CG * CPL == DP, "lane grid");
+  static_assert(NA <= 32 && RG * RPL == DP && CG * CPL == DP, "lane grid");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
+// N consecutive floats from shared memory (16-, 8- or 4-byte loads)
 template <int N>
 __device__ __forceinline__ void lds_n(const float* p, float (&v)[N]) {
   if constexpr (N % 4 == 0) {
@@ -91,13 +97,14 @@ __device__ __forceinline__ void lds_n(const float* p, float (&v)[N]) {
 }
 
 template <int CELL, int DP, int NWARP>
-__global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams P) {
+__global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MINB) dense_warp_kernel(const IterParams P) {
   using C = DenseWarpCfg<CELL, DP, NWARP>;
   constexpr int R = C::R;
   constexpr int L = C::L;
   constexpr int NCS = C::NCS;
   constexpr int CG = C::CG;
   constexpr int CPL = C::CPL;
+  constexpr int RPL = C::RPL;
   constexpr int SP = C::SP;
   constexpr int UP = C::UP;
   constexpr int WR = R * DP;   // row length of the transposed weights
@@ -149,36 +156,49 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
   __syncthreads();
   const float* sWj = banded ? sWb : sWf;
 
-  // chain / matvec lane grid: rows 4 rg .. 4 rg + 3, P columns (= k-slice) cg CPL .. cg CPL + CPL - 1
+  // chain / matvec lane grid: rows r0 .. r0 + RPL - 1, P columns (= k-slice) cg CPL .. cg CPL + CPL - 1
   const bool act = lane < C::NA;
   const int rg = act ? lane / CG : 0;
   const int cg = act ? lane % CG : 0;
-  const int r0 = 4 * rg;
+  const int r0 = RPL * rg;
   const int j0 = cg * CPL;
-  // band-limited k range of the chain's inner product for these four rows
+  // band-limited k range of the chain's inner product for these rows
   const int klo = banded ? max(0, r0 - band) : 0;
-  const int khi = banded ? min(DP - 1, r0 + 3 + band) : DP - 1;
-  const float bhn_l = (CELL == PN_CELL_GRU && lane < D) ? __ldg(P.bhn + lane) : 0.0f;
+  const int khi = banded ? min(DP - 1, r0 + RPL - 1 + band) : DP - 1;
+  // cell phase: lane = channel ci of step group ms (SPP steps per pass)
+  const int ci = lane % DP;
+  const int ms = lane / DP;
+  const float bhn_c = (CELL == PN_CELL_GRU && ci < D) ? __ldg(P.bhn + ci) : 0.0f;
+  // the chain's W rows in registers (one-gate cells, band off): wreg[r][k] = W[r0 + r][k]
+  float wreg[C::WREG ? RPL : 1][C::WREG ? DP : 1];
+  if constexpr (C::WREG) {
+#pragma unroll
+    for (int r = 0; r < RPL; ++r)
+#pragma unroll
+      for (int kk = 0; kk < DP; ++kk) wreg[r][kk] = sWf[kk * WR + r0 + r];
+  }
   unsigned rbits = 0u;
   bool aborted = false;
 
+  // W_q[r0 + r][k] of the Jacobian (band-masked when banded), RPL consecutive rows
+  auto wrows = [&](int kk, int q, float (&w)[RPL]) { lds_n<RPL>(sWj + kk * WR + q * DP + r0, w); };
+
   // y = sum over the k-slice of W_q[r0 + r][k] x[k], reduced over the column-group lanes
-  auto slice_matvec = [&](const float* x, float (&out)[R][4]) {
+  auto slice_matvec = [&](const float* x, float (&out)[R][RPL]) {
     float xs[CPL];
     lds_n<CPL>(x + j0, xs);
 #pragma unroll
     for (int q = 0; q < R; ++q)
 #pragma unroll
-      for (int r = 0; r < 4; ++r) out[q][r] = 0.0f;
+      for (int r = 0; r < RPL; ++r) out[q][r] = 0.0f;
 #pragma unroll
     for (int kk = 0; kk < CPL; ++kk) {
 #pragma unroll
       for (int q = 0; q < R; ++q) {
-        const float4 w = *reinterpret_cast<const float4*>(sWj + (j0 + kk) * WR + q * DP + r0);
-        out[q][0] = fmaf(w.x, xs[kk], out[q][0]);
-        out[q][1] = fmaf(w.y, xs[kk], out[q][1]);
-        out[q][2] = fmaf(w.z, xs[kk], out[q][2]);
-        out[q][3] = fmaf(w.w, xs[kk], out[q][3]);
+        float w[RPL];
+        wrows(j0 + kk, q, w);
+#pragma unroll
+        for (int r = 0; r < RPL; ++r) out[q][r] = fmaf(w[r], xs[kk], out[q][r]);
       }
     }
 #pragma unroll
@@ -186,7 +206,13 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
 #pragma unroll
       for (int q = 0; q < R; ++q)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) out[q][r] += __shfl_xor_sync(0xffffffffu, out[q][r], off);
+        for (int r = 0; r < RPL; ++r) out[q][r] += __shfl_xor_sync(0xffffffffu, out[q][r], off);
+  };
+  // RPL consecutive floats at p + r0 (rows of a per-step vector), and their store
+  auto ld_rows = [&](const float* p, float (&v)[RPL]) { lds_n<RPL>(p + r0, v); };
+  auto st_rows = [&](float* p, const float (&v)[RPL]) {
+    if constexpr (RPL == 4) *reinterpret_cast<float4*>(p + r0) = make_float4(v[0], v[1], v[2], v[3]);
+    else *reinterpret_cast<float2*>(p + r0) = make_float2(v[0], v[1]);
   };
 
   unsigned epoch = epoch0;
@@ -231,101 +257,76 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
       __syncwarp();
     };
 
-    // ---- 2. cell phase, lane = step m: coefficient vectors, b_m (and |F_m| on the first pass) --
+    // ---- 2. cell phase, lane = channel ci of step m = pass SPP + ms: the coefficient vectors, b_m (and
+    //         |F_m| on the first pass); the writes of a pass go to consecutive channels
     auto cell = [&](int t0, bool with_res) {
-      const int m = lane;
-      const bool tok = (t0 + m) < T;
-      float sp[DP];
-#pragma unroll
-      for (int kk = 0; kk < DP; ++kk) sp[kk] = sS[m * SP + kk];
 #pragma unroll 1
-      for (int i0 = 0; i0 < DP; i0 += 4) {
-        float z[R][4], zb[R][4];
+      for (int m = ms; m < L; m += C::SPP) {
+        const bool tok = (t0 + m) < T;
+        const float* sp = sS + m * SP;   // s^(i)_{t-1}: the same row for the lanes of a pass
+        float z[R], zb[R];
 #pragma unroll
-        for (int q = 0; q < R; ++q)
+        for (int q = 0; q < R; ++q) z[q] = zb[q] = 0.0f;
 #pragma unroll
-          for (int r = 0; r < 4; ++r) z[q][r] = 0.0f;
+        for (int kk = 0; kk < DP; kk += 4) {
+          const float4 s4 = *reinterpret_cast<const float4*>(sp + kk);
+          const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
-        for (int kk = 0; kk < DP; ++kk) {
-#pragma unroll
-          for (int q = 0; q < R; ++q) {
-            const float4 w = *reinterpret_cast<const float4*>(sWf + kk * WR + q * DP + i0);
-            z[q][0] = fmaf(w.x, sp[kk], z[q][0]);
-            z[q][1] = fmaf(w.y, sp[kk], z[q][1]);
-            z[q][2] = fmaf(w.z, sp[kk], z[q][2]);
-            z[q][3] = fmaf(w.w, sp[kk], z[q][3]);
-          }
-        }
-        if (banded) {   // the Jacobian's product W_band s for b_t = f - A s
-#pragma unroll
-          for (int q = 0; q < R; ++q)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) zb[q][r] = 0.0f;
-#pragma unroll
-          for (int kk = 0; kk < DP; ++kk) {
+          for (int u = 0; u < 4; ++u) {
 #pragma unroll
             for (int q = 0; q < R; ++q) {
-              const float4 w = *reinterpret_cast<const float4*>(sWb + kk * WR + q * DP + i0);
-              zb[q][0] = fmaf(w.x, sp[kk], zb[q][0]);
-              zb[q][1] = fmaf(w.y, sp[kk], zb[q][1]);
-              zb[q][2] = fmaf(w.z, sp[kk], zb[q][2]);
-              zb[q][3] = fmaf(w.w, sp[kk], zb[q][3]);
+              z[q] = fmaf(sWf[(kk + u) * WR + q * DP + ci], sv[u], z[q]);
+              if (banded) zb[q] = fmaf(sWb[(kk + u) * WR + q * DP + ci], sv[u], zb[q]);
             }
           }
+        }
+        if (!banded) {
+#pragma unroll
+          for (int q = 0; q < R; ++q) zb[q] = z[q];
+        }
+        const float spi = sp[ci];
+        const float sci = sS[(m + 1) * SP + ci];
+        float cf[NCS], bb, res;
+        if constexpr (CELL == PN_CELL_TANH_RNN) {
+          const float y = tanh_pn(z[0] + sU[m * UP + ci]);
+          cf[0] = 0.0f;
+          cf[1] = 1.0f - y * y;
+          bb = y - cf[1] * zb[0];
+          res = sci - y;
+        } else if constexpr (CELL == PN_CELL_EULER_TANH) {
+          const float gg = tanh_pn(z[0] + sU[m * UP + ci]);
+          const float eg = P.eps * gg;
+          cf[0] = 1.0f;
+          cf[1] = P.eps * (1.0f - gg * gg);
+          bb = eg - cf[1] * zb[0];
+          res = (sci - spi) - eg;
         } else {
+          const float rr = sigmoidf_acc(sU[m * UP + ci] + z[0]);
+          const float zz = sigmoidf_acc(sU[m * UP + DP + ci] + z[1]);
+          const float hn = z[2] + bhn_c;
+          const float nn = tanh_pn(sU[m * UP + 2 * DP + ci] + rr * hn);
+          const float y = nn + zz * (spi - nn);
+          const float omz = 1.0f - zz;
+          const float dn = omz * (1.0f - nn * nn);
+          cf[0] = zz;
+          cf[1] = dn * hn * rr * (1.0f - rr);   // gamma: W_hr
+          cf[2] = (spi - nn) * zz * omz;        // alpha: W_hz
+          cf[3] = dn * rr;                      // beta:  W_hn
+          // b_t = y - A s with the banded products of W_hr, W_hz, W_hn
+          bb = y - (zz * spi + cf[1] * zb[0] + cf[2] * zb[1] + cf[3] * zb[2]);
+          res = sci - y;
+        }
+        if (tok && ci < D) {
+          if (with_res) rbits = max(rbits, abs_bits(res));
+        } else {   // identity map
+          cf[0] = 1.0f;
 #pragma unroll
-          for (int q = 0; q < R; ++q)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) zb[q][r] = z[q][r];
+          for (int q = 1; q < NCS; ++q) cf[q] = 0.0f;
+          bb = 0.0f;
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int i = i0 + r;
-          const float spi = sS[m * SP + i];
-          const float sci = sS[(m + 1) * SP + i];
-          float cf[NCS], bb, res;
-          if constexpr (CELL == PN_CELL_TANH_RNN) {
-            const float y = tanh_pn(z[0][r] + sU[m * UP + i]);
-            cf[0] = 0.0f;
-            cf[1] = 1.0f - y * y;
-            bb = y - cf[1] * zb[0][r];
-            res = sci - y;
-          } else if constexpr (CELL == PN_CELL_EULER_TANH) {
-            const float gg = tanh_pn(z[0][r] + sU[m * UP + i]);
-            const float eg = P.eps * gg;
-            cf[0] = 1.0f;
-            cf[1] = P.eps * (1.0f - gg * gg);
-            bb = eg - cf[1] * zb[0][r];
-            res = (sci - spi) - eg;
-          } else {
-            const float bh = __shfl_sync(0xffffffffu, bhn_l, i);
-            const float rr = sigmoidf_acc(sU[m * UP + i] + z[0][r]);
-            const float zz = sigmoidf_acc(sU[m * UP + DP + i] + z[1][r]);
-            const float hn = z[2][r] + bh;
-            const float nn = tanh_pn(sU[m * UP + 2 * DP + i] + rr * hn);
-            const float y = nn + zz * (spi - nn);
-            const float omz = 1.0f - zz;
-            const float dn = omz * (1.0f - nn * nn);
-            cf[0] = zz;
-            cf[1] = dn * hn * rr * (1.0f - rr);   // gamma: W_hr
-            cf[2] = (spi - nn) * zz * omz;        // alpha: W_hz
-            cf[3] = dn * rr;                      // beta:  W_hn
-            // b_t = y - A s with the banded products of W_hr, W_hz, W_hn
-            bb = y - (zz * spi + cf[1] * zb[0][r] + cf[2] * zb[1][r] + cf[3] * zb[2][r]);
-            res = sci - y;
-          }
-          if (tok && i < D) {
-            if (with_res) rbits = max(rbits, abs_bits(res));
-          } else {   // identity map
-            cf[0] = 1.0f;
-#pragma unroll
-            for (int q = 1; q < NCS; ++q) cf[q] = 0.0f;
-            bb = 0.0f;
-          }
-#pragma unroll
-          for (int q = 0; q < NCS; ++q) sC[(m * NCS + q) * DP + i] = cf[q];
-          sB[m * DP + i] = bb;
-        }
+        for (int q = 0; q < NCS; ++q) sC[(m * NCS + q) * DP + ci] = cf[q];
+        sB[m * DP + ci] = bb;
       }
       __syncwarp();
     };
@@ -333,7 +334,7 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
     // ---- 3. chain [P | q] over the run, one chunk at a time --------------------------------
     // gs counts the run's composition steps: step 0 sets [P | q] = [A_0 | b_0], step gs > 0 composes
     // with A_m from buffer (gs - 1) & 1 into buffer gs & 1
-    float pold[4][CPL];
+    float pold[RPL][CPL];
     int gs = 0;
 #pragma unroll 1
     for (int c = c_first; c < c_end; ++c) {
@@ -342,16 +343,16 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
       cell(t0, true);
 #pragma unroll 1
       for (int m = 0; m < L; ++m, ++gs) {
-        float c0[4], cq[R][4], bm[4];
-        lds_n<4>(sC + (m * NCS) * DP + r0, c0);
+        float c0[RPL], cq[R][RPL], bm[RPL];
+        ld_rows(sC + (m * NCS) * DP, c0);
 #pragma unroll
-        for (int q = 0; q < R; ++q) lds_n<4>(sC + (m * NCS + 1 + q) * DP + r0, cq[q]);
-        lds_n<4>(sB + m * DP + r0, bm);
+        for (int q = 0; q < R; ++q) ld_rows(sC + (m * NCS + 1 + q) * DP, cq[q]);
+        ld_rows(sB + m * DP, bm);
         float* Pn = sP + (gs & 1) * DP * DP;
-        float qn[4];
+        float qn[RPL];
         if (gs == 0) {
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
+          for (int r = 0; r < RPL; ++r) {
 #pragma unroll
             for (int cc = 0; cc < CPL; ++cc) {
               const int i = r0 + r, j = j0 + cc;
@@ -365,35 +366,52 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
         } else {
           const float* Pk = sP + ((gs - 1) & 1) * DP * DP;
           const float* Qk = sQ + ((gs - 1) & 1) * DP;
-          float acc[R][4][CPL];
+          float acc[R][RPL][CPL];
 #pragma unroll
           for (int q = 0; q < R; ++q)
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
+            for (int r = 0; r < RPL; ++r)
 #pragma unroll
               for (int cc = 0; cc < CPL; ++cc) acc[q][r][cc] = 0.0f;
-          if (act) {
+          bool done = false;
+          if constexpr (C::WREG) {
+            if (!banded) {
+              // W rows from registers: per k, one load of this lane's P columns and RPL x CPL FMAs
+#pragma unroll
+              for (int kk = 0; kk < DP; ++kk) {
+                float p[CPL];
+                lds_n<CPL>(Pk + kk * DP + j0, p);
+#pragma unroll
+                for (int r = 0; r < RPL; ++r)
+#pragma unroll
+                  for (int cc = 0; cc < CPL; ++cc) acc[0][r][cc] = fmaf(wreg[r][kk], p[cc], acc[0][r][cc]);
+              }
+              done = true;
+            }
+          }
+          if (!done && act) {
+            // W rows from shared memory, over the band's k range only
 #pragma unroll 4
             for (int kk = klo; kk <= khi; ++kk) {
               float p[CPL];
               lds_n<CPL>(Pk + kk * DP + j0, p);
 #pragma unroll
               for (int q = 0; q < R; ++q) {
-                const float4 w = *reinterpret_cast<const float4*>(sWj + kk * WR + q * DP + r0);
-                const float wv[4] = {w.x, w.y, w.z, w.w};
+                float w[RPL];
+                wrows(kk, q, w);
 #pragma unroll
-                for (int r = 0; r < 4; ++r)
+                for (int r = 0; r < RPL; ++r)
 #pragma unroll
-                  for (int cc = 0; cc < CPL; ++cc) acc[q][r][cc] = fmaf(wv[r], p[cc], acc[q][r][cc]);
+                  for (int cc = 0; cc < CPL; ++cc) acc[q][r][cc] = fmaf(w[r], p[cc], acc[q][r][cc]);
               }
             }
           }
-          float qa[R][4];
+          float qa[R][RPL];
           slice_matvec(Qk, qa);
-          float qo[4];
-          lds_n<4>(Qk + r0, qo);
+          float qo[RPL];
+          ld_rows(Qk, qo);
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
+          for (int r = 0; r < RPL; ++r) {
 #pragma unroll
             for (int cc = 0; cc < CPL; ++cc) {
               float v = c0[r] * pold[r][cc];
@@ -409,7 +427,7 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
         }
         if (act) {
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
+          for (int r = 0; r < RPL; ++r) {
             if constexpr (CPL % 4 == 0) {
 #pragma unroll
               for (int cc = 0; cc < CPL; cc += 4)
@@ -421,7 +439,7 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
               Pn[(r0 + r) * DP + j0] = pold[r][0];
             }
           }
-          if (cg == 0) *reinterpret_cast<float4*>(sQ + (gs & 1) * DP + r0) = make_float4(qn[0], qn[1], qn[2], qn[3]);
+          if (cg == 0) st_rows(sQ + (gs & 1) * DP, qn);
         }
         __syncwarp();
       }
@@ -458,15 +476,15 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
     __syncwarp();
     // fold the aggregates at distances n_agg .. 1, farthest first: carry <- P_d carry + q_d.  Each
     // lane's blocks of FB aggregates are loaded together, so a batch costs one L2 round trip.
-    constexpr int FB = (CPL <= 2) ? 4 : 2;
+    constexpr int FB = (CPL <= 4) ? 4 : 2;
     for (int d = n_agg; d >= 1; d -= FB) {
-      float blk[FB][4][CPL], qd[FB][4];
+      float blk[FB][RPL][CPL], qd[FB][RPL];
 #pragma unroll
       for (int u = 0; u < FB; ++u) {
         const bool use = act && (d - u >= 1);
         const float* ag = P.agg + ((size_t)k - (size_t)max(d - u, 1) * stride) * P.agg_stride;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < RPL; ++r) {
 #pragma unroll
           for (int cc = 0; cc < CPL; ++cc) blk[u][r][cc] = use ? __ldcg(ag + (r0 + r) * (DP + 1) + j0 + cc) : 0.0f;
           qd[u][r] = use ? __ldcg(ag + (r0 + r) * (DP + 1) + DP) : 0.0f;
@@ -477,9 +495,9 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
         if (d - u < 1) break;   // uniform across the warp
         float xs[CPL];
         lds_n<CPL>(cur + j0, xs);
-        float part[4];
+        float part[RPL];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < RPL; ++r) {
           float v = 0.0f;
 #pragma unroll
           for (int cc = 0; cc < CPL; ++cc) v = fmaf(blk[u][r][cc], xs[cc], v);
@@ -488,10 +506,12 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
 #pragma unroll
         for (int off = 1; off < CG; off <<= 1)
 #pragma unroll
-          for (int r = 0; r < 4; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
-        if (act && cg == 0)
-          *reinterpret_cast<float4*>(nxt + r0) =
-              make_float4(part[0] + qd[u][0], part[1] + qd[u][1], part[2] + qd[u][2], part[3] + qd[u][3]);
+          for (int r = 0; r < RPL; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
+        if (act && cg == 0) {
+#pragma unroll
+          for (int r = 0; r < RPL; ++r) part[r] += qd[u][r];
+          st_rows(nxt, part);
+        }
         __syncwarp();
         float* tmp = cur;
         cur = nxt;
@@ -502,9 +522,9 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
     if (!stall) {
       float xs[CPL];
       lds_n<CPL>(cur + j0, xs);
-      float part[4];
+      float part[RPL];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
+      for (int r = 0; r < RPL; ++r) {
         float v = 0.0f;
 #pragma unroll
         for (int cc = 0; cc < CPL; ++cc) v = fmaf(Pl[(r0 + r) * DP + j0 + cc], xs[cc], v);
@@ -513,10 +533,10 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
 #pragma unroll
       for (int off = 1; off < CG; off <<= 1)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
+        for (int r = 0; r < RPL; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
       if (act && cg == 0) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) P.pref[(size_t)k * P.pref_stride + r0 + r] = part[r] + Ql[r0 + r];
+        for (int r = 0; r < RPL; ++r) P.pref[(size_t)k * P.pref_stride + r0 + r] = part[r] + Ql[r0 + r];
       }
       __threadfence();
       __syncwarp();
@@ -524,12 +544,12 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
     }
 
     // ---- 5. apply the carry step by step over the run, chunk by chunk, write the states ------
-    // (the carry moves to the end of sO's row space: sX keeps it across the chunks' restaging)
+    // (sX holds the running state across the chunks' restaging)
     {
-      float sold[4];
-      lds_n<4>(cur + r0, sold);
-      if (cur != sX) {   // keep the running state at sX[0 .. DP-1]
-        if (act && cg == 0) *reinterpret_cast<float4*>(sX + r0) = make_float4(sold[0], sold[1], sold[2], sold[3]);
+      float sold[RPL];
+      ld_rows(cur, sold);
+      if (cur != sX) {
+        if (act && cg == 0) st_rows(sX, sold);
         __syncwarp();
       }
 #pragma unroll 1
@@ -542,21 +562,21 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
         const float* xcur = sX;
 #pragma unroll 1
         for (int m = 0; m < L; ++m) {
-          float pa[R][4];
+          float pa[R][RPL];
           slice_matvec(xcur, pa);
-          float c0[4], cq[R][4], bm[4];
-          lds_n<4>(sC + (m * NCS) * DP + r0, c0);
+          float c0[RPL], cq[R][RPL], bm[RPL];
+          ld_rows(sC + (m * NCS) * DP, c0);
 #pragma unroll
-          for (int q = 0; q < R; ++q) lds_n<4>(sC + (m * NCS + 1 + q) * DP + r0, cq[q]);
-          lds_n<4>(sB + m * DP + r0, bm);
+          for (int q = 0; q < R; ++q) ld_rows(sC + (m * NCS + 1 + q) * DP, cq[q]);
+          ld_rows(sB + m * DP, bm);
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
+          for (int r = 0; r < RPL; ++r) {
             float v = fmaf(c0[r], sold[r], bm[r]);
 #pragma unroll
             for (int q = 0; q < R; ++q) v = fmaf(cq[q][r], pa[q][r], v);
             sold[r] = v;
           }
-          if (act && cg == 0) *reinterpret_cast<float4*>(sO + m * DP + r0) = make_float4(sold[0], sold[1], sold[2], sold[3]);
+          if (act && cg == 0) st_rows(sO + m * DP, sold);
           __syncwarp();
           xcur = sO + m * DP;
         }
@@ -573,11 +593,12 @@ __global__ void __launch_bounds__(32 * NWARP) dense_warp_kernel(const IterParams
           }
         }
         // the chunk's last state starts the next chunk
-        if (act && cg == 0) *reinterpret_cast<float4*>(sX + r0) = make_float4(sold[0], sold[1], sold[2], sold[3]);
+        if (act && cg == 0) st_rows(sX, sold);
         __syncwarp();
       }
     }
   }
+
   // ---- residual of this iteration; the next one (grid barrier) or the end of the launch
   rbits = warp_max_u32(rbits);
   if (lane == 0) sRed[warp] = __uint_as_float(rbits);

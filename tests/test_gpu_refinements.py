@@ -233,16 +233,17 @@ def _run_storage(prob, mode, fmt, store_until, max_iters, tol):
 @pytest.mark.parametrize("fmt", ["bf16", "f16"])
 @pytest.mark.parametrize("max_iters", [1, 2, 3])
 def test_narrow_iterates_are_representable(fmt, max_iters):
-    """Stopped while still narrow (tol 0, store_until huge), the returned s^(max_iters) is exactly
-    representable in the format (the result copy widens it exactly, from either iterate buffer),
-    and matches the oracle's narrow iterate element by element up to the double-rounding cases."""
+    """Stopped while still narrow (tol 0; store_until 0, so every residual is above it), the returned
+    s^(max_iters) is exactly representable in the format (the result copy widens it exactly, from
+    either iterate buffer), and matches the oracle's narrow iterate element by element up to the
+    double-rounding cases."""
     store, _, unit = STORE_FMT[fmt]
     prob = pi.random_problem(381, pi.CELL_TANH_RNN, 16, 15, T=300, B=2, rho=0.7, s0_scale=0.3)
-    s, it, r, st, hist = _run_storage(prob, "quasi", fmt, 1e30, max_iters, 0.0)
+    s, it, r, st, hist = _run_storage(prob, "quasi", fmt, 0.0, max_iters, 0.0)
     assert (it, st) == (max_iters, oracle.NOT_CONVERGED)
     np.testing.assert_array_equal(oracle.round_storage(s.astype(np.float64), store), s.astype(np.float64))
     m = oracle.Model.from_problem(prob)
-    s_or, it_or, *_ = m.iterate_ex(pi.MODE_QUASI, prob.x, prob.s0, max_iters, 0.0, store=store, store_until=1e30)
+    s_or, it_or, *_ = m.iterate_ex(pi.MODE_QUASI, prob.x, prob.s0, max_iters, 0.0, store=store, store_until=0.0)
     diff = np.abs(s.astype(np.float64) - s_or)
     rel_unit = unit * np.maximum(np.abs(s_or), 1e-30)
     assert np.mean(diff > 0) < 1e-2                      # rare double-rounding flips ...
