@@ -912,11 +912,13 @@ pn_status select_kernels(pn_ctx* h) {
     h->fam.ngroups[m] = (m == PN_NEWTON) ? 1 : (D + ki.G - 1) / ki.G;
     if (h->fam.ngroups[m] > kMaxGroups)
       return fail(h, PN_ERR_INVALID, "D=%d needs %d channel groups (max %d)", D, h->fam.ngroups[m], kMaxGroups);
-    if (ki.smem > 48 * 1024) {
+    // Set even below 48 KB: dynamic plus static shared memory above 48 KB needs the opt-in too
+    // (dynamic 47.2 KB and 1 KB static leave no resident CTA without it).
+    if (ki.smem > 0) {
       cudaError_t e = cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.smem);
       if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     }
-    if (ki.pre_fn && ki.pre_smem > 48 * 1024) {
+    if (ki.pre_fn && ki.pre_smem > 0) {
       cudaError_t e = cudaFuncSetAttribute(ki.pre_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.pre_smem);
       if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     }

@@ -217,7 +217,7 @@ PN_API pn_status pn_eval_static(const float* params, size_t n_params, int D, int
   P.agg_stride = 2 * G;
   P.pref_stride = G;
   P.cond = 0;
-  if (ki.smem > 48 * 1024)
+  if (ki.smem > 0)   // also below 48 KB: dynamic plus static shared memory above it needs the opt-in
     PN_STATIC_CUDA(cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.smem));
   int per_sm = 0, nsm = 0;
   PN_STATIC_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ki.fn, ki.nt, ki.smem));

@@ -236,7 +236,9 @@ def test_narrow_iterates_are_representable(fmt, max_iters):
     """Stopped while still narrow (tol 0; store_until 0, so every residual is above it), the returned
     s^(max_iters) is exactly representable in the format (the result copy widens it exactly, from
     either iterate buffer), and matches the oracle's narrow iterate element by element up to the
-    double-rounding cases."""
+    double-rounding cases.  After one iteration a flip stays in its own element; from the second on,
+    a flip in s^(i-1)_{t-1,j} reaches every channel of step t through W and the later steps through
+    the scan, so there the bound is a few units of the format relative to the largest state."""
     store, _, unit = STORE_FMT[fmt]
     prob = pi.random_problem(381, pi.CELL_TANH_RNN, 16, 15, T=300, B=2, rho=0.7, s0_scale=0.3)
     s, it, r, st, hist = _run_storage(prob, "quasi", fmt, 0.0, max_iters, 0.0)
@@ -245,9 +247,13 @@ def test_narrow_iterates_are_representable(fmt, max_iters):
     m = oracle.Model.from_problem(prob)
     s_or, it_or, *_ = m.iterate_ex(pi.MODE_QUASI, prob.x, prob.s0, max_iters, 0.0, store=store, store_until=0.0)
     diff = np.abs(s.astype(np.float64) - s_or)
-    rel_unit = unit * np.maximum(np.abs(s_or), 1e-30)
-    assert np.mean(diff > 0) < 1e-2                      # rare double-rounding flips ...
-    assert np.all(diff <= 2.0 * rel_unit + 1e-7), float(np.max(diff / (rel_unit + 1e-30)))   # ... of one unit
+    if max_iters == 1:
+        rel_unit = unit * np.maximum(np.abs(s_or), 1e-30)
+        assert np.mean(diff > 0) < 1e-2                  # rare double-rounding flips ...
+        assert np.all(diff <= 2.0 * rel_unit + 1e-7), float(np.max(diff / (rel_unit + 1e-30)))   # ... of one unit
+    else:
+        scale = float(np.abs(s_or).max())
+        assert np.max(diff) <= 8.0 * unit * scale, float(np.max(diff) / (unit * scale))
 
 
 @pytest.mark.parametrize("cell", CELLS)
