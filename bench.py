@@ -57,6 +57,15 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--window", type=int, default=0,
                     help="time the windowed solve (pn_eval_windowed) with windows of this many steps instead")
+    ap.add_argument("--band", type=int, default=-1,
+                    help="newton: banded Jacobian with this half-bandwidth (PN_OPT_NEWTON_BAND)")
+    ap.add_argument("--damping", type=float, default=1.0, help="damping coefficient lambda in (0, 1]")
+    ap.add_argument("--adaptive", type=float, default=-1.0,
+                    help="adaptive switching with this stall ratio (>= 0; default off)")
+    ap.add_argument("--store", default="f32", choices=["f32", "bf16", "f16"],
+                    help="iterate storage while the residual is above --store-until")
+    ap.add_argument("--store-until", type=float, default=0.0)
+    ap.add_argument("--run-length", type=int, default=0, help="PN_OPT_RUN_LENGTH (0: automatic)")
     ap.add_argument("--host-loop", action="store_true",
                     help="host-driven convergence loop (plain kernel launches, e.g. for ncu) instead of the "
                          "device-side CUDA graph loop")
@@ -194,14 +203,29 @@ class ClockSampler:
 # the oracle on the host cores (CPU baseline / reference arm)
 # ----------------------------------------------------------------------------
 
-def cpu_sample(prob, mode, b_sample):
+def cpu_sample(prob, mode, b_sample, args=None):
+    """The oracle's iteration in the same mode (and variant: band, damping, adaptive switching,
+    storage format) on the first b_sample sequences."""
     import oracle
     m = oracle.Model.from_problem(prob)
     x = np.ascontiguousarray(prob.x[:b_sample])
     s0 = np.ascontiguousarray(prob.s0[:b_sample])
     threads = oracle.default_threads(b_sample)
+    v = variant(args) if args is not None else {}
     t0 = time.perf_counter()
-    _, it, _, _, _ = m.iterate(mode, x, s0, prob.iters_cap, prob.tol, nthreads=threads)
+    if {k: val for k, val in v.items() if k != "run_length"}:
+        band = v.get("newton_band", -1)
+        omode, oband = (oracle.BANDED, band) if (mode == pi.MODE_NEWTON and 0 <= band < prob.D - 1) else (mode, 0)
+        store = {"bf16": oracle.STORE_BF16, "f16": oracle.STORE_F16}.get(v.get("store"), oracle.STORE_F64)
+        # the library holds lambda, the stall ratio and store_until in float32
+        f32 = lambda a: float(np.float32(a))   # noqa: E731
+        _, it, _, _, _, _, _ = m.iterate_ex(omode, x, s0, prob.iters_cap, prob.tol, band=oband,
+                                            damping=f32(v.get("damping", 1.0)),
+                                            adapt="adaptive_stall" in v, stall=f32(v.get("adaptive_stall", 0.9)),
+                                            store=store, store_until=f32(v.get("store_until", 0.0)),
+                                            nthreads=threads)
+    else:
+        _, it, _, _, _ = m.iterate(mode, x, s0, prob.iters_cap, prob.tol, nthreads=threads)
     wall = time.perf_counter() - t0
     return prob.T * b_sample / wall, wall, it, threads
 
@@ -229,9 +253,9 @@ def cpu_model() -> str:
     return platform.processor() or "unknown"
 
 
-def cpu_baseline(prob, mode):
+def cpu_baseline(prob, mode, args=None):
     b_sample = max(1, min(prob.B, os.cpu_count() or 1))
-    v, wall, it, threads = cpu_sample(prob, mode, b_sample)
+    v, wall, it, threads = cpu_sample(prob, mode, b_sample, args)
     # context: the sequential loop the method replaces, on the same sample and threads, and on one
     # sequence with one thread
     seq = cpu_sequential(prob, b_sample, threads)
@@ -244,13 +268,48 @@ def cpu_baseline(prob, mode):
             "cpu_model": cpu_model(), "nproc": os.cpu_count()}
 
 
-def workload_config(prob, mode, world):
+def variant(args) -> dict:
+    """Settings beyond the plain iteration (banded Jacobian, damping, adaptive switching, narrow
+    iterate storage, run length); empty for the plain one."""
+    v = {}
+    if getattr(args, "band", -1) >= 0:
+        v["newton_band"] = args.band
+    if getattr(args, "damping", 1.0) != 1.0:
+        v["damping"] = args.damping
+    if getattr(args, "adaptive", -1.0) >= 0:
+        v["adaptive_stall"] = args.adaptive
+    if getattr(args, "store", "f32") != "f32":
+        v["store"] = args.store
+        v["store_until"] = args.store_until
+    if getattr(args, "run_length", 0) > 0:
+        v["run_length"] = args.run_length
+    return v
+
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def working_set_bytes(prob) -> int:
+    """x, the hoisted step inputs and two iterate buffers."""
+    rin = 3 if prob.cell == pi.CELL_GRU else 1
+    return int(prob.x.nbytes + (rin + 2) * prob.B * prob.T * prob.D * 4)
+
+
+def flush_l2_needed(prob) -> bool:
+    return working_set_bytes(prob) < 2 * L2_BYTES
+
+
+def workload_config(prob, mode, world, args=None):
     """The workload a line measures; both arms print the same dict for the same workload."""
-    return {"workload": prob.name, "mode": pi.MODE_NAMES[mode], "cell": pi.CELL_NAMES[prob.cell],
+    v = variant(args) if args is not None else {}
+    return {"workload": prob.name + "".join(f"_{k}{val}" for k, val in v.items()), **v, "mode": pi.MODE_NAMES[mode], "cell": pi.CELL_NAMES[prob.cell],
             "D": prob.D, "d_in": prob.d_in, "T": prob.T, "B": prob.B, "tol": prob.tol,
             "max_iters": prob.iters_cap, "parallelism": f"independent instances x{world}",
-            "l2": "inputs larger than L2 (x, u, two iterate buffers: "
-                  f"{(prob.x.nbytes + 3 * prob.B * prob.T * prob.D * 4) / 1e6:.0f} MB)"}
+            "l2": (f"L2 flushed before every timed step (a {2 * L2_BYTES >> 20} MB write outside the events): "
+                   f"working set {working_set_bytes(prob) / 1e6:.1f} MB"
+                   if flush_l2_needed(prob) else
+                   f"inputs larger than L2 (x, step inputs, two iterate buffers: "
+                   f"{working_set_bytes(prob) / 1e6:.0f} MB)")}
 
 
 def reference_arm(args, prob, mode, rank, world):
@@ -258,10 +317,10 @@ def reference_arm(args, prob, mode, rank, world):
         return
     b_sample = max(1, min(prob.B, os.cpu_count() or 1))
     for _ in range(args.warmup):
-        cpu_sample(prob, mode, b_sample)
+        cpu_sample(prob, mode, b_sample, args)
     walls, its = [], []
     for _ in range(args.steps):
-        _, wall, it, threads = cpu_sample(prob, mode, b_sample)
+        _, wall, it, threads = cpu_sample(prob, mode, b_sample, args)
         walls.append(wall)
         its.append(it)
     tot = sum(walls)
@@ -270,7 +329,7 @@ def reference_arm(args, prob, mode, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": workload_config(prob, mode, world),
+            "config": workload_config(prob, mode, world, args),
             "run": {"iters": its[-1], "sample_sequences": b_sample, "loop": "host (serial over t)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": f"fp64 oracle {pi.MODE_NAMES[mode]} iteration on the first {b_sample} "
@@ -313,6 +372,16 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
     solver = pn.Solver.from_problem(prob, stream=stream, device=dev)
     if args.host_loop:
         solver.set_option(pn.PN_OPT_DEVICE_LOOP, 0)
+    if args.band >= 0:
+        solver.set_option(pn.PN_OPT_NEWTON_BAND, args.band)
+    if args.run_length > 0:
+        solver.set_option(pn.PN_OPT_RUN_LENGTH, args.run_length)
+    if args.damping != 1.0:
+        solver.set_damping(args.damping)
+    if args.adaptive >= 0:
+        solver.set_adaptive(args.adaptive)
+    if args.store != "f32":
+        solver.set_storage({"bf16": pn.PN_STORE_BF16, "f16": pn.PN_STORE_F16}[args.store], args.store_until)
     x = torch.from_numpy(prob.x).to(dev)
     s0 = torch.from_numpy(prob.s0).to(dev)
     states = torch.empty((prob.B, prob.T, prob.D), device=dev, dtype=torch.float32)
@@ -329,16 +398,30 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
         torch.cuda.synchronize(dev)
 
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush = flush_l2_needed(prob)
+    scrub = torch.empty(2 * L2_BYTES // 4, device=dev, dtype=torch.float32) if flush else None
     with ClockSampler(local_rank) as clk:
         barrier()
         clk.mark_start()
-        e0.record(stream)
-        for _ in range(args.steps):
-            _, iters, resid, st = solver.eval(x, s0, mode, mi, tol, states)
-        e1.record(stream)
+        if flush:
+            # a working set below twice the L2: every step starts from a flushed L2, timed step by step
+            t_ms = 0.0
+            for _ in range(args.steps):
+                scrub.fill_(1.0)
+                e0.record(stream)
+                _, iters, resid, st = solver.eval(x, s0, mode, mi, tol, states)
+                e1.record(stream)
+                e1.synchronize()
+                t_ms += e0.elapsed_time(e1)
+        else:
+            e0.record(stream)
+            for _ in range(args.steps):
+                _, iters, resid, st = solver.eval(x, s0, mode, mi, tol, states)
+            e1.record(stream)
         barrier()
         clk.mark_end()
-    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    ms = max_over_ranks(t_ms if flush else e0.elapsed_time(e1), dist, dev)
+    del scrub
     stats = solver.stats()
     value = job_throughput(prob.T * prob.B * args.steps, world, ms)
     looping = pn.pn_dim(solver.h, 5 + mode) == 1 and not args.host_loop
@@ -348,7 +431,7 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(prob, mode, world),
+            "config": workload_config(prob, mode, world, args),
             "run": {"iters": iters, "final_resid": resid, "status": st,
                     "loop": "host" if args.host_loop else ("device (one launch iterating to the stop rule)"
                                                             if looping else "device (CUDA graph WHILE node)")},
@@ -444,7 +527,10 @@ def bench_windowed(args, prob, mode, rank, world, local_rank, dist):
                        "windows": nwin, "iters": iters, "window_iters": [int(n) for n in wit],
                        "final_resid": resid, "status": st,
                        "parallelism": f"independent instances x{world}",
-                       "l2": "inputs larger than L2 (the whole sequence is read and written once per step)"},
+                       "l2": (f"inputs larger than L2 (the whole sequence, {working_set_bytes(prob) / 1e6:.0f} MB "
+                              "of x, step inputs and iterates, is read and written once per step)"
+                              if not flush_l2_needed(prob) else
+                              f"L2 not flushed: working set {working_set_bytes(prob) / 1e6:.1f} MB")},
             "clocks": clk.summary(), "gpu_launches": sum(per_window) * args.steps}
     win.close()
     if tail is not None:
@@ -488,7 +574,7 @@ def main():
                 line = bench_pn(args, prob, mode, rank, world, local_rank, dist)
             if rank == 0:
                 if world == 1 and not args.no_cpu_baseline and args.window <= 0:
-                    line["cpu_baseline"] = cpu_baseline(prob, mode)
+                    line["cpu_baseline"] = cpu_baseline(prob, mode, args)
                 print(json.dumps(line), flush=True)
     finally:
         if dist is not None:

@@ -87,10 +87,17 @@ typedef enum {
   /* PN_NEWTON with a banded Jacobian approximation (page §2.2.2, banded
    * structure of locally connected systems): k >= 0 keeps the entries of
    * df_t/ds with |row - col| <= k (k = 0 is the diagonal, as PN_QUASI;
-   * k >= D - 1 the exact Jacobian); -1 (default) the exact Jacobian.  The
-   * cost per iteration is that of PN_NEWTON: the scan's aggregates stay
-   * dense, since products of banded matrices fill in. */
-  PN_OPT_NEWTON_BAND = 4
+   * k >= D - 1 the exact Jacobian); -1 (default) the exact Jacobian.  At
+   * D <= 32 the in-chunk products run over the band only (4 + 2k columns
+   * instead of D); the aggregates that cross chunks stay dense, since
+   * products of banded matrices fill in. */
+  PN_OPT_NEWTON_BAND = 4,
+  /* Consecutive scan chunks one ticket of the Newton kernels at D <= 32
+   * covers (a run: one aggregate per run in the look-back, the cell phase
+   * evaluated twice per chunk when the run is longer than one): 0 (default)
+   * chooses one run per resident warp where the work allows, n >= 1 fixes
+   * it (capped at the chunks of a sequence).  Other kernels ignore it. */
+  PN_OPT_RUN_LENGTH = 5
 } pn_option;
 
 /* Per-handle counters, cumulative since pn_create (or pn_reset_stats). */
@@ -224,7 +231,7 @@ PN_API pn_status pn_reset_stats(pn_handle h);
 
 /* Set one pn_option.  Values: PN_OPT_WAIT_TIMEOUT_NS >= 1000;
  * PN_OPT_DEBUG_STALL_TICKET -1 or a ticket >= 0; PN_OPT_NEWTON_BAND -1 or a
- * half-bandwidth >= 0; PN_OPT_DEVICE_LOOP and
+ * half-bandwidth >= 0; PN_OPT_RUN_LENGTH >= 0; PN_OPT_DEVICE_LOOP and
  * PN_OPT_TENSOR_CORES 0 or 1 (tensor cores: ignored where the shape has no
  * tensor-core kernel; switching re-selects the kernels after synchronising the
  * stream).  Anything else: PN_ERR_INVALID, the handle unchanged. */

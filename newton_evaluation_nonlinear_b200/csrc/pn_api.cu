@@ -15,6 +15,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <type_traits>
 #include <vector>
 
 #include "pn_aux.cuh"
@@ -65,7 +66,8 @@ struct pn_ctx {
   unsigned* flags = nullptr;
   float* agg = nullptr;
   float* pref = nullptr;
-  size_t agg_floats = 0, pref_floats = 0, nflags = 0;
+  size_t agg_floats = 0, pref_floats = 0, nflags = 0;        // what the selected tilings need
+  size_t agg_cap = 0, pref_cap = 0, flags_cap = 0;            // what is allocated
   Ctrl* ctrl = nullptr;
   Args* args = nullptr;
   float* hist = nullptr;
@@ -109,6 +111,7 @@ struct pn_ctx {
   long long timeout_ns = 1000000000LL;
   int stall_ticket = -1;
   int newton_band = -1;        // PN_OPT_NEWTON_BAND
+  int run_opt = 0;             // PN_OPT_RUN_LENGTH (0: automatic)
   float damping = 1.0f;        // pn_set_damping
   int store_fmt = 0;           // pn_set_storage: PN_STORE_F32 / _BF16 / _F16
   float store_until = 0.0f;
@@ -922,6 +925,14 @@ pn_status select_kernels(pn_ctx* h) {
       cudaError_t e = cudaFuncSetAttribute(ki.pre_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.pre_smem);
       if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     }
+    if (ki.reg_need > 0) {
+      // the kernel's warpgroups trade registers (setmaxnreg); their shares assume this many per
+      // thread at launch, and a smaller count would leave a share waiting for registers forever
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, ki.fn) != cudaSuccess || fa.numRegs < ki.reg_need)
+        return fail(h, PN_ERR_CUDA, "mode %d kernel: %d registers per thread at launch, its register shares need %d",
+                    m, fa.numRegs, ki.reg_need);
+    }
     int per_sm = 0, nsm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ki.fn, ki.nt, ki.smem) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || per_sm < 1)
@@ -933,6 +944,7 @@ pn_status select_kernels(pn_ctx* h) {
     if (ki.tpc > 0) {
       const long long takers = (long long)per_sm * nsm * ki.tpc;
       run = (int)std::max<long long>(1, ((long long)chunks * B + takers - 1) / takers);
+      if (h->run_opt > 0) run = std::min(h->run_opt, chunks);
     }
     h->fam.run[m] = run;
     h->fam.nchunks[m] = (chunks + run - 1) / run;
@@ -941,7 +953,10 @@ pn_status select_kernels(pn_ctx* h) {
     h->fam.resident[m] = per_sm * nsm;
     long long want = (long long)per_sm * nsm;
     want = std::max<long long>(ng, (want / ng) * ng);
-    h->fam.grid[m] = (int)std::min<long long>(want, h->fam.ntiles[m]);
+    // kernels with several ticket-takers per CTA need only enough CTAs for the tickets
+    const long long ctas_needed =
+        ki.tpc > 0 ? ((long long)h->fam.ntiles[m] + ki.tpc - 1) / ki.tpc : (long long)h->fam.ntiles[m];
+    h->fam.grid[m] = (int)std::max<long long>(1, std::min<long long>(want, ctas_needed));
     const size_t G = (size_t)ki.G;
     const size_t nt = (size_t)h->fam.ntiles[m];
     // the tensor-core kernels publish 64-bit tagged words: twice the floats
@@ -952,6 +967,31 @@ pn_status select_kernels(pn_ctx* h) {
     h->nflags = std::max(h->nflags, nt);
   }
   destroy_graphs(h);
+  // a re-selection (an option changed the kernels or their tiling) may need larger look-back buffers
+  // than create allocated: replace those (the stream has been synchronised), cleared like new ones.
+  // If that fails, no mode has a kernel until a later re-selection succeeds.
+  if (h->flags) {
+    auto grow = [&](auto** buf, size_t need, size_t* cap, size_t elem) -> bool {
+      if (need <= *cap) return true;
+      void* nb = nullptr;
+      if (cudaMalloc(&nb, need * elem) != cudaSuccess) return false;
+      if (cudaMemset(nb, 0, need * elem) != cudaSuccess) {
+        cudaFree(nb);
+        return false;
+      }
+      cudaFree(*buf);
+      *buf = static_cast<std::remove_reference_t<decltype(**buf)>*>(nb);
+      *cap = need;
+      return true;
+    };
+    if (!grow(&h->flags, h->nflags, &h->flags_cap, sizeof(unsigned)) ||
+        !grow(&h->agg, h->agg_floats, &h->agg_cap, sizeof(float)) ||
+        !grow(&h->pref, h->pref_floats, &h->pref_cap, sizeof(float))) {
+      cudaGetLastError();
+      for (int m = 0; m < 4; ++m) h->fam.k[m].fn = nullptr;
+      return fail(h, PN_ERR_NOMEM, "growing the look-back buffers for the new tiling failed");
+    }
+  }
   return PN_OK;
 }
 
@@ -1194,6 +1234,9 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
     PN_TRY(dalloc(h, &h->flags, h->nflags));
     PN_TRY(dalloc(h, &h->agg, h->agg_floats));
     PN_TRY(dalloc(h, &h->pref, h->pref_floats));
+    h->flags_cap = h->nflags;
+    h->agg_cap = h->agg_floats;
+    h->pref_cap = h->pref_floats;
     PN_TRY(dalloc(h, &h->ctrl, 1));
     PN_TRY(dalloc(h, &h->args, 1));
     PN_TRY(dalloc(h, &h->hist, kHistCap));
@@ -1569,6 +1612,15 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
         return select_kernels(h);
       }
       return PN_OK;
+    }
+    case PN_OPT_RUN_LENGTH: {
+      if (value < 0 || value > INT_MAX) return fail(h, PN_ERR_INVALID, "run length must be >= 0");
+      if ((int)value == h->run_opt) return PN_OK;
+      h->run_opt = (int)value;
+      DeviceGuard dg(h->device);
+      if (h->stream) cudaStreamSynchronize(h->stream);
+      else cudaDeviceSynchronize();
+      return select_kernels(h);
     }
     case PN_OPT_DEVICE_LOOP:
       if (value != 0 && value != 1) return fail(h, PN_ERR_INVALID, "device loop option is 0 or 1");

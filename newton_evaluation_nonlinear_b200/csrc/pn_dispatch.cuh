@@ -35,6 +35,7 @@ struct KInfo {
   const void* pre_fn = nullptr;   // launched before fn in every iteration (the tensor-core product Y = S W^T)
   int pre_nt = 0;
   size_t pre_smem = 0;
+  int reg_need = 0;     // > 0: per-thread registers at launch its warpgroups' setmaxnreg shares assume
 };
 
 template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS>
@@ -102,8 +103,9 @@ inline KInfo diag_tc_kinfo() {
 template <int CELL, int MODE, int DP>
 inline KInfo diag_tct_kinfo() {
   using C = DiagTctCfg<CELL, MODE, DP>;
-  return KInfo{(const void*)&diag_tct_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTct,
-               true};
+  KInfo k{(const void*)&diag_tct_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTct, true};
+  k.reg_need = C::kRegSplit ? C::REG_LAUNCH : 0;
+  return k;
 }
 
 template <int CELL, int DP, int L>

@@ -51,16 +51,21 @@ struct DenseWarpCfg {
   static constexpr int NCS = R + 1;                     // coefficient vectors per step: c0, c_1 .. c_R
   static constexpr int SP = DP + 4;                     // row stride of the staged s rows (16-byte rows)
   static constexpr int UP = R * DP + 1;                 // row stride of the staged step inputs
+  // row stride of P: the lanes of one store phase (rows r0, r0 + RPL of neighbouring row groups)
+  // land in disjoint banks (D = 16: 8 lanes x 16 bytes, row groups 48 words apart; D = 8: 32 lanes,
+  // row groups 24 words apart); other widths keep D
+  static constexpr int PS = (DP == 16) ? 24 : (DP == 8 ? 12 : DP);
   static constexpr int a4(int v) { return (v + 3) / 4 * 4; }
   // per-warp shared memory, in floats
   static constexpr int O_S = 0;                         // s^(i) rows t0-1 .. t0+L-1: [L+1][SP]
   static constexpr int O_U = a4(O_S + (L + 1) * SP);    // step inputs [L][UP]
   static constexpr int O_C = a4(O_U + L * UP);          // coefficients [L][NCS][DP]
   static constexpr int O_B = O_C + L * NCS * DP;        // b_m [L][DP]
-  static constexpr int O_P = O_B + L * DP;              // P double buffer [2][DP][DP]
-  static constexpr int O_Q = O_P + 2 * DP * DP;         // q double buffer [2][DP]
-  static constexpr int O_O = O_Q + 2 * DP;              // new states [L][DP]
-  static constexpr int O_X = O_O + L * DP;              // carry and fold scratch [2][DP]
+  static constexpr int O_P = O_B + L * DP;              // P double buffer [2][DP][PS]
+  static constexpr int O_Q = O_P + 2 * DP * PS;         // q double buffer [2][DP]
+  static constexpr int O_O = O_U;                       // new states [L][DP], over the step inputs
+                                                        // (consumed by the cell phase before)
+  static constexpr int O_X = O_Q + 2 * DP;              // carry and fold scratch [2][DP]
   static constexpr int WARP_FLOATS = a4(O_X + 2 * DP);
   // per-CTA: W_q^T for the cell [DP][R*DP] (k-major rows: W_q[i][k] at k*R*DP + q*DP + i), the banded
   // copy used by the Jacobian (same layout), then the warps' slices
@@ -107,6 +112,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
   constexpr int RPL = C::RPL;
   constexpr int SP = C::SP;
   constexpr int UP = C::UP;
+  constexpr int PS = C::PS;
   constexpr int WR = R * DP;   // row length of the transposed weights
 
   extern __shared__ __align__(16) float smem_dw[];
@@ -183,8 +189,29 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
   // W_q[r0 + r][k] of the Jacobian (band-masked when banded), RPL consecutive rows
   auto wrows = [&](int kk, int q, float (&w)[RPL]) { lds_n<RPL>(sWj + kk * WR + q * DP + r0, w); };
 
-  // y = sum over the k-slice of W_q[r0 + r][k] x[k], reduced over the column-group lanes
+  // y = W_q x for rows r0 .. r0 + RPL - 1.  With the W rows in registers (one gate, no band) every
+  // lane forms the whole sum from x read by broadcast; otherwise the sum over the lane's k-slice,
+  // with W from shared memory, is reduced over the column-group lanes.
   auto slice_matvec = [&](const float* x, float (&out)[R][RPL]) {
+    if constexpr (C::WREG) {
+      if (!banded) {
+        float acc[RPL];
+#pragma unroll
+        for (int r = 0; r < RPL; ++r) acc[r] = 0.0f;
+#pragma unroll
+        for (int kk = 0; kk < DP; kk += 4) {
+          const float4 x4 = *reinterpret_cast<const float4*>(x + kk);
+          const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int r = 0; r < RPL; ++r) acc[r] = fmaf(wreg[r][kk + u], xv[u], acc[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < RPL; ++r) out[0][r] = acc[r];
+        return;
+      }
+    }
     float xs[CPL];
     lds_n<CPL>(x + j0, xs);
 #pragma unroll
@@ -348,7 +375,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
 #pragma unroll
         for (int q = 0; q < R; ++q) ld_rows(sC + (m * NCS + 1 + q) * DP, cq[q]);
         ld_rows(sB + m * DP, bm);
-        float* Pn = sP + (gs & 1) * DP * DP;
+        float* Pn = sP + (gs & 1) * DP * PS;
         float qn[RPL];
         if (gs == 0) {
 #pragma unroll
@@ -364,7 +391,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
             qn[r] = bm[r];
           }
         } else {
-          const float* Pk = sP + ((gs - 1) & 1) * DP * DP;
+          const float* Pk = sP + ((gs - 1) & 1) * DP * PS;
           const float* Qk = sQ + ((gs - 1) & 1) * DP;
           float acc[R][RPL][CPL];
 #pragma unroll
@@ -380,7 +407,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
 #pragma unroll
               for (int kk = 0; kk < DP; ++kk) {
                 float p[CPL];
-                lds_n<CPL>(Pk + kk * DP + j0, p);
+                lds_n<CPL>(Pk + kk * PS + j0, p);
 #pragma unroll
                 for (int r = 0; r < RPL; ++r)
 #pragma unroll
@@ -394,7 +421,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
 #pragma unroll 4
             for (int kk = klo; kk <= khi; ++kk) {
               float p[CPL];
-              lds_n<CPL>(Pk + kk * DP + j0, p);
+              lds_n<CPL>(Pk + kk * PS + j0, p);
 #pragma unroll
               for (int q = 0; q < R; ++q) {
                 float w[RPL];
@@ -431,12 +458,12 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
             if constexpr (CPL % 4 == 0) {
 #pragma unroll
               for (int cc = 0; cc < CPL; cc += 4)
-                *reinterpret_cast<float4*>(Pn + (r0 + r) * DP + j0 + cc) =
+                *reinterpret_cast<float4*>(Pn + (r0 + r) * PS + j0 + cc) =
                     make_float4(pold[r][cc], pold[r][cc + 1], pold[r][cc + 2], pold[r][cc + 3]);
             } else if constexpr (CPL == 2) {
-              *reinterpret_cast<float2*>(Pn + (r0 + r) * DP + j0) = make_float2(pold[r][0], pold[r][1]);
+              *reinterpret_cast<float2*>(Pn + (r0 + r) * PS + j0) = make_float2(pold[r][0], pold[r][1]);
             } else {
-              Pn[(r0 + r) * DP + j0] = pold[r][0];
+              Pn[(r0 + r) * PS + j0] = pold[r][0];
             }
           }
           if (cg == 0) st_rows(sQ + (gs & 1) * DP, qn);
@@ -444,7 +471,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
         __syncwarp();
       }
     }
-    const float* Pl = sP + ((gs - 1) & 1) * DP * DP;   // the run's aggregate [P | q]
+    const float* Pl = sP + ((gs - 1) & 1) * DP * PS;   // the run's aggregate [P | q]
     const float* Ql = sQ + ((gs - 1) & 1) * DP;
 
     // ---- 4. decoupled look-back over the runs of the sequence ---------------------------------
@@ -453,7 +480,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
       float* ag = P.agg + (size_t)k * P.agg_stride;
       for (int e = lane; e < DP * (DP + 1); e += 32) {
         const int i = e / (DP + 1), j = e % (DP + 1);
-        ag[e] = (j == DP) ? Ql[i] : Pl[i * DP + j];
+        ag[e] = (j == DP) ? Ql[i] : Pl[i * PS + j];
       }
       __threadfence();
       __syncwarp();
@@ -527,7 +554,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
       for (int r = 0; r < RPL; ++r) {
         float v = 0.0f;
 #pragma unroll
-        for (int cc = 0; cc < CPL; ++cc) v = fmaf(Pl[(r0 + r) * DP + j0 + cc], xs[cc], v);
+        for (int cc = 0; cc < CPL; ++cc) v = fmaf(Pl[(r0 + r) * PS + j0 + cc], xs[cc], v);
         part[r] = v;
       }
 #pragma unroll

@@ -28,12 +28,14 @@ def _pn():
     return pn
 
 
-def _run(prob, mode, tol=None, max_iters=None, device_loop=1, tc=1):
+def _run(prob, mode, tol=None, max_iters=None, device_loop=1, tc=1, opts=None):
     import torch
     pn = _pn()
     solver = pn.Solver.from_problem(prob)
     solver.set_option(pn.PN_OPT_DEVICE_LOOP, device_loop)
     solver.set_option(pn.PN_OPT_TENSOR_CORES, tc)
+    for name, value in (opts or {}).items():
+        solver.set_option(getattr(pn, name), value)
     x = torch.from_numpy(prob.x).cuda()
     s0 = torch.from_numpy(prob.s0).cuda()
     tol = prob.tol if tol is None else tol
@@ -50,7 +52,7 @@ def _relerr(a, ref):
     return float(np.abs(a.astype(np.float64) - ref).max()) / den
 
 
-def _check_against_oracle(prob, mode, tol=None, max_iters=None, device_loop=1, tc=1):
+def _check_against_oracle(prob, mode, tol=None, max_iters=None, device_loop=1, tc=1, opts=None):
     """tol defaults to prob.tol * max(1, max|s|): an fp32 iterate assembled by a parallel scan carries
     rounding of a few ulp(|s|) per step, so an absolute tol below ~1e-6 |s| would sit on the fp32
     floor (the Euler drift reaches |s| ~ 20 on these inputs; the tanh and GRU states stay within 1)."""
@@ -59,7 +61,7 @@ def _check_against_oracle(prob, mode, tol=None, max_iters=None, device_loop=1, t
     seq = m.sequential(prob.x, prob.s0)
     tol = prob.tol * max(1.0, float(np.abs(seq).max())) if tol is None else tol
     s_or, it_or, r_or, st_or, hist_or = m.iterate(mode, prob.x, prob.s0, mi, tol)
-    s, it, r, st, hist = _run(prob, mode, tol, mi, device_loop, tc)
+    s, it, r, st, hist = _run(prob, mode, tol, mi, device_loop, tc, opts)
     assert np.isfinite(s).all()
     margin = float(np.min(np.abs(hist_or / tol - 1.0))) if tol > 0 else 1.0
     if margin > 1e-2:
@@ -342,3 +344,48 @@ def test_wide_tensor_core_product(tc, cell, mode, D, T, B):
     if mode == pi.MODE_JACOBI:
         prob.max_iters = T
     _check_against_oracle(prob, mode, tc=tc)
+
+
+@pytest.mark.parametrize("device_loop", [1, 0])
+@pytest.mark.parametrize("run", [1, 3, 0])
+@pytest.mark.parametrize("cell,D", [(pi.CELL_TANH_RNN, 16), (pi.CELL_GRU, 8), (pi.CELL_EULER, 4),
+                                    (pi.CELL_TANH_RNN, 32)])
+def test_newton_run_lengths(run, cell, D, device_loop):
+    """The Newton kernel at D <= 32 gives a ticket a run of consecutive 32-step chunks (one
+    aggregate per run; the cell phase evaluated again in the write-out pass when the run is longer
+    than one): one chunk, three (the last run ragged) and the automatic length all match the oracle,
+    looping in one launch or launched per iteration."""
+    T, B = 1000, 3   # 32 chunks, the last one ragged
+    d_in = D if cell == pi.CELL_EULER else D - 1
+    prob = pi.random_problem(1700 + 5 * D + cell, cell, D, d_in, T=T, B=B, rho=0.6, eps=0.05,
+                             s0_scale=0.3, tol=1e-5)
+    _check_against_oracle(prob, pi.MODE_NEWTON, device_loop=device_loop, tc=0,
+                          opts={"PN_OPT_RUN_LENGTH": run})
+
+
+def test_run_length_change_regrows_lookback():
+    """More chunks per sequence than the automatic tiling gives tickets (D = 16: 2 x 148 x 7 warps
+    take tickets, here 8 x 300 chunks): the automatic run length is 2, so run length 1 needs twice
+    the look-back buffers create allocated; the handle must grow them, and every setting, switched
+    on one handle, still matches the oracle."""
+    import torch
+    pn = _pn()
+    prob = pi.random_problem(1811, pi.CELL_TANH_RNN, 16, 15, T=9600, B=8, rho=0.6, s0_scale=0.3, tol=1e-5)
+    m = oracle.Model.from_problem(prob)
+    seq = m.sequential(prob.x, prob.s0)
+    tol = prob.tol * max(1.0, float(np.abs(seq).max()))
+    s_or, it_or, _, st_or, hist_or = m.iterate(pi.MODE_NEWTON, prob.x, prob.s0, prob.T, tol)
+    exact = float(np.min(np.abs(hist_or / tol - 1.0))) > 1e-2   # no residual within 1% of tol
+    solver = pn.Solver.from_problem(prob)
+    solver.set_option(pn.PN_OPT_TENSOR_CORES, 0)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    for run in (0, 1, 3, 0, 1):
+        solver.set_option(pn.PN_OPT_RUN_LENGTH, run)
+        states, it, r, st = solver.eval(x, s0, "newton", prob.T, tol)
+        assert (it, st) == (it_or, st_or) if exact else abs(it - it_or) <= 1, (run, it, it_or)
+        if it == it_or:
+            assert _relerr(states.cpu().numpy(), s_or) <= REL_TOL, run
+    with pytest.raises(pn.PnError):
+        solver.set_option(pn.PN_OPT_RUN_LENGTH, -1)
+    solver.close()
