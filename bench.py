@@ -424,17 +424,22 @@ def bench_pn(args, prob, mode, rank, world, local_rank, dist, with_extras=True):
     del scrub
     stats = solver.stats()
     value = job_throughput(prob.T * prob.B * args.steps, world, ms)
-    looping = pn.pn_dim(solver.h, 5 + mode) == 1 and not args.host_loop
-    # projection (not for the Euler cell), init, the iteration kernel(s), result copy
-    launches_per_step = (1 if looping else iters + 1) + 2 + (0 if prob.cell == pi.CELL_EULER else 1)
+    loop_kind = pn.pn_dim(solver.h, 5 + mode)
+    looping = loop_kind >= 1 and not args.host_loop
+    single = loop_kind == 2 and not args.host_loop
+    # projection (not for the Euler cell), init, the iteration kernel(s), result copy; or the one
+    # single-CTA launch of the small solve
+    launches_per_step = 1 if single else (1 if looping else iters + 1) + 2 + (0 if prob.cell == pi.CELL_EULER else 1)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(prob, mode, world, args),
             "run": {"iters": iters, "final_resid": resid, "status": st,
-                    "loop": "host" if args.host_loop else ("device (one launch iterating to the stop rule)"
-                                                            if looping else "device (CUDA graph WHILE node)")},
+                    "loop": "host" if args.host_loop else (
+                        "device (one single-CTA launch: projection, iterations, stop rule, result copy)" if single
+                        else "device (one launch iterating to the stop rule)" if looping
+                        else "device (CUDA graph WHILE node)")},
             "clocks": clk.summary(), "gpu_launches": launches_per_step * args.steps}
     if not with_extras:
         solver.close()
@@ -515,8 +520,9 @@ def bench_windowed(args, prob, mode, rank, world, local_rank, dist):
         clk.mark_end()
     ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     nwin = len(wit)
-    looping = pn.pn_dim(win.h, 5 + mode) == 1
-    per_window = [(1 if looping else int(n) + 1) + 2 + (0 if prob.cell == pi.CELL_EULER else 1) for n in wit]
+    loop_kind = pn.pn_dim(win.h, 5 + mode)
+    per_window = [1 if loop_kind == 2 else (1 if loop_kind == 1 else int(n) + 1) + 2 +
+                  (0 if prob.cell == pi.CELL_EULER else 1) for n in wit]
     line = {"metric": METRIC, "value": job_throughput(prob.T * prob.B * args.steps, world, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",

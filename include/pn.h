@@ -97,7 +97,15 @@ typedef enum {
    * evaluated twice per chunk when the run is longer than one): 0 (default)
    * chooses one run per resident warp where the work allows, n >= 1 fixes
    * it (capped at the chunks of a sequence).  Other kernels ignore it. */
-  PN_OPT_RUN_LENGTH = 5
+  PN_OPT_RUN_LENGTH = 5,
+  /* 1 (default): PN_NEWTON at D <= 8, when the problem's step inputs,
+   * iterate, Jacobian coefficients and chunk aggregates fit in one SM's
+   * shared memory (about B*T <= 3000 at D = 4 for the one-gate cells), runs
+   * the whole solve -- projection, every iteration with its stop rule, the
+   * result copy -- in one launch of one CTA, with the scan's chunk hand-off
+   * in shared memory; 0: the multi-CTA kernels.  Used only with the device
+   * loop and without adaptive switching. */
+  PN_OPT_SMALL_SOLVE = 6
 } pn_option;
 
 /* Per-handle counters, cumulative since pn_create (or pn_reset_stats). */
@@ -231,7 +239,7 @@ PN_API pn_status pn_reset_stats(pn_handle h);
 
 /* Set one pn_option.  Values: PN_OPT_WAIT_TIMEOUT_NS >= 1000;
  * PN_OPT_DEBUG_STALL_TICKET -1 or a ticket >= 0; PN_OPT_NEWTON_BAND -1 or a
- * half-bandwidth >= 0; PN_OPT_RUN_LENGTH >= 0; PN_OPT_DEVICE_LOOP and
+ * half-bandwidth >= 0; PN_OPT_RUN_LENGTH >= 0; PN_OPT_SMALL_SOLVE, PN_OPT_DEVICE_LOOP and
  * PN_OPT_TENSOR_CORES 0 or 1 (tensor cores: ignored where the shape has no
  * tensor-core kernel; switching re-selects the kernels after synchronising the
  * stream).  Anything else: PN_ERR_INVALID, the handle unchanged. */
@@ -328,7 +336,9 @@ PN_API pn_status pn_activation(int which, const float* x, float* y, long long n,
 /* Shape queries (for the binding); each returns -1 for a NULL handle.
  * which = 0..4: D, d_in, T, B, cell.  which = 5 + mode: 1 when that mode's
  * iteration kernel loops over the iterations on the device (one launch per
- * evaluation), 0 when pn_eval launches it once per iteration. */
+ * evaluation, between the projection and the result copy), 2 when one
+ * single-CTA launch runs the whole evaluation (PN_OPT_SMALL_SOLVE), 0 when
+ * pn_eval launches the iteration kernel once per iteration. */
 PN_API int pn_dim(pn_handle h, int which);
 
 /* Last error message of this handle; with h NULL, the calling thread's last

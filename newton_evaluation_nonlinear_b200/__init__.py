@@ -12,7 +12,7 @@ This package is the ctypes binding of that library; see :mod:`._binding`.
 from ._binding import (MODES, PN_CELL_EULER_TANH, PN_CELL_GRU, PN_CELL_TANH_RNN, PN_ERR_CUDA,  # noqa: F401
                        PN_ERR_INVALID, PN_ERR_NOMEM, PN_ERR_NONFINITE, PN_ERR_TIMEOUT, PN_JACOBI,
                        PN_MAX_D_DIAG, PN_MAX_D_NEWTON, PN_NEWTON, PN_NOT_CONVERGED, PN_OK,
-                       PN_OPT_DEBUG_STALL_TICKET, PN_OPT_DEVICE_LOOP, PN_OPT_NEWTON_BAND, PN_OPT_RUN_LENGTH, PN_OPT_TENSOR_CORES,
+                       PN_OPT_DEBUG_STALL_TICKET, PN_OPT_DEVICE_LOOP, PN_OPT_NEWTON_BAND, PN_OPT_RUN_LENGTH, PN_OPT_SMALL_SOLVE, PN_OPT_TENSOR_CORES,
                        PN_OPT_WAIT_TIMEOUT_NS,
                        PN_PICARD, PN_QUASI, PN_STORE_BF16, PN_STORE_F16, PN_STORE_F32,
                        SIGNATURES, STATUS_NAMES, LIB_PATH, PnError, Solver, lib,

@@ -24,6 +24,7 @@ PN_JACOBI, PN_PICARD, PN_QUASI, PN_NEWTON = 0, 1, 2, 3
 PN_OPT_WAIT_TIMEOUT_NS, PN_OPT_DEBUG_STALL_TICKET, PN_OPT_DEVICE_LOOP, PN_OPT_TENSOR_CORES = 0, 1, 2, 3
 PN_OPT_NEWTON_BAND = 4
 PN_OPT_RUN_LENGTH = 5
+PN_OPT_SMALL_SOLVE = 6
 PN_STORE_F32, PN_STORE_BF16, PN_STORE_F16 = 0, 1, 2
 PN_MAX_D_DIAG, PN_MAX_D_NEWTON = 256, 64
 

@@ -112,6 +112,8 @@ struct pn_ctx {
   int stall_ticket = -1;
   int newton_band = -1;        // PN_OPT_NEWTON_BAND
   int run_opt = 0;             // PN_OPT_RUN_LENGTH (0: automatic)
+  int small_opt = 1;           // PN_OPT_SMALL_SOLVE
+  KInfo small_k{nullptr, 0, 0, 0, 0, 0};   // the single-CTA Newton solve, when the problem fits
   float damping = 1.0f;        // pn_set_damping
   int store_fmt = 0;           // pn_set_storage: PN_STORE_F32 / _BF16 / _F16
   float store_until = 0.0f;
@@ -808,6 +810,17 @@ pn_status run_adaptive(pn_ctx* h, int mode) {
 
 // The loop body shared by pn_eval and pn_eval_host: args already point at
 // device buffers.
+// The single-CTA Newton solve: projection, initial guess, iterations, stop rule and result copy.
+pn_status launch_small(pn_ctx* h) {
+  IterParams P = make_params(h, PN_NEWTON);
+  const float* pw = h->proj_w;
+  const float* pb = h->proj_b;
+  void* kargs[] = {(void*)&P, (void*)&pw, (void*)&pb};
+  PN_CUDA(h, cudaLaunchKernel(h->small_k.fn, dim3(1), dim3((unsigned)h->small_k.nt), kargs, h->small_k.smem,
+                              h->stream));
+  return PN_OK;
+}
+
 pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
   pn_status st = prepare_lookback(h, mode);
   if (st != PN_OK) return st;
@@ -840,6 +853,9 @@ pn_status run_eval(pn_ctx* h, int mode, int* iters_out, float* resid_out) {
     PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
     if ((st = run_adaptive(h, mode)) != PN_OK) return st;
     if ((st = launch_finish(h)) != PN_OK) return st;
+  } else if (h->device_loop && mode == PN_NEWTON && h->small_k.fn) {
+    // the whole solve in one launch of one CTA
+    if ((st = launch_small(h)) != PN_OK) return st;
   } else if (h->device_loop && h->fam.k[mode].loops) {
     // the iteration kernel loops on the device: four plain launches, no graph needed
     if ((st = launch_pre(h)) != PN_OK) return st;
@@ -925,14 +941,6 @@ pn_status select_kernels(pn_ctx* h) {
       cudaError_t e = cudaFuncSetAttribute(ki.pre_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ki.pre_smem);
       if (e != cudaSuccess) return fail(h, PN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     }
-    if (ki.reg_need > 0) {
-      // the kernel's warpgroups trade registers (setmaxnreg); their shares assume this many per
-      // thread at launch, and a smaller count would leave a share waiting for registers forever
-      cudaFuncAttributes fa{};
-      if (cudaFuncGetAttributes(&fa, ki.fn) != cudaSuccess || fa.numRegs < ki.reg_need)
-        return fail(h, PN_ERR_CUDA, "mode %d kernel: %d registers per thread at launch, its register shares need %d",
-                    m, fa.numRegs, ki.reg_need);
-    }
     int per_sm = 0, nsm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ki.fn, ki.nt, ki.smem) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || per_sm < 1)
@@ -965,6 +973,22 @@ pn_status select_kernels(pn_ctx* h) {
     h->agg_floats = std::max(h->agg_floats, aggf);
     h->pref_floats = std::max(h->pref_floats, nt * G * wf);
     h->nflags = std::max(h->nflags, nt);
+  }
+  // Newton on a problem that fits in one SM's shared memory: the single-CTA solve
+  h->small_k = KInfo{nullptr, 0, 0, 0, 0, 0};
+  if (h->small_opt && DP <= 8 && h->fam.k[PN_NEWTON].fn) {
+    const int dpp = DP <= 4 ? 4 : 8;
+    const size_t bytes = small_smem_bytes(h->cell, dpp, B, T);
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device) == cudaSuccess &&
+        bytes + 1024 <= (size_t)optin) {
+      KInfo k = lookup_small(h->cell, dpp);
+      if (k.fn && cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess) {
+        k.smem = bytes;
+        h->small_k = k;
+      }
+    }
+    cudaGetLastError();
   }
   destroy_graphs(h);
   // a re-selection (an option changed the kernels or their tiling) may need larger look-back buffers
@@ -1527,6 +1551,33 @@ pn_status pn_time_iterations(pn_handle h, pn_mode mode, int n_launches, float* a
   // timed the same way: one launch that runs n_launches iterations (a tolerance below zero never
   // stops it early, max_iters ends it), average = elapsed / n_launches.  The others: n_launches
   // launches that each re-evaluate the same iterate (r <= +inf stops after one iteration).
+  const bool small = (mode == PN_NEWTON && h->small_k.fn && h->device_loop);
+  if (small) {
+    // the single-CTA solve: one launch of n_launches residual evaluations (n_launches - 1 updates)
+    h->args_h->tol = -1.0f;
+    h->args_h->max_iters = n_launches - 1;
+    h->args_h->use_cond = 0;
+    PN_CUDA(h, cudaMemcpyAsync(h->args, h->args_h, sizeof(Args), cudaMemcpyHostToDevice, h->stream));
+    cudaEvent_t e0, e1;
+    PN_CUDA(h, cudaEventCreate(&e0));
+    PN_CUDA(h, cudaEventCreate(&e1));
+    cudaError_t ce = cudaEventRecord(e0, h->stream);
+    st = (ce == cudaSuccess) ? launch_small(h) : PN_OK;
+    if (ce == cudaSuccess) ce = cudaEventRecord(e1, h->stream);
+    if (ce == cudaSuccess) ce = cudaEventSynchronize(e1);
+    float ms = 0.0f;
+    if (ce == cudaSuccess) ce = cudaEventElapsedTime(&ms, e0, e1);
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    if (st != PN_OK) return st;
+    if (ce != cudaSuccess) return fail(h, PN_ERR_CUDA, "timing failed: %s", cudaGetErrorString(ce));
+    PN_CUDA(h, cudaMemcpy(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost));
+    if (h->ctrl_h->final_iter != n_launches - 1)
+      return fail(h, PN_ERR_CUDA, "timing run stopped at iteration %d, expected %d", h->ctrl_h->final_iter,
+                  n_launches - 1);
+    *avg_ms = ms / (float)n_launches;
+    return PN_OK;
+  }
   const bool looping = h->fam.k[mode].loops;
   if (looping) {
     PN_CUDA(h, cudaMemcpy(h->ctrl_h, h->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost));
@@ -1617,6 +1668,15 @@ pn_status pn_set_option(pn_handle h, pn_option opt, long long value) {
       if (value < 0 || value > INT_MAX) return fail(h, PN_ERR_INVALID, "run length must be >= 0");
       if ((int)value == h->run_opt) return PN_OK;
       h->run_opt = (int)value;
+      DeviceGuard dg(h->device);
+      if (h->stream) cudaStreamSynchronize(h->stream);
+      else cudaDeviceSynchronize();
+      return select_kernels(h);
+    }
+    case PN_OPT_SMALL_SOLVE: {
+      if (value != 0 && value != 1) return fail(h, PN_ERR_INVALID, "small-solve option is 0 or 1");
+      if ((int)value == h->small_opt) return PN_OK;
+      h->small_opt = (int)value;
       DeviceGuard dg(h->device);
       if (h->stream) cudaStreamSynchronize(h->stream);
       else cudaDeviceSynchronize();
@@ -1717,7 +1777,9 @@ int pn_dim(pn_handle h, int which) {
     case 5 + PN_JACOBI:
     case 5 + PN_PICARD:
     case 5 + PN_QUASI:
-    case 5 + PN_NEWTON: return h->fam.k[which - 5].loops ? 1 : 0;
+    case 5 + PN_NEWTON:
+      if (which - 5 == PN_NEWTON && h->small_k.fn && h->device_loop && h->adapt_stall < 0.0f) return 2;
+      return h->fam.k[which - 5].loops ? 1 : 0;
     default: return -1;
   }
 }

@@ -12,6 +12,7 @@
 #include "pn_iter_diag.cuh"
 #include "pn_iter_diag_tc.cuh"
 #include "pn_iter_diag_tct.cuh"
+#include "pn_small.cuh"
 #include "pn_iter_diag_tma.cuh"
 #include "pn_wide_gemm.cuh"
 
@@ -35,7 +36,6 @@ struct KInfo {
   const void* pre_fn = nullptr;   // launched before fn in every iteration (the tensor-core product Y = S W^T)
   int pre_nt = 0;
   size_t pre_smem = 0;
-  int reg_need = 0;     // > 0: per-thread registers at launch its warpgroups' setmaxnreg shares assume
 };
 
 template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS>
@@ -103,9 +103,8 @@ inline KInfo diag_tc_kinfo() {
 template <int CELL, int MODE, int DP>
 inline KInfo diag_tct_kinfo() {
   using C = DiagTctCfg<CELL, MODE, DP>;
-  KInfo k{(const void*)&diag_tct_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTct, true};
-  k.reg_need = C::kRegSplit ? C::REG_LAUNCH : 0;
-  return k;
+  return KInfo{(const void*)&diag_tct_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTct,
+               true};
 }
 
 template <int CELL, int DP, int L>
@@ -232,10 +231,40 @@ inline KInfo lookup_cell(int mode, int DP, bool tma, bool tc) {
 #undef PN_DIAG_CASES
 }
 
+// The single-CTA Newton solve (DP = 4, 8): its kernel (smem: set by the caller from small_smem_bytes).
+template <int CELL>
+inline KInfo small_cell(int DP) {
+  if (DP == 4) return KInfo{(const void*)&small_solve_kernel<CELL, 4>, SmallCfg<CELL, 4>::NT, 32, 4, 0, kKindDense};
+  if (DP == 8) return KInfo{(const void*)&small_solve_kernel<CELL, 8>, SmallCfg<CELL, 8>::NT, 32, 8, 0, kKindDense};
+  return KInfo{nullptr, 0, 0, 0, 0, 0};
+}
+inline size_t small_smem_bytes(int cell, int DP, int B, int T) {
+  auto pick = [&](auto cfg4, auto cfg8) -> size_t {
+    return DP == 4 ? decltype(cfg4)::smem_bytes(B, T) : decltype(cfg8)::smem_bytes(B, T);
+  };
+  switch (cell) {
+    case PN_CELL_TANH_RNN: return pick(SmallCfg<PN_CELL_TANH_RNN, 4>{}, SmallCfg<PN_CELL_TANH_RNN, 8>{});
+    case PN_CELL_GRU: return pick(SmallCfg<PN_CELL_GRU, 4>{}, SmallCfg<PN_CELL_GRU, 8>{});
+    default: return pick(SmallCfg<PN_CELL_EULER_TANH, 4>{}, SmallCfg<PN_CELL_EULER_TANH, 8>{});
+  }
+}
+
 // Defined in one translation unit per cell (compiled in parallel).
 KInfo lookup_tanh(int mode, int DP, bool tma, bool tc);
 KInfo lookup_gru(int mode, int DP, bool tma, bool tc);
 KInfo lookup_euler(int mode, int DP, bool tma, bool tc);
+KInfo small_tanh(int DP);
+KInfo small_gru(int DP);
+KInfo small_euler(int DP);
+
+inline KInfo lookup_small(int cell, int DP) {
+  switch (cell) {
+    case PN_CELL_TANH_RNN: return small_tanh(DP);
+    case PN_CELL_GRU: return small_gru(DP);
+    case PN_CELL_EULER_TANH: return small_euler(DP);
+    default: return KInfo{nullptr, 0, 0, 0, 0, 0};
+  }
+}
 
 inline KInfo lookup(int cell, int mode, int DP, bool tma, bool tc) {
   switch (cell) {

@@ -40,9 +40,8 @@
 // quarters x RS / 16 step groups).  The split warps form a tile's S_lo as soon as its stage has
 // landed and the previous tile's products have read the S_lo buffer, so the tensor cores compute
 // the next tile's products while the epilogue works on the current one, and the epilogue's own
-// chain per tile holds only its cell phase, piece combine and write-out.  At D = 64 (768
-// threads, 80 registers each at launch) the warpgroups rebalance registers once per launch:
-// the epilogue takes 96, warps 0-3 keep 56, the split warps 40.
+// chain per tile holds only its cell phase, piece combine and write-out (D = 64: 768 threads, 80
+// registers each).
 #pragma once
 
 #include "pn_iter_diag_tc.cuh"
@@ -147,13 +146,6 @@ struct DiagTctCfg {
   static constexpr int NTS = 32 * NSPLIT;
   static constexpr int WE0 = WS0 + NSPLIT;       // first epilogue warp
   static constexpr int NT = 32 * (WE0 + NEW);
-  // Registers: where the launch's even share is below what the epilogue needs (D = 64: 768 threads,
-  // 80 each), the warpgroups rebalance with setmaxnreg; the shares add up to the launch's total.
-  static constexpr int REG_LAUNCH = (65536 / NT) / 8 * 8;
-  static constexpr bool kRegSplit = REG_LAUNCH < 96;
-  static constexpr int REG_EPI = 96, REG_CTL = 56, REG_SPLIT = 40;
-  static_assert(!kRegSplit || 32 * (4 * REG_CTL + NSPLIT * REG_SPLIT + NEW * REG_EPI) <= NT * REG_LAUNCH,
-                "register shares exceed the launch's registers");
   static constexpr int NQ = DP / 32;             // channels per look-back lane
   static constexpr int NLASTW = 4 / NB;          // epilogue warps holding the last piece of a channel
   static constexpr int WROWS = 3 * MT - DP;      // banded W: Z(64-D) W_hi Z(64-D) W_lo Z(64-D)
@@ -269,11 +261,6 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   const int iter0 = *(volatile int*)&ctrl->iter;
   const bool has_tile0 = (int)blockIdx.x < P.tiles_per_group;
   unsigned epoch = epoch0;
-  if constexpr (C::kRegSplit) {   // one share per warpgroup, taken once for the whole launch
-    if (warp >= C::WE0) reg_alloc<C::REG_EPI>();
-    else if (warp >= C::WS0) reg_dealloc<C::REG_SPLIT>();
-    else reg_dealloc<C::REG_CTL>();
-  }
   for (int round = 0;; ++round) {
   if (tid == 0) {
     if (round == 0) {

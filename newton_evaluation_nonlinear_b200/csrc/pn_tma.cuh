@@ -94,18 +94,4 @@ __device__ __forceinline__ void named_barrier(unsigned id, unsigned nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Per-thread register limit of the calling warpgroup (every thread of its four warps executes the
-// same one): release down to N, or take up to N from what other warpgroups released (it waits
-// until that much is free, so the shares of a launch must add up to at most its registers).
-template <int N>
-__device__ __forceinline__ void reg_dealloc() {
-  static_assert(N >= 24 && N <= 256 && N % 8 == 0, "register count");
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void reg_alloc() {
-  static_assert(N >= 24 && N <= 256 && N % 8 == 0, "register count");
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 }  // namespace pn

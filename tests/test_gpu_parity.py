@@ -389,3 +389,43 @@ def test_run_length_change_regrows_lookback():
     with pytest.raises(pn.PnError):
         solver.set_option(pn.PN_OPT_RUN_LENGTH, -1)
     solver.close()
+
+
+@pytest.mark.parametrize("small", [1, 0])
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("D,T,B", [(4, 1024, 1), (8, 200, 3), (3, 77, 2), (1, 33, 1), (5, 64, 4)])
+def test_newton_single_cta_solve(small, cell, D, T, B):
+    """Newton on problems that fit one SM's shared memory: the single-CTA solve (projection, every
+    iteration and the stop rule in one launch) and the multi-CTA kernel both match the oracle,
+    across whole and ragged 32-step chunks."""
+    pn = _pn()
+    d_in = D if cell == pi.CELL_EULER else max(1, D - 1)
+    prob = pi.random_problem(1900 + 3 * D + T + cell, cell, D, d_in, T=T, B=B, rho=0.6, eps=0.05,
+                             s0_scale=0.3, tol=1e-5)
+    solver = pn.Solver.from_problem(prob)
+    solver.set_option(pn.PN_OPT_SMALL_SOLVE, small)
+    assert pn.pn_dim(solver.h, 5 + pi.MODE_NEWTON) == (2 if small else 1)
+    solver.close()
+    _check_against_oracle(prob, pi.MODE_NEWTON, opts={"PN_OPT_SMALL_SOLVE": small})
+
+
+def test_newton_single_cta_limits_and_timing():
+    """A problem too large for one SM's shared memory runs the multi-CTA kernel; the timing hook
+    times the single-CTA solve as one launch of n residual evaluations."""
+    import torch
+    pn = _pn()
+    big = pi.random_problem(1931, pi.CELL_TANH_RNN, 8, 7, T=4096, B=2, rho=0.6, s0_scale=0.3)
+    sb = pn.Solver.from_problem(big)
+    assert pn.pn_dim(sb.h, 5 + pi.MODE_NEWTON) == 1
+    sb.close()
+    prob = pi.random_problem(1932, pi.CELL_TANH_RNN, 4, 4, T=1024, B=1, rho=0.5, s0_scale=0.3)
+    solver = pn.Solver.from_problem(prob)
+    assert pn.pn_dim(solver.h, 5 + pi.MODE_NEWTON) == 2
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    solver.eval(x, s0, "newton", prob.T, 1e-6)
+    ms = solver.time_iterations("newton", 5)
+    assert 0.0 < ms < 10.0
+    with pytest.raises(pn.PnError):
+        solver.set_option(pn.PN_OPT_SMALL_SOLVE, 2)
+    solver.close()

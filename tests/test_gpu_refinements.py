@@ -27,10 +27,11 @@ def _relerr(a, ref):
     return float(np.abs(a.astype(np.float64) - ref).max()) / den
 
 
-def _run(prob, band, tol, max_iters, damping=1.0, mode="newton", tc=1):
+def _run(prob, band, tol, max_iters, damping=1.0, mode="newton", tc=1, small=1):
     import torch
     import newton_evaluation_nonlinear_b200 as pn
     solver = pn.Solver.from_problem(prob)
+    solver.set_option(pn.PN_OPT_SMALL_SOLVE, small)
     solver.set_option(pn.PN_OPT_NEWTON_BAND, band)
     solver.set_option(pn.PN_OPT_TENSOR_CORES, tc)
     solver.set_damping(damping)
@@ -43,7 +44,7 @@ def _run(prob, band, tol, max_iters, damping=1.0, mode="newton", tc=1):
     return out, it, r, st, hist
 
 
-def _check(cell, D, T, B, band, damping, seed, mode="newton", tc=1):
+def _check(cell, D, T, B, band, damping, seed, mode="newton", tc=1, small=1):
     d_in = D if cell == pi.CELL_EULER else D - 1
     prob = pi.random_problem(seed, cell, D, d_in, T=T, B=B, rho=0.7, s0_scale=0.3, eps=0.05)
     m = oracle.Model.from_problem(prob)
@@ -56,7 +57,7 @@ def _check(cell, D, T, B, band, damping, seed, mode="newton", tc=1):
     lam = float(np.float32(damping))           # the library holds lambda in float32
     s_or, it_or, r_or, st_or, hist_or, _, _ = m.iterate_ex(mode_or, prob.x, prob.s0, T, tol, band=band_or,
                                                            damping=lam)
-    s, it, r, st, hist = _run(prob, band, tol, T, damping, mode, tc)
+    s, it, r, st, hist = _run(prob, band, tol, T, damping, mode, tc, small)
     assert np.isfinite(s).all()
     margin = float(np.min(np.abs(hist_or / tol - 1.0)))
     if margin > 1e-2:
@@ -71,16 +72,19 @@ def _check(cell, D, T, B, band, damping, seed, mode="newton", tc=1):
 
 
 @pytest.mark.parametrize("cell", CELLS)
-@pytest.mark.parametrize("D,T,B", [(8, 300, 2), (16, 517, 3)])
+@pytest.mark.parametrize("D,T,B,small", [(8, 300, 2, 1), (8, 300, 2, 0), (16, 517, 3, 1)])
 @pytest.mark.parametrize("band", [0, 1, 3, -1])
-def test_banded_newton_matches_oracle(cell, D, T, B, band):
-    _check(cell, D, T, B, band, 1.0, 301 + cell + D + band)
+def test_banded_newton_matches_oracle(cell, D, T, B, small, band):
+    """D = 8 fits the single-CTA solve (small = 1) and runs the multi-CTA warp-per-chunk kernel too."""
+    _check(cell, D, T, B, band, 1.0, 301 + cell + D + band, small=small)
 
 
 @pytest.mark.parametrize("cell", CELLS)
 @pytest.mark.parametrize("band,damping", [(-1, 0.5), (-1, 0.8), (2, 0.7)])
-def test_damped_newton_matches_oracle(cell, band, damping):
-    _check(cell, 12, 400, 2, band, damping, 321 + cell)
+@pytest.mark.parametrize("D,T", [(12, 400), (6, 300)])
+def test_damped_newton_matches_oracle(cell, band, damping, D, T):
+    """D = 6 runs the single-CTA solve, D = 12 the multi-CTA kernel."""
+    _check(cell, D, T, 2, band, damping, 321 + cell + D)
 
 
 @pytest.mark.parametrize("cell", CELLS)
@@ -296,3 +300,39 @@ def test_storage_arguments():
     solver.set_storage(pn.PN_STORE_F16, 1e-3)
     solver.set_storage(pn.PN_STORE_F32, 0.0)
     solver.close()
+
+
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("fmt,store_until", [("bf16", 3e-2), ("f16", 3e-3)])
+@pytest.mark.parametrize("small", [1, 0])
+def test_narrow_storage_newton_small_problem(cell, fmt, store_until, small):
+    """Narrow iterate storage in Newton mode at D = 6: the single-CTA solve rounds the iterate it
+    keeps in shared memory, the multi-CTA kernel its global buffers; both follow the oracle's rule."""
+    import newton_evaluation_nonlinear_b200 as pn
+    store, _, unit = STORE_FMT[fmt]
+    D, T = 6, 300
+    d_in = D if cell == pi.CELL_EULER else D - 1
+    prob = pi.random_problem(397 + cell, cell, D, d_in, T=T, B=2, rho=0.7, s0_scale=0.3, eps=0.05)
+    m = oracle.Model.from_problem(prob)
+    seq = m.sequential(prob.x, prob.s0)
+    scale = max(1.0, float(np.abs(seq).max()))
+    tol = 1e-5 * scale
+    s_or, it_or, r_or, st_or, hist_or, _, _ = m.iterate_ex(pi.MODE_NEWTON, prob.x, prob.s0, T, tol, store=store,
+                                                           store_until=store_until * scale)
+    import torch
+    solver = pn.Solver.from_problem(prob)
+    solver.set_option(pn.PN_OPT_SMALL_SOLVE, small)
+    assert pn.pn_dim(solver.h, 5 + pi.MODE_NEWTON) == (2 if small else 1)
+    solver.set_storage(STORE_FMT[fmt][1], store_until * scale)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    states, it, r, st = solver.eval(x, s0, "newton", T, tol)
+    hist = solver.residual_history()
+    s = states.cpu().numpy()
+    solver.close()
+    assert st == st_or
+    assert abs(it - it_or) <= 1, (it, it_or, hist.tolist(), hist_or.tolist())
+    if st == oracle.OK:
+        assert _relerr(s, seq) <= max(REL_TOL, 2.0 * _relerr(s_or, seq))
+    n = min(len(hist), len(hist_or))
+    np.testing.assert_allclose(hist[:n], hist_or[:n], rtol=1e-2, atol=8 * unit * scale)
