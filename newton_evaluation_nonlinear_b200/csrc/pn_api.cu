@@ -249,8 +249,9 @@ IterParams make_params(const pn_ctx* h, int mode) {
   IterParams P{};
   const bool dense = (mode == PN_NEWTON);
   const int kind = h->fam.k[mode].kind;
-  P.wt = dense ? h->wt_dense
-               : (kind == kKindDiagTc ? h->wt_tc : (kind == kKindDiagTct ? h->wt_tct : h->wt_diag));
+  P.wt = (dense || kind == kKindDiagPost)
+             ? h->wt_dense
+             : (kind == kKindDiagTc ? h->wt_tc : (kind == kKindDiagTct ? h->wt_tct : h->wt_diag));
   P.wt_tc = h->wt_tc;
   P.ypre = h->ypre;
   P.mode_hist = h->mode_hist_d;
@@ -983,7 +984,12 @@ pn_status select_kernels(pn_ctx* h) {
     if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device) == cudaSuccess &&
         bytes + 1024 <= (size_t)optin) {
       KInfo k = lookup_small(h->cell, dpp);
-      if (k.fn && cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess) {
+      // the attribute belongs to the function, not the handle: only ever raise it, so a handle
+      // with a smaller problem never lowers the limit another handle's launches rely on
+      cudaFuncAttributes fa{};
+      if (k.fn && cudaFuncGetAttributes(&fa, k.fn) == cudaSuccess &&
+          ((size_t)fa.maxDynamicSharedSizeBytes >= bytes ||
+           cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess)) {
         k.smem = bytes;
         h->small_k = k;
       }

@@ -13,13 +13,14 @@
 #include "pn_iter_diag_tc.cuh"
 #include "pn_iter_diag_tct.cuh"
 #include "pn_small.cuh"
+#include "pn_iter_diag_post.cuh"
 #include "pn_iter_diag_tma.cuh"
 #include "pn_wide_gemm.cuh"
 
 namespace pn {
 
 // Which weight packing and look-back format a kernel uses.
-enum KKind { kKindDiag = 0, kKindDiagTc = 1, kKindDense = 2, kKindDiagTct = 3 };
+enum KKind { kKindDiag = 0, kKindDiagTc = 1, kKindDense = 2, kKindDiagTct = 3, kKindDiagPost = 4 };
 
 // Kernels whose look-back aggregates and states are tagged 64-bit words.
 inline bool tagged_lookback(int kind) { return kind == kKindDiagTc || kind == kKindDiagTct; }
@@ -142,10 +143,9 @@ inline KInfo dense_pick() {
 // (wide_gemm_kernel), then the FP32 diagonal kernel reading it.
 template <int CELL, int MODE, int DP>
 inline KInfo diag_wide_kinfo() {
-  using C = DiagCfg<CELL, MODE, DP, 64, 4, 4, 16, true>;
+  using C = PostCfg<CELL, MODE, DP>;
   using W = WideGemmCfg<DP>;   // N = K = DP
-  KInfo k{(const void*)&diag_iter_kernel<CELL, MODE, DP, 64, 4, 4, 16, true>, C::NT, C::L, 64, C::SMEM_BYTES,
-          kKindDiag};
+  KInfo k{(const void*)&diag_post_kernel<CELL, MODE, DP>, C::NT, C::L, C::G, 0, kKindDiagPost};
   k.pre_fn = (const void*)&wide_gemm_kernel<DP>;
   k.pre_nt = W::NT;
   k.pre_smem = (size_t)W::SMEM_BYTES;

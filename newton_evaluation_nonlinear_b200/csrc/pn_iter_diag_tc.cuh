@@ -228,8 +228,10 @@ __device__ __forceinline__ float tf32_tail(float x) { return x - __uint_as_float
 
 // Bounded mbarrier wait that never leaves the caller's control flow: on
 // timeout / error it records the failure in *abort and returns false.
+// `site` (> 0) names the wait in the control block's timeout_ticket word (as -site) when it is
+// the one that gives up, so a timeout report says which wait of which role ran out.
 __device__ __forceinline__ bool mbar_wait_flag(uint64_t* bar, unsigned parity, Ctrl* ctrl, long long timeout_ns,
-                                               volatile int* abort) {
+                                               volatile int* abort, int site = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   unsigned spins = 0;
@@ -245,7 +247,7 @@ __device__ __forceinline__ bool mbar_wait_flag(uint64_t* bar, unsigned parity, C
         return false;
       }
       if ((long long)(globaltimer() - t0) > timeout_ns) {
-        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+        if (atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT) == 0 && site > 0) ctrl->timeout_ticket = -site;
         *abort = 1;
         return false;
       }

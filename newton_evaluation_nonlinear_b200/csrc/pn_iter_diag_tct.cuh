@@ -36,12 +36,10 @@
 // them, so both are fetched two tiles ahead of their use.
 //
 // Warp roles (one CTA per SM): 0 producer (tickets, TMA loads and state stores); 1 MMA issuer;
-// 2-3 look-back (scan modes, alternate tiles); 4-7 S_lo split; the rest epilogue (4 TMEM lane
-// quarters x RS / 16 step groups).  The split warps form a tile's S_lo as soon as its stage has
-// landed and the previous tile's products have read the S_lo buffer, so the tensor cores compute
-// the next tile's products while the epilogue works on the current one, and the epilogue's own
-// chain per tile holds only its cell phase, piece combine and write-out (D = 64: 768 threads, 80
-// registers each).
+// 2-3 look-back (scan modes, alternate tiles); the rest epilogue (4 TMEM lane
+// quarters x RS / 16 step groups).  The epilogue forms the next tile's S_lo
+// right after the current tile's cell phase, so the tensor cores compute the
+// next tile's products while the epilogue finishes the current one.
 #pragma once
 
 #include "pn_iter_diag_tc.cuh"
@@ -141,10 +139,7 @@ struct DiagTctCfg {
       USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128 : USED_COLS <= 256 ? 256 : 512;
   static constexpr int NEW = 4 * NRG;            // epilogue warps
   static constexpr int NTE = 32 * NEW;
-  static constexpr int WS0 = 4;                  // first S_lo split warp (warps 0-3: producer, MMA, look-back)
-  static constexpr int NSPLIT = 4;               // split warps (one warpgroup)
-  static constexpr int NTS = 32 * NSPLIT;
-  static constexpr int WE0 = WS0 + NSPLIT;       // first epilogue warp
+  static constexpr int WE0 = 2 + NLB;            // first epilogue warp
   static constexpr int NT = 32 * (WE0 + NEW);
   static constexpr int NQ = DP / 32;             // channels per look-back lane
   static constexpr int NLASTW = 4 / NB;          // epilogue warps holding the last piece of a channel
@@ -166,7 +161,6 @@ struct DiagTctCfg {
   static constexpr int OFF_CARRY = OFF_AGG + NAG * DP * 8;        // [NSLOT][DP]
   static constexpr int OFF_RED = OFF_CARRY + NSLOT * DP * 4;      // NT/32 floats
   static constexpr int SMEM_USED = OFF_RED + (NT / 32) * 4;
-  static_assert(NKH * L * 8 % (NTS * 4) == 0, "split batches cover the stage exactly");
   static constexpr int SMEM_BYTES = SMEM_USED + 1024;             // + slack to align the base to 1024 bytes
   // first row of band j's 64-row window of the banded W (W_hi or W_lo at window rows j D .. j D + D - 1)
   static constexpr int win_hi(int j) { return (MT - DP) - j * DP; }
@@ -203,8 +197,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       bar_mma[2],
       bar_tempty[2], bar_lb[C::NAG], bar_cfull[NSLOT], bar_cempty[NSLOT];
   __shared__ int s_tk[2];        // ticket staged in s stage 0/1 (-1: no more tiles)
-  __shared__ int s_atk[2];       // ticket of tile i's operands, by the parity of i (-1: stop), for the MMA warp
-  __shared__ int s_etk[2];       // the same decision for the epilogue
+  __shared__ int s_atk[2];       // ticket of tile i's operands, by the parity of i (-1: stop)
   __shared__ int s_lbtk[C::NAG];  // ticket handed to the look-back per slot (-1: stop)
   __shared__ int s_otk[2];        // ticket of the states staged in step-input buffer i (-1: none)
   __shared__ uint32_t s_tmem;
@@ -240,7 +233,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       mbar_init(&bar_cfull[s], 1u);
       mbar_init(&bar_cempty[s], (unsigned)C::NEW);
     }
-    mbar_init(&bar_afull, (unsigned)C::NSPLIT);
+    mbar_init(&bar_afull, (unsigned)C::NEW);
     mbar_init_fence();
   };
   auto inval_barriers = [&]() {
@@ -344,7 +337,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     // bar_oempty, for the epilogue's last events).
     int n_served = 0;
     auto serve = [&](int e) -> bool {
-      if (!mbar_wait_flag(&bar_ofull[e & 1], ((unsigned)e >> 1) & 1u, ctrl, tmo, &s_abort)) return false;
+      if (!mbar_wait_flag(&bar_ofull[e & 1], ((unsigned)e >> 1) & 1u, ctrl, tmo, &s_abort, 101)) return false;
       if (lane == 0) {
         const int ko = s_otk[e & 1];
         if (ko >= 0) {
@@ -367,7 +360,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       const int st = it & 1;
       // stage st's S buffer is free once tile it-2's cell phase is done; the ticket is claimed
       // only then, so a CTA holds no ticket it cannot start loading
-      if (it >= 2 && !mbar_wait_flag(&bar_sempty[st], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
+      if (it >= 2 && !mbar_wait_flag(&bar_sempty[st], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort, 102)) break;
       int kg = 0;
       if (lane == 0) kg = (int)(gridDim.x + atomicAdd(&ctrl->ticket[0], 1u));
       kg = __shfl_sync(0xffffffffu, kg, 0);
@@ -460,17 +453,17 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     int issued = 0;
     for (int it = 0;; ++it) {
       const int buf = it & 1;
-      if (!mbar_wait_flag(&bar_sfull[it & 1], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort)) break;
+      if (!mbar_wait_flag(&bar_sfull[it & 1], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort, 103)) break;
       const int kn = s_tk[it & 1];
       bool early = false;
       if (kn >= 0 && kn / B != 0) {
-        if (it >= 2 && !mbar_wait_flag(&bar_tempty[buf], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort)) break;
+        if (it >= 2 && !mbar_wait_flag(&bar_tempty[buf], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort, 104)) break;
         tc_fence_after();
         if (lane == 0) issue(it, 0, 2);
         __syncwarp();
         early = true;
       }
-      const bool ok = mbar_wait_flag(&bar_afull, (unsigned)it & 1u, ctrl, tmo, &s_abort);
+      const bool ok = mbar_wait_flag(&bar_afull, (unsigned)it & 1u, ctrl, tmo, &s_abort, 105);
       if (!ok || s_atk[it & 1] < 0) {
         if (early) {   // let the issued products complete before the accumulator is released
           if (lane == 0) umma_commit(&bar_mma[buf]);
@@ -479,7 +472,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         }
         break;
       }
-      if (!early && it >= 2 && !mbar_wait_flag(&bar_tempty[buf], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort))
+      if (!early && it >= 2 && !mbar_wait_flag(&bar_tempty[buf], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort, 106))
         break;
       tc_fence_after();
       if (lane == 0) {
@@ -492,7 +485,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     for (int j = max(0, issued - 2); j < issued; ++j)
       if (!mbar_drain(&bar_mma[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
         atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
-  } else if (warp < C::WS0) {
+  } else if (warp < C::WE0) {
     // =========================== look-back ==================================
     // warp 2 + j takes tiles j, j + NLB, ...; self-validating words, flags as hints
     if constexpr (kScan) {
@@ -503,7 +496,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         const int aslot = it % C::NAG;   // aggregate hand-off slot
         const int slot = it % NSLOT;     // carry slot
         const unsigned ph = (unsigned)(it / NSLOT) & 1u;
-        if (!mbar_wait_flag(&bar_lb[aslot], (unsigned)(it / C::NAG) & 1u, ctrl, tmo, &s_abort)) break;
+        if (!mbar_wait_flag(&bar_lb[aslot], (unsigned)(it / C::NAG) & 1u, ctrl, tmo, &s_abort, 107)) break;
         const int kg = s_lbtk[aslot];
         if (kg < 0) break;
         const int b = kg % B;
@@ -540,7 +533,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         }
         if (n_agg < 0) s_abort = 1;
         // 3. hand the carry to the epilogue (its slot is free once tile it - NSLOT was formed)
-        if (it >= NSLOT && !mbar_wait_flag(&bar_cempty[slot], ph ^ 1u, ctrl, tmo, &s_abort)) break;
+        if (it >= NSLOT && !mbar_wait_flag(&bar_cempty[slot], ph ^ 1u, ctrl, tmo, &s_abort, 108)) break;
 #pragma unroll
         for (int q = 0; q < C::NQ; ++q) sCarry[slot * DP + lane + 32 * q] = carry[q];
         __syncwarp();
@@ -554,56 +547,6 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
           if (lane == 0) st_relaxed(P.flags + k, make_flag(epoch, kFlagPrefix));
         }
       }
-    }
-  } else if (warp < C::WE0) {
-    // =========================== S_lo split =================================
-    // S_lo = S - tf32(S) of every landed stage, swizzled like S, into the one S_lo buffer once the
-    // products of the previous tile have read it; for the first chunk of a sequence, row 0 (step
-    // -1, loaded as zero) becomes s0 first.  Then the operands' ticket (the exit decision) for the
-    // MMA warp.
-    const int ts = tid - 32 * C::WS0;
-    for (int it = 0;; ++it) {
-      const int stg = it & 1;
-      int kn = -1;
-      if (mbar_wait_flag(&bar_sfull[stg], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort)) kn = s_tk[stg];
-      if (kn >= 0 && it >= 1 &&
-          !mbar_wait_flag(&bar_mma[(it - 1) & 1], ((unsigned)(it - 1) >> 1) & 1u, ctrl, tmo, &s_abort))
-        kn = -1;
-      if (kn >= 0 && !s_abort) {
-        constexpr int NB4 = 4;                        // 16-byte chunks in flight per thread
-        constexpr int NU = NKH * L * 8 / C::NTS;      // 16-byte chunks per thread
-        const bool first = (kn / B) == 0;
-#pragma unroll 1
-        for (int k0 = 0; k0 < NU; k0 += NB4) {
-          float4 v[NB4];
-#pragma unroll
-          for (int k = 0; k < NB4; ++k) {
-            const int u = ts + (k0 + k) * C::NTS;
-            const int h = (u >> 3) / L;
-            v[k] = *reinterpret_cast<const float4*>(sS + (stg * NKH + h) * C::SH_BYTES +
-                                                    sw128_offset((u >> 3) % L, 4 * (u & 7)));
-          }
-#pragma unroll
-          for (int k = 0; k < NB4; ++k) {
-            const int u = ts + (k0 + k) * C::NTS;
-            const int r = (u >> 3) % L;
-            const int h = (u >> 3) / L;
-            const uint32_t off = sw128_offset(r, 4 * (u & 7));
-            if (first && r == 0) {
-              v[k] = __ldg(reinterpret_cast<const float4*>(A.s0 + (size_t)(kn % B) * D + 32 * h) + (u & 7));
-              *reinterpret_cast<float4*>(sS + (stg * NKH + h) * C::SH_BYTES + off) = v[k];
-            }
-            *reinterpret_cast<float4*>(sLo + h * C::LO_BYTES + off) =
-                make_float4(tf32_tail(v[k].x), tf32_tail(v[k].y), tf32_tail(v[k].z), tf32_tail(v[k].w));
-          }
-        }
-        fence_async_smem();   // generic writes -> the tensor cores (async proxy)
-      }
-      if (ts == 0) s_atk[it & 1] = s_abort ? -1 : kn;
-      named_barrier(2, C::NTS);   // every split warp's part written; one decision for all four
-      const int dec = s_atk[it & 1];
-      if (lane == 0) mbar_arrive(&bar_afull);
-      if (dec < 0) break;
     }
   } else {
     // =========================== epilogue ===================================
@@ -625,13 +568,56 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     const int cc = c & 31;                  // its column within the half
     const float wdc = sWd[c];
 
+    // S_lo of stage `stg` (rows 0..L-1), swizzled like S.  For the first chunk of a
+    // sequence, row 0 (step -1, loaded as zero) becomes s0 first.
+    auto split = [&](int stg, int kgs) {
+      constexpr int NU = NKH * L * 8 / NTE;   // 16-byte chunks per thread
+      static_assert(NU * NTE == NKH * L * 8, "split covers the stage exactly");
+      const bool first = (kgs / B) == 0;
+      float4 v[NU];
+#pragma unroll
+      for (int k = 0; k < NU; ++k) {   // all loads first
+        const int u = te + k * NTE;
+        const int h = (u >> 3) / L;
+        v[k] = *reinterpret_cast<const float4*>(sS + (stg * NKH + h) * C::SH_BYTES + sw128_offset((u >> 3) % L, 4 * (u & 7)));
+      }
+#pragma unroll
+      for (int k = 0; k < NU; ++k) {
+        const int u = te + k * NTE;
+        const int r = (u >> 3) % L;
+        const int h = (u >> 3) / L;
+        const uint32_t off = sw128_offset(r, 4 * (u & 7));
+        if (first && r == 0) {
+          v[k] = __ldg(reinterpret_cast<const float4*>(A.s0 + (size_t)(kgs % B) * D + 32 * h) + (u & 7));
+          *reinterpret_cast<float4*>(sS + (stg * NKH + h) * C::SH_BYTES + off) = v[k];
+        }
+        *reinterpret_cast<float4*>(sLo + h * C::LO_BYTES + off) =
+            make_float4(tf32_tail(v[k].x), tf32_tail(v[k].y), tf32_tail(v[k].z), tf32_tail(v[k].w));
+      }
+      fence_async_smem();   // generic writes -> the tensor cores (async proxy)
+    };
+
+    // operands of the tile after `itn - 1`: wait for its stage, split it, publish its ticket
+    // (the exit decision, read by everyone after the next named barrier) and wake the MMA warp
+    auto prepare = [&](int itn) {
+      const int stg = itn & 1;
+      int kn = -1;
+      if (mbar_wait_flag(&bar_sfull[stg], ((unsigned)itn >> 1) & 1u, ctrl, tmo, &s_abort, 109)) kn = s_tk[stg];
+      if (kn >= 0 && !s_abort) split(stg, kn);
+      __syncwarp();
+      if (lane == 0) {
+        if (te == 0) s_atk[itn & 1] = s_abort ? -1 : kn;
+        mbar_arrive(&bar_afull);
+      }
+    };
+
     // s^(i+1) of tile j: piece carry from the look-back carry, then the parked prefixes (the
     // stash holds [A 0-7 | B 0-7 | A 8-15 | B 8-15] per 16 steps; B only for Picard), staged for
     // the producer's tensor store in step-input buffer `stg` (whose inputs every epilogue warp
     // has consumed), eight steps at a time
     auto stage_out = [&](int j, float pa, float pb, int stg) {
       const int slot = j % NSLOT;
-      mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort);
+      mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort, 110);
       const float carry = sCarry[slot * DP + c];
       // Picard parks only B: its damped A_t = lambda enters here
       const float cp = kHasA ? fmaf(pa, carry, pb) : (carry + pb) * lambda;
@@ -654,18 +640,9 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
 
     // The loop's exit decision is one thread's reading of the next stage's ticket,
     // published before a named barrier, so every epilogue thread takes the same path.
-    // the ticket of tile `itn` once its stage has landed (the split warps prepare its operands),
-    // published for the whole epilogue by its first thread before the next named barrier
-    auto next_ticket = [&](int itn) {
-      if (e == 0) {
-        int kn = -1;
-        if (mbar_wait_flag(&bar_sfull[itn & 1], ((unsigned)itn >> 1) & 1u, ctrl, tmo, &s_abort)) kn = s_tk[itn & 1];
-        if (te == 0) s_etk[itn & 1] = s_abort ? -1 : kn;
-      }
-    };
-    next_ticket(0);
+    prepare(0);
     named_barrier(1, NTE);
-    int kg = s_etk[0];
+    int kg = s_atk[0];
     int it = 0;
     int kg_m1 = -1, kg_m2 = -1, kg_m3 = -1;  // tickets of tiles it-1, it-2, it-3
     float pa1 = 1.0f, pb1 = 0.0f, pa2 = 1.0f, pb2 = 0.0f, pa3 = 1.0f, pb3 = 0.0f;   // their piece prefixes
@@ -676,11 +653,11 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       const int t0 = (kg / B) * L;
 
       // ---- Z of this thread's channel and 16 steps, then cell + sequential scan
-      mbar_wait_flag(&bar_mma[buf], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort);
+      mbar_wait_flag(&bar_mma[buf], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort, 111);
       tc_fence_after();
       float z[16];
       tmem_ld16(tmem + (uint32_t)(buf * RS + 16 * rg) + lane_off, z);
-      mbar_wait_flag(&bar_xfull[st], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort);
+      mbar_wait_flag(&bar_xfull[st], ((unsigned)it >> 1) & 1u, ctrl, tmo, &s_abort, 112);
       // rows row0 .. row0 + 16 of the swizzled stage (row0 is a multiple of 16, so the swizzle
       // phase of row row0 + i is i mod 8): byte offset = 128 (row0 + i) + (cq ^ (i mod 8)) 16 + (cc mod 4) 4
       const unsigned char* Sh = sS + (st * NKH + hc) * C::SH_BYTES + row0 * 128 + (cc & 3) * 4;
@@ -747,7 +724,8 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         mbar_arrive(&bar_tempty[buf]);
         mbar_arrive(&bar_sempty[st]);
       }
-      next_ticket(it + 1);
+      // the next tile's operands (S_lo is free: this tile's products are done)
+      prepare(it + 1);
 
 
       if constexpr (!kScan) {
@@ -761,13 +739,13 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         if (te == 0) s_otk[st] = -1;   // nothing staged: the step-input buffer is free
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_ofull[st]);
-        kg = s_etk[(it + 1) & 1];
+        kg = s_atk[(it + 1) & 1];
       } else {
         // ---- combine the 8 pieces of each channel
         float* tot = sTot + (it & 1) * C::NPC * DP * 2;
         *reinterpret_cast<float2*>(tot + (piece * DP + c) * 2) = make_float2(SA, SB);
         named_barrier(1, NTE);   // piece totals, and the ticket of tile it+1
-        const int kg_next = s_etk[(it + 1) & 1];
+        const int kg_next = s_atk[(it + 1) & 1];
         float PA = 1.0f, PB = 0.0f;   // prefix of the earlier pieces
         {
           float2 w[C::NPC - 1];   // all loads in flight together
@@ -828,7 +806,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
         const int ev = it + j;
         const int tj = ev - C::DEFER;
         const int st = ev & 1;
-        if (ev >= 2) mbar_wait_flag(&bar_oempty[st], ((unsigned)(ev - 2) >> 1) & 1u, ctrl, tmo, &s_abort);
+        if (ev >= 2) mbar_wait_flag(&bar_oempty[st], ((unsigned)(ev - 2) >> 1) & 1u, ctrl, tmo, &s_abort, 113);
         const int kj = (j == 0) ? kg_m3 : (j == 1 ? kg_m2 : kg_m1);
         const float pa = (j == 0) ? pa3 : (j == 1 ? pa2 : pa1);
         const float pb = (j == 0) ? pb3 : (j == 1 ? pb2 : pb1);
