@@ -319,10 +319,11 @@ PN_API pn_status pn_set_stream(pn_handle h, void* cuda_stream);
  * PN_ERR_INVALID with the needed size in pn_last_error(NULL), which also holds
  * the text of every other error of this call.
  * The first call on each device looks up the array's device address (with that
- * device current); make that first call before any stream capture.  Every call
- * reuses the same array and leaves its contents behind: calls that overlap on
- * the GPU (other threads, other streams) race and corrupt each other.  The loop
- * runs from the host, one kernel launch per iteration. */
+ * device current).  Every call clears the look-back flags it will use, reuses
+ * the same array and leaves its contents behind: calls that overlap on the GPU
+ * (other threads, other streams) race and corrupt each other.  The loop runs
+ * from the host, one kernel launch per iteration, with the control block read
+ * back after each. */
 PN_API pn_status pn_eval_static(const float* params, size_t n_params, int D, int d_in, int T, int B,
                                 const float* x, const float* s0, pn_mode mode, int max_iters, float tol,
                                 float* states, int* iters_out, float* resid_out, void* cuda_stream);

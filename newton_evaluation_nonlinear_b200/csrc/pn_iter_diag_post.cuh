@@ -32,7 +32,7 @@ struct PostCfg {
 };
 
 template <int CELL, int MODE, int DP>
-__global__ void __launch_bounds__(PostCfg<CELL, MODE, DP>::NT, 4) diag_post_kernel(const IterParams P) {
+__global__ void __launch_bounds__(PostCfg<CELL, MODE, DP>::NT) diag_post_kernel(const IterParams P) {
   using C = PostCfg<CELL, MODE, DP>;
   constexpr int G = C::G;
   constexpr int L = C::L;
@@ -80,85 +80,98 @@ __global__ void __launch_bounds__(PostCfg<CELL, MODE, DP>::NT, 4) diag_post_kern
     const size_t row0 = (size_t)b * T + t0;        // row of step t0
 
     // s^(i)_{t0-1} and, for the first chunk, W s0
-    float sp = 0.0f, z0 = 0.0f;
+    float sp0 = 0.0f, z0 = 0.0f;
     if (cok) {
       if (t0 == 0) {
         const float* s0 = A.s0 + (size_t)b * D;
-        sp = __ldg(s0 + c);
+        sp0 = __ldg(s0 + c);
         for (int kk = 0; kk < D; ++kk) z0 = fmaf(__ldg(P.wt + (size_t)kk * DP + c), __ldg(s0 + kk), z0);
       } else {
-        sp = __ldg(src + (row0 - 1) * D + c);
+        sp0 = __ldg(src + (row0 - 1) * DP + c);
       }
     }
-
-    // ---- cell, diagonal Jacobian, residual and the in-tile prefixes, step by step
-    float pa[L], pb[L];
-    float SA = 1.0f, SB = 0.0f;
-#pragma unroll
-    for (int m0 = 0; m0 < L; m0 += U) {
-      float zv[U], xv[U], sv[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {   // the loads of U steps first
-        const int m = m0 + u;
-        const size_t r = row0 + m;
-        const bool ok = cok && m < n;
-        zv[u] = (ok && (t0 + m) > 0) ? __ldg(P.ypre + (r - 1) * D + c) : z0;
-        xv[u] = ok ? __ldg(xin + r * D + c) : 0.0f;
-        sv[u] = ok ? __ldg(src + r * D + c) : 0.0f;
+    // the cell, the diagonal Jacobian a_t, b_t = y_t - a_t s_{t-1} and F_t of a step from its loads:
+    // (a, b, F)
+    auto coef = [&](float z, float x, float sc, float sp) -> float3 {
+      float a, bb, res;
+      if constexpr (CELL == PN_CELL_TANH_RNN) {
+        const float y = tanh_pn(z + x);
+        res = sc - y;
+        a = (MODE == PN_QUASI) ? (1.0f - y * y) * wdc : (MODE == PN_PICARD ? 1.0f : 0.0f);
+        bb = (MODE == PN_JACOBI) ? y : y - a * sp;
+      } else {
+        const float gg = tanh_pn(z + x);
+        const float eg = P.eps * gg;
+        res = (sc - sp) - eg;
+        if (MODE == PN_QUASI) {
+          const float ed = P.eps * (1.0f - gg * gg) * wdc;
+          a = 1.0f + ed;
+          bb = eg - ed * sp;
+        } else if (MODE == PN_PICARD) {
+          a = 1.0f;
+          bb = eg;
+        } else {
+          a = 0.0f;
+          bb = sp + eg;
+        }
       }
+      return make_float3(a, bb, res);
+    };
+    // the loads of U steps from m0 on (all in flight together); rows are DP floats apart (the wide
+    // path runs only with D == DP), so every address is a base plus an immediate offset
+    const float* zrow = P.ypre + (row0 - 1) * DP + c;   // row of step t0 - 1 (never read for t = 0)
+    const float* xrow = xin + row0 * DP + c;
+    const float* srow = src + row0 * DP + c;
+    auto load = [&](int m0, float (&zv)[U], float (&xv)[U], float (&sv)[U]) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int m = m0 + u;
         const bool ok = cok && m < n;
-        const float sc = sv[u];
-        float y, a, bb, res;
-        if constexpr (CELL == PN_CELL_TANH_RNN) {
-          y = tanh_pn(zv[u] + xv[u]);
-          res = sc - y;
-          a = (MODE == PN_QUASI) ? (1.0f - y * y) * wdc : (MODE == PN_PICARD ? 1.0f : 0.0f);
-          bb = (MODE == PN_JACOBI) ? y : y - a * sp;
-        } else {
-          const float gg = tanh_pn(zv[u] + xv[u]);
-          const float eg = P.eps * gg;
-          y = sp + eg;
-          res = (sc - sp) - eg;
-          if (MODE == PN_QUASI) {
-            const float ed = P.eps * (1.0f - gg * gg) * wdc;
-            a = 1.0f + ed;
-            bb = eg - ed * sp;
-          } else if (MODE == PN_PICARD) {
-            a = 1.0f;
-            bb = eg;
+        zv[u] = (ok && (t0 + m) > 0) ? __ldg(zrow + m * DP) : z0;
+        xv[u] = ok ? __ldg(xrow + m * DP) : 0.0f;
+        sv[u] = ok ? __ldg(srow + m * DP) : 0.0f;
+      }
+    };
+
+    // ---- the residual, the tile's aggregate and its in-tile prefixes (Jacobi: the states)
+    float SA = 1.0f, SB = 0.0f;
+    float pa[L], pb[L];
+    {
+      float sp = sp0;
+#pragma unroll
+      for (int m0 = 0; m0 < L; m0 += U) {
+        float zv[U], xv[U], sv[U];
+        load(m0, zv, xv, sv);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int m = m0 + u;
+          const bool ok = cok && m < n;
+          const float3 f = coef(zv[u], xv[u], sv[u], sp);
+          float a = f.x, bb = f.y;
+          if (ok) {
+            rbits = max(rbits, abs_bits(f.z));
+            if constexpr (!kScan) dst[(row0 + m) * DP + c] = damped ? fmaf(lambda, bb - sv[u], sv[u]) : bb;
           } else {
-            a = 0.0f;
-            bb = y;
+            a = 1.0f;   // identity element: steps past T, channels past D
+            bb = 0.0f;
           }
-        }
-        if (ok) {
-          rbits = max(rbits, abs_bits(res));
-        } else {
-          a = 1.0f;   // identity element: steps past T, channels past D
-          bb = 0.0f;
-        }
-        if constexpr (kScan) {
           SB = fmaf(a, SB, bb);
           if (kHasA) SA *= a;
           pa[m] = SA;
           pb[m] = SB;
-        } else if (ok) {   // Jacobi: s^(i+1)_t = f_t(s^(i)_{t-1})
-          dst[(row0 + m) * D + c] = damped ? fmaf(lambda, bb - sc, sc) : bb;
+          sp = sv[u];
         }
-        sp = sc;
       }
     }
     if constexpr (!kScan) continue;
 
-    // ---- decoupled look-back: this tile's aggregate, the nearest published state, the carry
+    // ---- decoupled look-back: this tile's aggregate, the nearest published state, the carry.
+    // The barrier orders every thread's words before the releasing store (a cumulative release).
+    // Every thread writes its channel's words; the barrier orders them before the one releasing
+    // store of the flag (a release covers what precedes it in causality order).  Warp 0 acquires
+    // the predecessors' flags; the barrier after it orders every thread's loads of their words.
     const bool stall = (A.stall_ticket == (int)k);
-    if (chunk > 0 && !stall) {
-      reinterpret_cast<float2*>(P.agg + k * P.agg_stride)[tid] = make_float2(SA, SB);
-      __threadfence();
-    }
+    if (chunk > 0 && !stall) reinterpret_cast<float2*>(P.agg + k * P.agg_stride)[tid] = make_float2(SA, SB);
     __syncthreads();
     if (warp == 0) {
       if (lane == 0 && chunk > 0 && !stall) st_release(P.flags + k, make_flag(epoch, kFlagAgg));
@@ -168,7 +181,6 @@ __global__ void __launch_bounds__(PostCfg<CELL, MODE, DP>::NT, 4) diag_post_kern
     __syncthreads();
     const int n_agg = s_nagg;
     if (n_agg < 0) break;   // a wait gave up: the error is set, the launch winds down
-    fence_acquire_gpu();    // warp 0 saw the flags; this thread's loads of the words they cover follow
     float carry;
     if (chunk - 1 - n_agg >= 0) carry = __ldcg(P.pref + (k - (size_t)(n_agg + 1) * stride) * P.pref_stride + tid);
     else carry = cok ? __ldg(A.s0 + (size_t)b * D + c) : 0.0f;
@@ -182,14 +194,11 @@ __global__ void __launch_bounds__(PostCfg<CELL, MODE, DP>::NT, 4) diag_post_kern
 #pragma unroll
       for (int u = 0; u < 4; ++u) carry = fmaf(ab[u].x, carry, ab[u].y);
     }
-    if (!stall) {
-      P.pref[k * P.pref_stride + tid] = fmaf(SA, carry, SB);
-      __threadfence();
-    }
+    if (!stall) P.pref[k * P.pref_stride + tid] = fmaf(SA, carry, SB);
     __syncthreads();
     if (tid == 0 && !stall) st_release(P.flags + k, make_flag(epoch, kFlagPrefix));
 
-    // ---- the states of the tile: s_t = A_t carry + B_t (in-tile prefixes), damped against s^(i)_t
+    // ---- the states of the tile: s_t = A_t carry + B_t, damped against s^(i)_t
     if (cok) {
 #pragma unroll
       for (int m = 0; m < L; ++m) {
@@ -197,10 +206,10 @@ __global__ void __launch_bounds__(PostCfg<CELL, MODE, DP>::NT, 4) diag_post_kern
           const float v = fmaf(pa[m], carry, pb[m]);
           float o = v;
           if (damped) {
-            const float sc = __ldg(src + (row0 + m) * D + c);
+            const float sc = __ldg(srow + m * DP);
             o = fmaf(lambda, v - sc, sc);
           }
-          dst[(row0 + m) * D + c] = o;
+          dst[(row0 + m) * DP + c] = o;
         }
       }
     }

@@ -12,15 +12,19 @@
 //   1. one thread per (b, t, channel): y = f_t(s^(i)_{t-1}), the Jacobian's
 //      coefficient vectors (A_t = diag(c0) + sum_q diag(c_q) W_q), b_t and
 //      |F_t|; the block's max is r^(i), which decides the stop;
-//   2. one warp per 32-step chunk: the chunk's aggregate [P | q] (the product
-//      of its A_t, and the chunk's response to a zero entering state);
-//   3. one warp per sequence folds the aggregates chunk after chunk into each
-//      chunk's entering state (starting from s0), then one warp per chunk
-//      applies s_t = A_t s_{t-1} + b_t step by step and stores s^(i+1) in place
-//      of s^(i) (damped: s^(i) + lambda (s - s^(i)); narrow storage: rounded
-//      to the 16-bit format while the residual known at the update's start is
-//      above store_until).
-// Padded channels (D < DP) are identity maps with zero input.
+//   2. one thread per (32-step chunk, column j of [P | q]): the column of the
+//      chunk's aggregate, the product of its A_t applied to e_j (P) or the
+//      chunk's response to a zero entering state (q), held in registers step
+//      after step -- the columns of an affine product evolve independently;
+//   3. one thread per sequence folds the aggregates chunk after chunk into
+//      each chunk's entering state (starting from s0); then one thread per
+//      chunk applies s_t = A_t s_{t-1} + b_t step by step in registers and
+//      stores s^(i+1) in place of s^(i) (damped: s^(i) + lambda (s - s^(i));
+//      narrow storage: rounded to the 16-bit format while the residual known
+//      at the update's start is above store_until).
+// Per-step arrays are laid out chunk-interleaved (row m * ntiles + k for step
+// m of chunk k), so the threads of neighbouring chunks touch neighbouring
+// rows.  Padded channels (D < DP) are identity maps with zero input.
 #pragma once
 
 #include "pn_cells.cuh"
@@ -32,22 +36,36 @@ struct SmallCfg {
   static constexpr int R = CellInfo<CELL>::R;
   static constexpr int NCS = R + 1;   // coefficient vectors per step: c0, c_1 .. c_R
   static constexpr int L = 32;        // steps per chunk
-  static constexpr int NW = 32;       // warps
+  static constexpr int NW = 8;        // warps
   static constexpr int NT = 32 * NW;
   static constexpr int WR = R * DP;   // row length of the transposed weights
   static_assert(DP == 4 || DP == 8, "DP in {4, 8}");
-  // shared memory in floats: two weight copies, per-warp chain buffers, the block reduction, the
-  // s0 rows, then per step (step inputs, the iterate, coefficients, b_t) and per chunk (aggregate,
-  // entering state)
-  static constexpr size_t fixed_floats(int B) {
-    return 2 * (size_t)DP * WR + (size_t)NW * (2 * DP * DP + 2 * DP) + NW + (size_t)B * DP;
-  }
+  // shared memory in floats: two weight copies, the block reduction, the s0 rows, then per step
+  // (step inputs, the iterate, coefficients, b_t) and per chunk (aggregate, entering state)
+  static constexpr size_t fixed_floats(int B) { return 2 * (size_t)DP * WR + NW + (size_t)B * DP; }
+  // per-step arrays in chunk-interleaved rows: L rows per chunk (a ragged last chunk's rows past
+  // T are allocated and never read); step inputs in natural order, B T rows
   static constexpr size_t smem_bytes(int B, int T) {
     const size_t nbt = (size_t)B * T;
     const size_t ntiles = (size_t)B * ((T + L - 1) / L);
-    return 4 * (fixed_floats(B) + nbt * (WR + DP + NCS * DP + DP) + ntiles * (DP * DP + 2 * DP));
+    const size_t nrows = (size_t)L * ntiles;
+    return 4 * (fixed_floats(B) + nbt * WR + nrows * (DP + NCS * DP + DP) + ntiles * (DP * DP + 2 * DP));
   }
 };
+
+// N consecutive floats of shared memory (16-byte aligned) into registers, 16 bytes at a time
+template <int N>
+__device__ __forceinline__ void lds_vec(const float* p, float (&v)[N]) {
+  static_assert(N % 4 == 0, "whole float4s");
+#pragma unroll
+  for (int e = 0; e < N; e += 4) {
+    const float4 t = *reinterpret_cast<const float4*>(p + e);
+    v[e] = t.x;
+    v[e + 1] = t.y;
+    v[e + 2] = t.z;
+    v[e + 3] = t.w;
+  }
+}
 
 __device__ __forceinline__ float round_storage(float v, int fmt) {
   if (fmt == 1) return __bfloat162float(__float2bfloat16_rn(v));
@@ -77,24 +95,26 @@ __global__ void __launch_bounds__(SmallCfg<CELL, DP>::NT, 1)
   const int D = P.D, T = P.T, B = P.B, d_in = P.d_in;
   const int nch = (T + L - 1) / L;
   const int ntiles = B * nch;
-  const size_t nbt = (size_t)B * T;
+  const int nbt = B * T;   // the problem fits one SM's shared memory: far below 2^31
+  const int nrows = L * ntiles;   // chunk-interleaved rows (>= nbt: a ragged last chunk leaves gaps)
   const int band = A.newton_band;
   const bool banded = band >= 0 && band < D - 1;
   const float lambda = A.damping;
   const bool damped = lambda != 1.0f;
   const int sfmt = A.store_fmt;
 
-  float* sWf = smem_sm;                                   // W_q[i][k] at k * WR + q * DP + i
-  float* sWb = sWf + DP * WR;                             // the Jacobian's copy (band-masked)
-  float* sWarp = sWb + DP * WR;                           // per warp: P [2][DP*DP], q [2][DP]
-  float* sRed = sWarp + NW * (2 * DP * DP + 2 * DP);      // [NW]
-  float* sS0 = sRed + NW;                                 // s0 [B][DP]
-  float* sU = sS0 + (size_t)B * DP;                       // step inputs [B*T][WR]
-  float* sS = sU + nbt * WR;                              // the iterate [B*T][DP]
-  float* sCf = sS + nbt * DP;                             // coefficients [B*T][NCS][DP]
-  float* sBv = sCf + nbt * NCS * DP;                      // b_t [B*T][DP]
-  float* sAgg = sBv + nbt * DP;                           // [P | q] per chunk [ntiles][DP*DP + DP]
-  float* sCar = sAgg + (size_t)ntiles * (DP * DP + DP);   // entering state per chunk [ntiles][DP]
+  float* sWf = smem_sm;                                  // W_q[i][k] at k * WR + q * DP + i
+  float* sWb = sWf + DP * WR;                            // the Jacobian's copy (band-masked)
+  float* sRed = sWb + DP * WR;                           // [NW]
+  float* sS0 = sRed + NW;                                // s0 [B][DP]
+  float* sU = sS0 + B * DP;                              // step inputs [b T + t][WR]
+  float* sS = sU + nbt * WR;                             // the iterate [row][DP], nrows rows
+  float* sCf = sS + nrows * DP;                          // coefficients [row][NCS][DP]
+  float* sBv = sCf + nrows * NCS * DP;                   // b_t [row][DP]
+  float* sAgg = sBv + nrows * DP;                        // [P | q] per chunk: P row-major, then q
+  float* sCar = sAgg + ntiles * (DP * DP + DP);          // entering state per chunk [ntiles][DP]
+  // row of step t of sequence b: chunk-interleaved
+  auto row_of = [&](int b, int t) { return (t % L) * ntiles + b * nch + t / L; };
 
   // ---- set-up: weights, s0 rows, the input projection, s^(0) = s0 --------------------------------
   for (int e = tid; e < DP * WR; e += NT) {
@@ -107,12 +127,12 @@ __global__ void __launch_bounds__(SmallCfg<CELL, DP>::NT, 1)
     const int b = e / DP, c = e % DP;
     sS0[e] = c < D ? __ldg(A.s0 + (size_t)b * D + c) : 0.0f;
   }
-  for (size_t e = tid; e < nbt * WR; e += NT) {
-    const size_t bt = e / WR;
-    const int qc = (int)(e % WR), q = qc / DP, c = qc % DP;
+  for (int e = tid; e < nbt * WR; e += NT) {
+    const int bt = e / WR;
+    const int qc = e % WR, q = qc / DP, c = qc % DP;
     float v = 0.0f;
     if (c < D) {
-      const float* xr = A.x + bt * d_in;
+      const float* xr = A.x + (size_t)bt * d_in;
       if constexpr (CELL == PN_CELL_EULER_TANH) {
         v = __ldg(xr + c);   // c_t = x_t (d_in = D)
       } else {
@@ -125,8 +145,9 @@ __global__ void __launch_bounds__(SmallCfg<CELL, DP>::NT, 1)
     sU[e] = v;
   }
   __syncthreads();
-  for (size_t e = tid; e < nbt * DP; e += NT) {
-    const int b = (int)(e / DP / T), c = (int)(e % DP);
+  for (int e = tid; e < nrows * DP; e += NT) {
+    const int r = e / DP, c = e % DP;
+    const int b = (r % ntiles) / nch;   // row -> chunk -> sequence
     sS[e] = round_storage(sS0[b * DP + c], sfmt);   // s^(0) in the storage format
   }
   const float* sWj = banded ? sWb : sWf;
@@ -137,11 +158,12 @@ __global__ void __launch_bounds__(SmallCfg<CELL, DP>::NT, 1)
   for (;; ++i) {
     // ---- 1. cell phase: one thread per (b, t, channel) -------------------------------------------
     unsigned rb = 0u;
-    for (size_t e = tid; e < nbt * DP; e += NT) {
-      const size_t bt = e / DP;
-      const int ci = (int)(e % DP);
-      const int t = (int)(bt % T), b = (int)(bt / T);
-      const float* sp = (t == 0) ? sS0 + b * DP : sS + (bt - 1) * DP;   // s^(i)_{t-1}
+    for (int e = tid; e < nbt * DP; e += NT) {
+      const int bt = e / DP;
+      const int ci = e % DP;
+      const int b = bt / T, t = bt - b * T;
+      const int row = row_of(b, t);
+      const float* sp = (t == 0) ? sS0 + b * DP : sS + row_of(b, t - 1) * DP;   // s^(i)_{t-1}
       float z[R], zb[R];
 #pragma unroll
       for (int q = 0; q < R; ++q) z[q] = zb[q] = 0.0f;
@@ -155,7 +177,7 @@ __global__ void __launch_bounds__(SmallCfg<CELL, DP>::NT, 1)
         }
       }
       const float spi = sp[ci];
-      const float sci = sS[bt * DP + ci];
+      const float sci = sS[row * DP + ci];
       const float* u = sU + bt * WR;
       float cf[NCS], bb, res;
       if constexpr (CELL == PN_CELL_TANH_RNN) {
@@ -196,8 +218,8 @@ __global__ void __launch_bounds__(SmallCfg<CELL, DP>::NT, 1)
         bb = 0.0f;
       }
 #pragma unroll
-      for (int q = 0; q < NCS; ++q) sCf[(bt * NCS + q) * DP + ci] = cf[q];
-      sBv[bt * DP + ci] = bb;
+      for (int q = 0; q < NCS; ++q) sCf[(row * NCS + q) * DP + ci] = cf[q];
+      sBv[row * DP + ci] = bb;
     }
     rb = warp_max_u32(rb);
     if (lane == 0) sRed[warp] = __uint_as_float(rb);
@@ -221,120 +243,131 @@ __global__ void __launch_bounds__(SmallCfg<CELL, DP>::NT, 1)
     const int fmt_new = (sfmt != 0 && (i == 0 || r_prev > A.store_until)) ? sfmt : 0;
     r_prev = s_r;
 
-    // ---- 2. chunk aggregates [P | q]: one warp per chunk -----------------------------------------
-    float* wP = sWarp + warp * (2 * DP * DP + 2 * DP);
-    float* wQ = wP + 2 * DP * DP;
-    for (int k = warp; k < ntiles; k += NW) {
+    // ---- 2. chunk aggregates, one thread per (chunk, column of [P | q]) --------------------------
+    for (int e = tid; e < ntiles * (DP + 1); e += NT) {
+      const int k = e / (DP + 1), j = e % (DP + 1);   // column j: P e_j for j < DP, q for j = DP
       const int b = k / nch, t0 = (k % nch) * L;
       const int n = min(L, T - t0);
-      const size_t bt0 = (size_t)b * T + t0;
-      {
-        const float* cf = sCf + bt0 * NCS * DP;
-        for (int e = lane; e < DP * DP; e += 32) {
-          const int ii = e / DP, j = e % DP;
-          float v = (ii == j) ? cf[ii] : 0.0f;
+      float x[DP];
+      {   // step 0: A_{t0} e_j, or b_{t0}
+        const float* cf = sCf + (size_t)k * NCS * DP;
 #pragma unroll
-          for (int q = 0; q < R; ++q) v = fmaf(cf[(1 + q) * DP + ii], sWj[j * WR + q * DP + ii], v);
-          wP[e] = v;
+        for (int ii = 0; ii < DP; ++ii) {
+          float v;
+          if (j < DP) {
+            v = (ii == j) ? cf[ii] : 0.0f;
+#pragma unroll
+            for (int q = 0; q < R; ++q) v = fmaf(cf[(1 + q) * DP + ii], sWj[j * WR + q * DP + ii], v);
+          } else {
+            v = sBv[k * DP + ii];
+          }
+          x[ii] = v;
         }
-        if (lane < DP) wQ[lane] = sBv[bt0 * DP + lane];
       }
-      __syncwarp();
-      int cur = 0;
       for (int m = 1; m < n; ++m) {
-        const float* cf = sCf + (bt0 + m) * NCS * DP;
-        const float* Pk = wP + cur * DP * DP;
-        float* Pn = wP + (cur ^ 1) * DP * DP;
-        for (int e = lane; e < DP * DP; e += 32) {
-          const int ii = e / DP, j = e % DP;
-          float v = cf[ii] * Pk[e];
+        const int row = m * ntiles + k;
+        float cf[NCS * DP], bv[DP];
+        lds_vec<NCS * DP>(sCf + (size_t)row * NCS * DP, cf);
+        lds_vec<DP>(sBv + row * DP, bv);
+        float y[DP];
+#pragma unroll
+        for (int ii = 0; ii < DP; ++ii) {
+          float v = cf[ii] * x[ii];
+          if (j == DP) v += bv[ii];
 #pragma unroll
           for (int q = 0; q < R; ++q) {
             float acc = 0.0f;
 #pragma unroll
-            for (int kk = 0; kk < DP; ++kk) acc = fmaf(sWj[kk * WR + q * DP + ii], Pk[kk * DP + j], acc);
+            for (int kk = 0; kk < DP; ++kk) acc = fmaf(sWj[kk * WR + q * DP + ii], x[kk], acc);
             v = fmaf(cf[(1 + q) * DP + ii], acc, v);
           }
-          Pn[e] = v;
+          y[ii] = v;
         }
-        if (lane < DP) {
-          const float* qk = wQ + cur * DP;
-          float v = fmaf(cf[lane], qk[lane], sBv[(bt0 + m) * DP + lane]);
+#pragma unroll
+        for (int ii = 0; ii < DP; ++ii) x[ii] = y[ii];
+      }
+      float* ag = sAgg + k * (DP * DP + DP);
+#pragma unroll
+      for (int ii = 0; ii < DP; ++ii) {
+        if (j < DP) ag[ii * DP + j] = x[ii];
+        else ag[DP * DP + ii] = x[ii];
+      }
+    }
+    __syncthreads();
+
+    // ---- 3a. entering state of every chunk: one thread per sequence, chunk after chunk -----------
+    for (int b = tid; b < B; b += NT) {
+      float carry[DP];
+#pragma unroll
+      for (int ii = 0; ii < DP; ++ii) carry[ii] = sS0[b * DP + ii];
+      for (int c = 0; c < nch; ++c) {
+        const int k = b * nch + c;
+        float ag[DP * DP + DP];
+        lds_vec<DP * DP + DP>(sAgg + k * (DP * DP + DP), ag);
+        float nxt[DP];
+#pragma unroll
+        for (int ii = 0; ii < DP; ++ii) {
+          sCar[k * DP + ii] = carry[ii];
+          float v = ag[DP * DP + ii];
+#pragma unroll
+          for (int jj = 0; jj < DP; ++jj) v = fmaf(ag[ii * DP + jj], carry[jj], v);
+          nxt[ii] = v;
+        }
+#pragma unroll
+        for (int ii = 0; ii < DP; ++ii) carry[ii] = nxt[ii];
+      }
+    }
+    __syncthreads();
+
+    // ---- 3b. apply: s_t = A_t s_{t-1} + b_t within each chunk, one thread per chunk, stored in place
+    for (int k = tid; k < ntiles; k += NT) {
+      const int t0 = (k % nch) * L;
+      const int n = min(L, T - t0);
+      float s[DP];
+#pragma unroll
+      for (int ii = 0; ii < DP; ++ii) s[ii] = sCar[k * DP + ii];
+      for (int m = 0; m < n; ++m) {
+        const int row = m * ntiles + k;
+        float cf[NCS * DP], bv[DP];
+        lds_vec<NCS * DP>(sCf + (size_t)row * NCS * DP, cf);
+        lds_vec<DP>(sBv + row * DP, bv);
+        float v[DP];
+#pragma unroll
+        for (int ii = 0; ii < DP; ++ii) {
+          float w = fmaf(cf[ii], s[ii], bv[ii]);
 #pragma unroll
           for (int q = 0; q < R; ++q) {
             float acc = 0.0f;
 #pragma unroll
-            for (int kk = 0; kk < DP; ++kk) acc = fmaf(sWj[kk * WR + q * DP + lane], qk[kk], acc);
-            v = fmaf(cf[(1 + q) * DP + lane], acc, v);
+            for (int kk = 0; kk < DP; ++kk) acc = fmaf(sWj[kk * WR + q * DP + ii], s[kk], acc);
+            w = fmaf(cf[(1 + q) * DP + ii], acc, w);
           }
-          wQ[(cur ^ 1) * DP + lane] = v;
+          v[ii] = w;
         }
-        __syncwarp();
-        cur ^= 1;
-      }
-      float* ag = sAgg + (size_t)k * (DP * DP + DP);
-      for (int e = lane; e < DP * DP; e += 32) ag[e] = wP[cur * DP * DP + e];
-      if (lane < DP) ag[DP * DP + lane] = wQ[cur * DP + lane];
-      __syncwarp();
-    }
-    __syncthreads();
-
-    // ---- 3a. entering state of every chunk: one warp per sequence, chunk after chunk -------------
-    for (int b = warp; b < B; b += NW) {
-      float carry = (lane < DP) ? sS0[b * DP + lane] : 0.0f;
-      for (int c = 0; c < nch; ++c) {
-        const int k = b * nch + c;
-        if (lane < DP) sCar[k * DP + lane] = carry;
-        const float* ag = sAgg + (size_t)k * (DP * DP + DP);
-        float v = (lane < DP) ? ag[DP * DP + lane] : 0.0f;
+        float* dst = sS + row * DP;
+        float old[DP];   // s^(i)_t
+        lds_vec<DP>(dst, old);
 #pragma unroll
-        for (int j = 0; j < DP; ++j) {
-          const float cj = __shfl_sync(0xffffffffu, carry, j);
-          if (lane < DP) v = fmaf(ag[lane * DP + j], cj, v);
+        for (int ii = 0; ii < DP; ii += 4) {
+          float4 o;
+          o.x = round_storage(damped ? fmaf(lambda, v[ii] - old[ii], old[ii]) : v[ii], fmt_new);
+          o.y = round_storage(damped ? fmaf(lambda, v[ii + 1] - old[ii + 1], old[ii + 1]) : v[ii + 1], fmt_new);
+          o.z = round_storage(damped ? fmaf(lambda, v[ii + 2] - old[ii + 2], old[ii + 2]) : v[ii + 2], fmt_new);
+          o.w = round_storage(damped ? fmaf(lambda, v[ii + 3] - old[ii + 3], old[ii + 3]) : v[ii + 3], fmt_new);
+          *reinterpret_cast<float4*>(dst + ii) = o;
         }
-        carry = v;
-      }
-    }
-    __syncthreads();
-
-    // ---- 3b. apply: s_t = A_t s_{t-1} + b_t within each chunk, stored in place -------------------
-    for (int k = warp; k < ntiles; k += NW) {
-      const int b = k / nch, t0 = (k % nch) * L;
-      const int n = min(L, T - t0);
-      const size_t bt0 = (size_t)b * T + t0;
-      float sprev = (lane < DP) ? sCar[k * DP + lane] : 0.0f;
-      for (int m = 0; m < n; ++m) {
-        const float* cf = sCf + (bt0 + m) * NCS * DP;
-        float acc[R];
 #pragma unroll
-        for (int q = 0; q < R; ++q) acc[q] = 0.0f;
-#pragma unroll
-        for (int kk = 0; kk < DP; ++kk) {
-          const float sk = __shfl_sync(0xffffffffu, sprev, kk);
-          if (lane < DP) {
-#pragma unroll
-            for (int q = 0; q < R; ++q) acc[q] = fmaf(sWj[kk * WR + q * DP + lane], sk, acc[q]);
-          }
-        }
-        float v = 0.0f;
-        if (lane < DP) {
-          v = fmaf(cf[lane], sprev, sBv[(bt0 + m) * DP + lane]);
-#pragma unroll
-          for (int q = 0; q < R; ++q) v = fmaf(cf[(1 + q) * DP + lane], acc[q], v);
-          float* dst = sS + (bt0 + m) * DP + lane;
-          const float old = *dst;   // s^(i)_t
-          *dst = round_storage(damped ? fmaf(lambda, v - old, old) : v, fmt_new);
-        }
-        sprev = v;
+        for (int ii = 0; ii < DP; ++ii) s[ii] = v[ii];   // the scan runs undamped and unrounded
       }
     }
     __syncthreads();
   }
 
   // ---- the result s^(i), and the control block as the multi-CTA loop leaves it -------------------
-  for (size_t e = tid; e < nbt * DP; e += NT) {
-    const int c = (int)(e % DP);
-    if (c < D) A.states[(e / DP) * D + c] = sS[e];
+  for (int e = tid; e < nbt * DP; e += NT) {
+    const int bt = e / DP, c = e % DP;
+    const int b = bt / T, t = bt - b * T;
+    if (c < D) A.states[(size_t)bt * D + c] = sS[row_of(b, t) * DP + c];
   }
   if (tid == 0) {
     ctrl->iter = i;
