@@ -129,10 +129,7 @@ __global__ void __launch_bounds__(128, 1) dense_tc_kernel(const IterParams P) {
     fence_async_smem();
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
-                 "r"((uint32_t)C::TCOLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tmem_alloc(&s_tmem, (uint32_t)C::TCOLS);
   }
   tc_fence_before();
   __syncthreads();
@@ -386,8 +383,7 @@ __global__ void __launch_bounds__(128, 1) dense_tc_kernel(const IterParams P) {
   __syncthreads();
   tc_fence_after();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::TCOLS)
-                 : "memory");
+    tmem_dealloc(tmem, (uint32_t)C::TCOLS);
   if (tid == 0) {
     unsigned v = 0u;
     for (int w = 0; w < 4; ++w) v = max(v, __float_as_uint(sRed[w]));

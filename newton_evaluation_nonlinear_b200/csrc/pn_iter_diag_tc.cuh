@@ -101,8 +101,24 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// The tcgen05 instructions below are warp-aligned (.sync.aligned): every thread of the warp must
+// execute them together, which inline asm does not tell the compiler, so each helper reconverges
+// the warp first (the code before it may have diverged, e.g. in a spin-wait).
+// Allocate `cols` TMEM columns for the CTA (one warp calls it; the base address lands in *dst).
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t cols) {
+  __syncwarp();
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst)), "r"(cols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+  __syncwarp();
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+
 // 16 consecutive fp32 columns of this warp's 32 TMEM lanes: thread i gets lane i.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  __syncwarp();
   uint32_t r[16];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
@@ -116,6 +132,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 // Store 16 fp32 columns into this warp's 32 TMEM lanes (thread i -> lane i).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  __syncwarp();
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
           taddr),
@@ -125,10 +142,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
       : "memory");
 }
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st_wait() {
+  __syncwarp();
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 // 32 consecutive fp32 columns of this warp's 32 TMEM lanes in one load (thread i gets lane i).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  __syncwarp();
   uint32_t r[32];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -145,6 +166,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 // Store 32 fp32 columns into this warp's 32 TMEM lanes (thread i -> lane i): a[16] then b[16].
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&a)[16], const float (&b)[16]) {
+  __syncwarp();
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
       "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
@@ -492,10 +514,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     fence_async_smem();   // the tensor cores read sBH/sBL through the async proxy
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
-                 "r"((uint32_t)C::ALLOC_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tmem_alloc(&s_tmem, (uint32_t)C::ALLOC_COLS);
   }
   tc_fence_before();
   __syncthreads();
@@ -1027,8 +1046,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   __syncthreads();
   tc_fence_after();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::ALLOC_COLS)
-                 : "memory");
+    tmem_dealloc(tmem, (uint32_t)C::ALLOC_COLS);
   if (tid == 0) {
     unsigned v = 0u;
     for (int w = 0; w < C::NT / 32; ++w) v = max(v, __float_as_uint(sRed[w]));

@@ -309,10 +309,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     for (int e = tid; e < DP; e += C::NT) sWd[e] = __ldg(P.wdiag + e);
     fence_async_smem();   // the tensor cores read sW through the async proxy
     if (warp == 0) {
-      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
-                   "r"((uint32_t)C::ALLOC_COLS)
-                   : "memory");
-      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+      tmem_alloc(&s_tmem, (uint32_t)C::ALLOC_COLS);
     }
   }
   tc_fence_before();
@@ -860,8 +857,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   __syncthreads();
   tc_fence_after();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(s_tmem), "r"((uint32_t)C::ALLOC_COLS)
-                 : "memory");
+    tmem_dealloc(s_tmem, (uint32_t)C::ALLOC_COLS);
   if (!P.persist) finish_launch(P, A, epoch, s_last);
 }
 

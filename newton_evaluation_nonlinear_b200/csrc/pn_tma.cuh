@@ -90,7 +90,10 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, unsign
 }
 
 // Named barrier over the first `nthreads` threads (a multiple of 32).
+// bar.sync is warp-aligned: every thread of a warp must reach it together, which inline asm does not
+// tell the compiler, so the warp is reconverged first (the code before a barrier may have diverged).
 __device__ __forceinline__ void named_barrier(unsigned id, unsigned nthreads) {
+  __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 

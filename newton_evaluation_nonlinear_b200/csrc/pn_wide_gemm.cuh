@@ -105,10 +105,7 @@ __global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __
     s_issued = 0;
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
-                 "r"((uint32_t)C::TCOLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tmem_alloc(&s_tmem, (uint32_t)C::TCOLS);
   }
   tc_fence_before();
   __syncthreads();
@@ -234,8 +231,7 @@ __global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __
   __syncthreads();
   tc_fence_after();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::TCOLS)
-                 : "memory");
+    tmem_dealloc(tmem, (uint32_t)C::TCOLS);
 }
 
 }  // namespace pn
