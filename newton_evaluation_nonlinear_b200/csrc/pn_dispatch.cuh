@@ -97,7 +97,8 @@ inline KInfo diag_tma_pick() {
 template <int CELL, int MODE, int DP>
 inline KInfo diag_tc_kinfo() {
   using C = DiagTcCfg<CELL, MODE, DP>;
-  return KInfo{(const void*)&diag_tc_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTc};
+  return KInfo{(const void*)&diag_tc_kernel<CELL, MODE, DP>, C::NT, C::L, DP, (size_t)C::SMEM_BYTES, kKindDiagTc,
+               true};
 }
 
 // Channel-major tensor-core variant for the one-gate cells: D == DP in {32, 64}.

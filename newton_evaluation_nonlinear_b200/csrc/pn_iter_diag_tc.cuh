@@ -458,8 +458,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   const size_t stride = (size_t)B;   // one channel group: consecutive chunks are B tickets apart
   const long long tmo = A.timeout_ns;
 
-  if (tid == 0) {
-    atomicMin(&ctrl->t_start, globaltimer());
+  auto init_barriers = [&]() {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_sfull[s], 1u);
       mbar_init(&bar_sempty[s], (unsigned)C::NEW);
@@ -477,10 +476,42 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     mbar_init(&bar_ofull, (unsigned)C::NEW);
     mbar_init(&bar_oempty, 1u);
     mbar_init_fence();
+  };
+  auto inval_barriers = [&]() {
+    for (int s = 0; s < 2; ++s) {
+      mbar_inval(&bar_sfull[s]);
+      mbar_inval(&bar_sempty[s]);
+      mbar_inval(&bar_mma[s]);
+      mbar_inval(&bar_tempty[s]);
+    }
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_inval(&bar_lb[s]);
+      mbar_inval(&bar_cfull[s]);
+      mbar_inval(&bar_cempty[s]);
+    }
+    mbar_inval(&bar_xfull);
+    mbar_inval(&bar_xempty);
+    mbar_inval(&bar_afull);
+    mbar_inval(&bar_ofull);
+    mbar_inval(&bar_oempty);
+  };
+  // iteration and look-back epoch of this launch's first iteration; with P.persist each further
+  // iteration of the launch (one round of the loop below, after the grid barrier) adds one to both
+  const unsigned gen0 = *(volatile unsigned*)&ctrl->gen;
+  const unsigned epoch0 = *(volatile unsigned*)&ctrl->epoch;
+  const int iter0 = *(volatile int*)&ctrl->iter;
+  unsigned epoch = epoch0;
+  uint32_t tmem = 0u;
+  for (int round = 0;; ++round) {
+  if (tid == 0) {
+    if (round == 0) {
+      atomicMin(&ctrl->t_start, globaltimer());
+      init_barriers();   // later rounds: re-initialised at the end of the previous one
+    }
     s_abort = 0;
   }
-  const unsigned epoch = *(volatile unsigned*)&ctrl->epoch;
-  const int iter = *(volatile int*)&ctrl->iter;
+  epoch = epoch0 + (unsigned)round;
+  const int iter = iter0 + round;
   if (tid == 0) {
     // The first tile of every CTA has a static ticket (blockIdx.x < tiles: the grid is never
     // larger) and is fetched right away, overlapping the weight load and TMEM set-up below.
@@ -488,6 +519,9 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     const CUtensorMap* tm_x = P.tmaps + 2;
     tmap_acquire(tm_s);
     tmap_acquire(tm_x);
+    // the last round's states (other CTAs' stores, ordered before the grid barrier) are read by
+    // the tensor-copy loads below
+    asm volatile("fence.proxy.async.global;" ::: "memory");
     const int kg = (int)blockIdx.x;
     if (kg < P.tiles_per_group) {
       const int b = kg % B;
@@ -505,7 +539,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   }
 
   // weights: W_hi and W_lo in the K-major core-matrix layout (pre-packed), diagonals, b_hn
-  {
+  if (round == 0) {
     const float4* w4 = reinterpret_cast<const float4*>(P.wt);
     float4* d4 = reinterpret_cast<float4*>(sBH);   // sBH and sBL are contiguous
     for (int e = tid; e < 2 * C::B_BYTES / 16; e += C::NT) d4[e] = __ldg(w4 + e);
@@ -513,13 +547,13 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     for (int e = tid; e < DP; e += C::NT) sBhn[e] = (CELL == PN_CELL_GRU) ? __ldg(P.bhn + e) : 0.0f;
     fence_async_smem();   // the tensor cores read sBH/sBL through the async proxy
   }
-  if (warp == 0) {
+  if (warp == 0 && round == 0) {
     tmem_alloc(&s_tmem, (uint32_t)C::ALLOC_COLS);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = s_tmem;
+  tmem = s_tmem;
 
   unsigned rbits = 0u;
 
@@ -638,6 +672,12 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     // the remaining output tiles, up to the stop marker
     for (int j = nstored;; ++j)
       if (!store_tile(j)) break;
+    // the stored states are in global memory, ordered before this CTA's part of the grid barrier
+    if (lane == 0) {
+      bulk_wait_all();
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    __syncwarp();
     if (lane == 0) bulk_wait_all();   // the states are in global memory before the CTA retires
   } else if (warp < C::WE0) {
     // =========================== look-back ==================================
@@ -1039,20 +1079,32 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     }
   }
 
-  // ---- residual, TMEM release, end-of-launch decision ------------------------
+  // ---- residual of this iteration; the next one (grid barrier) or the end of the launch
   rbits = warp_max_u32(rbits);
   if (lane == 0) sRed[warp] = __uint_as_float(rbits);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0)
-    tmem_dealloc(tmem, (uint32_t)C::ALLOC_COLS);
   if (tid == 0) {
     unsigned v = 0u;
     for (int w = 0; w < C::NT / 32; ++w) v = max(v, __float_as_uint(sRed[w]));
     if (v) atomicMax(&ctrl->resid_bits, v);
   }
-  finish_launch(P, A, epoch, s_last);
+  if (!P.persist) break;
+  // fresh barriers for the next round (every operation on the old ones has completed)
+  if (tid == 0) {
+    inval_barriers();
+    init_barriers();
+  }
+  if (!finish_iteration(P, A, iter, epoch, s_last, (gen0 >> 1) + (unsigned)round)) break;
+  }   // rounds
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    tmem_dealloc(tmem, (uint32_t)C::ALLOC_COLS);
+  if (!P.persist) finish_launch(P, A, epoch, s_last);
 }
 
 }  // namespace pn
