@@ -24,8 +24,8 @@
 // The 8 sixteen-step pieces of a channel are combined through shared memory;
 // the piece prefix (PA, PB) stays in registers, the in-piece prefixes are
 // parked in TMEM, and the states are formed three tiles later from the carry
-// of the look-back warps, staged in the step-input buffer the tile has
-// consumed and written by one TMA tensor store from the producer warp.
+// of the look-back warps and stored to global memory by the epilogue threads
+// themselves (each warp store instruction covers two 64-byte row segments).
 //
 // With P.persist = 1 the kernel runs the whole fixed-point loop in one launch:
 // after each iteration the CTAs meet at a bounded grid barrier whose last
@@ -35,7 +35,7 @@
 // The step inputs are double-buffered with the S stages and released with
 // them, so both are fetched two tiles ahead of their use.
 //
-// Warp roles (one CTA per SM): 0 producer (tickets, TMA loads and state stores); 1 MMA issuer;
+// Warp roles (one CTA per SM): 0 producer (tickets and TMA loads); 1 MMA issuer;
 // 2-3 look-back (scan modes, alternate tiles); the rest epilogue (4 TMEM lane
 // quarters x RS / 16 step groups).  The epilogue forms the next tile's S_lo
 // right after the current tile's cell phase, so the tensor cores compute the
@@ -193,13 +193,11 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   float* sCarry = reinterpret_cast<float*>(smem_raw + C::OFF_CARRY);
   float* sRed = reinterpret_cast<float*>(smem_raw + C::OFF_RED);
 
-  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull[2], bar_ofull[2], bar_oempty[2], bar_afull,
-      bar_mma[2],
-      bar_tempty[2], bar_lb[C::NAG], bar_cfull[NSLOT], bar_cempty[NSLOT];
+  __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2], bar_xfull[2], bar_afull, bar_mma[2], bar_tempty[2],
+      bar_lb[C::NAG], bar_cfull[NSLOT], bar_cempty[NSLOT];
   __shared__ int s_tk[2];        // ticket staged in s stage 0/1 (-1: no more tiles)
   __shared__ int s_atk[2];       // ticket of tile i's operands, by the parity of i (-1: stop)
   __shared__ int s_lbtk[C::NAG];  // ticket handed to the look-back per slot (-1: stop)
-  __shared__ int s_otk[2];        // ticket of the states staged in step-input buffer i (-1: none)
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ int s_last;
@@ -222,8 +220,6 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_sfull[s], 1u);
       mbar_init(&bar_xfull[s], 1u);
-      mbar_init(&bar_ofull[s], (unsigned)C::NEW);
-      mbar_init(&bar_oempty[s], 1u);
       mbar_init(&bar_sempty[s], (unsigned)C::NEW);
       mbar_init(&bar_mma[s], 1u);
       mbar_init(&bar_tempty[s], (unsigned)C::NEW);
@@ -238,8 +234,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   };
   auto inval_barriers = [&]() {
     uint64_t* bars[] = {&bar_sfull[0], &bar_sfull[1], &bar_sempty[0], &bar_sempty[1], &bar_mma[0], &bar_mma[1],
-                        &bar_tempty[0], &bar_tempty[1], &bar_xfull[0], &bar_xfull[1], &bar_ofull[0],
-                        &bar_ofull[1], &bar_oempty[0], &bar_oempty[1], &bar_afull};
+                        &bar_tempty[0], &bar_tempty[1], &bar_xfull[0], &bar_xfull[1], &bar_afull};
     for (uint64_t* bb : bars) mbar_inval(bb);
     for (int s = 0; s < C::NAG; ++s) mbar_inval(&bar_lb[s]);
     for (int s = 0; s < NSLOT; ++s) {
@@ -271,8 +266,8 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     const CUtensorMap* tm_x = P.tmaps + 2;
     tmap_acquire(tm_s);
     tmap_acquire(tm_x);
-    // the last iteration's states (other CTAs' stores, ordered before the grid barrier) are
-    // read by the tensor-copy loads below
+    // the last iteration's states (other CTAs' generic stores, ordered before the grid barrier)
+    // are read by this thread's tensor-copy loads, here and for every later tile of the iteration
     asm volatile("fence.proxy.async.global;" ::: "memory");
     const int kg = (int)blockIdx.x;
     if (kg < P.tiles_per_group) {
@@ -323,40 +318,17 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     // =========================== producer ===================================
     const CUtensorMap* tm_s = P.tmaps + ((iter & 1) ? 1 : 0);   // s^(i)
     const CUtensorMap* tm_x = P.tmaps + 2;                      // step inputs
-    const CUtensorMap* tm_o = P.tmaps + ((iter & 1) ? 3 : 4);   // s^(i+1), into the other buffer
-    if (lane == 0) tmap_acquire(tm_o);
     // the step inputs are read by every iteration: kept in L2 ahead of the iterates, read once each
     const uint64_t pol_keep = l2_policy_evict_last();
     const uint64_t pol_stream = l2_policy_evict_first();
-    // The states the epilogue staged at its event e (one event per tile, and three more for the
-    // last write-outs) in step-input buffer e & 1: one tensor store, and a wait until it has
-    // read the buffer, which is then free again (for tile e + 2's step inputs, or, signalled on
-    // bar_oempty, for the epilogue's last events).
-    int n_served = 0;
-    auto serve = [&](int e) -> bool {
-      if (!mbar_wait_flag(&bar_ofull[e & 1], ((unsigned)e >> 1) & 1u, ctrl, tmo, &s_abort, 101)) return false;
-      if (lane == 0) {
-        const int ko = s_otk[e & 1];
-        if (ko >= 0) {
-          tma_store_3d(tm_o, 0, (ko / B) * L, ko % B, smem_raw + C::OFF_X + (e & 1) * C::X_BYTES);
-          bulk_commit();
-          bulk_wait_read();
-        }
-        mbar_arrive(&bar_oempty[e & 1]);
-      }
-      __syncwarp();
-      n_served = e + 1;
-      return true;
-    };
     // tile 0 was issued before the block-wide sync (static ticket blockIdx.x)
     const bool none = (int)blockIdx.x >= P.tiles_per_group;
     int it = 1;
-    int n_tiles = none ? 0 : 1;    // tiles claimed (their S loads issued)
-    int n_loaded = none ? 0 : 1;   // of them, with their step inputs issued too
+    int n_loaded = none ? 0 : 1;   // stages with their S and step-input loads issued
     for (; !none; ++it) {
       const int st = it & 1;
-      // stage st's S buffer is free once tile it-2's cell phase is done; the ticket is claimed
-      // only then, so a CTA holds no ticket it cannot start loading
+      // stage st (S and step inputs) is free once tile it-2's cell phase is done; the ticket is
+      // claimed only then, so a CTA holds no ticket it cannot start loading
       if (it >= 2 && !mbar_wait_flag(&bar_sempty[st], (((unsigned)it >> 1) & 1u) ^ 1u, ctrl, tmo, &s_abort, 102)) break;
       int kg = 0;
       if (lane == 0) kg = (int)(gridDim.x + atomicAdd(&ctrl->ticket[0], 1u));
@@ -378,37 +350,20 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
 #pragma unroll
         for (int h = 0; h < NKH; ++h)
           tma_load_3d_hint(sS + (st * NKH + h) * C::SH_BYTES, tm_s, 32 * h, t0 - 1, b, &bar_sfull[st], pol_stream);
-      }
-      __syncwarp();
-      n_tiles = it + 1;
-      // step-input buffer st: free once the states tile it-2's epilogue staged there are read
-      if (it >= 2 && !serve(it - 2)) {
-        ++it;
-        break;
-      }
-      if (lane == 0) {
         mbar_arrive_expect_tx(&bar_xfull[st], (unsigned)C::X_BYTES);
         tma_load_3d_hint(smem_raw + C::OFF_X + st * C::X_BYTES, tm_x, 0, t0, b, &bar_xfull[st], pol_keep);
       }
       __syncwarp();
       n_loaded = it + 1;
     }
-    // the remaining events: the last tiles', and three more for the last write-outs
-    for (int e = n_served; e < n_tiles + (kScan ? C::DEFER : 0) && !s_abort; ++e)
-      if (!serve(e)) break;
-    // the last two stages' loads (and the stop marker) complete before the CTA moves on
+    // the last two stages' loads (and the stop marker, which has no step-input load) complete
+    // before the CTA moves on
     for (int j = max(0, it - 2); j < it; ++j)
       if (!mbar_drain(&bar_sfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
         atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
     for (int j = max(0, n_loaded - 2); j < n_loaded; ++j)
       if (!mbar_drain(&bar_xfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
         atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
-    // the stored states are in global memory, ordered before this CTA's part of the grid barrier
-    if (lane == 0) {
-      bulk_wait_all();
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-    }
-    __syncwarp();
   } else if (warp == 1) {
     // =========================== MMA issuer =================================
     constexpr uint32_t idesc = umma_idesc_tf32(C::MT, RS);
@@ -608,18 +563,20 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       }
     };
 
-    // s^(i+1) of tile j: piece carry from the look-back carry, then the parked prefixes (the
-    // stash holds [A 0-7 | B 0-7 | A 8-15 | B 8-15] per 16 steps; B only for Picard), staged for
-    // the producer's tensor store in step-input buffer `stg` (whose inputs every epilogue warp
-    // has consumed), eight steps at a time
-    auto stage_out = [&](int j, float pa, float pb, int stg) {
+    // s^(i+1) of tile j (ticket kj): piece carry from the look-back carry, then the parked
+    // prefixes (the stash holds [A 0-7 | B 0-7 | A 8-15 | B 8-15] per 16 steps; B only for
+    // Picard), stored eight steps at a time.  The rows are D = DP floats apart (the kernel runs
+    // only with D == DP); steps past T are not stored.
+    auto stage_out = [&](int j, float pa, float pb, int kj) {
       const int slot = j % NSLOT;
       mbar_wait_flag(&bar_cfull[slot], (unsigned)(j / NSLOT) & 1u, ctrl, tmo, &s_abort, 110);
       const float carry = sCarry[slot * DP + c];
       // Picard parks only B: its damped A_t = lambda enters here
       const float cp = kHasA ? fmaf(pa, carry, pb) : (carry + pb) * lambda;
       const uint32_t sbase = tmem + (uint32_t)(C::STASH0 + slot * C::SCOLS + (kHasA ? 32 : 16) * rg) + lane_off;
-      float* xo = reinterpret_cast<float*>(smem_raw + C::OFF_X + stg * C::X_BYTES) + row0 * DP + c;
+      const int tj = (kj / B) * L + row0;   // this thread's first step of tile j
+      float* o = dst + ((size_t)(kj % B) * T + tj) * DP + c;
+      const bool fullj = tj + 16 <= T;
 #pragma unroll
       for (int h8 = 0; h8 < (kHasA ? 2 : 1); ++h8) {
         float v[16];   // quasi: A then B of steps 8 h8 .. 8 h8 + 7; Picard: B of all 16 steps
@@ -627,10 +584,9 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
 #pragma unroll
         for (int i = 0; i < (kHasA ? 8 : 16); ++i) {
           const int ii = (kHasA ? 8 * h8 : 0) + i;
-          xo[ii * DP] = kHasA ? fmaf(v[i], cp, v[8 + i]) : cp + v[i];
+          if (fullj || tj + ii < T) o[(size_t)ii * DP] = kHasA ? fmaf(v[i], cp, v[8 + i]) : cp + v[i];
         }
       }
-      fence_async_smem();   // generic writes -> the tensor store (async proxy)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_cempty[slot]);
     };
@@ -733,9 +689,6 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
             if (t0 + row0 + i < T) o[(size_t)i * D] = bv[i];
         }
         named_barrier(1, NTE);   // the ticket of tile it+1
-        if (te == 0) s_otk[st] = -1;   // nothing staged: the step-input buffer is free
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_ofull[st]);
         kg = s_atk[(it + 1) & 1];
       } else {
         // ---- combine the 8 pieces of each channel
@@ -767,13 +720,9 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
             mbar_arrive(&bar_lb[aslot]);
           }
         }
-        // the states of tile it-3 (its carry had three tiles of time to arrive), staged in this
-        // tile's step-input buffer for the producer's tensor store; this frees the stash slot
-        // this tile's prefixes take
-        if (it >= C::DEFER) stage_out(it - C::DEFER, pa3, pb3, st);
-        if (te == 0) s_otk[st] = (it >= C::DEFER && !s_abort) ? kg_m3 : -1;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_ofull[st]);
+        // the states of tile it-3 (its carry had three tiles of time to arrive); this frees the
+        // stash slot this tile's prefixes take
+        if (it >= C::DEFER) stage_out(it - C::DEFER, pa3, pb3, kg_m3);
         // ---- park the in-piece prefixes in TMEM
         {
           const uint32_t sbase =
@@ -795,23 +744,18 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
       }
     }
     if constexpr (kScan) {
-      // the last three tiles' states: events it .. it+2, each in the step-input buffer of its
-      // parity once the store of the event two before has read that buffer (a loop, not unrolled:
-      // one copy of the write-out code serves it, which keeps the epilogue's code smaller)
+      // the last three tiles' states (a loop, not unrolled: one copy of the write-out code
+      // serves it, which keeps the epilogue's code smaller)
 #pragma unroll 1
       for (int j = 0; j < C::DEFER; ++j) {
-        const int ev = it + j;
-        const int tj = ev - C::DEFER;
-        const int st = ev & 1;
-        if (ev >= 2) mbar_wait_flag(&bar_oempty[st], ((unsigned)(ev - 2) >> 1) & 1u, ctrl, tmo, &s_abort, 113);
+        const int tj = it + j - C::DEFER;
         const int kj = (j == 0) ? kg_m3 : (j == 1 ? kg_m2 : kg_m1);
         const float pa = (j == 0) ? pa3 : (j == 1 ? pa2 : pa1);
         const float pb = (j == 0) ? pb3 : (j == 1 ? pb2 : pb1);
-        if (tj >= 0) stage_out(tj, pa, pb, st);
-        if (te == 0) s_otk[st] = (tj >= 0 && !s_abort) ? kj : -1;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_ofull[st]);
+        if (tj >= 0) stage_out(tj, pa, pb, kj);
       }
+      // the next iteration reads these states with tensor copies (async proxy) after the grid barrier
+      asm volatile("fence.proxy.async.global;" ::: "memory");
       // stop the look-back warps: their next tiles are it .. it + NLB - 1
       if (lastw && lane == 0) {
         for (int j = it; j < it + C::NLB; ++j) {
