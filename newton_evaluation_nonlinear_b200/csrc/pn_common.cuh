@@ -49,7 +49,28 @@ struct Ctrl {
   alignas(128) unsigned resid_bits;  // running max of |F| for the current launch (float bits)
   unsigned done;       // CTAs finished in the current launch
   unsigned gen;        // grid barrier of the looping kernels: (iterations completed << 1) | (another follows)
+  // Arrivals at the grid barrier of the looping kernels, with the stop rule's inputs packed in
+  // (kArrive* below), and their residual maxima by iteration parity.
+  alignas(128) unsigned long long arrive;
+  unsigned resid_loop[2];
 };
+
+// Fields of Ctrl::arrive, each a count of CTAs (at most 2^20 - 1): arrived, with a residual
+// above tol (or NaN), with a non-finite residual; the top field counts raised errors.
+constexpr unsigned long long kArriveOne = 1ull;
+constexpr unsigned long long kArriveHot = 1ull << 20;
+constexpr unsigned long long kArriveBad = 1ull << 40;
+constexpr unsigned long long kArriveErr = 1ull << 60;
+constexpr unsigned long long kArriveMask = (1ull << 20) - 1ull;
+
+// Sets the sticky device error unless one is set already; the first raise also counts itself in
+// Ctrl::arrive, so the grid barrier's last arrival learns of it from the value its own atomic
+// returns (the raising CTA arrives only after the raise).  Returns whether this call set it.
+__device__ __forceinline__ bool raise_error(Ctrl* c, int code) {
+  if (atomicCAS(&c->error, 0, code) != 0) return false;
+  atomicAdd(&c->arrive, kArriveErr);
+  return true;
+}
 
 // Per-call arguments, written by the host before each evaluation.
 struct Args {
@@ -200,7 +221,7 @@ __device__ __forceinline__ int lookback_find_prefix(const unsigned* flags, size_
       if (lane == 0) {
         if (ld_volatile(&ctrl->error)) give_up = 1;
         else if ((long long)(globaltimer() - t0) > timeout_ns) {
-          if (atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT) == 0) ctrl->timeout_ticket = (int)k;
+          if (raise_error(ctrl, (int)PN_ERR_TIMEOUT)) ctrl->timeout_ticket = (int)k;
           give_up = 1;
         }
       }
@@ -245,7 +266,7 @@ __device__ __forceinline__ int lookback_nearest_state(const unsigned* flags, siz
       if (lane == 0) {
         if (ld_volatile(&ctrl->error)) give_up = 1;
         else if ((long long)(globaltimer() - t0) > timeout_ns) {
-          if (atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT) == 0) ctrl->timeout_ticket = (int)k;
+          if (raise_error(ctrl, (int)PN_ERR_TIMEOUT)) ctrl->timeout_ticket = (int)k;
           give_up = 1;
         }
       }
@@ -385,37 +406,54 @@ __device__ __forceinline__ void finish_launch(const IterParams& P, const Args& A
 }
 
 // Grid barrier between the iterations of a looping kernel.  Every CTA calls
-// it (all threads) after its part of the iteration, after all of its global
-// writes and with its residual folded into ctrl->resid_bits.  The last CTA to
-// arrive applies the stop rule exactly as finish_launch does (iteration `iter`,
-// look-back epoch `epoch`) and publishes the next generation of ctrl->gen
-// together with the decision in its low bit, so the other CTAs learn both from
-// the one word they wait on.  `gen_count` is the number of iterations this
-// handle completed before this one.  Returns, for every thread of the CTA,
-// whether another iteration follows (its iteration and epoch are one more).
+// it (all threads) after its part of the iteration and after all of its global
+// writes; `rbits` is the CTA's residual maximum (float bits, read on thread 0).
+// The last CTA to arrive applies the stop rule of finish_launch (iteration
+// `iter`, look-back epoch `epoch`) and publishes the next generation of
+// ctrl->gen together with the decision in its low bit, so the other CTAs learn
+// both from the one word they wait on.  `gen_count` is the number of
+// iterations this handle completed before this one.  Returns, for every thread
+// of the CTA, whether another iteration follows (its iteration and epoch are
+// one more).
+//
+// The decision needs no read after the arrival: each CTA adds to ctrl->arrive
+// its arrival, whether its residual is above tol (or NaN) and whether it is
+// non-finite, and every error raised counted itself there too, so the value
+// the last arrival's atomic returns holds the whole rule (r <= tol exactly when
+// no CTA's maximum is above it).  The residual value itself, for the history
+// and the result, is read by the last CTA after the release, from the word of
+// this iteration's parity, which it then clears for iteration iter + 2.
 __device__ __forceinline__ bool finish_iteration(const IterParams& P, const Args& A, int iter, unsigned epoch,
-                                                 int& flag_smem, unsigned gen_count) {
+                                                 int& flag_smem, unsigned gen_count, unsigned rbits) {
   __syncthreads();
   if (threadIdx.x == 0) {
     Ctrl* c = P.ctrl;
+    unsigned* rw = &c->resid_loop[iter & 1];
+    if (rbits) atomicMax(rw, rbits);
+    unsigned long long mine = kArriveOne;
+    if (__uint_as_float(rbits) > A.tol || rbits > 0x7f800000u) mine += kArriveHot;
+    if (rbits >= 0x7f800000u) mine += kArriveBad;
     __threadfence();
-    const unsigned prev = atomicAdd(&c->done, 1u);
+    const unsigned long long prev = atomicAdd(&c->arrive, mine);
     int go = 0;
-    if (prev == gridDim.x - 1) {
+    if ((prev & kArriveMask) == (unsigned long long)(gridDim.x - 1)) {
+      const unsigned long long tot = prev + mine;
       __threadfence();
-      const float r = __uint_as_float(atomicAdd(&c->resid_bits, 0u));
-      const int err = ld_volatile(&c->error);
-      if (iter < kHistCap) P.hist[iter] = r;
       int st = kRunning;
-      if (err) st = err;
-      else if (!(r <= 3.402823466e38f)) st = PN_ERR_NONFINITE;
-      else if (r <= A.tol) st = PN_OK;
-      else if (iter >= A.max_iters) st = PN_NOT_CONVERGED;
+      if (tot >> 60) {
+        st = ld_volatile(&c->error);
+        if (!st) st = PN_ERR_TIMEOUT;
+      } else if ((tot >> 40) & kArriveMask) {
+        st = PN_ERR_NONFINITE;
+      } else if (((tot >> 20) & kArriveMask) == 0ull) {
+        st = PN_OK;
+      } else if (iter >= A.max_iters) {
+        st = PN_NOT_CONVERGED;
+      }
       c->launches += 1ull;
       if (st != kRunning) {
         c->status = st;
         c->final_iter = iter;
-        c->final_resid = r;
         c->final_fmt = c->fmt_in;
         const unsigned long long t1 = globaltimer();
         const unsigned long long t0 = c->t_start;
@@ -424,23 +462,28 @@ __device__ __forceinline__ bool finish_iteration(const IterParams& P, const Args
       } else {
         c->iter = iter + 1;
         c->fmt_in = c->fmt_out;
-        c->fmt_out = (A.store_fmt != 0 && r > A.store_until) ? 1 : 0;
+        // narrow storage (not run by the looping kernels today) needs the value before the release
+        c->fmt_out = (A.store_fmt != 0 && __uint_as_float(atomicAdd(rw, 0u)) > A.store_until) ? 1 : 0;
         go = 1;
       }
-      c->resid_bits = 0u;
 #pragma unroll
       for (int g = 0; g < kMaxGroups; ++g) c->ticket[g] = 0u;
-      c->done = 0u;
+      c->arrive = 0ull;
       c->epoch = epoch + 1u;
       __threadfence();
       st_release(&c->gen, ((gen_count + 1u) << 1) | (unsigned)go);
+      // off the other CTAs' path: the residual of this iteration (every CTA folded its maximum
+      // in before arriving), and its word cleared for iteration iter + 2
+      const float r = __uint_as_float(atomicExch(rw, 0u));
+      if (iter < kHistCap) P.hist[iter] = r;
+      if (st != kRunning) c->final_resid = r;
     } else {
       const unsigned long long t0 = globaltimer();
       unsigned spins = 0;
       unsigned g;
       while (((g = ld_acquire(&c->gen)) >> 1) == (gen_count & 0x7fffffffu)) {
         if (((++spins) & 15u) == 0u && (long long)(globaltimer() - t0) > A.timeout_ns) {
-          atomicCAS(&c->error, 0, (int)PN_ERR_TIMEOUT);
+          raise_error(c, (int)PN_ERR_TIMEOUT);
           break;
         }
         if (spins > 64u) __nanosleep(64);

@@ -630,13 +630,13 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
   rbits = warp_max_u32(rbits);
   if (lane == 0) sRed[warp] = __uint_as_float(rbits);
   __syncthreads();
+  unsigned rmax = 0u;   // the CTA's residual maximum, on thread 0
   if (tid == 0) {
-    unsigned v = 0u;
-    for (int w = 0; w < NWARP; ++w) v = max(v, __float_as_uint(sRed[w]));
-    if (v) atomicMax(&ctrl->resid_bits, v);
+    for (int w = 0; w < NWARP; ++w) rmax = max(rmax, __float_as_uint(sRed[w]));
+    if (rmax && !P.persist) atomicMax(&ctrl->resid_bits, rmax);
   }
   if (!P.persist) break;
-  if (!finish_iteration(P, A, iter, epoch, s_last, (gen0 >> 1) + (unsigned)round)) break;
+  if (!finish_iteration(P, A, iter, epoch, s_last, (gen0 >> 1) + (unsigned)round, rmax)) break;
   }   // iterations
   if (!P.persist) finish_launch(P, A, epoch, s_last);
 }

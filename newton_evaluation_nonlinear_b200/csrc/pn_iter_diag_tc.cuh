@@ -269,7 +269,7 @@ __device__ __forceinline__ bool mbar_wait_flag(uint64_t* bar, unsigned parity, C
         return false;
       }
       if ((long long)(globaltimer() - t0) > timeout_ns) {
-        if (atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT) == 0 && site > 0) ctrl->timeout_ticket = -site;
+        if (raise_error(ctrl, (int)PN_ERR_TIMEOUT) && site > 0) ctrl->timeout_ticket = -site;
         *abort = 1;
         return false;
       }
@@ -288,7 +288,7 @@ __device__ __forceinline__ bool spin_give_up(unsigned& spins, unsigned long long
   if ((++spins & 15u) == 0u && (threadIdx.x & 31) == 0) {
     if (ld_volatile(&ctrl->error)) g = 1;
     else if ((long long)(globaltimer() - t0) > timeout_ns) {
-      atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+      raise_error(ctrl, (int)PN_ERR_TIMEOUT);
       g = 1;
     }
   }
@@ -603,9 +603,9 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     // drain every fill this warp issued
     for (int j = max(0, it - 2); j < it; ++j)
       if (!mbar_drain(&bar_sfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
-        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+        raise_error(ctrl, (int)PN_ERR_TIMEOUT);
     if (x_issued > 0 && !mbar_drain(&bar_xfull, ((unsigned)(x_issued - 1)) & 1u, tmo) && lane == 0)
-      atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+      raise_error(ctrl, (int)PN_ERR_TIMEOUT);
   } else if (warp == 1) {
     // ======================= MMA and store issuer ============================
     constexpr uint32_t idesc = umma_idesc_tf32(L, N);
@@ -668,7 +668,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     // every issued product must have completed before TMEM is released
     for (int j = max(0, issued - 2); j < issued; ++j)
       if (!mbar_drain(&bar_mma[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
-        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+        raise_error(ctrl, (int)PN_ERR_TIMEOUT);
     // the remaining output tiles, up to the stop marker
     for (int j = nstored;; ++j)
       if (!store_tile(j)) break;
@@ -1085,10 +1085,10 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  unsigned rmax = 0u;   // the CTA's residual maximum, on thread 0
   if (tid == 0) {
-    unsigned v = 0u;
-    for (int w = 0; w < C::NT / 32; ++w) v = max(v, __float_as_uint(sRed[w]));
-    if (v) atomicMax(&ctrl->resid_bits, v);
+    for (int w = 0; w < C::NT / 32; ++w) rmax = max(rmax, __float_as_uint(sRed[w]));
+    if (rmax && !P.persist) atomicMax(&ctrl->resid_bits, rmax);
   }
   if (!P.persist) break;
   // fresh barriers for the next round (every operation on the old ones has completed)
@@ -1096,7 +1096,7 @@ __global__ void __launch_bounds__(DiagTcCfg<CELL, MODE, DP>::NT, 1) diag_tc_kern
     inval_barriers();
     init_barriers();
   }
-  if (!finish_iteration(P, A, iter, epoch, s_last, (gen0 >> 1) + (unsigned)round)) break;
+  if (!finish_iteration(P, A, iter, epoch, s_last, (gen0 >> 1) + (unsigned)round, rmax)) break;
   }   // rounds
 
   tc_fence_before();

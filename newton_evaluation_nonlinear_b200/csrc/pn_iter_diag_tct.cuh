@@ -360,10 +360,10 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     // before the CTA moves on
     for (int j = max(0, it - 2); j < it; ++j)
       if (!mbar_drain(&bar_sfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
-        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+        raise_error(ctrl, (int)PN_ERR_TIMEOUT);
     for (int j = max(0, n_loaded - 2); j < n_loaded; ++j)
       if (!mbar_drain(&bar_xfull[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
-        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+        raise_error(ctrl, (int)PN_ERR_TIMEOUT);
   } else if (warp == 1) {
     // =========================== MMA issuer =================================
     constexpr uint32_t idesc = umma_idesc_tf32(C::MT, RS);
@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
     }
     for (int j = max(0, issued - 2); j < issued; ++j)
       if (!mbar_drain(&bar_mma[j & 1], ((unsigned)j >> 1) & 1u, tmo) && lane == 0)
-        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+        raise_error(ctrl, (int)PN_ERR_TIMEOUT);
   } else if (warp < C::WE0) {
     // =========================== look-back ==================================
     // warp 2 + j takes tiles j, j + NLB, ...; self-validating words, flags as hints
@@ -772,10 +772,10 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  unsigned rmax = 0u;   // the CTA's residual maximum, on thread 0
   if (tid == 0) {
-    unsigned v = 0u;
-    for (int w = 0; w < C::NT / 32; ++w) v = max(v, __float_as_uint(sRed[w]));
-    if (v) atomicMax(&ctrl->resid_bits, v);
+    for (int w = 0; w < C::NT / 32; ++w) rmax = max(rmax, __float_as_uint(sRed[w]));
+    if (rmax && !P.persist) atomicMax(&ctrl->resid_bits, rmax);
   }
   if (!P.persist) break;
   // Set-up of the next iteration ahead of the grid barrier: fresh barriers (every operation on
@@ -790,9 +790,9 @@ __global__ void __launch_bounds__(DiagTctCfg<CELL, MODE, DP>::NT, 1) diag_tct_ke
                        l2_policy_evict_last());
     }
   }
-  if (!finish_iteration(P, A, iter, epoch, s_last, (gen0 >> 1) + (unsigned)round)) {
+  if (!finish_iteration(P, A, iter, epoch, s_last, (gen0 >> 1) + (unsigned)round, rmax)) {
     // no next iteration: the prefetched step inputs land before the CTA exits
-    if (tid == 0 && has_tile0 && !mbar_drain(&bar_xfull[0], 0u, tmo)) atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+    if (tid == 0 && has_tile0 && !mbar_drain(&bar_xfull[0], 0u, tmo)) raise_error(ctrl, (int)PN_ERR_TIMEOUT);
     break;
   }
   }   // iterations

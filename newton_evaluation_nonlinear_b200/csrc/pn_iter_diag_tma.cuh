@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(DiagTmaCfg<CELL, MODE, DP, G, TM, TN, TS>::NT,
     // drain: every issued fill must land before the CTA may exit
     for (int j = max(0, it - STAGES); j < it; ++j)
       if (!mbar_drain(&s_full[j % STAGES], (unsigned)(j / STAGES) & 1u, A.timeout_ns) && lane == 0)
-        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+        raise_error(ctrl, (int)PN_ERR_TIMEOUT);
     (void)ok;
   } else {
     // ======================= consumer warps ================================

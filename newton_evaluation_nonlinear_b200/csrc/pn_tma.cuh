@@ -61,7 +61,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, Ctrl* 
     if (((++spins) & 31u) == 0u) {
       if (ld_volatile(&ctrl->error)) return false;
       if ((long long)(globaltimer() - t0) > timeout_ns) {
-        atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+        raise_error(ctrl, (int)PN_ERR_TIMEOUT);
         return false;
       }
     }

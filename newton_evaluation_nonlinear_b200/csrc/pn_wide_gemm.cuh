@@ -220,12 +220,12 @@ __global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __
   if (warp == 0 && lane == 0) {
     const int n = s_loaded;
     for (int u = max(0, n - NS); u < n; ++u)
-      if (!mbar_drain(&bar_full[u % NS], (unsigned)(u / NS) & 1u, tmo)) atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+      if (!mbar_drain(&bar_full[u % NS], (unsigned)(u / NS) & 1u, tmo)) raise_error(ctrl, (int)PN_ERR_TIMEOUT);
   }
   if (warp == 1 && lane == 0) {
     const int n = s_issued;
     for (int u = max(0, n - NS); u < n; ++u)
-      if (!mbar_drain(&bar_empty[u % NS], (unsigned)(u / NS) & 1u, tmo)) atomicCAS(&ctrl->error, 0, (int)PN_ERR_TIMEOUT);
+      if (!mbar_drain(&bar_empty[u % NS], (unsigned)(u / NS) & 1u, tmo)) raise_error(ctrl, (int)PN_ERR_TIMEOUT);
   }
   tc_fence_before();
   __syncthreads();
