@@ -77,7 +77,8 @@ struct pn_ctx {
   float* wt_hi = nullptr;          // TF32 split of W, row-major [D][D]
   float* wt_lo = nullptr;
   float* ypre = nullptr;           // [B*T][D]
-  CUtensorMap* wmaps = nullptr;    // [0]/[1] S of iterate buffer 0 / 1, [2] W_hi, [3] W_lo
+  CUtensorMap* wmaps = nullptr;    // kWideMaps: [0]/[1] S of iterate buffer 0 / 1, [2] W_hi, [3] W_lo;
+                                   // the per-channel kernel's tiles: [4] Y, [5] step inputs, [6]/[7] s^(i)
   CUtensorMap* wmaps_h = nullptr;
   // the input projection on the tensor cores (N = R*D a multiple of 16 up to 256, d_in % 4 == 0)
   const void* proj_gemm = nullptr;
@@ -266,6 +267,7 @@ IterParams make_params(const pn_ctx* h, int mode) {
   P.args = h->args;
   P.hist = h->hist;
   P.tmaps = h->tmaps ? h->tmaps + (size_t)mode * kTcMaps : nullptr;   // each mode's kernel has its own maps
+  if (kind == kKindDiagPost) P.tmaps = h->wmaps ? h->wmaps + 4 : nullptr;   // its tile loads
   P.eps = h->eps;
   P.D = h->D;
   P.d_in = h->d_in;
@@ -276,7 +278,8 @@ IterParams make_params(const pn_ctx* h, int mode) {
   P.tiles_per_group = h->B * h->fam.nchunks[mode];
   P.run = h->fam.run[mode];
   const int G = h->fam.k[mode].G;
-  P.agg_stride = dense ? G * (G + 1) : 2 * G;
+  // the wide per-channel kernel keeps two (A, B) pairs per channel: the tile's and its first half's
+  P.agg_stride = dense ? G * (G + 1) : (kind == kKindDiagPost ? 4 * G : 2 * G);
   P.pref_stride = G;
   P.cond = 0;
   return P;
@@ -336,13 +339,21 @@ bool encode_2d_sw128(CUtensorMap* m, const void* base, int cols, long long rows,
 }
 
 // The wide product's maps for the current call: S of both iterate buffers (128 rows x 32
-// floats per box) and W_hi, W_lo (D rows x 32 floats).
-bool encode_wide_maps(const pn_ctx* h, CUtensorMap* out) {
+// floats per box) and W_hi, W_lo (D rows x 32 floats); then the per-channel kernel's tile loads
+// (G channels of L steps of one sequence): Y (row b T + t - 1 read as step t - 1 of sequence b),
+// the step inputs, and s^(i) of both iterate buffers (L + 1 steps, from t0 - 1).
+bool encode_wide_maps(const pn_ctx* h, CUtensorMap* out, int G, int L) {
   const long long rows = (long long)h->B * h->T;
-  return encode_2d_sw128(&out[0], h->args_h->states, h->D, rows, 32, 128) &&
-         encode_2d_sw128(&out[1], h->buf1, h->D, rows, 32, 128) &&
-         encode_2d_sw128(&out[2], h->wt_hi, h->D, h->D, 32, h->D) &&
-         encode_2d_sw128(&out[3], h->wt_lo, h->D, h->D, 32, h->D);
+  const int D = h->D, T = h->T, B = h->B;
+  const void* xs = (h->cell == PN_CELL_EULER_TANH) ? (const void*)h->args_h->x : (const void*)h->xin;
+  return encode_2d_sw128(&out[0], h->args_h->states, D, rows, 32, 128) &&
+         encode_2d_sw128(&out[1], h->buf1, D, rows, 32, 128) &&
+         encode_2d_sw128(&out[2], h->wt_hi, D, D, 32, D) &&
+         encode_2d_sw128(&out[3], h->wt_lo, D, D, 32, D) &&
+         encode_seq(&out[4], h->ypre, D, T, B, G, L, false) &&
+         encode_seq(&out[5], xs, D, T, B, G, L, false) &&
+         encode_seq(&out[6], h->args_h->states, D, T, B, G, L + 1, false) &&
+         encode_seq(&out[7], h->buf1, D, T, B, G, L + 1, false);
 }
 
 // Fills the pinned mirror of the maps of the tensor-core kernels for the
@@ -557,7 +568,12 @@ pn_status build_graph(pn_ctx* h, int mode, bool adaptive = false) {
         if (err != cudaSuccess) return err;
         dep = &pnode;
       }
-      return add_kernel(gr, km.fn, dim3((unsigned)h->fam.grid[m]), dim3(km.nt), km.smem, kargs, dep, &knode);
+      err = add_kernel(gr, km.fn, dim3((unsigned)h->fam.grid[m]), dim3(km.nt), km.smem, kargs, dep, &knode);
+      if (err != cudaSuccess || !km.coop) return err;
+      if (h->fam.grid[m] > h->fam.resident[m]) return cudaErrorCooperativeLaunchTooLarge;
+      cudaLaunchAttributeValue cv{};
+      cv.cooperative = 1;
+      return cudaGraphKernelNodeSetAttribute(knode, cudaLaunchAttributeCooperative, &cv);
     };
     if (!adaptive) {
       e = add_iteration(body, mode, nullptr);
@@ -613,8 +629,9 @@ fail_graph:
 
 // The looping kernels' CTAs wait on one another (they meet at a grid barrier
 // after every iteration; the channel-major kernel also starts each CTA with a
-// static ticket, blockIdx.x, whose look-back may need any lower one), so all
-// of their CTAs must be resident at once.  They are launched cooperatively:
+// static ticket, blockIdx.x, whose look-back may need any lower one), and so
+// do those of the wide per-channel kernel (grid barriers between the phases of
+// its scan), so all of their CTAs must be resident at once.  They are launched cooperatively:
 // the runtime refuses a grid it cannot keep resident (another context's
 // kernels, an MPS limit) instead of every wait running out its timeout.  The
 // grid was sized from the occupancy query; the check below guards that sizing
@@ -630,7 +647,7 @@ pn_status launch_iter(pn_ctx* h, int mode, int persist = 0) {
     wide_launch(h, ki, wl);
     PN_CUDA(h, cudaLaunchKernel(wl.fn, dim3(wl.grid), dim3(wl.nt), wl.kargs, wl.smem, h->stream));
   }
-  if (!ki.loops) {
+  if (!ki.loops && !ki.coop) {
     PN_CUDA(h, cudaLaunchKernel(ki.fn, dim3(grid), dim3(ki.nt), kargs, ki.smem, h->stream));
     return PN_OK;
   }
@@ -749,9 +766,10 @@ pn_status upload_tc_maps(pn_ctx* h, int mode) {
     PN_CUDA(h, cudaMemcpyAsync(h->pmaps, h->pmaps_h, 4 * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
   }
   if (h->fam.k[mode].pre_fn) {
-    if (!encode_wide_maps(h, h->wmaps_h))
+    if (!encode_wide_maps(h, h->wmaps_h, h->fam.k[mode].G, h->fam.k[mode].L))
       return fail(h, PN_ERR_CUDA, "encoding the wide product's tensor maps failed (D=%d, T=%d, B=%d)", h->D, h->T, h->B);
-    PN_CUDA(h, cudaMemcpyAsync(h->wmaps, h->wmaps_h, 4 * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
+    PN_CUDA(h, cudaMemcpyAsync(h->wmaps, h->wmaps_h, kWideMaps * sizeof(CUtensorMap), cudaMemcpyHostToDevice,
+                               h->stream));
     return PN_OK;
   }
   if (!tagged_lookback(h->fam.k[mode].kind)) return PN_OK;
@@ -970,7 +988,7 @@ pn_status select_kernels(pn_ctx* h) {
     const size_t nt = (size_t)h->fam.ntiles[m];
     // the tensor-core kernels publish 64-bit tagged words: twice the floats
     const size_t wf = tagged_lookback(ki.kind) ? 2 : 1;
-    const size_t aggf = nt * ((m == PN_NEWTON) ? G * (G + 1) : 2 * G) * wf;
+    const size_t aggf = nt * ((m == PN_NEWTON) ? G * (G + 1) : (ki.kind == kKindDiagPost ? 4 * G : 2 * G)) * wf;
     h->agg_floats = std::max(h->agg_floats, aggf);
     h->pref_floats = std::max(h->pref_floats, nt * G * wf);
     h->nflags = std::max(h->nflags, nt);
@@ -1255,8 +1273,8 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
       PN_TRY(dalloc(h, &h->ypre, BT * D));
       if (cudaMemcpy(h->wt_hi, whi.data(), whi.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
           cudaMemcpy(h->wt_lo, wlo.data(), wlo.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
-          cudaMalloc((void**)&h->wmaps, 4 * sizeof(CUtensorMap)) != cudaSuccess ||
-          cudaMallocHost((void**)&h->wmaps_h, 4 * sizeof(CUtensorMap)) != cudaSuccess) {
+          cudaMalloc((void**)&h->wmaps, kWideMaps * sizeof(CUtensorMap)) != cudaSuccess ||
+          cudaMallocHost((void**)&h->wmaps_h, kWideMaps * sizeof(CUtensorMap)) != cudaSuccess) {
         st = fail(h, PN_ERR_NOMEM, "allocating the wide product's buffers failed");
         goto bad;
       }

@@ -99,6 +99,7 @@ __global__ void init_kernel(const Args* __restrict__ args, Ctrl* __restrict__ ct
     ctrl->arrive = 0ull;
     ctrl->resid_loop[0] = 0u;
     ctrl->resid_loop[1] = 0u;
+    ctrl->sync_count = 0u;
     ctrl->timeout_ticket = -1;
     ctrl->t_start = ~0ull;
     ctrl->fmt_in = fmt != 0;    // s^(0) and s^(1) are narrow when a narrow format is set

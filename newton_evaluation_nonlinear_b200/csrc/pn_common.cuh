@@ -20,6 +20,7 @@ constexpr unsigned kFlagAgg = 1u;      // tile published its aggregate
 constexpr unsigned kFlagPrefix = 2u;   // tile published its inclusive prefix (a state)
 constexpr int kMaxGroups = 8;          // channel groups of the diagonal-family kernels (D / G)
 constexpr int kTcMaps = 5;             // TMA tensor maps of the tensor-core kernels
+constexpr int kWideMaps = 8;           // TMA tensor maps of the wide product and its per-channel kernel
 
 // Device control block: one per handle, in device memory.
 struct Ctrl {
@@ -53,6 +54,9 @@ struct Ctrl {
   // (kArrive* below), and their residual maxima by iteration parity.
   alignas(128) unsigned long long arrive;
   unsigned resid_loop[2];
+  // plain grid barrier inside one cooperative launch (the phases of the wide per-channel kernel)
+  alignas(128) unsigned sync_count;
+  unsigned sync_gen;
 };
 
 // Fields of Ctrl::arrive, each a count of CTAs (at most 2^20 - 1): arrived, with a residual

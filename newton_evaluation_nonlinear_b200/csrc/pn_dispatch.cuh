@@ -37,6 +37,7 @@ struct KInfo {
   const void* pre_fn = nullptr;   // launched before fn in every iteration (the tensor-core product Y = S W^T)
   int pre_nt = 0;
   size_t pre_smem = 0;
+  bool coop = false;    // meets a grid barrier inside every launch: launched cooperatively
 };
 
 template <int CELL, int MODE, int DP, int G, int TM, int TN, int TS>
@@ -146,10 +147,11 @@ template <int CELL, int MODE, int DP>
 inline KInfo diag_wide_kinfo() {
   using C = PostCfg<CELL, MODE, DP>;
   using W = WideGemmCfg<DP>;   // N = K = DP
-  KInfo k{(const void*)&diag_post_kernel<CELL, MODE, DP>, C::NT, C::L, C::G, 0, kKindDiagPost};
+  KInfo k{(const void*)&diag_post_kernel<CELL, MODE, DP>, C::NT, C::L, C::G, C::SMEM_BYTES, kKindDiagPost};
   k.pre_fn = (const void*)&wide_gemm_kernel<DP>;
   k.pre_nt = W::NT;
   k.pre_smem = (size_t)W::SMEM_BYTES;
+  k.coop = true;   // the phases of the scan meet at grid barriers
   return k;
 }
 
