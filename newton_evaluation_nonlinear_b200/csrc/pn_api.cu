@@ -77,15 +77,15 @@ struct pn_ctx {
   float* wt_hi = nullptr;          // TF32 split of W, row-major [D][D]
   float* wt_lo = nullptr;
   float* ypre = nullptr;           // [B*T][D]
-  CUtensorMap* wmaps = nullptr;    // kWideMaps: [0]/[1] S of iterate buffer 0 / 1, [2] W_hi, [3] W_lo;
-                                   // the per-channel kernel's tiles: [4] Y, [5] step inputs, [6]/[7] s^(i)
+  CUtensorMap* wmaps = nullptr;    // kWideMaps: [0]/[1] S of iterate buffer 0 / 1, [2] W_hi, [3] W_lo, [4] Y
+                                   // stores; the per-channel kernel's tiles: [5] Y, [6] step inputs, [7]/[8] s^(i)
   CUtensorMap* wmaps_h = nullptr;
   // the input projection on the tensor cores (N = R*D a multiple of 16 up to 256, d_in % 4 == 0)
   const void* proj_gemm = nullptr;
   size_t proj_gemm_smem = 0;
   float* proj_hi = nullptr;        // TF32 split of U (or W_ih), row-major [R*D][d_in]
   float* proj_lo = nullptr;
-  CUtensorMap* pmaps = nullptr;    // [0], [1] x, [2] U_hi, [3] U_lo
+  CUtensorMap* pmaps = nullptr;    // kProjMaps: [0], [1] x, [2] U_hi, [3] U_lo, [4] u stores
   CUtensorMap* pmaps_h = nullptr;
   // host pinned mirrors
   Args* args_h = nullptr;
@@ -267,7 +267,7 @@ IterParams make_params(const pn_ctx* h, int mode) {
   P.args = h->args;
   P.hist = h->hist;
   P.tmaps = h->tmaps ? h->tmaps + (size_t)mode * kTcMaps : nullptr;   // each mode's kernel has its own maps
-  if (kind == kKindDiagPost) P.tmaps = h->wmaps ? h->wmaps + 4 : nullptr;   // its tile loads
+  if (kind == kKindDiagPost) P.tmaps = h->wmaps ? h->wmaps + 5 : nullptr;   // its tile loads
   P.eps = h->eps;
   P.D = h->D;
   P.d_in = h->d_in;
@@ -350,10 +350,11 @@ bool encode_wide_maps(const pn_ctx* h, CUtensorMap* out, int G, int L) {
          encode_2d_sw128(&out[1], h->buf1, D, rows, 32, 128) &&
          encode_2d_sw128(&out[2], h->wt_hi, D, D, 32, D) &&
          encode_2d_sw128(&out[3], h->wt_lo, D, D, 32, D) &&
-         encode_seq(&out[4], h->ypre, D, T, B, G, L, false) &&
-         encode_seq(&out[5], xs, D, T, B, G, L, false) &&
-         encode_seq(&out[6], h->args_h->states, D, T, B, G, L + 1, false) &&
-         encode_seq(&out[7], h->buf1, D, T, B, G, L + 1, false);
+         encode_2d_sw128(&out[4], h->ypre, D, rows, 32, 128) &&
+         encode_seq(&out[5], h->ypre, D, T, B, G, L, false) &&
+         encode_seq(&out[6], xs, D, T, B, G, L, false) &&
+         encode_seq(&out[7], h->args_h->states, D, T, B, G, L + 1, false) &&
+         encode_seq(&out[8], h->buf1, D, T, B, G, L + 1, false);
 }
 
 // Fills the pinned mirror of the maps of the tensor-core kernels for the
@@ -760,10 +761,12 @@ pn_status upload_tc_maps(pn_ctx* h, int mode) {
     const int N = cell_R(h->cell) * h->D;
     if (!encode_2d_sw128(&h->pmaps_h[0], h->args_h->x, h->d_in, rows, 32, 128) ||
         !encode_2d_sw128(&h->pmaps_h[2], h->proj_hi, h->d_in, N, 32, N) ||
-        !encode_2d_sw128(&h->pmaps_h[3], h->proj_lo, h->d_in, N, 32, N))
+        !encode_2d_sw128(&h->pmaps_h[3], h->proj_lo, h->d_in, N, 32, N) ||
+        (N % 32 == 0 && !encode_2d_sw128(&h->pmaps_h[4], h->xin, N, rows, 32, 128)))
       return fail(h, PN_ERR_CUDA, "encoding the input projection's tensor maps failed");
     h->pmaps_h[1] = h->pmaps_h[0];
-    PN_CUDA(h, cudaMemcpyAsync(h->pmaps, h->pmaps_h, 4 * sizeof(CUtensorMap), cudaMemcpyHostToDevice, h->stream));
+    PN_CUDA(h, cudaMemcpyAsync(h->pmaps, h->pmaps_h, kProjMaps * sizeof(CUtensorMap), cudaMemcpyHostToDevice,
+                               h->stream));
   }
   if (h->fam.k[mode].pre_fn) {
     if (!encode_wide_maps(h, h->wmaps_h, h->fam.k[mode].G, h->fam.k[mode].L))
@@ -1241,8 +1244,8 @@ pn_status pn_create(pn_handle* out, pn_cell cell, int D, int d_in, int T, int B,
         PN_TRY(dalloc(h, &h->proj_lo, plo.size()));
         if (cudaMemcpy(h->proj_hi, phi.data(), phi.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
             cudaMemcpy(h->proj_lo, plo.data(), plo.size() * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
-            cudaMalloc((void**)&h->pmaps, 4 * sizeof(CUtensorMap)) != cudaSuccess ||
-            cudaMallocHost((void**)&h->pmaps_h, 4 * sizeof(CUtensorMap)) != cudaSuccess) {
+            cudaMalloc((void**)&h->pmaps, kProjMaps * sizeof(CUtensorMap)) != cudaSuccess ||
+            cudaMallocHost((void**)&h->pmaps_h, kProjMaps * sizeof(CUtensorMap)) != cudaSuccess) {
           st = fail(h, PN_ERR_NOMEM, "allocating the projection's tensor-core operands failed");
           goto bad;
         }

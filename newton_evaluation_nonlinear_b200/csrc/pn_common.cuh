@@ -20,7 +20,8 @@ constexpr unsigned kFlagAgg = 1u;      // tile published its aggregate
 constexpr unsigned kFlagPrefix = 2u;   // tile published its inclusive prefix (a state)
 constexpr int kMaxGroups = 8;          // channel groups of the diagonal-family kernels (D / G)
 constexpr int kTcMaps = 5;             // TMA tensor maps of the tensor-core kernels
-constexpr int kWideMaps = 8;           // TMA tensor maps of the wide product and its per-channel kernel
+constexpr int kWideMaps = 9;           // TMA tensor maps of the wide product and its per-channel kernel
+constexpr int kProjMaps = 5;           // TMA tensor maps of the input projection
 
 // Device control block: one per handle, in device memory.
 struct Ctrl {

@@ -89,6 +89,20 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, unsign
       : "memory");
 }
 
+// Named barrier over the first `nthreads` threads that also returns, to every one of them, whether
+// `v` held on all of them (a warp-aligned instruction: the warp is reconverged first).
+__device__ __forceinline__ bool named_barrier_and(unsigned id, unsigned nthreads, bool v) {
+  __syncwarp();
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // Named barrier over the first `nthreads` threads (a multiple of 32).
 // bar.sync is warp-aligned: every thread of a warp must reach it together, which inline asm does not
 // tell the compiler, so the warp is reconverged first (the code before a barrier may have diverged).

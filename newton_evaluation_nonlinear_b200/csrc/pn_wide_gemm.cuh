@@ -23,7 +23,11 @@
 //            accumulators (128 lanes x D columns); a commit frees the stage;
 //   warps 2-3  S_lo of each landed S chunk (element-wise: the swizzled
 //            layout is the same for both);
-//   warps 4-7  epilogue: thread = row, TMEM -> registers -> Y.
+//   warps 4-7  epilogue: thread = row, TMEM -> registers -> Y; for N a multiple
+//            of 32 through a double-buffered 128 x 32 staging tile (128-byte
+//            swizzled) and one TMA tensor store per 32 columns, so that Y is
+//            written in whole lines (a warp's direct stores would touch 32
+//            rows each).
 // TMA loads never use cluster multicast.  Rows past B*T read as zero and are
 // not stored.
 #pragma once
@@ -44,11 +48,24 @@ struct WideGemmCfg {
   static constexpr int NSTAGE = (200 * 1024) / STAGE < 4 ? (200 * 1024) / STAGE : 4;
   static constexpr int TCOLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
   static constexpr int NT = 256;                  // 8 warps
-  static constexpr int SMEM_BYTES = NSTAGE * STAGE + 1024;   // + slack to align the ring to 1024 bytes
+  static constexpr bool kStaged = (N % 32) == 0;  // epilogue through the staging tile and TMA stores
+  static constexpr int OUT_BYTES = BM * 32 * 4;   // one staging buffer: 128 rows x 32 floats
+  static constexpr int OFF_OUT = NSTAGE * STAGE;  // two staging buffers after the ring
+  static constexpr int SMEM_BYTES = NSTAGE * STAGE + (kStaged ? 2 * OUT_BYTES : 0) + 1024;   // + alignment slack
   static_assert(NSTAGE >= 2, "two stages at least");
   static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
+
+// 2-D TMA tensor store of one box from shared memory (coordinates >= 0); elements outside the
+// array are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int c0, int c1, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(c0), "r"(c1),
+               "r"(smem_addr(src))
+               : "memory");
+}
+// this thread's committed bulk stores, all but the most recent group, have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_but1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 
 // 2-D TMA tensor load (coordinates: column c0, row c1), counted on bar.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
@@ -61,7 +78,8 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 
 // Y[r][n] = sum_k X[r][k] W[n][k] (+ bias[n]) for r < rows, n < N, k < K.  maps: [0] X of iterate
 // buffer 0 and [1] of buffer 1 (the iteration's parity picks one; the input projection passes the
-// same map twice), [2] W_hi, [3] W_lo.  K need not be a multiple of 32 (the loads zero-fill).
+// same map twice), [2] W_hi, [3] W_lo, [4] Y (stores, 128 rows x 32 floats, 128-byte swizzled;
+// used when N is a multiple of 32).  K need not be a multiple of 32 (the loads zero-fill).
 template <int N>
 __global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __restrict__ maps, float* __restrict__ Y,
                                                            int rows, int K, const float* __restrict__ bias, Ctrl* ctrl,
@@ -185,6 +203,53 @@ __global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_lo[s]);
     }
+  } else if constexpr (C::kStaged) {
+    // ---------------- epilogue: thread = row, staged TMA stores ----------------
+    const int q = warp & 3;   // TMEM lane quarter
+    const int r = 32 * q + lane;   // row of the tile
+    const bool issuer = (warp == 4 && lane == 0);
+    const CUtensorMap* mY = maps + 4;
+    if (issuer) tmap_acquire(mY);
+    int nst = 0;   // staging buffers filled so far (buffer nst & 1 next)
+    for (int j = 0; j < my_tiles; ++j) {
+      const int acc = j & 1;
+      // the four warps meet the staging barriers together: all go on, or all stop, here
+      const bool ok = mbar_wait_flag(&bar_acc[acc], (unsigned)(j >> 1) & 1u, ctrl, tmo, &s_abort);
+      if (!named_barrier_and(1, 128, ok)) break;
+      tc_fence_after();
+      const int tile = (int)blockIdx.x + j * (int)gridDim.x;
+      const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * DP);
+#pragma unroll 1
+      for (int c = 0; c < DP; c += 32, ++nst) {
+        unsigned char* ob = ring + C::OFF_OUT + (nst & 1) * C::OUT_BYTES;
+        // the store that last read this buffer (two back) is done with it
+        if (issuer && nst >= 2) bulk_wait_read_but1();
+        named_barrier(1, 128);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float v[16];
+          tmem_ld16(base + (uint32_t)(c + 16 * hh), v);
+          if (bias) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] += __ldg(bias + c + 16 * hh + e);
+          }
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(ob + sw128_offset(r, 16 * hh + e)) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+        fence_async_smem();   // generic writes -> the tensor store (async proxy)
+        named_barrier(1, 128);
+        if (issuer) {
+          tma_store_2d(mY, c, tile * C::BM, ob);
+          bulk_commit();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_accfree[acc]);
+    }
+    if (issuer) bulk_wait_all();   // Y is in global memory (and the staging buffers read) before the CTA retires
+    __syncwarp();
   } else {
     // ---------------- epilogue: thread = row ----------------
     const int q = warp & 3;   // TMEM lane quarter
