@@ -476,7 +476,7 @@ void wide_launch(pn_ctx* h, const KInfo& ki, GemmLaunch& g) {
 // the input projection on the tensor cores (h->proj_gemm set at create)
 void proj_launch(pn_ctx* h, GemmLaunch& g) {
   g.fn = h->proj_gemm;
-  g.nt = 256;
+  g.nt = WideGemmCfg<64>::NT;   // the same for every width
   g.smem = h->proj_gemm_smem;
   g.maps = h->pmaps;
   g.y = h->xin;

@@ -21,7 +21,7 @@
 //            128-byte swizzled, into a stage of the ring;
 //   warp 1   MMA issuer: 3 passes x 4 K-steps per chunk into one of two TMEM
 //            accumulators (128 lanes x D columns); a commit frees the stage;
-//   warps 2-3  S_lo of each landed S chunk (element-wise: the swizzled
+//   warps 2-3, 8-9  S_lo of each landed S chunk (element-wise: the swizzled
 //            layout is the same for both);
 //   warps 4-7  epilogue: thread = row, TMEM -> registers -> Y; for N a multiple
 //            of 32 through a double-buffered 128 x 32 staging tile (128-byte
@@ -47,7 +47,7 @@ struct WideGemmCfg {
   static constexpr int STAGE = 2 * S_BYTES + 2 * W_BYTES;   // S, S_lo, W_hi, W_lo
   static constexpr int NSTAGE = (200 * 1024) / STAGE < 4 ? (200 * 1024) / STAGE : 4;
   static constexpr int TCOLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
-  static constexpr int NT = 256;                  // 8 warps
+  static constexpr int NT = 320;                  // 10 warps: producer, MMA, 2 + 2 split, 4 epilogue
   static constexpr bool kStaged = (N % 32) == 0;  // epilogue through the staging tile and TMA stores
   static constexpr int OUT_BYTES = BM * 32 * 4;   // one staging buffer: 128 rows x 32 floats
   static constexpr int OFF_OUT = NSTAGE * STAGE;  // two staging buffers after the ring
@@ -81,7 +81,7 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 // same map twice), [2] W_hi, [3] W_lo, [4] Y (stores, 128 rows x 32 floats, 128-byte swizzled;
 // used when N is a multiple of 32).  K need not be a multiple of 32 (the loads zero-fill).
 template <int N>
-__global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __restrict__ maps, float* __restrict__ Y,
+__global__ void __launch_bounds__(WideGemmCfg<N>::NT, 1) wide_gemm_kernel(const CUtensorMap* __restrict__ maps, float* __restrict__ Y,
                                                            int rows, int K, const float* __restrict__ bias, Ctrl* ctrl,
                                                            const Args* __restrict__ args) {
   using C = WideGemmCfg<N>;
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bar_full[s], 1u);
-      mbar_init(&bar_lo[s], 2u);
+      mbar_init(&bar_lo[s], 4u);
       mbar_init(&bar_empty[s], 1u);
     }
     for (int a = 0; a < 2; ++a) {
@@ -186,16 +186,16 @@ __global__ void __launch_bounds__(256, 1) wide_gemm_kernel(const CUtensorMap* __
       }
       __syncwarp();
     }
-  } else if (warp < 4) {
-    // ---------------- S_lo ----------------
-    const int t = tid - 64;   // 0 .. 63
+  } else if (warp < 4 || warp >= 8) {
+    // ---------------- S_lo (warps 2, 3, 8, 9) ----------------
+    const int t = (warp < 4) ? tid - 64 : tid - 192;   // 0 .. 127
     for (int u = 0; u < units; ++u) {
       const int s = u % NS;
       if (!mbar_wait_flag(&bar_full[s], (unsigned)(u / NS) & 1u, ctrl, tmo, &s_abort)) break;
       const float4* src = reinterpret_cast<const float4*>(sbuf(s));
       float4* dst = reinterpret_cast<float4*>(lbuf(s));
 #pragma unroll 4
-      for (int e = t; e < C::S_BYTES / 16; e += 64) {
+      for (int e = t; e < C::S_BYTES / 16; e += 128) {
         const float4 v = src[e];
         dst[e] = make_float4(tf32_tail(v.x), tf32_tail(v.y), tf32_tail(v.z), tf32_tail(v.w));
       }
