@@ -491,7 +491,6 @@ void proj_launch(pn_ctx* h, GemmLaunch& g) {
 
 pn_status build_graph(pn_ctx* h, int mode, bool adaptive = false) {
   if ((adaptive ? h->exec_ad[mode] : h->exec[mode])) return PN_OK;
-  const KInfo& ki = h->fam.k[mode];
   const PreLaunch pl = pre_launch(h);
   cudaGraph_t g = nullptr;
   PN_CUDA(h, cudaGraphCreate(&g, 0));

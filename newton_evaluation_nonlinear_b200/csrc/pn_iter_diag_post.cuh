@@ -126,9 +126,7 @@ __global__ void __launch_bounds__(PostCfg<CELL, MODE, DP>::NT, 2) diag_post_kern
   __syncthreads();
   const unsigned epoch = *(volatile unsigned*)&ctrl->epoch;
   const int iter = *(volatile int*)&ctrl->iter;
-  const float* __restrict__ src = (iter & 1) ? P.buf1 : A.states;
-  float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;
-  const float* __restrict__ xin = (CELL == PN_CELL_EULER_TANH) ? A.x : P.xin;   // [B][T][D]
+  float* __restrict__ dst = (iter & 1) ? A.states : P.buf1;   // s^(i+1); s^(i) and the inputs come by TMA
   unsigned rbits = 0u;
 
   // this CTA's tiles, blockIdx.x + r gridDim.x: phase 1 takes them as units 0 .. n1-1, phase 3 as

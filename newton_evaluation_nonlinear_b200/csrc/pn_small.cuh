@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(SmallCfg<CELL, DP>::NT, 1)
     // ---- 2. chunk aggregates, one thread per (chunk, column of [P | q]) --------------------------
     for (int e = tid; e < ntiles * (DP + 1); e += NT) {
       const int k = e / (DP + 1), j = e % (DP + 1);   // column j: P e_j for j < DP, q for j = DP
-      const int b = k / nch, t0 = (k % nch) * L;
+      const int t0 = (k % nch) * L;
       const int n = min(L, T - t0);
       float x[DP];
       {   // step 0: A_{t0} e_j, or b_{t0}
