@@ -93,6 +93,9 @@ __global__ void __launch_bounds__(PostCfg<CELL, MODE, DP>::NT, 2) diag_post_kern
   constexpr int NT = C::NT;
   constexpr bool kScan = (MODE != PN_JACOBI);
   constexpr bool kHasA = (MODE == PN_QUASI);
+  // undamped Euler Picard forms its states from Y and the step inputs alone (b_t = eps g_t, the
+  // residual was taken in phase 1), so phase 3 does not load s^(i)
+  constexpr bool kEulerPicard = (CELL == PN_CELL_EULER_TANH && MODE == PN_PICARD);
   extern __shared__ __align__(128) unsigned char smem_post_raw[];
   float* smem_post = reinterpret_cast<float*>(smem_post_raw + ((128u - (smem_addr(smem_post_raw) & 127u)) & 127u));
   __shared__ __align__(8) uint64_t bar_full[NS], bar_empty[NS];
@@ -204,10 +207,11 @@ __global__ void __launch_bounds__(PostCfg<CELL, MODE, DP>::NT, 2) diag_post_kern
         const uint64_t pol = l2_policy_evict_first();
         float* st = smem_post + (size_t)s * C::STAGE_FLOATS;
         const int col = t.g * G;
-        mbar_arrive_expect_tx(&bar_full[s], (unsigned)(C::STAGE_FLOATS * 4));
+        const bool with_s = !(kEulerPicard && !damped && u >= n1);
+        mbar_arrive_expect_tx(&bar_full[s], (unsigned)((with_s ? C::STAGE_FLOATS : 2 * L * G) * 4));
         tma_load_3d_hint(st, mY, col, t.t0 - 1, t.b, &bar_full[s], pol);
         tma_load_3d_hint(st + L * G, mX, col, t.t0, t.b, &bar_full[s], pol);
-        tma_load_3d_hint(st + 2 * L * G, mS, col, t.t0 - 1, t.b, &bar_full[s], pol);
+        if (with_s) tma_load_3d_hint(st + 2 * L * G, mS, col, t.t0 - 1, t.b, &bar_full[s], pol);
       }
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -243,11 +247,12 @@ __global__ void __launch_bounds__(PostCfg<CELL, MODE, DP>::NT, 2) diag_post_kern
     const float* sX = sY + L * G;
     const float* sS = sY + 2 * L * G;                                            // row m0: step t0 + m0 - 1
     float* orow = dst + (t.row0 + m0) * DP + c;
-    float sp = (t.t0 + m0 == 0) ? s0c : sS[0];
+    float sp = (t.t0 + m0 == 0) ? s0c : ((kEulerPicard && apply && !damped) ? 0.0f : sS[0]);
     float SA = 1.0f, SB = 0.0f;
+    const bool no_s = kEulerPicard && apply && !damped;   // phase 3 loaded no s^(i) (see the producer)
     auto step = [&](int i) {
       const float z = (t.t0 + m0 + i > 0) ? sY[i * G] : z0;
-      const float sc = sS[(i + 1) * G];
+      const float sc = no_s ? 0.0f : sS[(i + 1) * G];
       const float3 f = coef(z, sX[i * G], sc, sp, wdc);
       sp = sc;
       if (!apply) {
