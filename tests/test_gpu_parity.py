@@ -346,6 +346,47 @@ def test_wide_tensor_core_product(tc, cell, mode, D, T, B):
     _check_against_oracle(prob, mode, tc=tc)
 
 
+@pytest.mark.parametrize("cell,mode", [(pi.CELL_EULER, pi.MODE_PICARD), (pi.CELL_TANH_RNN, pi.MODE_QUASI)])
+def test_wide_many_chunks(cell, mode):
+    """D = 128 with 66 chunks of 32 steps per sequence (the last ragged): the per-channel kernel's fold
+    of the tile aggregates per (sequence, channel group) runs in several batches of loads.  Twenty
+    iterations with tol = 0 on both sides, states compared element by element: over 2100 steps the
+    Euler states reach |s| ~ 100, where fp32 rounding of the scan moves the last residuals by tens
+    of percent of a 1e-5 |s| tolerance, so a stop-rule comparison would test the rounding, not the
+    kernel.  (Euler quasi-Newton passes through far larger unconverged iterates on the way, which
+    puts its fp32 distance to the fp64 iterate above 1e-4 here; it is covered at T <= 333.)"""
+    prob = pi.random_problem(2210 + cell + mode, cell, 128, 128, T=2100, B=2, rho=0.6, eps=0.05,
+                             s0_scale=0.2, tol=1e-5)
+    it, _ = _check_against_oracle(prob, mode, tol=0.0, max_iters=20, tc=1)
+    assert it == 20
+
+
+def test_wide_bounded_wait_times_out_and_recovers():
+    """The wide per-channel kernel's test hook: the CTA holding tile 0 never arrives at the grid barrier
+    after the aggregates, so every CTA's bounded wait there runs out; the call returns
+    PN_ERR_TIMEOUT and the handle evaluates normally afterwards."""
+    import torch
+    pn = _pn()
+    prob = pi.random_problem(2233, pi.CELL_EULER, 256, 256, T=333, B=2, rho=0.6, eps=0.05, s0_scale=0.2,
+                             tol=1e-5)
+    solver = pn.Solver.from_problem(prob)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    solver.set_option(pn.PN_OPT_WAIT_TIMEOUT_NS, 20_000_000)   # 20 ms
+    solver.set_option(pn.PN_OPT_DEBUG_STALL_TICKET, 0)
+    with pytest.raises(pn.PnError) as e:
+        solver.eval(x, s0, "picard", 10, 1e-6)
+    assert e.value.status == pn.PN_ERR_TIMEOUT
+    solver.set_option(pn.PN_OPT_DEBUG_STALL_TICKET, -1)
+    m = oracle.Model.from_problem(prob)
+    seq = m.sequential(prob.x, prob.s0)
+    tol = prob.tol * max(1.0, float(np.abs(seq).max()))
+    states, it, r, st = solver.eval(x, s0, "picard", prob.T, tol)
+    assert st == pn.PN_OK
+    assert _relerr(states.cpu().numpy(), seq) <= REL_TOL
+    solver.close()
+
+
 @pytest.mark.parametrize("device_loop", [1, 0])
 @pytest.mark.parametrize("run", [1, 3, 0])
 @pytest.mark.parametrize("cell,D", [(pi.CELL_TANH_RNN, 16), (pi.CELL_GRU, 8), (pi.CELL_EULER, 4),

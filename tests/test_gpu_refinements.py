@@ -98,6 +98,16 @@ def test_damped_diagonal_modes_match_oracle(cell, mode, D, tc):
     _check(cell, D, T, 2, -1, 0.7, 371 + cell + D, mode=mode, tc=tc)
 
 
+@pytest.mark.parametrize("cell", [pi.CELL_TANH_RNN, pi.CELL_EULER])
+@pytest.mark.parametrize("mode", ["jacobi", "picard", "quasi"])
+def test_damped_wide_modes_match_oracle(cell, mode):
+    """Damping on the wide path (D = 256: the tensor-core product, then the per-channel kernel's three
+    phases): the damped states come out of the last phase, which for Euler Picard then loads s^(i)
+    again (undamped it does not need it)."""
+    T = 12 if (mode == "picard" and cell != pi.CELL_EULER) else 300
+    _check(cell, 256, T, 2, -1, 0.7, 391 + cell, mode=mode, tc=1)
+
+
 def test_damping_arguments_and_switching():
     """Damping toggles the kernel choice of Picard (tensor-core row-major kernel undamped, FP32 kernel
     damped) and back; the Euler drift keeps Picard contractive over the whole sequence."""
