@@ -142,6 +142,34 @@ def test_wide_states(cell, mode, D):
     _check_against_oracle(prob, mode)
 
 
+@pytest.mark.parametrize("cell,D,mode", [(pi.CELL_TANH_RNN, 64, pi.MODE_QUASI), (pi.CELL_TANH_RNN, 64, pi.MODE_JACOBI),
+                                         (pi.CELL_GRU, 32, pi.MODE_QUASI), (pi.CELL_TANH_RNN, 16, pi.MODE_NEWTON)])
+def test_looping_stop_rule_edges(cell, D, mode):
+    """The looping kernels (channel-major, row-major and warp-per-chunk Newton) take the stop decision
+    from the grid barrier's packed arrival count: tol = 0 runs exactly max_iters iterations and
+    reports PN_NOT_CONVERGED with the oracle's iterate; a huge tol stops at iteration 0; a NaN in the
+    input reports PN_ERR_NONFINITE, after which the handle evaluates normally."""
+    import torch
+    pn = _pn()
+    prob = pi.random_problem(2301 + D + mode, cell, D, D, T=700, B=2, rho=0.6, eps=0.05, s0_scale=0.3,
+                             tol=1e-5)
+    it, s = _check_against_oracle(prob, mode, tol=0.0, max_iters=5)
+    assert it == 5
+    solver = pn.Solver.from_problem(prob)
+    x = torch.from_numpy(prob.x).cuda()
+    s0 = torch.from_numpy(prob.s0).cuda()
+    _, it, _, st = solver.eval(x, s0, pi.MODE_NAMES[mode], 50, 1e9)
+    assert (it, st) == (0, pn.PN_OK)
+    bad = x.clone()
+    bad[1, 300, 3] = float("nan")
+    with pytest.raises(pn.PnError) as e:
+        solver.eval(bad, s0, pi.MODE_NAMES[mode], 20, 1e-6)
+    assert e.value.status == pn.PN_ERR_NONFINITE
+    _, it, _, st = solver.eval(x, s0, pi.MODE_NAMES[mode], 3, 0.0)
+    assert (it, st) == (3, pn.PN_NOT_CONVERGED)
+    solver.close()
+
+
 def test_picard_divergence_is_reported():
     """Picard on a tanh RNN far from the identity: the tail grows until it overflows; the loop must
     stop with PN_ERR_NONFINITE (or run out of iterations), never hang or return garbage as PN_OK."""
