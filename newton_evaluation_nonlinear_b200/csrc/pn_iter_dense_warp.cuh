@@ -101,6 +101,53 @@ __device__ __forceinline__ void lds_n(const float* p, float (&v)[N]) {
   }
 }
 
+// The chain at D = 16 on the tensor cores (one-gate cells, no band).  With Q = P^T the step
+// P_m = (diag(c0) + diag(c1) W) P_{m-1} reads Q_m = Q_{m-1} diag(c0) + (Q_{m-1} W^T) diag(c1): a
+// 16 x 16 x 16 product with the constant W^T as the B operand.  Q lives in the f32 accumulator
+// layout of the m16n8k8 TF32 MMA (lane = 4 g + i holds rows g, g + 8 and columns 2 i, 2 i + 1 of
+// each 8-column tile j), and that layout is also an A operand once the K index is relabelled: in
+// K-step s, A column i stands for Q column 8 s + 2 i and column i + 4 for 8 s + 2 i + 1, and the B
+// fragments hold W^T's rows in the same order.  So one step needs no data movement between lanes.
+// Products are 3xTF32 (hi hi + hi lo + lo hi, hi the operand with its low 13 mantissa bits
+// cleared), the two small passes in an accumulator of their own.
+__device__ __forceinline__ uint32_t tf32_hi_bits(float x) { return __float_as_uint(x) & 0xFFFFE000u; }
+__device__ __forceinline__ void mma_m16n8k8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// One chain step on q = Q_{m-1} (q[j][e]: row g + 8 (e >> 1), column 8 j + 2 i + (e & 1)), with
+// bh / bl the hi / lo B fragments (bh[s][j][h] = W[8 j + g][8 s + 2 i + h]) and c0 / c1 the
+// scalings of this lane's columns (c[j][h] for column 8 j + 2 i + h).
+__device__ __forceinline__ void chain_step_mma16(float (&q)[2][4], const uint32_t (&bh)[2][2][2],
+                                                 const uint32_t (&bl)[2][2][2], const float (&c0)[2][2],
+                                                 const float (&c1)[2][2]) {
+  uint32_t ah[2][4], al[2][4];
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    const float v[4] = {q[s][0], q[s][2], q[s][1], q[s][3]};   // A rows g, g + 8 x columns i, i + 4
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      ah[s][e] = tf32_hi_bits(v[e]);
+      al[s][e] = tf32_hi_bits(v[e] - __uint_as_float(ah[s][e]));
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    float hh[4] = {0.0f, 0.0f, 0.0f, 0.0f}, lo[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      mma_m16n8k8_tf32(hh, ah[s], bh[s][j]);
+      mma_m16n8k8_tf32(lo, ah[s], bl[s][j]);
+      mma_m16n8k8_tf32(lo, al[s], bh[s][j]);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q[j][e] = fmaf(c1[j][e & 1], hh[e] + lo[e], c0[j][e & 1] * q[j][e]);
+  }
+}
+
 template <int CELL, int DP, int NWARP>
 __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MINB) dense_warp_kernel(const IterParams P) {
   using C = DenseWarpCfg<CELL, DP, NWARP>;
@@ -185,6 +232,11 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
   }
   unsigned rbits = 0u;
   bool aborted = false;
+  // the D = 16 tensor-core chain (one-gate cells, no band)
+  constexpr bool kMmaChain = (DP == 16 && R == 1);
+  static_assert(!kMmaChain || C::NA == 32, "every lane takes part in the chain");
+  const bool mma_chain = kMmaChain && !banded;
+  const int qg = lane >> 2, qi = lane & 3;   // the MMA fragments' row group and column pair
 
   // W_q[r0 + r][k] of the Jacobian (band-masked when banded), RPL consecutive rows
   auto wrows = [&](int kk, int q, float (&w)[RPL]) { lds_n<RPL>(sWj + kk * WR + q * DP + r0, w); };
@@ -195,9 +247,11 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
   auto slice_matvec = [&](const float* x, float (&out)[R][RPL]) {
     if constexpr (C::WREG) {
       if (!banded) {
-        float acc[RPL];
+        float acc[RPL][4];   // four partial sums per row (k mod 4): a short dependent chain
 #pragma unroll
-        for (int r = 0; r < RPL; ++r) acc[r] = 0.0f;
+        for (int r = 0; r < RPL; ++r)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) acc[r][u] = 0.0f;
 #pragma unroll
         for (int kk = 0; kk < DP; kk += 4) {
           const float4 x4 = *reinterpret_cast<const float4*>(x + kk);
@@ -205,10 +259,10 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
 #pragma unroll
           for (int u = 0; u < 4; ++u)
 #pragma unroll
-            for (int r = 0; r < RPL; ++r) acc[r] = fmaf(wreg[r][kk + u], xv[u], acc[r]);
+            for (int r = 0; r < RPL; ++r) acc[r][u] = fmaf(wreg[r][kk + u], xv[u], acc[r][u]);
         }
 #pragma unroll
-        for (int r = 0; r < RPL; ++r) out[0][r] = acc[r];
+        for (int r = 0; r < RPL; ++r) out[0][r] = (acc[r][0] + acc[r][1]) + (acc[r][2] + acc[r][3]);
         return;
       }
     }
@@ -291,9 +345,10 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
       for (int m = ms; m < L; m += C::SPP) {
         const bool tok = (t0 + m) < T;
         const float* sp = sS + m * SP;   // s^(i)_{t-1}: the same row for the lanes of a pass
-        float z[R], zb[R];
+        // W_q s: two partial sums per product (even and odd k) keep the dependent chain short
+        float z[R], zb[R], z2[R][2], zb2[R][2];
 #pragma unroll
-        for (int q = 0; q < R; ++q) z[q] = zb[q] = 0.0f;
+        for (int q = 0; q < R; ++q) z2[q][0] = z2[q][1] = zb2[q][0] = zb2[q][1] = 0.0f;
 #pragma unroll
         for (int kk = 0; kk < DP; kk += 4) {
           const float4 s4 = *reinterpret_cast<const float4*>(sp + kk);
@@ -302,10 +357,15 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
           for (int u = 0; u < 4; ++u) {
 #pragma unroll
             for (int q = 0; q < R; ++q) {
-              z[q] = fmaf(sWf[(kk + u) * WR + q * DP + ci], sv[u], z[q]);
-              if (banded) zb[q] = fmaf(sWb[(kk + u) * WR + q * DP + ci], sv[u], zb[q]);
+              z2[q][u & 1] = fmaf(sWf[(kk + u) * WR + q * DP + ci], sv[u], z2[q][u & 1]);
+              if (banded) zb2[q][u & 1] = fmaf(sWb[(kk + u) * WR + q * DP + ci], sv[u], zb2[q][u & 1]);
             }
           }
+        }
+#pragma unroll
+        for (int q = 0; q < R; ++q) {
+          z[q] = z2[q][0] + z2[q][1];
+          zb[q] = zb2[q][0] + zb2[q][1];
         }
         if (!banded) {
 #pragma unroll
@@ -361,13 +421,29 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
     // ---- 3. chain [P | q] over the run, one chunk at a time --------------------------------
     // gs counts the run's composition steps: step 0 sets [P | q] = [A_0 | b_0], step gs > 0 composes
     // with A_m from buffer (gs - 1) & 1 into buffer gs & 1
+    // the lane's P entries; the tensor-core chain keeps Q = P^T there instead (accumulator layout)
     float pold[RPL][CPL];
+    float (&qt)[2][4] = *reinterpret_cast<float (*)[2][4]>(&pold[0][0]);
+    static_assert(!kMmaChain || (RPL == 2 && CPL == 4), "Q fits the P registers");
     int gs = 0;
 #pragma unroll 1
     for (int c = c_first; c < c_end; ++c) {
       const int t0 = c * L;
       stage(t0);
       cell(t0, true);
+      uint32_t wbh[2][2][2], wbl[2][2][2];   // the tensor-core chain's W^T fragments, hi and lo
+      if (kMmaChain && mma_chain) {
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float w = sWf[(8 * ks + 2 * qi + h) * WR + 8 * j + qg];   // W[8 j + g][8 s + 2 i + h]
+              wbh[ks][j][h] = tf32_hi_bits(w);
+              wbl[ks][j][h] = tf32_hi_bits(w - __uint_as_float(wbh[ks][j][h]));
+            }
+      }
 #pragma unroll 1
       for (int m = 0; m < L; ++m, ++gs) {
         float c0[RPL], cq[R][RPL], bm[RPL];
@@ -377,6 +453,38 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
         ld_rows(sB + m * DP, bm);
         float* Pn = sP + (gs & 1) * DP * PS;
         float qn[RPL];
+        if (kMmaChain && mma_chain) {
+          // P on the tensor cores; q as below.  c0, c1 of this lane's Q columns 2 i, 2 i + 1, 8 + 2 i, 9 + 2 i
+          const float* cv = sC + (m * NCS) * DP;
+          const float2 u0 = *reinterpret_cast<const float2*>(cv + 2 * qi);
+          const float2 u1 = *reinterpret_cast<const float2*>(cv + 8 + 2 * qi);
+          const float2 v0 = *reinterpret_cast<const float2*>(cv + DP + 2 * qi);
+          const float2 v1 = *reinterpret_cast<const float2*>(cv + DP + 8 + 2 * qi);
+          const float sc0[2][2] = {{u0.x, u0.y}, {u1.x, u1.y}};
+          const float sc1[2][2] = {{v0.x, v0.y}, {v1.x, v1.y}};
+          if (gs == 0) {   // Q_0 = A_0^T: Q_0[n][r] = c0[r] [r == n] + c1[r] W[r][n]
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int n = qg + 8 * (e >> 1), r = 8 * j + 2 * qi + (e & 1);
+                qt[j][e] = fmaf(sc1[j][e & 1], sWf[n * WR + r], (r == n) ? sc0[j][e & 1] : 0.0f);
+              }
+#pragma unroll
+            for (int r = 0; r < RPL; ++r) qn[r] = bm[r];
+          } else {
+            chain_step_mma16(qt, wbh, wbl, sc0, sc1);
+            const float* Qk = sQ + ((gs - 1) & 1) * DP;
+            float qa[R][RPL], qo[RPL];
+            slice_matvec(Qk, qa);
+            ld_rows(Qk, qo);
+#pragma unroll
+            for (int r = 0; r < RPL; ++r) qn[r] = fmaf(cq[0][r], qa[0][r], fmaf(c0[r], qo[r], bm[r]));
+          }
+          if (cg == 0) st_rows(sQ + (gs & 1) * DP, qn);
+          __syncwarp();
+          continue;
+        }
         if (gs == 0) {
 #pragma unroll
           for (int r = 0; r < RPL; ++r) {
@@ -470,6 +578,14 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
         }
         __syncwarp();
       }
+    }
+    if (kMmaChain && mma_chain) {   // the tensor-core chain's aggregate into the shared-memory P
+      float* Pw = sP + ((gs - 1) & 1) * DP * PS;
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) Pw[(8 * j + 2 * qi + (e & 1)) * PS + qg + 8 * (e >> 1)] = qt[j][e];
+      __syncwarp();
     }
     const float* Pl = sP + ((gs - 1) & 1) * DP * PS;   // the run's aggregate [P | q]
     const float* Ql = sQ + ((gs - 1) & 1) * DP;
