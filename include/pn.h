@@ -240,9 +240,10 @@ PN_API pn_status pn_reset_stats(pn_handle h);
 /* Set one pn_option.  Values: PN_OPT_WAIT_TIMEOUT_NS >= 1000;
  * PN_OPT_DEBUG_STALL_TICKET -1 or a ticket >= 0; PN_OPT_NEWTON_BAND -1 or a
  * half-bandwidth >= 0; PN_OPT_RUN_LENGTH >= 0; PN_OPT_SMALL_SOLVE, PN_OPT_DEVICE_LOOP and
- * PN_OPT_TENSOR_CORES 0 or 1 (tensor cores: ignored where the shape has no
- * tensor-core kernel; switching re-selects the kernels after synchronising the
- * stream).  Anything else: PN_ERR_INVALID, the handle unchanged. */
+ * PN_OPT_TENSOR_CORES 0 or 1 (tensor cores, 3xTF32: the matvec kernels of the
+ * diagonal modes, the Newton compositions at padded width 16, 32 and 64; 0 runs
+ * the FP32 kernels; ignored where the shape has no tensor-core kernel;
+ * switching re-selects the kernels after synchronising the stream).  Anything else: PN_ERR_INVALID, the handle unchanged. */
 PN_API pn_status pn_set_option(pn_handle h, pn_option opt, long long value);
 
 /* Adaptive switching (page §5.3: when the residual curve stalls, switch to

@@ -277,6 +277,7 @@ IterParams make_params(const pn_ctx* h, int mode) {
   P.nchunks = h->fam.nchunks[mode];
   P.tiles_per_group = h->B * h->fam.nchunks[mode];
   P.run = h->fam.run[mode];
+  P.tc = h->tc_opt ? 1 : 0;
   const int G = h->fam.k[mode].G;
   // the wide per-channel kernel keeps two (A, B) pairs per channel: the tile's and its first half's
   P.agg_stride = dense ? G * (G + 1) : (kind == kKindDiagPost ? 4 * G : 2 * G);

@@ -121,6 +121,7 @@ struct IterParams {
   int agg_stride, pref_stride;
   int persist;          // looping kernels: 1 = run iterations until the stop rule, 0 = one iteration
   int run;              // chunks of L steps per ticket (a run; 1 for the kernels that take single chunks)
+  int tc;               // 1: the Newton kernel's D = 16 chunk chain on the tensor cores (PN_OPT_TENSOR_CORES)
   cudaGraphConditionalHandle cond;
   cudaGraphConditionalHandle mode_cond[4];   // adaptive graph: the IF node of each mode
   int* mode_hist;       // adaptive: the mode of each kept update [kHistCap]

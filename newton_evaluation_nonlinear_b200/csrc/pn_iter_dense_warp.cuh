@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
   // the D = 16 tensor-core chain (one-gate cells, no band)
   constexpr bool kMmaChain = (DP == 16 && R == 1);
   static_assert(!kMmaChain || C::NA == 32, "every lane takes part in the chain");
-  const bool mma_chain = kMmaChain && !banded;
+  const bool mma_chain = kMmaChain && !banded && P.tc != 0;   // PN_OPT_TENSOR_CORES = 0: the FMA chain
   const int qg = lane >> 2, qi = lane & 3;   // the MMA fragments' row group and column pair
 
   // W_q[r0 + r][k] of the Jacobian (band-masked when banded), RPL consecutive rows

@@ -415,23 +415,24 @@ def test_wide_bounded_wait_times_out_and_recovers():
     solver.close()
 
 
+@pytest.mark.parametrize("tc", [0, 1])
 @pytest.mark.parametrize("device_loop", [1, 0])
 @pytest.mark.parametrize("run", [1, 3, 0])
 @pytest.mark.parametrize("cell,D", [(pi.CELL_TANH_RNN, 16), (pi.CELL_GRU, 8), (pi.CELL_EULER, 4),
                                     (pi.CELL_TANH_RNN, 32), (pi.CELL_TANH_RNN, 12), (pi.CELL_EULER, 13),
                                     (pi.CELL_GRU, 16)])
-def test_newton_run_lengths(run, cell, D, device_loop):
+def test_newton_run_lengths(run, cell, D, device_loop, tc):
     """The Newton kernel at D <= 32 gives a ticket a run of consecutive 32-step chunks (one
     aggregate per run; the cell phase evaluated again in the write-out pass when the run is longer
     than one): one chunk, three (the last run ragged) and the automatic length all match the oracle,
     looping in one launch or launched per iteration.  At padded width 16 the one-gate cells run the
-    chunk chain on the tensor cores (D = 12, 13, 16: padded channels included), the GRU on the FMA
-    pipe."""
+    chunk chain on the tensor cores (D = 12, 13, 16: padded channels included) unless
+    PN_OPT_TENSOR_CORES = 0, the GRU always on the FMA pipe."""
     T, B = 1000, 3   # 32 chunks, the last one ragged
     d_in = D if cell == pi.CELL_EULER else D - 1
     prob = pi.random_problem(1700 + 5 * D + cell, cell, D, d_in, T=T, B=B, rho=0.6, eps=0.05,
                              s0_scale=0.3, tol=1e-5)
-    _check_against_oracle(prob, pi.MODE_NEWTON, device_loop=device_loop, tc=0,
+    _check_against_oracle(prob, pi.MODE_NEWTON, device_loop=device_loop, tc=tc,
                           opts={"PN_OPT_RUN_LENGTH": run})
 
 
