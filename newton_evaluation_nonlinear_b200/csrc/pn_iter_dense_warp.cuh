@@ -101,7 +101,8 @@ __device__ __forceinline__ void lds_n(const float* p, float (&v)[N]) {
   }
 }
 
-// The chain at D = 16 on the tensor cores (one-gate cells, no band).  With Q = P^T the step
+// The chain at D = 16 on the tensor cores (one-gate cells; banded: W is the band-masked copy, at the
+// dense cost -- the tensor cores gain nothing from the zeros).  With Q = P^T the step
 // P_m = (diag(c0) + diag(c1) W) P_{m-1} reads Q_m = Q_{m-1} diag(c0) + (Q_{m-1} W^T) diag(c1): a
 // 16 x 16 x 16 product with the constant W^T as the B operand.  Q lives in the f32 accumulator
 // layout of the m16n8k8 TF32 MMA (lane = 4 g + i holds rows g, g + 8 and columns 2 i, 2 i + 1 of
@@ -232,10 +233,10 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
   }
   unsigned rbits = 0u;
   bool aborted = false;
-  // the D = 16 tensor-core chain (one-gate cells, no band)
+  // the D = 16 tensor-core chain (one-gate cells, dense or banded)
   constexpr bool kMmaChain = (DP == 16 && R == 1);
   static_assert(!kMmaChain || C::NA == 32, "every lane takes part in the chain");
-  const bool mma_chain = kMmaChain && !banded && P.tc != 0;   // PN_OPT_TENSOR_CORES = 0: the FMA chain
+  const bool mma_chain = kMmaChain && P.tc != 0;   // PN_OPT_TENSOR_CORES = 0: the FMA chain
   const int qg = lane >> 2, qi = lane & 3;   // the MMA fragments' row group and column pair
 
   // W_q[r0 + r][k] of the Jacobian (band-masked when banded), RPL consecutive rows
@@ -439,7 +440,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
           for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const float w = sWf[(8 * ks + 2 * qi + h) * WR + 8 * j + qg];   // W[8 j + g][8 s + 2 i + h]
+              const float w = sWj[(8 * ks + 2 * qi + h) * WR + 8 * j + qg];   // W[8 j + g][8 s + 2 i + h]
               wbh[ks][j][h] = tf32_hi_bits(w);
               wbl[ks][j][h] = tf32_hi_bits(w - __uint_as_float(wbh[ks][j][h]));
             }
@@ -468,7 +469,7 @@ __global__ void __launch_bounds__(32 * NWARP, DenseWarpCfg<CELL, DP, NWARP>::MIN
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int n = qg + 8 * (e >> 1), r = 8 * j + 2 * qi + (e & 1);
-                qt[j][e] = fmaf(sc1[j][e & 1], sWf[n * WR + r], (r == n) ? sc0[j][e & 1] : 0.0f);
+                qt[j][e] = fmaf(sc1[j][e & 1], sWj[n * WR + r], (r == n) ? sc0[j][e & 1] : 0.0f);
               }
 #pragma unroll
             for (int r = 0; r < RPL; ++r) qn[r] = bm[r];

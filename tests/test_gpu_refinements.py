@@ -80,6 +80,14 @@ def test_banded_newton_matches_oracle(cell, D, T, B, small, band):
 
 
 @pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("band", [0, 2])
+def test_banded_newton_fma_chain(cell, band):
+    """At D = 16 the one-gate cells' banded chain runs on the tensor cores with the band-masked W
+    (the case above); PN_OPT_TENSOR_CORES = 0 runs it on the FMA pipe over the band's columns only."""
+    _check(cell, 16, 517, 3, band, 1.0, 311 + cell + band, tc=0)
+
+
+@pytest.mark.parametrize("cell", CELLS)
 @pytest.mark.parametrize("band,damping", [(-1, 0.5), (-1, 0.8), (2, 0.7)])
 @pytest.mark.parametrize("D,T", [(12, 400), (6, 300)])
 def test_damped_newton_matches_oracle(cell, band, damping, D, T):
