@@ -132,7 +132,7 @@ struct DiagTctCfg {
                                                  // that tile's prefixes take over its stash slot
   static constexpr int NAG = NSLOT + 1;          // slots of the aggregate hand-off to the look-back
   static constexpr int NLB = kScan ? 2 : 0;      // look-back warps, alternating tiles
-  static constexpr int FB = 6;                   // aggregates per look-back round trip
+  static constexpr int FB = 4;                   // aggregates per look-back round trip (4 measured fastest of 2-8)
   static constexpr int STASH0 = 2 * RS;          // accumulators: 2 x RS columns
   static constexpr int USED_COLS = STASH0 + (kScan ? NSLOT * SCOLS : 0);
   static constexpr int ALLOC_COLS =
