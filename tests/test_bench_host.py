@@ -56,3 +56,19 @@ def test_algorithmic_bytes_of_the_headline_workload():
 def test_job_throughput_and_cpu_model():
     assert bench.job_throughput(1000.0, 4, 2.0) == 2_000_000.0
     assert isinstance(bench.cpu_model(), str) and bench.cpu_model()
+
+
+def test_traffic_only_while_the_device_source_matches(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu figure only while the device code hashes to the
+    value recorded beside it; any other source, an unknown workload or no file gives None."""
+    import json
+    p = pi.benchmark_workload(1, T=64, B=2)
+    key = f"{p.name}:{pi.MODE_NAMES[pi.MODE_QUASI]}"
+    monkeypatch.setattr(bench, "PROFILES", str(tmp_path))
+    assert bench.traffic_from_profile(p, pi.MODE_QUASI) is None          # no file
+    sha = bench.kernel_source_sha()
+    (tmp_path / "traffic.json").write_text(json.dumps({key: {"source_sha": sha, "dram_bytes_per_launch": 1.5e8}}))
+    assert bench.traffic_from_profile(p, pi.MODE_QUASI) == 1.5e8
+    assert bench.traffic_from_profile(p, pi.MODE_JACOBI) is None         # no entry for that mode
+    (tmp_path / "traffic.json").write_text(json.dumps({key: {"source_sha": "0" * 16, "dram_bytes_per_launch": 1.5e8}}))
+    assert bench.traffic_from_profile(p, pi.MODE_QUASI) is None          # taken on another source
